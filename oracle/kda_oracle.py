@@ -1,0 +1,126 @@
+"""KDA oracle, Python side: builds and calls the fp64 C recurrence in
+``kda_oracle.c``.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this module.  It shares no code with
+the CUDA path and never imports the product package.
+
+The recurrence (page "Kimi Linear" on docsaid.org, section "KDA : une
+decroissance propre a chaque canal"; course page "Attention lineaire et
+recurrence", section "Kimi Delta Attention = les trois remedes combines"):
+
+    S_t = (I - beta_t k_t k_t^T) Diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T
+    o_t = S_t^T q_t
+
+Inputs are float64 numpy arrays holding exactly the values the GPU sees (bf16
+inputs are widened exactly).  Pins of this oracle (closed forms, exact
+retrieval, explicit transition products, invariants) are in
+``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "libkda_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP, IEEE semantics: no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math",
+             "-ffp-contract=off", "-std=c11", _SRC, "-o", tmp, "-lm"],
+            check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            dp = ctypes.POINTER(ctypes.c_double)
+            lib.kda_oracle_recurrence.argtypes = [
+                dp, dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                dp, dp, ctypes.c_int]
+            lib.kda_oracle_recurrence.restype = ctypes.c_int
+            lib.kda_oracle_max_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    """Threads the oracle's OpenMP region uses by default."""
+    return int(_load().kda_oracle_max_threads())
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def kda_recurrence(q, k, v, g, beta, init_state=None, cu_seqlens=None,
+                   nthreads: int = 0):
+    """Run the recurrence over packed sequences.
+
+    q, k, g: [T, H, d_k]; v: [T, H, d_v]; beta: [T, H];
+    init_state: [N, H, d_k, d_v] or None (zeros);
+    cu_seqlens: [N+1] int offsets or None (one sequence of length T).
+    Returns (o [T, H, d_v], final_state [N, H, d_k, d_v]) as float64.
+    """
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    if k.shape != (T, H, dk) or g.shape != (T, H, dk):
+        raise ValueError("q, k, g must share shape [T, H, d_k]")
+    if v.shape[:2] != (T, H) or beta.shape != (T, H):
+        raise ValueError("v must be [T, H, d_v] and beta [T, H]")
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    n = cu.shape[0] - 1
+    if cu[0] != 0 or cu[-1] != T:
+        raise ValueError("cu_seqlens must start at 0 and end at T")
+    s0 = None if init_state is None else _f64(init_state)
+    if s0 is not None and s0.shape != (n, H, dk, dv):
+        raise ValueError("init_state must be [N, H, d_k, d_v]")
+    o = np.zeros((T, H, dv), dtype=np.float64)
+    fs = np.zeros((n, H, dk, dv), dtype=np.float64)
+    rc = _load().kda_oracle_recurrence(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0),
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        n, H, dk, dv, _ptr(o), _ptr(fs), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_recurrence failed with code {rc}")
+    return o, fs
+
+
+def kda_decode_step(q, k, v, g, beta, state, nthreads: int = 0):
+    """One recurrence step for each of B independent sequences.
+
+    q, k, g: [B, H, d_k]; v: [B, H, d_v]; beta: [B, H]; state [B, H, d_k, d_v].
+    Returns (o [B, H, d_v], new_state).  A decode step is the recurrence on B
+    sequences of length one each.
+    """
+    B = np.asarray(q).shape[0]
+    cu = np.arange(B + 1, dtype=np.int64)
+    return kda_recurrence(q, k, v, g, beta, init_state=state, cu_seqlens=cu,
+                          nthreads=nthreads)
