@@ -1,0 +1,137 @@
+// C ABI of libkda.so: host-side validation and dispatch.  Declarations and
+// the contract of each entry point are in include/kda.h.
+#include <climits>
+
+#include "kda_internal.cuh"
+
+namespace {
+
+constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
+
+bool supported_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+bool aligned_to(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool aligned16(const void *p) { return aligned_to(p, 16); }
+
+size_t elem_bytes(kda_dtype t) { return t == KDA_BF16 ? 2 : 4; }
+
+bool overlaps(const void *a, size_t an, const void *b, size_t bn) {
+    if (!a || !b || an == 0 || bn == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + bn && b0 < a0 + an;
+}
+
+kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: shape or dtype not supported";
+        case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA runtime error";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+int kda_version(void) { return kVersion; }
+
+size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens,
+                                  int32_t H, int32_t d_k, int32_t d_v) {
+    if (num_seqs < 1 || total_tokens < 0 || H < 1) return 0;
+    if (!supported_dim(d_k) || !supported_dim(d_v)) return 0;
+    return kda::kWorkspaceHeader;
+}
+
+kda_status kda_prefill(const void *q, const void *k, const void *v,
+                       const void *log_alpha, const void *beta,
+                       const float *init_state, const int32_t *cu_seqlens,
+                       int32_t num_seqs, int64_t total_tokens, int32_t H,
+                       int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                       float *final_state, void *workspace,
+                       size_t workspace_bytes, kda_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (num_seqs < 1 || total_tokens < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_BF16 && dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(d_k) || !supported_dim(d_v)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)num_seqs * H > INT_MAX) return KDA_ERR_UNSUPPORTED;
+    if (!cu_seqlens && total_tokens % num_seqs != 0) return KDA_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !o))
+        return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, init_state, o, final_state};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (beta && !aligned_to(beta, elem_bytes(dtype))) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
+    const size_t need = kda_prefill_workspace_size(num_seqs, total_tokens, H, d_k, d_v);
+    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_INVALID_ARG;
+
+    const size_t eb = elem_bytes(dtype);
+    const size_t nk = (size_t)total_tokens * H * d_k * eb;
+    const size_t nv = (size_t)total_tokens * H * d_v * eb;
+    const size_t nb = (size_t)total_tokens * H * eb;
+    const size_t ns = (size_t)num_seqs * H * d_k * d_v * sizeof(float);
+    if (overlaps(o, nv, q, nk) || overlaps(o, nv, k, nk) || overlaps(o, nv, v, nv) ||
+        overlaps(o, nv, log_alpha, nk) || overlaps(o, nv, beta, nb) ||
+        overlaps(o, nv, init_state, ns) || overlaps(o, nv, final_state, ns) ||
+        overlaps(o, nv, workspace, need))
+        return KDA_ERR_INVALID_ARG;
+    if (init_state && final_state && init_state != final_state &&
+        overlaps(init_state, ns, final_state, ns))
+        return KDA_ERR_INVALID_ARG;
+
+    uint32_t *err_word = static_cast<uint32_t *>(workspace);
+    cudaError_t e = cudaMemsetAsync(err_word, 0, sizeof(uint32_t), stream);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    e = kda::launch_prefill_simt(q, k, v, log_alpha, beta, init_state, cu_seqlens,
+                                 num_seqs, total_tokens, H, d_k, d_v, dtype, o,
+                                 final_state, err_word, stream);
+    return from_cuda(e);
+}
+
+kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const void *log_alpha, const void *beta,
+                           float *state, int32_t batch, int32_t H,
+                           int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                           kda_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (batch < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_BF16 && dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(d_k) || !supported_dim(d_v)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)batch * H > INT_MAX) return KDA_ERR_UNSUPPORTED;
+    if (batch == 0) return KDA_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_INVALID_ARG;
+    const size_t eb = elem_bytes(dtype);
+    const void *ptrs[] = {q, k, v, log_alpha, beta, o};
+    for (const void *p : ptrs)
+        if (!aligned_to(p, eb)) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(state)) return KDA_ERR_INVALID_ARG;
+    const size_t nk = (size_t)batch * H * d_k * eb;
+    const size_t nv = (size_t)batch * H * d_v * eb;
+    const size_t nb = (size_t)batch * H * eb;
+    const size_t ns = (size_t)batch * H * d_k * d_v * sizeof(float);
+    if (overlaps(o, nv, q, nk) || overlaps(o, nv, k, nk) || overlaps(o, nv, v, nv) ||
+        overlaps(o, nv, log_alpha, nk) || overlaps(o, nv, beta, nb) ||
+        overlaps(o, nv, state, ns))
+        return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_decode(q, k, v, log_alpha, beta, state, batch, H,
+                                        d_k, d_v, dtype, o, stream));
+}
+
+kda_status kda_check_workspace_error(const void *workspace, kda_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (!workspace) return KDA_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    return word == kda::kDevErrNone ? KDA_OK : KDA_ERR_INVALID_ARG;
+}
+
+}  // extern "C"

@@ -1,0 +1,63 @@
+// Internal helpers shared by the KDA CUDA kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// Element I/O for the two supported input/output types.
+template <typename T> struct io;
+
+template <> struct io<float> {
+    static __device__ __forceinline__ float load(const float *p) { return *p; }
+    static __device__ __forceinline__ void store(float *p, float x) { *p = x; }
+};
+
+template <> struct io<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(const __nv_bfloat16 *p) {
+        return __bfloat162float(*p);
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, float x) {
+        *p = __float2bfloat16_rn(x);
+    }
+};
+
+// Per-token log-decay floor.  A retention factor exp(-80) ~ 1.8e-35 already
+// acts as zero against any state magnitude, and the floor keeps the
+// within-chunk running sums finite (so differences of running sums are
+// defined even for log_alpha = -inf).
+constexpr float kLogAlphaFloor = -80.0f;
+
+__device__ __forceinline__ float clamp_log_alpha(float g) {
+    return fmaxf(g, kLogAlphaFloor);
+}
+
+// Error word written by device-side checks into the workspace header.
+enum : uint32_t {
+    kDevErrNone = 0,
+    kDevErrCuSeqlens = 1u << 0,   // cu_seqlens not non-decreasing / bad ends
+};
+
+// Workspace layout: a 256-byte header holding the error word, then the
+// per-kernel scratch areas.
+constexpr size_t kWorkspaceHeader = 256;
+
+// Launchers (defined in the .cu files).  All return cudaGetLastError().
+cudaError_t launch_decode(const void *q, const void *k, const void *v,
+                          const void *g, const void *beta, float *state,
+                          int batch, int H, int dk, int dv, kda_dtype dtype,
+                          void *o, cudaStream_t stream);
+
+cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
+                                const void *g, const void *beta,
+                                const float *init_state, const int32_t *cu,
+                                int num_seqs, int64_t total_tokens, int H,
+                                int dk, int dv, kda_dtype dtype, void *o,
+                                float *final_state, uint32_t *err_word,
+                                cudaStream_t stream);
+
+}  // namespace kda

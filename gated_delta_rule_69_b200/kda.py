@@ -1,0 +1,141 @@
+"""Thin Python binding of libkda.so (the C ABI declared in include/kda.h).
+
+Argument marshalling only: every step of the operator runs in the library's
+CUDA kernels.  Functions carry the C names and take torch CUDA tensors (or
+None for the optional ones); outputs are allocated here when not supplied.
+There is no CPU path: without the built library, or without a CUDA device,
+every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
+_lib = None
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA = range(5)
+KDA_BF16, KDA_FP32 = 0, 1
+EXPORTED = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
+            "kda_prefill", "kda_decode_step", "kda_check_workspace_error")
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+def lib():
+    """Load libkda.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with "
+                "`python -m gated_delta_rule_69_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        L.kda_status_string.argtypes = [ctypes.c_int]
+        L.kda_status_string.restype = ctypes.c_char_p
+        L.kda_version.restype = ctypes.c_int
+        L.kda_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32]
+        L.kda_prefill_workspace_size.restype = sz
+        L.kda_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
+                                  ctypes.c_int, vp, vp, vp, sz, vp]
+        L.kda_prefill.restype = ctypes.c_int
+        L.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                      ctypes.c_int, vp, vp]
+        L.kda_decode_step.restype = ctypes.c_int
+        L.kda_check_workspace_error.argtypes = [vp, vp]
+        L.kda_check_workspace_error.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().kda_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}: use bfloat16 or float32")
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def kda_prefill_workspace_size(num_seqs: int, total_tokens: int, H: int, d_k: int, d_v: int) -> int:
+    return int(lib().kda_prefill_workspace_size(num_seqs, total_tokens, H, d_k, d_v))
+
+
+def kda_prefill(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None,
+                num_seqs=None, o=None, final_state=None, workspace=None,
+                output_final_state=True, stream=None):
+    """Chunkwise KDA prefill.  Shapes: q, k, log_alpha [T, H, d_k]; v [T, H, d_v];
+    beta [T, H]; init_state [N, H, d_k, d_v] fp32 or None; cu_seqlens int32
+    [N+1] on the device or None (num_seqs equal sequences, default 1).
+    Returns (o, final_state); final_state is None if output_final_state is False.
+    """
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is not None:
+        n = cu_seqlens.numel() - 1
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+    else:
+        n = 1 if num_seqs is None else int(num_seqs)
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = kda_prefill_workspace_size(n, T, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check_cuda(q, k, v, log_alpha, beta, init_state, cu_seqlens, o, final_state, workspace)
+    st = lib().kda_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
+        _ptr(cu_seqlens), n, T, H, dk, dv, _dtype_code(q), _ptr(o), _ptr(final_state),
+        _ptr(workspace), workspace.numel(), _stream(stream, q.device))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_prefill")
+    return o, final_state
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, state, o=None, stream=None):
+    """One KDA step per sequence; ``state`` [B, H, d_k, d_v] fp32 is updated in
+    place.  Returns o [B, H, d_v]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _check_cuda(q, k, v, log_alpha, beta, state, o)
+    st = lib().kda_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state),
+        B, H, dk, dv, _dtype_code(q), _ptr(o), _stream(stream, q.device))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode_step")
+    return o
+
+
+def kda_check_workspace_error(workspace, stream=None) -> int:
+    """Synchronise and return the status of the device-side checks."""
+    return int(lib().kda_check_workspace_error(_ptr(workspace), _stream(stream, workspace.device)))

@@ -1,0 +1,160 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention operator library
+ * (libkda.so).
+ *
+ * The operator is the per-head recurrence of Kimi Delta Attention (page
+ * "Kimi Linear" on docsaid.org, section "KDA : une decroissance propre a
+ * chaque canal", the KDA update equation; course page "Attention lineaire et
+ * recurrence", section "Kimi Delta Attention = les trois remedes combines"):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * with a per-key-channel forget gate alpha_t = exp(log_alpha_t) in (0, 1]^{d_k}
+ * and a scalar write strength beta_t in [0, 1] per token and head.  The state
+ * S is d_k x d_v per (sequence, head) and is kept in fp32.  The read-out uses
+ * the updated state S_t; no 1/sqrt(d_k) scale is applied (fold it into q).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no device memory and keeps no state between calls except a
+ *     cached per-device property query.
+ *   - Tensors are dense, row-major, token-major:
+ *       q, k, log_alpha : [T_total, H, d_k]
+ *       v, o            : [T_total, H, d_v]
+ *       beta            : [T_total, H]
+ *       states          : [N, H, d_k, d_v] fp32, d_v fastest
+ *     For decode, T_total is the batch size (one token per sequence).
+ *   - Alignment: fp32 state pointers, and q, k, v, log_alpha and o of
+ *     kda_prefill, must be 16-byte aligned; beta, cu_seqlens and every input
+ *     of kda_decode_step other than the state need only their element's
+ *     natural alignment.  The workspace is 256-byte aligned.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream) and never
+ *     synchronise, except kda_check_workspace_error.
+ *   - Arguments are validated on the host; a failed check returns a status
+ *     and launches nothing.  Launch failures return KDA_ERR_CUDA.  No C++
+ *     exception crosses this boundary and no kernel traps or asserts.
+ *   - Data preconditions that are documented but not checked: log_alpha <= 0
+ *     (alpha in (0, 1]; -inf is allowed and means alpha = 0), beta in [0, 1],
+ *     finite values, and, for the fast path's accuracy bound, L2-normalised
+ *     q and k (the pages normalise q and k before the operator).
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The stream type of the CUDA runtime, declared opaquely so that this header
+ * does not need cuda_runtime.h. */
+typedef struct CUstream_st *kda_stream_t;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer   */
+    KDA_ERR_UNSUPPORTED = 2,  /* shape or dtype without a kernel               */
+    KDA_ERR_WORKSPACE = 3,    /* workspace missing or too small                */
+    KDA_ERR_CUDA = 4          /* a CUDA runtime call or launch failed          */
+} kda_status;
+
+/* Element type of q, k, v, log_alpha, beta and o.  States are always fp32. */
+typedef enum {
+    KDA_BF16 = 0,
+    KDA_FP32 = 1
+} kda_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kda_status_string(kda_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int kda_version(void);
+
+/*
+ * Workspace bytes kda_prefill needs for this problem (a multiple of 256; may
+ * be 0 only if the library needs none).  Pure host arithmetic, no CUDA call.
+ * Returns 0 for arguments kda_prefill would reject.
+ */
+size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens,
+                                  int32_t H, int32_t d_k, int32_t d_v);
+
+/*
+ * Chunkwise prefill over a packed batch of sequences.
+ *
+ * Computes o_t for every token and, per sequence, the state after its last
+ * token.  The sequence is cut into chunks of 64 tokens; within a chunk the
+ * work is matrix products and between chunks the state is carried (news
+ * digest page on Kimi Linear, section "Algorithme parallele par chunks";
+ * course page "Attention lineaire et recurrence", section "Le calcul par
+ * blocs").  The chunked form is exact; only the rounding order differs from
+ * the token-by-token recurrence.
+ *
+ *   q, k, log_alpha : [T_total, H, d_k]  dtype
+ *   v               : [T_total, H, d_v]  dtype
+ *   beta            : [T_total, H]       dtype
+ *   init_state      : [N, H, d_k, d_v] fp32, or NULL for zero initial states
+ *   cu_seqlens      : device int32 [N + 1], cu_seqlens[0] = 0, non-decreasing,
+ *                     cu_seqlens[N] = T_total; or NULL for N sequences of
+ *                     equal length T_total / N (T_total % N must be 0).
+ *                     Zero-length sequences are allowed: their final state
+ *                     is their initial state.
+ *   num_seqs (N) >= 1, total_tokens >= 0, H >= 1.
+ *   o               : [T_total, H, d_v]  dtype, written
+ *   final_state     : [N, H, d_k, d_v] fp32, written, or NULL.  May alias
+ *                     init_state exactly (same pointer).
+ *   workspace       : device buffer of at least
+ *                     kda_prefill_workspace_size(...) bytes, 256-byte aligned;
+ *                     its contents on entry do not matter.
+ *
+ * Supported: dtype KDA_BF16 or KDA_FP32 with d_k, d_v in {16, 32, 64, 128}.
+ * KDA_BF16 with d_k = d_v = 128 runs the tensor-core (tcgen05) path; every
+ * other case runs the fp32 CUDA-core path (KDA_FP32 is the accurate test
+ * mode).  o must not overlap any input.
+ */
+kda_status kda_prefill(const void *q, const void *k, const void *v,
+                       const void *log_alpha, const void *beta,
+                       const float *init_state, const int32_t *cu_seqlens,
+                       int32_t num_seqs, int64_t total_tokens, int32_t H,
+                       int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                       float *final_state, void *workspace,
+                       size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * One decode step for `batch` independent sequences, state updated in place.
+ *
+ * Per (b, h): S <- Diag(exp(log_alpha)) S;  u = beta (v - S^T k);
+ * S <- S + k u^T;  o = S^T q  -- the KDA update for a single token, which is
+ * the step form the chunked prefill hands over to (the state is the whole
+ * memory of the sequence).
+ *
+ *   q, k, log_alpha : [batch, H, d_k] dtype;  v, o : [batch, H, d_v] dtype;
+ *   beta : [batch, H] dtype;  state : [batch, H, d_k, d_v] fp32, read and
+ *   written in place.
+ * Supported: dtype KDA_BF16 or KDA_FP32, d_k in {16, 32, 64, 128},
+ * d_v in {16, 32, 64, 128}.  o must not overlap the state or the inputs.
+ * batch = 0 is a valid no-op.
+ */
+kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const void *log_alpha, const void *beta,
+                           float *state, int32_t batch, int32_t H,
+                           int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                           kda_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads the error word that the prefill kernels
+ * leave at the start of `workspace` (non-zero when a device-side check failed,
+ * e.g. cu_seqlens not non-decreasing or not ending at T_total).  Returns
+ * KDA_ERR_INVALID_ARG in that case, KDA_OK otherwise.  Debugging aid; the
+ * only call here that blocks.
+ */
+kda_status kda_check_workspace_error(const void *workspace,
+                                     kda_stream_t stream);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* KDA_H_ */

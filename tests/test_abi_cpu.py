@@ -1,0 +1,113 @@
+"""libkda.so loads on a host without a GPU, exports every function that
+include/kda.h declares, and rejects bad arguments on the host before any CUDA
+call.  CPU only: the pointers passed here are never dereferenced."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_delta_rule_69_b200 import build, kda
+    build.build()
+    return kda.lib()
+
+
+def _declared_functions():
+    names = []
+    for path in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if path.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", path)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(kda_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared_functions()
+    assert "kda_prefill" in names and "kda_decode_step" in names
+    for n in names:
+        assert hasattr(L, n), f"libkda.so does not export {n}"
+
+
+def test_binding_names_match_header():
+    from gated_delta_rule_69_b200 import kda
+    for n in _declared_functions():
+        if n in ("kda_status_string", "kda_version"):
+            continue
+        assert hasattr(kda, n), f"binding lacks {n}"
+
+
+def test_status_strings(L):
+    for s in range(5):
+        assert L.kda_status_string(s).startswith(b"KDA_")
+    assert L.kda_status_string(99) == b"KDA_ERR_UNKNOWN"
+
+
+def test_workspace_size(L):
+    ws = L.kda_prefill_workspace_size
+    assert ws(1, 4096, 16, 128, 128) >= 256
+    assert ws(1, 4096, 16, 128, 128) % 256 == 0
+    assert ws(0, 10, 1, 16, 16) == 0
+    assert ws(1, 10, 1, 48, 16) == 0
+    assert ws(1, -1, 1, 16, 16) == 0
+
+
+FAKE = 1 << 20  # 16-byte aligned, never dereferenced on the host
+
+
+def _prefill(L, **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, g=FAKE * 4, b=FAKE * 5, s0=None, cu=None,
+             n=1, T=64, H=1, dk=16, dv=16, dt=1, o=FAKE * 64, fs=None, ws=FAKE * 128,
+             wsb=256)
+    a.update(kw)
+    return L.kda_prefill(a["q"], a["k"], a["v"], a["g"], a["b"], a["s0"], a["cu"],
+                         a["n"], a["T"], a["H"], a["dk"], a["dv"], a["dt"], a["o"],
+                         a["fs"], a["ws"], a["wsb"], None)
+
+
+def test_prefill_rejects_on_host(L):
+    assert _prefill(L, n=0) == 1
+    assert _prefill(L, H=0) == 1
+    assert _prefill(L, T=-1) == 1
+    assert _prefill(L, dt=7) == 1
+    assert _prefill(L, dk=48) == 2
+    assert _prefill(L, dv=256) == 2
+    assert _prefill(L, q=None) == 1
+    assert _prefill(L, q=FAKE + 4) == 1            # misaligned
+    assert _prefill(L, n=3, T=64) == 1             # T % N != 0 without cu_seqlens
+    assert _prefill(L, ws=None) == 3
+    assert _prefill(L, wsb=16) == 3
+    assert _prefill(L, ws=FAKE * 128 + 16) == 1    # workspace not 256-aligned
+    assert _prefill(L, o=FAKE + 64) == 1           # o overlaps q
+
+
+def _decode(L, **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, g=FAKE * 4, b=FAKE * 5, s=FAKE * 16,
+             B=4, H=2, dk=16, dv=16, dt=1, o=FAKE * 64)
+    a.update(kw)
+    return L.kda_decode_step(a["q"], a["k"], a["v"], a["g"], a["b"], a["s"], a["B"],
+                             a["H"], a["dk"], a["dv"], a["dt"], a["o"], None)
+
+
+def test_decode_rejects_on_host(L):
+    assert _decode(L, B=0) == 0                    # empty batch: no-op
+    assert _decode(L, B=-1) == 1
+    assert _decode(L, H=0) == 1
+    assert _decode(L, dk=8) == 2
+    assert _decode(L, s=None) == 1
+    assert _decode(L, o=FAKE * 16 + 32) == 1       # o overlaps the state
+    assert _decode(L, v=FAKE * 3 + 2) == 1         # not element-aligned (fp32)
+    assert _decode(L, s=FAKE * 16 + 8) == 1        # state not 16-byte aligned
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    from gated_delta_rule_69_b200 import kda
+    x = torch.zeros(4, 1, 16)
+    with pytest.raises((ValueError, RuntimeError, AssertionError)):
+        kda.kda_decode_step(x, x, x, x, torch.zeros(4, 1), torch.zeros(4, 1, 16, 16))
