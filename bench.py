@@ -1,0 +1,430 @@
+"""Benchmark of the KDA operator on B200: prefill tokens/s (headline) and
+decode tokens/s, each with its roofline, as ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed
+
+A step is one kda_prefill call over the prefill workload's batch (all chunks,
+all heads, final state written).  Inputs are resident in HBM when timing
+starts; L2 is flushed (a 256 MiB write) before every timed step, outside the
+timed interval.  The decode figures time chained kda_decode_step calls on the
+decode workload (state 512 MiB, larger than L2, so no flush is needed).
+Under torchrun every rank runs the same workload as an independent replica
+(the operator needs no exchange between GPUs); value = all ranks' tokens over
+the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s and decode tokens/s at 1 B200; fraction of tensor/HBM roofline"
+PREFILL_DEFAULT = "prefill_T4096_H16_d128"
+DECODE_DEFAULT = "decode_B256_H32_d128"
+DECODE_STEPS = 1000
+
+# Algorithmic work per (token, head) for prefill with chunk C and d_k = d_v = d:
+#   FLOP  = 6 d_k d_v + C (3 d_k + 2 d_v)          (state products + chunk products)
+#   bytes = (3 d_k + 2 d_v) * io_bytes + io_bytes  (q, k, log_alpha, v in; o out; beta in)
+# plus per (sequence, head) the fp32 state: read if an initial state is given,
+# written always.
+CHUNK = 64
+
+
+def prefill_work(w, lengths):
+    T = sum(lengths)
+    n = len(lengths)
+    eb = 2 if w.dtype == "bf16" else 4
+    per_tok_flop = 6 * w.d_k * w.d_v + CHUNK * (3 * w.d_k + 2 * w.d_v)
+    per_tok_bytes = (3 * w.d_k + 2 * w.d_v) * eb + eb
+    state_bytes = n * w.H * w.d_k * w.d_v * 4 * (2 if w.init_std > 0 else 1)
+    return dict(tokens=T, flop=per_tok_flop * T * w.H,
+                bytes=per_tok_bytes * T * w.H + state_bytes)
+
+
+def decode_work(w):
+    eb = 2 if w.dtype == "bf16" else 4
+    units = w.batch * w.H
+    return dict(tokens=w.batch,
+                flop=units * (6 * w.d_k * w.d_v + 2 * w.d_k),
+                bytes=units * (2 * w.d_k * w.d_v * 4 + (3 * w.d_k + 2 * w.d_v) * eb + eb))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p["bf16_tflops_sustained"]), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --- distributed plumbing -------------------------------------------------------
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --- the GPU arm -------------------------------------------------------------------
+
+def time_prefill(w, steps, warmup, world):
+    import torch
+    from gated_delta_rule_69_b200 import inputs as kin
+    from gated_delta_rule_69_b200 import kda
+    inp = kin.generate(w, device="cuda")
+    q, k, v, g, b = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta"))
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    n = len(inp["lengths"])
+    o = torch.empty((T, H, dv), dtype=q.dtype, device="cuda")
+    fs = torch.empty((n, H, dk, dv), dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(256, kda.kda_prefill_workspace_size(n, T, H, dk, dv)),
+                     dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.kda_prefill(q, k, v, g, b, init_state=inp["init_state"], cu_seqlens=inp["cu_seqlens"],
+                        o=o, final_state=fs, workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.fill_(i & 0xFF)                 # L2 flush, outside the timed interval
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    if kda.kda_check_workspace_error(ws) != kda.KDA_OK:
+        raise RuntimeError("device-side check failed during the benchmark")
+    return dict(ms_total=sum(ms), ms=ms, inputs=inp, launches=steps)
+
+
+def time_prefill_e2e(w, steps, warmup):
+    """Same workload through the public call, with each step's inputs copied
+    from pinned host memory and o + final state read back."""
+    import torch
+    from gated_delta_rule_69_b200 import inputs as kin
+    from gated_delta_rule_69_b200 import kda
+    inp = kin.generate(w, device="cuda")
+    names = ("q", "k", "v", "log_alpha", "beta")
+    host = {x: inp[x].cpu().pin_memory() for x in names}
+    dev = {x: torch.empty_like(inp[x]) for x in names}
+    T, H, dk = inp["q"].shape
+    dv = inp["v"].shape[-1]
+    n = len(inp["lengths"])
+    o_h = torch.empty((T, H, dv), dtype=inp["q"].dtype).pin_memory()
+    fs_h = torch.empty((n, H, dk, dv), dtype=torch.float32).pin_memory()
+    s0 = inp["init_state"]
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + fs_h.numel() * 4
+
+    def step():
+        for x in names:
+            dev[x].copy_(host[x], non_blocking=True)
+        o, fs = kda.kda_prefill(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
+                                init_state=s0, cu_seqlens=inp["cu_seqlens"])
+        o_h.copy_(o, non_blocking=True)
+        fs_h.copy_(fs, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    return dict(ms_per_step=e0.elapsed_time(e1) / steps, h2d=h2d, d2h=d2h)
+
+
+def time_decode(w, steps, warmup, world):
+    import torch
+    from gated_delta_rule_69_b200 import inputs as kin
+    from gated_delta_rule_69_b200 import kda
+    inp = kin.generate(w, device="cuda")
+    q, k, v, g, b, state = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta", "init_state"))
+    o = torch.empty((w.batch, w.H, w.d_v), dtype=q.dtype, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        kda.kda_decode_step(q, k, v, g, b, state, o=o, stream=stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        kda.kda_decode_step(q, k, v, g, b, state, o=o, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return dict(ms_total=e0.elapsed_time(e1), launches=steps)
+
+
+# --- the oracle on the host cores ------------------------------------------------------
+
+def oracle_prefill_sample(w, inp, budget_s=10.0, max_heads=None):
+    """Time the fp64 oracle on whole heads of the first sequence, adding heads
+    (as many per batch as there are oracle threads) until ``budget_s`` of CPU
+    work has run or every head is done.  Returns the oracle's tokens/s
+    extrapolated to the whole workload, and a description of the sample."""
+    import numpy as np
+    import oracle
+    from gated_delta_rule_69_b200.inputs import as_float64
+    cu = inp["cu_seqlens"].cpu().numpy()
+    L0 = int(cu[1] - cu[0])
+    threads = oracle.max_threads()
+    H = w.H if max_heads is None else min(w.H, max_heads)
+    done, t_total = 0, 0.0
+    while done < H and (done == 0 or t_total < budget_s):
+        hs = list(range(done, min(H, done + threads)))
+        sel = lambda t: as_float64(t[:L0, hs])
+        s0 = None if inp["init_state"] is None else as_float64(inp["init_state"][:1, hs])
+        args = [sel(inp[x]) for x in ("q", "k", "v", "log_alpha", "beta")]
+        t0 = time.perf_counter()
+        oracle.kda_recurrence(*args, init_state=s0, cu_seqlens=np.array([0, L0]))
+        t_total += time.perf_counter() - t0
+        done += len(hs)
+    total_tokens = sum(inp["lengths"])
+    # the oracle's cost is linear in (tokens x heads): scale the sampled rate
+    units_done = done * L0
+    units_all = total_tokens * w.H
+    value = total_tokens / (t_total * units_all / units_done)
+    sample = (f"{done} of {w.H} heads x {L0} tokens of sequence 0 "
+              f"({units_done} (token, head) pairs of {units_all}); tokens/s scaled by the pair count")
+    return value, threads, sample, t_total
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from gated_delta_rule_69_b200 import inputs as kin
+    inp = kin.generate(w, device="cpu")
+    import oracle
+    threads = oracle.max_threads()
+    vals, secs = [], []
+    for i in range(args.warmup + args.steps):
+        v, thr, sample, t = oracle_prefill_sample(w, inp, budget_s=0.0, max_heads=threads)
+        if i >= args.warmup:
+            vals.append(v)
+            secs.append(t)
+    value = statistics.median(vals)
+    work = prefill_work(w, inp["lengths"])
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * work["tokens"] / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, inp["lengths"], args.gpus),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, lengths, n_gpus):
+    c = {"workload": w.name, "tokens": sum(lengths), "num_seqs": len(lengths), "H": w.H,
+         "d_k": w.d_k, "d_v": w.d_v, "chunk": CHUNK, "io_dtype": w.dtype,
+         "state_dtype": "fp32", "init_state": "N(0, 0.02)" if w.init_std > 0 else "zeros",
+         "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
+         "l2": "flushed by a 256 MiB write before each timed prefill step"}
+    return c
+
+
+# --- main -------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=PREFILL_DEFAULT)
+    ap.add_argument("--decode-workload", default=DECODE_DEFAULT)
+    ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from gated_delta_rule_69_b200 import inputs as kin
+    w = kin.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    rank, world, local = dist_setup()
+    from gated_delta_rule_69_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    peaks = load_peaks()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    pf = time_prefill(w, args.steps, args.warmup, world)
+    dw = kin.WORKLOADS[args.decode_workload]
+    dec = time_decode(dw, args.decode_steps, args.warmup, world)
+    clocks = sampler.stop()
+
+    lengths = pf["inputs"]["lengths"]
+    work = prefill_work(w, lengths)
+    ms_step = max_over_ranks(pf["ms_total"] / args.steps, world)
+    value = world * work["tokens"] / (ms_step * 1e-3)
+    gbs = work["bytes"] / (ms_step * 1e-3) / 1e9
+    tfs = work["flop"] / (ms_step * 1e-3) / 1e12
+    dwork = decode_work(dw)
+    dms = max_over_ranks(dec["ms_total"] / args.decode_steps, world)
+    dgbs = dwork["bytes"] / (dms * 1e-3) / 1e9
+    src = "of " + peaks["source"]
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": config_of(w, lengths, world),
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm"], "traffic": None, "peak_source": src,
+                     "kernel": "kda_prefill", "algorithmic_bytes_per_launch": work["bytes"],
+                     "tensor_tflops": tfs, "tensor_frac": tfs / peaks["bf16"],
+                     "algorithmic_flop_per_launch": work["flop"]},
+        "decode": {"workload": dw.name, "value": world * dwork["tokens"] / (dms * 1e-3),
+                   "unit": "tokens/s", "ms_per_step": dms, "steps": args.decode_steps,
+                   "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm"],
+                                "unit": "GB/s", "frac": dgbs / peaks["hbm"], "traffic": None,
+                                "peak_source": src, "kernel": "kda_decode_step",
+                                "algorithmic_bytes_per_launch": dwork["bytes"]}},
+        "gpu_launches": pf["launches"] + dec["launches"],
+        "clocks": clocks,
+    }
+    if not args.no_e2e:
+        e2e = time_prefill_e2e(w, max(3, args.steps // 2), args.warmup)
+        e_ms = max_over_ranks(e2e["ms_per_step"], world)
+        line["e2e"] = {"value": world * work["tokens"] / (e_ms * 1e-3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, thr, sample, _ = oracle_prefill_sample(w, pf["inputs"], budget_s=10.0)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
