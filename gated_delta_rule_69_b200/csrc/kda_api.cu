@@ -24,6 +24,13 @@ bool overlaps(const void *a, size_t an, const void *b, size_t bn) {
 
 kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
 
+// The tensor-core path: bf16 I/O with 128 x 128 heads (token coordinates of
+// its tensor maps are 32-bit).
+bool use_tensor_cores(kda_dtype dtype, int d_k, int d_v, int64_t total_tokens) {
+    return dtype == KDA_BF16 && d_k == 128 && d_v == 128 && total_tokens > 0 &&
+           total_tokens <= INT_MAX;
+}
+
 }  // namespace
 
 extern "C" {
@@ -45,7 +52,7 @@ size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens,
                                   int32_t H, int32_t d_k, int32_t d_v) {
     if (num_seqs < 1 || total_tokens < 0 || H < 1) return 0;
     if (!supported_dim(d_k) || !supported_dim(d_v)) return 0;
-    return kda::kWorkspaceHeader;
+    return kda::prefill_tc_workspace(num_seqs);
 }
 
 kda_status kda_prefill(const void *q, const void *k, const void *v,
@@ -86,6 +93,10 @@ kda_status kda_prefill(const void *q, const void *k, const void *v,
         overlaps(init_state, ns, final_state, ns))
         return KDA_ERR_INVALID_ARG;
 
+    if (use_tensor_cores(dtype, d_k, d_v, total_tokens))
+        return from_cuda(kda::launch_prefill_tc(q, k, v, log_alpha, beta, init_state, cu_seqlens,
+                                                num_seqs, total_tokens, H, o, final_state,
+                                                workspace, stream));
     uint32_t *err_word = static_cast<uint32_t *>(workspace);
     cudaError_t e = cudaMemsetAsync(err_word, 0, sizeof(uint32_t), stream);
     if (e != cudaSuccess) return KDA_ERR_CUDA;

@@ -40,6 +40,7 @@ __device__ __forceinline__ float clamp_log_alpha(float g) {
 enum : uint32_t {
     kDevErrNone = 0,
     kDevErrCuSeqlens = 1u << 0,   // cu_seqlens not non-decreasing / bad ends
+    kDevErrTimeout = 1u << 1,     // a bounded wait gave up (internal error)
 };
 
 // Workspace layout: a 256-byte header holding the error word, then the
@@ -59,5 +60,13 @@ cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
                                 int dk, int dv, kda_dtype dtype, void *o,
                                 float *final_state, uint32_t *err_word,
                                 cudaStream_t stream);
+
+// Tensor-core prefill (bf16, d_k = d_v = 128).
+size_t prefill_tc_workspace(int num_seqs);
+
+cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const void *g,
+                              const void *beta, const float *init_state, const int32_t *cu,
+                              int num_seqs, int64_t total_tokens, int H, void *o,
+                              float *final_state, void *workspace, cudaStream_t stream);
 
 }  // namespace kda

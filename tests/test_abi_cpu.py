@@ -63,7 +63,7 @@ FAKE = 1 << 20  # 16-byte aligned, never dereferenced on the host
 def _prefill(L, **kw):
     a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, g=FAKE * 4, b=FAKE * 5, s0=None, cu=None,
              n=1, T=64, H=1, dk=16, dv=16, dt=1, o=FAKE * 64, fs=None, ws=FAKE * 128,
-             wsb=256)
+             wsb=4096)
     a.update(kw)
     return L.kda_prefill(a["q"], a["k"], a["v"], a["g"], a["b"], a["s0"], a["cu"],
                          a["n"], a["T"], a["H"], a["dk"], a["dv"], a["dt"], a["o"],
