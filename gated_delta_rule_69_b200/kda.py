@@ -19,7 +19,8 @@ _lib = None
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA = range(5)
 KDA_BF16, KDA_FP32 = 0, 1
 EXPORTED = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
-            "kda_prefill", "kda_decode_step", "kda_check_workspace_error")
+            "kda_prefill", "kda_decode_step", "kda_check_workspace_error",
+            "kda_prefill_noalloc")
 
 
 class KdaError(RuntimeError):
@@ -49,6 +50,9 @@ def lib():
         L.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                       ctypes.c_int, vp, vp]
         L.kda_decode_step.restype = ctypes.c_int
+        L.kda_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
+                                          ctypes.c_int, vp, vp, vp]
+        L.kda_prefill_noalloc.restype = ctypes.c_int
         L.kda_check_workspace_error.argtypes = [vp, vp]
         L.kda_check_workspace_error.restype = ctypes.c_int
         _lib = L
@@ -139,3 +143,31 @@ def kda_decode_step(q, k, v, log_alpha, beta, state, o=None, stream=None):
 def kda_check_workspace_error(workspace, stream=None) -> int:
     """Synchronise and return the status of the device-side checks."""
     return int(lib().kda_check_workspace_error(_ptr(workspace), _stream(stream, workspace.device)))
+
+
+def kda_prefill_noalloc(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None,
+                        num_seqs=None, o=None, final_state=None, output_final_state=True,
+                        stream=None):
+    """kda_prefill without a workspace: the library's own fixed device array
+    serves as scratch (see include/kda.h).  Same shapes and results as
+    kda_prefill; calls that overlap on the GPU must be serialised."""
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is not None:
+        n = cu_seqlens.numel() - 1
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+    else:
+        n = 1 if num_seqs is None else int(num_seqs)
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check_cuda(q, k, v, log_alpha, beta, init_state, cu_seqlens, o, final_state)
+    st = lib().kda_prefill_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
+        _ptr(cu_seqlens), n, T, H, dk, dv, _dtype_code(q), _ptr(o), _ptr(final_state),
+        _stream(stream, q.device))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_prefill_noalloc")
+    return o, final_state

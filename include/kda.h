@@ -153,6 +153,37 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
 kda_status kda_check_workspace_error(const void *workspace,
                                      kda_stream_t stream);
 
+/*
+ * kda_prefill without a workspace argument, for callers that cannot allocate
+ * device memory when they run the operator (an engine whose device memory
+ * all belongs to its own pool, a loop that cannot afford cudaMalloc's
+ * synchronisation, a plugin host that passes only a stream and tensors).
+ * This call has no counterpart in the method's description; it is a
+ * deployment convenience.
+ *
+ * Same arguments, results and errors as kda_prefill, minus the workspace.
+ * The scratch it needs (the error word and the sequence-order table) lives
+ * in a fixed array of this library's device memory, 256 + 4 *
+ * KDA_NOALLOC_MAX_SEQS bytes, which every GPU that loads the library holds
+ * until the process exits.  num_seqs above KDA_NOALLOC_MAX_SEQS returns
+ * KDA_ERR_UNSUPPORTED.  It calls no allocating function.
+ *
+ * The first call on a device (with that device current) looks up the
+ * array's device address and caches it; make that first call before any
+ * stream capture.  All calls share the one array: calls that may overlap on
+ * the GPU (different streams, or several host threads) race on it and must
+ * be serialised by the caller.  kda_check_workspace_error cannot be used
+ * with this entry point.
+ */
+#define KDA_NOALLOC_MAX_SEQS 4096
+
+kda_status kda_prefill_noalloc(const void *q, const void *k, const void *v,
+                               const void *log_alpha, const void *beta,
+                               const float *init_state, const int32_t *cu_seqlens,
+                               int32_t num_seqs, int64_t total_tokens, int32_t H,
+                               int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                               float *final_state, kda_stream_t stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif
