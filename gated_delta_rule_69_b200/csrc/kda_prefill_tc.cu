@@ -77,12 +77,12 @@ struct Smem {
     static constexpr uint32_t SB = 204800;        // 8 KB: S bf16 [128 c][32 j] (64-byte rows)
     static constexpr uint32_t VT = 212992;        // 2 x 4 KB: V [64 t][32 j]
     static constexpr uint32_t UB = 221184;        // 4 KB: U bf16 [64 t][32 j]
-    static constexpr uint32_t BETA = 225280;      // 64 fp32
-    static constexpr uint32_t EGL = 225536;       // 2 x 128 fp32: exp(G_L) per stage
-    static constexpr uint32_t CSUM = 226560;      // 4 x 128 fp32: running-sum partials
-    static constexpr uint32_t BARS = 228608;      // mbarriers
-    static constexpr uint32_t MISC = 228864;      // tmem base, flags
-    static constexpr uint32_t SIZE = 228928;
+    static constexpr uint32_t BETA = 225280;      // 2 x 64 fp32: beta per stage (zero past the end)
+    static constexpr uint32_t EGL = 225792;       // 2 x 128 fp32: exp(G_L) per stage
+    static constexpr uint32_t CSUM = 226816;      // 4 x 128 fp32: running-sum partials
+    static constexpr uint32_t BARS = 228864;      // mbarriers
+    static constexpr uint32_t MISC = 229120;      // tmem base, flags
+    static constexpr uint32_t SIZE = 229184;
     static constexpr uint32_t ALLOC = SIZE + 1024;  // room to align the base
 };
 static_assert(Smem::ALLOC <= 232448, "shared memory budget");
@@ -136,30 +136,38 @@ __device__ __forceinline__ int fidx(int t, int i) { return t * 64 + (i ^ (t & 31
 
 // ---- preparation step 1: running sums of log_alpha and the gated operands.
 // Thread pt (0..255) owns channels c, c+1 (c = 2 (pt mod 64)) for the 16
-// tokens of group pt / 64.  Returns whether the chunk takes the pairwise path.
-__device__ bool prep_gate(uint8_t *sm, int pt, int s, int L, const Params &p, int64_t tok0,
-                          int h) {
+// tokens of group pt / 64; a warp covers one 64-channel K-atom of one token
+// group, so every shared-memory access below is a full 128-byte row.
+// Returns whether the chunk takes the pairwise path.
+__device__ bool prep_gate(uint8_t *__restrict__ sm, int pt, int s, int L) {
     const int c = 2 * (pt & 63);
     const int tg = pt >> 6;
     const int t0 = tg * 16;
     float *csum = reinterpret_cast<float *>(sm + Smem::CSUM);
     uint32_t *flags = misc(sm);
     const uint8_t *graw = sm + Smem::GRAW + s * 16384;
+    const int katom = c >> 6, cc = c & 63;
+    uint8_t *stack = sm + Smem::STACK + s * 32768 + katom * 16384;
+    uint8_t *khat = sm + Smem::KHAT + katom * 8192;
+    uint8_t *kbar = sm + Smem::KBAR + s * 16384 + katom * 8192;
 
+    // issue every load of this thread's slice first
+    uint32_t graw_v[16], k_v[16], q_v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int t = t0 + i;
+        graw_v[i] = *reinterpret_cast<const uint32_t *>(graw + t * 256 + c * 2);
+        k_v[i] = *reinterpret_cast<const uint32_t *>(stack + sw128_off(t, cc));
+        q_v[i] = *reinterpret_cast<const uint32_t *>(stack + sw128_off(64 + t, cc));
+    }
     float g0[16], g1[16];
     float r0 = 0.f, r1 = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        const int t = t0 + i;
-        float a = 0.f, b = 0.f;
-        if (t < L) {
-            const __nv_bfloat162 gv =
-                *reinterpret_cast<const __nv_bfloat162 *>(graw + t * 256 + c * 2);
-            a = clamp_log_alpha(__low2float(gv));
-            b = clamp_log_alpha(__high2float(gv));
-        }
-        r0 += a;
-        r1 += b;
+        const bool valid = t0 + i < L;
+        const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162 *>(&graw_v[i]);
+        r0 += valid ? clamp_log_alpha(__low2float(gv)) : 0.f;
+        r1 += valid ? clamp_log_alpha(__high2float(gv)) : 0.f;
         g0[i] = r0;
         g1[i] = r1;
     }
@@ -186,21 +194,14 @@ __device__ bool prep_gate(uint8_t *sm, int pt, int s, int L, const Params &p, in
         egl[c] = eL0;
         egl[c + 1] = eL1;
     }
-    const int katom = c >> 6, cc = c & 63;
-    uint8_t *stack = sm + Smem::STACK + s * 32768 + katom * 16384;
-    uint8_t *khat = sm + Smem::KHAT + katom * 8192;
-    uint8_t *kbar = sm + Smem::KBAR + s * 16384 + katom * 8192;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int t = t0 + i;
-        const uint32_t ok = sw128_off(t, cc), oq = sw128_off(64 + t, cc);
-        float k0 = 0.f, k1 = 0.f, q0 = 0.f, q1 = 0.f;
-        if (t < L) {
-            const __nv_bfloat162 kv = *reinterpret_cast<const __nv_bfloat162 *>(stack + ok);
-            const __nv_bfloat162 qv = *reinterpret_cast<const __nv_bfloat162 *>(stack + oq);
-            k0 = __low2float(kv); k1 = __high2float(kv);
-            q0 = __low2float(qv); q1 = __high2float(qv);
-        }
+        const bool valid = t < L;
+        const __nv_bfloat162 kv = *reinterpret_cast<const __nv_bfloat162 *>(&k_v[i]);
+        const __nv_bfloat162 qv = *reinterpret_cast<const __nv_bfloat162 *>(&q_v[i]);
+        const float k0 = valid ? __low2float(kv) : 0.f, k1 = valid ? __high2float(kv) : 0.f;
+        const float q0 = valid ? __low2float(qv) : 0.f, q1 = valid ? __high2float(qv) : 0.f;
         const float G0 = g0[i] + off0, G1 = g1[i] + off1;
         const float e0 = exp_f(G0), e1 = exp_f(G1);
         const float ih0 = exp_f(fminf(-G0, 80.f)), ih1 = exp_f(fminf(-G1, 80.f));
@@ -212,15 +213,11 @@ __device__ bool prep_gate(uint8_t *sm, int pt, int s, int L, const Params &p, in
             b0 = eL0 * ih0;
             b1 = eL1 * ih1;
         }
+        const uint32_t ok = sw128_off(t, cc);
         *reinterpret_cast<uint32_t *>(stack + ok) = pack_bf16x2(k0 * e0, k1 * e1);
-        *reinterpret_cast<uint32_t *>(stack + oq) = pack_bf16x2(q0 * e0, q1 * e1);
+        *reinterpret_cast<uint32_t *>(stack + sw128_off(64 + t, cc)) = pack_bf16x2(q0 * e0, q1 * e1);
         *reinterpret_cast<uint32_t *>(khat + ok) = pack_bf16x2(k0 * ih0, k1 * ih1);
         *reinterpret_cast<uint32_t *>(kbar + ok) = pack_bf16x2(k0 * b0, k1 * b1);
-    }
-    if (pt < C) {
-        float b = 0.f;
-        if (pt < L) b = __bfloat162float(p.beta[(size_t)(tok0 + pt) * p.H + h]);
-        reinterpret_cast<float *>(sm + Smem::BETA)[pt] = b;
     }
     return slow;
 }
@@ -230,7 +227,7 @@ __device__ bool prep_gate(uint8_t *sm, int pt, int s, int L, const Params &p, in
 __device__ void prep_pairwise(uint8_t *sm, int pt, int s, int L, const Params &p,
                               int64_t tok0, int h) {
     const uint8_t *graw = sm + Smem::GRAW + s * 16384;
-    const float *beta = reinterpret_cast<const float *>(sm + Smem::BETA);
+    const float *beta = reinterpret_cast<const float *>(sm + Smem::BETA) + s * C;
     float *AF = reinterpret_cast<float *>(sm + Smem::KHAT);
     uint8_t *pb = sm + Smem::PB + s * 8192;
     for (int pidx = pt; pidx < C * C; pidx += kPrepThreads) {
@@ -263,7 +260,7 @@ __device__ void prep_read_ap(uint8_t *sm, uint32_t tmem, int warp, int lane, int
     float v[32];
     tmem_ld32(tmem_addr(tmem, 32 * quad, kColAP + 32 * half), v);
     tmem_wait_ld();
-    const float *beta = reinterpret_cast<const float *>(sm + Smem::BETA);
+    const float *beta = reinterpret_cast<const float *>(sm + Smem::BETA) + s * C;
     if (quad < 2) {
         float *AF = reinterpret_cast<float *>(sm + Smem::KHAT);
         const int t = 32 * quad + lane;
@@ -293,63 +290,90 @@ __device__ void prep_read_ap(uint8_t *sm, uint32_t tmem, int warp, int lane, int
 
 // ---- preparation step 3: T = (I + A)^{-1} for the unit lower-triangular
 // 64x64 system, by blocks of 16: the four diagonal blocks by forward
-// substitution (one warp each), then the off-diagonal blocks by increasing
-// distance from the diagonal, T_ab = -T_aa sum_{c=b}^{a-1} A_ac T_cb.
-// Writes T diag(beta) as bf16 into TB.
-__device__ void prep_solve(uint8_t *sm, int pt, int s) {
-    const float *AF = reinterpret_cast<const float *>(sm + Smem::KHAT);
-    float *TF = reinterpret_cast<float *>(sm + Smem::TF);
-    float *XF = reinterpret_cast<float *>(sm + Smem::GRAW + s * 16384);  // raw g is spent
-    const float *beta = reinterpret_cast<const float *>(sm + Smem::BETA);
-    const int pw = pt >> 5, lane = pt & 31;
+// substitution (one thread per column), then the off-diagonal blocks by
+// increasing distance d from the diagonal,
+//     X_ab = sum_{c=b}^{a-1} A_ac T_cb,   T_ab = -T_aa X_ab,   a = b + d,
+// each thread producing a 1x4 row segment.  Writes T diag(beta) as bf16 into TB.
 
-    if (pw < 4) {
-        if (lane < 16) {
-            const int a = pw, j = lane, base = 16 * a;
-            float x[16];
+// T tile layout: rows of 64 floats; the float4 group index is XORed with
+// (row mod 16), so that row segments load as float4 and threads on
+// different rows hit different banks.
+__device__ __forceinline__ int tfi(int row, int col) {
+    return row * 64 + ((((col >> 2) ^ (row & 15))) << 2) + (col & 3);
+}
+
+__device__ void prep_solve(uint8_t *__restrict__ sm, int pt, int s) {
+    const float *__restrict__ AF = reinterpret_cast<const float *>(sm + Smem::KHAT);
+    float *__restrict__ TF = reinterpret_cast<float *>(sm + Smem::TF);
+    float *__restrict__ XF = reinterpret_cast<float *>(sm + Smem::GRAW + s * 16384);  // raw g is spent
+    const float *__restrict__ beta = reinterpret_cast<const float *>(sm + Smem::BETA) + s * C;
+
+    if (pt < 64) {
+        const int a = pt >> 4, j = pt & 15, base = 16 * a;
+        float x[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = 0.f;
+        for (int r = 0; r < 16; ++r) {
+            float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < r; ++i) acc = fmaf(AF[fidx(base + r, base + i)], x[i], acc);
-                x[r] = (r == j) ? 1.f : ((r < j) ? 0.f : -acc);
+            for (int i = 0; i < r; ++i) {
+                const float av = AF[fidx(base + r, base + i)];
+                if (i & 1) acc1 = fmaf(av, x[i], acc1);
+                else acc0 = fmaf(av, x[i], acc0);
             }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) TF[fidx(base + r, base + j)] = x[r];
+            x[r] = (r == j) ? 1.f : ((r < j) ? 0.f : -(acc0 + acc1));
         }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) TF[tfi(base + r, base + j)] = x[r];
     } else {
-        // zero the six blocks above the diagonal
-        for (int e = pt - 128; e < 6 * 256; e += 128) {
-            const int blk = e >> 8, r = (e >> 4) & 15, col = e & 15;
+        // zero the six blocks above the diagonal (384 float4)
+        for (int v = pt - 64; v < 384; v += kPrepThreads - 64) {
+            const int blk = v >> 6, r = (v >> 2) & 15, c4 = (v & 3) * 4;
             const int a = (blk < 3) ? 0 : (blk < 5 ? 1 : 2);
             const int b = (blk < 3) ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            TF[fidx(16 * a + r, 16 * b + col)] = 0.f;
+            *reinterpret_cast<float4 *>(&TF[tfi(16 * a + r, 16 * b + c4)]) =
+                make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
     named_barrier(kBarPrep, kPrepThreads);
 
+#pragma unroll 1
     for (int d = 1; d <= 3; ++d) {
-        const int nblk = 4 - d;
-        // X_ab = sum_{c=b}^{a-1} A_ac T_cb  for (a, b) = (b + d, b)
-        for (int e = pt; e < nblk * 256; e += kPrepThreads) {
-            const int b = e >> 8, a = b + d, r = (e >> 4) & 15, col = e & 15;
-            float acc = 0.f;
-            for (int c = b; c < a; ++c) {
+        const int nthr = (4 - d) * 64;
+        const int blk = pt >> 6, r = (pt >> 2) & 15, c4 = (pt & 3) * 4;
+        const int b = blk, a = b + d;
+        if (pt < nthr) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int cb = b; cb < a; ++cb) {
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    acc = fmaf(AF[fidx(16 * a + r, 16 * c + k)], TF[fidx(16 * c + k, 16 * b + col)], acc);
+                for (int k = 0; k < 16; ++k) {
+                    const float av = AF[fidx(16 * a + r, 16 * cb + k)];
+                    const float4 tv = *reinterpret_cast<const float4 *>(&TF[tfi(16 * cb + k, 16 * b + c4)]);
+                    acc.x = fmaf(av, tv.x, acc.x);
+                    acc.y = fmaf(av, tv.y, acc.y);
+                    acc.z = fmaf(av, tv.z, acc.z);
+                    acc.w = fmaf(av, tv.w, acc.w);
+                }
             }
-            XF[e] = acc;
+            *reinterpret_cast<float4 *>(&XF[(blk * 16 + r) * 16 + c4]) = acc;
         }
         named_barrier(kBarPrep, kPrepThreads);
-        // T_ab = -T_aa X_ab
-        for (int e = pt; e < nblk * 256; e += kPrepThreads) {
-            const int b = e >> 8, a = b + d, r = (e >> 4) & 15, col = e & 15;
-            float acc = 0.f;
+        if (pt < nthr) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-                acc = fmaf(TF[fidx(16 * a + r, 16 * a + k)], XF[(b << 8) + (k << 4) + col], acc);
-            TF[fidx(16 * a + r, 16 * b + col)] = -acc;
+            for (int k4 = 0; k4 < 16; k4 += 4) {
+                const float4 tr = *reinterpret_cast<const float4 *>(&TF[tfi(16 * a + r, 16 * a + k4)]);
+                const float tk[4] = {tr.x, tr.y, tr.z, tr.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float4 xv = *reinterpret_cast<const float4 *>(&XF[(blk * 16 + k4 + e) * 16 + c4]);
+                    acc.x = fmaf(tk[e], xv.x, acc.x);
+                    acc.y = fmaf(tk[e], xv.y, acc.y);
+                    acc.z = fmaf(tk[e], xv.z, acc.z);
+                    acc.w = fmaf(tk[e], xv.w, acc.w);
+                }
+            }
+            *reinterpret_cast<float4 *>(&TF[tfi(16 * a + r, 16 * b + c4)]) =
+                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
         }
         named_barrier(kBarPrep, kPrepThreads);
     }
@@ -359,17 +383,14 @@ __device__ void prep_solve(uint8_t *sm, int pt, int s) {
     const int t = pt >> 2, i0 = (pt & 3) * 16;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-        float w[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int i = i0 + 8 * hh + e;
-            w[e] = TF[fidx(t, i)] * beta[i];
-        }
+        const float4 u0 = *reinterpret_cast<const float4 *>(&TF[tfi(t, i0 + 8 * hh)]);
+        const float4 u1 = *reinterpret_cast<const float4 *>(&TF[tfi(t, i0 + 8 * hh + 4)]);
+        const float *bb = beta + i0 + 8 * hh;
         uint4 pk;
-        pk.x = pack_bf16x2(w[0], w[1]);
-        pk.y = pack_bf16x2(w[2], w[3]);
-        pk.z = pack_bf16x2(w[4], w[5]);
-        pk.w = pack_bf16x2(w[6], w[7]);
+        pk.x = pack_bf16x2(u0.x * bb[0], u0.y * bb[1]);
+        pk.y = pack_bf16x2(u0.z * bb[2], u0.w * bb[3]);
+        pk.z = pack_bf16x2(u1.x * bb[4], u1.y * bb[5]);
+        pk.w = pack_bf16x2(u1.z * bb[6], u1.w * bb[7]);
         *reinterpret_cast<uint4 *>(tb + sw128_off(t, i0 + 8 * hh)) = pk;
     }
 }
@@ -483,7 +504,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
     volatile uint32_t *abort_flag = flags + 1;
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i)
-            mbar_init(&B[i], (i == RAW_EMPTY || i == RAW_EMPTY + 1) ? 2u : 1u);
+            mbar_init(&B[i], (i == RAW_EMPTY || i == RAW_EMPTY + 1 || i == RAW_FULL ||
+                                  i == RAW_FULL + 1) ? 2u : 1u);
         flags[1] = 0u;
         flags[2] = 0u;
         fence_mbar_init();
@@ -499,30 +521,54 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0 && nchunks > 0) {
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_g);
-            tma_prefetch_desc(&tm_v);
+        // Lane 0 issues the tensor copies; the whole warp then loads the
+        // chunk's 64 beta values (a strided gather TMA cannot do) into the
+        // matching ring slot and lane 0 adds the second arrival.
+        if (nchunks > 0) {
+            if (lane == 0) {
+                tma_prefetch_desc(&tm_k);
+                tma_prefetch_desc(&tm_q);
+                tma_prefetch_desc(&tm_g);
+                tma_prefetch_desc(&tm_v);
+            }
+            float *betar = reinterpret_cast<float *>(sm + Smem::BETA);
             int issued = 0;
             for (int n = 0; n < nchunks; ++n) {
                 const int s = n & 1;
-                if (n >= 2) mbar_wait(&B[RAW_EMPTY + s], ((n - 2) >> 1) & 1, abort_flag);
-                if (*abort_flag) break;
-                mbar_arrive_expect_tx(&B[RAW_FULL + s], kRawBytes);
+                int stop = 0;
+                if (lane == 0) {
+                    if (n >= 2) mbar_wait(&B[RAW_EMPTY + s], ((n - 2) >> 1) & 1, abort_flag);
+                    stop = *abort_flag ? 1 : 0;
+                }
+                stop = __shfl_sync(0xffffffffu, stop, 0);
+                if (stop) break;
                 const int tok = (int)(bos + (int64_t)n * C);
-                uint8_t *stk = sm + Smem::STACK + s * 32768;
-                tma_load_3d(stk, &tm_k, &B[RAW_FULL + s], 0, h, tok);
-                tma_load_3d(stk + 16384, &tm_k, &B[RAW_FULL + s], 64, h, tok);
-                tma_load_3d(stk + 8192, &tm_q, &B[RAW_FULL + s], 0, h, tok);
-                tma_load_3d(stk + 16384 + 8192, &tm_q, &B[RAW_FULL + s], 64, h, tok);
-                tma_load_3d(sm + Smem::GRAW + s * 16384, &tm_g, &B[RAW_FULL + s], 0, h, tok);
-                tma_load_3d(sm + Smem::VT + s * 4096, &tm_v, &B[RAW_FULL + s], j0, h, tok);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&B[RAW_FULL + s], kRawBytes);
+                    uint8_t *stk = sm + Smem::STACK + s * 32768;
+                    tma_load_3d(stk, &tm_k, &B[RAW_FULL + s], 0, h, tok);
+                    tma_load_3d(stk + 16384, &tm_k, &B[RAW_FULL + s], 64, h, tok);
+                    tma_load_3d(stk + 8192, &tm_q, &B[RAW_FULL + s], 0, h, tok);
+                    tma_load_3d(stk + 16384 + 8192, &tm_q, &B[RAW_FULL + s], 64, h, tok);
+                    tma_load_3d(sm + Smem::GRAW + s * 16384, &tm_g, &B[RAW_FULL + s], 0, h, tok);
+                    tma_load_3d(sm + Smem::VT + s * 4096, &tm_v, &B[RAW_FULL + s], j0, h, tok);
+                }
+                const int64_t rem = len - (int64_t)n * C;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int t = lane + 32 * e;
+                    float b = 0.f;
+                    if (t < rem) b = __bfloat162float(p.beta[(size_t)(tok + t) * p.H + h]);
+                    betar[s * C + t] = b;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&B[RAW_FULL + s]);
                 issued = n + 1;
             }
             // every issued copy must have landed before the CTA's memory is released
-            for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n)
-                mbar_wait_drain(&B[RAW_FULL + (n & 1)], (n >> 1) & 1);
+            if (lane == 0)
+                for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n)
+                    mbar_wait_drain(&B[RAW_FULL + (n & 1)], (n >> 1) & 1);
         }
     } else if (warp < kPrepWarp0) {
         // ------------------------------------------------ state chain
@@ -639,7 +685,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
             const int64_t tok0 = bos + (int64_t)n * C;
             mbar_wait(&B[RAW_FULL + s], (n >> 1) & 1, abort_flag);
             if (n >= 2) mbar_wait(&B[CHAIN_DONE + s], ((n - 2) >> 1) & 1, abort_flag);
-            const bool slow = prep_gate(sm, pt, s, L, p, tok0, h);
+            const bool slow = prep_gate(sm, pt, s, L);
             fence_async_smem();
             named_barrier(kBarPrep, kPrepThreads);
             if (leader) {

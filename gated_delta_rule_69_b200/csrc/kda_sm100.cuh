@@ -49,6 +49,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep up to `hint_ns` (it is woken
+// when the phase completes), so a waiting warp takes no issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns) : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Gives up
 // after `limit_ns` of wall time, or at once when *abort is already set;
 // on giving up it sets *abort (shared by the CTA) and returns false.  After
@@ -59,11 +72,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           uint64_t limit_ns = 2000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
-    uint32_t spins = 0;
     while (true) {
         if (*abort) return false;
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((++spins & 255u) == 0 && global_timer_ns() - t0 > limit_ns) {
+        if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+        if (global_timer_ns() - t0 > limit_ns) {
             *abort = 1u;
             return false;
         }
