@@ -60,20 +60,23 @@ constexpr float kSlowPathLogDecay = -60.0f;   // chunk log-decay below this -> p
 // TMEM column map (lane = row of the accumulator)
 constexpr uint32_t kColAP = 0;     // [Ktil;Qtil] Khat^T : M=128, N=64
 constexpr uint32_t kColW = 64;     // T_beta Ktil        : M=64,  N=128
-constexpr uint32_t kColU = 192;    // U (x2 stages)      : M=64,  N=32
-constexpr uint32_t kColO = 256;    // O (x2 stages)      : M=64,  N=32
+constexpr uint32_t kColUp = 192;   // U' (x2 stages)     : M=128, N=32 (rows 0-63 used)
+constexpr uint32_t kColUO = 256;   // [-W S; O] (x2)     : M=128, N=32 (rows 0-63: -W S, 64-127: O)
 constexpr uint32_t kColS = 320;    // state              : M=128, N=32
 
 // Shared memory map (bytes from a 1024-aligned base)
 struct Smem {
     static constexpr uint32_t STACK = 0;          // 2 x 32 KB: [Ktil rows 0-63 | Qtil rows 64-127] x 2 K-atoms
     static constexpr uint32_t KBAR = 65536;       // 2 x 16 KB: Kbar [64 t][128 c], 2 K-atoms of 8 KB
-    static constexpr uint32_t KHAT = 98304;       // 16 KB Khat; reused as A (fp32 64x64) after the product
-    static constexpr uint32_t WB = 114688;        // 16 KB: -W [64 t][128 c]
+    static constexpr uint32_t KHAT = 98304;       // 16 KB Khat [64 i][128 c]
+    static constexpr uint32_t AF = 114688;        // 16 KB: A fp32 64x64 (row-XOR layout)
     static constexpr uint32_t TF = 131072;        // 16 KB: T fp32 64x64
     static constexpr uint32_t GRAW = 147456;      // 2 x 16 KB: raw log_alpha [64 t][128 c]
     static constexpr uint32_t TB = 180224;        // 8 KB: T diag(beta), bf16 [64 t][64 i]
     static constexpr uint32_t PB = 188416;        // 2 x 8 KB: P bf16 [64 t][64 i]
+    // TB, PB[0], PB[1] are contiguous: an M = 128 operand that starts 64 rows
+    // before PB[s] (or at TB) reads rows 64-127 from PB[s] (or PB[0]); the
+    // first 64 rows only feed accumulator rows that are never read.
     static constexpr uint32_t SB = 204800;        // 8 KB: S bf16 [128 c][32 j] (64-byte rows)
     static constexpr uint32_t VT = 212992;        // 2 x 4 KB: V [64 t][32 j]
     static constexpr uint32_t UB = 221184;        // 4 KB: U bf16 [64 t][32 j]
@@ -94,9 +97,9 @@ enum Bar : int {
     GATE_READY = 4,   // [2] prep -> chain (exp(G_L) ready; Ktil/Qtil/Kbar written)
     AP_FULL = 6,      // product [A;P] done -> prep
     W_FULL = 7,       // W and U' products done -> prep
-    WB_READY = 8,     // -W written -> chain
-    ACCU_EMPTY = 9,   // [2] chain read U -> prep may write U' again
-    U_FULL = 11,      // [2] U = U' - W S done -> chain, prep
+    WB_READY = 8,     // -W written over Ktil in STACK[s] -> chain
+    ACCU_EMPTY = 9,   // [2] chain read U' -> prep may write U' again
+    U_FULL = 11,      // [2] [-W; Qtil] S done -> chain
     CHAIN_DONE = 13,  // [2] state update + output products done -> chain, prep
     FINAL = 15,       // end-of-kernel drain of this thread's MMAs
     FINAL2 = 16,
@@ -118,7 +121,14 @@ struct Params {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ float exp_f(float x) { return exp2f(x * kLog2e); }
+// e^x through the hardware base-2 exponential (ex2.approx, flush-to-zero):
+// its relative error (~2^-22) is far below the bf16 rounding of the operands
+// it scales.
+__device__ __forceinline__ float exp_f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * kLog2e));
+    return y;
+}
 
 __device__ __forceinline__ uint64_t *bars(uint8_t *sm) {
     return reinterpret_cast<uint64_t *>(sm + Smem::BARS);
@@ -228,7 +238,7 @@ __device__ void prep_pairwise(uint8_t *sm, int pt, int s, int L, const Params &p
                               int64_t tok0, int h) {
     const uint8_t *graw = sm + Smem::GRAW + s * 16384;
     const float *beta = reinterpret_cast<const float *>(sm + Smem::BETA) + s * C;
-    float *AF = reinterpret_cast<float *>(sm + Smem::KHAT);
+    float *AF = reinterpret_cast<float *>(sm + Smem::AF);
     uint8_t *pb = sm + Smem::PB + s * 8192;
     for (int pidx = pt; pidx < C * C; pidx += kPrepThreads) {
         const int t = pidx >> 6, i = pidx & 63;
@@ -262,7 +272,7 @@ __device__ void prep_read_ap(uint8_t *sm, uint32_t tmem, int warp, int lane, int
     tmem_wait_ld();
     const float *beta = reinterpret_cast<const float *>(sm + Smem::BETA) + s * C;
     if (quad < 2) {
-        float *AF = reinterpret_cast<float *>(sm + Smem::KHAT);
+        float *AF = reinterpret_cast<float *>(sm + Smem::AF);
         const int t = 32 * quad + lane;
         const float bt = beta[t];
 #pragma unroll
@@ -289,11 +299,12 @@ __device__ void prep_read_ap(uint8_t *sm, uint32_t tmem, int warp, int lane, int
 }
 
 // ---- preparation step 3: T = (I + A)^{-1} for the unit lower-triangular
-// 64x64 system, by blocks of 16: the four diagonal blocks by forward
-// substitution (one thread per column), then the off-diagonal blocks by
-// increasing distance d from the diagonal,
-//     X_ab = sum_{c=b}^{a-1} A_ac T_cb,   T_ab = -T_aa X_ab,   a = b + d,
-// each thread producing a 1x4 row segment.  Writes T diag(beta) as bf16 into TB.
+// 64x64 system by recursive doubling: the sixteen 4x4 diagonal blocks in
+// closed form (forward substitution written out), then four merge levels that
+// combine neighbouring m x m inverses into 2m x 2m ones,
+//     [[T1, 0], [T21, T2]],   T21 = -T2 (A21 T1),
+// for m = 4, 8, 16, 32.  Each level is two fully parallel products (one 1x4
+// row segment per thread).  Writes T diag(beta) as bf16 into TB.
 
 // T tile layout: rows of 64 floats; the float4 group index is XORed with
 // (row mod 16), so that row segments load as float4 and threads on
@@ -302,81 +313,82 @@ __device__ __forceinline__ int tfi(int row, int col) {
     return row * 64 + ((((col >> 2) ^ (row & 15))) << 2) + (col & 3);
 }
 
+template <int M>
+__device__ __forceinline__ void solve_merge(const float *__restrict__ AF, float *__restrict__ TF,
+                                            float *__restrict__ XF, int pt) {
+    constexpr int kThr = 8 * M;               // (64 / 2M) merges x M x (M / 4) segments
+    const int merge = pt / (M * M / 4);
+    const int rem = pt % (M * M / 4);
+    const int r = rem / (M / 4), c4 = (rem % (M / 4)) * 4;
+    const int base = merge * 2 * M;
+    if (pt < kThr) {   // X = A21 T1
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < M; ++k) {
+            const float av = AF[fidx(base + M + r, base + k)];
+            const float4 tv = *reinterpret_cast<const float4 *>(&TF[tfi(base + k, base + c4)]);
+            acc.x = fmaf(av, tv.x, acc.x);
+            acc.y = fmaf(av, tv.y, acc.y);
+            acc.z = fmaf(av, tv.z, acc.z);
+            acc.w = fmaf(av, tv.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(&XF[(merge * M + r) * M + c4]) = acc;
+    }
+    named_barrier(kBarPrep, kPrepThreads);
+    if (pt < kThr) {   // T21 = -T2 X
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k4 = 0; k4 < M; k4 += 4) {
+            const float4 tr = *reinterpret_cast<const float4 *>(&TF[tfi(base + M + r, base + M + k4)]);
+            const float tk[4] = {tr.x, tr.y, tr.z, tr.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float4 xv = *reinterpret_cast<const float4 *>(&XF[(merge * M + k4 + e) * M + c4]);
+                acc.x = fmaf(tk[e], xv.x, acc.x);
+                acc.y = fmaf(tk[e], xv.y, acc.y);
+                acc.z = fmaf(tk[e], xv.z, acc.z);
+                acc.w = fmaf(tk[e], xv.w, acc.w);
+            }
+        }
+        *reinterpret_cast<float4 *>(&TF[tfi(base + M + r, base + c4)]) =
+            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    named_barrier(kBarPrep, kPrepThreads);
+}
+
 __device__ void prep_solve(uint8_t *__restrict__ sm, int pt, int s) {
-    const float *__restrict__ AF = reinterpret_cast<const float *>(sm + Smem::KHAT);
+    const float *__restrict__ AF = reinterpret_cast<const float *>(sm + Smem::AF);
     float *__restrict__ TF = reinterpret_cast<float *>(sm + Smem::TF);
     float *__restrict__ XF = reinterpret_cast<float *>(sm + Smem::GRAW + s * 16384);  // raw g is spent
     const float *__restrict__ beta = reinterpret_cast<const float *>(sm + Smem::BETA) + s * C;
 
-    if (pt < 64) {
-        const int a = pt >> 4, j = pt & 15, base = 16 * a;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-            for (int i = 0; i < r; ++i) {
-                const float av = AF[fidx(base + r, base + i)];
-                if (i & 1) acc1 = fmaf(av, x[i], acc1);
-                else acc0 = fmaf(av, x[i], acc0);
-            }
-            x[r] = (r == j) ? 1.f : ((r < j) ? 0.f : -(acc0 + acc1));
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) TF[tfi(base + r, base + j)] = x[r];
-    } else {
-        // zero the six blocks above the diagonal (384 float4)
-        for (int v = pt - 64; v < 384; v += kPrepThreads - 64) {
-            const int blk = v >> 6, r = (v >> 2) & 15, c4 = (v & 3) * 4;
-            const int a = (blk < 3) ? 0 : (blk < 5 ? 1 : 2);
-            const int b = (blk < 3) ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            *reinterpret_cast<float4 *>(&TF[tfi(16 * a + r, 16 * b + c4)]) =
-                make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+    // zero every float4 group of T outside the 4x4 diagonal blocks
+    for (int v = pt; v < 1024; v += kPrepThreads) {
+        const int row = v >> 4, g4 = v & 15;
+        if (g4 != (row >> 2))
+            *reinterpret_cast<float4 *>(&TF[tfi(row, 4 * g4)]) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // 4x4 diagonal blocks: T = L^{-1} for unit lower-triangular L = I + N
+    if (pt < 16) {
+        const int b0 = 4 * pt;
+        const float n10 = AF[fidx(b0 + 1, b0)];
+        const float n20 = AF[fidx(b0 + 2, b0)], n21 = AF[fidx(b0 + 2, b0 + 1)];
+        const float n30 = AF[fidx(b0 + 3, b0)], n31 = AF[fidx(b0 + 3, b0 + 1)],
+                    n32 = AF[fidx(b0 + 3, b0 + 2)];
+        const float t10 = -n10, t21 = -n21, t32 = -n32;
+        const float t20 = -(n20 + n21 * t10);
+        const float t31 = -(n31 + n32 * t21);
+        const float t30 = -(n30 + n31 * t10 + n32 * t20);
+        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 0, b0)]) = make_float4(1.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 1, b0)]) = make_float4(t10, 1.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 2, b0)]) = make_float4(t20, t21, 1.f, 0.f);
+        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 3, b0)]) = make_float4(t30, t31, t32, 1.f);
     }
     named_barrier(kBarPrep, kPrepThreads);
-
-#pragma unroll 1
-    for (int d = 1; d <= 3; ++d) {
-        const int nthr = (4 - d) * 64;
-        const int blk = pt >> 6, r = (pt >> 2) & 15, c4 = (pt & 3) * 4;
-        const int b = blk, a = b + d;
-        if (pt < nthr) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int cb = b; cb < a; ++cb) {
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float av = AF[fidx(16 * a + r, 16 * cb + k)];
-                    const float4 tv = *reinterpret_cast<const float4 *>(&TF[tfi(16 * cb + k, 16 * b + c4)]);
-                    acc.x = fmaf(av, tv.x, acc.x);
-                    acc.y = fmaf(av, tv.y, acc.y);
-                    acc.z = fmaf(av, tv.z, acc.z);
-                    acc.w = fmaf(av, tv.w, acc.w);
-                }
-            }
-            *reinterpret_cast<float4 *>(&XF[(blk * 16 + r) * 16 + c4]) = acc;
-        }
-        named_barrier(kBarPrep, kPrepThreads);
-        if (pt < nthr) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int k4 = 0; k4 < 16; k4 += 4) {
-                const float4 tr = *reinterpret_cast<const float4 *>(&TF[tfi(16 * a + r, 16 * a + k4)]);
-                const float tk[4] = {tr.x, tr.y, tr.z, tr.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float4 xv = *reinterpret_cast<const float4 *>(&XF[(blk * 16 + k4 + e) * 16 + c4]);
-                    acc.x = fmaf(tk[e], xv.x, acc.x);
-                    acc.y = fmaf(tk[e], xv.y, acc.y);
-                    acc.z = fmaf(tk[e], xv.z, acc.z);
-                    acc.w = fmaf(tk[e], xv.w, acc.w);
-                }
-            }
-            *reinterpret_cast<float4 *>(&TF[tfi(16 * a + r, 16 * b + c4)]) =
-                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-        }
-        named_barrier(kBarPrep, kPrepThreads);
-    }
+    solve_merge<4>(AF, TF, XF, pt);
+    solve_merge<8>(AF, TF, XF, pt);
+    solve_merge<16>(AF, TF, XF, pt);
+    solve_merge<32>(AF, TF, XF, pt);
 
     // T diag(beta) -> bf16, K-major 128-byte-swizzled [64 t][64 i]
     uint8_t *tb = sm + Smem::TB;
@@ -396,10 +408,11 @@ __device__ void prep_solve(uint8_t *__restrict__ sm, int pt, int s) {
 }
 
 // ---- preparation step 4: -W from TMEM (M = 64 layout: row r sits in lane
-// (r mod 16) + 32 (r / 16)) into WB as bf16, K-major [64 t][128 c].
-__device__ void prep_read_w(uint8_t *sm, uint32_t tmem, int warp, int lane) {
+// (r mod 16) + 32 (r / 16)) as bf16 over Ktil, i.e. rows 0-63 of STACK[s]
+// (K-major, 64 channels per K-atom), so that [-W; Qtil] is one M = 128 operand.
+__device__ void prep_read_w(uint8_t *sm, uint32_t tmem, int warp, int lane, int s) {
     const int quad = warp & 3, half = (warp - kPrepWarp0) >> 2;
-    uint8_t *wb = sm + Smem::WB + half * 8192;
+    uint8_t *wdst = sm + Smem::STACK + s * 32768 + half * 16384;
     const int t = 16 * quad + lane;
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
@@ -414,7 +427,7 @@ __device__ void prep_read_w(uint8_t *sm, uint32_t tmem, int warp, int lane) {
                 pk.y = pack_bf16x2(-v[j + 2], -v[j + 3]);
                 pk.z = pack_bf16x2(-v[j + 4], -v[j + 5]);
                 pk.w = pack_bf16x2(-v[j + 6], -v[j + 7]);
-                *reinterpret_cast<uint4 *>(wb + sw128_off(t, 32 * part + j)) = pk;
+                *reinterpret_cast<uint4 *>(wdst + sw128_off(t, 32 * part + j)) = pk;
             }
         }
     }
@@ -433,17 +446,20 @@ constexpr uint32_t kRawBytes = 2 * 8192 + 2 * 8192 + 16384 + C * DVT * 2;
 
 // ---- chain step helpers ---------------------------------------------------------
 
-// O rows of chunk m from TMEM (M = 64 layout) to global memory, bf16.
+// O rows of chunk m from TMEM (rows 64-127 of the M = 128 accumulator
+// [-W S; O], i.e. lanes 64-127: the warps of quadrants 2 and 3) to global
+// memory, bf16.
 __device__ __forceinline__ void chain_store_o(uint32_t tmem, int quad, int lane, int m,
                                               int64_t bos, int64_t len, int h, int j0,
                                               const Params &p) {
+    if (quad < 2) return;
     const int st = m & 1;
     float v[32];
-    tmem_ld32(tmem_addr(tmem, 32 * quad, kColO + 32 * st), v);
+    tmem_ld32(tmem_addr(tmem, 32 * quad, kColUO + 32 * st), v);
     tmem_wait_ld();
-    const int t = 16 * quad + lane;
+    const int t = 32 * (quad - 2) + lane;
     const int64_t tok = bos + (int64_t)m * C + t;
-    if (lane < 16 && (int64_t)m * C + t < len) {
+    if ((int64_t)m * C + t < len) {
         uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)tok * p.H + h) * DV + j0);
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
@@ -611,20 +627,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
             if (leader) {
                 tc_fence_after();
                 mbar_wait(&B[WB_READY], n & 1, abort_flag);
-                const uint32_t aW = smem_addr(sm + Smem::WB), bS = smem_addr(sm + Smem::SB);
-                const uint32_t aQ = smem_addr(sm + Smem::STACK + s * 32768 + 8192);
-                const uint32_t id = idesc_bf16(64, DVT, false, true);
+                const uint32_t aWQ = smem_addr(sm + Smem::STACK + s * 32768);
+                const uint32_t bS = smem_addr(sm + Smem::SB);
+                const uint32_t id = idesc_bf16(128, DVT, false, true);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // U += (-W) S
-                    mma_bf16(tmem + kColU + 32 * s,
-                             smem_desc(aW + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                             smem_desc(bS + ks * 1024, 16, 512, kLayoutSW64), id, 1u);
-                mma_commit(&B[U_FULL + s]);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // O = Qtil S
-                    mma_bf16(tmem + kColO + 32 * s,
-                             smem_desc(aQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                for (int ks = 0; ks < 8; ++ks)   // [-W S; Qtil S] = [-W; Qtil] S
+                    mma_bf16(tmem + kColUO + 32 * s,
+                             smem_desc(aWQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
                              smem_desc(bS + ks * 1024, 16, 512, kLayoutSW64), id, ks > 0 ? 1u : 0u);
+                mma_commit(&B[U_FULL + s]);
                 mma_commit(&B[RAW_EMPTY + s]);
             }
             if (n >= 1) chain_store_o(tmem, quad, lane, n - 1, bos, len, h, j0, p);
@@ -632,9 +643,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
             mbar_wait(&B[U_FULL + s], (n >> 1) & 1, abort_flag);
             tc_fence_after();
             float U[32];
-            tmem_ld32(tmem_addr(tmem, 32 * quad, kColU + 32 * s), U);
-            tmem_wait_ld();
-            if (lane < 16) store_bf16_row_sw64(sm + Smem::UB, 16 * quad + lane, U);
+            if (quad < 2) {   // U = U' - W S for rows 0-63 (lanes 0-63)
+                float Wp[32];
+                tmem_ld32(tmem_addr(tmem, 32 * quad, kColUO + 32 * s), U);
+                tmem_ld32(tmem_addr(tmem, 32 * quad, kColUp + 32 * s), Wp);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) U[i] += Wp[i];
+                store_bf16_row_sw64(sm + Smem::UB, 32 * quad + lane, U);
+            }
             fence_async_smem();
             tc_fence_before();
             named_barrier(kBarChain, kChainThreads);
@@ -642,17 +659,17 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 tc_fence_after();
                 mbar_arrive(&B[ACCU_EMPTY + s]);
                 const uint32_t aK = smem_addr(sm + Smem::KBAR + s * 16384);
-                const uint32_t aP = smem_addr(sm + Smem::PB + s * 8192);
+                const uint32_t aP = smem_addr(sm + Smem::PB + s * 8192 - 8192);
                 const uint32_t bU = smem_addr(sm + Smem::UB);
                 const uint32_t idS = idesc_bf16(128, DVT, true, true);
-                const uint32_t idO = idesc_bf16(64, DVT, false, true);
+                const uint32_t idO = idesc_bf16(128, DVT, false, true);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)   // S += Kbar^T U
                     mma_bf16(tmem + kColS, smem_desc(aK + ks * 2048, 8192, 1024, kLayoutSW128),
                              smem_desc(bU + ks * 1024, 16, 512, kLayoutSW64), idS, 1u);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)   // O += P U
-                    mma_bf16(tmem + kColO + 32 * s, smem_desc(aP + ks * 32, 16, 1024, kLayoutSW128),
+                for (int ks = 0; ks < 4; ++ks)   // O += P U (rows 64-127 of an M = 128 product)
+                    mma_bf16(tmem + kColUO + 32 * s, smem_desc(aP + ks * 32, 16, 1024, kLayoutSW128),
                              smem_desc(bU + ks * 1024, 16, 512, kLayoutSW64), idO, 1u);
                 mma_commit(&B[CHAIN_DONE + s]);
             }
@@ -718,23 +735,22 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 const uint32_t bK = smem_addr(sm + Smem::STACK + s * 32768);
                 const uint32_t bV = smem_addr(sm + Smem::VT + s * 4096);
                 const uint32_t idW = idesc_bf16(64, DK, false, true);
-                const uint32_t idU = idesc_bf16(64, DVT, false, true);
+                const uint32_t idU = idesc_bf16(128, DVT, false, true);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)   // W = T diag(beta) Ktil
                     mma_bf16(tmem + kColW, smem_desc(aT + ks * 32, 16, 1024, kLayoutSW128),
                              smem_desc(bK + ks * 2048, 16384, 1024, kLayoutSW128), idW,
                              ks > 0 ? 1u : 0u);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)   // U' = T diag(beta) V
-                    mma_bf16(tmem + kColU + 32 * s, smem_desc(aT + ks * 32, 16, 1024, kLayoutSW128),
+                for (int ks = 0; ks < 4; ++ks)   // U' = T diag(beta) V (rows 0-63 of an M = 128 product)
+                    mma_bf16(tmem + kColUp + 32 * s, smem_desc(aT + ks * 32, 16, 1024, kLayoutSW128),
                              smem_desc(bV + ks * 1024, 16, 512, kLayoutSW64), idU,
                              ks > 0 ? 1u : 0u);
                 mma_commit(&B[W_FULL]);
             }
             mbar_wait(&B[W_FULL], n & 1, abort_flag);
-            if (n >= 1) mbar_wait(&B[U_FULL + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort_flag);
             tc_fence_after();
-            prep_read_w(sm, tmem, warp, lane);
+            prep_read_w(sm, tmem, warp, lane, s);
             tc_fence_before();
             fence_async_smem();
             named_barrier(kBarPrep, kPrepThreads);
