@@ -316,15 +316,22 @@ __device__ __forceinline__ int tfi(int row, int col) {
 template <int M>
 __device__ __forceinline__ void solve_merge(const float *__restrict__ AF, float *__restrict__ TF,
                                             float *__restrict__ XF, int pt) {
-    constexpr int kThr = 8 * M;               // (64 / 2M) merges x M x (M / 4) segments
-    const int merge = pt / (M * M / 4);
-    const int rem = pt % (M * M / 4);
-    const int r = rem / (M / 4), c4 = (rem % (M / 4)) * 4;
-    const int base = merge * 2 * M;
+    // (64 / 2M) merges, each M x M outputs in 1x4 segments: 8M threads.
+    // Thread layout for X = A21 T1: a warp shares one 4-column group, lanes
+    // run over rows, so the loop can start at k = c4 (T1 is lower
+    // triangular).  For T21 = -T2 X: a warp shares a group of rows, so the
+    // loop can stop after the group's last row (T2 is lower triangular).
+    constexpr int kThr = 8 * M;
+    constexpr int SEG = M / 4;                // 4-column groups per row
+    constexpr int PER = M * SEG;              // threads per merge
+    constexpr int XS = M + 4;                 // padded row stride of X (bank spread)
     if (pt < kThr) {   // X = A21 T1
+        const int merge = pt / PER, rem = pt % PER;
+        const int c4 = (rem / M) * 4, r = rem % M;   // column group outer, row inner
+        const int base = merge * 2 * M;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < M; ++k) {
+#pragma unroll 4
+        for (int k = c4; k < M; ++k) {
             const float av = AF[fidx(base + M + r, base + k)];
             const float4 tv = *reinterpret_cast<const float4 *>(&TF[tfi(base + k, base + c4)]);
             acc.x = fmaf(av, tv.x, acc.x);
@@ -332,18 +339,23 @@ __device__ __forceinline__ void solve_merge(const float *__restrict__ AF, float 
             acc.z = fmaf(av, tv.z, acc.z);
             acc.w = fmaf(av, tv.w, acc.w);
         }
-        *reinterpret_cast<float4 *>(&XF[(merge * M + r) * M + c4]) = acc;
+        *reinterpret_cast<float4 *>(&XF[(merge * M + r) * XS + c4]) = acc;
     }
     named_barrier(kBarPrep, kPrepThreads);
     if (pt < kThr) {   // T21 = -T2 X
+        const int merge = pt / PER, rem = pt % PER;
+        const int r = rem / SEG, c4 = (rem % SEG) * 4;   // row outer, column group inner
+        const int base = merge * 2 * M;
+        const int rlast = (pt | 31) % PER / SEG;          // last row handled by this warp
+        // warps of the M >= 16 levels hold whole row groups of one merge
+        const int kend = (M >= 16) ? ((rlast >> 2) + 1) * 4 : M;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int k4 = 0; k4 < M; k4 += 4) {
+        for (int k4 = 0; k4 < kend; k4 += 4) {
             const float4 tr = *reinterpret_cast<const float4 *>(&TF[tfi(base + M + r, base + M + k4)]);
             const float tk[4] = {tr.x, tr.y, tr.z, tr.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float4 xv = *reinterpret_cast<const float4 *>(&XF[(merge * M + k4 + e) * M + c4]);
+                const float4 xv = *reinterpret_cast<const float4 *>(&XF[(merge * M + k4 + e) * XS + c4]);
                 acc.x = fmaf(tk[e], xv.x, acc.x);
                 acc.y = fmaf(tk[e], xv.y, acc.y);
                 acc.z = fmaf(tk[e], xv.z, acc.z);
