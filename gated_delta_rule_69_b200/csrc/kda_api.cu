@@ -52,6 +52,8 @@ size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens,
                                   int32_t H, int32_t d_k, int32_t d_v) {
     if (num_seqs < 1 || total_tokens < 0 || H < 1) return 0;
     if (!supported_dim(d_k) || !supported_dim(d_v)) return 0;
+    if (d_k == 128 && d_v == 128 && total_tokens > 0)
+        return kda::prefill_split_workspace(num_seqs, total_tokens, H);
     return kda::prefill_tc_workspace(num_seqs);
 }
 
@@ -75,7 +77,9 @@ kda_status kda_prefill(const void *q, const void *k, const void *v,
         if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
     if (beta && !aligned_to(beta, elem_bytes(dtype))) return KDA_ERR_INVALID_ARG;
     if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
-    const size_t need = kda_prefill_workspace_size(num_seqs, total_tokens, H, d_k, d_v);
+    // The least workspace any path accepts; the two-kernel tensor-core path is
+    // taken when the workspace also holds its per-chunk records.
+    const size_t need = kda::prefill_tc_workspace(num_seqs);
     if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_INVALID_ARG;
 
@@ -87,12 +91,17 @@ kda_status kda_prefill(const void *q, const void *k, const void *v,
     if (overlaps(o, nv, q, nk) || overlaps(o, nv, k, nk) || overlaps(o, nv, v, nv) ||
         overlaps(o, nv, log_alpha, nk) || overlaps(o, nv, beta, nb) ||
         overlaps(o, nv, init_state, ns) || overlaps(o, nv, final_state, ns) ||
-        overlaps(o, nv, workspace, need))
+        overlaps(o, nv, workspace, workspace_bytes))
         return KDA_ERR_INVALID_ARG;
     if (init_state && final_state && init_state != final_state &&
         overlaps(init_state, ns, final_state, ns))
         return KDA_ERR_INVALID_ARG;
 
+    if (use_tensor_cores(dtype, d_k, d_v, total_tokens) &&
+        workspace_bytes >= kda::prefill_split_workspace(num_seqs, total_tokens, H))
+        return from_cuda(kda::launch_prefill_split(q, k, v, log_alpha, beta, init_state,
+                                                   cu_seqlens, num_seqs, total_tokens, H, o,
+                                                   final_state, workspace, stream));
     if (use_tensor_cores(dtype, d_k, d_v, total_tokens))
         return from_cuda(kda::launch_prefill_tc(q, k, v, log_alpha, beta, init_state, cu_seqlens,
                                                 num_seqs, total_tokens, H, o, final_state,

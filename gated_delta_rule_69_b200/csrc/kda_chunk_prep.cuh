@@ -1,0 +1,339 @@
+// Chunk preparation for the tensor-core KDA prefill: everything that does not
+// depend on the carried state.  For one chunk of C = 64 tokens of one head,
+// with G the running sum of log_alpha from the chunk start:
+//     Ktil = K e^G, Qtil = Q e^G, Khat = K e^-G, Kbar = K e^{G_L - G}
+//     [A; P] = [Ktil; Qtil] Khat^T  (tensor cores)
+//     A = diag(beta) strict_tril(.),  P = tril(.)
+//     T = (I + A)^-1 (fp32, recursive doubling),  T_beta = T diag(beta)
+//     W = T_beta Ktil (tensor cores)
+// (news digest page on Kimi Linear, section "Algorithme parallele par
+// chunks": WY/UT packing of the chunk's rank-1 updates and the triangular
+// inverse by forward substitution).  The routines take explicit buffer
+// pointers so that kernels with different shared-memory maps can use them;
+// the threads of one 256-thread group call each routine together.
+#pragma once
+
+#include "kda_internal.cuh"
+#include "kda_sm100.cuh"
+
+namespace kda {
+namespace prep {
+
+using namespace sm100;
+
+constexpr int C = 64;
+constexpr int DK = 128;
+constexpr int kGroupThreads = 256;
+constexpr float kSlowPathLogDecay = -60.0f;   // chunk log-decay below this -> pairwise path
+constexpr float kLog2e = 1.4426950408889634f;
+
+// e^x through the hardware base-2 exponential (ex2.approx, flush-to-zero):
+// its relative error (~2^-22) is far below the bf16 rounding of the operands
+// it scales.
+__device__ __forceinline__ float exp_f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * kLog2e));
+    return y;
+}
+
+// Shared-memory buffers of one chunk's preparation.
+struct Bufs {
+    uint8_t *stk;        // [Ktil rows 0-63 | Qtil rows 64-127], 2 K-atoms of 16 KB (128-byte swizzle);
+                         // raw k / q on entry, -W over Ktil on exit
+    uint8_t *khat;       // Khat [64][128], 2 K-atoms of 8 KB
+    uint8_t *kbar;       // Kbar [64][128], 2 K-atoms of 8 KB
+    const uint8_t *graw; // raw log_alpha [64][128] bf16, 256-byte rows
+    float *af;           // A, fp32 64x64 (row-XOR layout); may alias khat after the product
+    float *tf;           // T, fp32 64x64 (float4-XOR layout)
+    float *xf;           // solve scratch, >= 4608 bytes; may alias graw after gating
+    uint8_t *tb;         // T diag(beta) bf16 [64 t][64 i] (one K-atom)
+    uint8_t *pb;         // P bf16 [64 t][64 i]
+    const float *beta;   // 64 fp32, zero past the chunk end
+    float *egl;          // 128 fp32: exp(G_L)
+    float *csum;         // 4 x 128 fp32 scratch
+    uint32_t *slow_flag; // one word
+};
+
+// Index of A element (t, i): rows of 64 floats, column XORed with the row's
+// low 5 bits so that row-parallel accesses hit distinct banks.
+__device__ __forceinline__ int fidx(int t, int i) { return t * 64 + (i ^ (t & 31)); }
+
+// T layout: rows of 64 floats, float4 group index XORed with (row mod 16).
+__device__ __forceinline__ int tfi(int row, int col) {
+    return row * 64 + ((((col >> 2) ^ (row & 15))) << 2) + (col & 3);
+}
+
+// ---- running sums and gated operands.  Thread pt (0..255) owns channels
+// c, c+1 (c = 2 (pt mod 64)) for the 16 tokens of group pt / 64; a warp covers
+// one 64-channel K-atom of one token group.  Returns whether the chunk needs
+// the pairwise path.
+template <int BAR>
+__device__ bool gate(const Bufs &b, int pt, int L) {
+    const int c = 2 * (pt & 63);
+    const int tg = pt >> 6;
+    const int t0 = tg * 16;
+    const int katom = c >> 6, cc = c & 63;
+    uint8_t *stack = b.stk + katom * 16384;
+    uint8_t *khat = b.khat + katom * 8192;
+    uint8_t *kbar = b.kbar + katom * 8192;
+
+    uint32_t graw_v[16], k_v[16], q_v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int t = t0 + i;
+        graw_v[i] = *reinterpret_cast<const uint32_t *>(b.graw + t * 256 + c * 2);
+        k_v[i] = *reinterpret_cast<const uint32_t *>(stack + sw128_off(t, cc));
+        q_v[i] = *reinterpret_cast<const uint32_t *>(stack + sw128_off(64 + t, cc));
+    }
+    float g0[16], g1[16];
+    float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const bool valid = t0 + i < L;
+        const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162 *>(&graw_v[i]);
+        r0 += valid ? clamp_log_alpha(__low2float(gv)) : 0.f;
+        r1 += valid ? clamp_log_alpha(__high2float(gv)) : 0.f;
+        g0[i] = r0;
+        g1[i] = r1;
+    }
+    b.csum[tg * 128 + c] = r0;
+    b.csum[tg * 128 + c + 1] = r1;
+    if (pt == 0) *b.slow_flag = 0u;
+    named_barrier(BAR, kGroupThreads);
+
+    float off0 = 0.f, off1 = 0.f, GL0 = 0.f, GL1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float a = b.csum[j * 128 + c], bb = b.csum[j * 128 + c + 1];
+        if (j < tg) { off0 += a; off1 += bb; }
+        GL0 += a;
+        GL1 += bb;
+    }
+    if (tg == 0 && (GL0 < kSlowPathLogDecay || GL1 < kSlowPathLogDecay)) *b.slow_flag = 1u;
+    named_barrier(BAR, kGroupThreads);
+    const bool slow = *b.slow_flag != 0u;
+
+    const float eL0 = exp_f(GL0), eL1 = exp_f(GL1);
+    if (tg == 0) {
+        b.egl[c] = eL0;
+        b.egl[c + 1] = eL1;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int t = t0 + i;
+        const bool valid = t < L;
+        const __nv_bfloat162 kv = *reinterpret_cast<const __nv_bfloat162 *>(&k_v[i]);
+        const __nv_bfloat162 qv = *reinterpret_cast<const __nv_bfloat162 *>(&q_v[i]);
+        const float k0 = valid ? __low2float(kv) : 0.f, k1 = valid ? __high2float(kv) : 0.f;
+        const float q0 = valid ? __low2float(qv) : 0.f, q1 = valid ? __high2float(qv) : 0.f;
+        const float G0 = g0[i] + off0, G1 = g1[i] + off1;
+        const float e0 = exp_f(G0), e1 = exp_f(G1);
+        const float ih0 = exp_f(fminf(-G0, 80.f)), ih1 = exp_f(fminf(-G1, 80.f));
+        float b0, b1;
+        if (slow) {
+            b0 = exp_f(GL0 - G0);
+            b1 = exp_f(GL1 - G1);
+        } else {
+            b0 = eL0 * ih0;
+            b1 = eL1 * ih1;
+        }
+        const uint32_t ok = sw128_off(t, cc);
+        *reinterpret_cast<uint32_t *>(stack + ok) = pack_bf16x2(k0 * e0, k1 * e1);
+        *reinterpret_cast<uint32_t *>(stack + sw128_off(64 + t, cc)) = pack_bf16x2(q0 * e0, q1 * e1);
+        *reinterpret_cast<uint32_t *>(khat + ok) = pack_bf16x2(k0 * ih0, k1 * ih1);
+        *reinterpret_cast<uint32_t *>(kbar + ok) = pack_bf16x2(k0 * b0, k1 * b1);
+    }
+    return slow;
+}
+
+// ---- pairwise fallback for A and P when a chunk decays too fast for the
+// product form: differences of running sums taken pair by pair in fp32, from
+// the raw k and q rows in global memory (kt0 / qt0 point at token 0 of the
+// chunk for this head; row_stride is H * d_k elements).
+__device__ void pairwise(const Bufs &b, int pt, int L, const __nv_bfloat16 *kt0,
+                         const __nv_bfloat16 *qt0, size_t row_stride) {
+    for (int pidx = pt; pidx < C * C; pidx += kGroupThreads) {
+        const int t = pidx >> 6, i = pidx & 63;
+        float ak = 0.f, aq = 0.f;
+        if (i <= t && t < L) {
+            const __nv_bfloat16 *kt = kt0 + (size_t)t * row_stride;
+            const __nv_bfloat16 *ki = kt0 + (size_t)i * row_stride;
+            const __nv_bfloat16 *qt = qt0 + (size_t)t * row_stride;
+            for (int c = 0; c < DK; ++c) {
+                float d = 0.f;  // G_t - G_i = sum of log_alpha over tokens i+1..t
+                for (int u = i + 1; u <= t; ++u)
+                    d += clamp_log_alpha(__bfloat162float(
+                        *reinterpret_cast<const __nv_bfloat16 *>(b.graw + u * 256 + c * 2)));
+                const float kd = __bfloat162float(ki[c]) * exp_f(d);
+                ak = fmaf(__bfloat162float(kt[c]), kd, ak);
+                aq = fmaf(__bfloat162float(qt[c]), kd, aq);
+            }
+        }
+        b.af[fidx(t, i)] = (i < t) ? b.beta[t] * ak : 0.f;
+        *reinterpret_cast<__nv_bfloat16 *>(b.pb + sw128_off(t, i)) = __float2bfloat16_rn(aq);
+    }
+}
+
+// ---- [A; P] from TMEM.  A warp of TMEM quadrant `quad` (lanes 32 quad ..)
+// reads 32 of the 64 columns (`half`): rows 0-63 are Ktil Khat^T -> A (fp32,
+// beta-scaled, strictly lower), rows 64-127 are Qtil Khat^T -> P (bf16, lower).
+__device__ __forceinline__ void read_ap(const Bufs &b, uint32_t tmem_ap, int quad, int half,
+                                        int lane) {
+    float v[32];
+    tmem_ld32(tmem_addr(tmem_ap, 32 * quad, 32 * half), v);
+    tmem_wait_ld();
+    if (quad < 2) {
+        const int t = 32 * quad + lane;
+        const float bt = b.beta[t];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int i = 32 * half + j;
+            b.af[fidx(t, i)] = (i < t) ? bt * v[j] : 0.f;
+        }
+    } else {
+        const int t = 32 * (quad - 2) + lane;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+            float w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = (32 * half + j + e <= t) ? v[j + e] : 0.f;
+            uint4 pk;
+            pk.x = pack_bf16x2(w[0], w[1]);
+            pk.y = pack_bf16x2(w[2], w[3]);
+            pk.z = pack_bf16x2(w[4], w[5]);
+            pk.w = pack_bf16x2(w[6], w[7]);
+            *reinterpret_cast<uint4 *>(b.pb + sw128_off(t, 32 * half + j)) = pk;
+        }
+    }
+}
+
+// ---- one merge level of the recursive-doubling inverse: neighbouring M x M
+// lower-triangular inverses T1, T2 become [[T1, 0], [T21, T2]] with
+// T21 = -T2 (A21 T1).  1x4 row segments per thread; warps share a column
+// group (first product) or a row group (second product) so that the loops
+// skip the triangular zeros.
+template <int M, int BAR>
+__device__ __forceinline__ void merge(const float *__restrict__ AF, float *__restrict__ TF,
+                                      float *__restrict__ XF, int pt) {
+    constexpr int kThr = 8 * M;
+    constexpr int SEG = M / 4;
+    constexpr int PER = M * SEG;
+    constexpr int XS = M + 4;
+    if (pt < kThr) {   // X = A21 T1
+        const int merge_id = pt / PER, rem = pt % PER;
+        const int c4 = (rem / M) * 4, r = rem % M;
+        const int base = merge_id * 2 * M;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int k = c4; k < M; ++k) {
+            const float av = AF[fidx(base + M + r, base + k)];
+            const float4 tv = *reinterpret_cast<const float4 *>(&TF[tfi(base + k, base + c4)]);
+            acc.x = fmaf(av, tv.x, acc.x);
+            acc.y = fmaf(av, tv.y, acc.y);
+            acc.z = fmaf(av, tv.z, acc.z);
+            acc.w = fmaf(av, tv.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(&XF[(merge_id * M + r) * XS + c4]) = acc;
+    }
+    named_barrier(BAR, kGroupThreads);
+    if (pt < kThr) {   // T21 = -T2 X
+        const int merge_id = pt / PER, rem = pt % PER;
+        const int r = rem / SEG, c4 = (rem % SEG) * 4;
+        const int base = merge_id * 2 * M;
+        const int rlast = (pt | 31) % PER / SEG;
+        const int kend = (M >= 16) ? ((rlast >> 2) + 1) * 4 : M;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k4 = 0; k4 < kend; k4 += 4) {
+            const float4 tr = *reinterpret_cast<const float4 *>(&TF[tfi(base + M + r, base + M + k4)]);
+            const float tk[4] = {tr.x, tr.y, tr.z, tr.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float4 xv =
+                    *reinterpret_cast<const float4 *>(&XF[(merge_id * M + k4 + e) * XS + c4]);
+                acc.x = fmaf(tk[e], xv.x, acc.x);
+                acc.y = fmaf(tk[e], xv.y, acc.y);
+                acc.z = fmaf(tk[e], xv.z, acc.z);
+                acc.w = fmaf(tk[e], xv.w, acc.w);
+            }
+        }
+        *reinterpret_cast<float4 *>(&TF[tfi(base + M + r, base + c4)]) =
+            make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+    }
+    named_barrier(BAR, kGroupThreads);
+}
+
+// ---- T = (I + A)^-1 by recursive doubling from closed-form 4x4 diagonal
+// blocks; writes T diag(beta) as bf16 into b.tb.  Starts and ends with every
+// thread of the group past a barrier on its buffers.
+template <int BAR>
+__device__ void solve(const Bufs &b, int pt) {
+    const float *__restrict__ AF = b.af;
+    float *__restrict__ TF = b.tf;
+    float *__restrict__ XF = b.xf;
+    for (int v = pt; v < 1024; v += kGroupThreads) {   // zero outside the 4x4 diagonal blocks
+        const int row = v >> 4, g4 = v & 15;
+        if (g4 != (row >> 2))
+            *reinterpret_cast<float4 *>(&TF[tfi(row, 4 * g4)]) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (pt < 16) {   // 4x4 unit lower-triangular inverses, written out
+        const int b0 = 4 * pt;
+        const float n10 = AF[fidx(b0 + 1, b0)];
+        const float n20 = AF[fidx(b0 + 2, b0)], n21 = AF[fidx(b0 + 2, b0 + 1)];
+        const float n30 = AF[fidx(b0 + 3, b0)], n31 = AF[fidx(b0 + 3, b0 + 1)],
+                    n32 = AF[fidx(b0 + 3, b0 + 2)];
+        const float t10 = -n10, t21 = -n21, t32 = -n32;
+        const float t20 = -(n20 + n21 * t10);
+        const float t31 = -(n31 + n32 * t21);
+        const float t30 = -(n30 + n31 * t10 + n32 * t20);
+        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 0, b0)]) = make_float4(1.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 1, b0)]) = make_float4(t10, 1.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 2, b0)]) = make_float4(t20, t21, 1.f, 0.f);
+        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 3, b0)]) = make_float4(t30, t31, t32, 1.f);
+    }
+    named_barrier(BAR, kGroupThreads);
+    merge<4, BAR>(AF, TF, XF, pt);
+    merge<8, BAR>(AF, TF, XF, pt);
+    merge<16, BAR>(AF, TF, XF, pt);
+    merge<32, BAR>(AF, TF, XF, pt);
+
+    const int t = pt >> 2, i0 = (pt & 3) * 16;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const float4 u0 = *reinterpret_cast<const float4 *>(&TF[tfi(t, i0 + 8 * hh)]);
+        const float4 u1 = *reinterpret_cast<const float4 *>(&TF[tfi(t, i0 + 8 * hh + 4)]);
+        const float *bb = b.beta + i0 + 8 * hh;
+        uint4 pk;
+        pk.x = pack_bf16x2(u0.x * bb[0], u0.y * bb[1]);
+        pk.y = pack_bf16x2(u0.z * bb[2], u0.w * bb[3]);
+        pk.z = pack_bf16x2(u1.x * bb[4], u1.y * bb[5]);
+        pk.w = pack_bf16x2(u1.z * bb[6], u1.w * bb[7]);
+        *reinterpret_cast<uint4 *>(b.tb + sw128_off(t, i0 + 8 * hh)) = pk;
+    }
+}
+
+// ---- -W from TMEM (M = 64 layout: row r in lane (r mod 16) + 32 (r / 16))
+// over Ktil in b.stk (rows 0-63), so that [-W; Qtil] is one M = 128 operand.
+__device__ __forceinline__ void read_w(const Bufs &b, uint32_t tmem_w, int quad, int half, int lane) {
+    uint8_t *wdst = b.stk + half * 16384;
+    const int t = 16 * quad + lane;
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+        float v[32];
+        tmem_ld32(tmem_addr(tmem_w, 32 * quad, 64 * half + 32 * part), v);
+        tmem_wait_ld();
+        if (lane < 16) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+                uint4 pk;
+                pk.x = pack_bf16x2(-v[j + 0], -v[j + 1]);
+                pk.y = pack_bf16x2(-v[j + 2], -v[j + 3]);
+                pk.z = pack_bf16x2(-v[j + 4], -v[j + 5]);
+                pk.w = pack_bf16x2(-v[j + 6], -v[j + 7]);
+                *reinterpret_cast<uint4 *>(wdst + sw128_off(t, 32 * part + j)) = pk;
+            }
+        }
+    }
+}
+
+}  // namespace prep
+}  // namespace kda

@@ -69,4 +69,13 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                               int num_seqs, int64_t total_tokens, int H, void *o,
                               float *final_state, void *workspace, cudaStream_t stream);
 
+// Tensor-core prefill split into a chunk-parallel preparation kernel and a
+// state-chain kernel; its workspace holds one record per (chunk, head).
+size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H);
+
+cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const void *g,
+                                 const void *beta, const float *init_state, const int32_t *cu,
+                                 int num_seqs, int64_t total_tokens, int H, void *o,
+                                 float *final_state, void *workspace, cudaStream_t stream);
+
 }  // namespace kda

@@ -52,8 +52,9 @@ extern "C" kda_status kda_prefill_noalloc(const void *q, const void *k, const vo
                                           int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
                                           float *final_state, kda_stream_t stream) {
     if (num_seqs > kNoAllocMaxSeqs) return KDA_ERR_UNSUPPORTED;
-    const size_t need = kda_prefill_workspace_size(num_seqs, total_tokens, H, d_k, d_v);
-    if (need > kNoAllocBytes) return KDA_ERR_UNSUPPORTED;
+    // the array holds the workspace of the single-kernel paths (error word and
+    // sequence order); kda_prefill takes those paths for a workspace this size
+    if (kda::prefill_tc_workspace(num_seqs) > kNoAllocBytes) return KDA_ERR_UNSUPPORTED;
     void *scratch = scratch_for_current_device();
     if (!scratch) return KDA_ERR_CUDA;
     return kda_prefill(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, total_tokens,

@@ -1,0 +1,721 @@
+// KDA prefill as two kernels (bf16 I/O, d_k = d_v = 128, C = 64):
+//
+//   kda_prep_kernel  - one CTA per (chunk, head), all chunks at once: the
+//                      chunk preparation of kda_chunk_prep.cuh (running sums,
+//                      gated operands, [A; P] on the tensor cores, T = (I+A)^-1,
+//                      W), written to the workspace as a 65 KB record per
+//                      (chunk, head) in the exact shared-memory layout the
+//                      tensor cores read: [-W; Qtil], Kbar, T diag(beta), P,
+//                      exp(G_L).
+//   kda_chain_kernel - one CTA per (sequence, head, 32-column slice of d_v):
+//                      the serial state chain.  Per chunk it bulk-copies the
+//                      record into a 3-stage ring (plus its v slice by TMA),
+//                      and with the fp32 state S in TMEM computes
+//                          U' = T diag(beta) V,  [-W S; Qtil S] = [-W; Qtil] S
+//                          U = U' - W S,  O = Qtil S + P U
+//                          S <- Diag(e^{G_L}) S + Kbar^T U
+//                      on the tensor cores.
+//
+// The state-independent preparation (the long-latency part of a chunk: the
+// gating exponentials and the triangular solve) thus runs chunk-parallel
+// over the whole GPU, once per (chunk, head), and leaves the serial chain
+// (news digest page on Kimi Linear, section "Algorithme parallele par chunks":
+// the previous chunk's final state is the next chunk's initial state) with
+// only tensor-core products and their read-outs.  The price is the record's
+// round trip through global memory (written once, read once per d_v slice).
+#include <cuda.h>
+
+#include "kda_chunk_prep.cuh"
+#include "kda_internal.cuh"
+#include "kda_sm100.cuh"
+
+namespace kda {
+namespace split {
+
+using namespace sm100;
+
+constexpr int C = 64;
+constexpr int DK = 128;
+constexpr int DV = 128;
+constexpr int DVT = 32;
+constexpr int NTILE = DV / DVT;
+
+// ---- the per-(chunk, head) record, also the chain kernel's ring-slot layout
+struct Rec {
+    static constexpr uint32_t STK = 0;         // [-W rows 0-63 | Qtil rows 64-127], 2 K-atoms x 16 KB
+    static constexpr uint32_t KBAR = 32768;    // Kbar [64 t][128 c], 2 K-atoms x 8 KB
+    static constexpr uint32_t TB = 49152;      // T diag(beta) [64 t][64 i]; TB+PB form one M=128 operand
+    static constexpr uint32_t PB = 57344;      // P [64 t][64 i]
+    static constexpr uint32_t EGL = 65536;     // 128 fp32
+    static constexpr uint32_t BYTES = 66048;   // bytes carried
+    static constexpr uint32_t STRIDE = 66560;  // record stride (1024-aligned)
+};
+
+// ---- prep kernel
+constexpr int kPrepThreads = 288;              // warp 0: loads; warps 1-8: the 256-thread group
+constexpr uint32_t kPrepBar = 1;
+struct PrepSmem {
+    static constexpr uint32_t REC = 0;         // record image (STK, KBAR, TB, PB, EGL)
+    static constexpr uint32_t TF = Rec::KBAR;  // T fp32, after Kbar has been stored
+    static constexpr uint32_t KHAT = 66560;    // Khat, then A fp32
+    static constexpr uint32_t GRAW = 82944;    // raw log_alpha, then solve scratch
+    static constexpr uint32_t BETA = 99328;    // 64 fp32
+    static constexpr uint32_t CSUM = 99584;    // 4 x 128 fp32
+    static constexpr uint32_t BARS = 101632;   // 3 mbarriers
+    static constexpr uint32_t MISC = 101696;   // tmem base, abort, slow flag
+    static constexpr uint32_t SIZE = 101760;
+    static constexpr uint32_t ALLOC = SIZE + 1024;
+};
+static_assert(2 * PrepSmem::ALLOC <= 228 * 1024, "two prep CTAs per SM");
+constexpr uint32_t kPrepTmemCols = 256;        // [A;P] at 0 (64 cols), W at 64 (128 cols)
+constexpr uint32_t kRawBytes = 4 * 8192 + 16384;   // k, q (2 boxes each), log_alpha
+
+// ---- chain kernel
+constexpr int kChainThreads = 160;             // warp 0: loads; warps 1-4: the chain
+constexpr uint32_t kChainBar = 1;
+constexpr int NS = 3;                          // ring stages
+struct ChainSmem {
+    static constexpr uint32_t SLOT = 0;        // NS x (record + v slice)
+    static constexpr uint32_t VT_OFF = Rec::STRIDE;           // v slice [64 t][32 j], 64-byte swizzle
+    static constexpr uint32_t SLOT_STRIDE = Rec::STRIDE + 4096;   // 70656
+    static constexpr uint32_t SB = NS * SLOT_STRIDE;          // S bf16 [128 c][32 j]
+    static constexpr uint32_t UB = SB + 8192;                 // U bf16 [64 t][32 j]
+    static constexpr uint32_t BARS = UB + 4096;
+    static constexpr uint32_t MISC = BARS + 128;
+    static constexpr uint32_t SIZE = MISC + 64;
+    static constexpr uint32_t ALLOC = SIZE + 1024;
+};
+static_assert(ChainSmem::ALLOC <= 232448, "chain shared memory");
+constexpr uint32_t kChainTmemCols = 256;
+constexpr uint32_t kColUp = 0, kColUO = 64, kColS = 128;   // U' x2, [-W S; O] x2, S
+
+struct Params {
+    const __nv_bfloat16 *k, *q, *beta;
+    const float *init_state;
+    float *final_state;
+    __nv_bfloat16 *o;
+    const int32_t *cu;          // may be null: equal lengths
+    const int32_t *perm;        // longest-first order (chain kernel) or null
+    const int32_t *chunk_off;   // [N+1] first record index of each sequence
+    const int2 *chunk_tab;      // [max_chunks] (sequence, chunk) of each record
+    const uint32_t *total_chunks;
+    uint8_t *recs;              // records, STRIDE bytes each, index (chunk * H + h)
+    uint32_t *err_word;
+    int64_t total_tokens;
+    int num_seqs, H;
+};
+
+__device__ __forceinline__ void seq_bounds(const Params &p, int seq, int64_t &bos, int64_t &eos) {
+    if (p.cu) {
+        bos = p.cu[seq];
+        eos = p.cu[seq + 1];
+        if (bos < 0 || eos < bos || eos > p.total_tokens) bos = eos = 0;  // flagged by the plan kernel
+    } else {
+        const int64_t len = p.total_tokens / p.num_seqs;
+        bos = (int64_t)seq * len;
+        eos = bos + len;
+    }
+}
+
+// 1-D bulk copies between global and shared memory (16-byte aligned,
+// multiple-of-16 sizes).  Loads complete on an mbarrier; stores are tracked
+// as a bulk group of the issuing thread.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(dst), "r"(smem_addr(src)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > 1000000000ull) return;
+    }
+}
+
+// =============================================================== prep kernel
+
+__global__ void __launch_bounds__(kPrepThreads, 2)
+kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                const __grid_constant__ CUtensorMap tm_g, const Params p) {
+    const uint32_t total = *p.total_chunks;
+    const int h = blockIdx.x % p.H;
+    const uint32_t chunk = blockIdx.x / p.H;
+    if (chunk >= total) return;   // the grid is sized for the largest possible chunk count
+
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t *sm = dyn_smem + ((1024u - (smem_addr(dyn_smem) & 1023u)) & 1023u);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int2 sc = p.chunk_tab[chunk];
+    int64_t bos, eos;
+    seq_bounds(p, sc.x, bos, eos);
+    const int64_t tok0 = bos + (int64_t)sc.y * C;
+    const int L = (int)min((int64_t)C, eos - tok0);
+    uint8_t *rec = p.recs + ((size_t)chunk * p.H + h) * Rec::STRIDE;
+
+    uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);   // 0 raw, 1 [A;P], 2 W
+    uint32_t *misc = reinterpret_cast<uint32_t *>(sm + PrepSmem::MISC);
+    volatile uint32_t *abort_flag = misc + 1;
+    float *beta = reinterpret_cast<float *>(sm + PrepSmem::BETA);
+    if (tid == 0) {
+        mbar_init(&B[0], 2);
+        mbar_init(&B[1], 1);
+        mbar_init(&B[2], 1);
+        misc[1] = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&misc[0], kPrepTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&B[0], kRawBytes);
+            const int t = (int)tok0;
+            tma_load_3d(sm + Rec::STK, &tm_k, &B[0], 0, h, t);
+            tma_load_3d(sm + Rec::STK + 16384, &tm_k, &B[0], 64, h, t);
+            tma_load_3d(sm + Rec::STK + 8192, &tm_q, &B[0], 0, h, t);
+            tma_load_3d(sm + Rec::STK + 16384 + 8192, &tm_q, &B[0], 64, h, t);
+            tma_load_3d(sm + PrepSmem::GRAW, &tm_g, &B[0], 0, h, t);
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int t = lane + 32 * e;
+            beta[t] = (t < L) ? __bfloat162float(p.beta[(size_t)(tok0 + t) * p.H + h]) : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B[0]);
+        if (lane == 0) wait_drain(&B[0], 0);   // the copies land before this CTA may exit
+    } else {
+        const int pt = tid - 32;
+        const bool leader = pt == 0;
+        const int quad = warp & 3, half = (warp - 1) >> 2;
+        prep::Bufs b;
+        b.stk = sm + Rec::STK;
+        b.khat = sm + PrepSmem::KHAT;
+        b.kbar = sm + Rec::KBAR;
+        b.graw = sm + PrepSmem::GRAW;
+        b.af = reinterpret_cast<float *>(sm + PrepSmem::KHAT);
+        b.tf = reinterpret_cast<float *>(sm + PrepSmem::TF);
+        b.xf = reinterpret_cast<float *>(sm + PrepSmem::GRAW);
+        b.tb = sm + Rec::TB;
+        b.pb = sm + Rec::PB;
+        b.beta = beta;
+        b.egl = reinterpret_cast<float *>(sm + Rec::EGL);
+        b.csum = reinterpret_cast<float *>(sm + PrepSmem::CSUM);
+        b.slow_flag = misc + 2;
+
+        mbar_wait(&B[0], 0, abort_flag);
+        const bool slow = prep::gate<kPrepBar>(b, pt, L);
+        fence_async_smem();
+        named_barrier(kPrepBar, prep::kGroupThreads);
+        if (leader) {
+            tc_fence_after();
+            const uint32_t a0 = smem_addr(sm + Rec::STK), b0 = smem_addr(sm + PrepSmem::KHAT);
+            const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)   // [Ktil; Qtil] Khat^T
+                mma_bf16(tmem, smem_desc(a0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                         smem_desc(b0 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                         id, ks > 0 ? 1u : 0u);
+            mma_commit(&B[1]);
+            bulk_store(rec + Rec::KBAR, sm + Rec::KBAR, 16384);   // Kbar is final
+            bulk_commit();
+        }
+        mbar_wait(&B[1], 0, abort_flag);
+        tc_fence_after();
+        if (!slow) {
+            prep::read_ap(b, tmem, quad, half, lane);
+        } else {
+            const size_t stride = (size_t)p.H * DK;
+            prep::pairwise(b, pt, L, p.k + ((size_t)tok0 * p.H + h) * DK,
+                           p.q + ((size_t)tok0 * p.H + h) * DK, stride);
+        }
+        if (leader) bulk_wait_read_all();   // Kbar has left shared memory: T may overwrite it
+        tc_fence_before();
+        named_barrier(kPrepBar, prep::kGroupThreads);
+        prep::solve<kPrepBar>(b, pt);
+        fence_async_smem();
+        named_barrier(kPrepBar, prep::kGroupThreads);
+        if (leader) {
+            tc_fence_after();
+            const uint32_t aT = smem_addr(sm + Rec::TB), bK = smem_addr(sm + Rec::STK);
+            const uint32_t idW = idesc_bf16(64, DK, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)   // W = T diag(beta) Ktil
+                mma_bf16(tmem + 64, smem_desc(aT + ks * 32, 16, 1024, kLayoutSW128),
+                         smem_desc(bK + ks * 2048, 16384, 1024, kLayoutSW128), idW, ks > 0 ? 1u : 0u);
+            mma_commit(&B[2]);
+        }
+        mbar_wait(&B[2], 0, abort_flag);
+        tc_fence_after();
+        prep::read_w(b, tmem + 64, quad, half, lane);
+        fence_async_smem();
+        tc_fence_before();
+        named_barrier(kPrepBar, prep::kGroupThreads);
+        if (leader) {
+            bulk_store(rec + Rec::STK, sm + Rec::STK, 32768);
+            bulk_store(rec + Rec::TB, sm + Rec::TB, Rec::BYTES - Rec::TB);   // TB, PB, exp(G_L)
+            bulk_commit();
+            bulk_wait_all();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kPrepTmemCols);
+    }
+    if (tid == 0 && *abort_flag) atomicOr(p.err_word, kDevErrTimeout);
+}
+
+// =============================================================== chain kernel
+
+__device__ __forceinline__ void store_bf16_row_sw64(uint8_t *tile, int row, const float (&v)[32]) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+        uint4 pk;
+        pk.x = pack_bf16x2(v[j + 0], v[j + 1]);
+        pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
+        pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
+        pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
+        *reinterpret_cast<uint4 *>(tile + sw64_off(row, j)) = pk;
+    }
+}
+
+// O rows of chunk m: rows 64-127 of [-W S; O] (lanes 64-127, quadrants 2-3).
+__device__ __forceinline__ void store_o(uint32_t tmem, int quad, int lane, int m, int64_t bos,
+                                        int64_t len, int h, int j0, const Params &p) {
+    if (quad < 2) return;
+    float v[32];
+    tmem_ld32(tmem_addr(tmem, 32 * quad, kColUO + 32 * (m & 1)), v);
+    tmem_wait_ld();
+    const int t = 32 * (quad - 2) + lane;
+    if ((int64_t)m * C + t < len) {
+        uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)(bos + (int64_t)m * C + t) * p.H + h) * DV + j0);
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(v[j + 0], v[j + 1]);
+            pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
+            pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
+            pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
+            dst[j / 8] = pk;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kChainThreads, 1)
+kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t *sm = dyn_smem + ((1024u - (smem_addr(dyn_smem) & 1023u)) & 1023u);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tile = blockIdx.x % NTILE;
+    const int h = (blockIdx.x / NTILE) % p.H;
+    const int rank = blockIdx.x / (NTILE * p.H);
+    const int seq = p.perm ? p.perm[rank] : rank;
+    int64_t bos, eos;
+    seq_bounds(p, seq, bos, eos);
+    const int64_t len = eos - bos;
+    const int nchunks = (int)((len + C - 1) / C);
+    const int j0 = tile * DVT;
+    const size_t rec0 = (size_t)p.chunk_off[seq];
+
+    // mbarriers: FULL[NS], EMPTY[NS], U_FULL[2], DONE[2], FINAL
+    uint64_t *B = reinterpret_cast<uint64_t *>(sm + ChainSmem::BARS);
+    uint64_t *FULL = B, *EMPTY = B + NS, *UFULL = B + 2 * NS, *DONE = B + 2 * NS + 2,
+             *FIN = B + 2 * NS + 4;
+    uint32_t *misc = reinterpret_cast<uint32_t *>(sm + ChainSmem::MISC);
+    volatile uint32_t *abort_flag = misc + 1;
+    if (tid == 0) {
+        for (int i = 0; i < 2 * NS + 5; ++i) mbar_init(&B[i], 1);
+        misc[1] = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&misc[0], kChainTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+
+    if (warp == 0) {
+        // ---------------------------------------------- loader: records + v slices
+        if (lane == 0 && nchunks > 0) {
+            tma_prefetch_desc(&tm_v);
+            int issued = 0;
+            for (int n = 0; n < nchunks; ++n) {
+                const int s = n % NS;
+                if (n >= NS) mbar_wait(&EMPTY[s], ((n / NS) - 1) & 1, abort_flag);
+                if (*abort_flag) break;
+                uint8_t *slot = sm + ChainSmem::SLOT + s * ChainSmem::SLOT_STRIDE;
+                const uint8_t *rec = p.recs + ((rec0 + n) * p.H + h) * Rec::STRIDE;
+                mbar_arrive_expect_tx(&FULL[s], Rec::BYTES + 4096);
+                bulk_load(slot + Rec::STK, rec + Rec::STK, 32768, &FULL[s]);
+                bulk_load(slot + Rec::KBAR, rec + Rec::KBAR, 16384, &FULL[s]);
+                bulk_load(slot + Rec::TB, rec + Rec::TB, Rec::BYTES - Rec::TB, &FULL[s]);
+                tma_load_3d(slot + ChainSmem::VT_OFF, &tm_v, &FULL[s], j0, h, (int)(bos + (int64_t)n * C));
+                issued = n + 1;
+            }
+            for (int n = (issued > NS ? issued - NS : 0); n < issued; ++n)
+                wait_drain(&FULL[n % NS], (n / NS) & 1);
+        }
+    } else {
+        // ---------------------------------------------- the state chain
+        const int ct = tid - 32;
+        const bool leader = ct == 0;
+        const int quad = warp & 3;
+        const int crow = 32 * quad + lane;
+        const size_t soff = ((size_t)seq * p.H + h) * (size_t)(DK * DV) + (size_t)crow * DV + j0;
+        float S[32];
+        if (p.init_state) {
+            const float4 *src = reinterpret_cast<const float4 *>(p.init_state + soff);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 v = src[i];
+                S[4 * i] = v.x; S[4 * i + 1] = v.y; S[4 * i + 2] = v.z; S[4 * i + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) S[i] = 0.f;
+        }
+        for (int n = 0; n < nchunks; ++n) {
+            const int s = n % NS, u = n & 1;
+            uint8_t *slot = sm + ChainSmem::SLOT + s * ChainSmem::SLOT_STRIDE;
+            if (n >= 1) {
+                mbar_wait(&DONE[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
+                tc_fence_after();
+                tmem_ld32(tmem_addr(tmem, 32 * quad, kColS), S);
+                tmem_wait_ld();
+            }
+            store_bf16_row_sw64(sm + ChainSmem::SB, crow, S);
+            mbar_wait(&FULL[s], (n / NS) & 1, abort_flag);
+            const float d = reinterpret_cast<const float *>(slot + Rec::EGL)[crow];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) S[i] *= d;
+            tmem_st32(tmem_addr(tmem, 32 * quad, kColS), S);
+            tmem_wait_st();
+            fence_async_smem();
+            tc_fence_before();
+            named_barrier(kChainBar, 128);
+            if (leader) {
+                tc_fence_after();
+                const uint32_t aTP = smem_addr(slot + Rec::TB);
+                const uint32_t bV = smem_addr(slot + ChainSmem::VT_OFF);
+                const uint32_t aWQ = smem_addr(slot + Rec::STK);
+                const uint32_t bS = smem_addr(sm + ChainSmem::SB);
+                const uint32_t id = idesc_bf16(128, DVT, false, true);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)   // U' = T diag(beta) V (rows 0-63)
+                    mma_bf16(tmem + kColUp + 32 * u, smem_desc(aTP + ks * 32, 16, 1024, kLayoutSW128),
+                             smem_desc(bV + ks * 1024, 16, 512, kLayoutSW64), id, ks > 0 ? 1u : 0u);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)   // [-W S; Qtil S]
+                    mma_bf16(tmem + kColUO + 32 * u,
+                             smem_desc(aWQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                             smem_desc(bS + ks * 1024, 16, 512, kLayoutSW64), id, ks > 0 ? 1u : 0u);
+                mma_commit(&UFULL[u]);
+            }
+            if (n >= 1) store_o(tmem, quad, lane, n - 1, bos, len, h, j0, p);
+
+            mbar_wait(&UFULL[u], (n >> 1) & 1, abort_flag);
+            tc_fence_after();
+            if (quad < 2) {   // U = U' - W S, rows 0-63
+                float U[32], Wp[32];
+                tmem_ld32(tmem_addr(tmem, 32 * quad, kColUO + 32 * u), U);
+                tmem_ld32(tmem_addr(tmem, 32 * quad, kColUp + 32 * u), Wp);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) U[i] += Wp[i];
+                store_bf16_row_sw64(sm + ChainSmem::UB, crow, U);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            named_barrier(kChainBar, 128);
+            if (leader) {
+                tc_fence_after();
+                const uint32_t aK = smem_addr(slot + Rec::KBAR);
+                const uint32_t aTP = smem_addr(slot + Rec::TB);
+                const uint32_t bU = smem_addr(sm + ChainSmem::UB);
+                const uint32_t idS = idesc_bf16(128, DVT, true, true);
+                const uint32_t idO = idesc_bf16(128, DVT, false, true);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)   // S += Kbar^T U
+                    mma_bf16(tmem + kColS, smem_desc(aK + ks * 2048, 8192, 1024, kLayoutSW128),
+                             smem_desc(bU + ks * 1024, 16, 512, kLayoutSW64), idS, 1u);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)   // O += P U (rows 64-127 of [TB; PB] U)
+                    mma_bf16(tmem + kColUO + 32 * u, smem_desc(aTP + ks * 32, 16, 1024, kLayoutSW128),
+                             smem_desc(bU + ks * 1024, 16, 512, kLayoutSW64), idO, 1u);
+                mma_commit(&DONE[u]);
+                mma_commit(&EMPTY[s]);
+            }
+        }
+        if (nchunks > 0) {
+            const int n = nchunks - 1;
+            mbar_wait(&DONE[n & 1], (n >> 1) & 1, abort_flag);
+            tc_fence_after();
+            store_o(tmem, quad, lane, n, bos, len, h, j0, p);
+            tmem_ld32(tmem_addr(tmem, 32 * quad, kColS), S);
+            tmem_wait_ld();
+            if (leader) {
+                mma_commit(FIN);
+                wait_drain(FIN, 0);
+            }
+        }
+        if (p.final_state) {
+            float4 *dst = reinterpret_cast<float4 *>(p.final_state + soff);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kChainTmemCols);
+    }
+    if (tid == 0 && *abort_flag) atomicOr(p.err_word, kDevErrTimeout);
+}
+
+// =============================================================== plan kernel
+// One CTA: checks cu_seqlens (error word), counts each sequence's chunks,
+// writes the record offset of every sequence (exclusive prefix sum), the
+// (sequence, chunk) of every record, the record count, and the longest-first
+// sequence order used by the chain kernel.
+constexpr int kPlanThreads = 1024;
+constexpr int kMaxSortedSeqs = 4096;
+
+__device__ __forceinline__ int64_t seq_len_checked(const int32_t *cu, int i, int n, int64_t total) {
+    if (!cu) return total / n;
+    const int64_t a = cu[i], b = cu[i + 1];
+    return (a < 0 || b < a || b > total) ? 0 : b - a;
+}
+
+__global__ void __launch_bounds__(kPlanThreads)
+kda_split_plan_kernel(const int32_t *cu, int n, int64_t total, int32_t *perm, int32_t *chunk_off,
+                      int2 *chunk_tab, uint32_t *total_chunks, uint32_t *err) {
+    __shared__ int32_t warp_sums[kPlanThreads / 32];
+    __shared__ int32_t carry_s;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    int bad = 0;
+    if (cu) {
+        for (int i = tid; i < n; i += kPlanThreads) {
+            const int64_t a = cu[i], b = cu[i + 1];
+            if (a < 0 || b < a || b > total) bad = 1;
+        }
+        if (tid == 0 && (cu[0] != 0 || cu[n] != total)) bad = 1;
+    }
+    bad = __syncthreads_or(bad);
+    if (tid == 0) {
+        *err = bad ? kDevErrCuSeqlens : kDevErrNone;
+        carry_s = 0;
+    }
+    __syncthreads();
+    // exclusive scan of the chunk counts, 1024 sequences at a time
+    for (int base = 0; base < n; base += kPlanThreads) {
+        const int i = base + tid;
+        const int cnt = (i < n) ? (int)((seq_len_checked(cu, i, n, total) + C - 1) / C) : 0;
+        int incl = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (lane == 31) warp_sums[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            int w = warp_sums[lane];
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, off);
+                if (lane >= off) w += y;
+            }
+            warp_sums[lane] = w;   // inclusive over warps
+        }
+        __syncthreads();
+        const int carry = carry_s;
+        const int excl = carry + (wid > 0 ? warp_sums[wid - 1] : 0) + incl - cnt;
+        if (i < n) chunk_off[i] = excl;
+        __syncthreads();
+        if (tid == kPlanThreads - 1) carry_s = excl + cnt;
+        __syncthreads();
+    }
+    const int nchunks = carry_s;
+    if (tid == 0) {
+        chunk_off[n] = nchunks;
+        *total_chunks = (uint32_t)nchunks;
+    }
+    __syncthreads();
+    for (int c = tid; c < nchunks; c += kPlanThreads) {
+        int lo = 0, hi = n;   // last sequence i with chunk_off[i] <= c
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (chunk_off[mid] <= c) lo = mid;
+            else hi = mid;
+        }
+        chunk_tab[c] = make_int2(lo, c - chunk_off[lo]);
+    }
+    if (!perm) return;
+    for (int i = tid; i < n; i += kPlanThreads) {
+        if (n > kMaxSortedSeqs) {
+            perm[i] = i;
+            continue;
+        }
+        const int64_t li = seq_len_checked(cu, i, n, total);
+        int r = 0;
+        for (int j = 0; j < n; ++j) {
+            const int64_t lj = seq_len_checked(cu, j, n, total);
+            r += (lj > li) || (lj == li && j < i);
+        }
+        perm[r] = i;
+    }
+}
+
+}  // namespace split
+
+// ---- host side -------------------------------------------------------------------
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn_split() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+bool make_map_split(CUtensorMap *m, const void *base, int64_t T, int H, int inner, int box_inner,
+                    CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn_split();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)H, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * 2 * H};
+    const cuuint32_t box[3] = {(cuuint32_t)box_inner, 1, (cuuint32_t)split::C};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct SplitLayout {
+    size_t perm, chunk_off, chunk_tab, recs, total;
+    size_t max_chunks;
+};
+
+SplitLayout split_layout(int num_seqs, int64_t total_tokens, int H) {
+    SplitLayout l;
+    l.max_chunks = (size_t)(total_tokens / split::C) + (size_t)num_seqs;
+    l.perm = kWorkspaceHeader;
+    l.chunk_off = l.perm + round_up((size_t)num_seqs * 4, 256);
+    l.chunk_tab = l.chunk_off + round_up((size_t)(num_seqs + 1) * 4, 256);
+    l.recs = round_up(l.chunk_tab + l.max_chunks * 8, 1024);
+    l.total = l.recs + l.max_chunks * (size_t)H * split::Rec::STRIDE;
+    return l;
+}
+
+}  // namespace
+
+size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H) {
+    return split_layout(num_seqs, total_tokens, H).total;
+}
+
+cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const void *g,
+                                 const void *beta, const float *init_state, const int32_t *cu,
+                                 int num_seqs, int64_t total_tokens, int H, void *o,
+                                 float *final_state, void *workspace, cudaStream_t stream) {
+    using namespace split;
+    const SplitLayout l = split_layout(num_seqs, total_tokens, H);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *err = reinterpret_cast<uint32_t *>(ws);
+    uint32_t *total_chunks = reinterpret_cast<uint32_t *>(ws + 4);
+    int32_t *perm = cu ? reinterpret_cast<int32_t *>(ws + l.perm) : nullptr;
+    int32_t *chunk_off = reinterpret_cast<int32_t *>(ws + l.chunk_off);
+    int2 *chunk_tab = reinterpret_cast<int2 *>(ws + l.chunk_tab);
+
+    CUtensorMap mk, mq, mg, mv;
+    if (!make_map_split(&mk, k, total_tokens, H, DK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_split(&mq, q, total_tokens, H, DK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_split(&mg, g, total_tokens, H, DK, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_split(&mv, v, total_tokens, H, DV, DVT, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    kda_split_plan_kernel<<<1, kPlanThreads, 0, stream>>>(cu, num_seqs, total_tokens, perm,
+                                                          chunk_off, chunk_tab, total_chunks, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    static bool attr_set = false;
+    if (!attr_set) {
+        e = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)PrepSmem::ALLOC);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kda_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)ChainSmem::ALLOC);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    Params prm;
+    prm.k = static_cast<const __nv_bfloat16 *>(k);
+    prm.q = static_cast<const __nv_bfloat16 *>(q);
+    prm.beta = static_cast<const __nv_bfloat16 *>(beta);
+    prm.init_state = init_state;
+    prm.final_state = final_state;
+    prm.o = static_cast<__nv_bfloat16 *>(o);
+    prm.cu = cu;
+    prm.perm = perm;
+    prm.chunk_off = chunk_off;
+    prm.chunk_tab = chunk_tab;
+    prm.total_chunks = total_chunks;
+    prm.recs = ws + l.recs;
+    prm.err_word = err;
+    prm.total_tokens = total_tokens;
+    prm.num_seqs = num_seqs;
+    prm.H = H;
+    const unsigned prep_blocks = (unsigned)(l.max_chunks * (size_t)H);
+    kda_prep_kernel<<<prep_blocks, kPrepThreads, PrepSmem::ALLOC, stream>>>(mk, mq, mg, prm);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const unsigned chain_blocks = (unsigned)((size_t)num_seqs * H * NTILE);
+    kda_chain_kernel<<<chain_blocks, kChainThreads, ChainSmem::ALLOC, stream>>>(mv, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

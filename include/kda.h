@@ -74,9 +74,11 @@ const char *kda_status_string(kda_status s);
 int kda_version(void);
 
 /*
- * Workspace bytes kda_prefill needs for this problem (a multiple of 256; may
- * be 0 only if the library needs none).  Pure host arithmetic, no CUDA call.
- * Returns 0 for arguments kda_prefill would reject.
+ * Workspace bytes for kda_prefill's fastest path on this problem (a multiple
+ * of 256).  For d_k = d_v = 128 this includes one 65 KB record per (chunk of
+ * 64 tokens, head) for the two-kernel tensor-core path, i.e. about
+ * 1 KiB per (token, head): 4.4 GB for 131072 tokens x 32 heads.  Pure host
+ * arithmetic, no CUDA call.  Returns 0 for arguments kda_prefill would reject.
  */
 size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens,
                                   int32_t H, int32_t d_k, int32_t d_v);
@@ -105,9 +107,13 @@ size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens,
  *   o               : [T_total, H, d_v]  dtype, written
  *   final_state     : [N, H, d_k, d_v] fp32, written, or NULL.  May alias
  *                     init_state exactly (same pointer).
- *   workspace       : device buffer of at least
- *                     kda_prefill_workspace_size(...) bytes, 256-byte aligned;
- *                     its contents on entry do not matter.
+ *   workspace       : device buffer, 256-byte aligned, contents on entry do
+ *                     not matter.  At least 256 + 4 N bytes (rounded up to
+ *                     256) are required; with kda_prefill_workspace_size(...)
+ *                     bytes the bf16 d = 128 case runs the two-kernel path
+ *                     (chunk preparation for all chunks in parallel, then the
+ *                     state chain), with less it runs the single-kernel path
+ *                     (same results, slower).
  *
  * Supported: dtype KDA_BF16 or KDA_FP32 with d_k, d_v in {16, 32, 64, 128}.
  * KDA_BF16 with d_k = d_v = 128 runs the tensor-core (tcgen05) path; every
