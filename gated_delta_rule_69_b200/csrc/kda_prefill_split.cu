@@ -52,8 +52,11 @@ struct Rec {
 };
 
 // ---- prep kernel
-constexpr int kPrepThreads = 288;              // warp 0: loads; warps 1-8: the 256-thread group
-constexpr uint32_t kPrepBar = 1;
+// Two independent preparation pipelines per CTA (one CTA per SM), each of
+// 8 warps; pipeline P owns warps 8P..8P+7, its own shared-memory half and
+// its own 256 TMEM columns.
+constexpr int kPipeThreads = 256;
+constexpr int kPrepThreads = 2 * kPipeThreads;
 struct PrepSmem {
     static constexpr uint32_t REC = 0;         // record image (STK, KBAR, TB, PB, EGL)
     static constexpr uint32_t TF = Rec::KBAR;  // T fp32, after Kbar has been stored
@@ -62,12 +65,13 @@ struct PrepSmem {
     static constexpr uint32_t BETA = 99328;    // 64 fp32
     static constexpr uint32_t CSUM = 99584;    // 4 x 128 fp32
     static constexpr uint32_t BARS = 101632;   // 3 mbarriers
-    static constexpr uint32_t MISC = 101696;   // tmem base, abort, slow flag
+    static constexpr uint32_t MISC = 101696;   // tmem base, abort, slow flag, next-item slots at 4, 5
     static constexpr uint32_t SIZE = 101760;
-    static constexpr uint32_t ALLOC = SIZE + 1024;
+    static constexpr uint32_t PIPE = 102400;    // per-pipeline stride
+    static constexpr uint32_t ALLOC = 2 * PIPE + 1024;
 };
-static_assert(2 * PrepSmem::ALLOC <= 228 * 1024, "two prep CTAs per SM");
-constexpr uint32_t kPrepTmemCols = 256;        // [A;P] at 0 (64 cols), W at 64 (128 cols)
+static_assert(PrepSmem::ALLOC <= 232448, "two preparation pipelines per CTA");
+constexpr uint32_t kPrepTmemCols = 512;        // per pipeline: [A;P] at +0 (64 cols), W at +64 (128 cols)
 constexpr uint32_t kRawBytes = 4 * 8192 + 16384;   // k, q (2 boxes each), log_alpha
 
 // ---- chain kernel
@@ -100,6 +104,9 @@ struct Params {
     const int2 *chunk_tab;      // [max_chunks] (sequence, chunk) of each record
     const uint32_t *total_chunks;
     uint8_t *recs;              // records, STRIDE bytes each, index (chunk * H + h)
+    uint32_t *rec_ready;        // [max_chunks * H] set to 1 once a record is complete; null
+                                // when the chain kernel starts only after the prep grid
+    uint32_t *work_next;        // prep items handed out after each pipeline's first one
     uint32_t *err_word;
     int64_t total_tokens;
     int num_seqs, H;
@@ -143,6 +150,34 @@ __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+
+// Record hand-off between the kernels: the writer completes its bulk stores,
+// orders them before a release store of the flag; the reader acquires the
+// flag and orders it before its own bulk (async-proxy) reads.
+__device__ __forceinline__ void publish_flag(uint32_t *flag) {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(1u) : "memory");
+}
+
+__device__ __forceinline__ bool acquire_flag(const uint32_t *flag, volatile uint32_t *abort) {
+    const uint64_t t0 = global_timer_ns();
+    uint32_t ns = 32;
+    while (true) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v) break;
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > 2000000000ull) {
+            *abort = 1u;
+            return false;
+        }
+        __nanosleep(ns);
+        if (ns < 1024) ns <<= 1;
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return true;
+}
+
 __device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity) {
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
@@ -152,46 +187,46 @@ __device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity) {
 
 // =============================================================== prep kernel
 
-__global__ void __launch_bounds__(kPrepThreads, 2)
-kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
-                const __grid_constant__ CUtensorMap tm_g, const Params p) {
-    const uint32_t total = *p.total_chunks;
-    const int h = blockIdx.x % p.H;
-    const uint32_t chunk = blockIdx.x / p.H;
-    if (chunk >= total) return;   // the grid is sized for the largest possible chunk count
-
-    extern __shared__ uint8_t dyn_smem[];
-    uint8_t *sm = dyn_smem + ((1024u - (smem_addr(dyn_smem) & 1023u)) & 1023u);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int2 sc = p.chunk_tab[chunk];
-    int64_t bos, eos;
-    seq_bounds(p, sc.x, bos, eos);
-    const int64_t tok0 = bos + (int64_t)sc.y * C;
-    const int L = (int)min((int64_t)C, eos - tok0);
-    uint8_t *rec = p.recs + ((size_t)chunk * p.H + h) * Rec::STRIDE;
-
+template <int P>
+__device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int tid, int warp, int lane,
+                                              const CUtensorMap &tm_k, const CUtensorMap &tm_q,
+                                              const CUtensorMap &tm_g, const Params &p,
+                                              uint32_t total_items) {
+    constexpr uint32_t BAR = 1 + P;          // this pipeline's 256 threads
+    const int wp = warp - 8 * P;
+    const int pt = tid - P * kPipeThreads;
+    const bool leader = pt == 0;
+    const int quad = warp & 3, half = wp >> 2;
     uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);   // 0 raw, 1 [A;P], 2 W
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + PrepSmem::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     float *beta = reinterpret_cast<float *>(sm + PrepSmem::BETA);
-    if (tid == 0) {
-        mbar_init(&B[0], 2);
-        mbar_init(&B[1], 1);
-        mbar_init(&B[2], 1);
-        misc[1] = 0u;
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(&misc[0], kPrepTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = misc[0];
-
-    if (warp == 0) {
-        if (lane == 0) {
+    // The leader publishes a record one step late: it waits only for the
+    // stores to have read shared memory before it loads the next item, and
+    // for their writes to complete once the next item's first product has
+    // been issued, by which time they have long landed.
+    uint32_t *pending = nullptr;
+    // Items: each pipeline starts with its own, then takes the next free one
+    // from a global counter (SMs do not run at the same speed, so a fixed
+    // share would leave the slowest as the tail).  The leader draws the
+    // following item early in the current one and leaves it in a two-entry
+    // slot, which every thread reads after the current item's last barrier.
+    volatile uint32_t *next_slot = misc + 4;
+    uint32_t item = 2 * blockIdx.x + P;
+#pragma unroll 1
+    for (int it = 0; item < total_items; ++it) {
+        const int h = item % p.H;
+        const uint32_t chunk = item / p.H;
+        const int2 sc = p.chunk_tab[chunk];
+        int64_t bos, eos;
+        seq_bounds(p, sc.x, bos, eos);
+        const int64_t tok0 = bos + (int64_t)sc.y * C;
+        const int L = (int)min((int64_t)C, eos - tok0);
+        uint8_t *rec = p.recs + ((size_t)chunk * p.H + h) * Rec::STRIDE;
+        // Loads.  The leader reaches this point only after the previous
+        // item's record has left shared memory and every thread has passed
+        // that item's last barrier, so the buffers are free.
+        if (leader) {
             mbar_arrive_expect_tx(&B[0], kRawBytes);
             const int t = (int)tok0;
             tma_load_3d(sm + Rec::STK, &tm_k, &B[0], 0, h, t);
@@ -200,18 +235,12 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tma_load_3d(sm + Rec::STK + 16384 + 8192, &tm_q, &B[0], 64, h, t);
             tma_load_3d(sm + PrepSmem::GRAW, &tm_g, &B[0], 0, h, t);
         }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int t = lane + 32 * e;
-            beta[t] = (t < L) ? __bfloat162float(p.beta[(size_t)(tok0 + t) * p.H + h]) : 0.f;
+        if (pt < C) {
+            beta[pt] = (pt < L) ? __bfloat162float(p.beta[(size_t)(tok0 + pt) * p.H + h]) : 0.f;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&B[0]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&B[0]);
-        if (lane == 0) wait_drain(&B[0], 0);   // the copies land before this CTA may exit
-    } else {
-        const int pt = tid - 32;
-        const bool leader = pt == 0;
-        const int quad = warp & 3, half = (warp - 1) >> 2;
+
         prep::Bufs b;
         b.stk = sm + Rec::STK;
         b.khat = sm + PrepSmem::KHAT;
@@ -227,11 +256,13 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         b.csum = reinterpret_cast<float *>(sm + PrepSmem::CSUM);
         b.slow_flag = misc + 2;
 
-        mbar_wait(&B[0], 0, abort_flag);
-        const bool slow = prep::gate<kPrepBar>(b, pt, L);
+        mbar_wait(&B[0], it & 1, abort_flag);
+        const bool slow = prep::gate<BAR>(b, pt, L);
         fence_async_smem();
-        named_barrier(kPrepBar, prep::kGroupThreads);
+        named_barrier(BAR, prep::kGroupThreads);
+        uint32_t drawn = 0;
         if (leader) {
+            drawn = atomicAdd(p.work_next, 1u);   // consumed at the end of the item
             tc_fence_after();
             const uint32_t a0 = smem_addr(sm + Rec::STK), b0 = smem_addr(sm + PrepSmem::KHAT);
             const uint32_t id = idesc_bf16(128, 64, false, false);
@@ -241,10 +272,15 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                          smem_desc(b0 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
                          id, ks > 0 ? 1u : 0u);
             mma_commit(&B[1]);
+            if (pending) {   // before the next bulk store, which the fence would wait for
+                bulk_wait_all();
+                publish_flag(pending);
+                pending = nullptr;
+            }
             bulk_store(rec + Rec::KBAR, sm + Rec::KBAR, 16384);   // Kbar is final
             bulk_commit();
         }
-        mbar_wait(&B[1], 0, abort_flag);
+        mbar_wait(&B[1], it & 1, abort_flag);
         tc_fence_after();
         if (!slow) {
             prep::read_ap(b, tmem, quad, half, lane);
@@ -255,10 +291,10 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         if (leader) bulk_wait_read_all();   // Kbar has left shared memory: T may overwrite it
         tc_fence_before();
-        named_barrier(kPrepBar, prep::kGroupThreads);
-        prep::solve<kPrepBar>(b, pt);
+        named_barrier(BAR, prep::kGroupThreads);
+        prep::solve<BAR>(b, pt);
         fence_async_smem();
-        named_barrier(kPrepBar, prep::kGroupThreads);
+        named_barrier(BAR, prep::kGroupThreads);
         if (leader) {
             tc_fence_after();
             const uint32_t aT = smem_addr(sm + Rec::TB), bK = smem_addr(sm + Rec::STK);
@@ -269,26 +305,69 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                          smem_desc(bK + ks * 2048, 16384, 1024, kLayoutSW128), idW, ks > 0 ? 1u : 0u);
             mma_commit(&B[2]);
         }
-        mbar_wait(&B[2], 0, abort_flag);
+        mbar_wait(&B[2], it & 1, abort_flag);
         tc_fence_after();
         prep::read_w(b, tmem + 64, quad, half, lane);
+        if (leader) next_slot[(it + 1) & 1] = 2 * gridDim.x + drawn;
         fence_async_smem();
         tc_fence_before();
-        named_barrier(kPrepBar, prep::kGroupThreads);
+        named_barrier(BAR, prep::kGroupThreads);
+        const uint32_t next_item = next_slot[(it + 1) & 1];
         if (leader) {
             bulk_store(rec + Rec::STK, sm + Rec::STK, 32768);
             bulk_store(rec + Rec::TB, sm + Rec::TB, Rec::BYTES - Rec::TB);   // TB, PB, exp(G_L)
             bulk_commit();
-            bulk_wait_all();
+            bulk_wait_read_all();
+            if (p.rec_ready) pending = p.rec_ready + (size_t)chunk * p.H + h;
         }
+        item = next_item;
     }
+    if (leader) {
+        bulk_wait_all();
+        if (pending) publish_flag(pending);
+        if (*abort_flag) atomicOr(p.err_word, kDevErrTimeout);
+    }
+}
+
+__global__ void __launch_bounds__(kPrepThreads, 1)
+kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                const __grid_constant__ CUtensorMap tm_g, const Params p) {
+    // Let a dependent chain kernel start now: it waits on per-record flags,
+    // not on this grid's completion.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const uint32_t total_items = *p.total_chunks * (uint32_t)p.H;
+    if (2 * blockIdx.x >= total_items) return;
+
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t *sm0 = dyn_smem + ((1024u - (smem_addr(dyn_smem) & 1023u)) & 1023u);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int P = warp / 8;
+    uint8_t *sm = sm0 + P * PrepSmem::PIPE;
+    uint32_t *misc0 = reinterpret_cast<uint32_t *>(sm0 + PrepSmem::MISC);
+    if (tid == 0 || tid == kPipeThreads) {
+        uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);
+        mbar_init(&B[0], 3);   // the leader's expect_tx, and one arrive per beta warp
+        mbar_init(&B[1], 1);
+        mbar_init(&B[2], 1);
+        reinterpret_cast<uint32_t *>(sm + PrepSmem::MISC)[1] = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&misc0[0], kPrepTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc0[0] + 256u * P;
+    if (P == 0) prep_pipeline<0>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
+    else prep_pipeline<1>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kPrepTmemCols);
+        tmem_dealloc(misc0[0], kPrepTmemCols);
     }
-    if (tid == 0 && *abort_flag) atomicOr(p.err_word, kDevErrTimeout);
 }
 
 // =============================================================== chain kernel
@@ -373,7 +452,9 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 if (n >= NS) mbar_wait(&EMPTY[s], ((n / NS) - 1) & 1, abort_flag);
                 if (*abort_flag) break;
                 uint8_t *slot = sm + ChainSmem::SLOT + s * ChainSmem::SLOT_STRIDE;
-                const uint8_t *rec = p.recs + ((rec0 + n) * p.H + h) * Rec::STRIDE;
+                const size_t ri = (rec0 + n) * p.H + h;
+                const uint8_t *rec = p.recs + ri * Rec::STRIDE;
+                if (p.rec_ready && !acquire_flag(p.rec_ready + ri, abort_flag)) break;   // the record is complete
                 mbar_arrive_expect_tx(&FULL[s], Rec::BYTES + 4096);
                 bulk_load(slot + Rec::STK, rec + Rec::STK, 32768, &FULL[s]);
                 bulk_load(slot + Rec::KBAR, rec + Rec::KBAR, 16384, &FULL[s]);
@@ -519,7 +600,10 @@ __device__ __forceinline__ int64_t seq_len_checked(const int32_t *cu, int i, int
 
 __global__ void __launch_bounds__(kPlanThreads)
 kda_split_plan_kernel(const int32_t *cu, int n, int64_t total, int32_t *perm, int32_t *chunk_off,
-                      int2 *chunk_tab, uint32_t *total_chunks, uint32_t *err) {
+                      int2 *chunk_tab, uint32_t *total_chunks, uint32_t *err,
+                      uint32_t *rec_ready, size_t n_flags, uint32_t *work_next) {
+    for (size_t i = threadIdx.x; i < n_flags; i += kPlanThreads) rec_ready[i] = 0u;
+    if (threadIdx.x == 0) *work_next = 0u;
     __shared__ int32_t warp_sums[kPlanThreads / 32];
     __shared__ int32_t carry_s;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -638,7 +722,7 @@ bool make_map_split(CUtensorMap *m, const void *base, int64_t T, int H, int inne
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct SplitLayout {
-    size_t perm, chunk_off, chunk_tab, recs, total;
+    size_t perm, chunk_off, chunk_tab, flags, recs, total;
     size_t max_chunks;
 };
 
@@ -648,7 +732,8 @@ SplitLayout split_layout(int num_seqs, int64_t total_tokens, int H) {
     l.perm = kWorkspaceHeader;
     l.chunk_off = l.perm + round_up((size_t)num_seqs * 4, 256);
     l.chunk_tab = l.chunk_off + round_up((size_t)(num_seqs + 1) * 4, 256);
-    l.recs = round_up(l.chunk_tab + l.max_chunks * 8, 1024);
+    l.flags = round_up(l.chunk_tab + l.max_chunks * 8, 256);
+    l.recs = round_up(l.flags + l.max_chunks * (size_t)H * 4, 1024);
     l.total = l.recs + l.max_chunks * (size_t)H * split::Rec::STRIDE;
     return l;
 }
@@ -668,6 +753,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint32_t *err = reinterpret_cast<uint32_t *>(ws);
     uint32_t *total_chunks = reinterpret_cast<uint32_t *>(ws + 4);
+    uint32_t *work_next = reinterpret_cast<uint32_t *>(ws + 8);
     int32_t *perm = cu ? reinterpret_cast<int32_t *>(ws + l.perm) : nullptr;
     int32_t *chunk_off = reinterpret_cast<int32_t *>(ws + l.chunk_off);
     int2 *chunk_tab = reinterpret_cast<int2 *>(ws + l.chunk_tab);
@@ -678,8 +764,25 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         !make_map_split(&mg, g, total_tokens, H, DK, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map_split(&mv, v, total_tokens, H, DV, DVT, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
+    // Prep runs as a persistent grid (one CTA per SM).  When the chain needs
+    // few SMs, the prep grid leaves those SMs free and the chain kernel is
+    // launched as a programmatic dependent of it, so that it starts at once
+    // and consumes records as they are published; otherwise the two kernels
+    // run one after the other and the records need no flags.
+    static int sm_count = 0;
+    if (!sm_count) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            sm_count = 148;
+    }
+    const unsigned chain_blocks = (unsigned)((size_t)num_seqs * H * NTILE);
+    const bool overlap = chain_blocks * 10 <= (unsigned)sm_count * 6;   // chain needs <= 60 % of SMs
+    uint32_t *rec_ready = overlap ? reinterpret_cast<uint32_t *>(ws + l.flags) : nullptr;
     kda_split_plan_kernel<<<1, kPlanThreads, 0, stream>>>(cu, num_seqs, total_tokens, perm,
-                                                          chunk_off, chunk_tab, total_chunks, err);
+                                                          chunk_off, chunk_tab, total_chunks, err,
+                                                          rec_ready, overlap ? l.max_chunks * (size_t)H : 0,
+                                                          work_next);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     static bool attr_set = false;
@@ -705,16 +808,30 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     prm.chunk_tab = chunk_tab;
     prm.total_chunks = total_chunks;
     prm.recs = ws + l.recs;
+    prm.rec_ready = rec_ready;
+    prm.work_next = work_next;
     prm.err_word = err;
     prm.total_tokens = total_tokens;
     prm.num_seqs = num_seqs;
     prm.H = H;
-    const unsigned prep_blocks = (unsigned)(l.max_chunks * (size_t)H);
-    kda_prep_kernel<<<prep_blocks, kPrepThreads, PrepSmem::ALLOC, stream>>>(mk, mq, mg, prm);
+    const size_t max_items = l.max_chunks * (size_t)H;
+    size_t prep_blocks = (size_t)(overlap ? sm_count - chain_blocks : sm_count);
+    if (2 * prep_blocks > max_items) prep_blocks = (max_items + 1) / 2;
+    kda_prep_kernel<<<(unsigned)prep_blocks, kPrepThreads, PrepSmem::ALLOC, stream>>>(mk, mq, mg, prm);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const unsigned chain_blocks = (unsigned)((size_t)num_seqs * H * NTILE);
-    kda_chain_kernel<<<chain_blocks, kChainThreads, ChainSmem::ALLOC, stream>>>(mv, prm);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(chain_blocks);
+    cfg.blockDim = dim3(kChainThreads);
+    cfg.dynamicSmemBytes = ChainSmem::ALLOC;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = overlap ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kda_chain_kernel, mv, prm);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
