@@ -40,15 +40,23 @@ constexpr int DV = 128;
 constexpr int DVT = 32;
 constexpr int NTILE = DV / DVT;
 
-// ---- the per-(chunk, head) record, also the chain kernel's ring-slot layout
+// ---- the per-(chunk, head) record: bf16 tensor-core operands in the
+// K-major 128-byte-swizzled layout the chain kernel's products read.
+//   MP = -Kbar^T W      [128 c_out][128 c_in]  (2 K-atoms x 16 KB)
+//   YT = Kbar^T T_beta  [128 c][64 t]          (1 K-atom)
+//   QP = Qtil - P W     [64 t][128 c]          (2 K-atoms x 8 KB)
+//   ZB = P T_beta       [64 t][64 i]           (1 K-atom)
+//   EGL = exp(G_L)      128 fp32
+// so that, for a chunk with input state S and values V,
+//   S_next = Diag(exp(G_L)) S + MP S + YT V,   O = QP S + ZB V.
 struct Rec {
-    static constexpr uint32_t STK = 0;         // [-W rows 0-63 | Qtil rows 64-127], 2 K-atoms x 16 KB
-    static constexpr uint32_t KBAR = 32768;    // Kbar [64 t][128 c], 2 K-atoms x 8 KB
-    static constexpr uint32_t TB = 49152;      // T diag(beta) [64 t][64 i]; TB+PB form one M=128 operand
-    static constexpr uint32_t PB = 57344;      // P [64 t][64 i]
-    static constexpr uint32_t EGL = 65536;     // 128 fp32
-    static constexpr uint32_t BYTES = 66048;   // bytes carried
-    static constexpr uint32_t STRIDE = 66560;  // record stride (1024-aligned)
+    static constexpr uint32_t MP = 0;
+    static constexpr uint32_t YT = 32768;
+    static constexpr uint32_t QP = 49152;
+    static constexpr uint32_t ZB = 65536;
+    static constexpr uint32_t EGL = 73728;
+    static constexpr uint32_t BYTES = 74240;   // bytes carried
+    static constexpr uint32_t STRIDE = 74752;  // record stride (1024-aligned)
 };
 
 // ---- prep kernel
@@ -58,40 +66,53 @@ struct Rec {
 constexpr int kPipeThreads = 256;
 constexpr int kPrepThreads = 2 * kPipeThreads;
 struct PrepSmem {
-    static constexpr uint32_t REC = 0;         // record image (STK, KBAR, TB, PB, EGL)
-    static constexpr uint32_t TF = Rec::KBAR;  // T fp32, after Kbar has been stored
-    static constexpr uint32_t KHAT = 66560;    // Khat, then A fp32
-    static constexpr uint32_t GRAW = 82944;    // raw log_alpha, then solve scratch
-    static constexpr uint32_t BETA = 99328;    // 64 fp32
-    static constexpr uint32_t CSUM = 99584;    // 4 x 128 fp32
-    static constexpr uint32_t BARS = 101632;   // 3 mbarriers
-    static constexpr uint32_t MISC = 101696;   // tmem base, abort, slow flag, next-item slots at 4, 5
-    static constexpr uint32_t SIZE = 101760;
-    static constexpr uint32_t PIPE = 102400;    // per-pipeline stride
+    static constexpr uint32_t STK = 0;         // raw k | q -> [Ktil | Qtil] -> [-W | QP], 2 K-atoms x 16 KB
+                                               // (rows 0-63 and 64-127 of each atom)
+    static constexpr uint32_t KBAR = 32768;    // Kbar [64 t][128 c] (2 K-atoms x 8 KB), then YT
+    static constexpr uint32_t TB = 49152;      // T diag(beta) [64 t][64 i], then ZB
+    static constexpr uint32_t PB = 57344;      // P [64 t][64 i]
+    static constexpr uint32_t EGL = 65536;     // 128 fp32
+    static constexpr uint32_t KHAT = 66560;    // Khat, then A fp32, then MP K-atom 0
+    static constexpr uint32_t GRAW = 82944;    // raw log_alpha, then T fp32, then MP K-atom 1
+    static constexpr uint32_t XF = 99328;      // solve scratch (4608 bytes)
+    static constexpr uint32_t BETA = 103936;   // 64 fp32
+    static constexpr uint32_t CSUM = 104192;   // 4 x 128 fp32
+    static constexpr uint32_t BARS = 106240;   // 5 mbarriers
+    static constexpr uint32_t MISC = 106304;   // tmem base, abort, slow flag, next-item slots at 4, 5
+    static constexpr uint32_t SIZE = 106368;
+    static constexpr uint32_t PIPE = 107520;   // per-pipeline stride
     static constexpr uint32_t ALLOC = 2 * PIPE + 1024;
 };
 static_assert(PrepSmem::ALLOC <= 232448, "two preparation pipelines per CTA");
-constexpr uint32_t kPrepTmemCols = 512;        // per pipeline: [A;P] at +0 (64 cols), W at +64 (128 cols)
+// per pipeline (256 columns): [A;P] at 0 and W at 64; then MP at 0, YT at 128,
+// ZB at 192 (M = 64); then -P W at 0 (M = 64)
+constexpr uint32_t kPrepTmemCols = 512;
 constexpr uint32_t kRawBytes = 4 * 8192 + 16384;   // k, q (2 boxes each), log_alpha
 
 // ---- chain kernel
-constexpr int kChainThreads = 160;             // warp 0: loads; warps 1-4: the chain
-constexpr uint32_t kChainBar = 1;
-constexpr int NS = 3;                          // ring stages
+constexpr int kChainThreads = 192;             // warp 0: loads; warps 1-4: the chain; warp 5: products
+constexpr int NSA = 3;                         // ring A: state-update operands + v slice
+constexpr int NSB = 2;                         // ring B: output operands
 struct ChainSmem {
-    static constexpr uint32_t SLOT = 0;        // NS x (record + v slice)
-    static constexpr uint32_t VT_OFF = Rec::STRIDE;           // v slice [64 t][32 j], 64-byte swizzle
-    static constexpr uint32_t SLOT_STRIDE = Rec::STRIDE + 4096;   // 70656
-    static constexpr uint32_t SB = NS * SLOT_STRIDE;          // S bf16 [128 c][32 j]
-    static constexpr uint32_t UB = SB + 8192;                 // U bf16 [64 t][32 j]
-    static constexpr uint32_t BARS = UB + 4096;
+    static constexpr uint32_t A_MP = 0, A_YT = 32768, A_V = 49152, A_EGL = 53248;
+    static constexpr uint32_t A_STRIDE = 54272;
+    static constexpr uint32_t B_QP = 0, B_ZB = 16384;
+    static constexpr uint32_t B_STRIDE = 24576;
+    static constexpr uint32_t RA = 0;
+    static constexpr uint32_t RB = NSA * A_STRIDE;          // 162816
+    static constexpr uint32_t SB = RB + NSB * B_STRIDE;     // 2 x S bf16 [128 c][32 j], 64-byte swizzle
+    static constexpr uint32_t BARS = SB + 2 * 8192;
     static constexpr uint32_t MISC = BARS + 128;
     static constexpr uint32_t SIZE = MISC + 64;
     static constexpr uint32_t ALLOC = SIZE + 1024;
 };
 static_assert(ChainSmem::ALLOC <= 232448, "chain shared memory");
-constexpr uint32_t kChainTmemCols = 256;
-constexpr uint32_t kColUp = 0, kColUO = 64, kColS = 128;   // U' x2, [-W S; O] x2, S
+static_assert(Rec::YT == Rec::MP + 32768 && ChainSmem::A_YT == ChainSmem::A_MP + 32768,
+              "MP and YT travel as one copy");
+static_assert(Rec::ZB == Rec::QP + 16384 && ChainSmem::B_ZB == ChainSmem::B_QP + 16384,
+              "QP and ZB travel as one copy");
+constexpr uint32_t kChainTmemCols = 128;
+constexpr uint32_t kColS = 0, kColO = 32;      // S (32 columns), O x2 (M = 64, 32 columns each)
 
 struct Params {
     const __nv_bfloat16 *k, *q, *beta;
@@ -187,6 +208,83 @@ __device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity) {
 
 // =============================================================== prep kernel
 
+// ---- read-outs of the record's products (TMEM -> bf16, K-major 128-byte
+// swizzle).  A warp of TMEM quadrant `quad` handles half `half` of the
+// columns.  M = 64 products keep row r in lane (r mod 16) + 32 (r / 16).
+__device__ __forceinline__ void store8(uint8_t *tile, uint32_t row, uint32_t col, const float *v) {
+    uint4 pk;
+    pk.x = pack_bf16x2(v[0], v[1]);
+    pk.y = pack_bf16x2(v[2], v[3]);
+    pk.z = pack_bf16x2(v[4], v[5]);
+    pk.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4 *>(tile + sw128_off(row, col)) = pk;
+}
+
+// MP [128 c_out][128 c_in]: K-atom `half` holds c_in 64 half .. + 63.
+__device__ __forceinline__ void write_mp(uint8_t *mp, uint32_t tmem, int quad, int half, int lane) {
+    uint8_t *atom = mp + half * 16384;
+    const int row = 32 * quad + lane;
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+        float v[32];
+        tmem_ld32(tmem_addr(tmem, 32 * quad, 64 * half + 32 * part), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) store8(atom, row, 32 * part + j, v + j);
+    }
+}
+
+// YT [128 c][64 t].
+__device__ __forceinline__ void write_yt(uint8_t *yt, uint32_t tmem, int quad, int half, int lane) {
+    float v[32];
+    tmem_ld32(tmem_addr(tmem, 32 * quad, 32 * half), v);
+    tmem_wait_ld();
+    const int row = 32 * quad + lane;
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) store8(yt, row, 32 * half + j, v + j);
+}
+
+// ZB [64 t][64 i] (M = 64).
+__device__ __forceinline__ void write_zb(uint8_t *zb, uint32_t tmem, int quad, int half, int lane) {
+    float v[32];
+    tmem_ld32(tmem_addr(tmem, 32 * quad, 32 * half), v);
+    tmem_wait_ld();
+    if (lane < 16) {
+        const int t = 16 * quad + lane;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) store8(zb, t, 32 * half + j, v + j);
+    }
+}
+
+// QP = Qtil + P (-W) (M = 64), in place over Qtil: rows 64-127 of the two
+// 16 KB K-atoms of `stk`, K-atom `half` holding channels 64 half .. + 63.
+__device__ __forceinline__ void write_qp(uint8_t *stk, uint32_t tmem, int quad, int half, int lane) {
+    uint8_t *atom = stk + half * 16384;
+    const int t = 16 * quad + lane;
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+        float v[32];
+        tmem_ld32(tmem_addr(tmem, 32 * quad, 64 * half + 32 * part), v);
+        tmem_wait_ld();
+        if (lane < 16) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+                uint4 *q8 = reinterpret_cast<uint4 *>(atom + sw128_off(64 + t, 32 * part + j));
+                const uint4 qv = *q8;
+                const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&w[e]);
+                    f[2 * e] = __low2float(h2) + v[j + 2 * e];
+                    f[2 * e + 1] = __high2float(h2) + v[j + 2 * e + 1];
+                }
+                store8(atom, 64 + t, 32 * part + j, f);
+            }
+        }
+    }
+}
+
 template <int P>
 __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int tid, int warp, int lane,
                                               const CUtensorMap &tm_k, const CUtensorMap &tm_q,
@@ -197,7 +295,7 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
     const int pt = tid - P * kPipeThreads;
     const bool leader = pt == 0;
     const int quad = warp & 3, half = wp >> 2;
-    uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);   // 0 raw, 1 [A;P], 2 W
+    uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);   // raw, [A;P], W, MP/YT/ZB, PW
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + PrepSmem::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     float *beta = reinterpret_cast<float *>(sm + PrepSmem::BETA);
@@ -229,10 +327,10 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         if (leader) {
             mbar_arrive_expect_tx(&B[0], kRawBytes);
             const int t = (int)tok0;
-            tma_load_3d(sm + Rec::STK, &tm_k, &B[0], 0, h, t);
-            tma_load_3d(sm + Rec::STK + 16384, &tm_k, &B[0], 64, h, t);
-            tma_load_3d(sm + Rec::STK + 8192, &tm_q, &B[0], 0, h, t);
-            tma_load_3d(sm + Rec::STK + 16384 + 8192, &tm_q, &B[0], 64, h, t);
+            tma_load_3d(sm + PrepSmem::STK, &tm_k, &B[0], 0, h, t);
+            tma_load_3d(sm + PrepSmem::STK + 16384, &tm_k, &B[0], 64, h, t);
+            tma_load_3d(sm + PrepSmem::STK + 8192, &tm_q, &B[0], 0, h, t);
+            tma_load_3d(sm + PrepSmem::STK + 16384 + 8192, &tm_q, &B[0], 64, h, t);
             tma_load_3d(sm + PrepSmem::GRAW, &tm_g, &B[0], 0, h, t);
         }
         if (pt < C) {
@@ -242,17 +340,17 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         }
 
         prep::Bufs b;
-        b.stk = sm + Rec::STK;
+        b.stk = sm + PrepSmem::STK;
         b.khat = sm + PrepSmem::KHAT;
-        b.kbar = sm + Rec::KBAR;
+        b.kbar = sm + PrepSmem::KBAR;
         b.graw = sm + PrepSmem::GRAW;
         b.af = reinterpret_cast<float *>(sm + PrepSmem::KHAT);
-        b.tf = reinterpret_cast<float *>(sm + PrepSmem::TF);
-        b.xf = reinterpret_cast<float *>(sm + PrepSmem::GRAW);
-        b.tb = sm + Rec::TB;
-        b.pb = sm + Rec::PB;
+        b.tf = reinterpret_cast<float *>(sm + PrepSmem::GRAW);
+        b.xf = reinterpret_cast<float *>(sm + PrepSmem::XF);
+        b.tb = sm + PrepSmem::TB;
+        b.pb = sm + PrepSmem::PB;
         b.beta = beta;
-        b.egl = reinterpret_cast<float *>(sm + Rec::EGL);
+        b.egl = reinterpret_cast<float *>(sm + PrepSmem::EGL);
         b.csum = reinterpret_cast<float *>(sm + PrepSmem::CSUM);
         b.slow_flag = misc + 2;
 
@@ -264,7 +362,7 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         if (leader) {
             drawn = atomicAdd(p.work_next, 1u);   // consumed at the end of the item
             tc_fence_after();
-            const uint32_t a0 = smem_addr(sm + Rec::STK), b0 = smem_addr(sm + PrepSmem::KHAT);
+            const uint32_t a0 = smem_addr(sm + PrepSmem::STK), b0 = smem_addr(sm + PrepSmem::KHAT);
             const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)   // [Ktil; Qtil] Khat^T
@@ -272,13 +370,11 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
                          smem_desc(b0 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
                          id, ks > 0 ? 1u : 0u);
             mma_commit(&B[1]);
-            if (pending) {   // before the next bulk store, which the fence would wait for
+            if (pending) {
                 bulk_wait_all();
                 publish_flag(pending);
                 pending = nullptr;
             }
-            bulk_store(rec + Rec::KBAR, sm + Rec::KBAR, 16384);   // Kbar is final
-            bulk_commit();
         }
         mbar_wait(&B[1], it & 1, abort_flag);
         tc_fence_after();
@@ -289,33 +385,80 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
             prep::pairwise(b, pt, L, p.k + ((size_t)tok0 * p.H + h) * DK,
                            p.q + ((size_t)tok0 * p.H + h) * DK, stride);
         }
-        if (leader) bulk_wait_read_all();   // Kbar has left shared memory: T may overwrite it
         tc_fence_before();
         named_barrier(BAR, prep::kGroupThreads);
         prep::solve<BAR>(b, pt);
         fence_async_smem();
         named_barrier(BAR, prep::kGroupThreads);
+        const uint32_t sK = smem_addr(sm + PrepSmem::STK), sKb = smem_addr(sm + PrepSmem::KBAR);
+        const uint32_t sT = smem_addr(sm + PrepSmem::TB), sP = smem_addr(sm + PrepSmem::PB);
         if (leader) {
             tc_fence_after();
-            const uint32_t aT = smem_addr(sm + Rec::TB), bK = smem_addr(sm + Rec::STK);
             const uint32_t idW = idesc_bf16(64, DK, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)   // W = T diag(beta) Ktil
-                mma_bf16(tmem + 64, smem_desc(aT + ks * 32, 16, 1024, kLayoutSW128),
-                         smem_desc(bK + ks * 2048, 16384, 1024, kLayoutSW128), idW, ks > 0 ? 1u : 0u);
+                mma_bf16(tmem + 64, smem_desc(sT + ks * 32, 16, 1024, kLayoutSW128),
+                         smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idW, ks > 0 ? 1u : 0u);
             mma_commit(&B[2]);
         }
         mbar_wait(&B[2], it & 1, abort_flag);
         tc_fence_after();
-        prep::read_w(b, tmem + 64, quad, half, lane);
+        prep::read_w(b, tmem + 64, quad, half, lane);   // -W over Ktil
+        fence_async_smem();
+        tc_fence_before();
+        named_barrier(BAR, prep::kGroupThreads);
+        if (leader) {
+            tc_fence_after();
+            const uint32_t idM = idesc_bf16(128, DK, true, true);
+            const uint32_t idY = idesc_bf16(128, C, true, true);
+            const uint32_t idZ = idesc_bf16(64, C, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {   // K = 64 tokens
+                const uint64_t aKb = smem_desc(sKb + ks * 2048, 8192, 1024, kLayoutSW128);   // Kbar^T
+                // MP = Kbar^T (-W)
+                mma_bf16(tmem, aKb, smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idM,
+                         ks > 0 ? 1u : 0u);
+                // YT = Kbar^T T_beta
+                mma_bf16(tmem + 128, aKb, smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idY,
+                         ks > 0 ? 1u : 0u);
+                // ZB = P T_beta
+                mma_bf16(tmem + 192, smem_desc(sP + ks * 32, 16, 1024, kLayoutSW128),
+                         smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idZ, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(&B[3]);
+        }
+        mbar_wait(&B[3], it & 1, abort_flag);
+        tc_fence_after();
+        write_mp(sm + PrepSmem::KHAT, tmem, quad, half, lane);
+        tc_fence_before();
+        named_barrier(BAR, prep::kGroupThreads);
+        if (leader) {
+            tc_fence_after();
+            const uint32_t idQ = idesc_bf16(64, DK, false, true);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)   // P (-W), into the columns MP has left
+                mma_bf16(tmem, smem_desc(sP + ks * 32, 16, 1024, kLayoutSW128),
+                         smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idQ, ks > 0 ? 1u : 0u);
+            mma_commit(&B[4]);
+        }
+        // Kbar, T_beta are no longer read: YT and ZB go over them
+        write_yt(sm + PrepSmem::KBAR, tmem + 128, quad, half, lane);
+        write_zb(sm + PrepSmem::TB, tmem + 192, quad, half, lane);
+        mbar_wait(&B[4], it & 1, abort_flag);
+        tc_fence_after();
+        write_qp(sm + PrepSmem::STK, tmem, quad, half, lane);
         if (leader) next_slot[(it + 1) & 1] = 2 * gridDim.x + drawn;
         fence_async_smem();
         tc_fence_before();
         named_barrier(BAR, prep::kGroupThreads);
         const uint32_t next_item = next_slot[(it + 1) & 1];
         if (leader) {
-            bulk_store(rec + Rec::STK, sm + Rec::STK, 32768);
-            bulk_store(rec + Rec::TB, sm + Rec::TB, Rec::BYTES - Rec::TB);   // TB, PB, exp(G_L)
+            bulk_store(rec + Rec::MP, sm + PrepSmem::KHAT, 32768);
+            bulk_store(rec + Rec::YT, sm + PrepSmem::KBAR, 16384);
+            bulk_store(rec + Rec::QP, sm + PrepSmem::STK + 8192, 8192);
+            bulk_store(rec + Rec::QP + 8192, sm + PrepSmem::STK + 16384 + 8192, 8192);
+            bulk_store(rec + Rec::ZB, sm + PrepSmem::TB, 8192);
+            bulk_store(rec + Rec::EGL, sm + PrepSmem::EGL, 512);
             bulk_commit();
             bulk_wait_read_all();
             if (p.rec_ready) pending = p.rec_ready + (size_t)chunk * p.H + h;
@@ -347,8 +490,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     if (tid == 0 || tid == kPipeThreads) {
         uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);
         mbar_init(&B[0], 3);   // the leader's expect_tx, and one arrive per beta warp
-        mbar_init(&B[1], 1);
-        mbar_init(&B[2], 1);
+        for (int i = 1; i < 5; ++i) mbar_init(&B[i], 1);
         reinterpret_cast<uint32_t *>(sm + PrepSmem::MISC)[1] = 0u;
         fence_mbar_init();
     }
@@ -384,15 +526,15 @@ __device__ __forceinline__ void store_bf16_row_sw64(uint8_t *tile, int row, cons
     }
 }
 
-// O rows of chunk m: rows 64-127 of [-W S; O] (lanes 64-127, quadrants 2-3).
+// O of chunk m from TMEM (M = 64 layout: row t in lane (t mod 16) + 32 (t / 16))
+// to global memory; the whole warp reads, lanes 0-15 hold rows.
 __device__ __forceinline__ void store_o(uint32_t tmem, int quad, int lane, int m, int64_t bos,
                                         int64_t len, int h, int j0, const Params &p) {
-    if (quad < 2) return;
     float v[32];
-    tmem_ld32(tmem_addr(tmem, 32 * quad, kColUO + 32 * (m & 1)), v);
+    tmem_ld32(tmem_addr(tmem, 32 * quad, kColO + 32 * (m & 1)), v);
     tmem_wait_ld();
-    const int t = 32 * (quad - 2) + lane;
-    if ((int64_t)m * C + t < len) {
+    const int t = 16 * quad + lane;
+    if (lane < 16 && (int64_t)m * C + t < len) {
         uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)(bos + (int64_t)m * C + t) * p.H + h) * DV + j0);
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
@@ -406,6 +548,12 @@ __device__ __forceinline__ void store_o(uint32_t tmem, int quad, int lane, int m
     }
 }
 
+// Per chunk n, with S_n (fp32) in TMEM:
+//   chain warps: S_n -> bf16 SB[n mod 2];  TMEM S <- Diag(exp(G_L)) S_n
+//   product warp, S products (the serial path):  S += MP SB,  S += YT V
+//                 O products (off it):           O[n mod 2] = QP SB + ZB V
+// The chain warps read the O of chunk n out while chunk n + 1 runs; the
+// product warp issues chunk n's O products while they convert S_{n+1}.
 __global__ void __launch_bounds__(kChainThreads, 1)
 kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     extern __shared__ uint8_t dyn_smem[];
@@ -422,14 +570,17 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     const int j0 = tile * DVT;
     const size_t rec0 = (size_t)p.chunk_off[seq];
 
-    // mbarriers: FULL[NS], EMPTY[NS], U_FULL[2], DONE[2], FINAL
+    // mbarriers: FULLA[NSA], EMPTYA[NSA], FULLB[NSB], EMPTYB[NSB], SDONE, ODONE[2], FIN, SREADY
     uint64_t *B = reinterpret_cast<uint64_t *>(sm + ChainSmem::BARS);
-    uint64_t *FULL = B, *EMPTY = B + NS, *UFULL = B + 2 * NS, *DONE = B + 2 * NS + 2,
-             *FIN = B + 2 * NS + 4;
+    uint64_t *FULLA = B, *EMPTYA = B + NSA, *FULLB = B + 2 * NSA, *EMPTYB = B + 2 * NSA + NSB;
+    uint64_t *SDONE = B + 2 * NSA + 2 * NSB, *ODONE = SDONE + 1, *FIN = SDONE + 3, *SREADY = SDONE + 4;
+    constexpr int kBars = 2 * NSA + 2 * NSB + 5;
+    static_assert(kBars * 8 <= 128, "barrier area");
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + ChainSmem::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     if (tid == 0) {
-        for (int i = 0; i < 2 * NS + 5; ++i) mbar_init(&B[i], 1);
+        for (int i = 0; i < kBars - 1; ++i) mbar_init(&B[i], 1);
+        mbar_init(SREADY, 4);   // one arrive per chain warp
         misc[1] = 0u;
         fence_mbar_init();
     }
@@ -446,29 +597,80 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         // ---------------------------------------------- loader: records + v slices
         if (lane == 0 && nchunks > 0) {
             tma_prefetch_desc(&tm_v);
-            int issued = 0;
+            int issued_a = 0, issued_b = 0;
             for (int n = 0; n < nchunks; ++n) {
-                const int s = n % NS;
-                if (n >= NS) mbar_wait(&EMPTY[s], ((n / NS) - 1) & 1, abort_flag);
+                const int sa = n % NSA, sb = n % NSB;
+                if (n >= NSA) mbar_wait(&EMPTYA[sa], ((n / NSA) - 1) & 1, abort_flag);
                 if (*abort_flag) break;
-                uint8_t *slot = sm + ChainSmem::SLOT + s * ChainSmem::SLOT_STRIDE;
                 const size_t ri = (rec0 + n) * p.H + h;
                 const uint8_t *rec = p.recs + ri * Rec::STRIDE;
                 if (p.rec_ready && !acquire_flag(p.rec_ready + ri, abort_flag)) break;   // the record is complete
-                mbar_arrive_expect_tx(&FULL[s], Rec::BYTES + 4096);
-                bulk_load(slot + Rec::STK, rec + Rec::STK, 32768, &FULL[s]);
-                bulk_load(slot + Rec::KBAR, rec + Rec::KBAR, 16384, &FULL[s]);
-                bulk_load(slot + Rec::TB, rec + Rec::TB, Rec::BYTES - Rec::TB, &FULL[s]);
-                tma_load_3d(slot + ChainSmem::VT_OFF, &tm_v, &FULL[s], j0, h, (int)(bos + (int64_t)n * C));
-                issued = n + 1;
+                uint8_t *slot_a = sm + ChainSmem::RA + sa * ChainSmem::A_STRIDE;
+                mbar_arrive_expect_tx(&FULLA[sa], 49152 + 512 + 4096);
+                bulk_load(slot_a + ChainSmem::A_MP, rec + Rec::MP, 49152, &FULLA[sa]);   // MP, YT
+                bulk_load(slot_a + ChainSmem::A_EGL, rec + Rec::EGL, 512, &FULLA[sa]);
+                tma_load_3d(slot_a + ChainSmem::A_V, &tm_v, &FULLA[sa], j0, h, (int)(bos + (int64_t)n * C));
+                issued_a = n + 1;
+                if (n >= NSB) mbar_wait(&EMPTYB[sb], ((n / NSB) - 1) & 1, abort_flag);
+                if (*abort_flag) break;
+                uint8_t *slot_b = sm + ChainSmem::RB + sb * ChainSmem::B_STRIDE;
+                mbar_arrive_expect_tx(&FULLB[sb], 24576);
+                bulk_load(slot_b + ChainSmem::B_QP, rec + Rec::QP, 24576, &FULLB[sb]);   // QP, ZB
+                issued_b = n + 1;
             }
-            for (int n = (issued > NS ? issued - NS : 0); n < issued; ++n)
-                wait_drain(&FULL[n % NS], (n / NS) & 1);
+            // the copies land before this CTA may exit
+            for (int n = (issued_a > NSA ? issued_a - NSA : 0); n < issued_a; ++n)
+                wait_drain(&FULLA[n % NSA], (n / NSA) & 1);
+            for (int n = (issued_b > NSB ? issued_b - NSB : 0); n < issued_b; ++n)
+                wait_drain(&FULLB[n % NSB], (n / NSB) & 1);
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------- tensor-core products
+        const uint32_t idS = idesc_bf16(128, DVT, false, true);
+        const uint32_t idO = idesc_bf16(64, DVT, false, true);
+        for (int n = 0; n < nchunks; ++n) {
+            const int sa = n % NSA, sb = n % NSB;
+            uint8_t *slot_a = sm + ChainSmem::RA + sa * ChainSmem::A_STRIDE;
+            uint8_t *slot_b = sm + ChainSmem::RB + sb * ChainSmem::B_STRIDE;
+            const uint32_t aM = smem_addr(slot_a + ChainSmem::A_MP);
+            const uint32_t aY = smem_addr(slot_a + ChainSmem::A_YT);
+            const uint32_t bV = smem_addr(slot_a + ChainSmem::A_V);
+            const uint32_t bS = smem_addr(sm + ChainSmem::SB + (n & 1) * 8192);
+            mbar_wait(SREADY, n & 1, abort_flag);
+            mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)   // S += MP SB
+                mma_bf16_warp(tmem + kColS,
+                              smem_desc(aM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(bS + ks * 1024, 16, 512, kLayoutSW64), idS, 1u);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)   // S += YT V
+                mma_bf16_warp(tmem + kColS, smem_desc(aY + ks * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(bV + ks * 1024, 16, 512, kLayoutSW64), idS, 1u);
+            mma_commit_warp(SDONE);
+            mbar_wait(&FULLB[sb], (n / NSB) & 1, abort_flag);
+            const uint32_t aQ = smem_addr(slot_b + ChainSmem::B_QP);
+            const uint32_t aZ = smem_addr(slot_b + ChainSmem::B_ZB);
+            const uint32_t dO = tmem + kColO + 32 * (n & 1);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)   // O = QP SB
+                mma_bf16_warp(dO, smem_desc(aQ + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(bS + ks * 1024, 16, 512, kLayoutSW64), idO, ks > 0 ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)   // O += ZB V
+                mma_bf16_warp(dO, smem_desc(aZ + ks * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(bV + ks * 1024, 16, 512, kLayoutSW64), idO, 1u);
+            mma_commit_warp(&ODONE[n & 1]);
+            mma_commit_warp(&EMPTYA[sa]);
+            mma_commit_warp(&EMPTYB[sb]);
+        }
+        if (nchunks > 0) {   // every arrive of the commits above lands before the CTA exits
+            mma_commit_warp(FIN);
+            wait_drain(FIN, 0);
         }
     } else {
         // ---------------------------------------------- the state chain
-        const int ct = tid - 32;
-        const bool leader = ct == 0;
         const int quad = warp & 3;
         const int crow = 32 * quad + lane;
         const size_t soff = ((size_t)seq * p.H + h) * (size_t)(DK * DV) + (size_t)crow * DV + j0;
@@ -485,88 +687,41 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             for (int i = 0; i < 32; ++i) S[i] = 0.f;
         }
         for (int n = 0; n < nchunks; ++n) {
-            const int s = n % NS, u = n & 1;
-            uint8_t *slot = sm + ChainSmem::SLOT + s * ChainSmem::SLOT_STRIDE;
+            const int sa = n % NSA;
+            const uint8_t *slot_a = sm + ChainSmem::RA + sa * ChainSmem::A_STRIDE;
             if (n >= 1) {
-                mbar_wait(&DONE[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
+                mbar_wait(SDONE, (n - 1) & 1, abort_flag);
                 tc_fence_after();
                 tmem_ld32(tmem_addr(tmem, 32 * quad, kColS), S);
                 tmem_wait_ld();
             }
-            store_bf16_row_sw64(sm + ChainSmem::SB, crow, S);
-            mbar_wait(&FULL[s], (n / NS) & 1, abort_flag);
-            const float d = reinterpret_cast<const float *>(slot + Rec::EGL)[crow];
+            store_bf16_row_sw64(sm + ChainSmem::SB + (n & 1) * 8192, crow, S);
+            mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
+            const float d = reinterpret_cast<const float *>(slot_a + ChainSmem::A_EGL)[crow];
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] *= d;
             tmem_st32(tmem_addr(tmem, 32 * quad, kColS), S);
             tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
-            named_barrier(kChainBar, 128);
-            if (leader) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(SREADY);
+            if (n >= 1) {
+                const int m = n - 1;
+                mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
                 tc_fence_after();
-                const uint32_t aTP = smem_addr(slot + Rec::TB);
-                const uint32_t bV = smem_addr(slot + ChainSmem::VT_OFF);
-                const uint32_t aWQ = smem_addr(slot + Rec::STK);
-                const uint32_t bS = smem_addr(sm + ChainSmem::SB);
-                const uint32_t id = idesc_bf16(128, DVT, false, true);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)   // U' = T diag(beta) V (rows 0-63)
-                    mma_bf16(tmem + kColUp + 32 * u, smem_desc(aTP + ks * 32, 16, 1024, kLayoutSW128),
-                             smem_desc(bV + ks * 1024, 16, 512, kLayoutSW64), id, ks > 0 ? 1u : 0u);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // [-W S; Qtil S]
-                    mma_bf16(tmem + kColUO + 32 * u,
-                             smem_desc(aWQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                             smem_desc(bS + ks * 1024, 16, 512, kLayoutSW64), id, ks > 0 ? 1u : 0u);
-                mma_commit(&UFULL[u]);
-            }
-            if (n >= 1) store_o(tmem, quad, lane, n - 1, bos, len, h, j0, p);
-
-            mbar_wait(&UFULL[u], (n >> 1) & 1, abort_flag);
-            tc_fence_after();
-            if (quad < 2) {   // U = U' - W S, rows 0-63
-                float U[32], Wp[32];
-                tmem_ld32(tmem_addr(tmem, 32 * quad, kColUO + 32 * u), U);
-                tmem_ld32(tmem_addr(tmem, 32 * quad, kColUp + 32 * u), Wp);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) U[i] += Wp[i];
-                store_bf16_row_sw64(sm + ChainSmem::UB, crow, U);
-            }
-            fence_async_smem();
-            tc_fence_before();
-            named_barrier(kChainBar, 128);
-            if (leader) {
-                tc_fence_after();
-                const uint32_t aK = smem_addr(slot + Rec::KBAR);
-                const uint32_t aTP = smem_addr(slot + Rec::TB);
-                const uint32_t bU = smem_addr(sm + ChainSmem::UB);
-                const uint32_t idS = idesc_bf16(128, DVT, true, true);
-                const uint32_t idO = idesc_bf16(128, DVT, false, true);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)   // S += Kbar^T U
-                    mma_bf16(tmem + kColS, smem_desc(aK + ks * 2048, 8192, 1024, kLayoutSW128),
-                             smem_desc(bU + ks * 1024, 16, 512, kLayoutSW64), idS, 1u);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)   // O += P U (rows 64-127 of [TB; PB] U)
-                    mma_bf16(tmem + kColUO + 32 * u, smem_desc(aTP + ks * 32, 16, 1024, kLayoutSW128),
-                             smem_desc(bU + ks * 1024, 16, 512, kLayoutSW64), idO, 1u);
-                mma_commit(&DONE[u]);
-                mma_commit(&EMPTY[s]);
+                store_o(tmem, quad, lane, m, bos, len, h, j0, p);
             }
         }
         if (nchunks > 0) {
-            const int n = nchunks - 1;
-            mbar_wait(&DONE[n & 1], (n >> 1) & 1, abort_flag);
+            const int m = nchunks - 1;
+            mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
             tc_fence_after();
-            store_o(tmem, quad, lane, n, bos, len, h, j0, p);
+            store_o(tmem, quad, lane, m, bos, len, h, j0, p);
+            mbar_wait(SDONE, m & 1, abort_flag);
+            tc_fence_after();
             tmem_ld32(tmem_addr(tmem, 32 * quad, kColS), S);
             tmem_wait_ld();
-            if (leader) {
-                mma_commit(FIN);
-                wait_drain(FIN, 0);
-            }
         }
         if (p.final_state) {
             float4 *dst = reinterpret_cast<float4 *>(p.final_state + soff);
