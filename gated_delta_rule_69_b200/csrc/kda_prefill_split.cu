@@ -167,6 +167,11 @@ __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// all but the most recently committed bulk group have read their sources
+__device__ __forceinline__ void bulk_wait_read_all_but_last() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
@@ -321,17 +326,21 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         const int64_t tok0 = bos + (int64_t)sc.y * C;
         const int L = (int)min((int64_t)C, eos - tok0);
         uint8_t *rec = p.recs + ((size_t)chunk * p.H + h) * Rec::STRIDE;
-        // Loads.  The leader reaches this point only after the previous
-        // item's record has left shared memory and every thread has passed
-        // that item's last barrier, so the buffers are free.
+        // Loads.  The leader reaches this point after every thread has
+        // passed the previous item's last barrier and after the record
+        // stores have read the buffers these loads overwrite (STK, GRAW);
+        // the rest of the record may still be leaving shared memory, so the
+        // leader's arrive, which lets the group write again, waits for that.
         if (leader) {
-            mbar_arrive_expect_tx(&B[0], kRawBytes);
+            mbar_expect_tx(&B[0], kRawBytes);
             const int t = (int)tok0;
             tma_load_3d(sm + PrepSmem::STK, &tm_k, &B[0], 0, h, t);
             tma_load_3d(sm + PrepSmem::STK + 16384, &tm_k, &B[0], 64, h, t);
             tma_load_3d(sm + PrepSmem::STK + 8192, &tm_q, &B[0], 0, h, t);
             tma_load_3d(sm + PrepSmem::STK + 16384 + 8192, &tm_q, &B[0], 64, h, t);
             tma_load_3d(sm + PrepSmem::GRAW, &tm_g, &B[0], 0, h, t);
+            bulk_wait_read_all();
+            mbar_arrive(&B[0]);
         }
         if (pt < C) {
             beta[pt] = (pt < L) ? __bfloat162float(p.beta[(size_t)(tok0 + pt) * p.H + h]) : 0.f;
@@ -359,17 +368,19 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         fence_async_smem();
         named_barrier(BAR, prep::kGroupThreads);
         uint32_t drawn = 0;
-        if (leader) {
-            drawn = atomicAdd(p.work_next, 1u);   // consumed at the end of the item
+        if (wp == 0) {   // tensor-core products: issued by the group's first warp
             tc_fence_after();
             const uint32_t a0 = smem_addr(sm + PrepSmem::STK), b0 = smem_addr(sm + PrepSmem::KHAT);
             const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)   // [Ktil; Qtil] Khat^T
-                mma_bf16(tmem, smem_desc(a0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                         smem_desc(b0 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                         id, ks > 0 ? 1u : 0u);
-            mma_commit(&B[1]);
+                mma_bf16_warp(tmem, smem_desc(a0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(b0 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              id, ks > 0 ? 1u : 0u);
+            mma_commit_warp(&B[1]);
+        }
+        if (leader) {
+            drawn = atomicAdd(p.work_next, 1u);   // consumed at the end of the item
             if (pending) {
                 bulk_wait_all();
                 publish_flag(pending);
@@ -392,14 +403,14 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         named_barrier(BAR, prep::kGroupThreads);
         const uint32_t sK = smem_addr(sm + PrepSmem::STK), sKb = smem_addr(sm + PrepSmem::KBAR);
         const uint32_t sT = smem_addr(sm + PrepSmem::TB), sP = smem_addr(sm + PrepSmem::PB);
-        if (leader) {
+        if (wp == 0) {
             tc_fence_after();
             const uint32_t idW = idesc_bf16(64, DK, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)   // W = T diag(beta) Ktil
-                mma_bf16(tmem + 64, smem_desc(sT + ks * 32, 16, 1024, kLayoutSW128),
-                         smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idW, ks > 0 ? 1u : 0u);
-            mma_commit(&B[2]);
+                mma_bf16_warp(tmem + 64, smem_desc(sT + ks * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idW, ks > 0 ? 1u : 0u);
+            mma_commit_warp(&B[2]);
         }
         mbar_wait(&B[2], it & 1, abort_flag);
         tc_fence_after();
@@ -407,7 +418,7 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         fence_async_smem();
         tc_fence_before();
         named_barrier(BAR, prep::kGroupThreads);
-        if (leader) {
+        if (wp == 0) {
             tc_fence_after();
             const uint32_t idM = idesc_bf16(128, DK, true, true);
             const uint32_t idY = idesc_bf16(128, C, true, true);
@@ -416,30 +427,30 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
             for (int ks = 0; ks < 4; ++ks) {   // K = 64 tokens
                 const uint64_t aKb = smem_desc(sKb + ks * 2048, 8192, 1024, kLayoutSW128);   // Kbar^T
                 // MP = Kbar^T (-W)
-                mma_bf16(tmem, aKb, smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idM,
-                         ks > 0 ? 1u : 0u);
+                mma_bf16_warp(tmem, aKb, smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idM,
+                              ks > 0 ? 1u : 0u);
                 // YT = Kbar^T T_beta
-                mma_bf16(tmem + 128, aKb, smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idY,
-                         ks > 0 ? 1u : 0u);
+                mma_bf16_warp(tmem + 128, aKb, smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idY,
+                              ks > 0 ? 1u : 0u);
                 // ZB = P T_beta
-                mma_bf16(tmem + 192, smem_desc(sP + ks * 32, 16, 1024, kLayoutSW128),
-                         smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idZ, ks > 0 ? 1u : 0u);
+                mma_bf16_warp(tmem + 192, smem_desc(sP + ks * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idZ, ks > 0 ? 1u : 0u);
             }
-            mma_commit(&B[3]);
+            mma_commit_warp(&B[3]);
         }
         mbar_wait(&B[3], it & 1, abort_flag);
         tc_fence_after();
         write_mp(sm + PrepSmem::KHAT, tmem, quad, half, lane);
         tc_fence_before();
         named_barrier(BAR, prep::kGroupThreads);
-        if (leader) {
+        if (wp == 0) {
             tc_fence_after();
             const uint32_t idQ = idesc_bf16(64, DK, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)   // P (-W), into the columns MP has left
-                mma_bf16(tmem, smem_desc(sP + ks * 32, 16, 1024, kLayoutSW128),
-                         smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idQ, ks > 0 ? 1u : 0u);
-            mma_commit(&B[4]);
+                mma_bf16_warp(tmem, smem_desc(sP + ks * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idQ, ks > 0 ? 1u : 0u);
+            mma_commit_warp(&B[4]);
         }
         // Kbar, T_beta are no longer read: YT and ZB go over them
         write_yt(sm + PrepSmem::KBAR, tmem + 128, quad, half, lane);
@@ -453,14 +464,17 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         named_barrier(BAR, prep::kGroupThreads);
         const uint32_t next_item = next_slot[(it + 1) & 1];
         if (leader) {
-            bulk_store(rec + Rec::MP, sm + PrepSmem::KHAT, 32768);
-            bulk_store(rec + Rec::YT, sm + PrepSmem::KBAR, 16384);
+            // first group: the sources the next item's loads overwrite
             bulk_store(rec + Rec::QP, sm + PrepSmem::STK + 8192, 8192);
             bulk_store(rec + Rec::QP + 8192, sm + PrepSmem::STK + 16384 + 8192, 8192);
+            bulk_store(rec + Rec::MP + 16384, sm + PrepSmem::GRAW, 16384);
+            bulk_commit();
+            bulk_store(rec + Rec::MP, sm + PrepSmem::KHAT, 16384);
+            bulk_store(rec + Rec::YT, sm + PrepSmem::KBAR, 16384);
             bulk_store(rec + Rec::ZB, sm + PrepSmem::TB, 8192);
             bulk_store(rec + Rec::EGL, sm + PrepSmem::EGL, 512);
             bulk_commit();
-            bulk_wait_read_all();
+            bulk_wait_read_all_but_last();
             if (p.rec_ready) pending = p.rec_ready + (size_t)chunk * p.H + h;
         }
         item = next_item;
@@ -489,7 +503,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint32_t *misc0 = reinterpret_cast<uint32_t *>(sm0 + PrepSmem::MISC);
     if (tid == 0 || tid == kPipeThreads) {
         uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);
-        mbar_init(&B[0], 3);   // the leader's expect_tx, and one arrive per beta warp
+        mbar_init(&B[0], 3);   // the leader, and one arrive per beta warp
         for (int i = 1; i < 5; ++i) mbar_init(&B[i], 1);
         reinterpret_cast<uint32_t *>(sm + PrepSmem::MISC)[1] = 0u;
         fence_mbar_init();
