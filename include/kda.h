@@ -75,9 +75,9 @@ int kda_version(void);
 
 /*
  * Workspace bytes for kda_prefill's fastest path on this problem (a multiple
- * of 256).  For d_k = d_v = 128 this includes one 65 KB record per (chunk of
+ * of 256).  For d_k = d_v = 128 this includes one 73 KB record per (chunk of
  * 64 tokens, head) for the two-kernel tensor-core path, i.e. about
- * 1 KiB per (token, head): 4.4 GB for 131072 tokens x 32 heads.  Pure host
+ * 1.2 KB per (token, head): 4.9 GB for 131072 tokens x 32 heads.  Pure host
  * arithmetic, no CUDA call.  Returns 0 for arguments kda_prefill would reject.
  */
 size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens,
