@@ -30,11 +30,13 @@ constexpr float kLog2e = 1.4426950408889634f;
 // e^x through the hardware base-2 exponential (ex2.approx, flush-to-zero):
 // its relative error (~2^-22) is far below the bf16 rounding of the operands
 // it scales.
-__device__ __forceinline__ float exp_f(float x) {
+__device__ __forceinline__ float exp2_f(float x) {
     float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * kLog2e));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+
+__device__ __forceinline__ float exp_f(float x) { return exp2_f(x * kLog2e); }
 
 // Shared-memory buffers of one chunk's preparation.
 struct Bufs {
@@ -43,8 +45,8 @@ struct Bufs {
     uint8_t *khat;       // Khat [64][128], 2 K-atoms of 8 KB
     uint8_t *kbar;       // Kbar [64][128], 2 K-atoms of 8 KB
     const uint8_t *graw; // raw log_alpha [64][128] bf16, 256-byte rows
-    float *af;           // A, fp32 64x64 (row-XOR layout); may alias khat after the product
-    float *tf;           // T, fp32 64x64 (float4-XOR layout)
+    float *af;           // A, fp32 64x64, rows of 65 (16,640 bytes); may alias khat after the product
+    float *tf;           // T, fp32 64x64, rows of 68 (17,408 bytes)
     float *xf;           // solve scratch, >= 4608 bytes; may alias graw after gating
     uint8_t *tb;         // T diag(beta) bf16 [64 t][64 i] (one K-atom)
     uint8_t *pb;         // P bf16 [64 t][64 i]
@@ -54,19 +56,24 @@ struct Bufs {
     uint32_t *slow_flag; // one word
 };
 
-// Index of A element (t, i): rows of 64 floats, column XORed with the row's
-// low 5 bits so that row-parallel accesses hit distinct banks.
-__device__ __forceinline__ int fidx(int t, int i) { return t * 64 + (i ^ (t & 31)); }
+// Index of A element (t, i): rows padded to 65 floats, so that a warp
+// reading one column across 32 rows hits 32 distinct banks, and a thread
+// walking a row or a column steps by a constant.
+constexpr int kAStride = 65;
+__device__ __forceinline__ int fidx(int t, int i) { return t * kAStride + i; }
 
-// T layout: rows of 64 floats, float4 group index XORed with (row mod 16).
-__device__ __forceinline__ int tfi(int row, int col) {
-    return row * 64 + ((((col >> 2) ^ (row & 15))) << 2) + (col & 3);
-}
+// T layout: rows padded to 68 floats (float4-aligned); the four rows a warp
+// reads at once in the second product of a merge fall in distinct banks.
+constexpr int kTStride = 68;
+__device__ __forceinline__ int tfi(int row, int col) { return row * kTStride + col; }
 
 // ---- running sums and gated operands.  Thread pt (0..255) owns channels
 // c, c+1 (c = 2 (pt mod 64)) for the 16 tokens of group pt / 64; a warp covers
-// one 64-channel K-atom of one token group.  Returns whether the chunk needs
-// the pairwise path.
+// one 64-channel K-atom of one token group.  Rows past the chunk's end (a
+// sequence's last chunk) are zeroed first, so that they add nothing to the
+// running sums and give zero operand rows.  The running sums are kept in
+// base-2 units (log_alpha log2(e)).  Returns whether the chunk needs the
+// pairwise path.
 template <int BAR>
 __device__ bool gate(const Bufs &b, int pt, int L) {
     const int c = 2 * (pt & 63);
@@ -76,6 +83,19 @@ __device__ bool gate(const Bufs &b, int pt, int L) {
     uint8_t *stack = b.stk + katom * 16384;
     uint8_t *khat = b.khat + katom * 8192;
     uint8_t *kbar = b.kbar + katom * 8192;
+
+    if (L < C) {   // uniform over the group
+        uint8_t *graw = const_cast<uint8_t *>(b.graw);
+        for (int v = pt; v < (C - L) * 16; v += kGroupThreads) {   // 16-byte pieces of a 256-byte row
+            const int t = L + (v >> 4), piece = v & 15;
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(graw + t * 256 + piece * 16) = z;
+            uint8_t *atom = b.stk + (piece >> 3) * 16384;
+            *reinterpret_cast<uint4 *>(atom + sw128_off(t, (piece & 7) * 8)) = z;
+            *reinterpret_cast<uint4 *>(atom + sw128_off(64 + t, (piece & 7) * 8)) = z;
+        }
+        named_barrier(BAR, kGroupThreads);
+    }
 
     uint32_t graw_v[16], k_v[16], q_v[16];
 #pragma unroll
@@ -89,10 +109,9 @@ __device__ bool gate(const Bufs &b, int pt, int L) {
     float r0 = 0.f, r1 = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        const bool valid = t0 + i < L;
         const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162 *>(&graw_v[i]);
-        r0 += valid ? clamp_log_alpha(__low2float(gv)) : 0.f;
-        r1 += valid ? clamp_log_alpha(__high2float(gv)) : 0.f;
+        r0 = fmaf(clamp_log_alpha(__low2float(gv)), kLog2e, r0);
+        r1 = fmaf(clamp_log_alpha(__high2float(gv)), kLog2e, r1);
         g0[i] = r0;
         g1[i] = r1;
     }
@@ -109,34 +128,31 @@ __device__ bool gate(const Bufs &b, int pt, int L) {
         GL0 += a;
         GL1 += bb;
     }
-    if (tg == 0 && (GL0 < kSlowPathLogDecay || GL1 < kSlowPathLogDecay)) *b.slow_flag = 1u;
+    constexpr float kSlow2 = kSlowPathLogDecay * kLog2e;
+    if (tg == 0 && (GL0 < kSlow2 || GL1 < kSlow2)) *b.slow_flag = 1u;
     named_barrier(BAR, kGroupThreads);
     const bool slow = *b.slow_flag != 0u;
 
-    const float eL0 = exp_f(GL0), eL1 = exp_f(GL1);
+    const float eL0 = exp2_f(GL0), eL1 = exp2_f(GL1);
     if (tg == 0) {
         b.egl[c] = eL0;
         b.egl[c + 1] = eL1;
     }
+    constexpr float kMaxInv2 = 80.f * kLog2e;   // Khat's factor is capped at e^80
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int t = t0 + i;
-        const bool valid = t < L;
         const __nv_bfloat162 kv = *reinterpret_cast<const __nv_bfloat162 *>(&k_v[i]);
         const __nv_bfloat162 qv = *reinterpret_cast<const __nv_bfloat162 *>(&q_v[i]);
-        const float k0 = valid ? __low2float(kv) : 0.f, k1 = valid ? __high2float(kv) : 0.f;
-        const float q0 = valid ? __low2float(qv) : 0.f, q1 = valid ? __high2float(qv) : 0.f;
+        const float k0 = __low2float(kv), k1 = __high2float(kv);
+        const float q0 = __low2float(qv), q1 = __high2float(qv);
         const float G0 = g0[i] + off0, G1 = g1[i] + off1;
-        const float e0 = exp_f(G0), e1 = exp_f(G1);
-        const float ih0 = exp_f(fminf(-G0, 80.f)), ih1 = exp_f(fminf(-G1, 80.f));
-        float b0, b1;
-        if (slow) {
-            b0 = exp_f(GL0 - G0);
-            b1 = exp_f(GL1 - G1);
-        } else {
-            b0 = eL0 * ih0;
-            b1 = eL1 * ih1;
-        }
+        const float e0 = exp2_f(G0), e1 = exp2_f(G1);
+        const float ih0 = exp2_f(fminf(-G0, kMaxInv2)), ih1 = exp2_f(fminf(-G1, kMaxInv2));
+        // Kbar's factor e^{G_L - G}: a product of two factors, or (pairwise
+        // path, where e^{-G} may be capped) one exponential
+        const float b0 = slow ? exp2_f(GL0 - G0) : eL0 * ih0;
+        const float b1 = slow ? exp2_f(GL1 - G1) : eL1 * ih1;
         const uint32_t ok = sw128_off(t, cc);
         *reinterpret_cast<uint32_t *>(stack + ok) = pack_bf16x2(k0 * e0, k1 * e1);
         *reinterpret_cast<uint32_t *>(stack + sw128_off(64 + t, cc)) = pack_bf16x2(q0 * e0, q1 * e1);

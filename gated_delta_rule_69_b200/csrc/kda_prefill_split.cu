@@ -72,18 +72,23 @@ struct PrepSmem {
     static constexpr uint32_t TB = 49152;      // T diag(beta) [64 t][64 i], then ZB
     static constexpr uint32_t PB = 57344;      // P [64 t][64 i]
     static constexpr uint32_t EGL = 65536;     // 128 fp32
-    static constexpr uint32_t KHAT = 66560;    // Khat, then A fp32, then MP K-atom 0
-    static constexpr uint32_t GRAW = 82944;    // raw log_alpha, then T fp32, then MP K-atom 1
-    static constexpr uint32_t XF = 99328;      // solve scratch (4608 bytes)
-    static constexpr uint32_t BETA = 103936;   // 64 fp32
-    static constexpr uint32_t CSUM = 104192;   // 4 x 128 fp32
-    static constexpr uint32_t BARS = 106240;   // 5 mbarriers
-    static constexpr uint32_t MISC = 106304;   // tmem base, abort, slow flag, next-item slots at 4, 5
-    static constexpr uint32_t SIZE = 106368;
-    static constexpr uint32_t PIPE = 107520;   // per-pipeline stride
+    static constexpr uint32_t KHAT = 66560;    // Khat, then A fp32 (16,640 bytes), then MP K-atom 0
+    static constexpr uint32_t GRAW = 83968;    // raw log_alpha, then T fp32 (17,408 bytes), then MP K-atom 1
+    static constexpr uint32_t XF = 101376;     // solve scratch (4608 bytes)
+    static constexpr uint32_t BETA = 105984;   // 64 fp32
+    static constexpr uint32_t CSUM = 106240;   // 4 x 128 fp32
+    static constexpr uint32_t BARS = 108288;   // 5 mbarriers
+    static constexpr uint32_t MISC = 108352;   // tmem base, abort, slow flag, next-item slots at 4, 5
+    static constexpr uint32_t SIZE = 108416;
+    static constexpr uint32_t PIPE = 109568;   // per-pipeline stride
     static constexpr uint32_t ALLOC = 2 * PIPE + 1024;
 };
-static_assert(PrepSmem::ALLOC <= 232448, "two preparation pipelines per CTA");
+static_assert(PrepSmem::ALLOC <= 232448 && PrepSmem::SIZE <= PrepSmem::PIPE,
+              "two preparation pipelines per CTA");
+static_assert(PrepSmem::KHAT + 64 * prep::kAStride * 4 <= PrepSmem::GRAW &&
+                  PrepSmem::GRAW + 64 * prep::kTStride * 4 <= PrepSmem::XF &&
+                  PrepSmem::XF + 4608 <= PrepSmem::BETA,
+              "solve scratch");
 // per pipeline (256 columns): [A;P] at 0 and W at 64; then MP at 0, YT at 128,
 // ZB at 192 (M = 64); then -P W at 0 (M = 64)
 constexpr uint32_t kPrepTmemCols = 512;
@@ -225,9 +230,11 @@ __device__ __forceinline__ void store8(uint8_t *tile, uint32_t row, uint32_t col
     *reinterpret_cast<uint4 *>(tile + sw128_off(row, col)) = pk;
 }
 
-// MP [128 c_out][128 c_in]: K-atom `half` holds c_in 64 half .. + 63.
-__device__ __forceinline__ void write_mp(uint8_t *mp, uint32_t tmem, int quad, int half, int lane) {
-    uint8_t *atom = mp + half * 16384;
+// MP [128 c_out][128 c_in]: K-atom `half` (at atom0 or atom1) holds c_in
+// 64 half .. + 63.
+__device__ __forceinline__ void write_mp(uint8_t *atom0, uint8_t *atom1, uint32_t tmem, int quad,
+                                         int half, int lane) {
+    uint8_t *atom = half ? atom1 : atom0;
     const int row = 32 * quad + lane;
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
@@ -440,7 +447,7 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         }
         mbar_wait(&B[3], it & 1, abort_flag);
         tc_fence_after();
-        write_mp(sm + PrepSmem::KHAT, tmem, quad, half, lane);
+        write_mp(sm + PrepSmem::KHAT, sm + PrepSmem::GRAW, tmem, quad, half, lane);
         tc_fence_before();
         named_barrier(BAR, prep::kGroupThreads);
         if (wp == 0) {
