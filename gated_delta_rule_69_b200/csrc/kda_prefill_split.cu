@@ -1,19 +1,18 @@
 // KDA prefill as two kernels (bf16 I/O, d_k = d_v = 128, C = 64):
 //
-//   kda_prep_kernel  - one CTA per (chunk, head), all chunks at once: the
+//   kda_prep_kernel  - persistent, chunk-parallel: for every (chunk, head) the
 //                      chunk preparation of kda_chunk_prep.cuh (running sums,
 //                      gated operands, [A; P] on the tensor cores, T = (I+A)^-1,
-//                      W), written to the workspace as a 65 KB record per
-//                      (chunk, head) in the exact shared-memory layout the
-//                      tensor cores read: [-W; Qtil], Kbar, T diag(beta), P,
-//                      exp(G_L).
-//   kda_chain_kernel - one CTA per (sequence, head, 32-column slice of d_v):
-//                      the serial state chain.  Per chunk it bulk-copies the
-//                      record into a 3-stage ring (plus its v slice by TMA),
-//                      and with the fp32 state S in TMEM computes
-//                          U' = T diag(beta) V,  [-W S; Qtil S] = [-W; Qtil] S
-//                          U = U' - W S,  O = Qtil S + P U
-//                          S <- Diag(e^{G_L}) S + Kbar^T U
+//                      W), then the chunk's transition operands
+//                          MP = -Kbar^T W,  YT = Kbar^T T_beta,
+//                          QP = Qtil - P W, ZB = P T_beta,  exp(G_L)
+//                      on the tensor cores, written to the workspace as a
+//                      73 KB record in the layout the chain's products read.
+//   kda_chain_kernel - the serial state chain, one CTA per (sequence, head,
+//                      slice of d_v; 32 columns or the whole 128): per chunk it
+//                      bulk-copies the record (plus its v slice by TMA) into
+//                      rings and, with the fp32 state S in TMEM, computes
+//                          S <- Diag(exp(G_L)) S + MP S + YT V,  O = QP S + ZB V
 //                      on the tensor cores.
 //
 // The state-independent preparation (the long-latency part of a chunk: the
@@ -21,8 +20,8 @@
 // over the whole GPU, once per (chunk, head), and leaves the serial chain
 // (news digest page on Kimi Linear, section "Algorithme parallele par chunks":
 // the previous chunk's final state is the next chunk's initial state) with
-// only tensor-core products and their read-outs.  The price is the record's
-// round trip through global memory (written once, read once per d_v slice).
+// one product group per chunk on its serial path.  The price is the record's
+// round trip through L2 / global memory.
 #include <cuda.h>
 
 #include "kda_chunk_prep.cuh"
@@ -37,8 +36,6 @@ using namespace sm100;
 constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int DV = 128;
-constexpr int DVT = 32;
-constexpr int NTILE = DV / DVT;
 
 // ---- the per-(chunk, head) record: bf16 tensor-core operands in the
 // K-major 128-byte-swizzled layout the chain kernel's products read.
@@ -94,30 +91,42 @@ static_assert(PrepSmem::KHAT + 64 * prep::kAStride * 4 <= PrepSmem::GRAW &&
 constexpr uint32_t kPrepTmemCols = 512;
 constexpr uint32_t kRawBytes = 4 * 8192 + 16384;   // k, q (2 boxes each), log_alpha
 
-// ---- chain kernel
-constexpr int kChainThreads = 192;             // warp 0: loads; warps 1-4: the chain; warp 5: products
-constexpr int NSA = 3;                         // ring A: state-update operands + v slice
-constexpr int NSB = 2;                         // ring B: output operands
-struct ChainSmem {
-    static constexpr uint32_t A_MP = 0, A_YT = 32768, A_V = 49152, A_EGL = 53248;
-    static constexpr uint32_t A_STRIDE = 54272;
+// ---- chain kernel, one CTA per (sequence, head, DVT-column slice of d_v).
+// Warp 0 loads; warps 1 .. NCW hold the state (warp w: TMEM lanes of quadrant
+// w mod 4, columns 32 ((w - 1) / 4) .. + 31 of the slice); warp NCW + 1 issues
+// the products.  Ring A carries MP, YT, the v slice and exp(G_L); ring B QP,
+// ZB; the bf16 copy of the state is double-buffered.
+constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
+
+template <int DVT_>
+struct ChainCfg {
+    static constexpr int DVT = DVT_;
+    static constexpr int NTILE = DV / DVT;
+    static constexpr int NCW = 4 * (DVT / 32);
+    static constexpr int THREADS = 32 * (NCW + 2);
+    static constexpr int NSA = DVT == 32 ? 3 : 2;
+    static constexpr int NSB = DVT == 128 ? 1 : 2;
+    static constexpr uint32_t V_BYTES = (uint32_t)DVT * C * 2;
+    static constexpr uint32_t A_MP = 0, A_YT = 32768, A_V = 49152, A_EGL = A_V + V_BYTES;
+    static constexpr uint32_t A_STRIDE = align1k(A_EGL + 512);
     static constexpr uint32_t B_QP = 0, B_ZB = 16384;
     static constexpr uint32_t B_STRIDE = 24576;
+    static constexpr uint32_t SB_BYTES = (uint32_t)DK * DVT * 2;   // S bf16 [128 c][DVT j]
     static constexpr uint32_t RA = 0;
-    static constexpr uint32_t RB = NSA * A_STRIDE;          // 162816
-    static constexpr uint32_t SB = RB + NSB * B_STRIDE;     // 2 x S bf16 [128 c][32 j], 64-byte swizzle
-    static constexpr uint32_t BARS = SB + 2 * 8192;
+    static constexpr uint32_t RB = NSA * A_STRIDE;
+    static constexpr uint32_t SB = RB + NSB * B_STRIDE;
+    static constexpr uint32_t BARS = SB + 2 * SB_BYTES;
     static constexpr uint32_t MISC = BARS + 128;
     static constexpr uint32_t SIZE = MISC + 64;
     static constexpr uint32_t ALLOC = SIZE + 1024;
+    static constexpr uint32_t TMEM_COLS = DVT == 32 ? 128 : (DVT == 64 ? 256 : 512);
+    static constexpr uint32_t COL_S = 0, COL_O = DVT;   // S; O x2 at DVT + DVT b (M = 64)
+    static_assert(ALLOC <= 232448, "chain shared memory");
+    static_assert(3 * DVT <= (int)TMEM_COLS, "chain TMEM");
+    static_assert(2 * NSA + 2 * NSB + 5 <= 16, "barrier area");
 };
-static_assert(ChainSmem::ALLOC <= 232448, "chain shared memory");
-static_assert(Rec::YT == Rec::MP + 32768 && ChainSmem::A_YT == ChainSmem::A_MP + 32768,
-              "MP and YT travel as one copy");
-static_assert(Rec::ZB == Rec::QP + 16384 && ChainSmem::B_ZB == ChainSmem::B_QP + 16384,
-              "QP and ZB travel as one copy");
-constexpr uint32_t kChainTmemCols = 128;
-constexpr uint32_t kColS = 0, kColO = 32;      // S (32 columns), O x2 (M = 64, 32 columns each)
+static_assert(Rec::YT == Rec::MP + 32768 && Rec::ZB == Rec::QP + 16384,
+              "MP and YT, QP and ZB travel as one copy each");
 
 struct Params {
     const __nv_bfloat16 *k, *q, *beta;
@@ -535,7 +544,12 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 // =============================================================== chain kernel
 
-__device__ __forceinline__ void store_bf16_row_sw64(uint8_t *tile, int row, const float (&v)[32]) {
+// One thread's 32 state columns (slice columns col0 .. col0 + 31 of row
+// `row`) as bf16 into the B-operand copy of S: for a 32-column slice one
+// 64-byte-swizzled tile [128 c][32 j]; for wider slices 128-byte-swizzled
+// atoms [128 c][64 j], 16 KB apart.
+template <int DVT>
+__device__ __forceinline__ void store_sb_row(uint8_t *sb, int row, int col0, const float (&v)[32]) {
 #pragma unroll
     for (int j = 0; j < 32; j += 8) {
         uint4 pk;
@@ -543,20 +557,43 @@ __device__ __forceinline__ void store_bf16_row_sw64(uint8_t *tile, int row, cons
         pk.y = pack_bf16x2(v[j + 2], v[j + 3]);
         pk.z = pack_bf16x2(v[j + 4], v[j + 5]);
         pk.w = pack_bf16x2(v[j + 6], v[j + 7]);
-        *reinterpret_cast<uint4 *>(tile + sw64_off(row, j)) = pk;
+        if (DVT == 32) {
+            *reinterpret_cast<uint4 *>(sb + sw64_off(row, j)) = pk;
+        } else {
+            const int col = col0 + j;
+            *reinterpret_cast<uint4 *>(sb + (col >> 6) * 16384 + sw128_off(row, col & 63)) = pk;
+        }
     }
 }
 
-// O of chunk m from TMEM (M = 64 layout: row t in lane (t mod 16) + 32 (t / 16))
-// to global memory; the whole warp reads, lanes 0-15 hold rows.
-__device__ __forceinline__ void store_o(uint32_t tmem, int quad, int lane, int m, int64_t bos,
-                                        int64_t len, int h, int j0, const Params &p) {
+// B-operand descriptor of k-step ks for the state copy (K = 128 rows of c)
+// and the v slice (K = 64 rows of t).
+template <int DVT>
+__device__ __forceinline__ uint64_t desc_sb(uint32_t base, int ks) {
+    return DVT == 32 ? smem_desc(base + ks * 1024, 16, 512, kLayoutSW64)
+                     : smem_desc(base + ks * 2048, 16384, 1024, kLayoutSW128);
+}
+
+template <int DVT>
+__device__ __forceinline__ uint64_t desc_v(uint32_t base, int ks) {
+    return DVT == 32 ? smem_desc(base + ks * 1024, 16, 512, kLayoutSW64)
+                     : smem_desc(base + ks * 2048, 8192, 1024, kLayoutSW128);
+}
+
+// O of chunk m, 32 columns (slice columns col0 ..) from TMEM (M = 64 layout:
+// row t in lane (t mod 16) + 32 (t / 16)) to global memory; the whole warp
+// reads, lanes 0-15 hold rows.
+template <int DVT>
+__device__ __forceinline__ void store_o(uint32_t tmem, int quad, int lane, int col0, int m,
+                                        int64_t bos, int64_t len, int h, int j0, const Params &p) {
+    using Cfg = ChainCfg<DVT>;
     float v[32];
-    tmem_ld32(tmem_addr(tmem, 32 * quad, kColO + 32 * (m & 1)), v);
+    tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_O + DVT * (m & 1) + col0), v);
     tmem_wait_ld();
     const int t = 16 * quad + lane;
     if (lane < 16 && (int64_t)m * C + t < len) {
-        uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)(bos + (int64_t)m * C + t) * p.H + h) * DV + j0);
+        uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)(bos + (int64_t)m * C + t) * p.H + h) * DV +
+                                               j0 + col0);
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
             uint4 pk;
@@ -575,8 +612,11 @@ __device__ __forceinline__ void store_o(uint32_t tmem, int quad, int lane, int m
 //                 O products (off it):           O[n mod 2] = QP SB + ZB V
 // The chain warps read the O of chunk n out while chunk n + 1 runs; the
 // product warp issues chunk n's O products while they convert S_{n+1}.
-__global__ void __launch_bounds__(kChainThreads, 1)
+template <int DVT>
+__global__ void __launch_bounds__(ChainCfg<DVT>::THREADS, 1)
 kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    using Cfg = ChainCfg<DVT>;
+    constexpr int NSA = Cfg::NSA, NSB = Cfg::NSB, NCW = Cfg::NCW, NTILE = Cfg::NTILE;
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *sm = dyn_smem + ((1024u - (smem_addr(dyn_smem) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -592,21 +632,20 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     const size_t rec0 = (size_t)p.chunk_off[seq];
 
     // mbarriers: FULLA[NSA], EMPTYA[NSA], FULLB[NSB], EMPTYB[NSB], SDONE, ODONE[2], FIN, SREADY
-    uint64_t *B = reinterpret_cast<uint64_t *>(sm + ChainSmem::BARS);
+    uint64_t *B = reinterpret_cast<uint64_t *>(sm + Cfg::BARS);
     uint64_t *FULLA = B, *EMPTYA = B + NSA, *FULLB = B + 2 * NSA, *EMPTYB = B + 2 * NSA + NSB;
     uint64_t *SDONE = B + 2 * NSA + 2 * NSB, *ODONE = SDONE + 1, *FIN = SDONE + 3, *SREADY = SDONE + 4;
     constexpr int kBars = 2 * NSA + 2 * NSB + 5;
-    static_assert(kBars * 8 <= 128, "barrier area");
-    uint32_t *misc = reinterpret_cast<uint32_t *>(sm + ChainSmem::MISC);
+    uint32_t *misc = reinterpret_cast<uint32_t *>(sm + Cfg::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     if (tid == 0) {
         for (int i = 0; i < kBars - 1; ++i) mbar_init(&B[i], 1);
-        mbar_init(SREADY, 4);   // one arrive per chain warp
+        mbar_init(SREADY, NCW);   // one arrive per chain warp
         misc[1] = 0u;
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(&misc[0], kChainTmemCols);
+        tmem_alloc(&misc[0], Cfg::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -626,17 +665,19 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 const size_t ri = (rec0 + n) * p.H + h;
                 const uint8_t *rec = p.recs + ri * Rec::STRIDE;
                 if (p.rec_ready && !acquire_flag(p.rec_ready + ri, abort_flag)) break;   // the record is complete
-                uint8_t *slot_a = sm + ChainSmem::RA + sa * ChainSmem::A_STRIDE;
-                mbar_arrive_expect_tx(&FULLA[sa], 49152 + 512 + 4096);
-                bulk_load(slot_a + ChainSmem::A_MP, rec + Rec::MP, 49152, &FULLA[sa]);   // MP, YT
-                bulk_load(slot_a + ChainSmem::A_EGL, rec + Rec::EGL, 512, &FULLA[sa]);
-                tma_load_3d(slot_a + ChainSmem::A_V, &tm_v, &FULLA[sa], j0, h, (int)(bos + (int64_t)n * C));
+                uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
+                const int t = (int)(bos + (int64_t)n * C);
+                mbar_arrive_expect_tx(&FULLA[sa], 49152 + 512 + Cfg::V_BYTES);
+                bulk_load(slot_a + Cfg::A_MP, rec + Rec::MP, 49152, &FULLA[sa]);   // MP, YT
+                bulk_load(slot_a + Cfg::A_EGL, rec + Rec::EGL, 512, &FULLA[sa]);
+                tma_load_3d(slot_a + Cfg::A_V, &tm_v, &FULLA[sa], j0, h, t);
+                if (DVT == 128) tma_load_3d(slot_a + Cfg::A_V + 8192, &tm_v, &FULLA[sa], j0 + 64, h, t);
                 issued_a = n + 1;
                 if (n >= NSB) mbar_wait(&EMPTYB[sb], ((n / NSB) - 1) & 1, abort_flag);
                 if (*abort_flag) break;
-                uint8_t *slot_b = sm + ChainSmem::RB + sb * ChainSmem::B_STRIDE;
+                uint8_t *slot_b = sm + Cfg::RB + sb * Cfg::B_STRIDE;
                 mbar_arrive_expect_tx(&FULLB[sb], 24576);
-                bulk_load(slot_b + ChainSmem::B_QP, rec + Rec::QP, 24576, &FULLB[sb]);   // QP, ZB
+                bulk_load(slot_b + Cfg::B_QP, rec + Rec::QP, 24576, &FULLB[sb]);   // QP, ZB
                 issued_b = n + 1;
             }
             // the copies land before this CTA may exit
@@ -645,43 +686,43 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             for (int n = (issued_b > NSB ? issued_b - NSB : 0); n < issued_b; ++n)
                 wait_drain(&FULLB[n % NSB], (n / NSB) & 1);
         }
-    } else if (warp == 5) {
+    } else if (warp == NCW + 1) {
         // ---------------------------------------------- tensor-core products
         const uint32_t idS = idesc_bf16(128, DVT, false, true);
         const uint32_t idO = idesc_bf16(64, DVT, false, true);
         for (int n = 0; n < nchunks; ++n) {
             const int sa = n % NSA, sb = n % NSB;
-            uint8_t *slot_a = sm + ChainSmem::RA + sa * ChainSmem::A_STRIDE;
-            uint8_t *slot_b = sm + ChainSmem::RB + sb * ChainSmem::B_STRIDE;
-            const uint32_t aM = smem_addr(slot_a + ChainSmem::A_MP);
-            const uint32_t aY = smem_addr(slot_a + ChainSmem::A_YT);
-            const uint32_t bV = smem_addr(slot_a + ChainSmem::A_V);
-            const uint32_t bS = smem_addr(sm + ChainSmem::SB + (n & 1) * 8192);
+            uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
+            uint8_t *slot_b = sm + Cfg::RB + sb * Cfg::B_STRIDE;
+            const uint32_t aM = smem_addr(slot_a + Cfg::A_MP);
+            const uint32_t aY = smem_addr(slot_a + Cfg::A_YT);
+            const uint32_t bV = smem_addr(slot_a + Cfg::A_V);
+            const uint32_t bS = smem_addr(sm + Cfg::SB + (n & 1) * Cfg::SB_BYTES);
             mbar_wait(SREADY, n & 1, abort_flag);
             mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)   // S += MP SB
-                mma_bf16_warp(tmem + kColS,
+                mma_bf16_warp(tmem + Cfg::COL_S,
                               smem_desc(aM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                              smem_desc(bS + ks * 1024, 16, 512, kLayoutSW64), idS, 1u);
+                              desc_sb<DVT>(bS, ks), idS, 1u);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)   // S += YT V
-                mma_bf16_warp(tmem + kColS, smem_desc(aY + ks * 32, 16, 1024, kLayoutSW128),
-                              smem_desc(bV + ks * 1024, 16, 512, kLayoutSW64), idS, 1u);
+                mma_bf16_warp(tmem + Cfg::COL_S, smem_desc(aY + ks * 32, 16, 1024, kLayoutSW128),
+                              desc_v<DVT>(bV, ks), idS, 1u);
             mma_commit_warp(SDONE);
             mbar_wait(&FULLB[sb], (n / NSB) & 1, abort_flag);
-            const uint32_t aQ = smem_addr(slot_b + ChainSmem::B_QP);
-            const uint32_t aZ = smem_addr(slot_b + ChainSmem::B_ZB);
-            const uint32_t dO = tmem + kColO + 32 * (n & 1);
+            const uint32_t aQ = smem_addr(slot_b + Cfg::B_QP);
+            const uint32_t aZ = smem_addr(slot_b + Cfg::B_ZB);
+            const uint32_t dO = tmem + Cfg::COL_O + DVT * (n & 1);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)   // O = QP SB
                 mma_bf16_warp(dO, smem_desc(aQ + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                              smem_desc(bS + ks * 1024, 16, 512, kLayoutSW64), idO, ks > 0 ? 1u : 0u);
+                              desc_sb<DVT>(bS, ks), idO, ks > 0 ? 1u : 0u);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)   // O += ZB V
-                mma_bf16_warp(dO, smem_desc(aZ + ks * 32, 16, 1024, kLayoutSW128),
-                              smem_desc(bV + ks * 1024, 16, 512, kLayoutSW64), idO, 1u);
+                mma_bf16_warp(dO, smem_desc(aZ + ks * 32, 16, 1024, kLayoutSW128), desc_v<DVT>(bV, ks),
+                              idO, 1u);
             mma_commit_warp(&ODONE[n & 1]);
             mma_commit_warp(&EMPTYA[sa]);
             mma_commit_warp(&EMPTYB[sb]);
@@ -693,8 +734,9 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     } else {
         // ---------------------------------------------- the state chain
         const int quad = warp & 3;
+        const int col0 = 32 * ((warp - 1) >> 2);
         const int crow = 32 * quad + lane;
-        const size_t soff = ((size_t)seq * p.H + h) * (size_t)(DK * DV) + (size_t)crow * DV + j0;
+        const size_t soff = ((size_t)seq * p.H + h) * (size_t)(DK * DV) + (size_t)crow * DV + j0 + col0;
         float S[32];
         if (p.init_state) {
             const float4 *src = reinterpret_cast<const float4 *>(p.init_state + soff);
@@ -709,19 +751,19 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         }
         for (int n = 0; n < nchunks; ++n) {
             const int sa = n % NSA;
-            const uint8_t *slot_a = sm + ChainSmem::RA + sa * ChainSmem::A_STRIDE;
+            const uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
             if (n >= 1) {
                 mbar_wait(SDONE, (n - 1) & 1, abort_flag);
                 tc_fence_after();
-                tmem_ld32(tmem_addr(tmem, 32 * quad, kColS), S);
+                tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + col0), S);
                 tmem_wait_ld();
             }
-            store_bf16_row_sw64(sm + ChainSmem::SB + (n & 1) * 8192, crow, S);
+            store_sb_row<DVT>(sm + Cfg::SB + (n & 1) * Cfg::SB_BYTES, crow, col0, S);
             mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
-            const float d = reinterpret_cast<const float *>(slot_a + ChainSmem::A_EGL)[crow];
+            const float d = reinterpret_cast<const float *>(slot_a + Cfg::A_EGL)[crow];
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] *= d;
-            tmem_st32(tmem_addr(tmem, 32 * quad, kColS), S);
+            tmem_st32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + col0), S);
             tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
@@ -731,17 +773,17 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 const int m = n - 1;
                 mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
                 tc_fence_after();
-                store_o(tmem, quad, lane, m, bos, len, h, j0, p);
+                store_o<DVT>(tmem, quad, lane, col0, m, bos, len, h, j0, p);
             }
         }
         if (nchunks > 0) {
             const int m = nchunks - 1;
             mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
             tc_fence_after();
-            store_o(tmem, quad, lane, m, bos, len, h, j0, p);
+            store_o<DVT>(tmem, quad, lane, col0, m, bos, len, h, j0, p);
             mbar_wait(SDONE, m & 1, abort_flag);
             tc_fence_after();
-            tmem_ld32(tmem_addr(tmem, 32 * quad, kColS), S);
+            tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + col0), S);
             tmem_wait_ld();
         }
         if (p.final_state) {
@@ -755,7 +797,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kChainTmemCols);
+        tmem_dealloc(tmem, Cfg::TMEM_COLS);
     }
     if (tid == 0 && *abort_flag) atomicOr(p.err_word, kDevErrTimeout);
 }
@@ -914,6 +956,84 @@ SplitLayout split_layout(int num_seqs, int64_t total_tokens, int H) {
     return l;
 }
 
+// The chain kernel for one slice width: grid = sequences x heads x slices.
+// With `overlap` it is launched as a programmatic dependent of the prep grid.
+template <int DVT>
+cudaError_t launch_chain(const void *v, int64_t total_tokens, int H, const split::Params &prm,
+                         unsigned units, bool overlap, cudaStream_t stream) {
+    using namespace split;
+    using Cfg = ChainCfg<DVT>;
+    CUtensorMap mv;
+    if (!make_map_split(&mv, v, total_tokens, H, DV, DVT == 32 ? 32 : 64,
+                        DVT == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    static bool attr_set = false;
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(kda_chain_kernel<DVT>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)Cfg::ALLOC);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(units * Cfg::NTILE);
+    cfg.blockDim = dim3(Cfg::THREADS);
+    cfg.dynamicSmemBytes = Cfg::ALLOC;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = overlap ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kda_chain_kernel<DVT>, mv, prm);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+// Chain slice width and overlap, from a cost model in SM cycles:
+//   prep ~ items x c_p / (SMs it gets), c_p ~ 12 K cycles per (chunk, head)
+//     per SM (two pipelines per SM, ~24 K cycles per item each);
+//   chain ~ chunks per sequence x period when its CTAs fit on the GPU at
+//     once, else (CTA-chunks x period / SMs); period ~ 1.6 K cycles for a
+//     32-column slice and ~2.7 K for the whole d_v (a burst of N = 128
+//     products costs little more per instruction than N = 32, so the wide
+//     CTA does four times the work per chunk in under twice the time);
+//   overlap (prep on the SMs the chain leaves free, chain consuming
+//     records as they appear) costs the larger of the two, otherwise their
+//     sum.
+// Few (sequence, head) units and short chains favour narrow slices with
+// overlap; many units or long chains the whole-d_v CTA.
+struct ChainPlan {
+    int dvt;
+    bool overlap;
+};
+
+ChainPlan choose_chain(unsigned units, uint64_t items, int64_t total_tokens, int num_seqs,
+                       unsigned sm_count) {
+    const double c_p = 12e3, sm = (double)sm_count;
+    const double chunks = (double)((total_tokens / num_seqs + split::C - 1) / split::C);
+    ChainPlan best = {128, false};
+    double best_cost = -1.0;
+    const int widths[2] = {32, 128};
+    for (int wi = 0; wi < 2; ++wi) {
+        const int dvt = widths[wi];
+        const double per = dvt == 32 ? 1.6e3 : 2.7e3;
+        const double ctas = (double)units * (split::DV / dvt);
+        const double chain = ctas <= sm ? chunks * per : ctas * chunks * per / sm;
+        for (int ov = 0; ov < 2; ++ov) {
+            if (ov && ctas >= sm) continue;
+            const double cost = ov ? fmax((double)items * c_p / (sm - ctas), chain)
+                                   : (double)items * c_p / sm + chain;
+            if (best_cost < 0.0 || cost < best_cost) {
+                best_cost = cost;
+                best.dvt = dvt;
+                best.overlap = ov != 0;
+            }
+        }
+    }
+    return best;
+}
+
 }  // namespace
 
 size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H) {
@@ -934,17 +1054,16 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     int32_t *chunk_off = reinterpret_cast<int32_t *>(ws + l.chunk_off);
     int2 *chunk_tab = reinterpret_cast<int2 *>(ws + l.chunk_tab);
 
-    CUtensorMap mk, mq, mg, mv;
+    CUtensorMap mk, mq, mg;
     if (!make_map_split(&mk, k, total_tokens, H, DK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_split(&mq, q, total_tokens, H, DK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_split(&mg, g, total_tokens, H, DK, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map_split(&mv, v, total_tokens, H, DV, DVT, CU_TENSOR_MAP_SWIZZLE_64B))
+        !make_map_split(&mg, g, total_tokens, H, DK, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    // Prep runs as a persistent grid (one CTA per SM).  When the chain needs
-    // few SMs, the prep grid leaves those SMs free and the chain kernel is
-    // launched as a programmatic dependent of it, so that it starts at once
-    // and consumes records as they are published; otherwise the two kernels
-    // run one after the other and the records need no flags.
+    // Prep runs as a persistent grid (one CTA per SM).  With overlap the prep
+    // grid leaves the chain's SMs free and the chain kernel is launched as a
+    // programmatic dependent of it, so that it starts at once and consumes
+    // records as they are published; otherwise the two kernels run one after
+    // the other and the records need no flags.
     static int sm_count = 0;
     if (!sm_count) {
         int dev = 0;
@@ -952,8 +1071,11 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
             cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             sm_count = 148;
     }
-    const unsigned chain_blocks = (unsigned)((size_t)num_seqs * H * NTILE);
-    const bool overlap = chain_blocks * 10 <= (unsigned)sm_count * 6;   // chain needs <= 60 % of SMs
+    const unsigned units = (unsigned)((size_t)num_seqs * H);
+    const ChainPlan plan = choose_chain(units, (uint64_t)(total_tokens / C + num_seqs) * H, total_tokens,
+                                        num_seqs, (unsigned)sm_count);
+    const bool overlap = plan.overlap;
+    const unsigned chain_blocks = units * (unsigned)(DV / plan.dvt);
     uint32_t *rec_ready = overlap ? reinterpret_cast<uint32_t *>(ws + l.flags) : nullptr;
     kda_split_plan_kernel<<<1, kPlanThreads, 0, stream>>>(cu, num_seqs, total_tokens, perm,
                                                           chunk_off, chunk_tab, total_chunks, err,
@@ -965,9 +1087,6 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     if (!attr_set) {
         e = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)PrepSmem::ALLOC);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kda_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)ChainSmem::ALLOC);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -996,19 +1115,8 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     kda_prep_kernel<<<(unsigned)prep_blocks, kPrepThreads, PrepSmem::ALLOC, stream>>>(mk, mq, mg, prm);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(chain_blocks);
-    cfg.blockDim = dim3(kChainThreads);
-    cfg.dynamicSmemBytes = ChainSmem::ALLOC;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = overlap ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kda_chain_kernel, mv, prm);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    return plan.dvt == 32 ? launch_chain<32>(v, total_tokens, H, prm, units, overlap, stream)
+                          : launch_chain<128>(v, total_tokens, H, prm, units, overlap, stream);
 }
 
 }  // namespace kda

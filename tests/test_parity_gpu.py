@@ -249,3 +249,32 @@ def test_prefill_single_kernel_path_with_small_workspace():
     ref_o, ref_s, cu, _, _ = run_oracle(inp)
     assert o_err(f64(o), ref_o, cu, 2) <= TOL["bf16"]
     assert state_err(f64(fs), ref_s) <= TOL["bf16"]
+
+
+def test_prefill_many_short_sequences():
+    """180 (sequence, head) units of ragged lengths, empty ones included: more
+    units than SMs, so the chain runs one CTA per (sequence, head) over the
+    whole d_v, after the preparation."""
+    rng = np.random.default_rng(123)
+    lens = [int(x) for x in rng.integers(0, 200, size=60)]
+    lens[3] = 0
+    lens[17] = 64
+    inp = make(0, 3, 128, 128, dtype="bf16", seed=123, lengths=lens, init_std=0.02)
+    o, fs = gpu_prefill(inp)
+    ref_o, ref_s, cu, _, _ = run_oracle(inp)
+    assert o_err(f64(o), ref_o, cu, 3) <= TOL["bf16"]
+    assert state_err(f64(fs), ref_s) <= TOL["bf16"]
+    assert torch.equal(fs[3], inp["init_state"][3])
+
+
+def test_prefill_whole_dv_chain_overlapped():
+    """40 units of 500-1500 tokens: the chain runs one CTA per (sequence,
+    head) over the whole d_v, overlapped with the preparation (records
+    consumed as their ready flags appear)."""
+    rng = np.random.default_rng(321)
+    lens = [int(x) for x in rng.integers(500, 1500, size=10)]
+    inp = make(0, 4, 128, 128, dtype="bf16", seed=321, lengths=lens, init_std=0.02)
+    o, fs = gpu_prefill(inp)
+    ref_o, ref_s, cu, _, _ = run_oracle(inp)
+    assert o_err(f64(o), ref_o, cu, 4) <= TOL["bf16"]
+    assert state_err(f64(fs), ref_s) <= TOL["bf16"]
