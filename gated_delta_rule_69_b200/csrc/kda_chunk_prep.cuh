@@ -327,26 +327,26 @@ __device__ void solve(const Bufs &b, int pt) {
     }
 }
 
-// ---- -W from TMEM (M = 64 layout: row r in lane (r mod 16) + 32 (r / 16))
-// over Ktil in b.stk (rows 0-63), so that [-W; Qtil] is one M = 128 operand.
+// ---- -W from TMEM over Ktil in b.stk (rows 0-63).  W is rows 0-63 of the
+// M = 128 product [T_beta; P] Ktil (row r in lane r), so the warps of TMEM
+// quadrants 0 and 1 read it, each half `half` of the 128 columns.
 __device__ __forceinline__ void read_w(const Bufs &b, uint32_t tmem_w, int quad, int half, int lane) {
+    if (quad >= 2) return;
     uint8_t *wdst = b.stk + half * 16384;
-    const int t = 16 * quad + lane;
+    const int t = 32 * quad + lane;
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
         float v[32];
         tmem_ld32(tmem_addr(tmem_w, 32 * quad, 64 * half + 32 * part), v);
         tmem_wait_ld();
-        if (lane < 16) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-                uint4 pk;
-                pk.x = pack_bf16x2(-v[j + 0], -v[j + 1]);
-                pk.y = pack_bf16x2(-v[j + 2], -v[j + 3]);
-                pk.z = pack_bf16x2(-v[j + 4], -v[j + 5]);
-                pk.w = pack_bf16x2(-v[j + 6], -v[j + 7]);
-                *reinterpret_cast<uint4 *>(wdst + sw128_off(t, 32 * part + j)) = pk;
-            }
+        for (int j = 0; j < 32; j += 8) {
+            uint4 pk;
+            pk.x = pack_bf16x2(-v[j + 0], -v[j + 1]);
+            pk.y = pack_bf16x2(-v[j + 2], -v[j + 3]);
+            pk.z = pack_bf16x2(-v[j + 4], -v[j + 5]);
+            pk.w = pack_bf16x2(-v[j + 6], -v[j + 7]);
+            *reinterpret_cast<uint4 *>(wdst + sw128_off(t, 32 * part + j)) = pk;
         }
     }
 }

@@ -87,7 +87,7 @@ static_assert(PrepSmem::KHAT + 64 * prep::kAStride * 4 <= PrepSmem::GRAW &&
                   PrepSmem::XF + 4608 <= PrepSmem::BETA,
               "solve scratch");
 // per pipeline (256 columns): [A;P] at 0 and W at 64; then MP at 0, YT at 128,
-// ZB at 192 (M = 64); then -P W at 0 (M = 64)
+// ZB at 192; then -P W at 0 (all M = 128 products)
 constexpr uint32_t kPrepTmemCols = 512;
 constexpr uint32_t kRawBytes = 4 * 8192 + 16384;   // k, q (2 boxes each), log_alpha
 
@@ -265,29 +265,33 @@ __device__ __forceinline__ void write_yt(uint8_t *yt, uint32_t tmem, int quad, i
     for (int j = 0; j < 32; j += 8) store8(yt, row, 32 * half + j, v + j);
 }
 
-// ZB [64 t][64 i] (M = 64).
+// ZB [64 t][64 i]: rows 0-63 of an M = 128 product whose A operand starts
+// at P (rows 64-127 multiply whatever follows P in shared memory and are not
+// read), read by the warps of TMEM quadrants 0 and 1.
 __device__ __forceinline__ void write_zb(uint8_t *zb, uint32_t tmem, int quad, int half, int lane) {
+    if (quad >= 2) return;
     float v[32];
     tmem_ld32(tmem_addr(tmem, 32 * quad, 32 * half), v);
     tmem_wait_ld();
-    if (lane < 16) {
-        const int t = 16 * quad + lane;
+    const int t = 32 * quad + lane;
 #pragma unroll
-        for (int j = 0; j < 32; j += 8) store8(zb, t, 32 * half + j, v + j);
-    }
+    for (int j = 0; j < 32; j += 8) store8(zb, t, 32 * half + j, v + j);
 }
 
-// QP = Qtil + P (-W) (M = 64), in place over Qtil: rows 64-127 of the two
-// 16 KB K-atoms of `stk`, K-atom `half` holding channels 64 half .. + 63.
+// QP = Qtil + P (-W), in place over Qtil: rows 64-127 of the two 16 KB
+// K-atoms of `stk`, K-atom `half` holding channels 64 half .. + 63.  P (-W)
+// is rows 0-63 of an M = 128 product whose A operand starts at P, read by the
+// warps of TMEM quadrants 0 and 1.
 __device__ __forceinline__ void write_qp(uint8_t *stk, uint32_t tmem, int quad, int half, int lane) {
+    if (quad >= 2) return;
     uint8_t *atom = stk + half * 16384;
-    const int t = 16 * quad + lane;
+    const int t = 32 * quad + lane;
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
         float v[32];
         tmem_ld32(tmem_addr(tmem, 32 * quad, 64 * half + 32 * part), v);
         tmem_wait_ld();
-        if (lane < 16) {
+        {
 #pragma unroll
             for (int j = 0; j < 32; j += 8) {
                 uint4 *q8 = reinterpret_cast<uint4 *>(atom + sw128_off(64 + t, 32 * part + j));
@@ -421,9 +425,9 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         const uint32_t sT = smem_addr(sm + PrepSmem::TB), sP = smem_addr(sm + PrepSmem::PB);
         if (wp == 0) {
             tc_fence_after();
-            const uint32_t idW = idesc_bf16(64, DK, false, true);
+            const uint32_t idW = idesc_bf16(128, DK, false, true);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)   // W = T diag(beta) Ktil
+            for (int ks = 0; ks < 4; ++ks)   // [T_beta; P] Ktil: rows 0-63 are W = T_beta Ktil
                 mma_bf16_warp(tmem + 64, smem_desc(sT + ks * 32, 16, 1024, kLayoutSW128),
                               smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idW, ks > 0 ? 1u : 0u);
             mma_commit_warp(&B[2]);
@@ -438,7 +442,7 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
             tc_fence_after();
             const uint32_t idM = idesc_bf16(128, DK, true, true);
             const uint32_t idY = idesc_bf16(128, C, true, true);
-            const uint32_t idZ = idesc_bf16(64, C, false, true);
+            const uint32_t idZ = idesc_bf16(128, C, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {   // K = 64 tokens
                 const uint64_t aKb = smem_desc(sKb + ks * 2048, 8192, 1024, kLayoutSW128);   // Kbar^T
@@ -448,7 +452,7 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
                 // YT = Kbar^T T_beta
                 mma_bf16_warp(tmem + 128, aKb, smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idY,
                               ks > 0 ? 1u : 0u);
-                // ZB = P T_beta
+                // ZB = P T_beta: rows 0-63 of an M = 128 product whose A starts at P
                 mma_bf16_warp(tmem + 192, smem_desc(sP + ks * 32, 16, 1024, kLayoutSW128),
                               smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idZ, ks > 0 ? 1u : 0u);
             }
@@ -461,9 +465,11 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         named_barrier(BAR, prep::kGroupThreads);
         if (wp == 0) {
             tc_fence_after();
-            const uint32_t idQ = idesc_bf16(64, DK, false, true);
+            const uint32_t idQ = idesc_bf16(128, DK, false, true);
+            // P (-W), into the columns MP has left: rows 0-63 of an M = 128
+            // product whose A starts at P
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)   // P (-W), into the columns MP has left
+            for (int ks = 0; ks < 4; ++ks)
                 mma_bf16_warp(tmem, smem_desc(sP + ks * 32, 16, 1024, kLayoutSW128),
                               smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idQ, ks > 0 ? 1u : 0u);
             mma_commit_warp(&B[4]);
