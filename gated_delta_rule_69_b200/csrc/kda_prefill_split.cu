@@ -136,7 +136,7 @@ struct Params {
     const int32_t *cu;          // may be null: equal lengths
     const int32_t *perm;        // longest-first order (chain kernel) or null
     const int32_t *chunk_off;   // [N+1] first record index of each sequence
-    const int2 *chunk_tab;      // [max_chunks] (sequence, chunk) of each record
+    const int2 *chunk_tab;      // [max_chunks] (first token, length) of each record's chunk
     const uint32_t *total_chunks;
     uint8_t *recs;              // records, STRIDE bytes each, index (chunk * H + h)
     uint32_t *rec_ready;        // [max_chunks * H] set to 1 once a record is complete; null
@@ -340,11 +340,9 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
     for (int it = 0; item < total_items; ++it) {
         const int h = item % p.H;
         const uint32_t chunk = item / p.H;
-        const int2 sc = p.chunk_tab[chunk];
-        int64_t bos, eos;
-        seq_bounds(p, sc.x, bos, eos);
-        const int64_t tok0 = bos + (int64_t)sc.y * C;
-        const int L = (int)min((int64_t)C, eos - tok0);
+        const int2 ct = p.chunk_tab[chunk];   // one load: the token range was planned
+        const int64_t tok0 = ct.x;
+        const int L = ct.y;
         uint8_t *rec = p.recs + ((size_t)chunk * p.H + h) * Rec::STRIDE;
         // Loads.  The leader reaches this point after every thread has
         // passed the previous item's last barrier and after the record
@@ -811,7 +809,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 // =============================================================== plan kernel
 // One CTA: checks cu_seqlens (error word), counts each sequence's chunks,
 // writes the record offset of every sequence (exclusive prefix sum), the
-// (sequence, chunk) of every record, the record count, and the longest-first
+// first token and length of every record's chunk, the record count, and the longest-first
 // sequence order used by the chain kernel.
 constexpr int kPlanThreads = 1024;
 constexpr int kMaxSortedSeqs = 4096;
@@ -887,7 +885,10 @@ kda_split_plan_kernel(const int32_t *cu, int n, int64_t total, int32_t *perm, in
             if (chunk_off[mid] <= c) lo = mid;
             else hi = mid;
         }
-        chunk_tab[c] = make_int2(lo, c - chunk_off[lo]);
+        const int64_t bos = cu ? (int64_t)cu[lo] : (int64_t)lo * (total / n);
+        const int64_t t0 = bos + (int64_t)(c - chunk_off[lo]) * C;
+        const int64_t len = seq_len_checked(cu, lo, n, total);
+        chunk_tab[c] = make_int2((int)t0, (int)min((int64_t)C, bos + len - t0));
     }
     if (!perm) return;
     for (int i = tid; i < n; i += kPlanThreads) {
