@@ -59,6 +59,11 @@ WORKLOADS = {
         "varlen_16seq_256to16384_H32_d128", "prefill", H=32, d_k=128, d_v=128,
         dtype="bf16", seed=1003, num_seqs=16, varlen=(256, 16384),
         init_std=0.02),
+    # a smaller case of the 131072-token workload's kernels (same heads and
+    # chain plan), small enough for a full profiler capture
+    "prefill_T16384_H32_d128": Workload(
+        "prefill_T16384_H32_d128", "prefill", H=32, d_k=128, d_v=128,
+        dtype="bf16", seed=1005, T=16384, init_std=0.02),
     "decode_B256_H32_d128": Workload(
         "decode_B256_H32_d128", "decode", H=32, d_k=128, d_v=128,
         dtype="bf16", seed=1004, batch=256, init_std=0.02),
