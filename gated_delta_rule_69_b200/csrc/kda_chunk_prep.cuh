@@ -24,7 +24,10 @@ using namespace sm100;
 constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int kGroupThreads = 256;
-constexpr float kSlowPathLogDecay = -60.0f;   // chunk log-decay below this -> pairwise path
+// A chunk whose log-decay on some channel is below this takes the pairwise
+// path: above it, e^{G} and e^{-G} (<= e^80 ~ 5.5e34) are normal numbers in
+// bf16 and fp32, so the product form keeps its relative precision.
+constexpr float kSlowPathLogDecay = -80.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // e^x through the hardware base-2 exponential (ex2.approx, flush-to-zero):

@@ -190,6 +190,10 @@ def _stress(kind, T=256, H=2):
     elif kind == "beta_one_qk":       # replace completely, read back with q = k
         inp["beta"] = torch.ones_like(inp["beta"])
         inp["q"] = inp["k"].clone()
+    elif kind == "decay_near_limit":  # a chunk decays by e^-76.8: still the product form
+        inp["log_alpha"] = torch.full_like(g, -1.2)
+    elif kind == "decay_past_limit":  # e^-83.2 per chunk: the pairwise path
+        inp["log_alpha"] = torch.full_like(g, -1.3)
     elif kind == "mixed_extremes":    # half the channels keep, half forget fast
         g2 = g.clone()
         g2[..., ::2] = 0.0
@@ -199,7 +203,8 @@ def _stress(kind, T=256, H=2):
 
 
 @pytest.mark.parametrize("kind", ["alpha_half", "gate_floor", "alpha_one", "alpha_zero",
-                                  "beta_zero", "beta_one_qk", "mixed_extremes"])
+                                  "beta_zero", "beta_one_qk", "mixed_extremes",
+                                  "decay_near_limit", "decay_past_limit"])
 def test_prefill_stress(kind):
     inp = _stress(kind)
     o, fs = gpu_prefill(inp)
