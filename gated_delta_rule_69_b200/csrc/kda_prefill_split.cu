@@ -95,7 +95,8 @@ constexpr uint32_t kRawBytes = 4 * 8192 + 16384;   // k, q (2 boxes each), log_a
 // Warp 0 loads; warps 1 .. NCW hold the state (warp w: TMEM lanes of quadrant
 // w mod 4, columns 32 ((w - 1) / 4) .. + 31 of the slice); warp NCW + 1 issues
 // the products.  Ring A carries MP, YT, the v slice and exp(G_L); ring B QP,
-// ZB; the bf16 copy of the state is double-buffered.
+// ZB; the bf16 copy of the state is double-buffered.  Stages (A, B): (3, 2)
+// for 32 columns, (3, 1) for 64, (2, 1) for 128: what shared memory holds.
 constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 
 template <int DVT_>
@@ -104,18 +105,19 @@ struct ChainCfg {
     static constexpr int NTILE = DV / DVT;
     static constexpr int NCW = 4 * (DVT / 32);
     static constexpr int THREADS = 32 * (NCW + 2);
-    static constexpr int NSA = DVT == 32 ? 3 : 2;
-    static constexpr int NSB = DVT == 128 ? 1 : 2;
+    static constexpr int NSA = DVT == 128 ? 2 : 3;
+    static constexpr int NSB = DVT == 32 ? 2 : 1;
     static constexpr uint32_t V_BYTES = (uint32_t)DVT * C * 2;
-    static constexpr uint32_t A_MP = 0, A_YT = 32768, A_V = 49152, A_EGL = A_V + V_BYTES;
-    static constexpr uint32_t A_STRIDE = align1k(A_EGL + 512);
+    static constexpr uint32_t A_MP = 0, A_YT = 32768, A_V = 49152;
+    static constexpr uint32_t A_STRIDE = align1k(A_V + V_BYTES);
     static constexpr uint32_t B_QP = 0, B_ZB = 16384;
     static constexpr uint32_t B_STRIDE = 24576;
     static constexpr uint32_t SB_BYTES = (uint32_t)DK * DVT * 2;   // S bf16 [128 c][DVT j]
     static constexpr uint32_t RA = 0;
     static constexpr uint32_t RB = NSA * A_STRIDE;
     static constexpr uint32_t SB = RB + NSB * B_STRIDE;
-    static constexpr uint32_t BARS = SB + 2 * SB_BYTES;
+    static constexpr uint32_t EGLR = SB + 2 * SB_BYTES;     // NSA x exp(G_L), 128 fp32 each
+    static constexpr uint32_t BARS = EGLR + NSA * 512;
     static constexpr uint32_t MISC = BARS + 128;
     static constexpr uint32_t SIZE = MISC + 64;
     static constexpr uint32_t ALLOC = SIZE + 1024;
@@ -673,7 +675,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 const int t = (int)(bos + (int64_t)n * C);
                 mbar_arrive_expect_tx(&FULLA[sa], 49152 + 512 + Cfg::V_BYTES);
                 bulk_load(slot_a + Cfg::A_MP, rec + Rec::MP, 49152, &FULLA[sa]);   // MP, YT
-                bulk_load(slot_a + Cfg::A_EGL, rec + Rec::EGL, 512, &FULLA[sa]);
+                bulk_load(sm + Cfg::EGLR + sa * 512, rec + Rec::EGL, 512, &FULLA[sa]);
                 tma_load_3d(slot_a + Cfg::A_V, &tm_v, &FULLA[sa], j0, h, t);
                 if (DVT == 128) tma_load_3d(slot_a + Cfg::A_V + 8192, &tm_v, &FULLA[sa], j0 + 64, h, t);
                 issued_a = n + 1;
@@ -764,7 +766,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             }
             store_sb_row<DVT>(sm + Cfg::SB + (n & 1) * Cfg::SB_BYTES, crow, col0, S);
             mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
-            const float d = reinterpret_cast<const float *>(slot_a + Cfg::A_EGL)[crow];
+            const float d = reinterpret_cast<const float *>(sm + Cfg::EGLR + sa * 512)[crow];
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] *= d;
             tmem_st32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + col0), S);
