@@ -232,33 +232,85 @@ __device__ bool prep_gate(uint8_t *__restrict__ sm, int pt, int s, int L) {
     return slow;
 }
 
+// 32 consecutive bf16 of a global row as fp32 (zeros when !valid).
+__device__ __forceinline__ void row32_f(const __nv_bfloat16 *src, float (&v)[32], bool valid) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) w = reinterpret_cast<const uint4 *>(src)[q];
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&ww[e]);
+            v[8 * q + 2 * e] = __low2float(h2);
+            v[8 * q + 2 * e + 1] = __high2float(h2);
+        }
+    }
+}
+
 // ---- pairwise fallback for A and P when a chunk decays too fast for the
-// product form: differences of running sums taken pair by pair in fp32.
+// product form.  A quad of lanes (four groups of 32 channels) owns column i
+// and walks the rows t = i .. 63 in order, carrying d = G_t - G_i (the sum of
+// log_alpha over tokens i+1 .. t) per channel, so every exponent is a
+// difference of running sums taken in fp32 and is <= 0; the quad's partial
+// sums are combined with shuffles.  All lanes of a warp walk the same rows
+// (from the warp's first column), so the shuffles stay converged.
 __device__ void prep_pairwise(uint8_t *sm, int pt, int s, int L, const Params &p,
                               int64_t tok0, int h) {
     const uint8_t *graw = sm + Smem::GRAW + s * 16384;
     const float *beta = reinterpret_cast<const float *>(sm + Smem::BETA) + s * C;
     float *AF = reinterpret_cast<float *>(sm + Smem::AF);
     uint8_t *pb = sm + Smem::PB + s * 8192;
-    for (int pidx = pt; pidx < C * C; pidx += kPrepThreads) {
-        const int t = pidx >> 6, i = pidx & 63;
-        float ak = 0.f, aq = 0.f;
-        if (i <= t && t < L) {
-            const __nv_bfloat16 *kt = p.k + ((size_t)(tok0 + t) * p.H + h) * DK;
-            const __nv_bfloat16 *ki = p.k + ((size_t)(tok0 + i) * p.H + h) * DK;
-            const __nv_bfloat16 *qt = p.q + ((size_t)(tok0 + t) * p.H + h) * DK;
-            for (int c = 0; c < DK; ++c) {
-                float d = 0.f;  // G_t - G_i = sum of log_alpha over tokens i+1..t
-                for (int u = i + 1; u <= t; ++u)
-                    d += clamp_log_alpha(__bfloat162float(
-                        *reinterpret_cast<const __nv_bfloat16 *>(graw + u * 256 + c * 2)));
-                const float kd = __bfloat162float(ki[c]) * exp_f(d);
-                ak = fmaf(__bfloat162float(kt[c]), kd, ak);
-                aq = fmaf(__bfloat162float(qt[c]), kd, aq);
+    const size_t row_stride = (size_t)p.H * DK;
+    const __nv_bfloat16 *kt0 = p.k + ((size_t)tok0 * p.H + h) * DK;
+    const __nv_bfloat16 *qt0 = p.q + ((size_t)tok0 * p.H + h) * DK;
+    const int i = pt >> 2, cg = pt & 3, c0 = 32 * cg;
+    const bool lead = cg == 0;
+    const int t_first = (pt >> 5) * 8;
+    float ki[32], d[32];
+    row32_f(kt0 + (size_t)i * row_stride + c0, ki, i < L);
+#pragma unroll
+    for (int c = 0; c < 32; ++c) d[c] = 0.f;
+    if (lead) {   // rows above the diagonal
+        for (int t = 0; t < i; ++t) {
+            AF[fidx(t, i)] = 0.f;
+            *reinterpret_cast<__nv_bfloat16 *>(pb + sw128_off(t, i)) = __float2bfloat16_rn(0.f);
+        }
+    }
+    for (int t = t_first; t < C; ++t) {
+        const bool active = t >= i;
+        if (t > i) {
+            const uint4 *gr = reinterpret_cast<const uint4 *>(graw + t * 256 + c0 * 2);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 w = gr[q];
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&ww[e]);
+                    d[8 * q + 2 * e] += clamp_log_alpha(__low2float(h2));
+                    d[8 * q + 2 * e + 1] += clamp_log_alpha(__high2float(h2));
+                }
             }
         }
-        AF[fidx(t, i)] = (i < t) ? beta[t] * ak : 0.f;
-        *reinterpret_cast<__nv_bfloat16 *>(pb + sw128_off(t, i)) = __float2bfloat16_rn(aq);
+        float kt[32], qt[32];
+        row32_f(kt0 + (size_t)t * row_stride + c0, kt, active && t < L);
+        row32_f(qt0 + (size_t)t * row_stride + c0, qt, active && t < L);
+        float a = 0.f, pq = 0.f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+            const float w = ki[c] * exp_f(d[c]);
+            a = fmaf(kt[c], w, a);
+            pq = fmaf(qt[c], w, pq);
+        }
+        a += __shfl_xor_sync(0xffffffffu, a, 1);
+        a += __shfl_xor_sync(0xffffffffu, a, 2);
+        pq += __shfl_xor_sync(0xffffffffu, pq, 1);
+        pq += __shfl_xor_sync(0xffffffffu, pq, 2);
+        if (lead && active) {
+            AF[fidx(t, i)] = (t > i) ? beta[t] * a : 0.f;
+            *reinterpret_cast<__nv_bfloat16 *>(pb + sw128_off(t, i)) = __float2bfloat16_rn(pq);
+        }
     }
 }
 

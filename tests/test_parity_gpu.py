@@ -283,3 +283,23 @@ def test_prefill_whole_dv_chain_overlapped():
     ref_o, ref_s, cu, _, _ = run_oracle(inp)
     assert o_err(f64(o), ref_o, cu, 4) <= TOL["bf16"]
     assert state_err(f64(fs), ref_s) <= TOL["bf16"]
+
+
+def test_prefill_single_kernel_path_fast_decay():
+    """The single-kernel path on gates of -2 per token (a chunk decays by
+    e^-128): every chunk takes the pairwise path."""
+    lens = [130, 0, 64, 257, 1]
+    inp = make(0, 2, 128, 128, dtype="bf16", seed=37, lengths=lens, init_std=0.02)
+    inp["log_alpha"] = torch.full_like(inp["log_alpha"], -2.0)
+    k = kda()
+    small = (256 + ((len(lens) * 4 + 255) // 256) * 256)
+    ws = torch.empty(small, dtype=torch.uint8, device=DEV)
+    o = torch.full((sum(lens), 2, 128), float("nan"), dtype=torch.bfloat16, device=DEV)
+    o, fs = k.kda_prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                          init_state=inp["init_state"], cu_seqlens=inp["cu_seqlens"], o=o,
+                          workspace=ws)
+    torch.cuda.synchronize()
+    assert k.kda_check_workspace_error(ws) == k.KDA_OK
+    ref_o, ref_s, cu, _, _ = run_oracle(inp)
+    assert o_err(f64(o), ref_o, cu, 2) <= TOL["bf16"]
+    assert state_err(f64(fs), ref_s) <= TOL["bf16"]
