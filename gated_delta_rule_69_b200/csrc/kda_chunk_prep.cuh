@@ -75,10 +75,14 @@ __device__ __forceinline__ int tfi(int row, int col) { return row * kTStride + c
 // one 64-channel K-atom of one token group.  Rows past the chunk's end (a
 // sequence's last chunk) are zeroed first, so that they add nothing to the
 // running sums and give zero operand rows.  The running sums are kept in
-// base-2 units (log_alpha log2(e)).  Returns whether the chunk needs the
-// pairwise path.
+// base-2 units (log_alpha log2(e)).  Returns how [A; P] is to be formed:
+// kProductForm (one reference, the chunk start), kSecondary (the chunk
+// decays below e^-80 on some channel, but no 16-token block does: one
+// reference per block) or kPairwise.
+enum : int { kProductForm = 0, kSecondary = 1, kPairwise = 2 };
+
 template <int BAR>
-__device__ bool gate(const Bufs &b, int pt, int L) {
+__device__ int gate(const Bufs &b, int pt, int L) {
     const int c = 2 * (pt & 63);
     const int tg = pt >> 6;
     const int t0 = tg * 16;
@@ -132,9 +136,11 @@ __device__ bool gate(const Bufs &b, int pt, int L) {
         GL1 += bb;
     }
     constexpr float kSlow2 = kSlowPathLogDecay * kLog2e;
-    if (tg == 0 && (GL0 < kSlow2 || GL1 < kSlow2)) *b.slow_flag = 1u;
+    if (tg == 0 && (GL0 < kSlow2 || GL1 < kSlow2)) atomicOr(b.slow_flag, 1u);
+    if (r0 < kSlow2 || r1 < kSlow2) atomicOr(b.slow_flag, 2u);   // this 16-token block alone
     named_barrier(BAR, kGroupThreads);
-    const bool slow = *b.slow_flag != 0u;
+    const uint32_t flag = *b.slow_flag;
+    const bool slow = (flag & 1u) != 0u;
 
     const float eL0 = exp2_f(GL0), eL1 = exp2_f(GL1);
     if (tg == 0) {
@@ -162,7 +168,105 @@ __device__ bool gate(const Bufs &b, int pt, int L) {
         *reinterpret_cast<uint32_t *>(khat + ok) = pack_bf16x2(k0 * ih0, k1 * ih1);
         *reinterpret_cast<uint32_t *>(kbar + ok) = pack_bf16x2(k0 * b0, k1 * b1);
     }
-    return slow;
+    return !slow ? kProductForm : ((flag & 2u) ? kPairwise : kSecondary);
+}
+
+// ---- secondary chunking, for a chunk that decays too fast for one reference
+// but not within any 16-token block.  For each column block bb, with the
+// running sum just before the block as reference (off_bb, per channel), the
+// rows t >= 16 bb scaled by e^{G_t - off_bb} (<= 1) and the block's columns
+// by e^{off_bb - G_i} (<= e^80) give columns 16 bb .. + 15 of
+// [Ktil Khat^T; Qtil Khat^T] as one M = 128, N = 16 product; rows above the
+// block hold leftovers of earlier blocks, which the read-out masks.  The four
+// products fill the TMEM columns the one-reference product does, so the same
+// read-out follows.  Operand tiles: rows [k; q] in two K-atoms at opa0 and
+// opa1 (16 KB each), the block's columns in two 2 KB K-atoms at opc; raw g
+// is read from b.graw before opa1 may overwrite it; raw k and q come from
+// global memory (kt0 / qt0, as for the pairwise path).  `round` counts the
+// phases of `bar` across calls.
+template <int BAR>
+__device__ void secondary(const Bufs &b, int pt, int L, const __nv_bfloat16 *kt0,
+                          const __nv_bfloat16 *qt0, size_t row_stride, uint8_t *opa0,
+                          uint8_t *opa1, uint8_t *opc, uint32_t tmem_ap, bool issue_warp,
+                          uint64_t *bar, uint32_t &round, volatile uint32_t *abort) {
+    const int c = 2 * (pt & 63);
+    const int tg = pt >> 6;
+    const int t0 = tg * 16;
+    const int katom = c >> 6, cc = c & 63;
+    uint8_t *atom_a = katom ? opa1 : opa0;
+    uint8_t *atom_c = opc + katom * 2048;
+    float G0[16], G1[16];
+    {
+        float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 gv =
+                *reinterpret_cast<const __nv_bfloat162 *>(b.graw + (t0 + i) * 256 + c * 2);
+            r0 = fmaf(clamp_log_alpha(__low2float(gv)), kLog2e, r0);
+            r1 = fmaf(clamp_log_alpha(__high2float(gv)), kLog2e, r1);
+            G0[i] = r0;
+            G1[i] = r1;
+        }
+    }
+    float off0[4], off1[4];   // running sum before each block
+    off0[0] = off1[0] = 0.f;
+#pragma unroll
+    for (int j = 1; j < 4; ++j) {
+        off0[j] = off0[j - 1] + b.csum[(j - 1) * 128 + c];
+        off1[j] = off1[j - 1] + b.csum[(j - 1) * 128 + c + 1];
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        G0[i] += off0[tg];
+        G1[i] += off1[tg];
+    }
+    uint32_t kv[16], qv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int t = t0 + i;
+        kv[i] = t < L ? *reinterpret_cast<const uint32_t *>(kt0 + (size_t)t * row_stride + c) : 0u;
+        qv[i] = t < L ? *reinterpret_cast<const uint32_t *>(qt0 + (size_t)t * row_stride + c) : 0u;
+    }
+    named_barrier(BAR, kGroupThreads);   // raw g read everywhere before opa1 is written
+    for (int bb = 0; bb < 4; ++bb) {
+        const float ob0 = off0[bb], ob1 = off1[bb];
+        if (tg >= bb) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int t = t0 + i;
+                const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(&kv[i]);
+                const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(&qv[i]);
+                const float e0 = exp2_f(G0[i] - ob0), e1 = exp2_f(G1[i] - ob1);
+                *reinterpret_cast<uint32_t *>(atom_a + sw128_off(t, cc)) =
+                    pack_bf16x2(__low2float(k2) * e0, __high2float(k2) * e1);
+                *reinterpret_cast<uint32_t *>(atom_a + sw128_off(64 + t, cc)) =
+                    pack_bf16x2(__low2float(q2) * e0, __high2float(q2) * e1);
+                if (tg == bb) {
+                    const float f0 = exp2_f(ob0 - G0[i]), f1 = exp2_f(ob1 - G1[i]);
+                    *reinterpret_cast<uint32_t *>(atom_c + sw128_off(i, cc)) =
+                        pack_bf16x2(__low2float(k2) * f0, __high2float(k2) * f1);
+                }
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        named_barrier(BAR, kGroupThreads);
+        if (issue_warp) {
+            tc_fence_after();
+            const uint32_t a0 = smem_addr(opa0), a1 = smem_addr(opa1), c0 = smem_addr(opc);
+            const uint32_t id = idesc_bf16(128, 16, false, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16_warp(tmem_ap + 16 * bb,
+                              smem_desc((ks >> 2 ? a1 : a0) + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(c0 + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              id, ks > 0 ? 1u : 0u);
+            mma_commit_warp(bar);
+        }
+        mbar_wait(bar, round & 1u, abort);   // this block's operands are free again
+        ++round;
+        tc_fence_after();
+    }
 }
 
 // 32 consecutive bf16 of a global row as fp32 (zeros when !valid).

@@ -74,7 +74,7 @@ struct PrepSmem {
     static constexpr uint32_t XF = 101376;     // solve scratch (4608 bytes)
     static constexpr uint32_t BETA = 105984;   // 64 fp32
     static constexpr uint32_t CSUM = 106240;   // 4 x 128 fp32
-    static constexpr uint32_t BARS = 108288;   // 5 mbarriers
+    static constexpr uint32_t BARS = 108288;   // 6 mbarriers
     static constexpr uint32_t MISC = 108352;   // tmem base, abort, slow flag, next-item slots at 4, 5
     static constexpr uint32_t SIZE = 108416;
     static constexpr uint32_t PIPE = 109568;   // per-pipeline stride
@@ -322,7 +322,8 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
     const int pt = tid - P * kPipeThreads;
     const bool leader = pt == 0;
     const int quad = warp & 3, half = wp >> 2;
-    uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);   // raw, [A;P], W, MP/YT/ZB, PW
+    uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);   // raw, [A;P], W, MP/YT/ZB, PW,
+                                                                      // secondary-chunking blocks
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + PrepSmem::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     float *beta = reinterpret_cast<float *>(sm + PrepSmem::BETA);
@@ -331,6 +332,7 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
     // for their writes to complete once the next item's first product has
     // been issued, by which time they have long landed.
     uint32_t *pending = nullptr;
+    uint32_t sec_round = 0;   // phases of B[5] (secondary-chunking products) so far
     // Items: each pipeline starts with its own, then takes the next free one
     // from a global counter (SMs do not run at the same speed, so a fixed
     // share would leave the slowest as the tail).  The leader draws the
@@ -384,7 +386,7 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         b.slow_flag = misc + 2;
 
         mbar_wait(&B[0], it & 1, abort_flag);
-        const bool slow = prep::gate<BAR>(b, pt, L);
+        const int form = prep::gate<BAR>(b, pt, L);
         fence_async_smem();
         named_barrier(BAR, prep::kGroupThreads);
         uint32_t drawn = 0;
@@ -409,12 +411,19 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         }
         mbar_wait(&B[1], it & 1, abort_flag);
         tc_fence_after();
-        if (!slow) {
+        if (form == prep::kProductForm) {
             prep::read_ap(b, tmem, quad, half, lane);
         } else {
             const size_t stride = (size_t)p.H * DK;
-            prep::pairwise(b, pt, L, p.k + ((size_t)tok0 * p.H + h) * DK,
-                           p.q + ((size_t)tok0 * p.H + h) * DK, stride);
+            const __nv_bfloat16 *kt0 = p.k + ((size_t)tok0 * p.H + h) * DK;
+            const __nv_bfloat16 *qt0 = p.q + ((size_t)tok0 * p.H + h) * DK;
+            if (form == prep::kSecondary) {
+                prep::secondary<BAR>(b, pt, L, kt0, qt0, stride, sm + PrepSmem::KHAT, sm + PrepSmem::GRAW,
+                                     sm + PrepSmem::XF, tmem, wp == 0, &B[5], sec_round, abort_flag);
+                prep::read_ap(b, tmem, quad, half, lane);
+            } else {
+                prep::pairwise(b, pt, L, kt0, qt0, stride);
+            }
         }
         tc_fence_before();
         named_barrier(BAR, prep::kGroupThreads);
@@ -526,7 +535,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     if (tid == 0 || tid == kPipeThreads) {
         uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);
         mbar_init(&B[0], 3);   // the leader, and one arrive per beta warp
-        for (int i = 1; i < 5; ++i) mbar_init(&B[i], 1);
+        for (int i = 1; i < 6; ++i) mbar_init(&B[i], 1);
         reinterpret_cast<uint32_t *>(sm + PrepSmem::MISC)[1] = 0u;
         fence_mbar_init();
     }

@@ -192,8 +192,21 @@ def _stress(kind, T=256, H=2):
         inp["q"] = inp["k"].clone()
     elif kind == "decay_near_limit":  # a chunk decays by e^-76.8: still the product form
         inp["log_alpha"] = torch.full_like(g, -1.2)
-    elif kind == "decay_past_limit":  # e^-83.2 per chunk: the pairwise path
+    elif kind == "decay_past_limit":  # e^-83.2 per chunk: one reference per 16-token block
         inp["log_alpha"] = torch.full_like(g, -1.3)
+    elif kind == "decay_blocks":      # e^-48 per 16-token block, e^-192 per chunk
+        inp["log_alpha"] = torch.full_like(g, -3.0)
+    elif kind == "decay_past_block":  # e^-96 within a 16-token block: the pairwise path
+        inp["log_alpha"] = torch.full_like(g, -6.0)
+    elif kind == "decay_spikes":      # a -60 spike every 16 tokens on half the channels
+        g2 = g.clone()
+        g2[::16, :, 1::2] = -60.0
+        inp["log_alpha"] = g2
+    elif kind == "spikes_in_block":   # two -50 spikes in one block on a few channels
+        g2 = g.clone()
+        g2[3::64, :, :8] = -50.0
+        g2[9::64, :, :8] = -50.0
+        inp["log_alpha"] = g2
     elif kind == "mixed_extremes":    # half the channels keep, half forget fast
         g2 = g.clone()
         g2[..., ::2] = 0.0
@@ -204,7 +217,8 @@ def _stress(kind, T=256, H=2):
 
 @pytest.mark.parametrize("kind", ["alpha_half", "gate_floor", "alpha_one", "alpha_zero",
                                   "beta_zero", "beta_one_qk", "mixed_extremes",
-                                  "decay_near_limit", "decay_past_limit"])
+                                  "decay_near_limit", "decay_past_limit", "decay_blocks",
+                                  "decay_past_block", "decay_spikes", "spikes_in_block"])
 def test_prefill_stress(kind):
     inp = _stress(kind)
     o, fs = gpu_prefill(inp)
