@@ -106,7 +106,12 @@ struct ChainCfg {
     static constexpr int NCW = 4 * (DVT / 32);
     static constexpr int THREADS = 32 * (NCW + 2);
     static constexpr int NSA = DVT == 128 ? 2 : 3;
-    static constexpr int NSB = DVT == 32 ? 2 : 1;
+    static constexpr int NSB = DVT == 64 ? 1 : 2;
+    // Copies of the bf16 state: two let the chain warps write S_{n+1} while
+    // chunk n's output products still read S_n; whole-d_v CTAs keep one (and
+    // a second ring-B stage in its place), the chain warps waiting for those
+    // products first.
+    static constexpr int NSBC = DVT == 128 ? 1 : 2;
     static constexpr uint32_t V_BYTES = (uint32_t)DVT * C * 2;
     static constexpr uint32_t A_MP = 0, A_YT = 32768, A_V = 49152;
     static constexpr uint32_t A_STRIDE = align1k(A_V + V_BYTES);
@@ -116,7 +121,7 @@ struct ChainCfg {
     static constexpr uint32_t RA = 0;
     static constexpr uint32_t RB = NSA * A_STRIDE;
     static constexpr uint32_t SB = RB + NSB * B_STRIDE;
-    static constexpr uint32_t EGLR = SB + 2 * SB_BYTES;     // NSA x exp(G_L), 128 fp32 each
+    static constexpr uint32_t EGLR = SB + NSBC * SB_BYTES;  // NSA x exp(G_L), 128 fp32 each
     static constexpr uint32_t BARS = EGLR + NSA * 512;
     static constexpr uint32_t MISC = BARS + 128;
     static constexpr uint32_t SIZE = MISC + 64;
@@ -520,12 +525,6 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
 __global__ void __launch_bounds__(kPrepThreads, 1)
 kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_g, const Params p) {
-    // Let a dependent chain kernel start now: it waits on per-record flags,
-    // not on this grid's completion.
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const uint32_t total_items = *p.total_chunks * (uint32_t)p.H;
-    if (2 * blockIdx.x >= total_items) return;
-
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *sm0 = dyn_smem + ((1024u - (smem_addr(dyn_smem) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -543,12 +542,26 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         tmem_alloc(&misc0[0], kPrepTmemCols);
         tmem_relinquish();
     }
+    if (tid == 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_g);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // The set-up above overlaps the plan kernel (this grid is its
+    // programmatic dependent); its output is read only past this wait.
+    // Then a dependent chain kernel may start: it waits on per-record flags,
+    // not on this grid's completion.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const uint32_t total_items = *p.total_chunks * (uint32_t)p.H;
     const uint32_t tmem = misc0[0] + 256u * P;
-    if (P == 0) prep_pipeline<0>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
-    else prep_pipeline<1>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
+    if (2 * blockIdx.x < total_items) {
+        if (P == 0) prep_pipeline<0>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
+        else prep_pipeline<1>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -712,7 +725,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             const uint32_t aM = smem_addr(slot_a + Cfg::A_MP);
             const uint32_t aY = smem_addr(slot_a + Cfg::A_YT);
             const uint32_t bV = smem_addr(slot_a + Cfg::A_V);
-            const uint32_t bS = smem_addr(sm + Cfg::SB + (n & 1) * Cfg::SB_BYTES);
+            const uint32_t bS = smem_addr(sm + Cfg::SB + (Cfg::NSBC == 2 ? (n & 1) : 0) * Cfg::SB_BYTES);
             mbar_wait(SREADY, n & 1, abort_flag);
             mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
             tc_fence_after();
@@ -773,7 +786,11 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + col0), S);
                 tmem_wait_ld();
             }
-            store_sb_row<DVT>(sm + Cfg::SB + (n & 1) * Cfg::SB_BYTES, crow, col0, S);
+            if (Cfg::NSBC == 1 && n >= 1) {   // chunk n-1's output products have read S_{n-1}
+                mbar_wait(&ODONE[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
+                tc_fence_after();
+            }
+            store_sb_row<DVT>(sm + Cfg::SB + (Cfg::NSBC == 2 ? (n & 1) : 0) * Cfg::SB_BYTES, crow, col0, S);
             mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
             const float d = reinterpret_cast<const float *>(sm + Cfg::EGLR + sa * 512)[crow];
 #pragma unroll
@@ -835,6 +852,9 @@ __global__ void __launch_bounds__(kPlanThreads)
 kda_split_plan_kernel(const int32_t *cu, int n, int64_t total, int32_t *perm, int32_t *chunk_off,
                       int2 *chunk_tab, uint32_t *total_chunks, uint32_t *err,
                       uint32_t *rec_ready, size_t n_flags, uint32_t *work_next) {
+    // The prep grid may start its set-up now; it reads nothing of this
+    // grid's output before this grid has completed.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (size_t i = threadIdx.x; i < n_flags; i += kPlanThreads) rec_ready[i] = 0u;
     if (threadIdx.x == 0) *work_next = 0u;
     __shared__ int32_t warp_sums[kPlanThreads / 32];
@@ -1130,9 +1150,22 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     const size_t max_items = l.max_chunks * (size_t)H;
     size_t prep_blocks = (size_t)(overlap ? sm_count - chain_blocks : sm_count);
     if (2 * prep_blocks > max_items) prep_blocks = (max_items + 1) / 2;
-    kda_prep_kernel<<<(unsigned)prep_blocks, kPrepThreads, PrepSmem::ALLOC, stream>>>(mk, mq, mg, prm);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    {   // a programmatic dependent of the plan kernel: its set-up overlaps it
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)prep_blocks);
+        cfg.blockDim = dim3(kPrepThreads);
+        cfg.dynamicSmemBytes = PrepSmem::ALLOC;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kda_prep_kernel, mk, mq, mg, prm);
+        if (e != cudaSuccess) return e;
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     return plan.dvt == 32 ? launch_chain<32>(v, total_tokens, H, prm, units, overlap, stream)
                           : launch_chain<128>(v, total_tokens, H, prm, units, overlap, stream);
 }
