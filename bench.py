@@ -8,7 +8,9 @@ A step is one kda_prefill call over the prefill workload's batch (all chunks,
 all heads, final state written).  Inputs are resident in HBM when timing
 starts; L2 is flushed (a 256 MiB write) before every timed step, outside the
 timed interval.  The decode figures time chained kda_decode_step calls on the
-decode workload (state 512 MiB, larger than L2, so no flush is needed).
+decode workload (state 512 MiB, larger than L2, so no flush is needed).  The
+"gdn_prefill" object times gdn_prefill (Gated DeltaNet: one gate value per
+token and head) on the prefill workload the same way.
 Under torchrun every rank runs the same workload as an independent replica
 (the operator needs no exchange between GPUs); value = all ranks' tokens over
 the slowest rank's time.
@@ -40,12 +42,16 @@ DECODE_STEPS = 1000
 CHUNK = 64
 
 
-def prefill_work(w, lengths):
+def prefill_work(w, lengths, scalar_gate=False):
+    """Algorithmic work of one prefill call; with ``scalar_gate`` (Gated
+    DeltaNet) log_alpha is one value per (token, head) instead of d_k."""
     T = sum(lengths)
     n = len(lengths)
     eb = 2 if w.dtype == "bf16" else 4
     per_tok_flop = 6 * w.d_k * w.d_v + CHUNK * (3 * w.d_k + 2 * w.d_v)
     per_tok_bytes = (3 * w.d_k + 2 * w.d_v) * eb + eb
+    if scalar_gate:
+        per_tok_bytes -= (w.d_k - 1) * eb
     state_bytes = n * w.H * w.d_k * w.d_v * 4 * (2 if w.init_std > 0 else 1)
     return dict(tokens=T, flop=per_tok_flop * T * w.H,
                 bytes=per_tok_bytes * T * w.H + state_bytes)
@@ -162,12 +168,18 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # --- the GPU arm -------------------------------------------------------------------
 
-def time_prefill(w, steps, warmup, world):
+def time_prefill(w, steps, warmup, world, scalar_gate=False):
+    """kda_prefill (or, with ``scalar_gate``, gdn_prefill with channel 0 of
+    the gate draw as the per-head gate) on the workload, L2 flushed."""
     import torch
     from gated_delta_rule_69_b200 import inputs as kin
     from gated_delta_rule_69_b200 import kda
     inp = kin.generate(w, device="cuda")
     q, k, v, g, b = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta"))
+    fn = kda.kda_prefill
+    if scalar_gate:
+        g = g[..., 0].contiguous()
+        fn = kda.gdn_prefill
     T, H, dk = q.shape
     dv = v.shape[-1]
     n = len(inp["lengths"])
@@ -179,8 +191,8 @@ def time_prefill(w, steps, warmup, world):
     stream = torch.cuda.current_stream()
 
     def step():
-        kda.kda_prefill(q, k, v, g, b, init_state=inp["init_state"], cu_seqlens=inp["cu_seqlens"],
-                        o=o, final_state=fs, workspace=ws, stream=stream)
+        fn(q, k, v, g, b, init_state=inp["init_state"], cu_seqlens=inp["cu_seqlens"],
+           o=o, final_state=fs, workspace=ws, stream=stream)
 
     for _ in range(warmup):
         flush.fill_(1)
@@ -398,6 +410,7 @@ def main():
     pf = time_prefill(w, args.steps, args.warmup, world)
     dw = kin.WORKLOADS[args.decode_workload]
     dec = time_decode(dw, args.decode_steps, args.warmup, world)
+    gdn = time_prefill(w, args.steps, args.warmup, world, scalar_gate=True)
     clocks = sampler.stop()
 
     lengths = pf["inputs"]["lengths"]
@@ -409,6 +422,9 @@ def main():
     dwork = decode_work(dw)
     dms = max_over_ranks(dec["ms_total"] / args.decode_steps, world)
     dgbs = dwork["bytes"] / (dms * 1e-3) / 1e9
+    gwork = prefill_work(w, lengths, scalar_gate=True)
+    gms = max_over_ranks(gdn["ms_total"] / args.steps, world)
+    ggbs = gwork["bytes"] / (gms * 1e-3) / 1e9
     src = "of " + peaks["source"]
 
     line = {
@@ -428,7 +444,14 @@ def main():
                                 "unit": "GB/s", "frac": dgbs / peaks["hbm"], "traffic": None,
                                 "peak_source": src, "kernel": "kda_decode_step",
                                 "algorithmic_bytes_per_launch": dwork["bytes"]}},
-        "gpu_launches": pf["launches"] + dec["launches"],
+        "gdn_prefill": {"workload": w.name + " with one gate value per (token, head)",
+                        "value": world * gwork["tokens"] / (gms * 1e-3), "unit": "tokens/s",
+                        "ms_per_step": gms, "steps": args.steps,
+                        "roofline": {"bound": "hbm", "achieved": ggbs, "peak": peaks["hbm"],
+                                     "unit": "GB/s", "frac": ggbs / peaks["hbm"], "traffic": None,
+                                     "peak_source": src, "kernel": "gdn_prefill",
+                                     "algorithmic_bytes_per_launch": gwork["bytes"]}},
+        "gpu_launches": pf["launches"] + dec["launches"] + gdn["launches"],
         "clocks": clocks,
     }
     if not args.no_e2e:

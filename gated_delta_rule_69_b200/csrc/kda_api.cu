@@ -31,6 +31,98 @@ bool use_tensor_cores(kda_dtype dtype, int d_k, int d_v, int64_t total_tokens) {
            total_tokens <= INT_MAX;
 }
 
+// The prefill and the decode step for either gate: one log_alpha per key
+// channel (KDA) or one per head (Gated DeltaNet).
+kda_status prefill_impl(const void *q, const void *k, const void *v,
+                        const void *log_alpha, const void *beta,
+                        const float *init_state, const int32_t *cu_seqlens,
+                        int32_t num_seqs, int64_t total_tokens, int32_t H,
+                        int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                        float *final_state, void *workspace,
+                        size_t workspace_bytes, kda_stream_t stream_, bool scalar_gate) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (num_seqs < 1 || total_tokens < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_BF16 && dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(d_k) || !supported_dim(d_v)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)num_seqs * H > INT_MAX) return KDA_ERR_UNSUPPORTED;
+    if (!cu_seqlens && total_tokens % num_seqs != 0) return KDA_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !o))
+        return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, scalar_gate ? nullptr : log_alpha, init_state, o, final_state};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (beta && !aligned_to(beta, elem_bytes(dtype))) return KDA_ERR_INVALID_ARG;
+    if (scalar_gate && log_alpha && !aligned_to(log_alpha, elem_bytes(dtype))) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
+    // The least workspace any path accepts; the two-kernel tensor-core path is
+    // taken when the workspace also holds its per-chunk records.
+    const size_t need = kda::prefill_tc_workspace(num_seqs);
+    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_INVALID_ARG;
+
+    const size_t eb = elem_bytes(dtype);
+    const size_t nk = (size_t)total_tokens * H * d_k * eb;
+    const size_t nv = (size_t)total_tokens * H * d_v * eb;
+    const size_t nb = (size_t)total_tokens * H * eb;
+    const size_t ng = scalar_gate ? nb : nk;
+    const size_t ns = (size_t)num_seqs * H * d_k * d_v * sizeof(float);
+    if (overlaps(o, nv, q, nk) || overlaps(o, nv, k, nk) || overlaps(o, nv, v, nv) ||
+        overlaps(o, nv, log_alpha, ng) || overlaps(o, nv, beta, nb) ||
+        overlaps(o, nv, init_state, ns) || overlaps(o, nv, final_state, ns) ||
+        overlaps(o, nv, workspace, workspace_bytes))
+        return KDA_ERR_INVALID_ARG;
+    if (init_state && final_state && init_state != final_state &&
+        overlaps(init_state, ns, final_state, ns))
+        return KDA_ERR_INVALID_ARG;
+
+    if (use_tensor_cores(dtype, d_k, d_v, total_tokens) &&
+        workspace_bytes >= kda::prefill_split_workspace(num_seqs, total_tokens, H))
+        return from_cuda(kda::launch_prefill_split(q, k, v, log_alpha, beta, init_state,
+                                                   cu_seqlens, num_seqs, total_tokens, H, o,
+                                                   final_state, workspace, scalar_gate, stream));
+    if (use_tensor_cores(dtype, d_k, d_v, total_tokens))
+        return from_cuda(kda::launch_prefill_tc(q, k, v, log_alpha, beta, init_state, cu_seqlens,
+                                                num_seqs, total_tokens, H, o, final_state,
+                                                workspace, scalar_gate, stream));
+    uint32_t *err_word = static_cast<uint32_t *>(workspace);
+    cudaError_t e = cudaMemsetAsync(err_word, 0, sizeof(uint32_t), stream);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    e = kda::launch_prefill_simt(q, k, v, log_alpha, beta, init_state, cu_seqlens,
+                                 num_seqs, total_tokens, H, d_k, d_v, dtype, o,
+                                 final_state, err_word, scalar_gate, stream);
+    return from_cuda(e);
+}
+
+kda_status decode_impl(const void *q, const void *k, const void *v,
+                       const void *log_alpha, const void *beta,
+                       float *state, int32_t batch, int32_t H,
+                       int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                       kda_stream_t stream_, bool scalar_gate) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (batch < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_BF16 && dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(d_k) || !supported_dim(d_v)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)batch * H > INT_MAX) return KDA_ERR_UNSUPPORTED;
+    if (batch == 0) return KDA_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_INVALID_ARG;
+    const size_t eb = elem_bytes(dtype);
+    const void *ptrs[] = {q, k, v, log_alpha, beta, o};
+    for (const void *p : ptrs)
+        if (!aligned_to(p, eb)) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(state)) return KDA_ERR_INVALID_ARG;
+    const size_t nk = (size_t)batch * H * d_k * eb;
+    const size_t nv = (size_t)batch * H * d_v * eb;
+    const size_t nb = (size_t)batch * H * eb;
+    const size_t ng = scalar_gate ? nb : nk;
+    const size_t ns = (size_t)batch * H * d_k * d_v * sizeof(float);
+    if (overlaps(o, nv, q, nk) || overlaps(o, nv, k, nk) || overlaps(o, nv, v, nv) ||
+        overlaps(o, nv, log_alpha, ng) || overlaps(o, nv, beta, nb) ||
+        overlaps(o, nv, state, ns))
+        return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_decode(q, k, v, log_alpha, beta, state, batch, H,
+                                        d_k, d_v, dtype, o, scalar_gate, stream));
+}
+
 }  // namespace
 
 extern "C" {
@@ -63,85 +155,40 @@ kda_status kda_prefill(const void *q, const void *k, const void *v,
                        int32_t num_seqs, int64_t total_tokens, int32_t H,
                        int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
                        float *final_state, void *workspace,
-                       size_t workspace_bytes, kda_stream_t stream_) {
-    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    if (num_seqs < 1 || total_tokens < 0 || H < 1) return KDA_ERR_INVALID_ARG;
-    if (dtype != KDA_BF16 && dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
-    if (!supported_dim(d_k) || !supported_dim(d_v)) return KDA_ERR_UNSUPPORTED;
-    if ((int64_t)num_seqs * H > INT_MAX) return KDA_ERR_UNSUPPORTED;
-    if (!cu_seqlens && total_tokens % num_seqs != 0) return KDA_ERR_INVALID_ARG;
-    if (total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !o))
-        return KDA_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, k, v, log_alpha, init_state, o, final_state};
-    for (const void *p : ptrs)
-        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
-    if (beta && !aligned_to(beta, elem_bytes(dtype))) return KDA_ERR_INVALID_ARG;
-    if (cu_seqlens && !aligned_to(cu_seqlens, 4)) return KDA_ERR_INVALID_ARG;
-    // The least workspace any path accepts; the two-kernel tensor-core path is
-    // taken when the workspace also holds its per-chunk records.
-    const size_t need = kda::prefill_tc_workspace(num_seqs);
-    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_INVALID_ARG;
+                       size_t workspace_bytes, kda_stream_t stream) {
+    return prefill_impl(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, total_tokens,
+                        H, d_k, d_v, dtype, o, final_state, workspace, workspace_bytes, stream,
+                        false);
+}
 
-    const size_t eb = elem_bytes(dtype);
-    const size_t nk = (size_t)total_tokens * H * d_k * eb;
-    const size_t nv = (size_t)total_tokens * H * d_v * eb;
-    const size_t nb = (size_t)total_tokens * H * eb;
-    const size_t ns = (size_t)num_seqs * H * d_k * d_v * sizeof(float);
-    if (overlaps(o, nv, q, nk) || overlaps(o, nv, k, nk) || overlaps(o, nv, v, nv) ||
-        overlaps(o, nv, log_alpha, nk) || overlaps(o, nv, beta, nb) ||
-        overlaps(o, nv, init_state, ns) || overlaps(o, nv, final_state, ns) ||
-        overlaps(o, nv, workspace, workspace_bytes))
-        return KDA_ERR_INVALID_ARG;
-    if (init_state && final_state && init_state != final_state &&
-        overlaps(init_state, ns, final_state, ns))
-        return KDA_ERR_INVALID_ARG;
-
-    if (use_tensor_cores(dtype, d_k, d_v, total_tokens) &&
-        workspace_bytes >= kda::prefill_split_workspace(num_seqs, total_tokens, H))
-        return from_cuda(kda::launch_prefill_split(q, k, v, log_alpha, beta, init_state,
-                                                   cu_seqlens, num_seqs, total_tokens, H, o,
-                                                   final_state, workspace, stream));
-    if (use_tensor_cores(dtype, d_k, d_v, total_tokens))
-        return from_cuda(kda::launch_prefill_tc(q, k, v, log_alpha, beta, init_state, cu_seqlens,
-                                                num_seqs, total_tokens, H, o, final_state,
-                                                workspace, stream));
-    uint32_t *err_word = static_cast<uint32_t *>(workspace);
-    cudaError_t e = cudaMemsetAsync(err_word, 0, sizeof(uint32_t), stream);
-    if (e != cudaSuccess) return KDA_ERR_CUDA;
-    e = kda::launch_prefill_simt(q, k, v, log_alpha, beta, init_state, cu_seqlens,
-                                 num_seqs, total_tokens, H, d_k, d_v, dtype, o,
-                                 final_state, err_word, stream);
-    return from_cuda(e);
+kda_status gdn_prefill(const void *q, const void *k, const void *v,
+                       const void *log_alpha, const void *beta,
+                       const float *init_state, const int32_t *cu_seqlens,
+                       int32_t num_seqs, int64_t total_tokens, int32_t H,
+                       int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                       float *final_state, void *workspace,
+                       size_t workspace_bytes, kda_stream_t stream) {
+    return prefill_impl(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, total_tokens,
+                        H, d_k, d_v, dtype, o, final_state, workspace, workspace_bytes, stream,
+                        true);
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            const void *log_alpha, const void *beta,
                            float *state, int32_t batch, int32_t H,
                            int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
-                           kda_stream_t stream_) {
-    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    if (batch < 0 || H < 1) return KDA_ERR_INVALID_ARG;
-    if (dtype != KDA_BF16 && dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
-    if (!supported_dim(d_k) || !supported_dim(d_v)) return KDA_ERR_UNSUPPORTED;
-    if ((int64_t)batch * H > INT_MAX) return KDA_ERR_UNSUPPORTED;
-    if (batch == 0) return KDA_OK;
-    if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_INVALID_ARG;
-    const size_t eb = elem_bytes(dtype);
-    const void *ptrs[] = {q, k, v, log_alpha, beta, o};
-    for (const void *p : ptrs)
-        if (!aligned_to(p, eb)) return KDA_ERR_INVALID_ARG;
-    if (!aligned16(state)) return KDA_ERR_INVALID_ARG;
-    const size_t nk = (size_t)batch * H * d_k * eb;
-    const size_t nv = (size_t)batch * H * d_v * eb;
-    const size_t nb = (size_t)batch * H * eb;
-    const size_t ns = (size_t)batch * H * d_k * d_v * sizeof(float);
-    if (overlaps(o, nv, q, nk) || overlaps(o, nv, k, nk) || overlaps(o, nv, v, nv) ||
-        overlaps(o, nv, log_alpha, nk) || overlaps(o, nv, beta, nb) ||
-        overlaps(o, nv, state, ns))
-        return KDA_ERR_INVALID_ARG;
-    return from_cuda(kda::launch_decode(q, k, v, log_alpha, beta, state, batch, H,
-                                        d_k, d_v, dtype, o, stream));
+                           kda_stream_t stream) {
+    return decode_impl(q, k, v, log_alpha, beta, state, batch, H, d_k, d_v, dtype, o, stream,
+                       false);
+}
+
+kda_status gdn_decode_step(const void *q, const void *k, const void *v,
+                           const void *log_alpha, const void *beta,
+                           float *state, int32_t batch, int32_t H,
+                           int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                           kda_stream_t stream) {
+    return decode_impl(q, k, v, log_alpha, beta, state, batch, H, d_k, d_v, dtype, o, stream,
+                       true);
 }
 
 kda_status kda_check_workspace_error(const void *workspace, kda_stream_t stream_) {

@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
 kda_decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
                   const T *__restrict__ v, const T *__restrict__ g,
                   const T *__restrict__ beta, float *__restrict__ state,
-                  T *__restrict__ o) {
+                  T *__restrict__ o, int g_bh, int g_c) {
     using Sh = DecodeShape<DK, DV>;
     constexpr int LX = Sh::LX, NT = Sh::NT, R = Sh::R, RPT = Sh::RPT;
     __shared__ float sk[DK], sq[DK], sa[DK], sv[DV], su[DV];
@@ -64,7 +64,7 @@ kda_decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
     for (int i = tid; i < DK; i += NT) {
         sk[i] = io<T>::load(k + bh * DK + i);
         sq[i] = io<T>::load(q + bh * DK + i);
-        sa[i] = expf(io<T>::load(g + bh * DK + i));
+        sa[i] = expf(io<T>::load(g + bh * g_bh + i * g_c));
     }
     for (int i = tid; i < DV; i += NT) sv[i] = io<T>::load(v + bh * DV + i);
     __syncthreads();
@@ -117,24 +117,24 @@ kda_decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
 template <typename T, int DK, int DV>
 cudaError_t launch_typed(const void *q, const void *k, const void *v,
                          const void *g, const void *beta, float *state,
-                         int batch, int H, void *o, cudaStream_t stream) {
+                         int batch, int H, void *o, bool sg, cudaStream_t stream) {
     const unsigned blocks = (unsigned)((size_t)batch * (size_t)H);
     kda_decode_kernel<T, DK, DV><<<blocks, DecodeShape<DK, DV>::NT, 0, stream>>>(
         static_cast<const T *>(q), static_cast<const T *>(k),
         static_cast<const T *>(v), static_cast<const T *>(g),
-        static_cast<const T *>(beta), state, static_cast<T *>(o));
+        static_cast<const T *>(beta), state, static_cast<T *>(o), sg ? 1 : DK, sg ? 0 : 1);
     return cudaGetLastError();
 }
 
 template <typename T, int DK>
 cudaError_t dispatch_dv(int dv, const void *q, const void *k, const void *v,
                         const void *g, const void *beta, float *state,
-                        int batch, int H, void *o, cudaStream_t stream) {
+                        int batch, int H, void *o, bool sg, cudaStream_t stream) {
     switch (dv) {
-        case 16: return launch_typed<T, DK, 16>(q, k, v, g, beta, state, batch, H, o, stream);
-        case 32: return launch_typed<T, DK, 32>(q, k, v, g, beta, state, batch, H, o, stream);
-        case 64: return launch_typed<T, DK, 64>(q, k, v, g, beta, state, batch, H, o, stream);
-        case 128: return launch_typed<T, DK, 128>(q, k, v, g, beta, state, batch, H, o, stream);
+        case 16: return launch_typed<T, DK, 16>(q, k, v, g, beta, state, batch, H, o, sg, stream);
+        case 32: return launch_typed<T, DK, 32>(q, k, v, g, beta, state, batch, H, o, sg, stream);
+        case 64: return launch_typed<T, DK, 64>(q, k, v, g, beta, state, batch, H, o, sg, stream);
+        case 128: return launch_typed<T, DK, 128>(q, k, v, g, beta, state, batch, H, o, sg, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -142,13 +142,13 @@ cudaError_t dispatch_dv(int dv, const void *q, const void *k, const void *v,
 template <typename T>
 cudaError_t dispatch_dk(int dk, int dv, const void *q, const void *k,
                         const void *v, const void *g, const void *beta,
-                        float *state, int batch, int H, void *o,
+                        float *state, int batch, int H, void *o, bool sg,
                         cudaStream_t stream) {
     switch (dk) {
-        case 16: return dispatch_dv<T, 16>(dv, q, k, v, g, beta, state, batch, H, o, stream);
-        case 32: return dispatch_dv<T, 32>(dv, q, k, v, g, beta, state, batch, H, o, stream);
-        case 64: return dispatch_dv<T, 64>(dv, q, k, v, g, beta, state, batch, H, o, stream);
-        case 128: return dispatch_dv<T, 128>(dv, q, k, v, g, beta, state, batch, H, o, stream);
+        case 16: return dispatch_dv<T, 16>(dv, q, k, v, g, beta, state, batch, H, o, sg, stream);
+        case 32: return dispatch_dv<T, 32>(dv, q, k, v, g, beta, state, batch, H, o, sg, stream);
+        case 64: return dispatch_dv<T, 64>(dv, q, k, v, g, beta, state, batch, H, o, sg, stream);
+        case 128: return dispatch_dv<T, 128>(dv, q, k, v, g, beta, state, batch, H, o, sg, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -158,10 +158,11 @@ cudaError_t dispatch_dk(int dk, int dv, const void *q, const void *k,
 cudaError_t launch_decode(const void *q, const void *k, const void *v,
                           const void *g, const void *beta, float *state,
                           int batch, int H, int dk, int dv, kda_dtype dtype,
-                          void *o, cudaStream_t stream) {
+                          void *o, bool scalar_gate, cudaStream_t stream) {
     if (dtype == KDA_BF16)
-        return dispatch_dk<__nv_bfloat16>(dk, dv, q, k, v, g, beta, state, batch, H, o, stream);
-    return dispatch_dk<float>(dk, dv, q, k, v, g, beta, state, batch, H, o, stream);
+        return dispatch_dk<__nv_bfloat16>(dk, dv, q, k, v, g, beta, state, batch, H, o, scalar_gate,
+                                          stream);
+    return dispatch_dk<float>(dk, dv, q, k, v, g, beta, state, batch, H, o, scalar_gate, stream);
 }
 
 }  // namespace kda

@@ -48,17 +48,19 @@ enum : uint32_t {
 constexpr size_t kWorkspaceHeader = 256;
 
 // Launchers (defined in the .cu files).  All return cudaGetLastError().
+// `scalar_gate`: log_alpha holds one value per (token, head) ([T, H], the
+// Gated DeltaNet gate) instead of one per key channel ([T, H, d_k]).
 cudaError_t launch_decode(const void *q, const void *k, const void *v,
                           const void *g, const void *beta, float *state,
                           int batch, int H, int dk, int dv, kda_dtype dtype,
-                          void *o, cudaStream_t stream);
+                          void *o, bool scalar_gate, cudaStream_t stream);
 
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
                                 const void *g, const void *beta,
                                 const float *init_state, const int32_t *cu,
                                 int num_seqs, int64_t total_tokens, int H,
                                 int dk, int dv, kda_dtype dtype, void *o,
-                                float *final_state, uint32_t *err_word,
+                                float *final_state, uint32_t *err_word, bool scalar_gate,
                                 cudaStream_t stream);
 
 // Tensor-core prefill (bf16, d_k = d_v = 128).
@@ -67,7 +69,8 @@ size_t prefill_tc_workspace(int num_seqs);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const void *g,
                               const void *beta, const float *init_state, const int32_t *cu,
                               int num_seqs, int64_t total_tokens, int H, void *o,
-                              float *final_state, void *workspace, cudaStream_t stream);
+                              float *final_state, void *workspace, bool scalar_gate,
+                              cudaStream_t stream);
 
 // Tensor-core prefill split into a chunk-parallel preparation kernel and a
 // state-chain kernel; its workspace holds one record per (chunk, head).
@@ -76,6 +79,7 @@ size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H);
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const void *g,
                                  const void *beta, const float *init_state, const int32_t *cu,
                                  int num_seqs, int64_t total_tokens, int H, void *o,
-                                 float *final_state, void *workspace, cudaStream_t stream);
+                                 float *final_state, void *workspace, bool scalar_gate,
+                                 cudaStream_t stream);
 
 }  // namespace kda

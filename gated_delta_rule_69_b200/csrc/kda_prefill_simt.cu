@@ -56,7 +56,7 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
                         const float *init_state, const int32_t *__restrict__ cu,
                         int num_seqs, int64_t total_tokens, int H,
                         T *__restrict__ o, float *final_state,
-                        uint32_t *err_word) {
+                        uint32_t *err_word, int scalar_gate) {
     using L = SimtSmem<DK, DV>;
     constexpr int KP = L::KP, AP = L::AP;
     extern __shared__ __align__(16) float sm[];
@@ -97,7 +97,8 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
             const size_t gi = ((size_t)(cs + t) * H + h) * DK + c;
             Ks[t * KP + c] = io<T>::load(k + gi);
             Qs[t * KP + c] = io<T>::load(q + gi);
-            Gs[t * KP + c] = clamp_log_alpha(io<T>::load(g + gi));
+            const size_t gg = scalar_gate ? (size_t)(cs + t) * H + h : gi;
+            Gs[t * KP + c] = clamp_log_alpha(io<T>::load(g + gg));
         }
         for (int idx = tid; idx < Lc * DV; idx += kThreads) {
             const int t = idx / DV, j = idx % DV;
@@ -201,7 +202,7 @@ template <typename T, int DK, int DV>
 cudaError_t launch_typed(const void *q, const void *k, const void *v,
                          const void *g, const void *beta, const float *init,
                          const int32_t *cu, int n, int64_t T_tot, int H,
-                         void *o, float *fin, uint32_t *err, cudaStream_t st) {
+                         void *o, float *fin, uint32_t *err, bool sg, cudaStream_t st) {
     constexpr size_t smem = SimtSmem<DK, DV>::bytes;
     auto kern = kda_prefill_simt_kernel<T, DK, DV>;
     cudaError_t e = cudaFuncSetAttribute(
@@ -212,7 +213,7 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v,
         static_cast<const T *>(q), static_cast<const T *>(k),
         static_cast<const T *>(v), static_cast<const T *>(g),
         static_cast<const T *>(beta), init, cu, n, T_tot, H,
-        static_cast<T *>(o), fin, err);
+        static_cast<T *>(o), fin, err, sg ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -220,12 +221,12 @@ template <typename T, int DK>
 cudaError_t dispatch_dv(int dv, const void *q, const void *k, const void *v,
                         const void *g, const void *beta, const float *init,
                         const int32_t *cu, int n, int64_t T_tot, int H,
-                        void *o, float *fin, uint32_t *err, cudaStream_t st) {
+                        void *o, float *fin, uint32_t *err, bool sg, cudaStream_t st) {
     switch (dv) {
-        case 16: return launch_typed<T, DK, 16>(q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, st);
-        case 32: return launch_typed<T, DK, 32>(q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, st);
-        case 64: return launch_typed<T, DK, 64>(q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, st);
-        case 128: return launch_typed<T, DK, 128>(q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, st);
+        case 16: return launch_typed<T, DK, 16>(q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, sg, st);
+        case 32: return launch_typed<T, DK, 32>(q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, sg, st);
+        case 64: return launch_typed<T, DK, 64>(q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, sg, st);
+        case 128: return launch_typed<T, DK, 128>(q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, sg, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -235,12 +236,12 @@ cudaError_t dispatch_dk(int dk, int dv, const void *q, const void *k,
                         const void *v, const void *g, const void *beta,
                         const float *init, const int32_t *cu, int n,
                         int64_t T_tot, int H, void *o, float *fin,
-                        uint32_t *err, cudaStream_t st) {
+                        uint32_t *err, bool sg, cudaStream_t st) {
     switch (dk) {
-        case 16: return dispatch_dv<T, 16>(dv, q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, st);
-        case 32: return dispatch_dv<T, 32>(dv, q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, st);
-        case 64: return dispatch_dv<T, 64>(dv, q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, st);
-        case 128: return dispatch_dv<T, 128>(dv, q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, st);
+        case 16: return dispatch_dv<T, 16>(dv, q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, sg, st);
+        case 32: return dispatch_dv<T, 32>(dv, q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, sg, st);
+        case 64: return dispatch_dv<T, 64>(dv, q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, sg, st);
+        case 128: return dispatch_dv<T, 128>(dv, q, k, v, g, beta, init, cu, n, T_tot, H, o, fin, err, sg, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -252,13 +253,14 @@ cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
                                 const float *init_state, const int32_t *cu,
                                 int num_seqs, int64_t total_tokens, int H,
                                 int dk, int dv, kda_dtype dtype, void *o,
-                                float *final_state, uint32_t *err_word,
+                                float *final_state, uint32_t *err_word, bool scalar_gate,
                                 cudaStream_t stream) {
     if (dtype == KDA_BF16)
         return dispatch_dk<__nv_bfloat16>(dk, dv, q, k, v, g, beta, init_state, cu, num_seqs,
-                                          total_tokens, H, o, final_state, err_word, stream);
+                                          total_tokens, H, o, final_state, err_word, scalar_gate,
+                                          stream);
     return dispatch_dk<float>(dk, dv, q, k, v, g, beta, init_state, cu, num_seqs,
-                              total_tokens, H, o, final_state, err_word, stream);
+                              total_tokens, H, o, final_state, err_word, scalar_gate, stream);
 }
 
 }  // namespace kda

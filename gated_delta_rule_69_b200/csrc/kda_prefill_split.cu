@@ -137,6 +137,8 @@ static_assert(Rec::YT == Rec::MP + 32768 && Rec::ZB == Rec::QP + 16384,
 
 struct Params {
     const __nv_bfloat16 *k, *q, *beta;
+    const __nv_bfloat16 *g;     // log_alpha [T, H] when scalar_gate
+    int scalar_gate;
     const float *init_state;
     float *final_state;
     __nv_bfloat16 *o;
@@ -359,18 +361,32 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         // the rest of the record may still be leaving shared memory, so the
         // leader's arrive, which lets the group write again, waits for that.
         if (leader) {
-            mbar_expect_tx(&B[0], kRawBytes);
+            mbar_expect_tx(&B[0], p.scalar_gate ? kRawBytes - 16384 : kRawBytes);
             const int t = (int)tok0;
             tma_load_3d(sm + PrepSmem::STK, &tm_k, &B[0], 0, h, t);
             tma_load_3d(sm + PrepSmem::STK + 16384, &tm_k, &B[0], 64, h, t);
             tma_load_3d(sm + PrepSmem::STK + 8192, &tm_q, &B[0], 0, h, t);
             tma_load_3d(sm + PrepSmem::STK + 16384 + 8192, &tm_q, &B[0], 64, h, t);
-            tma_load_3d(sm + PrepSmem::GRAW, &tm_g, &B[0], 0, h, t);
+            if (!p.scalar_gate) tma_load_3d(sm + PrepSmem::GRAW, &tm_g, &B[0], 0, h, t);
             bulk_wait_read_all();
             mbar_arrive(&B[0]);
         }
         if (pt < C) {
             beta[pt] = (pt < L) ? __bfloat162float(p.beta[(size_t)(tok0 + pt) * p.H + h]) : 0.f;
+            if (p.scalar_gate) {
+                // One log_alpha per token, broadcast over its 128 channels.  GRAW
+                // is a source of the previous record's stores: the leader has
+                // waited for every store to read its source before this
+                // barrier of the 64 threads that write it.
+                __nv_bfloat16 gv = __float2bfloat16(0.f);
+                if (pt < L) gv = p.g[(size_t)(tok0 + pt) * p.H + h];
+                named_barrier(BAR + 2, C);
+                const __nv_bfloat162 g2 = __halves2bfloat162(gv, gv);
+                const uint32_t gw = *reinterpret_cast<const uint32_t *>(&g2);
+                uint4 *row = reinterpret_cast<uint4 *>(sm + PrepSmem::GRAW + pt * 256);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) row[i] = make_uint4(gw, gw, gw, gw);
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&B[0]);
         }
@@ -1081,7 +1097,8 @@ size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H) {
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const void *g,
                                  const void *beta, const float *init_state, const int32_t *cu,
                                  int num_seqs, int64_t total_tokens, int H, void *o,
-                                 float *final_state, void *workspace, cudaStream_t stream) {
+                                 float *final_state, void *workspace, bool scalar_gate,
+                                 cudaStream_t stream) {
     using namespace split;
     const SplitLayout l = split_layout(num_seqs, total_tokens, H);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1095,7 +1112,8 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     CUtensorMap mk, mq, mg;
     if (!make_map_split(&mk, k, total_tokens, H, DK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_split(&mq, q, total_tokens, H, DK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_split(&mg, g, total_tokens, H, DK, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+        // with a scalar gate the map is never used (log_alpha comes in by plain loads)
+        !make_map_split(&mg, scalar_gate ? k : g, total_tokens, H, DK, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     // Prep runs as a persistent grid (one CTA per SM).  With overlap the prep
     // grid leaves the chain's SMs free and the chain kernel is launched as a
@@ -1132,6 +1150,8 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     prm.k = static_cast<const __nv_bfloat16 *>(k);
     prm.q = static_cast<const __nv_bfloat16 *>(q);
     prm.beta = static_cast<const __nv_bfloat16 *>(beta);
+    prm.g = static_cast<const __nv_bfloat16 *>(g);
+    prm.scalar_gate = scalar_gate ? 1 : 0;
     prm.init_state = init_state;
     prm.final_state = final_state;
     prm.o = static_cast<__nv_bfloat16 *>(o);

@@ -108,6 +108,8 @@ enum Bar : int {
 
 struct Params {
     const __nv_bfloat16 *k, *q, *beta;            // raw pointers for the pairwise path
+    const __nv_bfloat16 *g;                       // log_alpha [T, H] when scalar_gate
+    int scalar_gate;
     const float *init_state;
     float *final_state;
     __nv_bfloat16 *o;
@@ -622,15 +624,17 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                 }
                 stop = __shfl_sync(0xffffffffu, stop, 0);
                 if (stop) break;
+                __syncwarp();   // lane 0's wait for the free slot orders the warp's stores below
                 const int tok = (int)(bos + (int64_t)n * C);
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&B[RAW_FULL + s], kRawBytes);
+                    mbar_arrive_expect_tx(&B[RAW_FULL + s], p.scalar_gate ? kRawBytes - 16384 : kRawBytes);
                     uint8_t *stk = sm + Smem::STACK + s * 32768;
                     tma_load_3d(stk, &tm_k, &B[RAW_FULL + s], 0, h, tok);
                     tma_load_3d(stk + 16384, &tm_k, &B[RAW_FULL + s], 64, h, tok);
                     tma_load_3d(stk + 8192, &tm_q, &B[RAW_FULL + s], 0, h, tok);
                     tma_load_3d(stk + 16384 + 8192, &tm_q, &B[RAW_FULL + s], 64, h, tok);
-                    tma_load_3d(sm + Smem::GRAW + s * 16384, &tm_g, &B[RAW_FULL + s], 0, h, tok);
+                    if (!p.scalar_gate)
+                        tma_load_3d(sm + Smem::GRAW + s * 16384, &tm_g, &B[RAW_FULL + s], 0, h, tok);
                     tma_load_3d(sm + Smem::VT + s * 4096, &tm_v, &B[RAW_FULL + s], j0, h, tok);
                 }
                 const int64_t rem = len - (int64_t)n * C;
@@ -640,6 +644,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                     float b = 0.f;
                     if (t < rem) b = __bfloat162float(p.beta[(size_t)(tok + t) * p.H + h]);
                     betar[s * C + t] = b;
+                    if (p.scalar_gate) {   // one log_alpha per token: broadcast over its 128 channels
+                        __nv_bfloat16 gv = __float2bfloat16(0.f);
+                        if (t < rem) gv = p.g[(size_t)(tok + t) * p.H + h];
+                        const __nv_bfloat162 g2 = __halves2bfloat162(gv, gv);
+                        const uint32_t gw = *reinterpret_cast<const uint32_t *>(&g2);
+                        uint4 *row = reinterpret_cast<uint4 *>(sm + Smem::GRAW + s * 16384 + t * 256);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) row[i] = make_uint4(gw, gw, gw, gw);
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&B[RAW_FULL + s]);
@@ -920,7 +933,8 @@ size_t prefill_tc_workspace(int num_seqs) {
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const void *g,
                               const void *beta, const float *init_state, const int32_t *cu,
                               int num_seqs, int64_t total_tokens, int H, void *o,
-                              float *final_state, void *workspace, cudaStream_t stream) {
+                              float *final_state, void *workspace, bool scalar_gate,
+                              cudaStream_t stream) {
     using namespace tc;
     uint32_t *err = static_cast<uint32_t *>(workspace);
     int32_t *perm = cu ? reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) +
@@ -929,7 +943,8 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     CUtensorMap mk, mq, mg, mv;
     if (!make_map(&mk, k, total_tokens, H, DK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mq, q, total_tokens, H, DK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mg, g, total_tokens, H, DK, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        // with a scalar gate the map is never used (log_alpha comes in by plain loads)
+        !make_map(&mg, scalar_gate ? k : g, total_tokens, H, DK, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map(&mv, v, total_tokens, H, DV, DVT, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     kda_plan_kernel<<<1, kPlanThreads, 0, stream>>>(cu, num_seqs, total_tokens, perm, err);
@@ -946,6 +961,8 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     prm.k = static_cast<const __nv_bfloat16 *>(k);
     prm.q = static_cast<const __nv_bfloat16 *>(q);
     prm.beta = static_cast<const __nv_bfloat16 *>(beta);
+    prm.g = static_cast<const __nv_bfloat16 *>(g);
+    prm.scalar_gate = scalar_gate ? 1 : 0;
     prm.init_state = init_state;
     prm.final_state = final_state;
     prm.o = static_cast<__nv_bfloat16 *>(o);

@@ -20,7 +20,7 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUD
 KDA_BF16, KDA_FP32 = 0, 1
 EXPORTED = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
             "kda_prefill", "kda_decode_step", "kda_check_workspace_error",
-            "kda_prefill_noalloc")
+            "kda_prefill_noalloc", "gdn_prefill", "gdn_decode_step")
 
 
 class KdaError(RuntimeError):
@@ -50,6 +50,10 @@ def lib():
         L.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
                                       ctypes.c_int, vp, vp]
         L.kda_decode_step.restype = ctypes.c_int
+        L.gdn_prefill.argtypes = L.kda_prefill.argtypes
+        L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_decode_step.argtypes = L.kda_decode_step.argtypes
+        L.gdn_decode_step.restype = ctypes.c_int
         L.kda_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
                                           ctypes.c_int, vp, vp, vp]
         L.kda_prefill_noalloc.restype = ctypes.c_int
@@ -99,6 +103,25 @@ def kda_prefill(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None,
     [N+1] on the device or None (num_seqs equal sequences, default 1).
     Returns (o, final_state); final_state is None if output_final_state is False.
     """
+    if log_alpha.shape != q.shape:
+        raise ValueError("log_alpha must have q's shape [T, H, d_k]")
+    return _prefill("kda_prefill", q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
+                    o, final_state, workspace, output_final_state, stream)
+
+
+def gdn_prefill(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None,
+                num_seqs=None, o=None, final_state=None, workspace=None,
+                output_final_state=True, stream=None):
+    """Chunkwise Gated DeltaNet prefill: as kda_prefill with one gate value per
+    (token, head), log_alpha [T, H]."""
+    if log_alpha.shape != q.shape[:2]:
+        raise ValueError("log_alpha must be [T, H]")
+    return _prefill("gdn_prefill", q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
+                    o, final_state, workspace, output_final_state, stream)
+
+
+def _prefill(fn, q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, o, final_state,
+             workspace, output_final_state, stream):
     T, H, dk = q.shape
     dv = v.shape[-1]
     if cu_seqlens is not None:
@@ -115,28 +138,42 @@ def kda_prefill(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None,
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     _check_cuda(q, k, v, log_alpha, beta, init_state, cu_seqlens, o, final_state, workspace)
-    st = lib().kda_prefill(
+    st = getattr(lib(), fn)(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
         _ptr(cu_seqlens), n, T, H, dk, dv, _dtype_code(q), _ptr(o), _ptr(final_state),
         _ptr(workspace), workspace.numel(), _stream(stream, q.device))
     if st != KDA_OK:
-        raise KdaError(st, "kda_prefill")
+        raise KdaError(st, fn)
     return o, final_state
 
 
 def kda_decode_step(q, k, v, log_alpha, beta, state, o=None, stream=None):
     """One KDA step per sequence; ``state`` [B, H, d_k, d_v] fp32 is updated in
     place.  Returns o [B, H, d_v]."""
+    if log_alpha.shape != q.shape:
+        raise ValueError("log_alpha must have q's shape [B, H, d_k]")
+    return _decode("kda_decode_step", q, k, v, log_alpha, beta, state, o, stream)
+
+
+def gdn_decode_step(q, k, v, log_alpha, beta, state, o=None, stream=None):
+    """One Gated DeltaNet step per sequence (log_alpha [B, H]); ``state`` is
+    updated in place.  Returns o [B, H, d_v]."""
+    if log_alpha.shape != q.shape[:2]:
+        raise ValueError("log_alpha must be [B, H]")
+    return _decode("gdn_decode_step", q, k, v, log_alpha, beta, state, o, stream)
+
+
+def _decode(fn, q, k, v, log_alpha, beta, state, o, stream):
     B, H, dk = q.shape
     dv = v.shape[-1]
     if o is None:
         o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
     _check_cuda(q, k, v, log_alpha, beta, state, o)
-    st = lib().kda_decode_step(
+    st = getattr(lib(), fn)(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state),
         B, H, dk, dv, _dtype_code(q), _ptr(o), _stream(stream, q.device))
     if st != KDA_OK:
-        raise KdaError(st, "kda_decode_step")
+        raise KdaError(st, fn)
     return o
 
 

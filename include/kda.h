@@ -150,6 +150,40 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            kda_stream_t stream);
 
 /*
+ * The same two calls for Gated DeltaNet, whose forget gate is one scalar per
+ * token and head (page "Kimi Linear" on docsaid.org, section "KDA : une
+ * decroissance propre a chaque canal", the Gated DeltaNet update that opens
+ * it; news digest page on Kimi Linear, section "De l'attention lineaire a
+ * Gated DeltaNet"):
+ *
+ *     S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,
+ *     o_t = S_t^T q_t,   alpha_t = exp(log_alpha_t) a scalar in (0, 1].
+ *
+ * A scalar gate commutes with (I - beta k k^T), so this is the KDA update
+ * with the gate repeated over the d_k key channels; the kernels take it that
+ * way (each 64-token chunk's gate values are spread over the channels in
+ * shared memory) and run the same paths as kda_prefill / kda_decode_step.
+ *
+ * Arguments, layouts, workspace (kda_prefill_workspace_size), alignment and
+ * errors are those of kda_prefill / kda_decode_step except:
+ *   log_alpha : [T_total, H] (prefill) or [batch, H] (decode), dtype, with
+ *               only its element's natural alignment.
+ */
+kda_status gdn_prefill(const void *q, const void *k, const void *v,
+                       const void *log_alpha, const void *beta,
+                       const float *init_state, const int32_t *cu_seqlens,
+                       int32_t num_seqs, int64_t total_tokens, int32_t H,
+                       int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                       float *final_state, void *workspace,
+                       size_t workspace_bytes, kda_stream_t stream);
+
+kda_status gdn_decode_step(const void *q, const void *k, const void *v,
+                           const void *log_alpha, const void *beta,
+                           float *state, int32_t batch, int32_t H,
+                           int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                           kda_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads the error word that the prefill kernels
  * leave at the start of `workspace` (non-zero when a device-side check failed,
  * e.g. cu_seqlens not non-decreasing or not ending at T_total).  Returns

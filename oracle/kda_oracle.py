@@ -12,6 +12,9 @@ recurrence", section "Kimi Delta Attention = les trois remedes combines"):
     S_t = (I - beta_t k_t k_t^T) Diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T
     o_t = S_t^T q_t
 
+``gdn_recurrence`` is the Gated DeltaNet special case (one scalar gate per
+token and head), written from its own update equation.
+
 Inputs are float64 numpy arrays holding exactly the values the GPU sees (bf16
 inputs are widened exactly).  Pins of this oracle (closed forms, exact
 retrieval, explicit transition products, invariants) are in
@@ -56,6 +59,8 @@ def _load():
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 dp, dp, ctypes.c_int]
             lib.kda_oracle_recurrence.restype = ctypes.c_int
+            lib.gdn_oracle_recurrence.argtypes = lib.kda_oracle_recurrence.argtypes
+            lib.gdn_oracle_recurrence.restype = ctypes.c_int
             lib.kda_oracle_max_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -111,6 +116,47 @@ def kda_recurrence(q, k, v, g, beta, init_state=None, cu_seqlens=None,
     if rc != 0:
         raise RuntimeError(f"kda_oracle_recurrence failed with code {rc}")
     return o, fs
+
+
+def gdn_recurrence(q, k, v, g, beta, init_state=None, cu_seqlens=None,
+                   nthreads: int = 0):
+    """Gated DeltaNet over packed sequences: as kda_recurrence with one gate
+    value per (token, head), g [T, H] (the scalar-gate update, taken as
+    printed: erase, then decay, then write)."""
+    q, k, v, g, beta = (_f64(x) for x in (q, k, v, g, beta))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    if k.shape != (T, H, dk) or g.shape != (T, H):
+        raise ValueError("q, k must share shape [T, H, d_k] and g be [T, H]")
+    if v.shape[:2] != (T, H) or beta.shape != (T, H):
+        raise ValueError("v must be [T, H, d_v] and beta [T, H]")
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    n = cu.shape[0] - 1
+    if cu[0] != 0 or cu[-1] != T:
+        raise ValueError("cu_seqlens must start at 0 and end at T")
+    s0 = None if init_state is None else _f64(init_state)
+    if s0 is not None and s0.shape != (n, H, dk, dv):
+        raise ValueError("init_state must be [N, H, d_k, d_v]")
+    o = np.zeros((T, H, dv), dtype=np.float64)
+    fs = np.zeros((n, H, dk, dv), dtype=np.float64)
+    rc = _load().gdn_oracle_recurrence(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0),
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        n, H, dk, dv, _ptr(o), _ptr(fs), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"gdn_oracle_recurrence failed with code {rc}")
+    return o, fs
+
+
+def gdn_decode_step(q, k, v, g, beta, state, nthreads: int = 0):
+    """One Gated DeltaNet step for each of B sequences (g [B, H])."""
+    B = np.asarray(q).shape[0]
+    cu = np.arange(B + 1, dtype=np.int64)
+    return gdn_recurrence(q, k, v, g, beta, init_state=state, cu_seqlens=cu,
+                          nthreads=nthreads)
 
 
 def kda_decode_step(q, k, v, g, beta, state, nthreads: int = 0):

@@ -23,13 +23,14 @@ def _declared_functions():
         if path.endswith(".h"):
             text = open(os.path.join(ROOT, "include", path)).read()
             text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-            names += re.findall(r"\b(kda_\w+)\s*\(", text)
+            names += re.findall(r"\b((?:kda|gdn)_\w+)\s*\(", text)
     return sorted(set(names))
 
 
 def test_exports_every_declared_symbol(L):
     names = _declared_functions()
     assert "kda_prefill" in names and "kda_decode_step" in names
+    assert "gdn_prefill" in names and "gdn_decode_step" in names
     for n in names:
         assert hasattr(L, n), f"libkda.so does not export {n}"
 
@@ -60,14 +61,14 @@ def test_workspace_size(L):
 FAKE = 1 << 20  # 16-byte aligned, never dereferenced on the host
 
 
-def _prefill(L, **kw):
+def _prefill(L, fn="kda_prefill", **kw):
     a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, g=FAKE * 4, b=FAKE * 5, s0=None, cu=None,
              n=1, T=64, H=1, dk=16, dv=16, dt=1, o=FAKE * 64, fs=None, ws=FAKE * 128,
              wsb=4096)
     a.update(kw)
-    return L.kda_prefill(a["q"], a["k"], a["v"], a["g"], a["b"], a["s0"], a["cu"],
-                         a["n"], a["T"], a["H"], a["dk"], a["dv"], a["dt"], a["o"],
-                         a["fs"], a["ws"], a["wsb"], None)
+    return getattr(L, fn)(a["q"], a["k"], a["v"], a["g"], a["b"], a["s0"], a["cu"],
+                          a["n"], a["T"], a["H"], a["dk"], a["dv"], a["dt"], a["o"],
+                          a["fs"], a["ws"], a["wsb"], None)
 
 
 def test_prefill_rejects_on_host(L):
@@ -86,11 +87,11 @@ def test_prefill_rejects_on_host(L):
     assert _prefill(L, o=FAKE + 64) == 1           # o overlaps q
 
 
-def _decode(L, **kw):
+def _decode(L, fn="kda_decode_step", **kw):
     a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, g=FAKE * 4, b=FAKE * 5, s=FAKE * 16,
              B=4, H=2, dk=16, dv=16, dt=1, o=FAKE * 64)
     a.update(kw)
-    return L.kda_decode_step(a["q"], a["k"], a["v"], a["g"], a["b"], a["s"], a["B"],
+    return getattr(L, fn)(a["q"], a["k"], a["v"], a["g"], a["b"], a["s"], a["B"],
                              a["H"], a["dk"], a["dv"], a["dt"], a["o"], None)
 
 
@@ -103,6 +104,30 @@ def test_decode_rejects_on_host(L):
     assert _decode(L, o=FAKE * 16 + 32) == 1       # o overlaps the state
     assert _decode(L, v=FAKE * 3 + 2) == 1         # not element-aligned (fp32)
     assert _decode(L, s=FAKE * 16 + 8) == 1        # state not 16-byte aligned
+
+
+def test_gdn_rejects_on_host(L):
+    # the scalar gate needs only element alignment; everything else as for KDA
+    assert _prefill(L, "gdn_prefill", g=FAKE * 4 + 4, ws=None) == 3   # alignment passed, no workspace
+    assert _prefill(L, "gdn_prefill", g=FAKE * 4 + 2) == 1            # fp32 gate not 4-byte aligned
+    assert _prefill(L, "gdn_prefill", n=0) == 1
+    assert _prefill(L, "gdn_prefill", dk=48) == 2
+    assert _prefill(L, "gdn_prefill", q=FAKE + 4) == 1
+    # o [64, 1, 16] fp32 at FAKE * 64 (4 KB) overlaps a gate placed right below its end
+    assert _prefill(L, "gdn_prefill", g=FAKE * 64 + 4096 - 128) == 1
+    assert _decode(L, "gdn_decode_step", B=0) == 0
+    assert _decode(L, "gdn_decode_step", g=FAKE * 4 + 2) == 1
+    assert _decode(L, "gdn_decode_step", s=None) == 1
+
+
+def test_binding_checks_gate_shape():
+    import torch
+    from gated_delta_rule_69_b200 import kda
+    x = torch.zeros(4, 2, 16)
+    with pytest.raises(ValueError):
+        kda.gdn_decode_step(x, x, x, x, torch.zeros(4, 2), torch.zeros(4, 2, 16, 16))
+    with pytest.raises(ValueError):
+        kda.kda_decode_step(x, x, x, torch.zeros(4, 2), torch.zeros(4, 2), torch.zeros(4, 2, 16, 16))
 
 
 def test_binding_refuses_cpu_tensors():

@@ -8,6 +8,8 @@ Each test names the plausible oracle mistake it catches:
   * wrong sign of the correction / dropped beta         -> DeltaNet solve, explicit product
   * transposed state (S q instead of S^T q)             -> explicit product (d_k != d_v)
   * state not reset per sequence                        -> varlen split invariant
+  * Gated DeltaNet: gate inside the erase, or missing    -> scalar-gate commutation,
+    scalar beta=0 closed form, orthonormal overwrite
 """
 import json
 import math
@@ -279,3 +281,56 @@ def test_empty_sequence_keeps_initial_state(oracle_mod):
     cu = np.concatenate([[0], np.cumsum(lens)])
     _, fs = oracle_mod.kda_recurrence(q, k, v, g, beta, init_state=s0, cu_seqlens=cu)
     np.testing.assert_array_equal(fs[1], s0[1])
+
+
+# --- Gated DeltaNet (scalar gate) ----------------------------------------------
+
+def test_gdn_equals_kda_with_repeated_gate(oracle_mod):
+    """A scalar alpha commutes with (I - beta k k^T): the GDN update taken as
+    printed (erase, then decay) equals the KDA update (decay, then erase) with
+    the gate repeated over the channels.  The two oracle loops share no step
+    order, so a misplaced or missing gate in either shows here."""
+    rng = np.random.default_rng(41)
+    T, H, dk, dv = 37, 2, 8, 5
+    q, k, v, g3, beta, s0 = _rand_case(rng, T, H, dk, dv, n_seqs=2)
+    g = g3[..., 0]
+    cu = np.array([0, 15, T])
+    o1, f1 = oracle_mod.gdn_recurrence(q, k, v, g, beta, s0, cu)
+    o2, f2 = oracle_mod.kda_recurrence(q, k, v, np.repeat(g[..., None], dk, axis=-1), beta, s0, cu)
+    assert np.abs(o1 - o2).max() < 1e-12 * max(1.0, np.abs(o2).max())
+    assert np.abs(f1 - f2).max() < 1e-12 * max(1.0, np.abs(f2).max())
+
+
+def test_gdn_beta0_scalar_decay(oracle_mod):
+    """beta = 0: S_t = (prod_{s<=t} alpha_s) S_0 and o_t = S_t^T q_t."""
+    rng = np.random.default_rng(42)
+    T, H, dk, dv = 9, 1, 4, 3
+    q, k, v, g3, beta, s0 = _rand_case(rng, T, H, dk, dv)
+    g = g3[..., 0]
+    o, fs = oracle_mod.gdn_recurrence(q, k, v, g, np.zeros_like(beta), s0)
+    cum = np.exp(np.cumsum(g[:, 0]))
+    for t in range(T):
+        expect = cum[t] * (s0[0, 0].T @ q[t, 0])
+        assert np.allclose(o[t, 0], expect, rtol=1e-13, atol=1e-13)
+    assert np.allclose(fs[0, 0], cum[-1] * s0[0, 0], rtol=1e-13, atol=1e-13)
+
+
+def test_gdn_orthonormal_overwrite(oracle_mod):
+    """alpha = 1, beta = 1 and orthonormal keys: each write replaces the value
+    stored under its key, so S_T = (I - sum e_i e_i^T) S_0 + sum e_i v_i^T and
+    reading key e_i returns v_i."""
+    rng = np.random.default_rng(43)
+    dk, dv, m = 6, 4, 4
+    basis, _ = np.linalg.qr(rng.normal(size=(dk, dk)))
+    keys = basis[:, :m].T                      # m orthonormal rows
+    T = m
+    k = keys[:, None, :]
+    q = keys[:, None, :]
+    v = rng.normal(size=(T, 1, dv))
+    s0 = rng.normal(size=(1, 1, dk, dv))
+    o, fs = oracle_mod.gdn_recurrence(q, k, v, np.zeros((T, 1)), np.ones((T, 1)), s0)
+    P = keys.T @ keys
+    expect = (np.eye(dk) - P) @ s0[0, 0] + keys.T @ v[:, 0, :]
+    assert np.allclose(fs[0, 0], expect, atol=1e-12)
+    for t in range(T):
+        assert np.allclose(o[t, 0], v[t, 0], atol=1e-12)
