@@ -92,11 +92,12 @@ constexpr uint32_t kPrepTmemCols = 512;
 constexpr uint32_t kRawBytes = 4 * 8192 + 16384;   // k, q (2 boxes each), log_alpha
 
 // ---- chain kernel, one CTA per (sequence, head, DVT-column slice of d_v).
-// Warp 0 loads; warps 1 .. NCW hold the state (warp w: TMEM lanes of quadrant
-// w mod 4, columns 32 ((w - 1) / 4) .. + 31 of the slice); warp NCW + 1 issues
-// the products.  Ring A carries MP, YT, the v slice and exp(G_L); ring B QP,
-// ZB; the bf16 copy of the state is double-buffered.  Stages (A, B): (3, 2)
-// for 32 columns, (3, 1) for 64, (2, 1) for 128: what shared memory holds.
+// Warp 0 loads ring A, warp NCW + 2 ring B (each ring runs ahead on its own);
+// warps 1 .. NCW hold the state (warp w: TMEM lanes of quadrant w mod 4,
+// columns 32 ((w - 1) / 4) .. + 31 of the slice); warp NCW + 1 issues the
+// products.  Ring A carries MP, YT, the v slice and exp(G_L); ring B QP, ZB.
+// Stages (A, B) and bf16 state copies: (3, 2) and 2 for 32 columns, (3, 1)
+// and 2 for 64, (2, 2) and 1 for 128: what shared memory holds.
 constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 
 template <int DVT_>
@@ -104,7 +105,7 @@ struct ChainCfg {
     static constexpr int DVT = DVT_;
     static constexpr int NTILE = DV / DVT;
     static constexpr int NCW = 4 * (DVT / 32);
-    static constexpr int THREADS = 32 * (NCW + 2);
+    static constexpr int THREADS = 32 * (NCW + 3);
     static constexpr int NSA = DVT == 128 ? 2 : 3;
     static constexpr int NSB = DVT == 64 ? 1 : 2;
     // Copies of the bf16 state: two let the chain warps write S_{n+1} while
@@ -698,12 +699,12 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     const uint32_t tmem = misc[0];
 
     if (warp == 0) {
-        // ---------------------------------------------- loader: records + v slices
+        // ---------------------------------------------- ring A: MP, YT, v slice, exp(G_L)
         if (lane == 0 && nchunks > 0) {
             tma_prefetch_desc(&tm_v);
-            int issued_a = 0, issued_b = 0;
+            int issued_a = 0;
             for (int n = 0; n < nchunks; ++n) {
-                const int sa = n % NSA, sb = n % NSB;
+                const int sa = n % NSA;
                 if (n >= NSA) mbar_wait(&EMPTYA[sa], ((n / NSA) - 1) & 1, abort_flag);
                 if (*abort_flag) break;
                 const size_t ri = (rec0 + n) * p.H + h;
@@ -717,16 +718,27 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 tma_load_3d(slot_a + Cfg::A_V, &tm_v, &FULLA[sa], j0, h, t);
                 if (DVT == 128) tma_load_3d(slot_a + Cfg::A_V + 8192, &tm_v, &FULLA[sa], j0 + 64, h, t);
                 issued_a = n + 1;
+            }
+            // the copies land before this CTA may exit
+            for (int n = (issued_a > NSA ? issued_a - NSA : 0); n < issued_a; ++n)
+                wait_drain(&FULLA[n % NSA], (n / NSA) & 1);
+        }
+    } else if (warp == NCW + 2) {
+        // ---------------------------------------------- ring B: QP, ZB
+        if (lane == 0 && nchunks > 0) {
+            int issued_b = 0;
+            for (int n = 0; n < nchunks; ++n) {
+                const int sb = n % NSB;
                 if (n >= NSB) mbar_wait(&EMPTYB[sb], ((n / NSB) - 1) & 1, abort_flag);
                 if (*abort_flag) break;
+                const size_t ri = (rec0 + n) * p.H + h;
+                const uint8_t *rec = p.recs + ri * Rec::STRIDE;
+                if (p.rec_ready && !acquire_flag(p.rec_ready + ri, abort_flag)) break;
                 uint8_t *slot_b = sm + Cfg::RB + sb * Cfg::B_STRIDE;
                 mbar_arrive_expect_tx(&FULLB[sb], 24576);
                 bulk_load(slot_b + Cfg::B_QP, rec + Rec::QP, 24576, &FULLB[sb]);   // QP, ZB
                 issued_b = n + 1;
             }
-            // the copies land before this CTA may exit
-            for (int n = (issued_a > NSA ? issued_a - NSA : 0); n < issued_a; ++n)
-                wait_drain(&FULLA[n % NSA], (n / NSA) & 1);
             for (int n = (issued_b > NSB ? issued_b - NSB : 0); n < issued_b; ++n)
                 wait_drain(&FULLB[n % NSB], (n / NSB) & 1);
         }
@@ -839,6 +851,269 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 dst[i] = make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, Cfg::TMEM_COLS);
+    }
+    if (tid == 0 && *abort_flag) atomicOr(p.err_word, kDevErrTimeout);
+}
+
+// =============================================================== whole-d_v chain, transposed
+//
+// One CTA per (sequence, head) carrying the state transposed, S^T [j = d_v
+// lanes][c = d_k columns] fp32 in TMEM, with its bf16 copy SB^T also in TMEM
+// as the A operand of the products:
+//     S_{n+1}^T = S_n^T Diag(exp(G_L)) + SB_n^T MP_n^T + V_n^T YT_n^T
+//     O_n^T     = SB_n^T QP_n^T + V_n^T ZB_n^T
+// The record operands keep their layout and descriptors; they only change
+// side (B instead of A), and V (its two 64-column atoms) is the A operand in
+// the MN-major form.  Against the row-major chain this removes the bf16 state
+// from shared memory (its store, the proxy fence, and the two reads per chunk
+// by the products), about a third of the chunk's shared-memory traffic, and
+// makes the output products M = 128.
+// Three rings, each with its own loader: A (MP, YT, exp(G_L)), V (the v
+// tile, read from HBM, so four stages ahead) and B (QP, ZB).
+//   warp 0: ring A;  warp 18: ring B;  warp 19: ring V
+//   warps 1..16: the state; warp w holds lanes j of quadrant w mod 4 and
+//                columns c in 32 ((w - 1) / 4) .. + 31
+//   warp 17: issues the products
+struct ChainT {
+    static constexpr int NCW = 16;
+    static constexpr int THREADS = 32 * (NCW + 4);
+    static constexpr int NSA = 2, NSB = 2, NSV = 4;
+    static constexpr uint32_t A_MP = 0, A_YT = 32768, A_STRIDE = 49152;
+    static constexpr uint32_t B_QP = 0, B_ZB = 16384, B_STRIDE = 24576;
+    static constexpr uint32_t V_STRIDE = 16384;
+    static constexpr uint32_t RA = 0;
+    static constexpr uint32_t RV = NSA * A_STRIDE;
+    static constexpr uint32_t RB = RV + NSV * V_STRIDE;
+    static constexpr uint32_t EGLR = RB + NSB * B_STRIDE;   // NSA x exp(G_L), 128 fp32 each
+    static constexpr uint32_t BARS = EGLR + NSA * 512;
+    static constexpr uint32_t MISC = BARS + 256;
+    static constexpr uint32_t SIZE = MISC + 64;
+    static constexpr uint32_t ALLOC = SIZE + 1024;
+    // TMEM columns: S^T fp32 (128), SB^T bf16 pairs x 2 (64 each), O^T fp32 x 2 (64 each)
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t COL_S = 0, COL_SB = 128, COL_O = 256;
+    static_assert(ALLOC <= 232448, "chain shared memory");
+    static_assert(2 * NSA + 2 * NSB + 2 * NSV + 5 <= 32, "barrier area");
+};
+
+__global__ void __launch_bounds__(ChainT::THREADS, 1)
+kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    using Cfg = ChainT;
+    constexpr int NSA = Cfg::NSA, NSB = Cfg::NSB, NSV = Cfg::NSV, NCW = Cfg::NCW;
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t *sm = dyn_smem + ((1024u - (smem_addr(dyn_smem) & 1023u)) & 1023u);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.x % p.H;
+    const int rank = blockIdx.x / p.H;
+    const int seq = p.perm ? p.perm[rank] : rank;
+    int64_t bos, eos;
+    seq_bounds(p, seq, bos, eos);
+    const int64_t len = eos - bos;
+    const int nchunks = (int)((len + C - 1) / C);
+    const size_t rec0 = (size_t)p.chunk_off[seq];
+
+    // mbarriers: FULLA[NSA], EMPTYA[NSA], FULLB[NSB], EMPTYB[NSB], FULLV[NSV], EMPTYV[NSV],
+    // SDONE, ODONE[2], FIN, SREADY
+    uint64_t *B = reinterpret_cast<uint64_t *>(sm + Cfg::BARS);
+    uint64_t *FULLA = B, *EMPTYA = B + NSA, *FULLB = B + 2 * NSA, *EMPTYB = B + 2 * NSA + NSB;
+    uint64_t *FULLV = B + 2 * NSA + 2 * NSB, *EMPTYV = FULLV + NSV;
+    uint64_t *SDONE = EMPTYV + NSV, *ODONE = SDONE + 1, *FIN = SDONE + 3, *SREADY = SDONE + 4;
+    constexpr int kBars = 2 * NSA + 2 * NSB + 2 * NSV + 5;
+    uint32_t *misc = reinterpret_cast<uint32_t *>(sm + Cfg::MISC);
+    volatile uint32_t *abort_flag = misc + 1;
+    if (tid == 0) {
+        for (int i = 0; i < kBars - 1; ++i) mbar_init(&B[i], 1);
+        mbar_init(SREADY, NCW);   // one arrive per chain warp
+        misc[1] = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&misc[0], Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+
+    if (warp == 0) {
+        // ---------------------------------------------- ring A: MP, YT, exp(G_L)
+        if (lane == 0 && nchunks > 0) {
+            int issued_a = 0;
+            for (int n = 0; n < nchunks; ++n) {
+                const int sa = n % NSA;
+                if (n >= NSA) mbar_wait(&EMPTYA[sa], ((n / NSA) - 1) & 1, abort_flag);
+                if (*abort_flag) break;
+                const size_t ri = (rec0 + n) * p.H + h;
+                const uint8_t *rec = p.recs + ri * Rec::STRIDE;
+                if (p.rec_ready && !acquire_flag(p.rec_ready + ri, abort_flag)) break;   // the record is complete
+                uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
+                mbar_arrive_expect_tx(&FULLA[sa], 49152 + 512);
+                bulk_load(slot_a + Cfg::A_MP, rec + Rec::MP, 49152, &FULLA[sa]);   // MP, YT
+                bulk_load(sm + Cfg::EGLR + sa * 512, rec + Rec::EGL, 512, &FULLA[sa]);
+                issued_a = n + 1;
+            }
+            // the copies land before this CTA may exit
+            for (int n = (issued_a > NSA ? issued_a - NSA : 0); n < issued_a; ++n)
+                wait_drain(&FULLA[n % NSA], (n / NSA) & 1);
+        }
+    } else if (warp == NCW + 3) {
+        // ---------------------------------------------- ring V: the v tile (from HBM)
+        if (lane == 0 && nchunks > 0) {
+            tma_prefetch_desc(&tm_v);
+            int issued_v = 0;
+            for (int n = 0; n < nchunks; ++n) {
+                const int sv = n % NSV;
+                if (n >= NSV) mbar_wait(&EMPTYV[sv], ((n / NSV) - 1) & 1, abort_flag);
+                if (*abort_flag) break;
+                uint8_t *slot_v = sm + Cfg::RV + sv * Cfg::V_STRIDE;
+                const int t = (int)(bos + (int64_t)n * C);
+                mbar_arrive_expect_tx(&FULLV[sv], 16384);
+                tma_load_3d(slot_v, &tm_v, &FULLV[sv], 0, h, t);
+                tma_load_3d(slot_v + 8192, &tm_v, &FULLV[sv], 64, h, t);
+                issued_v = n + 1;
+            }
+            for (int n = (issued_v > NSV ? issued_v - NSV : 0); n < issued_v; ++n)
+                wait_drain(&FULLV[n % NSV], (n / NSV) & 1);
+        }
+    } else if (warp == NCW + 2) {
+        // ---------------------------------------------- ring B: QP, ZB
+        if (lane == 0 && nchunks > 0) {
+            int issued_b = 0;
+            for (int n = 0; n < nchunks; ++n) {
+                const int sb = n % NSB;
+                if (n >= NSB) mbar_wait(&EMPTYB[sb], ((n / NSB) - 1) & 1, abort_flag);
+                if (*abort_flag) break;
+                const size_t ri = (rec0 + n) * p.H + h;
+                const uint8_t *rec = p.recs + ri * Rec::STRIDE;
+                if (p.rec_ready && !acquire_flag(p.rec_ready + ri, abort_flag)) break;
+                uint8_t *slot_b = sm + Cfg::RB + sb * Cfg::B_STRIDE;
+                mbar_arrive_expect_tx(&FULLB[sb], 24576);
+                bulk_load(slot_b + Cfg::B_QP, rec + Rec::QP, 24576, &FULLB[sb]);   // QP, ZB
+                issued_b = n + 1;
+            }
+            for (int n = (issued_b > NSB ? issued_b - NSB : 0); n < issued_b; ++n)
+                wait_drain(&FULLB[n % NSB], (n / NSB) & 1);
+        }
+    } else if (warp == NCW + 1) {
+        // ---------------------------------------------- tensor-core products
+        const uint32_t idS = idesc_bf16(128, 128, false, false);   // A = SB^T (TMEM), B = MP^T
+        const uint32_t idSV = idesc_bf16(128, 128, true, false);   // A = V^T (MN-major), B = YT^T
+        const uint32_t idO = idesc_bf16(128, 64, false, false);    // A = SB^T (TMEM), B = QP^T
+        const uint32_t idOV = idesc_bf16(128, 64, true, false);    // A = V^T (MN-major), B = ZB^T
+        for (int n = 0; n < nchunks; ++n) {
+            const int sa = n % NSA, sb = n % NSB, sv = n % NSV;
+            uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
+            uint8_t *slot_b = sm + Cfg::RB + sb * Cfg::B_STRIDE;
+            const uint32_t bM = smem_addr(slot_a + Cfg::A_MP);
+            const uint32_t bY = smem_addr(slot_a + Cfg::A_YT);
+            const uint32_t aV = smem_addr(sm + Cfg::RV + sv * Cfg::V_STRIDE);
+            const uint32_t aSB = tmem + Cfg::COL_SB + 64u * (uint32_t)(n & 1);
+            mbar_wait(SREADY, n & 1, abort_flag);
+            mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
+            mbar_wait(&FULLV[sv], (n / NSV) & 1, abort_flag);
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)   // S^T += SB^T MP^T  (K = c')
+                mma_bf16_ts_warp(tmem + Cfg::COL_S, aSB + 8 * ks,
+                                 smem_desc(bM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                                 idS, 1u);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)   // S^T += V^T YT^T  (K = t)
+                mma_bf16_warp(tmem + Cfg::COL_S, smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
+                              smem_desc(bY + ks * 32, 16, 1024, kLayoutSW128), idSV, 1u);
+            mma_commit_warp(SDONE);
+            mbar_wait(&FULLB[sb], (n / NSB) & 1, abort_flag);
+            const uint32_t bQ = smem_addr(slot_b + Cfg::B_QP);
+            const uint32_t bZ = smem_addr(slot_b + Cfg::B_ZB);
+            const uint32_t dO = tmem + Cfg::COL_O + 64u * (uint32_t)(n & 1);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)   // O^T = SB^T QP^T  (K = c)
+                mma_bf16_ts_warp(dO, aSB + 8 * ks,
+                                 smem_desc(bQ + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                                 idO, ks > 0 ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)   // O^T += V^T ZB^T  (K = t')
+                mma_bf16_warp(dO, smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
+                              smem_desc(bZ + ks * 32, 16, 1024, kLayoutSW128), idOV, 1u);
+            mma_commit_warp(&ODONE[n & 1]);
+            mma_commit_warp(&EMPTYA[sa]);
+            mma_commit_warp(&EMPTYB[sb]);
+            mma_commit_warp(&EMPTYV[sv]);
+        }
+        if (nchunks > 0) {   // every arrive of the commits above lands before the CTA exits
+            mma_commit_warp(FIN);
+            wait_drain(FIN, 0);
+        }
+    } else {
+        // ---------------------------------------------- the state chain
+        const int quad = warp & 3;
+        const int g = (warp - 1) >> 2;
+        const int j = 32 * quad + lane;
+        const size_t sbase = ((size_t)seq * p.H + h) * (size_t)(DK * DV) + (size_t)(32 * g) * DV + j;
+        float S[32];
+        if (p.init_state) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) S[i] = p.init_state[sbase + (size_t)i * DV];
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) S[i] = 0.f;
+        }
+        // O^T of chunk m: this warp's 16 t columns, lane j, bf16 to o[t][h][j]
+        auto store_o_t = [&](int m) {
+            mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
+            tc_fence_after();
+            float v[16];
+            tmem_ld16(tmem_addr(tmem, 32 * quad, Cfg::COL_O + 64 * (m & 1) + 16 * g), v);
+            tmem_wait_ld();
+            const int64_t t0 = (int64_t)m * C + 16 * g;
+            __nv_bfloat16 *dst = p.o + ((size_t)(bos + t0) * p.H + h) * DV + j;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (t0 + i < len) dst[(size_t)i * p.H * DV] = __float2bfloat16(v[i]);
+        };
+        for (int n = 0; n < nchunks; ++n) {
+            const int sa = n % NSA;
+            if (n >= 1) {
+                mbar_wait(SDONE, (n - 1) & 1, abort_flag);
+                tc_fence_after();
+                tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + 32 * g), S);
+                tmem_wait_ld();
+            }
+            // SB_n^T: column COL_SB + 64 (n mod 2) + c / 2 holds (c, c + 1)
+            uint32_t w16[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w16[i] = pack_bf16x2(S[2 * i], S[2 * i + 1]);
+            tmem_st16u(tmem_addr(tmem, 32 * quad, Cfg::COL_SB + 64 * (n & 1) + 16 * g), w16);
+            mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
+            const float *egl = reinterpret_cast<const float *>(sm + Cfg::EGLR + sa * 512) + 32 * g;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) S[i] *= egl[i];
+            tmem_st32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + 32 * g), S);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(SREADY);
+            if (n >= 1) store_o_t(n - 1);
+        }
+        if (nchunks > 0) {
+            const int m = nchunks - 1;
+            store_o_t(m);
+            mbar_wait(SDONE, m & 1, abort_flag);
+            tc_fence_after();
+            tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + 32 * g), S);
+            tmem_wait_ld();
+        }
+        if (p.final_state) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) p.final_state[sbase + (size_t)i * DV] = S[i];
         }
     }
     tc_fence_before();
@@ -1044,6 +1319,36 @@ cudaError_t launch_chain(const void *v, int64_t total_tokens, int H, const split
     return cudaGetLastError();
 }
 
+// The transposed whole-d_v chain: grid = sequences x heads.
+cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const split::Params &prm,
+                           unsigned units, bool overlap, cudaStream_t stream) {
+    using namespace split;
+    CUtensorMap mv;
+    if (!make_map_split(&mv, v, total_tokens, H, DV, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    static bool attr_set = false;
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(kda_chain_t_kernel,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)ChainT::ALLOC);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(units);
+    cfg.blockDim = dim3(ChainT::THREADS);
+    cfg.dynamicSmemBytes = ChainT::ALLOC;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = overlap ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kda_chain_t_kernel, mv, prm);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 // Chain slice width and overlap, from a cost model in SM cycles:
 //   prep ~ items x c_p / (SMs it gets), c_p ~ 12 K cycles per (chunk, head)
 //     per SM (two pipelines per SM, ~24 K cycles per item each);
@@ -1187,7 +1492,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         if (e != cudaSuccess) return e;
     }
     return plan.dvt == 32 ? launch_chain<32>(v, total_tokens, H, prm, units, overlap, stream)
-                          : launch_chain<128>(v, total_tokens, H, prm, units, overlap, stream);
+                          : launch_chain_t(v, total_tokens, H, prm, units, overlap, stream);
 }
 
 }  // namespace kda
