@@ -39,7 +39,8 @@ kda_status prefill_impl(const void *q, const void *k, const void *v,
                         int32_t num_seqs, int64_t total_tokens, int32_t H,
                         int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
                         float *final_state, void *workspace,
-                        size_t workspace_bytes, kda_stream_t stream_, bool scalar_gate) {
+                        size_t workspace_bytes, kda_stream_t stream_, bool scalar_gate,
+                        const kda::LayerArgs *layer = nullptr) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (num_seqs < 1 || total_tokens < 0 || H < 1) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_BF16 && dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
@@ -75,11 +76,25 @@ kda_status prefill_impl(const void *q, const void *k, const void *v,
         overlaps(init_state, ns, final_state, ns))
         return KDA_ERR_INVALID_ARG;
 
+    if (layer) {   // the fused layer runs on the two-kernel tensor-core path only
+        if (total_tokens > 0 && !use_tensor_cores(dtype, d_k, d_v, total_tokens))
+            return KDA_ERR_UNSUPPORTED;
+        if (total_tokens > 0 &&
+            workspace_bytes < kda::prefill_split_workspace(num_seqs, total_tokens, H))
+            return KDA_ERR_WORKSPACE;
+        if (!layer->A_log || !aligned_to(layer->A_log, 4) ||
+            (layer->norm_weight && !aligned_to(layer->norm_weight, 4)) ||
+            (layer->out_gate && !aligned_to(layer->out_gate, eb)) ||
+            !(layer->qk_eps >= 0.f) || !(layer->norm_eps >= 0.f) ||
+            overlaps(o, nv, layer->out_gate, nv))
+            return KDA_ERR_INVALID_ARG;
+    }
     if (use_tensor_cores(dtype, d_k, d_v, total_tokens) &&
         workspace_bytes >= kda::prefill_split_workspace(num_seqs, total_tokens, H))
         return from_cuda(kda::launch_prefill_split(q, k, v, log_alpha, beta, init_state,
                                                    cu_seqlens, num_seqs, total_tokens, H, o,
-                                                   final_state, workspace, scalar_gate, stream));
+                                                   final_state, workspace, scalar_gate, layer,
+                                                   stream));
     if (use_tensor_cores(dtype, d_k, d_v, total_tokens))
         return from_cuda(kda::launch_prefill_tc(q, k, v, log_alpha, beta, init_state, cu_seqlens,
                                                 num_seqs, total_tokens, H, o, final_state,
@@ -97,7 +112,8 @@ kda_status decode_impl(const void *q, const void *k, const void *v,
                        const void *log_alpha, const void *beta,
                        float *state, int32_t batch, int32_t H,
                        int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
-                       kda_stream_t stream_, bool scalar_gate) {
+                       kda_stream_t stream_, bool scalar_gate,
+                       const kda::LayerArgs *layer = nullptr) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (batch < 0 || H < 1) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_BF16 && dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
@@ -119,8 +135,14 @@ kda_status decode_impl(const void *q, const void *k, const void *v,
         overlaps(o, nv, log_alpha, ng) || overlaps(o, nv, beta, nb) ||
         overlaps(o, nv, state, ns))
         return KDA_ERR_INVALID_ARG;
+    if (layer && (!layer->A_log || !aligned_to(layer->A_log, 4) ||
+                  (layer->norm_weight && !aligned_to(layer->norm_weight, 4)) ||
+                  (layer->out_gate && !aligned_to(layer->out_gate, eb)) ||
+                  !(layer->qk_eps >= 0.f) || !(layer->norm_eps >= 0.f) ||
+                  overlaps(o, nv, layer->out_gate, nv)))
+        return KDA_ERR_INVALID_ARG;
     return from_cuda(kda::launch_decode(q, k, v, log_alpha, beta, state, batch, H,
-                                        d_k, d_v, dtype, o, scalar_gate, stream));
+                                        d_k, d_v, dtype, o, scalar_gate, layer, stream));
 }
 
 }  // namespace
@@ -189,6 +211,30 @@ kda_status gdn_decode_step(const void *q, const void *k, const void *v,
                            kda_stream_t stream) {
     return decode_impl(q, k, v, log_alpha, beta, state, batch, H, d_k, d_v, dtype, o, stream,
                        true);
+}
+
+kda_status kda_layer_prefill(const void *q, const void *k, const void *v, const void *gate_z,
+                             const float *A_log, const void *beta_logit, const void *out_gate,
+                             const float *norm_weight, float qk_eps, float norm_eps,
+                             const float *init_state, const int32_t *cu_seqlens,
+                             int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                             int32_t d_v, kda_dtype dtype, void *o, float *final_state,
+                             void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+    const kda::LayerArgs la = {gate_z, A_log, beta_logit, out_gate, norm_weight, qk_eps, norm_eps};
+    return prefill_impl(q, k, v, gate_z, beta_logit, init_state, cu_seqlens, num_seqs,
+                        total_tokens, H, d_k, d_v, dtype, o, final_state, workspace,
+                        workspace_bytes, stream, false, &la);
+}
+
+kda_status kda_layer_decode_step(const void *q, const void *k, const void *v,
+                                 const void *gate_z, const float *A_log, const void *beta_logit,
+                                 const void *out_gate, const float *norm_weight, float qk_eps,
+                                 float norm_eps, float *state, int32_t batch, int32_t H,
+                                 int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                                 kda_stream_t stream) {
+    const kda::LayerArgs la = {gate_z, A_log, beta_logit, out_gate, norm_weight, qk_eps, norm_eps};
+    return decode_impl(q, k, v, gate_z, beta_logit, state, batch, H, d_k, d_v, dtype, o, stream,
+                       false, &la);
 }
 
 kda_status kda_check_workspace_error(const void *workspace, kda_stream_t stream_) {

@@ -57,6 +57,13 @@ struct Bufs {
     float *egl;          // 128 fp32: exp(G_L)
     float *csum;         // 4 x 128 fp32 scratch
     uint32_t *slow_flag; // one word
+    // The layer prologue (null nrm: off).  graw then holds the gate
+    // pre-activation z on entry and log_alpha = neg_eA softplus(z) (bf16) on
+    // exit; q and k are L2-normalised with the factors left in nrm
+    // (1 / |k_t| at t, 1 / |q_t| at 64 + t).
+    float *nrm;          // 128 fp32, or null
+    float neg_eA;        // -exp(A_log[h])
+    float qk_eps;
 };
 
 // Index of A element (t, i): rows padded to 65 floats, so that a warp
@@ -81,7 +88,7 @@ __device__ __forceinline__ int tfi(int row, int col) { return row * kTStride + c
 // reference per block) or kPairwise.
 enum : int { kProductForm = 0, kSecondary = 1, kPairwise = 2 };
 
-template <int BAR>
+template <int BAR, bool LAYER>
 __device__ int gate(const Bufs &b, int pt, int L) {
     const int c = 2 * (pt & 63);
     const int tg = pt >> 6;
@@ -104,21 +111,59 @@ __device__ int gate(const Bufs &b, int pt, int L) {
         named_barrier(BAR, kGroupThreads);
     }
 
+    constexpr bool layer = LAYER;   // the prologue (b.nrm set)
     uint32_t graw_v[16], k_v[16], q_v[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int t = t0 + i;
-        graw_v[i] = *reinterpret_cast<const uint32_t *>(b.graw + t * 256 + c * 2);
         k_v[i] = *reinterpret_cast<const uint32_t *>(stack + sw128_off(t, cc));
         q_v[i] = *reinterpret_cast<const uint32_t *>(stack + sw128_off(64 + t, cc));
     }
+    if (layer) {
+        // Sums of squares of k and q per token: this warp's 64 channels by a
+        // reduce-scatter over the lanes (slot s = lane: k of token s for
+        // s < 16, q of token s - 16), the two channel halves added after
+        // the next barrier.
+        const int lane = pt & 31;
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 kv = *reinterpret_cast<const __nv_bfloat162 *>(&k_v[i]);
+            const __nv_bfloat162 qv = *reinterpret_cast<const __nv_bfloat162 *>(&q_v[i]);
+            v[i] = __low2float(kv) * __low2float(kv) + __high2float(kv) * __high2float(kv);
+            v[16 + i] = __low2float(qv) * __low2float(qv) + __high2float(qv) * __high2float(qv);
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) {
+            const bool up = (lane & m) != 0;
+#pragma unroll
+            for (int j = 0; j < m; ++j) {
+                const float lo = v[j], hi = v[j + m];
+                const float send = up ? lo : hi;
+                const float keep = up ? hi : lo;
+                v[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            }
+        }
+        b.xf[katom * 128 + tg * 32 + lane] = v[0];
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        graw_v[i] = *reinterpret_cast<const uint32_t *>(b.graw + (t0 + i) * 256 + c * 2);
     float g0[16], g1[16];
     float r0 = 0.f, r1 = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162 *>(&graw_v[i]);
-        r0 = fmaf(clamp_log_alpha(__low2float(gv)), kLog2e, r0);
-        r1 = fmaf(clamp_log_alpha(__high2float(gv)), kLog2e, r1);
+        float x0 = __low2float(gv), x1 = __high2float(gv);
+        if (layer) {   // log_alpha = -e^A softplus(z); rows past the chunk end decay nothing
+            const bool valid = t0 + i < L;
+            x0 = valid ? b.neg_eA * (x0 > 15.f ? x0 : __logf(1.f + __expf(x0))) : 0.f;
+            x1 = valid ? b.neg_eA * (x1 > 15.f ? x1 : __logf(1.f + __expf(x1))) : 0.f;
+            *reinterpret_cast<uint32_t *>(const_cast<uint8_t *>(b.graw) + (t0 + i) * 256 + c * 2) =
+                pack_bf16x2(x0, x1);
+        }
+        r0 = fmaf(clamp_log_alpha(x0), kLog2e, r0);
+        r1 = fmaf(clamp_log_alpha(x1), kLog2e, r1);
         g0[i] = r0;
         g1[i] = r1;
     }
@@ -126,6 +171,11 @@ __device__ int gate(const Bufs &b, int pt, int L) {
     b.csum[tg * 128 + c + 1] = r1;
     if (pt == 0) *b.slow_flag = 0u;
     named_barrier(BAR, kGroupThreads);
+    if (layer && katom == 0) {   // one lane per (token, k / q): the inverse norm
+        const int lane = pt & 31;
+        const float tot = b.xf[tg * 32 + lane] + b.xf[128 + tg * 32 + lane];
+        b.nrm[(lane < 16 ? 0 : 64) + t0 + (lane & 15)] = rsqrtf(tot + b.qk_eps);
+    }
 
     float off0 = 0.f, off1 = 0.f, GL0 = 0.f, GL1 = 0.f;
 #pragma unroll
@@ -153,8 +203,9 @@ __device__ int gate(const Bufs &b, int pt, int L) {
         const int t = t0 + i;
         const __nv_bfloat162 kv = *reinterpret_cast<const __nv_bfloat162 *>(&k_v[i]);
         const __nv_bfloat162 qv = *reinterpret_cast<const __nv_bfloat162 *>(&q_v[i]);
-        const float k0 = __low2float(kv), k1 = __high2float(kv);
-        const float q0 = __low2float(qv), q1 = __high2float(qv);
+        const float nk = layer ? b.nrm[t] : 1.f, nq = layer ? b.nrm[64 + t] : 1.f;
+        const float k0 = __low2float(kv) * nk, k1 = __high2float(kv) * nk;
+        const float q0 = __low2float(qv) * nq, q1 = __high2float(qv) * nq;
         const float G0 = g0[i] + off0, G1 = g1[i] + off1;
         const float e0 = exp2_f(G0), e1 = exp2_f(G1);
         const float ih0 = exp2_f(fminf(-G0, kMaxInv2)), ih1 = exp2_f(fminf(-G1, kMaxInv2));
@@ -236,15 +287,16 @@ __device__ void secondary(const Bufs &b, int pt, int L, const __nv_bfloat16 *kt0
                 const int t = t0 + i;
                 const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(&kv[i]);
                 const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(&qv[i]);
+                const float nk = b.nrm ? b.nrm[t] : 1.f, nq = b.nrm ? b.nrm[64 + t] : 1.f;
                 const float e0 = exp2_f(G0[i] - ob0), e1 = exp2_f(G1[i] - ob1);
                 *reinterpret_cast<uint32_t *>(atom_a + sw128_off(t, cc)) =
-                    pack_bf16x2(__low2float(k2) * e0, __high2float(k2) * e1);
+                    pack_bf16x2(__low2float(k2) * (e0 * nk), __high2float(k2) * (e1 * nk));
                 *reinterpret_cast<uint32_t *>(atom_a + sw128_off(64 + t, cc)) =
-                    pack_bf16x2(__low2float(q2) * e0, __high2float(q2) * e1);
+                    pack_bf16x2(__low2float(q2) * (e0 * nq), __high2float(q2) * (e1 * nq));
                 if (tg == bb) {
                     const float f0 = exp2_f(ob0 - G0[i]), f1 = exp2_f(ob1 - G1[i]);
                     *reinterpret_cast<uint32_t *>(atom_c + sw128_off(i, cc)) =
-                        pack_bf16x2(__low2float(k2) * f0, __high2float(k2) * f1);
+                        pack_bf16x2(__low2float(k2) * (f0 * nk), __high2float(k2) * (f1 * nk));
                 }
             }
         }
@@ -342,6 +394,10 @@ __device__ void pairwise(const Bufs &b, int pt, int L, const __nv_bfloat16 *kt0,
         pq += __shfl_xor_sync(0xffffffffu, pq, 1);
         pq += __shfl_xor_sync(0xffffffffu, pq, 2);
         if (lead && active) {
+            if (b.nrm) {   // the dot products of the raw rows, scaled to the normalised ones
+                a *= b.nrm[t] * b.nrm[i];
+                pq *= b.nrm[64 + t] * b.nrm[i];
+            }
             b.af[fidx(t, i)] = (t > i) ? b.beta[t] * a : 0.f;
             *reinterpret_cast<__nv_bfloat16 *>(b.pb + sw128_off(t, i)) = __float2bfloat16_rn(pq);
         }

@@ -36,6 +36,26 @@ __device__ __forceinline__ float clamp_log_alpha(float g) {
     return fmaxf(g, kLogAlphaFloor);
 }
 
+// The layer's prologue and epilogue, fused into the kernels for the
+// kda_layer_* entry points (page "Kimi Linear" on docsaid.org, section "Les
+// autres pieces"; course page "Attention lineaire et recurrence", the gate
+// -e^A Softplus(z) of Kimi Linear):
+//   q, k <- x / sqrt(sum_c x_c^2 + qk_eps)           (L2 normalisation)
+//   log_alpha = -exp(A_log[h]) softplus(z),  beta = sigmoid(beta_logit)
+//   o <- o / sqrt(mean_j o_j^2 + norm_eps) * w_j * sigmoid(out_gate_j)
+struct LayerArgs {
+    const void *gate_z;        // [T, H, d_k], the I/O dtype
+    const float *A_log;        // [H] fp32
+    const void *beta_logit;    // [T, H], the I/O dtype
+    const void *out_gate;      // [T, H, d_v], the I/O dtype, or null (no output gate)
+    const float *norm_weight;  // [d_v] fp32, or null (ones)
+    float qk_eps, norm_eps;
+};
+
+__device__ __forceinline__ float softplus_f(float x) { return x > 20.f ? x : log1pf(expf(x)); }
+
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + expf(-x)); }
+
 // Error word written by device-side checks into the workspace header.
 enum : uint32_t {
     kDevErrNone = 0,
@@ -50,10 +70,13 @@ constexpr size_t kWorkspaceHeader = 256;
 // Launchers (defined in the .cu files).  All return cudaGetLastError().
 // `scalar_gate`: log_alpha holds one value per (token, head) ([T, H], the
 // Gated DeltaNet gate) instead of one per key channel ([T, H, d_k]).
+// `layer` (or null): the kda_layer_* prologue and epilogue; then g and beta
+// are unused.
 cudaError_t launch_decode(const void *q, const void *k, const void *v,
                           const void *g, const void *beta, float *state,
                           int batch, int H, int dk, int dv, kda_dtype dtype,
-                          void *o, bool scalar_gate, cudaStream_t stream);
+                          void *o, bool scalar_gate, const LayerArgs *layer,
+                          cudaStream_t stream);
 
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v,
                                 const void *g, const void *beta,
@@ -76,10 +99,12 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
 // state-chain kernel; its workspace holds one record per (chunk, head).
 size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H);
 
+// With `layer`, g is the gate pre-activation and beta the logits (bf16,
+// d = 128 only; the chain is then always whole-d_v).
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const void *g,
                                  const void *beta, const float *init_state, const int32_t *cu,
                                  int num_seqs, int64_t total_tokens, int H, void *o,
                                  float *final_state, void *workspace, bool scalar_gate,
-                                 cudaStream_t stream);
+                                 const LayerArgs *layer, cudaStream_t stream);
 
 }  // namespace kda

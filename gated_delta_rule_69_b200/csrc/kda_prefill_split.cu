@@ -76,7 +76,8 @@ struct PrepSmem {
     static constexpr uint32_t CSUM = 106240;   // 4 x 128 fp32
     static constexpr uint32_t BARS = 108288;   // 6 mbarriers
     static constexpr uint32_t MISC = 108352;   // tmem base, abort, slow flag, next-item slots at 4, 5
-    static constexpr uint32_t SIZE = 108416;
+    static constexpr uint32_t NRM = 108416;    // layer prologue: 128 fp32 inverse norms
+    static constexpr uint32_t SIZE = 108928;
     static constexpr uint32_t PIPE = 109568;   // per-pipeline stride
     static constexpr uint32_t ALLOC = 2 * PIPE + 1024;
 };
@@ -140,6 +141,13 @@ struct Params {
     const __nv_bfloat16 *k, *q, *beta;
     const __nv_bfloat16 *g;     // log_alpha [T, H] when scalar_gate
     int scalar_gate;
+    // layer prologue / epilogue (layer != 0): the g map carries the gate
+    // pre-activation, beta holds logits; the chain normalises and gates o
+    int layer;
+    const float *A_log;
+    const __nv_bfloat16 *out_gate;
+    const float *norm_weight;
+    float qk_eps, norm_eps;
     const float *init_state;
     float *final_state;
     __nv_bfloat16 *o;
@@ -320,7 +328,7 @@ __device__ __forceinline__ void write_qp(uint8_t *stk, uint32_t tmem, int quad, 
     }
 }
 
-template <int P>
+template <int P, bool LAYER>
 __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int tid, int warp, int lane,
                                               const CUtensorMap &tm_k, const CUtensorMap &tm_q,
                                               const CUtensorMap &tm_g, const Params &p,
@@ -373,7 +381,9 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
             mbar_arrive(&B[0]);
         }
         if (pt < C) {
-            beta[pt] = (pt < L) ? __bfloat162float(p.beta[(size_t)(tok0 + pt) * p.H + h]) : 0.f;
+            float bv = (pt < L) ? __bfloat162float(p.beta[(size_t)(tok0 + pt) * p.H + h]) : 0.f;
+            if (LAYER && pt < L) bv = 1.f / (1.f + __expf(-bv));   // beta = sigmoid(logit)
+            beta[pt] = bv;
             if (p.scalar_gate) {
                 // One log_alpha per token, broadcast over its 128 channels.  GRAW
                 // is a source of the previous record's stores: the leader has
@@ -406,9 +416,12 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         b.egl = reinterpret_cast<float *>(sm + PrepSmem::EGL);
         b.csum = reinterpret_cast<float *>(sm + PrepSmem::CSUM);
         b.slow_flag = misc + 2;
+        b.nrm = LAYER ? reinterpret_cast<float *>(sm + PrepSmem::NRM) : nullptr;
+        b.neg_eA = LAYER ? -__expf(p.A_log[h]) : 0.f;
+        b.qk_eps = p.qk_eps;
 
         mbar_wait(&B[0], it & 1, abort_flag);
-        const int form = prep::gate<BAR>(b, pt, L);
+        const int form = prep::gate<BAR, LAYER>(b, pt, L);
         fence_async_smem();
         named_barrier(BAR, prep::kGroupThreads);
         uint32_t drawn = 0;
@@ -539,6 +552,9 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
     }
 }
 
+// LAYER: the layer prologue (gate activation, q / k normalisation, beta
+// sigmoid) fused in; a separate instantiation keeps the plain kernel as it is.
+template <bool LAYER>
 __global__ void __launch_bounds__(kPrepThreads, 1)
 kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_g, const Params p) {
@@ -576,8 +592,8 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t total_items = *p.total_chunks * (uint32_t)p.H;
     const uint32_t tmem = misc0[0] + 256u * P;
     if (2 * blockIdx.x < total_items) {
-        if (P == 0) prep_pipeline<0>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
-        else prep_pipeline<1>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
+        if (P == 0) prep_pipeline<0, LAYER>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
+        else prep_pipeline<1, LAYER>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
     }
     tc_fence_before();
     __syncthreads();
@@ -894,7 +910,8 @@ struct ChainT {
     static constexpr uint32_t EGLR = RB + NSB * B_STRIDE;   // NSA x exp(G_L), 128 fp32 each
     static constexpr uint32_t BARS = EGLR + NSA * 512;
     static constexpr uint32_t MISC = BARS + 256;
-    static constexpr uint32_t SIZE = MISC + 64;
+    static constexpr uint32_t EPI = MISC + 64;              // layer epilogue: 2 x 4 x 4 x 16 fp32
+    static constexpr uint32_t SIZE = EPI + 2048;
     static constexpr uint32_t ALLOC = SIZE + 1024;
     // TMEM columns: S^T fp32 (128), SB^T bf16 pairs x 2 (64 each), O^T fp32 x 2 (64 each)
     static constexpr uint32_t TMEM_COLS = 512;
@@ -1066,6 +1083,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] = 0.f;
         }
+        const float wj = (p.layer && p.norm_weight) ? p.norm_weight[j] : 1.f;
         // O^T of chunk m: this warp's 16 t columns, lane j, bf16 to o[t][h][j]
         auto store_o_t = [&](int m) {
             mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
@@ -1074,6 +1092,37 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             tmem_ld16(tmem_addr(tmem, 32 * quad, Cfg::COL_O + 64 * (m & 1) + 16 * g), v);
             tmem_wait_ld();
             const int64_t t0 = (int64_t)m * C + 16 * g;
+            if (p.layer) {
+                // RMSNorm over d_v: this warp's 32 lanes by a reduce-scatter (lane
+                // ends with the sum for t = 16 g + lane mod 16), the four
+                // quadrant warps of column group g through shared memory
+                float r[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) r[i] = v[i] * v[i];
+#pragma unroll
+                for (int mm = 8; mm >= 1; mm >>= 1) {
+                    const bool up = (lane & mm) != 0;
+#pragma unroll
+                    for (int i = 0; i < mm; ++i) {
+                        const float lo = r[i], hi = r[i + mm];
+                        r[i] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, mm);
+                    }
+                }
+                r[0] += __shfl_xor_sync(0xffffffffu, r[0], 16);
+                float *ep = reinterpret_cast<float *>(sm + Cfg::EPI) + (m & 1) * 256 + g * 64;
+                if (lane < 16) ep[quad * 16 + lane] = r[0];
+                named_barrier(1 + g, 128);   // the four quadrant warps of column group g
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float ss = ep[i] + ep[16 + i] + ep[32 + i] + ep[48 + i];
+                    float y = v[i] * rsqrtf(ss * (1.f / DV) + p.norm_eps) * wj;
+                    if (p.out_gate && t0 + i < len) {
+                        const float og = __bfloat162float(p.out_gate[((size_t)(bos + t0 + i) * p.H + h) * DV + j]);
+                        y *= 1.f / (1.f + __expf(-og));
+                    }
+                    v[i] = y;
+                }
+            }
             __nv_bfloat16 *dst = p.o + ((size_t)(bos + t0) * p.H + h) * DV + j;
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -1368,13 +1417,13 @@ struct ChainPlan {
 };
 
 ChainPlan choose_chain(unsigned units, uint64_t items, int64_t total_tokens, int num_seqs,
-                       unsigned sm_count) {
+                       unsigned sm_count, bool whole_dv_only) {
     const double c_p = 12e3, sm = (double)sm_count;
     const double chunks = (double)((total_tokens / num_seqs + split::C - 1) / split::C);
     ChainPlan best = {128, false};
     double best_cost = -1.0;
     const int widths[2] = {32, 128};
-    for (int wi = 0; wi < 2; ++wi) {
+    for (int wi = whole_dv_only ? 1 : 0; wi < 2; ++wi) {
         const int dvt = widths[wi];
         const double per = dvt == 32 ? 1.6e3 : 2.7e3;
         const double ctas = (double)units * (split::DV / dvt);
@@ -1403,7 +1452,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                  const void *beta, const float *init_state, const int32_t *cu,
                                  int num_seqs, int64_t total_tokens, int H, void *o,
                                  float *final_state, void *workspace, bool scalar_gate,
-                                 cudaStream_t stream) {
+                                 const LayerArgs *layer, cudaStream_t stream) {
     using namespace split;
     const SplitLayout l = split_layout(num_seqs, total_tokens, H);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1433,8 +1482,9 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
             sm_count = 148;
     }
     const unsigned units = (unsigned)((size_t)num_seqs * H);
+    // the layer epilogue normalises whole rows of o: whole-d_v chain CTAs only
     const ChainPlan plan = choose_chain(units, (uint64_t)(total_tokens / C + num_seqs) * H, total_tokens,
-                                        num_seqs, (unsigned)sm_count);
+                                        num_seqs, (unsigned)sm_count, layer != nullptr);
     const bool overlap = plan.overlap;
     const unsigned chain_blocks = units * (unsigned)(DV / plan.dvt);
     uint32_t *rec_ready = overlap ? reinterpret_cast<uint32_t *>(ws + l.flags) : nullptr;
@@ -1446,7 +1496,10 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     if (e != cudaSuccess) return e;
     static bool attr_set = false;
     if (!attr_set) {
-        e = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(kda_prep_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)PrepSmem::ALLOC);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kda_prep_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)PrepSmem::ALLOC);
         if (e != cudaSuccess) return e;
         attr_set = true;
@@ -1457,6 +1510,12 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     prm.beta = static_cast<const __nv_bfloat16 *>(beta);
     prm.g = static_cast<const __nv_bfloat16 *>(g);
     prm.scalar_gate = scalar_gate ? 1 : 0;
+    prm.layer = layer ? 1 : 0;
+    prm.A_log = layer ? layer->A_log : nullptr;
+    prm.out_gate = layer ? static_cast<const __nv_bfloat16 *>(layer->out_gate) : nullptr;
+    prm.norm_weight = layer ? layer->norm_weight : nullptr;
+    prm.qk_eps = layer ? layer->qk_eps : 0.f;
+    prm.norm_eps = layer ? layer->norm_eps : 0.f;
     prm.init_state = init_state;
     prm.final_state = final_state;
     prm.o = static_cast<__nv_bfloat16 *>(o);
@@ -1486,7 +1545,8 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, kda_prep_kernel, mk, mq, mg, prm);
+        e = layer ? cudaLaunchKernelEx(&cfg, kda_prep_kernel<true>, mk, mq, mg, prm)
+                  : cudaLaunchKernelEx(&cfg, kda_prep_kernel<false>, mk, mq, mg, prm);
         if (e != cudaSuccess) return e;
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

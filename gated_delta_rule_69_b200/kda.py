@@ -20,7 +20,8 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUD
 KDA_BF16, KDA_FP32 = 0, 1
 EXPORTED = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
             "kda_prefill", "kda_decode_step", "kda_check_workspace_error",
-            "kda_prefill_noalloc", "gdn_prefill", "gdn_decode_step")
+            "kda_prefill_noalloc", "gdn_prefill", "gdn_decode_step", "kda_layer_prefill",
+            "kda_layer_decode_step")
 
 
 class KdaError(RuntimeError):
@@ -54,6 +55,13 @@ def lib():
         L.gdn_prefill.restype = ctypes.c_int
         L.gdn_decode_step.argtypes = L.kda_decode_step.argtypes
         L.gdn_decode_step.restype = ctypes.c_int
+        f32 = ctypes.c_float
+        L.kda_layer_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, f32, f32, vp, vp, i32, i64,
+                                        i32, i32, i32, ctypes.c_int, vp, vp, vp, sz, vp]
+        L.kda_layer_prefill.restype = ctypes.c_int
+        L.kda_layer_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, f32, f32, vp, i32, i32,
+                                            i32, i32, ctypes.c_int, vp, vp]
+        L.kda_layer_decode_step.restype = ctypes.c_int
         L.kda_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
                                           ctypes.c_int, vp, vp, vp]
         L.kda_prefill_noalloc.restype = ctypes.c_int
@@ -208,3 +216,64 @@ def kda_prefill_noalloc(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=No
     if st != KDA_OK:
         raise KdaError(st, "kda_prefill_noalloc")
     return o, final_state
+
+
+def kda_layer_prefill(q, k, v, gate_z, A_log, beta_logit, out_gate=None, norm_weight=None,
+                      qk_eps=1e-6, norm_eps=1e-6, init_state=None, cu_seqlens=None,
+                      num_seqs=None, o=None, final_state=None, workspace=None,
+                      output_final_state=True, stream=None):
+    """KDA prefill with the layer prologue / epilogue fused in (see
+    include/kda.h): raw q, k, gate pre-activation gate_z [T, H, d_k], A_log [H]
+    fp32, beta_logit [T, H]; optional out_gate [T, H, d_v] and norm_weight
+    [d_v] fp32.  bf16, d = 128."""
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    if gate_z.shape != q.shape or beta_logit.shape != q.shape[:2] or A_log.shape != (H,):
+        raise ValueError("gate_z [T, H, d_k], beta_logit [T, H], A_log [H] expected")
+    if A_log.dtype != torch.float32 or (norm_weight is not None and norm_weight.dtype != torch.float32):
+        raise TypeError("A_log and norm_weight must be float32")
+    if cu_seqlens is not None:
+        n = cu_seqlens.numel() - 1
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+    else:
+        n = 1 if num_seqs is None else int(num_seqs)
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = kda_prefill_workspace_size(n, T, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check_cuda(q, k, v, gate_z, A_log, beta_logit, out_gate, norm_weight, init_state,
+                cu_seqlens, o, final_state, workspace)
+    st = lib().kda_layer_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gate_z), _ptr(A_log), _ptr(beta_logit), _ptr(out_gate),
+        _ptr(norm_weight), float(qk_eps), float(norm_eps), _ptr(init_state), _ptr(cu_seqlens),
+        n, T, H, dk, dv, _dtype_code(q), _ptr(o), _ptr(final_state), _ptr(workspace),
+        workspace.numel(), _stream(stream, q.device))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_layer_prefill")
+    return o, final_state
+
+
+def kda_layer_decode_step(q, k, v, gate_z, A_log, beta_logit, state, out_gate=None,
+                          norm_weight=None, qk_eps=1e-6, norm_eps=1e-6, o=None, stream=None):
+    """One KDA step per sequence with the layer prologue / epilogue fused in;
+    ``state`` [B, H, d_k, d_v] fp32 is updated in place.  Returns o [B, H, d_v]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if gate_z.shape != q.shape or beta_logit.shape != q.shape[:2] or A_log.shape != (H,):
+        raise ValueError("gate_z [B, H, d_k], beta_logit [B, H], A_log [H] expected")
+    if A_log.dtype != torch.float32 or (norm_weight is not None and norm_weight.dtype != torch.float32):
+        raise TypeError("A_log and norm_weight must be float32")
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _check_cuda(q, k, v, gate_z, A_log, beta_logit, out_gate, norm_weight, state, o)
+    st = lib().kda_layer_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gate_z), _ptr(A_log), _ptr(beta_logit), _ptr(out_gate),
+        _ptr(norm_weight), float(qk_eps), float(norm_eps), _ptr(state), B, H, dk, dv,
+        _dtype_code(q), _ptr(o), _stream(stream, q.device))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_layer_decode_step")
+    return o

@@ -184,6 +184,47 @@ kda_status gdn_decode_step(const void *q, const void *k, const void *v,
                            kda_stream_t stream);
 
 /*
+ * The operator with the layer's prologue and epilogue fused in (page "Kimi
+ * Linear" on docsaid.org, section "Les autres pieces": q, k L2-normalised,
+ * beta a sigmoid, the decay a GDN / Mamba-like function of a pre-activation,
+ * the output RMS-normalised per head and multiplied by a data-dependent
+ * sigmoid gate; the course page "Attention lineaire et recurrence" gives
+ * Kimi Linear's decay as -e^A Softplus(z)):
+ *
+ *   q_t <- q_t / sqrt(|q_t|^2 + qk_eps),   k_t <- k_t / sqrt(|k_t|^2 + qk_eps)
+ *   log_alpha_t = -exp(A_log[h]) * softplus(gate_z_t)      (per key channel)
+ *   beta_t = sigmoid(beta_logit_t)
+ *   (the KDA recurrence of kda_prefill / kda_decode_step)
+ *   o_t <- o_t / sqrt(mean_j o_tj^2 + norm_eps) * norm_weight_j * sigmoid(out_gate_tj)
+ *
+ *   q, k, gate_z : [T, H, d_k] raw;  v : [T, H, d_v];  beta_logit : [T, H]
+ *   A_log        : [H] fp32 (device), required
+ *   out_gate     : [T, H, d_v] pre-sigmoid, or NULL (no output gate)
+ *   norm_weight  : [d_v] fp32 (device), or NULL (weight 1)
+ * Other arguments, layouts and errors as kda_prefill / kda_decode_step.
+ * kda_layer_prefill runs on the two-kernel tensor-core path only: bf16,
+ * d_k = d_v = 128 and a workspace of kda_prefill_workspace_size(...) bytes
+ * (else KDA_ERR_UNSUPPORTED / KDA_ERR_WORKSPACE); the state chain then always
+ * keeps whole rows of o in one CTA.  kda_layer_decode_step takes every shape
+ * kda_decode_step takes.  Weights of the projections that produce these
+ * activations are the caller's.
+ */
+kda_status kda_layer_prefill(const void *q, const void *k, const void *v, const void *gate_z,
+                             const float *A_log, const void *beta_logit, const void *out_gate,
+                             const float *norm_weight, float qk_eps, float norm_eps,
+                             const float *init_state, const int32_t *cu_seqlens,
+                             int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                             int32_t d_v, kda_dtype dtype, void *o, float *final_state,
+                             void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+kda_status kda_layer_decode_step(const void *q, const void *k, const void *v,
+                                 const void *gate_z, const float *A_log, const void *beta_logit,
+                                 const void *out_gate, const float *norm_weight, float qk_eps,
+                                 float norm_eps, float *state, int32_t batch, int32_t H,
+                                 int32_t d_k, int32_t d_v, kda_dtype dtype, void *o,
+                                 kda_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads the error word that the prefill kernels
  * leave at the start of `workspace` (non-zero when a device-side check failed,
  * e.g. cu_seqlens not non-decreasing or not ending at T_total).  Returns

@@ -170,3 +170,53 @@ def kda_decode_step(q, k, v, g, beta, state, nthreads: int = 0):
     cu = np.arange(B + 1, dtype=np.int64)
     return kda_recurrence(q, k, v, g, beta, init_state=state, cu_seqlens=cu,
                           nthreads=nthreads)
+
+
+# ---- the layer's prologue and epilogue around the recurrence ----------------
+# (page "Kimi Linear" on docsaid.org, section "Les autres pieces": q and k
+# L2-normalised, beta a sigmoid, the output RMS-normalised per head then gated
+# by a sigmoid; course page "Attention lineaire et recurrence": Kimi Linear's
+# decay -e^A Softplus(z).)  Elementwise, in fp64.
+
+def l2_normalize(x, eps):
+    """x / sqrt(sum over the last axis of x^2 + eps)."""
+    x = _f64(x)
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
+
+
+def softplus(z):
+    """log(1 + e^z), overflow-free: max(z, 0) + log1p(e^{-|z|})."""
+    z = _f64(z)
+    return np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))
+
+
+def sigmoid(x):
+    """1 / (1 + e^{-x}), as e^x / (1 + e^x) for x < 0 (no cancellation)."""
+    x = _f64(x)
+    e = np.exp(-np.abs(x))
+    return np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def kimi_log_alpha(gate_z, A_log):
+    """log alpha = -exp(A_log[h]) softplus(z); gate_z [T, H, d_k], A_log [H]."""
+    return -np.exp(_f64(A_log))[None, :, None] * softplus(gate_z)
+
+
+def rms_norm_gate(o, out_gate, norm_weight, eps):
+    """o / sqrt(mean over d_v of o^2 + eps) * w * sigmoid(out_gate) per (token, head)."""
+    o = _f64(o)
+    y = o / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
+    if norm_weight is not None:
+        y = y * _f64(norm_weight)
+    if out_gate is not None:
+        y = y * sigmoid(out_gate)
+    return y
+
+
+def kda_layer(q, k, v, gate_z, A_log, beta_logit, out_gate=None, norm_weight=None,
+              qk_eps=1e-6, norm_eps=1e-6, init_state=None, cu_seqlens=None, nthreads: int = 0):
+    """Prologue, the KDA recurrence, epilogue.  Returns (o, final_state)."""
+    o, fs = kda_recurrence(l2_normalize(q, qk_eps), l2_normalize(k, qk_eps), v,
+                           kimi_log_alpha(gate_z, A_log), sigmoid(beta_logit),
+                           init_state=init_state, cu_seqlens=cu_seqlens, nthreads=nthreads)
+    return rms_norm_gate(o, out_gate, norm_weight, norm_eps), fs

@@ -10,6 +10,8 @@ Each test names the plausible oracle mistake it catches:
   * state not reset per sequence                        -> varlen split invariant
   * Gated DeltaNet: gate inside the erase, or missing    -> scalar-gate commutation,
     scalar beta=0 closed form, orthonormal overwrite
+  * layer prologue / epilogue: a wrong axis, sign or
+    constant in the norms, softplus or sigmoid           -> closed forms and invariants
 """
 import json
 import math
@@ -334,3 +336,50 @@ def test_gdn_orthonormal_overwrite(oracle_mod):
     assert np.allclose(fs[0, 0], expect, atol=1e-12)
     for t in range(T):
         assert np.allclose(o[t, 0], v[t, 0], atol=1e-12)
+
+
+# --- the layer prologue and epilogue ---------------------------------------------
+
+def test_l2_normalize_unit_rows(oracle_mod):
+    rng = np.random.default_rng(51)
+    x = rng.normal(size=(7, 3, 16)) * 5.0
+    y = oracle_mod.l2_normalize(x, 0.0)
+    assert np.allclose(np.linalg.norm(y, axis=-1), 1.0, atol=1e-14)
+    # direction kept: y is x scaled by a positive number per row
+    ratio = y / x
+    assert np.allclose(ratio, ratio[..., :1], rtol=1e-12)
+    assert np.all(ratio > 0)
+    # a [3, 4] row has norm 5
+    assert np.allclose(oracle_mod.l2_normalize(np.array([3.0, 4.0]), 0.0), [0.6, 0.8])
+
+
+def test_kimi_gate_closed_forms(oracle_mod):
+    """log alpha = -e^A softplus(z): z = 0, A = 0 gives -ln 2; A = ln 3 triples
+    it; z -> +inf gives -e^A z; z -> -inf gives -e^A e^z."""
+    z = np.array([0.0, 0.0, 40.0, -40.0]).reshape(4, 1, 1)
+    A0 = np.zeros(1)
+    g = oracle_mod.kimi_log_alpha(z, A0)[:, 0, 0]
+    assert abs(g[0] + math.log(2.0)) < 1e-15
+    assert abs(g[2] + 40.0) < 1e-12
+    assert abs(g[3] + math.exp(-40.0)) < 1e-28
+    g3 = oracle_mod.kimi_log_alpha(z, np.array([math.log(3.0)]))[:, 0, 0]
+    assert abs(g3[0] + 3.0 * math.log(2.0)) < 1e-14
+    assert np.all(oracle_mod.kimi_log_alpha(np.linspace(-5, 5, 11).reshape(11, 1, 1), A0) < 0)
+
+
+def test_sigmoid_values(oracle_mod):
+    assert oracle_mod.sigmoid(0.0) == 0.5
+    assert abs(oracle_mod.sigmoid(math.log(3.0)) - 0.75) < 1e-15
+    assert abs(oracle_mod.sigmoid(-40.0) - math.exp(-40.0)) < 1e-30
+
+
+def test_rms_norm_gate(oracle_mod):
+    rng = np.random.default_rng(52)
+    o = rng.normal(size=(5, 2, 8)) * 3.0
+    y = oracle_mod.rms_norm_gate(o, None, None, 0.0)
+    assert np.allclose(np.sqrt(np.mean(y * y, axis=-1)), 1.0, atol=1e-14)   # unit RMS per row
+    w = rng.normal(size=8)
+    yw = oracle_mod.rms_norm_gate(o, np.zeros((5, 2, 8)), w, 0.0)
+    assert np.allclose(yw, 0.5 * y * w, atol=1e-14)                        # sigmoid(0) = 1/2
+    # RMS of (1, 1, 1, 1) * 2 is 2: the row becomes (1, 1, 1, 1)
+    assert np.allclose(oracle_mod.rms_norm_gate(np.full((1, 1, 4), 2.0), None, None, 0.0), 1.0)
