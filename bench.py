@@ -10,7 +10,8 @@ starts; L2 is flushed (a 256 MiB write) before every timed step, outside the
 timed interval.  The decode figures time chained kda_decode_step calls on the
 decode workload (state 512 MiB, larger than L2, so no flush is needed).  The
 "gdn_prefill" object times gdn_prefill (Gated DeltaNet: one gate value per
-token and head) on the prefill workload the same way.
+token and head) and "layer_prefill" times kda_layer_prefill (raw activations,
+the layer's prologue and epilogue fused) on the prefill workload the same way.
 Under torchrun every rank runs the same workload as an independent replica
 (the operator needs no exchange between GPUs); value = all ranks' tokens over
 the slowest rank's time.
@@ -42,9 +43,10 @@ DECODE_STEPS = 1000
 CHUNK = 64
 
 
-def prefill_work(w, lengths, scalar_gate=False):
+def prefill_work(w, lengths, scalar_gate=False, layer=False):
     """Algorithmic work of one prefill call; with ``scalar_gate`` (Gated
-    DeltaNet) log_alpha is one value per (token, head) instead of d_k."""
+    DeltaNet) log_alpha is one value per (token, head) instead of d_k; with
+    ``layer`` the fused layer also reads the output gate (d_v per token)."""
     T = sum(lengths)
     n = len(lengths)
     eb = 2 if w.dtype == "bf16" else 4
@@ -52,6 +54,8 @@ def prefill_work(w, lengths, scalar_gate=False):
     per_tok_bytes = (3 * w.d_k + 2 * w.d_v) * eb + eb
     if scalar_gate:
         per_tok_bytes -= (w.d_k - 1) * eb
+    if layer:
+        per_tok_bytes += w.d_v * eb
     state_bytes = n * w.H * w.d_k * w.d_v * 4 * (2 if w.init_std > 0 else 1)
     return dict(tokens=T, flop=per_tok_flop * T * w.H,
                 bytes=per_tok_bytes * T * w.H + state_bytes)
@@ -168,9 +172,10 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # --- the GPU arm -------------------------------------------------------------------
 
-def time_prefill(w, steps, warmup, world, scalar_gate=False):
+def time_prefill(w, steps, warmup, world, scalar_gate=False, layer=False):
     """kda_prefill (or, with ``scalar_gate``, gdn_prefill with channel 0 of
-    the gate draw as the per-head gate) on the workload, L2 flushed."""
+    the gate draw as the per-head gate; with ``layer``, kda_layer_prefill on
+    raw activations) on the workload, L2 flushed."""
     import torch
     from gated_delta_rule_69_b200 import inputs as kin
     from gated_delta_rule_69_b200 import kda
@@ -180,6 +185,24 @@ def time_prefill(w, steps, warmup, world, scalar_gate=False):
     if scalar_gate:
         g = g[..., 0].contiguous()
         fn = kda.gdn_prefill
+    if layer:
+        # raw activations of the same shapes: q, k ~ N(0, 2^2), gate
+        # pre-activation ~ N(-1, 1), A_log ~ N(0, 0.25^2), beta logits and
+        # output-gate pre-activations ~ N(0, 1), RMSNorm weight 1 + N(0, 0.1^2)
+        gen = torch.Generator(device="cuda").manual_seed(w.seed + 7)
+        T0, H0, dk0 = q.shape
+        rn = lambda *sh: torch.randn(*sh, generator=gen, device="cuda")
+        q = (rn(T0, H0, dk0) * 2.0).to(q.dtype)
+        k = (rn(T0, H0, dk0) * 2.0).to(q.dtype)
+        g = (rn(T0, H0, dk0) - 1.0).to(q.dtype)
+        b = rn(T0, H0).to(q.dtype)
+        A_log = rn(H0) * 0.25
+        out_gate = rn(T0, H0, v.shape[-1]).to(q.dtype)
+        norm_weight = 1.0 + 0.1 * rn(v.shape[-1])
+
+        def fn(q, k, v, g, b, **kw):
+            return kda.kda_layer_prefill(q, k, v, g, A_log, b, out_gate=out_gate,
+                                         norm_weight=norm_weight, **kw)
     T, H, dk = q.shape
     dv = v.shape[-1]
     n = len(inp["lengths"])
@@ -411,6 +434,7 @@ def main():
     dw = kin.WORKLOADS[args.decode_workload]
     dec = time_decode(dw, args.decode_steps, args.warmup, world)
     gdn = time_prefill(w, args.steps, args.warmup, world, scalar_gate=True)
+    lay = time_prefill(w, args.steps, args.warmup, world, layer=True)
     clocks = sampler.stop()
 
     lengths = pf["inputs"]["lengths"]
@@ -425,6 +449,9 @@ def main():
     gwork = prefill_work(w, lengths, scalar_gate=True)
     gms = max_over_ranks(gdn["ms_total"] / args.steps, world)
     ggbs = gwork["bytes"] / (gms * 1e-3) / 1e9
+    lwork = prefill_work(w, lengths, layer=True)
+    lms = max_over_ranks(lay["ms_total"] / args.steps, world)
+    lgbs = lwork["bytes"] / (lms * 1e-3) / 1e9
     src = "of " + peaks["source"]
 
     line = {
@@ -451,7 +478,15 @@ def main():
                                      "unit": "GB/s", "frac": ggbs / peaks["hbm"], "traffic": None,
                                      "peak_source": src, "kernel": "gdn_prefill",
                                      "algorithmic_bytes_per_launch": gwork["bytes"]}},
-        "gpu_launches": pf["launches"] + dec["launches"] + gdn["launches"],
+        "layer_prefill": {"workload": w.name + ", raw activations, layer prologue and epilogue fused",
+                          "value": world * lwork["tokens"] / (lms * 1e-3), "unit": "tokens/s",
+                          "ms_per_step": lms, "steps": args.steps,
+                          "roofline": {"bound": "hbm", "achieved": lgbs, "peak": peaks["hbm"],
+                                       "unit": "GB/s", "frac": lgbs / peaks["hbm"],
+                                       "traffic": None, "peak_source": src,
+                                       "kernel": "kda_layer_prefill",
+                                       "algorithmic_bytes_per_launch": lwork["bytes"]}},
+        "gpu_launches": pf["launches"] + dec["launches"] + gdn["launches"] + lay["launches"],
         "clocks": clocks,
     }
     if not args.no_e2e:

@@ -1109,17 +1109,49 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                     }
                 }
                 r[0] += __shfl_xor_sync(0xffffffffu, r[0], 16);
+                // partials as [t][quadrant], so that a thread reads a t's four with one load
                 float *ep = reinterpret_cast<float *>(sm + Cfg::EPI) + (m & 1) * 256 + g * 64;
-                if (lane < 16) ep[quad * 16 + lane] = r[0];
+                if (lane < 16) ep[lane * 4 + quad] = r[0];
                 named_barrier(1 + g, 128);   // the four quadrant warps of column group g
+                // the output gate (its rows were sent towards L2 a chunk earlier);
+                // loaded only here, after the state hand-off, whose release
+                // would otherwise wait for these loads
+                float og[16];
+                if (p.out_gate) {
+                    // sixteen rows 8 KB apart: issued together in one block (left to
+                    // itself the compiler interleaves each load with its use);
+                    // rows past the end read the last row and are not stored
+                    const __nv_bfloat16 *a[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int64_t tt = t0 + i < len ? t0 + i : len - 1;
+                        a[i] = p.out_gate + ((size_t)(bos + tt) * p.H + h) * DV + j;
+                    }
+                    unsigned short u[16];
+                    asm volatile(
+                        "ld.global.nc.b16 %0, [%16];\n\tld.global.nc.b16 %1, [%17];\n\t"
+                        "ld.global.nc.b16 %2, [%18];\n\tld.global.nc.b16 %3, [%19];\n\t"
+                        "ld.global.nc.b16 %4, [%20];\n\tld.global.nc.b16 %5, [%21];\n\t"
+                        "ld.global.nc.b16 %6, [%22];\n\tld.global.nc.b16 %7, [%23];\n\t"
+                        "ld.global.nc.b16 %8, [%24];\n\tld.global.nc.b16 %9, [%25];\n\t"
+                        "ld.global.nc.b16 %10, [%26];\n\tld.global.nc.b16 %11, [%27];\n\t"
+                        "ld.global.nc.b16 %12, [%28];\n\tld.global.nc.b16 %13, [%29];\n\t"
+                        "ld.global.nc.b16 %14, [%30];\n\tld.global.nc.b16 %15, [%31];"
+                        : "=h"(u[0]), "=h"(u[1]), "=h"(u[2]), "=h"(u[3]), "=h"(u[4]), "=h"(u[5]),
+                          "=h"(u[6]), "=h"(u[7]), "=h"(u[8]), "=h"(u[9]), "=h"(u[10]), "=h"(u[11]),
+                          "=h"(u[12]), "=h"(u[13]), "=h"(u[14]), "=h"(u[15])
+                        : "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(a[4]), "l"(a[5]),
+                          "l"(a[6]), "l"(a[7]), "l"(a[8]), "l"(a[9]), "l"(a[10]), "l"(a[11]),
+                          "l"(a[12]), "l"(a[13]), "l"(a[14]), "l"(a[15]));
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) og[i] = __bfloat162float(__ushort_as_bfloat16(u[i]));
+                }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float ss = ep[i] + ep[16 + i] + ep[32 + i] + ep[48 + i];
+                    const float4 pq = reinterpret_cast<const float4 *>(ep)[i];
+                    const float ss = (pq.x + pq.y) + (pq.z + pq.w);
                     float y = v[i] * rsqrtf(ss * (1.f / DV) + p.norm_eps) * wj;
-                    if (p.out_gate && t0 + i < len) {
-                        const float og = __bfloat162float(p.out_gate[((size_t)(bos + t0 + i) * p.H + h) * DV + j]);
-                        y *= 1.f / (1.f + __expf(-og));
-                    }
+                    if (p.out_gate) y *= 1.f / (1.f + __expf(-og[i]));
                     v[i] = y;
                 }
             }
@@ -1130,6 +1162,15 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         };
         for (int n = 0; n < nchunks; ++n) {
             const int sa = n % NSA;
+            if (p.layer && p.out_gate) {
+                // chunk n's output-gate rows towards L2 for the next iteration
+                const int64_t tp = (int64_t)n * C + 16 * g;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (tp + i < len)
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(
+                            p.out_gate + ((size_t)(bos + tp + i) * p.H + h) * DV + j));
+            }
             if (n >= 1) {
                 mbar_wait(SDONE, (n - 1) & 1, abort_flag);
                 tc_fence_after();
