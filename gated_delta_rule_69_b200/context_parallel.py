@@ -1,0 +1,67 @@
+"""KDA context parallelism: one sequence cut into consecutive segments, one per
+rank (course page "Attention lineaire et recurrence", section "Verification de
+comprehension": a segment carries its cumulative transition M and the state it
+generates locally, S~; the state entering segment r is S_in(r) = M_{r-1}
+S_in(r-1) + S~_{r-1}).
+
+Per rank, all on the GPU in the library's kernels:
+  1. local pass: S~ = final state of kda_prefill on the segment from a zero
+     state; M = final state of kda_prefill on the segment with v = 0 and the
+     identity as initial state (the chain then multiplies the transitions);
+  2. exchange: all-gather of (M, S~) over the group (NCCL over NVLink);
+  3. combine: kda_cp_combine forms S_in(rank) from the pairs of lower ranks;
+  4. final pass: kda_prefill on the segment from S_in(rank): the outputs, and
+     on the last rank the sequence's final state.
+The pages give the decomposition, not a schedule; this one spends three
+preparation passes per rank (the local pair and the final pass each run one),
+which a library call that keeps the first pass's records would avoid.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import kda
+
+
+def local_pair(q, k, v, log_alpha, beta, workspace=None, stream=None):
+    """(M, S~) of one segment, each [1, H, d_k, d_*]."""
+    T, H, dk = q.shape
+    if v.shape[-1] != dk:
+        raise ValueError("context parallelism needs d_v = d_k (M is d_k x d_k)")
+    _, s_tilde = kda.kda_prefill(q, k, v, log_alpha, beta, workspace=workspace, stream=stream)
+    eye = torch.eye(dk, dtype=torch.float32, device=q.device).expand(1, H, dk, dk).contiguous()
+    _, m = kda.kda_prefill(q, k, torch.zeros_like(v), log_alpha, beta, init_state=eye,
+                           workspace=workspace, stream=stream)
+    return m, s_tilde
+
+
+def exchange(m, s_tilde, group=None):
+    """All-gather of every rank's (M, S~): returns [world, H, d_k, d_*] each, in
+    rank order."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    ms = [torch.empty_like(m) for _ in range(world)]
+    ss = [torch.empty_like(s_tilde) for _ in range(world)]
+    dist.all_gather(ms, m.contiguous(), group=group)
+    dist.all_gather(ss, s_tilde.contiguous(), group=group)
+    return torch.cat(ms), torch.cat(ss)
+
+
+def cp_prefill(q, k, v, log_alpha, beta, init_state=None, group=None, workspace=None,
+               stream=None, exchange_fn=None, rank=None):
+    """Context-parallel KDA prefill of one sequence.  This rank holds the
+    segment q, k, v, log_alpha, beta ([T_r, H, ...]) at position `rank` (its
+    rank in `group`); init_state [1, H, d_k, d_v] is the sequence's initial
+    state, the same on every rank (or None).  Returns (o for the segment, the
+    state after it); the last rank's is the sequence's final state.
+    ``exchange_fn(m, s_tilde)`` replaces the collective (returns the stacked
+    pairs of all ranks), e.g. to run the ranks one after another on one GPU."""
+    if rank is None:
+        import torch.distributed as dist
+        rank = dist.get_rank(group)
+    m, s_tilde = local_pair(q, k, v, log_alpha, beta, workspace=workspace, stream=stream)
+    ms, ss = exchange_fn(m, s_tilde) if exchange_fn is not None else exchange(m, s_tilde, group)
+    s0 = None if init_state is None else init_state.reshape(init_state.shape[-3:]).contiguous()
+    s_in = kda.kda_cp_combine(ms[:rank].contiguous(), ss[:rank].contiguous(), s0, stream=stream)
+    return kda.kda_prefill(q, k, v, log_alpha, beta, init_state=s_in.unsqueeze(0),
+                           workspace=workspace, stream=stream)

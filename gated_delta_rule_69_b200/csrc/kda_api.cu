@@ -237,6 +237,24 @@ kda_status kda_layer_decode_step(const void *q, const void *k, const void *v,
                        false, &la);
 }
 
+kda_status kda_cp_combine(const float *M, const float *S_tilde, const float *S0, float *S_in,
+                          int32_t n_prev, int32_t H, int32_t d_k, int32_t d_v,
+                          kda_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (n_prev < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (!supported_dim(d_k) || !supported_dim(d_v) || d_v < 32) return KDA_ERR_UNSUPPORTED;
+    if (!S_in || (n_prev > 0 && (!M || !S_tilde))) return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {M, S_tilde, S0, S_in};
+    for (const void *p : ptrs)
+        if (p && !aligned_to(p, 4)) return KDA_ERR_INVALID_ARG;
+    const size_t ns = (size_t)H * d_k * d_v * sizeof(float);
+    const size_t nm = (size_t)n_prev * H * d_k * d_k * sizeof(float);
+    if (overlaps(S_in, ns, M, nm) || overlaps(S_in, ns, S_tilde, (size_t)n_prev * ns) ||
+        (S0 && S0 != S_in && overlaps(S_in, ns, S0, ns)))
+        return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_cp_combine(M, S_tilde, S0, S_in, n_prev, H, d_k, d_v, stream));
+}
+
 kda_status kda_check_workspace_error(const void *workspace, kda_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (!workspace) return KDA_ERR_INVALID_ARG;

@@ -107,4 +107,9 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                  float *final_state, void *workspace, bool scalar_gate,
                                  const LayerArgs *layer, cudaStream_t stream);
 
+// Context parallelism: S_out = the state a segment starts from, given the
+// (M_i, S~_i) of the n_prev segments before it and the sequence's S_0 (or null).
+cudaError_t launch_cp_combine(const float *M, const float *S_tilde, const float *S0, float *S_out,
+                              int n_prev, int H, int dk, int dv, cudaStream_t stream);
+
 }  // namespace kda

@@ -21,7 +21,7 @@ KDA_BF16, KDA_FP32 = 0, 1
 EXPORTED = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
             "kda_prefill", "kda_decode_step", "kda_check_workspace_error",
             "kda_prefill_noalloc", "gdn_prefill", "gdn_decode_step", "kda_layer_prefill",
-            "kda_layer_decode_step")
+            "kda_layer_decode_step", "kda_cp_combine")
 
 
 class KdaError(RuntimeError):
@@ -62,6 +62,8 @@ def lib():
         L.kda_layer_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, f32, f32, vp, i32, i32,
                                             i32, i32, ctypes.c_int, vp, vp]
         L.kda_layer_decode_step.restype = ctypes.c_int
+        L.kda_cp_combine.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
+        L.kda_cp_combine.restype = ctypes.c_int
         L.kda_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
                                           ctypes.c_int, vp, vp, vp]
         L.kda_prefill_noalloc.restype = ctypes.c_int
@@ -277,3 +279,19 @@ def kda_layer_decode_step(q, k, v, gate_z, A_log, beta_logit, state, out_gate=No
     if st != KDA_OK:
         raise KdaError(st, "kda_layer_decode_step")
     return o
+
+
+def kda_cp_combine(M, S_tilde, S0=None, S_in=None, stream=None):
+    """The state a segment starts from, given the stacked (M, S~) of the
+    segments before it: M [n, H, d_k, d_k], S_tilde [n, H, d_k, d_v] fp32, S0
+    [H, d_k, d_v] or None.  Returns S_in [H, d_k, d_v]."""
+    n, H, dk, _ = M.shape
+    dv = S_tilde.shape[-1]
+    if S_in is None:
+        S_in = torch.empty((H, dk, dv), dtype=torch.float32, device=M.device)
+    _check_cuda(M, S_tilde, S0, S_in)
+    st = lib().kda_cp_combine(_ptr(M), _ptr(S_tilde), _ptr(S0), _ptr(S_in), n, H, dk, dv,
+                              _stream(stream, M.device))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_cp_combine")
+    return S_in

@@ -225,6 +225,28 @@ kda_status kda_layer_decode_step(const void *q, const void *k, const void *v,
                                  kda_stream_t stream);
 
 /*
+ * Context parallelism across devices (course page "Attention lineaire et
+ * recurrence", section "Verification de comprehension": a segment of a
+ * sequence acts on the state it receives through its cumulative transition
+ * M = prod_t (I - beta_t k_t k_t^T) Diag(alpha_t), then adds the state it
+ * generates from zero, S~).  A device holding segment r starts from
+ *     S_in(0) = S_0,   S_in(i + 1) = M_i S_in(i) + S~_i,   i < r.
+ * This call forms S_in(n_prev) from the gathered pairs of the n_prev segments
+ * before it:
+ *   M       : [n_prev, H, d_k, d_k] fp32;   S_tilde : [n_prev, H, d_k, d_v] fp32
+ *   S0      : [H, d_k, d_v] fp32 or NULL (zero);   S_in : [H, d_k, d_v] fp32, written
+ * n_prev = 0 copies S0 (or writes zeros).  A segment's M is the final state
+ * of kda_prefill on that segment with v = 0 (d_v = d_k) and the identity as
+ * initial state; S~ is its final state from a zero state (the Python module
+ * context_parallel.py does this and the exchange).  Supported: d_k in
+ * {16, 32, 64, 128}, d_v in {32, 64, 128}; 4-byte aligned pointers; S_in must
+ * not overlap M or S_tilde.
+ */
+kda_status kda_cp_combine(const float *M, const float *S_tilde, const float *S0, float *S_in,
+                          int32_t n_prev, int32_t H, int32_t d_k, int32_t d_v,
+                          kda_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads the error word that the prefill kernels
  * leave at the start of `workspace` (non-zero when a device-side check failed,
  * e.g. cu_seqlens not non-decreasing or not ending at T_total).  Returns
