@@ -37,7 +37,9 @@ __device__ __forceinline__ float4 fma4(float4 a, float s, float4 acc) {
     return acc;
 }
 
-template <typename T, int DK, int DV>
+// LAYER: the layer prologue / epilogue (kda_layer_decode_step); a separate
+// instantiation keeps the plain step as lean as before.
+template <typename T, int DK, int DV, bool LAYER>
 __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
 kda_decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
                   const T *__restrict__ v, const T *__restrict__ g,
@@ -49,8 +51,8 @@ kda_decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
     __shared__ __align__(16) float red_k[R][DV];
     __shared__ __align__(16) float red_q[R][DV];
     __shared__ float s_kq, s_nk, s_nq, s_no;
-    __shared__ float so[DV];
-    const bool layer = la.gate_z != nullptr;
+    __shared__ float so[LAYER ? DV : 1];
+    constexpr bool layer = LAYER;
 
     const int tid = threadIdx.x;
     const int lx = tid % LX;
@@ -172,11 +174,18 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v,
                          cudaStream_t stream) {
     const unsigned blocks = (unsigned)((size_t)batch * (size_t)H);
     LayerArgs la = {};
-    if (layer) la = *layer;
-    kda_decode_kernel<T, DK, DV><<<blocks, DecodeShape<DK, DV>::NT, 0, stream>>>(
-        static_cast<const T *>(q), static_cast<const T *>(k),
-        static_cast<const T *>(v), static_cast<const T *>(g),
-        static_cast<const T *>(beta), state, static_cast<T *>(o), sg ? 1 : DK, sg ? 0 : 1, H, la);
+    if (layer) {
+        la = *layer;
+        kda_decode_kernel<T, DK, DV, true><<<blocks, DecodeShape<DK, DV>::NT, 0, stream>>>(
+            static_cast<const T *>(q), static_cast<const T *>(k),
+            static_cast<const T *>(v), static_cast<const T *>(g),
+            static_cast<const T *>(beta), state, static_cast<T *>(o), sg ? 1 : DK, sg ? 0 : 1, H, la);
+    } else {
+        kda_decode_kernel<T, DK, DV, false><<<blocks, DecodeShape<DK, DV>::NT, 0, stream>>>(
+            static_cast<const T *>(q), static_cast<const T *>(k),
+            static_cast<const T *>(v), static_cast<const T *>(g),
+            static_cast<const T *>(beta), state, static_cast<T *>(o), sg ? 1 : DK, sg ? 0 : 1, H, la);
+    }
     return cudaGetLastError();
 }
 

@@ -920,6 +920,9 @@ struct ChainT {
     static_assert(2 * NSA + 2 * NSB + 2 * NSV + 5 <= 32, "barrier area");
 };
 
+// LAYER: the layer epilogue on o (a separate instantiation keeps the plain
+// chain as lean as before).
+template <bool LAYER>
 __global__ void __launch_bounds__(ChainT::THREADS, 1)
 kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     using Cfg = ChainT;
@@ -1083,7 +1086,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] = 0.f;
         }
-        const float wj = (p.layer && p.norm_weight) ? p.norm_weight[j] : 1.f;
+        const float wj = (LAYER && p.norm_weight) ? p.norm_weight[j] : 1.f;
         // O^T of chunk m: this warp's 16 t columns, lane j, bf16 to o[t][h][j]
         auto store_o_t = [&](int m) {
             mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
@@ -1092,7 +1095,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             tmem_ld16(tmem_addr(tmem, 32 * quad, Cfg::COL_O + 64 * (m & 1) + 16 * g), v);
             tmem_wait_ld();
             const int64_t t0 = (int64_t)m * C + 16 * g;
-            if (p.layer) {
+            if (LAYER) {
                 // RMSNorm over d_v: this warp's 32 lanes by a reduce-scatter (lane
                 // ends with the sum for t = 16 g + lane mod 16), the four
                 // quadrant warps of column group g through shared memory
@@ -1162,7 +1165,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         };
         for (int n = 0; n < nchunks; ++n) {
             const int sa = n % NSA;
-            if (p.layer && p.out_gate) {
+            if (LAYER && p.out_gate) {
                 // chunk n's output-gate rows towards L2 for the next iteration
                 const int64_t tp = (int64_t)n * C + 16 * g;
 #pragma unroll
@@ -1418,9 +1421,12 @@ cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const spl
         return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(kda_chain_t_kernel,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)ChainT::ALLOC);
+        cudaError_t e = cudaFuncSetAttribute(kda_chain_t_kernel<false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)ChainT::ALLOC);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kda_chain_t_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)ChainT::ALLOC);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -1434,7 +1440,8 @@ cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const spl
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = overlap ? 1 : 0;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kda_chain_t_kernel, mv, prm);
+    const cudaError_t e = prm.layer ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<true>, mv, prm)
+                                    : cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<false>, mv, prm);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
