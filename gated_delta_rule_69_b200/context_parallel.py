@@ -4,17 +4,16 @@ comprehension": a segment carries its cumulative transition M and the state it
 generates locally, S~; the state entering segment r is S_in(r) = M_{r-1}
 S_in(r-1) + S~_{r-1}).
 
-Per rank, all on the GPU in the library's kernels:
-  1. local pass: S~ = final state of kda_prefill on the segment from a zero
-     state; M = final state of kda_prefill on the segment with v = 0 and the
-     identity as initial state (the chain then multiplies the transitions);
+Per rank, all on the GPU in the library's kernels, with one chunk
+preparation:
+  1. kda_cp_local: the segment's chunk records, then over them the state
+     chain from zero (S~) and from the identity with v counting as zero (M);
   2. exchange: all-gather of (M, S~) over the group (NCCL over NVLink);
-  3. combine: kda_cp_combine forms S_in(rank) from the pairs of lower ranks;
-  4. final pass: kda_prefill on the segment from S_in(rank): the outputs, and
-     on the last rank the sequence's final state.
-The pages give the decomposition, not a schedule; this one spends three
-preparation passes per rank (the local pair and the final pass each run one),
-which a library call that keeps the first pass's records would avoid.
+  3. kda_cp_combine forms S_in(rank) from the pairs of lower ranks;
+  4. kda_cp_finish: the chain once more over the same records from S_in(rank):
+     the outputs, and on the last rank the sequence's final state.
+The pages give the decomposition, not a schedule: this one runs the chain
+three times per rank (two before the exchange), the preparation once.
 """
 from __future__ import annotations
 
@@ -23,16 +22,20 @@ import torch
 from . import kda
 
 
-def local_pair(q, k, v, log_alpha, beta, workspace=None, stream=None):
-    """(M, S~) of one segment, each [1, H, d_k, d_*]."""
+def workspace_for(q):
     T, H, dk = q.shape
-    if v.shape[-1] != dk:
+    n = kda.kda_prefill_workspace_size(1, T, H, dk, dk)
+    return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+
+def local_pair(q, k, v, log_alpha, beta, workspace=None, stream=None):
+    """(M, S~) of one segment, each [1, H, d_k, d_*]; the segment's chunk
+    records stay in ``workspace`` (allocated if None) for the final pass."""
+    if v.shape[-1] != q.shape[-1]:
         raise ValueError("context parallelism needs d_v = d_k (M is d_k x d_k)")
-    _, s_tilde = kda.kda_prefill(q, k, v, log_alpha, beta, workspace=workspace, stream=stream)
-    eye = torch.eye(dk, dtype=torch.float32, device=q.device).expand(1, H, dk, dk).contiguous()
-    _, m = kda.kda_prefill(q, k, torch.zeros_like(v), log_alpha, beta, init_state=eye,
-                           workspace=workspace, stream=stream)
-    return m, s_tilde
+    if workspace is None:
+        workspace = workspace_for(q)
+    return kda.kda_cp_local(q, k, v, log_alpha, beta, workspace, stream=stream)
 
 
 def exchange(m, s_tilde, group=None):
@@ -59,9 +62,10 @@ def cp_prefill(q, k, v, log_alpha, beta, init_state=None, group=None, workspace=
     if rank is None:
         import torch.distributed as dist
         rank = dist.get_rank(group)
+    if workspace is None:
+        workspace = workspace_for(q)
     m, s_tilde = local_pair(q, k, v, log_alpha, beta, workspace=workspace, stream=stream)
     ms, ss = exchange_fn(m, s_tilde) if exchange_fn is not None else exchange(m, s_tilde, group)
     s0 = None if init_state is None else init_state.reshape(init_state.shape[-3:]).contiguous()
     s_in = kda.kda_cp_combine(ms[:rank].contiguous(), ss[:rank].contiguous(), s0, stream=stream)
-    return kda.kda_prefill(q, k, v, log_alpha, beta, init_state=s_in.unsqueeze(0),
-                           workspace=workspace, stream=stream)
+    return kda.kda_cp_finish(v, s_in.unsqueeze(0), workspace, stream=stream)

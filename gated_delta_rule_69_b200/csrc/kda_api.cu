@@ -255,6 +255,61 @@ kda_status kda_cp_combine(const float *M, const float *S_tilde, const float *S0,
     return from_cuda(kda::launch_cp_combine(M, S_tilde, S0, S_in, n_prev, H, d_k, d_v, stream));
 }
 
+kda_status kda_cp_local(const void *q, const void *k, const void *v, const void *log_alpha,
+                        const void *beta, int64_t total_tokens, int32_t H, int32_t d_k,
+                        int32_t d_v, kda_dtype dtype, float *M, float *S_tilde, void *o_scratch,
+                        void *workspace, size_t workspace_bytes, kda_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (total_tokens < 1 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (!use_tensor_cores(dtype, d_k, d_v, total_tokens)) return KDA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !log_alpha || !beta || !M || !S_tilde || !o_scratch)
+        return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, M, S_tilde, o_scratch};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (!aligned_to(beta, 2)) return KDA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kda::prefill_split_workspace(1, total_tokens, H))
+        return KDA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_INVALID_ARG;
+    const size_t nk = (size_t)total_tokens * H * d_k * 2, nb = (size_t)total_tokens * H * 2;
+    const size_t ns = (size_t)H * d_k * d_v * sizeof(float);
+    const void *ins[] = {q, k, v, log_alpha};
+    for (const void *in : ins)
+        if (overlaps(M, ns, in, nk) || overlaps(S_tilde, ns, in, nk) || overlaps(o_scratch, nk, in, nk))
+            return KDA_ERR_INVALID_ARG;
+    if (overlaps(M, ns, S_tilde, ns) || overlaps(M, ns, o_scratch, nk) ||
+        overlaps(S_tilde, ns, o_scratch, nk) || overlaps(o_scratch, nk, beta, nb) ||
+        overlaps(o_scratch, nk, workspace, workspace_bytes))
+        return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_prefill_split(q, k, v, log_alpha, beta, nullptr, nullptr, 1,
+                                               total_tokens, H, o_scratch, S_tilde, workspace,
+                                               false, nullptr, stream, kda::kCpLocal, M));
+}
+
+kda_status kda_cp_finish(const void *v, const float *S_in, int64_t total_tokens, int32_t H,
+                         int32_t d_k, int32_t d_v, kda_dtype dtype, void *o, float *final_state,
+                         void *workspace, size_t workspace_bytes, kda_stream_t stream_) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (total_tokens < 1 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (!use_tensor_cores(dtype, d_k, d_v, total_tokens)) return KDA_ERR_UNSUPPORTED;
+    if (!v || !o) return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {v, S_in, o, final_state};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kda::prefill_split_workspace(1, total_tokens, H))
+        return KDA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_INVALID_ARG;
+    const size_t nv = (size_t)total_tokens * H * d_v * 2;
+    const size_t ns = (size_t)H * d_k * d_v * sizeof(float);
+    if (overlaps(o, nv, v, nv) || overlaps(o, nv, S_in, ns) || overlaps(o, nv, final_state, ns) ||
+        overlaps(o, nv, workspace, workspace_bytes) ||
+        (S_in && final_state && S_in != final_state && overlaps(S_in, ns, final_state, ns)))
+        return KDA_ERR_INVALID_ARG;
+    return from_cuda(kda::launch_prefill_split(nullptr, nullptr, v, nullptr, nullptr, S_in, nullptr,
+                                               1, total_tokens, H, o, final_state, workspace,
+                                               false, nullptr, stream, kda::kCpFinish, nullptr));
+}
+
 kda_status kda_check_workspace_error(const void *workspace, kda_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (!workspace) return KDA_ERR_INVALID_ARG;

@@ -101,11 +101,18 @@ size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H);
 
 // With `layer`, g is the gate pre-activation and beta the logits (bf16,
 // d = 128 only; the chain is then always whole-d_v).
+// cp_mode (context parallelism, one segment of a sequence): kCpLocal also
+// forms the segment's transition into cp_transition [N, H, d_k, d_k]
+// (final_state then receives the state generated from init_state, o is
+// scratch); kCpFinish runs only the chain over the records a kCpLocal call
+// left in the same workspace.
+enum : int { kCpNone = 0, kCpLocal = 1, kCpFinish = 2 };
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const void *g,
                                  const void *beta, const float *init_state, const int32_t *cu,
                                  int num_seqs, int64_t total_tokens, int H, void *o,
                                  float *final_state, void *workspace, bool scalar_gate,
-                                 const LayerArgs *layer, cudaStream_t stream);
+                                 const LayerArgs *layer, cudaStream_t stream,
+                                 int cp_mode = kCpNone, float *cp_transition = nullptr);
 
 // Context parallelism: S_out = the state a segment starts from, given the
 // (M_i, S~_i) of the n_prev segments before it and the sequence's S_0 (or null).

@@ -920,11 +920,19 @@ struct ChainT {
     static_assert(2 * NSA + 2 * NSB + 2 * NSV + 5 <= 32, "barrier area");
 };
 
-// LAYER: the layer epilogue on o (a separate instantiation keeps the plain
-// chain as lean as before).
-template <bool LAYER>
+// MODE (separate instantiations, so that the plain chain stays as lean as
+// it was): kChainPlain; kChainLayer adds the layer epilogue on o;
+// kChainTransition forms a segment's cumulative transition for context
+// parallelism: the state starts as the identity, v counts as zero (the v
+// ring and the YT V products are skipped), no output is formed, and the
+// final state is the transition.
+enum : int { kChainPlain = 0, kChainLayer = 1, kChainTransition = 2 };
+
+template <int MODE>
 __global__ void __launch_bounds__(ChainT::THREADS, 1)
 kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    constexpr bool LAYER = MODE == kChainLayer;
+    constexpr bool TRANS = MODE == kChainTransition;
     using Cfg = ChainT;
     constexpr int NSA = Cfg::NSA, NSB = Cfg::NSB, NSV = Cfg::NSV, NCW = Cfg::NCW;
     extern __shared__ uint8_t dyn_smem[];
@@ -986,7 +994,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         }
     } else if (warp == NCW + 3) {
         // ---------------------------------------------- ring V: the v tile (from HBM)
-        if (lane == 0 && nchunks > 0) {
+        if (!TRANS && lane == 0 && nchunks > 0) {
             tma_prefetch_desc(&tm_v);
             int issued_v = 0;
             for (int n = 0; n < nchunks; ++n) {
@@ -1005,7 +1013,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         }
     } else if (warp == NCW + 2) {
         // ---------------------------------------------- ring B: QP, ZB
-        if (lane == 0 && nchunks > 0) {
+        if (!TRANS && lane == 0 && nchunks > 0) {
             int issued_b = 0;
             for (int n = 0; n < nchunks; ++n) {
                 const int sb = n % NSB;
@@ -1038,18 +1046,24 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             const uint32_t aSB = tmem + Cfg::COL_SB + 64u * (uint32_t)(n & 1);
             mbar_wait(SREADY, n & 1, abort_flag);
             mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
-            mbar_wait(&FULLV[sv], (n / NSV) & 1, abort_flag);
+            if (!TRANS) mbar_wait(&FULLV[sv], (n / NSV) & 1, abort_flag);
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)   // S^T += SB^T MP^T  (K = c')
                 mma_bf16_ts_warp(tmem + Cfg::COL_S, aSB + 8 * ks,
                                  smem_desc(bM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
                                  idS, 1u);
+            if (!TRANS) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)   // S^T += V^T YT^T  (K = t)
-                mma_bf16_warp(tmem + Cfg::COL_S, smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
-                              smem_desc(bY + ks * 32, 16, 1024, kLayoutSW128), idSV, 1u);
+                for (int ks = 0; ks < 4; ++ks)   // S^T += V^T YT^T  (K = t)
+                    mma_bf16_warp(tmem + Cfg::COL_S, smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
+                                  smem_desc(bY + ks * 32, 16, 1024, kLayoutSW128), idSV, 1u);
+            }
             mma_commit_warp(SDONE);
+            if (TRANS) {   // no output: the slot is free once the state products are done
+                mma_commit_warp(&EMPTYA[sa]);
+                continue;
+            }
             mbar_wait(&FULLB[sb], (n / NSB) & 1, abort_flag);
             const uint32_t bQ = smem_addr(slot_b + Cfg::B_QP);
             const uint32_t bZ = smem_addr(slot_b + Cfg::B_ZB);
@@ -1079,7 +1093,10 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         const int j = 32 * quad + lane;
         const size_t sbase = ((size_t)seq * p.H + h) * (size_t)(DK * DV) + (size_t)(32 * g) * DV + j;
         float S[32];
-        if (p.init_state) {
+        if (TRANS) {   // the identity: S[c][j] = (c == j)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) S[i] = (32 * g + i == j) ? 1.f : 0.f;
+        } else if (p.init_state) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] = p.init_state[sbase + (size_t)i * DV];
         } else {
@@ -1194,11 +1211,11 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(SREADY);
-            if (n >= 1) store_o_t(n - 1);
+            if (!TRANS && n >= 1) store_o_t(n - 1);
         }
         if (nchunks > 0) {
             const int m = nchunks - 1;
-            store_o_t(m);
+            if (!TRANS) store_o_t(m);
             mbar_wait(SDONE, m & 1, abort_flag);
             tc_fence_after();
             tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + 32 * g), S);
@@ -1414,19 +1431,23 @@ cudaError_t launch_chain(const void *v, int64_t total_tokens, int H, const split
 
 // The transposed whole-d_v chain: grid = sequences x heads.
 cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const split::Params &prm,
-                           unsigned units, bool overlap, cudaStream_t stream) {
+                           unsigned units, bool overlap, cudaStream_t stream,
+                           int mode = split::kChainPlain) {
     using namespace split;
     CUtensorMap mv;
     if (!make_map_split(&mv, v, total_tokens, H, DV, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kda_chain_t_kernel<false>,
+        cudaError_t e = cudaFuncSetAttribute(kda_chain_t_kernel<kChainPlain>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)ChainT::ALLOC);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kda_chain_t_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)ChainT::ALLOC);
+        e = cudaFuncSetAttribute(kda_chain_t_kernel<kChainLayer>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ChainT::ALLOC);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kda_chain_t_kernel<kChainTransition>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ChainT::ALLOC);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -1440,8 +1461,10 @@ cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const spl
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = overlap ? 1 : 0;
-    const cudaError_t e = prm.layer ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<true>, mv, prm)
-                                    : cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<false>, mv, prm);
+    const cudaError_t e =
+        mode == kChainTransition ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainTransition>, mv, prm)
+        : prm.layer              ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainLayer>, mv, prm)
+                                 : cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainPlain>, mv, prm);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1500,7 +1523,8 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                  const void *beta, const float *init_state, const int32_t *cu,
                                  int num_seqs, int64_t total_tokens, int H, void *o,
                                  float *final_state, void *workspace, bool scalar_gate,
-                                 const LayerArgs *layer, cudaStream_t stream) {
+                                 const LayerArgs *layer, cudaStream_t stream, int cp_mode,
+                                 float *cp_transition) {
     using namespace split;
     const SplitLayout l = split_layout(num_seqs, total_tokens, H);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1510,6 +1534,27 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     int32_t *perm = cu ? reinterpret_cast<int32_t *>(ws + l.perm) : nullptr;
     int32_t *chunk_off = reinterpret_cast<int32_t *>(ws + l.chunk_off);
     int2 *chunk_tab = reinterpret_cast<int2 *>(ws + l.chunk_tab);
+    if (cp_mode == kCpFinish) {
+        // the records, chunk tables and sequence order are those a kCpLocal
+        // call left in this workspace: only the chain runs, from init_state
+        Params prm = {};
+        prm.init_state = init_state;
+        prm.final_state = final_state;
+        prm.o = static_cast<__nv_bfloat16 *>(o);
+        prm.cu = cu;
+        prm.perm = perm;
+        prm.chunk_off = chunk_off;
+        prm.chunk_tab = chunk_tab;
+        prm.total_chunks = total_chunks;
+        prm.recs = ws + l.recs;
+        prm.rec_ready = nullptr;
+        prm.work_next = work_next;
+        prm.err_word = err;
+        prm.total_tokens = total_tokens;
+        prm.num_seqs = num_seqs;
+        prm.H = H;
+        return launch_chain_t(v, total_tokens, H, prm, (unsigned)((size_t)num_seqs * H), false, stream);
+    }
 
     CUtensorMap mk, mq, mg;
     if (!make_map_split(&mk, k, total_tokens, H, DK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1530,9 +1575,11 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
             sm_count = 148;
     }
     const unsigned units = (unsigned)((size_t)num_seqs * H);
-    // the layer epilogue normalises whole rows of o: whole-d_v chain CTAs only
+    // the layer epilogue normalises whole rows of o, and a segment's transition
+    // is d_k x d_k: whole-d_v chain CTAs only
     const ChainPlan plan = choose_chain(units, (uint64_t)(total_tokens / C + num_seqs) * H, total_tokens,
-                                        num_seqs, (unsigned)sm_count, layer != nullptr);
+                                        num_seqs, (unsigned)sm_count,
+                                        layer != nullptr || cp_mode == kCpLocal);
     const bool overlap = plan.overlap;
     const unsigned chain_blocks = units * (unsigned)(DV / plan.dvt);
     uint32_t *rec_ready = overlap ? reinterpret_cast<uint32_t *>(ws + l.flags) : nullptr;
@@ -1598,6 +1645,17 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         if (e != cudaSuccess) return e;
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
+    }
+    if (cp_mode == kCpLocal) {
+        // the locally generated state (from zero), then over the same records
+        // the segment's transition (from the identity, v counting as zero)
+        e = launch_chain_t(v, total_tokens, H, prm, units, overlap, stream);
+        if (e != cudaSuccess) return e;
+        Params pt = prm;
+        pt.init_state = nullptr;
+        pt.final_state = cp_transition;
+        pt.rec_ready = nullptr;   // the records are complete once the first chain has run
+        return launch_chain_t(v, total_tokens, H, pt, units, false, stream, kChainTransition);
     }
     return plan.dvt == 32 ? launch_chain<32>(v, total_tokens, H, prm, units, overlap, stream)
                           : launch_chain_t(v, total_tokens, H, prm, units, overlap, stream);

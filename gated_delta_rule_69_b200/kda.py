@@ -21,7 +21,7 @@ KDA_BF16, KDA_FP32 = 0, 1
 EXPORTED = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
             "kda_prefill", "kda_decode_step", "kda_check_workspace_error",
             "kda_prefill_noalloc", "gdn_prefill", "gdn_decode_step", "kda_layer_prefill",
-            "kda_layer_decode_step", "kda_cp_combine")
+            "kda_layer_decode_step", "kda_cp_combine", "kda_cp_local", "kda_cp_finish")
 
 
 class KdaError(RuntimeError):
@@ -64,6 +64,11 @@ def lib():
         L.kda_layer_decode_step.restype = ctypes.c_int
         L.kda_cp_combine.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.kda_cp_combine.restype = ctypes.c_int
+        L.kda_cp_local.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, ctypes.c_int, vp, vp, vp,
+                                   vp, sz, vp]
+        L.kda_cp_local.restype = ctypes.c_int
+        L.kda_cp_finish.argtypes = [vp, vp, i64, i32, i32, i32, ctypes.c_int, vp, vp, vp, sz, vp]
+        L.kda_cp_finish.restype = ctypes.c_int
         L.kda_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
                                           ctypes.c_int, vp, vp, vp]
         L.kda_prefill_noalloc.restype = ctypes.c_int
@@ -295,3 +300,40 @@ def kda_cp_combine(M, S_tilde, S0=None, S_in=None, stream=None):
     if st != KDA_OK:
         raise KdaError(st, "kda_cp_combine")
     return S_in
+
+
+def kda_cp_local(q, k, v, log_alpha, beta, workspace, o_scratch=None, stream=None):
+    """One segment's (M [1, H, d_k, d_k], S~ [1, H, d_k, d_v]); the chunk records
+    stay in ``workspace`` for kda_cp_finish.  bf16, d = 128, one sequence."""
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    M = torch.empty((1, H, dk, dk), dtype=torch.float32, device=q.device)
+    S = torch.empty((1, H, dk, dv), dtype=torch.float32, device=q.device)
+    if o_scratch is None:
+        o_scratch = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    _check_cuda(q, k, v, log_alpha, beta, workspace, o_scratch)
+    st = lib().kda_cp_local(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), T, H, dk, dv,
+                            _dtype_code(q), _ptr(M), _ptr(S), _ptr(o_scratch), _ptr(workspace),
+                            workspace.numel(), _stream(stream, q.device))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_cp_local")
+    return M, S
+
+
+def kda_cp_finish(v, S_in, workspace, o=None, final_state=None, output_final_state=True,
+                  stream=None):
+    """The segment's outputs and end state from S_in, over the records a
+    kda_cp_local call left in ``workspace``."""
+    T, H, dv = v.shape
+    dk = S_in.shape[-2] if S_in is not None else dv
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=v.dtype, device=v.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((1, H, dk, dv), dtype=torch.float32, device=v.device)
+    _check_cuda(v, S_in, workspace, o, final_state)
+    st = lib().kda_cp_finish(_ptr(v), _ptr(S_in), T, H, dk, dv, _dtype_code(v), _ptr(o),
+                             _ptr(final_state), _ptr(workspace), workspace.numel(),
+                             _stream(stream, v.device))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_cp_finish")
+    return o, final_state

@@ -235,16 +235,39 @@ kda_status kda_layer_decode_step(const void *q, const void *k, const void *v,
  * before it:
  *   M       : [n_prev, H, d_k, d_k] fp32;   S_tilde : [n_prev, H, d_k, d_v] fp32
  *   S0      : [H, d_k, d_v] fp32 or NULL (zero);   S_in : [H, d_k, d_v] fp32, written
- * n_prev = 0 copies S0 (or writes zeros).  A segment's M is the final state
- * of kda_prefill on that segment with v = 0 (d_v = d_k) and the identity as
- * initial state; S~ is its final state from a zero state (the Python module
- * context_parallel.py does this and the exchange).  Supported: d_k in
+ * n_prev = 0 copies S0 (or writes zeros).  A segment's (M, S~) come from
+ * kda_cp_local below (the Python module context_parallel.py runs the passes
+ * and the exchange).  Supported: d_k in
  * {16, 32, 64, 128}, d_v in {32, 64, 128}; 4-byte aligned pointers; S_in must
  * not overlap M or S_tilde.
  */
 kda_status kda_cp_combine(const float *M, const float *S_tilde, const float *S0, float *S_in,
                           int32_t n_prev, int32_t H, int32_t d_k, int32_t d_v,
                           kda_stream_t stream);
+
+/*
+ * The two passes of one segment (a single sequence of total_tokens tokens,
+ * bf16, d_k = d_v = 128, a workspace of kda_prefill_workspace_size(1,
+ * total_tokens, H) bytes), sharing one chunk preparation:
+ *   kda_cp_local  prepares every chunk (the records stay in `workspace`) and
+ *                 runs the state chain twice over them: S_tilde [1, H, d_k, d_v]
+ *                 from a zero state, M [1, H, d_k, d_k] from the identity with
+ *                 v counting as zero; o_scratch [T, H, d_v] is written and
+ *                 holds nothing useful.
+ *   kda_cp_finish runs the chain once more over the same workspace's records
+ *                 from S_in [1, H, d_k, d_v] (NULL: zero), writing o and
+ *                 final_state (NULL: not written).  The workspace must not have
+ *                 been used for anything else in between, and v must be the
+ *                 same tensor.
+ */
+kda_status kda_cp_local(const void *q, const void *k, const void *v, const void *log_alpha,
+                        const void *beta, int64_t total_tokens, int32_t H, int32_t d_k,
+                        int32_t d_v, kda_dtype dtype, float *M, float *S_tilde, void *o_scratch,
+                        void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+kda_status kda_cp_finish(const void *v, const float *S_in, int64_t total_tokens, int32_t H,
+                         int32_t d_k, int32_t d_v, kda_dtype dtype, void *o, float *final_state,
+                         void *workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads the error word that the prefill kernels

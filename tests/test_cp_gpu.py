@@ -77,3 +77,30 @@ def test_cp_combine_matches_host_products():
         assert np.abs(f64(out) - ref).max() <= 1e-4 * max(1.0, np.abs(ref).max())
     zero = kda.kda_cp_combine(M[:0].contiguous(), St[:0].contiguous(), None)
     assert float(zero.abs().max()) == 0.0
+
+
+def test_cp_local_and_finish_match_plain_prefills():
+    """kda_cp_local's pair equals the two plain prefills it stands for (v = 0
+    from the identity, and from zero), and kda_cp_finish over the kept
+    records equals a plain prefill from the same entering state."""
+    from gated_delta_rule_69_b200 import context_parallel as cp
+    from gated_delta_rule_69_b200 import kda
+    T, H = 333, 3
+    w = kin.Workload("cpl", "prefill", H=H, d_k=128, d_v=128, dtype="bf16", seed=73, T=T,
+                     init_std=0.02)
+    inp = kin.generate(w, device=DEV)
+    args = tuple(inp[x] for x in ("q", "k", "v", "log_alpha", "beta"))
+    ws = cp.workspace_for(inp["q"])
+    m, st = kda.kda_cp_local(*args, ws)
+    eye = torch.eye(128, device=DEV).expand(1, H, 128, 128).contiguous()
+    _, m_ref = kda.kda_prefill(args[0], args[1], torch.zeros_like(args[2]), args[3], args[4],
+                               init_state=eye)
+    _, st_ref = kda.kda_prefill(*args)
+    torch.cuda.synchronize()
+    assert torch.equal(m, m_ref)
+    assert torch.equal(st, st_ref)
+    o, fs = kda.kda_cp_finish(args[2], inp["init_state"], ws)
+    o_ref, fs_ref = kda.kda_prefill(*args, init_state=inp["init_state"])
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref)
+    assert torch.equal(fs, fs_ref)
