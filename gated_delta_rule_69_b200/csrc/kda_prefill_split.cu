@@ -1260,14 +1260,23 @@ kda_split_plan_kernel(const int32_t *cu, int n, int64_t total, int32_t *perm, in
     if (threadIdx.x == 0) *work_next = 0u;
     __shared__ int32_t warp_sums[kPlanThreads / 32];
     __shared__ int32_t carry_s;
+    // up to kMaxSortedSeqs sequences, cu_seqlens and the chunk offsets are
+    // worked on in shared memory (one read of cu, no global round trips)
+    __shared__ int32_t s_cu[kMaxSortedSeqs + 1], s_off[kMaxSortedSeqs + 1];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const bool small = n <= kMaxSortedSeqs;
+    if (cu && small)
+        for (int i = tid; i <= n; i += kPlanThreads) s_cu[i] = cu[i];
+    __syncthreads();
+    const int32_t *cuv = (cu && small) ? s_cu : cu;
+    int32_t *offv = small ? s_off : chunk_off;
     int bad = 0;
     if (cu) {
         for (int i = tid; i < n; i += kPlanThreads) {
-            const int64_t a = cu[i], b = cu[i + 1];
+            const int64_t a = cuv[i], b = cuv[i + 1];
             if (a < 0 || b < a || b > total) bad = 1;
         }
-        if (tid == 0 && (cu[0] != 0 || cu[n] != total)) bad = 1;
+        if (tid == 0 && (cuv[0] != 0 || cuv[n] != total)) bad = 1;
     }
     bad = __syncthreads_or(bad);
     if (tid == 0) {
@@ -1278,7 +1287,7 @@ kda_split_plan_kernel(const int32_t *cu, int n, int64_t total, int32_t *perm, in
     // exclusive scan of the chunk counts, 1024 sequences at a time
     for (int base = 0; base < n; base += kPlanThreads) {
         const int i = base + tid;
-        const int cnt = (i < n) ? (int)((seq_len_checked(cu, i, n, total) + C - 1) / C) : 0;
+        const int cnt = (i < n) ? (int)((seq_len_checked(cuv, i, n, total) + C - 1) / C) : 0;
         int incl = cnt;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -1299,27 +1308,29 @@ kda_split_plan_kernel(const int32_t *cu, int n, int64_t total, int32_t *perm, in
         __syncthreads();
         const int carry = carry_s;
         const int excl = carry + (wid > 0 ? warp_sums[wid - 1] : 0) + incl - cnt;
-        if (i < n) chunk_off[i] = excl;
+        if (i < n) offv[i] = excl;
         __syncthreads();
         if (tid == kPlanThreads - 1) carry_s = excl + cnt;
         __syncthreads();
     }
     const int nchunks = carry_s;
     if (tid == 0) {
-        chunk_off[n] = nchunks;
+        offv[n] = nchunks;
         *total_chunks = (uint32_t)nchunks;
     }
     __syncthreads();
+    if (small)
+        for (int i = tid; i <= n; i += kPlanThreads) chunk_off[i] = s_off[i];
     for (int c = tid; c < nchunks; c += kPlanThreads) {
         int lo = 0, hi = n;   // last sequence i with chunk_off[i] <= c
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (chunk_off[mid] <= c) lo = mid;
+            if (offv[mid] <= c) lo = mid;
             else hi = mid;
         }
-        const int64_t bos = cu ? (int64_t)cu[lo] : (int64_t)lo * (total / n);
-        const int64_t t0 = bos + (int64_t)(c - chunk_off[lo]) * C;
-        const int64_t len = seq_len_checked(cu, lo, n, total);
+        const int64_t bos = cu ? (int64_t)cuv[lo] : (int64_t)lo * (total / n);
+        const int64_t t0 = bos + (int64_t)(c - offv[lo]) * C;
+        const int64_t len = seq_len_checked(cuv, lo, n, total);
         chunk_tab[c] = make_int2((int)t0, (int)min((int64_t)C, bos + len - t0));
     }
     if (!perm) return;
@@ -1328,10 +1339,10 @@ kda_split_plan_kernel(const int32_t *cu, int n, int64_t total, int32_t *perm, in
             perm[i] = i;
             continue;
         }
-        const int64_t li = seq_len_checked(cu, i, n, total);
+        const int64_t li = seq_len_checked(cuv, i, n, total);
         int r = 0;
         for (int j = 0; j < n; ++j) {
-            const int64_t lj = seq_len_checked(cu, j, n, total);
+            const int64_t lj = seq_len_checked(cuv, j, n, total);
             r += (lj > li) || (lj == li && j < i);
         }
         perm[r] = i;
