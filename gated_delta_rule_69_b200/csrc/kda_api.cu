@@ -84,7 +84,7 @@ kda_status prefill_impl(const void *q, const void *k, const void *v,
             return KDA_ERR_WORKSPACE;
         if (!layer->A_log || !aligned_to(layer->A_log, 4) ||
             (layer->norm_weight && !aligned_to(layer->norm_weight, 4)) ||
-            (layer->out_gate && !aligned_to(layer->out_gate, eb)) ||
+            (layer->out_gate && !aligned16(layer->out_gate)) ||
             !(layer->qk_eps >= 0.f) || !(layer->norm_eps >= 0.f) ||
             overlaps(o, nv, layer->out_gate, nv))
             return KDA_ERR_INVALID_ARG;

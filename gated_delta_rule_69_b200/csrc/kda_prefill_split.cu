@@ -910,8 +910,7 @@ struct ChainT {
     static constexpr uint32_t EGLR = RB + NSB * B_STRIDE;   // NSA x exp(G_L), 128 fp32 each
     static constexpr uint32_t BARS = EGLR + NSA * 512;
     static constexpr uint32_t MISC = BARS + 256;
-    static constexpr uint32_t EPI = MISC + 64;              // layer epilogue: 2 x 4 x 4 x 16 fp32
-    static constexpr uint32_t SIZE = EPI + 2048;
+    static constexpr uint32_t SIZE = MISC + 64;
     static constexpr uint32_t ALLOC = SIZE + 1024;
     // TMEM columns: S^T fp32 (128), SB^T bf16 pairs x 2 (64 each), O^T fp32 x 2 (64 each)
     static constexpr uint32_t TMEM_COLS = 512;
@@ -920,18 +919,15 @@ struct ChainT {
     static_assert(2 * NSA + 2 * NSB + 2 * NSV + 5 <= 32, "barrier area");
 };
 
-// MODE (separate instantiations, so that the plain chain stays as lean as
-// it was): kChainPlain; kChainLayer adds the layer epilogue on o;
-// kChainTransition forms a segment's cumulative transition for context
-// parallelism: the state starts as the identity, v counts as zero (the v
-// ring and the YT V products are skipped), no output is formed, and the
-// final state is the transition.
-enum : int { kChainPlain = 0, kChainLayer = 1, kChainTransition = 2 };
+// MODE (separate instantiations): kChainPlain; kChainTransition forms a
+// segment's cumulative transition for context parallelism: the state starts
+// as the identity, v counts as zero (the v ring and the YT V products are
+// skipped), no output is formed, and the final state is the transition.
+enum : int { kChainPlain = 0, kChainTransition = 2 };
 
 template <int MODE>
 __global__ void __launch_bounds__(ChainT::THREADS, 1)
 kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
-    constexpr bool LAYER = MODE == kChainLayer;
     constexpr bool TRANS = MODE == kChainTransition;
     using Cfg = ChainT;
     constexpr int NSA = Cfg::NSA, NSB = Cfg::NSB, NSV = Cfg::NSV, NCW = Cfg::NCW;
@@ -1103,7 +1099,6 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] = 0.f;
         }
-        const float wj = (LAYER && p.norm_weight) ? p.norm_weight[j] : 1.f;
         // O^T of chunk m: this warp's 16 t columns, lane j, bf16 to o[t][h][j]
         auto store_o_t = [&](int m) {
             mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
@@ -1112,69 +1107,6 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             tmem_ld16(tmem_addr(tmem, 32 * quad, Cfg::COL_O + 64 * (m & 1) + 16 * g), v);
             tmem_wait_ld();
             const int64_t t0 = (int64_t)m * C + 16 * g;
-            if (LAYER) {
-                // RMSNorm over d_v: this warp's 32 lanes by a reduce-scatter (lane
-                // ends with the sum for t = 16 g + lane mod 16), the four
-                // quadrant warps of column group g through shared memory
-                float r[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) r[i] = v[i] * v[i];
-#pragma unroll
-                for (int mm = 8; mm >= 1; mm >>= 1) {
-                    const bool up = (lane & mm) != 0;
-#pragma unroll
-                    for (int i = 0; i < mm; ++i) {
-                        const float lo = r[i], hi = r[i + mm];
-                        r[i] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, mm);
-                    }
-                }
-                r[0] += __shfl_xor_sync(0xffffffffu, r[0], 16);
-                // partials as [t][quadrant], so that a thread reads a t's four with one load
-                float *ep = reinterpret_cast<float *>(sm + Cfg::EPI) + (m & 1) * 256 + g * 64;
-                if (lane < 16) ep[lane * 4 + quad] = r[0];
-                named_barrier(1 + g, 128);   // the four quadrant warps of column group g
-                // the output gate (its rows were sent towards L2 a chunk earlier);
-                // loaded only here, after the state hand-off, whose release
-                // would otherwise wait for these loads
-                float og[16];
-                if (p.out_gate) {
-                    // sixteen rows 8 KB apart: issued together in one block (left to
-                    // itself the compiler interleaves each load with its use);
-                    // rows past the end read the last row and are not stored
-                    const __nv_bfloat16 *a[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int64_t tt = t0 + i < len ? t0 + i : len - 1;
-                        a[i] = p.out_gate + ((size_t)(bos + tt) * p.H + h) * DV + j;
-                    }
-                    unsigned short u[16];
-                    asm volatile(
-                        "ld.global.nc.b16 %0, [%16];\n\tld.global.nc.b16 %1, [%17];\n\t"
-                        "ld.global.nc.b16 %2, [%18];\n\tld.global.nc.b16 %3, [%19];\n\t"
-                        "ld.global.nc.b16 %4, [%20];\n\tld.global.nc.b16 %5, [%21];\n\t"
-                        "ld.global.nc.b16 %6, [%22];\n\tld.global.nc.b16 %7, [%23];\n\t"
-                        "ld.global.nc.b16 %8, [%24];\n\tld.global.nc.b16 %9, [%25];\n\t"
-                        "ld.global.nc.b16 %10, [%26];\n\tld.global.nc.b16 %11, [%27];\n\t"
-                        "ld.global.nc.b16 %12, [%28];\n\tld.global.nc.b16 %13, [%29];\n\t"
-                        "ld.global.nc.b16 %14, [%30];\n\tld.global.nc.b16 %15, [%31];"
-                        : "=h"(u[0]), "=h"(u[1]), "=h"(u[2]), "=h"(u[3]), "=h"(u[4]), "=h"(u[5]),
-                          "=h"(u[6]), "=h"(u[7]), "=h"(u[8]), "=h"(u[9]), "=h"(u[10]), "=h"(u[11]),
-                          "=h"(u[12]), "=h"(u[13]), "=h"(u[14]), "=h"(u[15])
-                        : "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(a[4]), "l"(a[5]),
-                          "l"(a[6]), "l"(a[7]), "l"(a[8]), "l"(a[9]), "l"(a[10]), "l"(a[11]),
-                          "l"(a[12]), "l"(a[13]), "l"(a[14]), "l"(a[15]));
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) og[i] = __bfloat162float(__ushort_as_bfloat16(u[i]));
-                }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float4 pq = reinterpret_cast<const float4 *>(ep)[i];
-                    const float ss = (pq.x + pq.y) + (pq.z + pq.w);
-                    float y = v[i] * rsqrtf(ss * (1.f / DV) + p.norm_eps) * wj;
-                    if (p.out_gate) y *= 1.f / (1.f + __expf(-og[i]));
-                    v[i] = y;
-                }
-            }
             __nv_bfloat16 *dst = p.o + ((size_t)(bos + t0) * p.H + h) * DV + j;
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -1182,15 +1114,6 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         };
         for (int n = 0; n < nchunks; ++n) {
             const int sa = n % NSA;
-            if (LAYER && p.out_gate) {
-                // chunk n's output-gate rows towards L2 for the next iteration
-                const int64_t tp = (int64_t)n * C + 16 * g;
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (tp + i < len)
-                        asm volatile("prefetch.global.L2 [%0];" ::"l"(
-                            p.out_gate + ((size_t)(bos + tp + i) * p.H + h) * DV + j));
-            }
             if (n >= 1) {
                 mbar_wait(SDONE, (n - 1) & 1, abort_flag);
                 tc_fence_after();
@@ -1233,6 +1156,50 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         tmem_dealloc(tmem, Cfg::TMEM_COLS);
     }
     if (tid == 0 && *abort_flag) atomicOr(p.err_word, kDevErrTimeout);
+}
+
+// =============================================================== layer epilogue
+// o <- o / sqrt(mean_j o_j^2 + eps) * w_j * sigmoid(g_j) per (token, head) row,
+// in place after the chain: one warp per row of 128, four channels per lane.
+// A pass of its own: inside the chain's loop the same work sat on the serial
+// state path (about 1.5 us per chunk); here it is a stream over o and the gate.
+constexpr int kEpiThreads = 256;
+
+__global__ void __launch_bounds__(kEpiThreads)
+kda_layer_epilogue_kernel(__nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ gate,
+                          const float *__restrict__ w, float eps, int64_t rows) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * (kEpiThreads / 32) + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    uint2 *orow = reinterpret_cast<uint2 *>(o + row * DV) + lane;
+    const uint2 ov = *orow;
+    float x[4];
+    {
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&ov.x);
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&ov.y);
+        x[0] = __low2float(a); x[1] = __high2float(a); x[2] = __low2float(b); x[3] = __high2float(b);
+    }
+    float gv[4] = {0.f, 0.f, 0.f, 0.f};
+    if (gate) {
+        const uint2 g2 = reinterpret_cast<const uint2 *>(gate + row * DV)[lane];
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&g2.x);
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&g2.y);
+        gv[0] = __low2float(a); gv[1] = __high2float(a); gv[2] = __low2float(b); gv[3] = __high2float(b);
+    }
+    float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float r = rsqrtf(ss * (1.f / DV) + eps);
+    float y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        y[e] = x[e] * r * (w ? w[4 * lane + e] : 1.f);
+        if (gate) y[e] *= 1.f / (1.f + __expf(-gv[e]));
+    }
+    uint2 out;
+    out.x = pack_bf16x2(y[0], y[1]);
+    out.y = pack_bf16x2(y[2], y[3]);
+    *orow = out;
 }
 
 // =============================================================== plan kernel
@@ -1454,9 +1421,6 @@ cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const spl
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)ChainT::ALLOC);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kda_chain_t_kernel<kChainLayer>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ChainT::ALLOC);
-        if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(kda_chain_t_kernel<kChainTransition>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ChainT::ALLOC);
         if (e != cudaSuccess) return e;
@@ -1474,7 +1438,6 @@ cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const spl
     cfg.numAttrs = overlap ? 1 : 0;
     const cudaError_t e =
         mode == kChainTransition ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainTransition>, mv, prm)
-        : prm.layer              ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainLayer>, mv, prm)
                                  : cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainPlain>, mv, prm);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
@@ -1586,11 +1549,9 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
             sm_count = 148;
     }
     const unsigned units = (unsigned)((size_t)num_seqs * H);
-    // the layer epilogue normalises whole rows of o, and a segment's transition
-    // is d_k x d_k: whole-d_v chain CTAs only
+    // a segment's transition is d_k x d_k: whole-d_v chain CTAs only
     const ChainPlan plan = choose_chain(units, (uint64_t)(total_tokens / C + num_seqs) * H, total_tokens,
-                                        num_seqs, (unsigned)sm_count,
-                                        layer != nullptr || cp_mode == kCpLocal);
+                                        num_seqs, (unsigned)sm_count, cp_mode == kCpLocal);
     const bool overlap = plan.overlap;
     const unsigned chain_blocks = units * (unsigned)(DV / plan.dvt);
     uint32_t *rec_ready = overlap ? reinterpret_cast<uint32_t *>(ws + l.flags) : nullptr;
@@ -1668,8 +1629,15 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         pt.rec_ready = nullptr;   // the records are complete once the first chain has run
         return launch_chain_t(v, total_tokens, H, pt, units, false, stream, kChainTransition);
     }
-    return plan.dvt == 32 ? launch_chain<32>(v, total_tokens, H, prm, units, overlap, stream)
-                          : launch_chain_t(v, total_tokens, H, prm, units, overlap, stream);
+    e = plan.dvt == 32 ? launch_chain<32>(v, total_tokens, H, prm, units, overlap, stream)
+                       : launch_chain_t(v, total_tokens, H, prm, units, overlap, stream);
+    if (e != cudaSuccess || !layer) return e;
+    const int64_t rows = total_tokens * H;
+    kda_layer_epilogue_kernel<<<(unsigned)((rows + kEpiThreads / 32 - 1) / (kEpiThreads / 32)),
+                                kEpiThreads, 0, stream>>>(
+        static_cast<__nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(layer->out_gate),
+        layer->norm_weight, layer->norm_eps, rows);
+    return cudaGetLastError();
 }
 
 }  // namespace kda

@@ -199,13 +199,15 @@ kda_status gdn_decode_step(const void *q, const void *k, const void *v,
  *
  *   q, k, gate_z : [T, H, d_k] raw;  v : [T, H, d_v];  beta_logit : [T, H]
  *   A_log        : [H] fp32 (device), required
- *   out_gate     : [T, H, d_v] pre-sigmoid, or NULL (no output gate)
+ *   out_gate     : [T, H, d_v] pre-sigmoid, or NULL (no output gate); 16-byte
+ *                  aligned for kda_layer_prefill
  *   norm_weight  : [d_v] fp32 (device), or NULL (weight 1)
  * Other arguments, layouts and errors as kda_prefill / kda_decode_step.
  * kda_layer_prefill runs on the two-kernel tensor-core path only: bf16,
  * d_k = d_v = 128 and a workspace of kda_prefill_workspace_size(...) bytes
- * (else KDA_ERR_UNSUPPORTED / KDA_ERR_WORKSPACE); the state chain then always
- * keeps whole rows of o in one CTA.  kda_layer_decode_step takes every shape
+ * (else KDA_ERR_UNSUPPORTED / KDA_ERR_WORKSPACE); its prologue runs inside
+ * the chunk preparation and its epilogue as one pass over o after the state
+ * chain.  kda_layer_decode_step takes every shape
  * kda_decode_step takes.  Weights of the projections that produce these
  * activations are the caller's.
  */
