@@ -13,7 +13,8 @@ recurrence", section "Kimi Delta Attention = les trois remedes combines"):
     o_t = S_t^T q_t
 
 ``gdn_recurrence`` is the Gated DeltaNet special case (one scalar gate per
-token and head), written from its own update equation.
+token and head), written from its own update equation.  ``kda_backward`` and
+``gdn_backward`` are the recurrence's reverse-mode derivative.
 
 Inputs are float64 numpy arrays holding exactly the values the GPU sees (bf16
 inputs are widened exactly).  Pins of this oracle (closed forms, exact
@@ -62,6 +63,11 @@ def _load():
             lib.gdn_oracle_recurrence.argtypes = lib.kda_oracle_recurrence.argtypes
             lib.gdn_oracle_recurrence.restype = ctypes.c_int
             lib.kda_oracle_max_threads.restype = ctypes.c_int
+            lib.kda_oracle_backward.argtypes = [
+                dp, dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+            lib.kda_oracle_backward.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -170,6 +176,63 @@ def kda_decode_step(q, k, v, g, beta, state, nthreads: int = 0):
     cu = np.arange(B + 1, dtype=np.int64)
     return kda_recurrence(q, k, v, g, beta, init_state=state, cu_seqlens=cu,
                           nthreads=nthreads)
+
+
+# ---- backward pass ------------------------------------------------------------
+# The reverse-mode derivative of the recurrence, step by step (the chain rule
+# written out in kda_oracle.c, kda_oracle_backward).
+
+def kda_backward(q, k, v, g, beta, d_o, init_state=None, d_final_state=None,
+                 cu_seqlens=None, nthreads: int = 0):
+    """Gradients of a loss L through kda_recurrence.
+
+    d_o = dL/do [T, H, d_v]; d_final_state = dL/dS_T [N, H, d_k, d_v] or None
+    (zero).  Returns (dq, dk, dv, dg, dbeta, d_init_state) as float64 arrays in
+    the inputs' shapes (d_init_state = dL/dS_0, [N, H, d_k, d_v]).
+    """
+    q, k, v, g, beta, d_o = (_f64(x) for x in (q, k, v, g, beta, d_o))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    if k.shape != (T, H, dk) or g.shape != (T, H, dk):
+        raise ValueError("q, k, g must share shape [T, H, d_k]")
+    if v.shape[:2] != (T, H) or beta.shape != (T, H) or d_o.shape != v.shape:
+        raise ValueError("v and d_o must be [T, H, d_v] and beta [T, H]")
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    n = cu.shape[0] - 1
+    if cu[0] != 0 or cu[-1] != T:
+        raise ValueError("cu_seqlens must start at 0 and end at T")
+    s0 = None if init_state is None else _f64(init_state)
+    dsT = None if d_final_state is None else _f64(d_final_state)
+    for x in (s0, dsT):
+        if x is not None and x.shape != (n, H, dk, dv):
+            raise ValueError("states must be [N, H, d_k, d_v]")
+    dq = np.zeros((T, H, dk)); dkk = np.zeros((T, H, dk)); dg = np.zeros((T, H, dk))
+    dvv = np.zeros((T, H, dv)); db = np.zeros((T, H)); ds0 = np.zeros((n, H, dk, dv))
+    rc = _load().kda_oracle_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0),
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n, H, dk, dv,
+        _ptr(d_o), _ptr(dsT), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dg), _ptr(db),
+        _ptr(ds0), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_backward failed with code {rc}")
+    return dq, dkk, dvv, dg, db, ds0
+
+
+def gdn_backward(q, k, v, g, beta, d_o, init_state=None, d_final_state=None,
+                 cu_seqlens=None, nthreads: int = 0):
+    """Gradients through gdn_recurrence (g [T, H]).  A scalar gate is the
+    per-channel gate with every channel equal, so its derivative is the sum of
+    the per-channel derivatives over the key channels (the chain rule for a
+    broadcast); the rest is kda_backward."""
+    g = _f64(g)
+    dk_ = np.asarray(q).shape[2]
+    dq, dkk, dvv, dg, db, ds0 = kda_backward(
+        q, k, v, np.repeat(g[:, :, None], dk_, axis=2), beta, d_o, init_state=init_state,
+        d_final_state=d_final_state, cu_seqlens=cu_seqlens, nthreads=nthreads)
+    return dq, dkk, dvv, dg.sum(axis=2), db, ds0
 
 
 # ---- the layer's prologue and epilogue around the recurrence ----------------
