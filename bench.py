@@ -11,7 +11,9 @@ timed interval.  The decode figures time chained kda_decode_step calls on the
 decode workload (state 512 MiB, larger than L2, so no flush is needed).  The
 "gdn_prefill" object times gdn_prefill (Gated DeltaNet: one gate value per
 token and head) and "layer_prefill" times kda_layer_prefill (raw activations,
-the layer's prologue and epilogue fused) on the prefill workload the same way.
+the layer's prologue and epilogue fused) on the prefill workload the same way;
+"backward" times kda_backward (the gradients, given seeded upstream gradients)
+on the same workload.
 Under torchrun every rank runs the same workload as an independent replica
 (the operator needs no exchange between GPUs); value = all ranks' tokens over
 the slowest rank's time.
@@ -59,6 +61,27 @@ def prefill_work(w, lengths, scalar_gate=False, layer=False):
     state_bytes = n * w.H * w.d_k * w.d_v * 4 * (2 if w.init_std > 0 else 1)
     return dict(tokens=T, flop=per_tok_flop * T * w.H,
                 bytes=per_tok_bytes * T * w.H + state_bytes)
+
+
+# Backward pass, per (token, head) with a d_k x d_v state: one forward step
+# (decay, r, update: 5 FLOP per state element) and the backward step (q do^T,
+# dq, du, dk, the erase term, dk's second term, dg, the decay of dS, Sp and
+# S_t again: 18 FLOP per element), on CUDA cores in fp32.  Bytes: q, k,
+# log_alpha, v, do read in the I/O dtype, beta read; dq, dk, dlog_alpha, dv,
+# dbeta written in fp32; per (sequence, head) the initial state and dL/dS_T
+# read and dL/dS_0 written.
+BWD_FLOP_PER_ELEM = 5 + 18
+# fp32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 FLOP (FMA) x 1.965 GHz
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def backward_work(w, lengths):
+    T, n = sum(lengths), len(lengths)
+    eb = 2 if w.dtype == "bf16" else 4
+    per_tok = (3 * w.d_k + 2 * w.d_v) * eb + eb + (3 * w.d_k + w.d_v + 1) * 4
+    states = n * w.H * w.d_k * w.d_v * 4 * 3
+    return dict(tokens=T, flop=BWD_FLOP_PER_ELEM * w.d_k * w.d_v * T * w.H,
+                bytes=per_tok * T * w.H + states)
 
 
 def decode_work(w):
@@ -239,6 +262,50 @@ def time_prefill(w, steps, warmup, world, scalar_gate=False, layer=False):
     # the plan, the preparation and the state chain
     per_call = 3 if (w.dtype == "bf16" and w.d_k == 128 and w.d_v == 128) else 2
     return dict(ms_total=sum(ms), ms=ms, inputs=inp, launches=steps * per_call)
+
+
+def time_backward(w, steps, warmup, world):
+    """kda_backward on the prefill workload with seeded upstream gradients,
+    L2 flushed before each step."""
+    import torch
+    from gated_delta_rule_69_b200 import inputs as kin
+    from gated_delta_rule_69_b200 import kda
+    inp = kin.generate(w, device="cuda")
+    ct = kin.cotangents(w, inp["lengths"], device="cuda")
+    q, k, v, g, b = (inp[x] for x in ("q", "k", "v", "log_alpha", "beta"))
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    n = len(inp["lengths"])
+    ws = torch.empty(max(256, kda.kda_backward_workspace_size(n, T, H, dk, dv)),
+                     dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.kda_backward(q, k, v, g, b, ct["d_o"], init_state=inp["init_state"],
+                         d_final_state=ct["d_final_state"], cu_seqlens=inp["cu_seqlens"],
+                         workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    if kda.kda_check_workspace_error(ws) != kda.KDA_OK:
+        raise RuntimeError("device-side check failed during the backward benchmark")
+    ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    # one kernel per call (the gradient zeroing is four memsets)
+    return dict(ms_total=sum(ms), ms=ms, lengths=inp["lengths"], launches=steps)
 
 
 def time_prefill_e2e(w, steps, warmup):
@@ -435,6 +502,7 @@ def main():
     dec = time_decode(dw, args.decode_steps, args.warmup, world)
     gdn = time_prefill(w, args.steps, args.warmup, world, scalar_gate=True)
     lay = time_prefill(w, args.steps, args.warmup, world, layer=True)
+    bwd = time_backward(w, max(3, args.steps // 4), args.warmup, world)
     clocks = sampler.stop()
 
     lengths = pf["inputs"]["lengths"]
@@ -452,6 +520,9 @@ def main():
     lwork = prefill_work(w, lengths, layer=True)
     lms = max_over_ranks(lay["ms_total"] / args.steps, world)
     lgbs = lwork["bytes"] / (lms * 1e-3) / 1e9
+    bwork = backward_work(w, bwd["lengths"])
+    bms = max_over_ranks(bwd["ms_total"] / len(bwd["ms"]), world)
+    btfs = bwork["flop"] / (bms * 1e-3) / 1e12
     src = "of " + peaks["source"]
 
     line = {
@@ -486,7 +557,19 @@ def main():
                                        "traffic": None, "peak_source": src,
                                        "kernel": "kda_layer_prefill",
                                        "algorithmic_bytes_per_launch": lwork["bytes"]}},
-        "gpu_launches": pf["launches"] + dec["launches"] + gdn["launches"] + lay["launches"],
+        "backward": {"workload": w.name + ", backward pass (kda_backward), seeded upstream gradients",
+                     "value": world * bwork["tokens"] / (bms * 1e-3), "unit": "tokens/s",
+                     "ms_per_step": bms, "steps": len(bwd["ms"]),
+                     "roofline": {"bound": "alu", "achieved": btfs, "peak": FP32_SIMT_TFLOPS,
+                                  "unit": "TFLOP/s", "frac": btfs / FP32_SIMT_TFLOPS,
+                                  "traffic": None,
+                                  "peak_source": "nominal fp32 CUDA-core rate (148 SMs x 128 lanes x 2 x 1.965 GHz)",
+                                  "kernel": "kda_backward",
+                                  "algorithmic_flop_per_launch": bwork["flop"],
+                                  "algorithmic_bytes_per_launch": bwork["bytes"],
+                                  "hbm_frac": bwork["bytes"] / (bms * 1e-3) / 1e9 / peaks["hbm"]}},
+        "gpu_launches": pf["launches"] + dec["launches"] + gdn["launches"] + lay["launches"]
+                        + bwd["launches"],
         "clocks": clocks,
     }
     if not args.no_e2e:

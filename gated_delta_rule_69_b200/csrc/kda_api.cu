@@ -145,6 +145,63 @@ kda_status decode_impl(const void *q, const void *k, const void *v,
                                         d_k, d_v, dtype, o, scalar_gate, layer, stream));
 }
 
+// The backward pass for either gate (gradients in fp32).
+kda_status backward_impl(const void *q, const void *k, const void *v, const void *log_alpha,
+                         const void *beta, const float *init_state, const int32_t *cu_seqlens,
+                         int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                         int32_t d_v, kda_dtype dtype, const void *d_o,
+                         const float *d_final_state, float *dq, float *dk, float *dv,
+                         float *dlog_alpha, float *dbeta, float *d_init_state, void *workspace,
+                         size_t workspace_bytes, kda_stream_t stream_, bool scalar_gate) {
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    if (num_seqs < 1 || total_tokens < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_BF16 && dtype != KDA_FP32) return KDA_ERR_INVALID_ARG;
+    const bool dims_ok = (d_k == 32 || d_k == 64 || d_k == 128) && d_v % 32 == 0 &&
+                         d_v >= 32 && d_v <= 128;
+    if (!dims_ok) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)num_seqs * H * (d_v / 32) > INT_MAX) return KDA_ERR_UNSUPPORTED;
+    if (!cu_seqlens && total_tokens % num_seqs != 0) return KDA_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !d_o || !dq || !dk ||
+                             !dv || !dlog_alpha || !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    const size_t eb = elem_bytes(dtype);
+    // v and d_o are read 4 columns at a time; states and dv 16 bytes at a time
+    const void *p16[] = {v, d_o, init_state, d_final_state, dv, d_init_state};
+    for (const void *p : p16)
+        if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    const void *pe[] = {q, k, log_alpha, beta};
+    for (const void *p : pe)
+        if (p && !aligned_to(p, eb)) return KDA_ERR_INVALID_ARG;
+    const void *p4[] = {dq, dk, dlog_alpha, dbeta, cu_seqlens};
+    for (const void *p : p4)
+        if (p && !aligned_to(p, 4)) return KDA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kda::backward_workspace(num_seqs, total_tokens, H, d_k, d_v))
+        return KDA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_INVALID_ARG;
+
+    // no output may overlap an input, the workspace or another output
+    const size_t nk = (size_t)total_tokens * H * d_k, nv = (size_t)total_tokens * H * d_v;
+    const size_t nb = (size_t)total_tokens * H, ng = scalar_gate ? nb : nk;
+    const size_t ns = (size_t)num_seqs * H * d_k * d_v;
+    struct Span { const void *p; size_t n; };
+    const Span ins[] = {{q, nk * eb}, {k, nk * eb}, {v, nv * eb}, {log_alpha, ng * eb},
+                        {beta, nb * eb}, {d_o, nv * eb}, {init_state, ns * 4},
+                        {d_final_state, ns * 4}, {cu_seqlens, ((size_t)num_seqs + 1) * 4},
+                        {workspace, workspace_bytes}};
+    const Span outs[] = {{dq, nk * 4}, {dk, nk * 4}, {dv, nv * 4}, {dlog_alpha, ng * 4},
+                         {dbeta, nb * 4}, {d_init_state, ns * 4}};
+    for (const Span &o : outs) {
+        for (const Span &i : ins)
+            if (overlaps(o.p, o.n, i.p, i.n)) return KDA_ERR_INVALID_ARG;
+        for (const Span &o2 : outs)
+            if (&o2 != &o && overlaps(o.p, o.n, o2.p, o2.n)) return KDA_ERR_INVALID_ARG;
+    }
+    return from_cuda(kda::launch_backward(q, k, v, log_alpha, beta, init_state, cu_seqlens,
+                                          num_seqs, total_tokens, H, d_k, d_v, dtype, d_o,
+                                          d_final_state, dq, dk, dv, dlog_alpha, dbeta,
+                                          d_init_state, workspace, scalar_gate, stream));
+}
+
 }  // namespace
 
 extern "C" {
@@ -308,6 +365,40 @@ kda_status kda_cp_finish(const void *v, const float *S_in, int64_t total_tokens,
     return from_cuda(kda::launch_prefill_split(nullptr, nullptr, v, nullptr, nullptr, S_in, nullptr,
                                                1, total_tokens, H, o, final_state, workspace,
                                                false, nullptr, stream, kda::kCpFinish, nullptr));
+}
+
+size_t kda_backward_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                   int32_t d_k, int32_t d_v) {
+    if (num_seqs < 1 || total_tokens < 0 || H < 1 || d_k < 32 || d_k > 128 || d_v < 32 ||
+        d_v > 128 || d_v % 32 != 0)
+        return 0;
+    return kda::backward_workspace(num_seqs, total_tokens, H, d_k, d_v);
+}
+
+kda_status kda_backward(const void *q, const void *k, const void *v, const void *log_alpha,
+                        const void *beta, const float *init_state, const int32_t *cu_seqlens,
+                        int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                        int32_t d_v, kda_dtype dtype, const void *d_o,
+                        const float *d_final_state, float *dq, float *dk, float *dv,
+                        float *dlog_alpha, float *dbeta, float *d_init_state, void *workspace,
+                        size_t workspace_bytes, kda_stream_t stream) {
+    return backward_impl(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
+                         total_tokens, H, d_k, d_v, dtype, d_o, d_final_state, dq, dk, dv,
+                         dlog_alpha, dbeta, d_init_state, workspace, workspace_bytes, stream,
+                         false);
+}
+
+kda_status gdn_backward(const void *q, const void *k, const void *v, const void *log_alpha,
+                        const void *beta, const float *init_state, const int32_t *cu_seqlens,
+                        int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                        int32_t d_v, kda_dtype dtype, const void *d_o,
+                        const float *d_final_state, float *dq, float *dk, float *dv,
+                        float *dlog_alpha, float *dbeta, float *d_init_state, void *workspace,
+                        size_t workspace_bytes, kda_stream_t stream) {
+    return backward_impl(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs,
+                         total_tokens, H, d_k, d_v, dtype, d_o, d_final_state, dq, dk, dv,
+                         dlog_alpha, dbeta, d_init_state, workspace, workspace_bytes, stream,
+                         true);
 }
 
 kda_status kda_check_workspace_error(const void *workspace, kda_stream_t stream_) {

@@ -1,0 +1,440 @@
+// KDA backward pass (training): the reverse-mode derivative of the recurrence
+//
+//     Sp = Diag(exp(g_t)) S_{t-1},  r = Sp^T k_t,  u = beta_t (v_t - r),
+//     S_t = Sp + k_t u^T,           o_t = S_t^T q_t
+//
+// (page "Kimi Linear" on docsaid.org, section "KDA : une decroissance propre
+// a chaque canal", the KDA update; the news digest page on Kimi Linear,
+// section "Algorithme parallele par chunks", organises the operator for
+// training).  Step t read backwards, with dS = dL/dS_t:
+//
+//     dS += q do^T;         dq = S_t do
+//     du  = dS^T k;         dk = dS u
+//     dbeta = du . (v - r); dv = beta du;   dr = -beta du
+//     dS += k dr^T;         dk += Sp dr          (dS is now dL/dSp)
+//     dg[c] = sum_j Sp[c][j] dS[c][j];      dS = Diag(exp(g_t)) dS
+//
+// Layout.  Every column of the state follows its own recurrence (the step
+// reads column j only through r_j and u_j), so a CTA owns a 32-column slice of
+// one (sequence, head) and runs the whole sequence: 8 warps of 4 columns, a
+// lane holding d_k/32 key rows of its warp's columns (16 fp32 of S and 16 of
+// dS at d_k = 128, in registers).  Column sums over the key rows (r, du) are
+// warp shuffles; row sums over the columns (dq, dk, dg, dbeta) are partials
+// per warp, summed over the CTA's warps in shared memory every 4 steps and
+// over the head's slices by fp32 atomic adds into the zeroed gradients.
+//
+// States entering the steps come from a forward pass that keeps the state
+// entering every block of 64 steps in the workspace; each block is then run
+// forward once more from its kept state, writing the 64 states entering its
+// steps into the CTA's own scratch (L2-resident), and backward from its end.
+// The same thread writes and reads every scratch element, so no barrier
+// orders them.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kBwdWarps = 8;
+constexpr int kBwdThreads = 32 * kBwdWarps;
+constexpr int kBwdCols = 4;                        // d_v columns per warp
+constexpr int kBwdSlice = kBwdWarps * kBwdCols;    // d_v columns per CTA
+constexpr int kBwdBlock = 64;                      // steps between kept states
+constexpr int kBwdGroup = 4;                       // steps per shared-memory reduction
+constexpr int kBwdMaxCtas = 2 * 148;               // resident CTAs on a B200 (2 per SM)
+
+template <int DK>
+struct BwdShape {
+    static constexpr int RPL = DK / 32;                  // key rows per lane
+    static constexpr int E = 3 * DK + 2;                 // a warp's partials of one step
+    static constexpr int STATE4 = DK * kBwdSlice / 4;    // float4s in a state slice
+    static constexpr size_t SMEM = 2ull * kBwdGroup * kBwdWarps * E * sizeof(float);
+    static_assert(DK % 32 == 0, "d_k must be a multiple of 32");
+};
+
+struct BwdArgs {
+    const void *q, *k, *v, *g, *beta, *d_o;
+    const float *init_state, *d_final_state;
+    const int32_t *cu_seqlens;
+    float *dq, *dk, *dv, *dg, *dbeta, *d_init_state;
+    float4 *ckpt, *scratch;
+    uint32_t *err_word;
+    int64_t seq_len;     // tokens per sequence when cu_seqlens is null
+    int64_t total_tokens;
+    int H, dv_total, nslices, units, scalar_gate;
+};
+
+template <typename T> __device__ __forceinline__ float4 load4(const T *p);
+template <> __device__ __forceinline__ float4 load4<float>(const float *p) {
+    return *reinterpret_cast<const float4 *>(p);
+}
+template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16 *p) {
+    const uint2 w = *reinterpret_cast<const uint2 *>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ float4 f4(float x) { return make_float4(x, x, x, x); }
+__device__ __forceinline__ float4 sub4(float4 a, float4 b) {
+    return make_float4(a.x - b.x, a.y - b.y, a.z - b.z, a.w - b.w);
+}
+__device__ __forceinline__ float4 mul4(float4 a, float s) {
+    return make_float4(a.x * s, a.y * s, a.z * s, a.w * s);
+}
+// acc + a * s
+__device__ __forceinline__ float4 fma4s(float4 a, float s, float4 acc) {
+    return make_float4(fmaf(a.x, s, acc.x), fmaf(a.y, s, acc.y), fmaf(a.z, s, acc.z),
+                       fmaf(a.w, s, acc.w));
+}
+__device__ __forceinline__ float dot4(float4 a, float4 b) {
+    return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
+}
+__device__ __forceinline__ float4 warp_sum4(float4 x) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        x.x += __shfl_xor_sync(0xffffffffu, x.x, off);
+        x.y += __shfl_xor_sync(0xffffffffu, x.y, off);
+        x.z += __shfl_xor_sync(0xffffffffu, x.z, off);
+        x.w += __shfl_xor_sync(0xffffffffu, x.w, off);
+    }
+    return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+// One step's inputs as a lane needs them: its key rows of k, q and the decay,
+// its warp's 4 columns of v and do, and beta.
+template <int RPL>
+struct StepIn {
+    float k[RPL], q[RPL], a[RPL];
+    float4 v, d;
+    float b;
+};
+
+template <typename T, int DK, bool BWD>
+__device__ __forceinline__ void load_step(StepIn<DK / 32> &s, const BwdArgs &p, int64_t t, int h,
+                                          int lane, int j0) {
+    constexpr int RPL = DK / 32;
+    const size_t row = (size_t)t * p.H + h;
+    const T *kp = static_cast<const T *>(p.k) + row * DK + lane;
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) s.k[i] = io<T>::load(kp + 32 * i);
+    if (p.scalar_gate) {
+        const float a = expf(io<T>::load(static_cast<const T *>(p.g) + row));
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) s.a[i] = a;
+    } else {
+        const T *gp = static_cast<const T *>(p.g) + row * DK + lane;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) s.a[i] = expf(io<T>::load(gp + 32 * i));
+    }
+    s.v = load4<T>(static_cast<const T *>(p.v) + row * p.dv_total + j0);
+    s.b = io<T>::load(static_cast<const T *>(p.beta) + row);
+    if (BWD) {
+        const T *qp = static_cast<const T *>(p.q) + row * DK + lane;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) s.q[i] = io<T>::load(qp + 32 * i);
+        s.d = load4<T>(static_cast<const T *>(p.d_o) + row * p.dv_total + j0);
+    }
+}
+
+// S <- S_t from S_{t-1}.
+template <int RPL>
+__device__ __forceinline__ void forward_step(float4 (&S)[RPL], const StepIn<RPL> &in) {
+    float4 rp = f4(0.f);
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+        S[i] = mul4(S[i], in.a[i]);
+        rp = fma4s(S[i], in.k[i], rp);
+    }
+    const float4 u = mul4(sub4(in.v, warp_sum4(rp)), in.b);
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) S[i] = fma4s(u, in.k[i], S[i]);
+}
+
+// Forward over steps [t0, t1) with the next step's inputs loaded one step ahead;
+// with `keep`, the state entering each step is written to keep[step - t0].
+template <typename T, int DK>
+__device__ __forceinline__ void forward_run(float4 (&S)[DK / 32], const BwdArgs &p, int64_t t0,
+                                            int64_t t1, int h, int lane, int j0, float4 *keep,
+                                            int idx) {
+    constexpr int RPL = DK / 32;
+    constexpr int S4 = BwdShape<DK>::STATE4;
+    StepIn<RPL> cur, nxt;
+    if (t0 < t1) load_step<T, DK, false>(nxt, p, t0, h, lane, j0);
+#pragma unroll 1
+    for (int64_t t = t0; t < t1; ++t) {
+        cur = nxt;
+        if (t + 1 < t1) load_step<T, DK, false>(nxt, p, t + 1, h, lane, j0);
+        if (keep) {
+#pragma unroll
+            for (int i = 0; i < RPL; ++i) keep[(size_t)(t - t0) * S4 + idx + i * kBwdThreads] = S[i];
+        }
+        forward_step<RPL>(S, cur);
+    }
+}
+
+// Sums the group's per-warp partials over the warps and adds them to the
+// gradients (count steps, the first of them at token t_hi, then t_hi - 1, ...).
+template <int DK>
+__device__ __forceinline__ void flush_group(const float *red, int count, int64_t t_hi, int h,
+                                            const BwdArgs &p) {
+    constexpr int E = BwdShape<DK>::E;
+    for (int idx = threadIdx.x; idx < count * E; idx += kBwdThreads) {
+        const int gi = idx / E, e = idx - gi * E;
+        const float *src = red + (size_t)gi * kBwdWarps * E + e;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kBwdWarps; ++w) acc += src[w * E];
+        const size_t row = (size_t)(t_hi - gi) * p.H + h;
+        if (e < DK) {
+            atomicAdd(p.dq + row * DK + e, acc);
+        } else if (e < 2 * DK) {
+            atomicAdd(p.dk + row * DK + (e - DK), acc);
+        } else if (e < 3 * DK) {
+            if (!p.scalar_gate) atomicAdd(p.dg + row * DK + (e - 2 * DK), acc);
+        } else if (e == 3 * DK) {
+            atomicAdd(p.dbeta + row, acc);
+        } else if (p.scalar_gate) {
+            atomicAdd(p.dg + row, acc);
+        }
+    }
+}
+
+template <typename T, int DK>
+__global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_kernel(const BwdArgs p) {
+    using Sh = BwdShape<DK>;
+    constexpr int RPL = Sh::RPL, E = Sh::E, S4 = Sh::STATE4;
+    extern __shared__ float red[];   // [2][kBwdGroup][kBwdWarps][E]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // a thread's float4 i of a state slice: key row lane + 32 i, its warp's columns
+    const int idx = warp * 32 + lane;
+    float4 *scratch = p.scratch + (size_t)blockIdx.x * kBwdBlock * S4;
+    int buf = 0;
+
+#pragma unroll 1
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+        const int s = u % p.nslices;
+        const int h = (u / p.nslices) % p.H;
+        const int n = u / (p.nslices * p.H);
+        int64_t bos, eos;
+        if (p.cu_seqlens) {
+            bos = p.cu_seqlens[n];
+            eos = p.cu_seqlens[n + 1];
+            if (bos < 0 || eos < bos || eos > p.total_tokens) {   // uniform over the CTA
+                if (threadIdx.x == 0) atomicOr(p.err_word, kDevErrCuSeqlens);
+                continue;
+            }
+        } else {
+            bos = (int64_t)n * p.seq_len;
+            eos = bos + p.seq_len;
+        }
+        const int j0 = s * kBwdSlice + warp * kBwdCols;
+        const int64_t nb = (eos - bos + kBwdBlock - 1) / kBwdBlock;
+        // Kept states: sequence n's blocks start at slot bos / 64 + n, which
+        // leaves the slot ranges of consecutive sequences disjoint.
+        const int64_t slot0 = bos / kBwdBlock + n;
+        const size_t st = ((size_t)n * p.H + h) * DK * p.dv_total + j0;   // [N, H, d_k, d_v]
+
+        float4 S[RPL];
+#pragma unroll
+        for (int i = 0; i < RPL; ++i)
+            S[i] = p.init_state ? *reinterpret_cast<const float4 *>(
+                                      p.init_state + st + (size_t)(lane + 32 * i) * p.dv_total)
+                                : f4(0.f);
+        // Forward: keep the state entering every block.
+#pragma unroll 1
+        for (int64_t b = 0; b < nb; ++b) {
+            float4 *ck = p.ckpt + (((size_t)(slot0 + b) * p.H + h) * p.nslices + s) * S4;
+#pragma unroll
+            for (int i = 0; i < RPL; ++i) ck[idx + i * kBwdThreads] = S[i];
+            if (b == nb - 1) break;
+            const int64_t t0 = bos + b * kBwdBlock;
+            forward_run<T, DK>(S, p, t0, t0 + kBwdBlock, h, lane, j0, nullptr, idx);
+        }
+
+        float4 dS[RPL];
+#pragma unroll
+        for (int i = 0; i < RPL; ++i)
+            dS[i] = p.d_final_state ? *reinterpret_cast<const float4 *>(
+                                          p.d_final_state + st + (size_t)(lane + 32 * i) * p.dv_total)
+                                    : f4(0.f);
+        int gi = 0;
+        int64_t g_hi = 0;
+#pragma unroll 1
+        for (int64_t b = nb - 1; b >= 0; --b) {
+            const int64_t tb = bos + b * kBwdBlock;
+            const int64_t te = (tb + kBwdBlock < eos) ? tb + kBwdBlock : eos;
+            const float4 *ck = p.ckpt + (((size_t)(slot0 + b) * p.H + h) * p.nslices + s) * S4;
+#pragma unroll
+            for (int i = 0; i < RPL; ++i) S[i] = ck[idx + i * kBwdThreads];
+            forward_run<T, DK>(S, p, tb, te, h, lane, j0, scratch, idx);
+
+            // Backward over the block, the next step's inputs and entering
+            // state loaded one step ahead.
+            StepIn<RPL> cur, nxt;
+            float4 Sn[RPL];
+            load_step<T, DK, true>(nxt, p, te - 1, h, lane, j0);
+#pragma unroll
+            for (int i = 0; i < RPL; ++i) Sn[i] = scratch[(size_t)(te - 1 - tb) * S4 + idx + i * kBwdThreads];
+#pragma unroll 1
+            for (int64_t t = te - 1; t >= tb; --t) {
+                cur = nxt;
+                float4 sp[RPL];
+#pragma unroll
+                for (int i = 0; i < RPL; ++i) sp[i] = Sn[i];
+                if (t - 1 >= tb) {
+                    load_step<T, DK, true>(nxt, p, t - 1, h, lane, j0);
+#pragma unroll
+                    for (int i = 0; i < RPL; ++i)
+                        Sn[i] = scratch[(size_t)(t - 1 - tb) * S4 + idx + i * kBwdThreads];
+                }
+                // the step again: Sp, r, u
+                float4 rp = f4(0.f);
+#pragma unroll
+                for (int i = 0; i < RPL; ++i) {
+                    sp[i] = mul4(sp[i], cur.a[i]);
+                    rp = fma4s(sp[i], cur.k[i], rp);
+                }
+                const float4 r = warp_sum4(rp);
+                const float4 vr = sub4(cur.v, r);
+                const float4 uu = mul4(vr, cur.b);
+                // o_t = S_t^T q, S_t = Sp + k u^T
+                float dq_r[RPL], dk_r[RPL], dg_r[RPL];
+                float4 dup = f4(0.f);
+#pragma unroll
+                for (int i = 0; i < RPL; ++i) {
+                    dS[i] = fma4s(cur.d, cur.q[i], dS[i]);
+                    dq_r[i] = dot4(fma4s(uu, cur.k[i], sp[i]), cur.d);
+                    dup = fma4s(dS[i], cur.k[i], dup);
+                    dk_r[i] = dot4(dS[i], uu);
+                }
+                const float4 du = warp_sum4(dup);
+                const float dbeta = dot4(du, vr);
+                const size_t row = (size_t)t * p.H + h;
+                if (lane == 0)
+                    *reinterpret_cast<float4 *>(p.dv + row * p.dv_total + j0) = mul4(du, cur.b);
+                const float4 dr = mul4(du, -cur.b);
+                float gsum = 0.f;
+#pragma unroll
+                for (int i = 0; i < RPL; ++i) {
+                    dS[i] = fma4s(dr, cur.k[i], dS[i]);
+                    dk_r[i] += dot4(sp[i], dr);
+                    dg_r[i] = dot4(sp[i], dS[i]);
+                    gsum += dg_r[i];
+                    dS[i] = mul4(dS[i], cur.a[i]);
+                }
+                // this warp's row partials of the step
+                float *slot = red + ((size_t)(buf * kBwdGroup + gi) * kBwdWarps + warp) * E;
+#pragma unroll
+                for (int i = 0; i < RPL; ++i) {
+                    slot[lane + 32 * i] = dq_r[i];
+                    slot[DK + lane + 32 * i] = dk_r[i];
+                    slot[2 * DK + lane + 32 * i] = dg_r[i];
+                }
+                if (p.scalar_gate) gsum = warp_sum(gsum);
+                if (lane == 0) {
+                    slot[3 * DK] = dbeta;
+                    slot[3 * DK + 1] = gsum;
+                }
+                if (gi == 0) g_hi = t;
+                ++gi;
+                if (gi == kBwdGroup || t == bos) {
+                    // One barrier per group: the two buffers alternate, and a
+                    // buffer is written again only after the next group's
+                    // barrier, which every thread reaches after this flush.
+                    __syncthreads();
+                    flush_group<DK>(red + (size_t)buf * kBwdGroup * kBwdWarps * E, gi, g_hi, h, p);
+                    buf ^= 1;
+                    gi = 0;
+                }
+            }
+        }
+        if (p.d_init_state) {
+#pragma unroll
+            for (int i = 0; i < RPL; ++i)
+                *reinterpret_cast<float4 *>(p.d_init_state + st + (size_t)(lane + 32 * i) * p.dv_total) = dS[i];
+        }
+    }
+}
+
+template <typename T, int DK>
+cudaError_t launch_dk(const BwdArgs &p, int grid, cudaStream_t stream) {
+    const size_t smem = BwdShape<DK>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(kda_backward_kernel<T, DK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kda_backward_kernel<T, DK><<<grid, kBwdThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+size_t bwd_slots(int num_seqs, int64_t total_tokens) {
+    return (size_t)(total_tokens / kBwdBlock) + (size_t)num_seqs + 1;
+}
+
+int bwd_grid(int num_seqs, int H, int d_v) {
+    const int64_t units = (int64_t)num_seqs * H * (d_v / kBwdSlice);
+    return (int)(units < kBwdMaxCtas ? units : kBwdMaxCtas);
+}
+
+}  // namespace
+
+size_t backward_workspace(int num_seqs, int64_t total_tokens, int H, int dk, int dv) {
+    const size_t state = (size_t)dk * kBwdSlice * sizeof(float);   // one slice
+    const size_t nsl = (size_t)(dv / kBwdSlice);
+    return kWorkspaceHeader + bwd_slots(num_seqs, total_tokens) * H * nsl * state +
+           (size_t)bwd_grid(num_seqs, H, dv) * kBwdBlock * state;
+}
+
+cudaError_t launch_backward(const void *q, const void *k, const void *v, const void *g,
+                            const void *beta, const float *init_state, const int32_t *cu,
+                            int num_seqs, int64_t total_tokens, int H, int dk, int dv,
+                            kda_dtype dtype, const void *d_o, const float *d_final_state,
+                            float *dq, float *dk_out, float *dv_out, float *dg, float *dbeta,
+                            float *d_init_state, void *workspace, bool scalar_gate,
+                            cudaStream_t stream) {
+    const size_t ng = (size_t)total_tokens * H * (scalar_gate ? 1 : dk);
+    const size_t nk = (size_t)total_tokens * H * dk;
+    uint32_t *err_word = static_cast<uint32_t *>(workspace);
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(err_word, 0, sizeof(uint32_t), stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dq, 0, nk * sizeof(float), stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dk_out, 0, nk * sizeof(float), stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dg, 0, ng * sizeof(float), stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dbeta, 0, (size_t)total_tokens * H * sizeof(float), stream)) != cudaSuccess)
+        return e;
+
+    BwdArgs p;
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.d_o = d_o;
+    p.init_state = init_state;
+    p.d_final_state = d_final_state;
+    p.cu_seqlens = cu;
+    p.dq = dq; p.dk = dk_out; p.dv = dv_out; p.dg = dg; p.dbeta = dbeta;
+    p.d_init_state = d_init_state;
+    p.err_word = err_word;
+    p.seq_len = cu ? 0 : total_tokens / num_seqs;
+    p.total_tokens = total_tokens;
+    p.H = H;
+    p.dv_total = dv;
+    p.nslices = dv / kBwdSlice;
+    p.units = num_seqs * H * p.nslices;
+    p.scalar_gate = scalar_gate ? 1 : 0;
+    const size_t state = (size_t)dk * kBwdSlice * sizeof(float);
+    uint8_t *base = static_cast<uint8_t *>(workspace) + kWorkspaceHeader;
+    p.ckpt = reinterpret_cast<float4 *>(base);
+    p.scratch = reinterpret_cast<float4 *>(base + bwd_slots(num_seqs, total_tokens) * H * p.nslices * state);
+    const int grid = bwd_grid(num_seqs, H, dv);
+    if (grid == 0) return cudaGetLastError();
+    const bool bf = dtype == KDA_BF16;
+    switch (dk) {
+        case 32: return bf ? launch_dk<__nv_bfloat16, 32>(p, grid, stream) : launch_dk<float, 32>(p, grid, stream);
+        case 64: return bf ? launch_dk<__nv_bfloat16, 64>(p, grid, stream) : launch_dk<float, 64>(p, grid, stream);
+        case 128: return bf ? launch_dk<__nv_bfloat16, 128>(p, grid, stream) : launch_dk<float, 128>(p, grid, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace kda

@@ -114,6 +114,19 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                  const LayerArgs *layer, cudaStream_t stream,
                                  int cp_mode = kCpNone, float *cp_transition = nullptr);
 
+// Backward pass (fp32 gradients; d_k and d_v multiples of 32 up to 128).
+// Its workspace keeps the state entering every 64-step block of every
+// (sequence, head) and gives each CTA a 64-state scratch.
+size_t backward_workspace(int num_seqs, int64_t total_tokens, int H, int dk, int dv);
+
+cudaError_t launch_backward(const void *q, const void *k, const void *v, const void *g,
+                            const void *beta, const float *init_state, const int32_t *cu,
+                            int num_seqs, int64_t total_tokens, int H, int dk, int dv,
+                            kda_dtype dtype, const void *d_o, const float *d_final_state,
+                            float *dq, float *dk_out, float *dv_out, float *dg, float *dbeta,
+                            float *d_init_state, void *workspace, bool scalar_gate,
+                            cudaStream_t stream);
+
 // Context parallelism: S_out = the state a segment starts from, given the
 // (M_i, S~_i) of the n_prev segments before it and the sequence's S_0 (or null).
 cudaError_t launch_cp_combine(const float *M, const float *S_tilde, const float *S0, float *S_out,

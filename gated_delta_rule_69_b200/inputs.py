@@ -131,6 +131,19 @@ def generate(w: Workload, device: str = "cpu", lengths=None) -> dict:
                 cu_seqlens=cu.to(device), lengths=lengths)
 
 
+def cotangents(w: Workload, lengths, device: str = "cpu", seed_offset: int = 500) -> dict:
+    """Seeded upstream gradients for the backward pass (the pages train the
+    layer but give no gradient statistics; a loss's gradients are taken as
+    N(0, 1) per output element and N(0, 0.02^2) per final-state element):
+    d_o [T_tot, H, d_v] in the I/O dtype, d_final_state [N, H, d_k, d_v] fp32.
+    Drawn from their own generator (seed + seed_offset)."""
+    gen = torch.Generator(device=device).manual_seed(w.seed + seed_offset)
+    T, n = int(sum(lengths)), len(lengths)
+    d_o = _normal((T, w.H, w.d_v), gen, device=device).to(_TORCH_DTYPE[w.dtype])
+    d_fs = _normal((n, w.H, w.d_k, w.d_v), gen, std=0.02, device=device)
+    return dict(d_o=d_o, d_final_state=d_fs)
+
+
 def as_float64(t):
     """Exact widening of a tensor's values to a float64 numpy array (for the
     oracle)."""

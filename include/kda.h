@@ -272,9 +272,58 @@ kda_status kda_cp_finish(const void *v, const float *S_in, int64_t total_tokens,
                          void *workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
- * Synchronises `stream`, then reads the error word that the prefill kernels
- * leave at the start of `workspace` (non-zero when a device-side check failed,
- * e.g. cu_seqlens not non-decreasing or not ending at T_total).  Returns
+ * Backward pass (training): the gradients of a loss L through the recurrence
+ * of kda_prefill, given dL/do and dL/dS_T (news digest page on Kimi Linear,
+ * section "Algorithme parallele par chunks", which organises the operator for
+ * training; the derivative is the chain rule through each step of the KDA
+ * update of page "Kimi Linear" on docsaid.org, section "KDA : une
+ * decroissance propre a chaque canal").
+ *
+ * Inputs are those of kda_prefill (same layouts, dtype, init_state NULL =
+ * zeros, cu_seqlens NULL = num_seqs equal sequences), plus
+ *   d_o            [T_total, H, d_v] in `dtype`: dL/do
+ *   d_final_state  [N, H, d_k, d_v] fp32 or NULL (zero): dL/dS_T
+ * Outputs, fp32, written in full (never accumulated):
+ *   dq, dk, dlog_alpha [T_total, H, d_k];  dv [T_total, H, d_v];
+ *   dbeta [T_total, H];  d_init_state [N, H, d_k, d_v] or NULL (not wanted).
+ * gdn_backward is the same for the Gated DeltaNet gate: log_alpha and
+ * dlog_alpha are [T_total, H].
+ *
+ * Shapes: d_k in {32, 64, 128}; d_v in {32, 64, 96, 128}; else
+ * KDA_ERR_UNSUPPORTED.  Alignment: v, d_o, the fp32 states and dv 16 bytes;
+ * the other inputs their element; the other outputs 4 bytes.  No output may
+ * overlap an input, the workspace or another output (KDA_ERR_INVALID_ARG).
+ * The workspace (256-byte aligned, kda_backward_workspace_size bytes) keeps
+ * the state entering every 64-token block of every (sequence, head), about
+ * T_total * H * d_k * d_v / 16 bytes, plus a per-CTA scratch.  The gradients
+ * are summed with fp32 atomic adds, so their last bits may differ from run to
+ * run.  A cu_seqlens entry out of order or past T_total skips that sequence
+ * and sets the workspace error word (kda_check_workspace_error).
+ */
+size_t kda_backward_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                   int32_t d_k, int32_t d_v);
+
+kda_status kda_backward(const void *q, const void *k, const void *v, const void *log_alpha,
+                        const void *beta, const float *init_state, const int32_t *cu_seqlens,
+                        int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                        int32_t d_v, kda_dtype dtype, const void *d_o,
+                        const float *d_final_state, float *dq, float *dk, float *dv,
+                        float *dlog_alpha, float *dbeta, float *d_init_state, void *workspace,
+                        size_t workspace_bytes, kda_stream_t stream);
+
+kda_status gdn_backward(const void *q, const void *k, const void *v, const void *log_alpha,
+                        const void *beta, const float *init_state, const int32_t *cu_seqlens,
+                        int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                        int32_t d_v, kda_dtype dtype, const void *d_o,
+                        const float *d_final_state, float *dq, float *dk, float *dv,
+                        float *dlog_alpha, float *dbeta, float *d_init_state, void *workspace,
+                        size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads the error word that the prefill and
+ * backward kernels leave at the start of `workspace` (non-zero when a
+ * device-side check failed, e.g. cu_seqlens not non-decreasing or not ending
+ * at T_total).  Returns
  * KDA_ERR_INVALID_ARG in that case, KDA_OK otherwise.  Debugging aid; the
  * only call here that blocks.
  */

@@ -136,3 +136,42 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(4, 1, 16)
     with pytest.raises((ValueError, RuntimeError, AssertionError)):
         kda.kda_decode_step(x, x, x, x, torch.zeros(4, 1), torch.zeros(4, 1, 16, 16))
+
+
+def _backward(L, fn="kda_backward", **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, g=FAKE * 4, b=FAKE * 5, s0=None, cu=None,
+             n=1, T=64, H=1, dk=32, dv=32, dt=1, do=FAKE * 6, dfs=None, dq=FAKE * 64,
+             dkk=FAKE * 65, dvv=FAKE * 66, dg=FAKE * 67, db=FAKE * 68, ds0=None,
+             ws=FAKE * 128, wsb=1 << 30)
+    a.update(kw)
+    return getattr(L, fn)(a["q"], a["k"], a["v"], a["g"], a["b"], a["s0"], a["cu"], a["n"],
+                          a["T"], a["H"], a["dk"], a["dv"], a["dt"], a["do"], a["dfs"],
+                          a["dq"], a["dkk"], a["dvv"], a["dg"], a["db"], a["ds0"], a["ws"],
+                          a["wsb"], None)
+
+
+def test_backward_workspace_size(L):
+    ws = L.kda_backward_workspace_size
+    # kept states: one 128 x 128 fp32 state per 64 tokens per head, plus slack per sequence
+    assert ws(1, 4096, 16, 128, 128) >= 4096 // 64 * 16 * 128 * 128 * 4
+    assert ws(0, 64, 1, 32, 32) == 0
+    assert ws(1, 64, 1, 16, 32) == 0
+    assert ws(1, 64, 1, 32, 48) == 0
+
+
+def test_backward_rejects_on_host(L):
+    for fn in ("kda_backward", "gdn_backward"):
+        assert _backward(L, fn, n=0) == 1
+        assert _backward(L, fn, dt=5) == 1
+        assert _backward(L, fn, dk=16) == 2
+        assert _backward(L, fn, dv=48) == 2
+        assert _backward(L, fn, do=None) == 1
+        assert _backward(L, fn, dq=None) == 1
+        assert _backward(L, fn, n=3) == 1                   # T % N != 0 without cu_seqlens
+        assert _backward(L, fn, v=FAKE * 3 + 4) == 1        # v not 16-byte aligned
+        assert _backward(L, fn, dvv=FAKE * 66 + 8) == 1     # dv not 16-byte aligned
+        assert _backward(L, fn, wsb=1024) == 3
+        assert _backward(L, fn, ws=FAKE * 128 + 16) == 1    # workspace not 256-aligned
+        assert _backward(L, fn, dq=FAKE + 64) == 1          # dq overlaps q
+        assert _backward(L, fn, dkk=FAKE * 64 + 64) == 1    # dk overlaps dq
+        assert _backward(L, fn, ds0=FAKE * 128 + 4096) == 1  # d_init_state inside the workspace
