@@ -63,17 +63,6 @@ struct BwdArgs {
     int H, dv_total, nslices, units, scalar_gate;
 };
 
-template <typename T> __device__ __forceinline__ float4 load4(const T *p);
-template <> __device__ __forceinline__ float4 load4<float>(const float *p) {
-    return *reinterpret_cast<const float4 *>(p);
-}
-template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16 *p) {
-    const uint2 w = *reinterpret_cast<const uint2 *>(p);
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.y));
-    return make_float4(a.x, a.y, b.x, b.y);
-}
-
 __device__ __forceinline__ float4 f4(float x) { return make_float4(x, x, x, x); }
 __device__ __forceinline__ float4 sub4(float4 a, float4 b) {
     return make_float4(a.x - b.x, a.y - b.y, a.z - b.z, a.w - b.w);
@@ -114,66 +103,121 @@ struct StepIn {
     float b;
 };
 
+// The same inputs as loaded, unconverted: a load issued a step ahead is then
+// first waited for in the step that uses it (converting at the load would
+// wait for it there).
+template <typename T> struct Raw4;
+template <> struct Raw4<float> { using type = float4; };
+template <> struct Raw4<__nv_bfloat16> { using type = uint2; };
+
+template <typename T, int RPL>
+struct StepRaw {
+    T k[RPL], q[RPL], g[RPL];
+    typename Raw4<T>::type v, d;
+    T b;
+};
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float4 to_f4(float4 x) { return x; }
+__device__ __forceinline__ float4 to_f4(uint2 w) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
 template <typename T, int DK, bool BWD>
-__device__ __forceinline__ void load_step(StepIn<DK / 32> &s, const BwdArgs &p, int64_t t, int h,
-                                          int lane, int j0) {
+__device__ __forceinline__ void load_step(StepRaw<T, DK / 32> &s, const BwdArgs &p, int64_t t,
+                                          int h, int lane, int j0) {
     constexpr int RPL = DK / 32;
+    using R4 = typename Raw4<T>::type;
     const size_t row = (size_t)t * p.H + h;
     const T *kp = static_cast<const T *>(p.k) + row * DK + lane;
 #pragma unroll
-    for (int i = 0; i < RPL; ++i) s.k[i] = io<T>::load(kp + 32 * i);
+    for (int i = 0; i < RPL; ++i) s.k[i] = kp[32 * i];
     if (p.scalar_gate) {
-        const float a = expf(io<T>::load(static_cast<const T *>(p.g) + row));
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) s.a[i] = a;
+        s.g[0] = static_cast<const T *>(p.g)[row];
     } else {
         const T *gp = static_cast<const T *>(p.g) + row * DK + lane;
 #pragma unroll
-        for (int i = 0; i < RPL; ++i) s.a[i] = expf(io<T>::load(gp + 32 * i));
+        for (int i = 0; i < RPL; ++i) s.g[i] = gp[32 * i];
     }
-    s.v = load4<T>(static_cast<const T *>(p.v) + row * p.dv_total + j0);
-    s.b = io<T>::load(static_cast<const T *>(p.beta) + row);
+    s.v = *reinterpret_cast<const R4 *>(static_cast<const T *>(p.v) + row * p.dv_total + j0);
+    s.b = static_cast<const T *>(p.beta)[row];
     if (BWD) {
         const T *qp = static_cast<const T *>(p.q) + row * DK + lane;
 #pragma unroll
-        for (int i = 0; i < RPL; ++i) s.q[i] = io<T>::load(qp + 32 * i);
-        s.d = load4<T>(static_cast<const T *>(p.d_o) + row * p.dv_total + j0);
+        for (int i = 0; i < RPL; ++i) s.q[i] = qp[32 * i];
+        s.d = *reinterpret_cast<const R4 *>(static_cast<const T *>(p.d_o) + row * p.dv_total + j0);
     }
 }
 
-// S <- S_t from S_{t-1}.
+template <typename T, int RPL, bool BWD>
+__device__ __forceinline__ void decode_step(StepIn<RPL> &s, const StepRaw<T, RPL> &r,
+                                            int scalar_gate) {
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) s.k[i] = to_f(r.k[i]);
+    if (scalar_gate) {
+        const float a = expf(to_f(r.g[0]));
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) s.a[i] = a;
+    } else {
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) s.a[i] = expf(to_f(r.g[i]));
+    }
+    s.v = to_f4(r.v);
+    s.b = to_f(r.b);
+    if (BWD) {
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) s.q[i] = to_f(r.q[i]);
+        s.d = to_f4(r.d);
+    }
+}
+
+// S <- S_t from S_{t-1}; returns r = (Diag(a) S_{t-1})^T k.
 template <int RPL>
-__device__ __forceinline__ void forward_step(float4 (&S)[RPL], const StepIn<RPL> &in) {
+__device__ __forceinline__ float4 forward_step(float4 (&S)[RPL], const StepIn<RPL> &in) {
     float4 rp = f4(0.f);
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
         S[i] = mul4(S[i], in.a[i]);
         rp = fma4s(S[i], in.k[i], rp);
     }
-    const float4 u = mul4(sub4(in.v, warp_sum4(rp)), in.b);
+    const float4 r = warp_sum4(rp);
+    const float4 u = mul4(sub4(in.v, r), in.b);
 #pragma unroll
     for (int i = 0; i < RPL; ++i) S[i] = fma4s(u, in.k[i], S[i]);
+    return r;
 }
 
+// A step's record in a CTA's scratch: the state slice entering it, then r of
+// each warp's 4 columns.
+template <int DK>
+constexpr int scratch_step4() { return BwdShape<DK>::STATE4 + kBwdWarps; }
+
 // Forward over steps [t0, t1) with the next step's inputs loaded one step ahead;
-// with `keep`, the state entering each step is written to keep[step - t0].
+// with `keep`, each step's record (entering state, r) is written to
+// keep[step - t0].
 template <typename T, int DK>
 __device__ __forceinline__ void forward_run(float4 (&S)[DK / 32], const BwdArgs &p, int64_t t0,
                                             int64_t t1, int h, int lane, int j0, float4 *keep,
                                             int idx) {
     constexpr int RPL = DK / 32;
-    constexpr int S4 = BwdShape<DK>::STATE4;
-    StepIn<RPL> cur, nxt;
+    constexpr int R4 = scratch_step4<DK>();
+    StepRaw<T, RPL> nxt;
     if (t0 < t1) load_step<T, DK, false>(nxt, p, t0, h, lane, j0);
 #pragma unroll 1
     for (int64_t t = t0; t < t1; ++t) {
-        cur = nxt;
+        StepIn<RPL> cur;
+        decode_step<T, RPL, false>(cur, nxt, p.scalar_gate);
         if (t + 1 < t1) load_step<T, DK, false>(nxt, p, t + 1, h, lane, j0);
-        if (keep) {
+        float4 *rec = keep ? keep + (size_t)(t - t0) * R4 : nullptr;
+        if (rec) {
 #pragma unroll
-            for (int i = 0; i < RPL; ++i) keep[(size_t)(t - t0) * S4 + idx + i * kBwdThreads] = S[i];
+            for (int i = 0; i < RPL; ++i) rec[idx + i * kBwdThreads] = S[i];
         }
-        forward_step<RPL>(S, cur);
+        const float4 r = forward_step<RPL>(S, cur);
+        if (rec && lane == 0) rec[BwdShape<DK>::STATE4 + (idx >> 5)] = r;
     }
 }
 
@@ -212,7 +256,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_kernel(const BwdA
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // a thread's float4 i of a state slice: key row lane + 32 i, its warp's columns
     const int idx = warp * 32 + lane;
-    float4 *scratch = p.scratch + (size_t)blockIdx.x * kBwdBlock * S4;
+    float4 *scratch = p.scratch + (size_t)blockIdx.x * kBwdBlock * scratch_step4<DK>();
     int buf = 0;
 
 #pragma unroll 1
@@ -273,33 +317,38 @@ __global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_kernel(const BwdA
             for (int i = 0; i < RPL; ++i) S[i] = ck[idx + i * kBwdThreads];
             forward_run<T, DK>(S, p, tb, te, h, lane, j0, scratch, idx);
 
-            // Backward over the block, the next step's inputs and entering
-            // state loaded one step ahead.
-            StepIn<RPL> cur, nxt;
-            float4 Sn[RPL];
+            // Lane 0 wrote each step's r; the warp's lanes read it below.
+            __syncwarp();
+            // Backward over the block, the next step's inputs and record
+            // loaded one step ahead.
+            constexpr int R4 = scratch_step4<DK>();
+            StepRaw<T, RPL> nxt;
+            float4 Sn[RPL], rn;
             load_step<T, DK, true>(nxt, p, te - 1, h, lane, j0);
+            {
+                const float4 *rec = scratch + (size_t)(te - 1 - tb) * R4;
 #pragma unroll
-            for (int i = 0; i < RPL; ++i) Sn[i] = scratch[(size_t)(te - 1 - tb) * S4 + idx + i * kBwdThreads];
+                for (int i = 0; i < RPL; ++i) Sn[i] = rec[idx + i * kBwdThreads];
+                rn = rec[S4 + warp];
+            }
 #pragma unroll 1
             for (int64_t t = te - 1; t >= tb; --t) {
-                cur = nxt;
+                StepIn<RPL> cur;
+                decode_step<T, RPL, true>(cur, nxt, p.scalar_gate);
                 float4 sp[RPL];
 #pragma unroll
                 for (int i = 0; i < RPL; ++i) sp[i] = Sn[i];
+                const float4 r = rn;
                 if (t - 1 >= tb) {
                     load_step<T, DK, true>(nxt, p, t - 1, h, lane, j0);
+                    const float4 *rec = scratch + (size_t)(t - 1 - tb) * R4;
 #pragma unroll
-                    for (int i = 0; i < RPL; ++i)
-                        Sn[i] = scratch[(size_t)(t - 1 - tb) * S4 + idx + i * kBwdThreads];
+                    for (int i = 0; i < RPL; ++i) Sn[i] = rec[idx + i * kBwdThreads];
+                    rn = rec[S4 + warp];
                 }
-                // the step again: Sp, r, u
-                float4 rp = f4(0.f);
+                // Sp = Diag(a) S_{t-1}; r and u as the forward had them
 #pragma unroll
-                for (int i = 0; i < RPL; ++i) {
-                    sp[i] = mul4(sp[i], cur.a[i]);
-                    rp = fma4s(sp[i], cur.k[i], rp);
-                }
-                const float4 r = warp_sum4(rp);
+                for (int i = 0; i < RPL; ++i) sp[i] = mul4(sp[i], cur.a[i]);
                 const float4 vr = sub4(cur.v, r);
                 const float4 uu = mul4(vr, cur.b);
                 // o_t = S_t^T q, S_t = Sp + k u^T
@@ -384,9 +433,10 @@ int bwd_grid(int num_seqs, int H, int d_v) {
 
 size_t backward_workspace(int num_seqs, int64_t total_tokens, int H, int dk, int dv) {
     const size_t state = (size_t)dk * kBwdSlice * sizeof(float);   // one slice
+    const size_t record = state + kBwdWarps * sizeof(float4);       // state and r per step
     const size_t nsl = (size_t)(dv / kBwdSlice);
     return kWorkspaceHeader + bwd_slots(num_seqs, total_tokens) * H * nsl * state +
-           (size_t)bwd_grid(num_seqs, H, dv) * kBwdBlock * state;
+           (size_t)bwd_grid(num_seqs, H, dv) * kBwdBlock * record;
 }
 
 cudaError_t launch_backward(const void *q, const void *k, const void *v, const void *g,
