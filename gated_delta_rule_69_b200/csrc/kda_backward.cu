@@ -158,12 +158,12 @@ __device__ __forceinline__ void decode_step(StepIn<RPL> &s, const StepRaw<T, RPL
 #pragma unroll
     for (int i = 0; i < RPL; ++i) s.k[i] = to_f(r.k[i]);
     if (scalar_gate) {
-        const float a = expf(to_f(r.g[0]));
+        const float a = __expf(to_f(r.g[0]));
 #pragma unroll
         for (int i = 0; i < RPL; ++i) s.a[i] = a;
     } else {
 #pragma unroll
-        for (int i = 0; i < RPL; ++i) s.a[i] = expf(to_f(r.g[i]));
+        for (int i = 0; i < RPL; ++i) s.a[i] = __expf(to_f(r.g[i]));
     }
     s.v = to_f4(r.v);
     s.b = to_f(r.b);
