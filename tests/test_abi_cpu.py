@@ -175,3 +175,14 @@ def test_backward_rejects_on_host(L):
         assert _backward(L, fn, dq=FAKE + 64) == 1          # dq overlaps q
         assert _backward(L, fn, dkk=FAKE * 64 + 64) == 1    # dk overlaps dq
         assert _backward(L, fn, ds0=FAKE * 128 + 4096) == 1  # d_init_state inside the workspace
+
+
+def test_binding_checks_backward_gate_shape():
+    import torch
+    from gated_delta_rule_69_b200 import kda
+    x = torch.zeros(4, 2, 32)
+    b = torch.zeros(4, 2)
+    with pytest.raises(ValueError):   # per-head gate given to the per-channel entry
+        kda.kda_backward(x, x, x, b, b, x)
+    with pytest.raises(ValueError):   # per-channel gate given to the per-head entry
+        kda.gdn_backward(x, x, x, x, b, x)
