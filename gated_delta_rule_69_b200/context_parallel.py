@@ -17,6 +17,8 @@ three times per rank (two before the exchange), the preparation once.
 """
 from __future__ import annotations
 
+import contextlib
+
 import torch
 
 from . import kda
@@ -58,14 +60,22 @@ def cp_prefill(q, k, v, log_alpha, beta, init_state=None, group=None, workspace=
     state, the same on every rank (or None).  Returns (o for the segment, the
     state after it); the last rank's is the sequence's final state.
     ``exchange_fn(m, s_tilde)`` replaces the collective (returns the stacked
-    pairs of all ranks), e.g. to run the ranks one after another on one GPU."""
+    pairs of all ranks), e.g. to run the ranks one after another on one GPU.
+    With ``stream``, every step, the collective included, is ordered on it
+    (it becomes torch's current stream for the call)."""
     if rank is None:
         import torch.distributed as dist
         rank = dist.get_rank(group)
     if workspace is None:
         workspace = workspace_for(q)
-    m, s_tilde = local_pair(q, k, v, log_alpha, beta, workspace=workspace, stream=stream)
-    ms, ss = exchange_fn(m, s_tilde) if exchange_fn is not None else exchange(m, s_tilde, group)
-    s0 = None if init_state is None else init_state.reshape(init_state.shape[-3:]).contiguous()
-    s_in = kda.kda_cp_combine(ms[:rank].contiguous(), ss[:rank].contiguous(), s0, stream=stream)
-    return kda.kda_cp_finish(v, s_in.unsqueeze(0), workspace, stream=stream)
+    ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+    with ctx:
+        m, s_tilde = local_pair(q, k, v, log_alpha, beta, workspace=workspace, stream=stream)
+        if exchange_fn is not None:
+            ms, ss = exchange_fn(m, s_tilde)
+        else:
+            ms, ss = exchange(m, s_tilde, group)
+        s0 = None if init_state is None else init_state.reshape(init_state.shape[-3:]).contiguous()
+        s_in = kda.kda_cp_combine(ms[:rank].contiguous(), ss[:rank].contiguous(), s0,
+                                  stream=stream)
+        return kda.kda_cp_finish(v, s_in.unsqueeze(0), workspace, stream=stream)
