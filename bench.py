@@ -5,15 +5,19 @@ decode tokens/s, each with its roofline, as ONE JSON line on rank 0.
     python bench.py --impl reference ...      # the fp64 CPU oracle, timed
 
 A step is one kda_prefill call over the prefill workload's batch (all chunks,
-all heads, final state written).  Inputs are resident in HBM when timing
-starts; L2 is flushed (a 256 MiB write) before every timed step, outside the
-timed interval.  The decode figures time chained kda_decode_step calls on the
+all heads, final state written).  The headline workload is the long
+single-sequence prefill (131072 tokens, 32 heads, d = 128), the largest
+single-GPU configuration; the 4096-token / 16-head prefill and the packed
+16-sequence varlen batch are timed the same way as the extra objects
+"prefill_T4096" and "varlen".  Inputs are resident in HBM when timing starts;
+L2 is flushed (a 256 MiB write) before every timed step, outside the timed
+interval.  The decode figures time chained kda_decode_step calls on the
 decode workload (state 512 MiB, larger than L2, so no flush is needed).  The
 "gdn_prefill" object times gdn_prefill (Gated DeltaNet: one gate value per
 token and head) and "layer_prefill" times kda_layer_prefill (raw activations,
-the layer's prologue and epilogue fused) on the prefill workload the same way;
-"backward" times kda_backward (the gradients, given seeded upstream gradients)
-on the same workload.
+the layer's prologue and epilogue fused) on the headline workload the same
+way; "backward" times kda_backward (the gradients, given seeded upstream
+gradients) on the 4096-token workload.
 Under torchrun every rank runs the same workload as an independent replica
 (the operator needs no exchange between GPUs); value = all ranks' tokens over
 the slowest rank's time.
@@ -33,8 +37,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "KDA prefill tokens/s and decode tokens/s at 1 B200; fraction of tensor/HBM roofline"
-PREFILL_DEFAULT = "prefill_T4096_H16_d128"
+PREFILL_DEFAULT = "prefill_T131072_H32_d128"
+EXTRA_PREFILL = (("prefill_T4096", "prefill_T4096_H16_d128"),
+                 ("varlen", "varlen_16seq_256to16384_H32_d128"))
+BACKWARD_DEFAULT = "prefill_T4096_H16_d128"
 DECODE_DEFAULT = "decode_B256_H32_d128"
+# the oracle's sample: whole heads of the first sequence, at most this many
+# of its first tokens (its cost is linear in (token, head) pairs)
+ORACLE_PREFIX = 32768
 DECODE_STEPS = 1000
 
 # Algorithmic work per (token, head) for prefill with chunk C and d_k = d_v = d:
@@ -391,16 +401,18 @@ def time_decode(w, steps, warmup, world):
 
 # --- the oracle on the host cores ------------------------------------------------------
 
-def oracle_prefill_sample(w, inp, budget_s=10.0, max_heads=None):
-    """Time the fp64 oracle on whole heads of the first sequence, adding heads
-    (as many per batch as there are oracle threads) until ``budget_s`` of CPU
-    work has run or every head is done.  Returns the oracle's tokens/s
-    extrapolated to the whole workload, and a description of the sample."""
+def oracle_prefill_sample(w, inp, budget_s=10.0, max_heads=None, total_tokens=None):
+    """Time the fp64 oracle on heads of the first sequence (its first
+    ORACLE_PREFIX tokens at most), adding heads (as many per batch as there
+    are oracle threads) until ``budget_s`` of CPU work has run or every head is
+    done.  Returns the oracle's tokens/s extrapolated to the whole workload
+    (``total_tokens`` of it, default the tokens in ``inp``), and a description
+    of the sample."""
     import numpy as np
     import oracle
     from gated_delta_rule_69_b200.inputs import as_float64
     cu = inp["cu_seqlens"].cpu().numpy()
-    L0 = int(cu[1] - cu[0])
+    L0 = min(int(cu[1] - cu[0]), ORACLE_PREFIX)
     threads = oracle.max_threads()
     H = w.H if max_heads is None else min(w.H, max_heads)
     done, t_total = 0, 0.0
@@ -413,12 +425,13 @@ def oracle_prefill_sample(w, inp, budget_s=10.0, max_heads=None):
         oracle.kda_recurrence(*args, init_state=s0, cu_seqlens=np.array([0, L0]))
         t_total += time.perf_counter() - t0
         done += len(hs)
-    total_tokens = sum(inp["lengths"])
+    if total_tokens is None:
+        total_tokens = sum(inp["lengths"])
     # the oracle's cost is linear in (tokens x heads): scale the sampled rate
     units_done = done * L0
     units_all = total_tokens * w.H
     value = total_tokens / (t_total * units_all / units_done)
-    sample = (f"{done} of {w.H} heads x {L0} tokens of sequence 0 "
+    sample = (f"{done} of {w.H} heads x the first {L0} tokens of sequence 0 "
               f"({units_done} (token, head) pairs of {units_all}); tokens/s scaled by the pair count")
     return value, threads, sample, t_total
 
@@ -429,23 +442,28 @@ def run_reference(args, w):
         return 0
     import torch
     from gated_delta_rule_69_b200 import inputs as kin
-    inp = kin.generate(w, device="cpu")
+    # the sample's inputs only: the first sequence's first ORACLE_PREFIX
+    # tokens, drawn with the workload's seed and distributions (drawing the
+    # whole 131072-token batch on the host would take longer than timing it)
+    lengths = kin.seq_lengths(w)
+    inp = kin.generate(w, device="cpu", lengths=[min(lengths[0], ORACLE_PREFIX)])
     import oracle
     threads = oracle.max_threads()
     vals, secs = [], []
     for i in range(args.warmup + args.steps):
-        v, thr, sample, t = oracle_prefill_sample(w, inp, budget_s=0.0, max_heads=threads)
+        v, thr, sample, t = oracle_prefill_sample(w, inp, budget_s=0.0, max_heads=threads,
+                                                  total_tokens=sum(lengths))
         if i >= args.warmup:
             vals.append(v)
             secs.append(t)
     value = statistics.median(vals)
-    work = prefill_work(w, inp["lengths"])
+    work = prefill_work(w, lengths)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * work["tokens"] / value, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w, inp["lengths"], args.gpus),
+        "config": config_of(w, lengths, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -474,6 +492,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=PREFILL_DEFAULT)
     ap.add_argument("--decode-workload", default=DECODE_DEFAULT)
+    ap.add_argument("--backward-workload", default=BACKWARD_DEFAULT)
     ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -498,11 +517,17 @@ def main():
     sampler = ClockSampler(local)
     sampler.start()
     pf = time_prefill(w, args.steps, args.warmup, world)
+    extra = []
+    for key, name in EXTRA_PREFILL:
+        if name != w.name:
+            ew = kin.WORKLOADS[name]
+            extra.append((key, ew, time_prefill(ew, args.steps, args.warmup, world)))
     dw = kin.WORKLOADS[args.decode_workload]
     dec = time_decode(dw, args.decode_steps, args.warmup, world)
     gdn = time_prefill(w, args.steps, args.warmup, world, scalar_gate=True)
     lay = time_prefill(w, args.steps, args.warmup, world, layer=True)
-    bwd = time_backward(w, max(3, args.steps // 4), args.warmup, world)
+    bw = kin.WORKLOADS[args.backward_workload]
+    bwd = time_backward(bw, max(3, args.steps // 4), args.warmup, world)
     clocks = sampler.stop()
 
     lengths = pf["inputs"]["lengths"]
@@ -520,7 +545,7 @@ def main():
     lwork = prefill_work(w, lengths, layer=True)
     lms = max_over_ranks(lay["ms_total"] / args.steps, world)
     lgbs = lwork["bytes"] / (lms * 1e-3) / 1e9
-    bwork = backward_work(w, bwd["lengths"])
+    bwork = backward_work(bw, bwd["lengths"])
     bms = max_over_ranks(bwd["ms_total"] / len(bwd["ms"]), world)
     btfs = bwork["flop"] / (bms * 1e-3) / 1e12
     src = "of " + peaks["source"]
@@ -557,7 +582,7 @@ def main():
                                        "traffic": None, "peak_source": src,
                                        "kernel": "kda_layer_prefill",
                                        "algorithmic_bytes_per_launch": lwork["bytes"]}},
-        "backward": {"workload": w.name + ", backward pass (kda_backward), seeded upstream gradients",
+        "backward": {"workload": bw.name + ", backward pass (kda_backward), seeded upstream gradients",
                      "value": world * bwork["tokens"] / (bms * 1e-3), "unit": "tokens/s",
                      "ms_per_step": bms, "steps": len(bwd["ms"]),
                      "roofline": {"bound": "alu", "achieved": btfs, "peak": FP32_SIMT_TFLOPS,
@@ -569,9 +594,23 @@ def main():
                                   "algorithmic_bytes_per_launch": bwork["bytes"],
                                   "hbm_frac": bwork["bytes"] / (bms * 1e-3) / 1e9 / peaks["hbm"]}},
         "gpu_launches": pf["launches"] + dec["launches"] + gdn["launches"] + lay["launches"]
-                        + bwd["launches"],
+                        + bwd["launches"] + sum(x[2]["launches"] for x in extra),
         "clocks": clocks,
     }
+    for key, ew, r in extra:
+        ework = prefill_work(ew, r["inputs"]["lengths"])
+        ems = max_over_ranks(r["ms_total"] / args.steps, world)
+        egbs = ework["bytes"] / (ems * 1e-3) / 1e9
+        etfs = ework["flop"] / (ems * 1e-3) / 1e12
+        line[key] = {"workload": ew.name, "config": config_of(ew, r["inputs"]["lengths"], world),
+                     "value": world * ework["tokens"] / (ems * 1e-3), "unit": "tokens/s",
+                     "ms_per_step": ems, "steps": args.steps,
+                     "roofline": {"bound": "hbm", "achieved": egbs, "peak": peaks["hbm"],
+                                  "unit": "GB/s", "frac": egbs / peaks["hbm"], "traffic": None,
+                                  "peak_source": src, "kernel": "kda_prefill",
+                                  "algorithmic_bytes_per_launch": ework["bytes"],
+                                  "tensor_tflops": etfs, "tensor_frac": etfs / peaks["bf16"],
+                                  "algorithmic_flop_per_launch": ework["flop"]}}
     if not args.no_e2e:
         e2e = time_prefill_e2e(w, max(6, args.steps), args.warmup)
         e_ms = max_over_ranks(e2e["ms_per_step"], world)

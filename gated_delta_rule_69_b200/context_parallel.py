@@ -36,7 +36,9 @@ def local_pair(q, k, v, log_alpha, beta, workspace=None, stream=None):
     if v.shape[-1] != q.shape[-1]:
         raise ValueError("context parallelism needs d_v = d_k (M is d_k x d_k)")
     if workspace is None:
-        workspace = workspace_for(q)
+        ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+        with ctx:   # the workspace belongs to the stream its kernels run on
+            workspace = workspace_for(q)
     return kda.kda_cp_local(q, k, v, log_alpha, beta, workspace, stream=stream)
 
 
@@ -66,10 +68,13 @@ def cp_prefill(q, k, v, log_alpha, beta, init_state=None, group=None, workspace=
     if rank is None:
         import torch.distributed as dist
         rank = dist.get_rank(group)
-    if workspace is None:
-        workspace = workspace_for(q)
+    # every allocation below, the workspace included, belongs to the stream
+    # the work runs on, so torch's allocator reuses its memory only after
+    # that work in the stream's order
     ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
     with ctx:
+        if workspace is None:
+            workspace = workspace_for(q)
         m, s_tilde = local_pair(q, k, v, log_alpha, beta, workspace=workspace, stream=stream)
         if exchange_fn is not None:
             ms, ss = exchange_fn(m, s_tilde)

@@ -413,8 +413,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_kernel(const BwdA
 template <typename T, int DK>
 cudaError_t launch_dk(const BwdArgs &p, int grid, cudaStream_t stream) {
     const size_t smem = BwdShape<DK>::SMEM;
-    cudaError_t e = cudaFuncSetAttribute(kda_backward_kernel<T, DK>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem((const void *)kda_backward_kernel<T, DK>, (int)smem);
     if (e != cudaSuccess) return e;
     kda_backward_kernel<T, DK><<<grid, kBwdThreads, smem, stream>>>(p);
     return cudaGetLastError();

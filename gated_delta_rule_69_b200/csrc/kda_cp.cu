@@ -75,14 +75,9 @@ kda_cp_combine_kernel(const float *__restrict__ M, const float *__restrict__ St,
 cudaError_t launch_cp_combine(const float *M, const float *S_tilde, const float *S0, float *S_out,
                               int n_prev, int H, int dk, int dv, cudaStream_t stream) {
     const size_t smem = (size_t)(dk * dk + dk * kCpCols) * sizeof(float);
-    static bool attr_set = false;
-    if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(kda_cp_combine_kernel,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)((128 * 128 + 128 * kCpCols) * sizeof(float)));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    const cudaError_t e = set_max_dynamic_smem((const void *)kda_cp_combine_kernel,
+                                               (int)((128 * 128 + 128 * kCpCols) * sizeof(float)));
+    if (e != cudaSuccess) return e;
     kda_cp_combine_kernel<<<dim3(H, dv / kCpCols), kCpThreads, smem, stream>>>(M, S_tilde, S0, S_out,
                                                                             n_prev, H, dk, dv);
     return cudaGetLastError();

@@ -67,6 +67,12 @@ enum : uint32_t {
 // per-kernel scratch areas.
 constexpr size_t kWorkspaceHeader = 256;
 
+// Launch set-up cached per (device, kernel) under a lock (kda_launch_setup.cu):
+// the dynamic shared-memory limit of `func` on the current device, and the
+// current device's SM count (148 if the query fails).
+cudaError_t set_max_dynamic_smem(const void *func, int bytes);
+int device_sm_count();
+
 // Launchers (defined in the .cu files).  All return cudaGetLastError().
 // `scalar_gate`: log_alpha holds one value per (token, head) ([T, H], the
 // Gated DeltaNet gate) instead of one per key channel ([T, H, d_k]).

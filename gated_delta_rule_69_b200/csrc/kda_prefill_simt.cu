@@ -205,8 +205,7 @@ cudaError_t launch_typed(const void *q, const void *k, const void *v,
                          void *o, float *fin, uint32_t *err, bool sg, cudaStream_t st) {
     constexpr size_t smem = SimtSmem<DK, DV>::bytes;
     auto kern = kda_prefill_simt_kernel<T, DK, DV>;
-    cudaError_t e = cudaFuncSetAttribute(
-        kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem((const void *)kern, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned blocks = (unsigned)((size_t)n * (size_t)H);
     kern<<<blocks, kThreads, smem, st>>>(

@@ -1327,17 +1327,17 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's encoder, looked up once per process (a function-local static
+// is initialised once even when several threads arrive together).
 EncodeTiledFn encode_fn_split() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
                 cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
+            return reinterpret_cast<EncodeTiledFn>(ptr);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -1384,13 +1384,9 @@ cudaError_t launch_chain(const void *v, int64_t total_tokens, int H, const split
     if (!make_map_split(&mv, v, total_tokens, H, DV, DVT == 32 ? 32 : 64,
                         DVT == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(kda_chain_kernel<DVT>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)Cfg::ALLOC);
+    {
+        const cudaError_t e = set_max_dynamic_smem((const void *)kda_chain_kernel<DVT>, (int)Cfg::ALLOC);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(units * Cfg::NTILE);
@@ -1415,16 +1411,12 @@ cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const spl
     CUtensorMap mv;
     if (!make_map_split(&mv, v, total_tokens, H, DV, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kda_chain_t_kernel<kChainPlain>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+    {
+        cudaError_t e = set_max_dynamic_smem((const void *)kda_chain_t_kernel<kChainPlain>,
                                              (int)ChainT::ALLOC);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kda_chain_t_kernel<kChainTransition>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ChainT::ALLOC);
+        e = set_max_dynamic_smem((const void *)kda_chain_t_kernel<kChainTransition>, (int)ChainT::ALLOC);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(units);
@@ -1541,13 +1533,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     // programmatic dependent of it, so that it starts at once and consumes
     // records as they are published; otherwise the two kernels run one after
     // the other and the records need no flags.
-    static int sm_count = 0;
-    if (!sm_count) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            sm_count = 148;
-    }
+    const int sm_count = device_sm_count();
     const unsigned units = (unsigned)((size_t)num_seqs * H);
     // a segment's transition is d_k x d_k: whole-d_v chain CTAs only
     const ChainPlan plan = choose_chain(units, (uint64_t)(total_tokens / C + num_seqs) * H, total_tokens,
@@ -1561,16 +1547,10 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                                           work_next);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    static bool attr_set = false;
-    if (!attr_set) {
-        e = cudaFuncSetAttribute(kda_prep_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)PrepSmem::ALLOC);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(kda_prep_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)PrepSmem::ALLOC);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    e = set_max_dynamic_smem((const void *)kda_prep_kernel<false>, (int)PrepSmem::ALLOC);
+    if (e != cudaSuccess) return e;
+    e = set_max_dynamic_smem((const void *)kda_prep_kernel<true>, (int)PrepSmem::ALLOC);
+    if (e != cudaSuccess) return e;
     Params prm;
     prm.k = static_cast<const __nv_bfloat16 *>(k);
     prm.q = static_cast<const __nv_bfloat16 *>(q);

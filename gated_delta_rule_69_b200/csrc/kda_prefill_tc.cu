@@ -896,17 +896,17 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's encoder, looked up once per process (a function-local static
+// is initialised once even when several threads arrive together).
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
                 cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
+            return reinterpret_cast<EncodeTiledFn>(ptr);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -950,13 +950,8 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     kda_plan_kernel<<<1, kPlanThreads, 0, stream>>>(cu, num_seqs, total_tokens, perm, err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    static bool attr_set = false;
-    if (!attr_set) {
-        e = cudaFuncSetAttribute(kda_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)Smem::ALLOC);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    e = set_max_dynamic_smem((const void *)kda_prefill_tc_kernel, (int)Smem::ALLOC);
+    if (e != cudaSuccess) return e;
     Params prm;
     prm.k = static_cast<const __nv_bfloat16 *>(k);
     prm.q = static_cast<const __nv_bfloat16 *>(q);

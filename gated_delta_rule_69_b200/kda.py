@@ -8,6 +8,7 @@ every call raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -108,6 +109,14 @@ def _stream(stream, device):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _on(stream):
+    """Allocations made for a call that runs on ``stream`` belong to that
+    stream: torch's caching allocator then hands their memory to later work
+    only in that stream's order, so a buffer the call frees on return cannot
+    be reused while the call's kernels still read it."""
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+
+
 def _check_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -153,13 +162,14 @@ def _prefill(fn, q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, o, 
             raise TypeError("cu_seqlens must be int32")
     else:
         n = 1 if num_seqs is None else int(num_seqs)
-    if o is None:
-        o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
-    if final_state is None and output_final_state:
-        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
     need = kda_prefill_workspace_size(n, T, H, dk, dv)
-    if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    with _on(stream):
+        if o is None:
+            o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+        if final_state is None and output_final_state:
+            final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+        if workspace is None:
+            workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     _check_cuda(q, k, v, log_alpha, beta, init_state, cu_seqlens, o, final_state, workspace)
     st = getattr(lib(), fn)(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
@@ -190,7 +200,8 @@ def _decode(fn, q, k, v, log_alpha, beta, state, o, stream):
     B, H, dk = q.shape
     dv = v.shape[-1]
     if o is None:
-        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+        with _on(stream):
+            o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
     _check_cuda(q, k, v, log_alpha, beta, state, o)
     st = getattr(lib(), fn)(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state),
@@ -219,10 +230,11 @@ def kda_prefill_noalloc(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=No
             raise TypeError("cu_seqlens must be int32")
     else:
         n = 1 if num_seqs is None else int(num_seqs)
-    if o is None:
-        o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
-    if final_state is None and output_final_state:
-        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+    with _on(stream):
+        if o is None:
+            o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+        if final_state is None and output_final_state:
+            final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
     _check_cuda(q, k, v, log_alpha, beta, init_state, cu_seqlens, o, final_state)
     st = lib().kda_prefill_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
@@ -253,13 +265,14 @@ def kda_layer_prefill(q, k, v, gate_z, A_log, beta_logit, out_gate=None, norm_we
             raise TypeError("cu_seqlens must be int32")
     else:
         n = 1 if num_seqs is None else int(num_seqs)
-    if o is None:
-        o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
-    if final_state is None and output_final_state:
-        final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
     need = kda_prefill_workspace_size(n, T, H, dk, dv)
-    if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    with _on(stream):
+        if o is None:
+            o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+        if final_state is None and output_final_state:
+            final_state = torch.empty((n, H, dk, dv), dtype=torch.float32, device=q.device)
+        if workspace is None:
+            workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     _check_cuda(q, k, v, gate_z, A_log, beta_logit, out_gate, norm_weight, init_state,
                 cu_seqlens, o, final_state, workspace)
     st = lib().kda_layer_prefill(
@@ -283,7 +296,8 @@ def kda_layer_decode_step(q, k, v, gate_z, A_log, beta_logit, state, out_gate=No
     if A_log.dtype != torch.float32 or (norm_weight is not None and norm_weight.dtype != torch.float32):
         raise TypeError("A_log and norm_weight must be float32")
     if o is None:
-        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+        with _on(stream):
+            o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
     _check_cuda(q, k, v, gate_z, A_log, beta_logit, out_gate, norm_weight, state, o)
     st = lib().kda_layer_decode_step(
         _ptr(q), _ptr(k), _ptr(v), _ptr(gate_z), _ptr(A_log), _ptr(beta_logit), _ptr(out_gate),
@@ -301,7 +315,8 @@ def kda_cp_combine(M, S_tilde, S0=None, S_in=None, stream=None):
     n, H, dk, _ = M.shape
     dv = S_tilde.shape[-1]
     if S_in is None:
-        S_in = torch.empty((H, dk, dv), dtype=torch.float32, device=M.device)
+        with _on(stream):
+            S_in = torch.empty((H, dk, dv), dtype=torch.float32, device=M.device)
     _check_cuda(M, S_tilde, S0, S_in)
     st = lib().kda_cp_combine(_ptr(M), _ptr(S_tilde), _ptr(S0), _ptr(S_in), n, H, dk, dv,
                               _stream(stream, M.device))
@@ -315,10 +330,11 @@ def kda_cp_local(q, k, v, log_alpha, beta, workspace, o_scratch=None, stream=Non
     stay in ``workspace`` for kda_cp_finish.  bf16, d = 128, one sequence."""
     T, H, dk = q.shape
     dv = v.shape[-1]
-    M = torch.empty((1, H, dk, dk), dtype=torch.float32, device=q.device)
-    S = torch.empty((1, H, dk, dv), dtype=torch.float32, device=q.device)
-    if o_scratch is None:
-        o_scratch = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    with _on(stream):
+        M = torch.empty((1, H, dk, dk), dtype=torch.float32, device=q.device)
+        S = torch.empty((1, H, dk, dv), dtype=torch.float32, device=q.device)
+        if o_scratch is None:
+            o_scratch = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
     _check_cuda(q, k, v, log_alpha, beta, workspace, o_scratch)
     st = lib().kda_cp_local(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), T, H, dk, dv,
                             _dtype_code(q), _ptr(M), _ptr(S), _ptr(o_scratch), _ptr(workspace),
@@ -334,10 +350,11 @@ def kda_cp_finish(v, S_in, workspace, o=None, final_state=None, output_final_sta
     kda_cp_local call left in ``workspace``."""
     T, H, dv = v.shape
     dk = S_in.shape[-2] if S_in is not None else dv
-    if o is None:
-        o = torch.empty((T, H, dv), dtype=v.dtype, device=v.device)
-    if final_state is None and output_final_state:
-        final_state = torch.empty((1, H, dk, dv), dtype=torch.float32, device=v.device)
+    with _on(stream):
+        if o is None:
+            o = torch.empty((T, H, dv), dtype=v.dtype, device=v.device)
+        if final_state is None and output_final_state:
+            final_state = torch.empty((1, H, dk, dv), dtype=torch.float32, device=v.device)
     _check_cuda(v, S_in, workspace, o, final_state)
     st = lib().kda_cp_finish(_ptr(v), _ptr(S_in), T, H, dk, dv, _dtype_code(v), _ptr(o),
                              _ptr(final_state), _ptr(workspace), workspace.numel(),
@@ -384,15 +401,16 @@ def _backward(fn, q, k, v, log_alpha, beta, d_o, init_state, d_final_state, cu_s
     else:
         n = 1 if num_seqs is None else int(num_seqs)
     f32 = dict(dtype=torch.float32, device=q.device)
-    dq = torch.empty((T, H, dk), **f32)
-    dkk = torch.empty((T, H, dk), **f32)
-    dvv = torch.empty((T, H, dv), **f32)
-    dg = torch.empty(tuple(log_alpha.shape), **f32)
-    db = torch.empty((T, H), **f32)
-    ds0 = torch.empty((n, H, dk, dv), **f32) if want_d_init_state else None
-    if workspace is None:
-        need = kda_backward_workspace_size(n, T, H, dk, dv)
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    with _on(stream):
+        dq = torch.empty((T, H, dk), **f32)
+        dkk = torch.empty((T, H, dk), **f32)
+        dvv = torch.empty((T, H, dv), **f32)
+        dg = torch.empty(tuple(log_alpha.shape), **f32)
+        db = torch.empty((T, H), **f32)
+        ds0 = torch.empty((n, H, dk, dv), **f32) if want_d_init_state else None
+        if workspace is None:
+            need = kda_backward_workspace_size(n, T, H, dk, dv)
+            workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     _check_cuda(q, k, v, log_alpha, beta, d_o, init_state, d_final_state, cu_seqlens, workspace)
     st = getattr(lib(), fn)(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),

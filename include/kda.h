@@ -17,8 +17,10 @@
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *     allocates no device memory and keeps no state between calls except a
- *     cached per-device property query.
+ *     allocates no device memory and keeps no state between calls except
+ *     launch settings cached per device under a lock (each kernel's shared-
+ *     memory limit, the SM count), so several host threads and several GPUs
+ *     may share one process.
  *   - Tensors are dense, row-major, token-major:
  *       q, k, log_alpha : [T_total, H, d_k]
  *       v, o            : [T_total, H, d_v]

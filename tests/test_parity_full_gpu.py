@@ -39,7 +39,7 @@ def _check(inp, o, fs, heads, seqs):
     got_s = fs.index_select(0, torch.as_tensor(seqs, device="cuda")).index_select(1, hh)
     e_o = o_err(got_o, ref_o, sub_cu, len(hs))
     e_s = state_err(got_s.double().cpu().numpy(), ref_s)
-    assert np.isfinite(o.float().cpu().numpy()).all(), "unwritten or non-finite outputs"
+    assert bool(torch.isfinite(o).all()), "unwritten or non-finite outputs"
     assert e_o <= TOL["bf16"], e_o
     assert e_s <= TOL["bf16"], e_s
     return e_o, e_s
@@ -61,15 +61,18 @@ def test_prefill_T131072_H32_sampled_heads():
     _check(inp, o, fs, heads=heads, seqs=[0])
 
 
-def test_varlen_16seq_sampled_units():
-    """Packed varlen batch: 4 sampled sequences x 2 sampled heads, plus the
-    shortest and longest sequence."""
+def test_varlen_16seq_all_units():
+    """Packed varlen batch: every one of the 16 sequences and all 32 heads
+    (512 units, about 4.3 M (token, head) pairs), each checked on every
+    output and final-state element, so that every sequence's state reset and
+    ragged last chunk is compared.  The oracle runs on 4 heads at a time to
+    bound host memory (its fp64 copies of 4 heads are ~3 GB)."""
     w = kin.WORKLOADS["varlen_16seq_256to16384_H32_d128"]
     inp = kin.generate(w, device="cuda")
     o, fs = _run(inp)
-    lens = np.array(inp["lengths"])
-    rng = np.random.default_rng(w.seed)
-    seqs = sorted(set(rng.choice(16, 4, replace=False).tolist()
-                      + [int(lens.argmin()), int(lens.argmax())]))
-    heads = sorted(rng.choice(32, 2, replace=False).tolist())
-    _check(inp, o, fs, heads=heads, seqs=seqs)
+    seqs = list(range(len(inp["lengths"])))
+    worst_o = worst_s = 0.0
+    for h0 in range(0, 32, 4):
+        e_o, e_s = _check(inp, o, fs, heads=list(range(h0, h0 + 4)), seqs=seqs)
+        worst_o, worst_s = max(worst_o, e_o), max(worst_s, e_s)
+    print(f"varlen all units: worst o error {worst_o:.3e}, worst state error {worst_s:.3e}")
