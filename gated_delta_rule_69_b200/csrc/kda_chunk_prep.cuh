@@ -5,7 +5,6 @@
 //     [A; P] = [Ktil; Qtil] Khat^T  (tensor cores)
 //     A = diag(beta) strict_tril(.),  P = tril(.)
 //     T = (I + A)^-1 (fp32, recursive doubling),  T_beta = T diag(beta)
-//     W = T_beta Ktil (tensor cores)
 // (news digest page on Kimi Linear, section "Algorithme parallele par
 // chunks": WY/UT packing of the chunk's rank-1 updates and the triangular
 // inverse by forward substitution).  The routines take explicit buffer
@@ -44,7 +43,7 @@ __device__ __forceinline__ float exp_f(float x) { return exp2_f(x * kLog2e); }
 // Shared-memory buffers of one chunk's preparation.
 struct Bufs {
     uint8_t *stk;        // [Ktil rows 0-63 | Qtil rows 64-127], 2 K-atoms of 16 KB (128-byte swizzle);
-                         // raw k / q on entry, -W over Ktil on exit
+                         // raw k / q on entry
     uint8_t *khat;       // Khat [64][128], 2 K-atoms of 8 KB
     uint8_t *kbar;       // Kbar [64][128], 2 K-atoms of 8 KB
     const uint8_t *graw; // raw log_alpha [64][128] bf16, 256-byte rows
@@ -538,30 +537,6 @@ __device__ void solve(const Bufs &b, int pt) {
         pk.z = pack_bf16x2(u1.x * bb[4], u1.y * bb[5]);
         pk.w = pack_bf16x2(u1.z * bb[6], u1.w * bb[7]);
         *reinterpret_cast<uint4 *>(b.tb + sw128_off(t, i0 + 8 * hh)) = pk;
-    }
-}
-
-// ---- -W from TMEM over Ktil in b.stk (rows 0-63).  W is rows 0-63 of the
-// M = 128 product [T_beta; P] Ktil (row r in lane r), so the warps of TMEM
-// quadrants 0 and 1 read it, each half `half` of the 128 columns.
-__device__ __forceinline__ void read_w(const Bufs &b, uint32_t tmem_w, int quad, int half, int lane) {
-    if (quad >= 2) return;
-    uint8_t *wdst = b.stk + half * 16384;
-    const int t = 32 * quad + lane;
-#pragma unroll
-    for (int part = 0; part < 2; ++part) {
-        float v[32];
-        tmem_ld32(tmem_addr(tmem_w, 32 * quad, 64 * half + 32 * part), v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-            uint4 pk;
-            pk.x = pack_bf16x2(-v[j + 0], -v[j + 1]);
-            pk.y = pack_bf16x2(-v[j + 2], -v[j + 3]);
-            pk.z = pack_bf16x2(-v[j + 4], -v[j + 5]);
-            pk.w = pack_bf16x2(-v[j + 6], -v[j + 7]);
-            *reinterpret_cast<uint4 *>(wdst + sw128_off(t, 32 * part + j)) = pk;
-        }
     }
 }
 

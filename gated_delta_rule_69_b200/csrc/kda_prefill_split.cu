@@ -87,8 +87,8 @@ static_assert(PrepSmem::KHAT + 64 * prep::kAStride * 4 <= PrepSmem::GRAW &&
                   PrepSmem::GRAW + 64 * prep::kTStride * 4 <= PrepSmem::XF &&
                   PrepSmem::XF + 4608 <= PrepSmem::BETA,
               "solve scratch");
-// per pipeline (256 columns): [A;P] at 0 and W at 64; then MP at 0, YT at 128,
-// ZB at 192; then -P W at 0 (all M = 128 products)
+// per pipeline (256 columns): [A;P] at 0; then YT at 128, ZB at 192; then
+// YT Ktil at 0 and ZB Ktil at 128 (all M = 128 products)
 constexpr uint32_t kPrepTmemCols = 512;
 constexpr uint32_t kRawBytes = 4 * 8192 + 16384;   // k, q (2 boxes each), log_alpha
 
@@ -257,8 +257,8 @@ __device__ __forceinline__ void store8(uint8_t *tile, uint32_t row, uint32_t col
     *reinterpret_cast<uint4 *>(tile + sw128_off(row, col)) = pk;
 }
 
-// MP [128 c_out][128 c_in]: K-atom `half` (at atom0 or atom1) holds c_in
-// 64 half .. + 63.
+// MP = -(YT Ktil) [128 c_out][128 c_in] from the product YT Ktil in TMEM:
+// K-atom `half` (at atom0 or atom1) holds c_in 64 half .. + 63.
 __device__ __forceinline__ void write_mp(uint8_t *atom0, uint8_t *atom1, uint32_t tmem, int quad,
                                          int half, int lane) {
     uint8_t *atom = half ? atom1 : atom0;
@@ -268,6 +268,8 @@ __device__ __forceinline__ void write_mp(uint8_t *atom0, uint8_t *atom1, uint32_
         float v[32];
         tmem_ld32(tmem_addr(tmem, 32 * quad, 64 * half + 32 * part), v);
         tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = -v[j];
 #pragma unroll
         for (int j = 0; j < 32; j += 8) store8(atom, row, 32 * part + j, v + j);
     }
@@ -296,9 +298,9 @@ __device__ __forceinline__ void write_zb(uint8_t *zb, uint32_t tmem, int quad, i
     for (int j = 0; j < 32; j += 8) store8(zb, t, 32 * half + j, v + j);
 }
 
-// QP = Qtil + P (-W), in place over Qtil: rows 64-127 of the two 16 KB
-// K-atoms of `stk`, K-atom `half` holding channels 64 half .. + 63.  P (-W)
-// is rows 0-63 of an M = 128 product whose A operand starts at P, read by the
+// QP = Qtil - ZB Ktil, in place over Qtil: rows 64-127 of the two 16 KB
+// K-atoms of `stk`, K-atom `half` holding channels 64 half .. + 63.  ZB Ktil
+// is rows 0-63 of an M = 128 product whose A operand starts at ZB, read by the
 // warps of TMEM quadrants 0 and 1.
 __device__ __forceinline__ void write_qp(uint8_t *stk, uint32_t tmem, int quad, int half, int lane) {
     if (quad >= 2) return;
@@ -319,8 +321,8 @@ __device__ __forceinline__ void write_qp(uint8_t *stk, uint32_t tmem, int quad, 
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&w[e]);
-                    f[2 * e] = __low2float(h2) + v[j + 2 * e];
-                    f[2 * e + 1] = __high2float(h2) + v[j + 2 * e + 1];
+                    f[2 * e] = __low2float(h2) - v[j + 2 * e];
+                    f[2 * e + 1] = __high2float(h2) - v[j + 2 * e + 1];
                 }
                 store8(atom, 64 + t, 32 * part + j, f);
             }
@@ -338,8 +340,8 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
     const int pt = tid - P * kPipeThreads;
     const bool leader = pt == 0;
     const int quad = warp & 3, half = wp >> 2;
-    uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);   // raw, [A;P], W, MP/YT/ZB, PW,
-                                                                      // secondary-chunking blocks
+    uint64_t *B = reinterpret_cast<uint64_t *>(sm + PrepSmem::BARS);   // raw, [A;P], YT/ZB, MP/QP,
+                                                                      // (unused), secondary-chunking blocks
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + PrepSmem::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     float *beta = reinterpret_cast<float *>(sm + PrepSmem::BETA);
@@ -467,63 +469,51 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         named_barrier(BAR, prep::kGroupThreads);
         const uint32_t sK = smem_addr(sm + PrepSmem::STK), sKb = smem_addr(sm + PrepSmem::KBAR);
         const uint32_t sT = smem_addr(sm + PrepSmem::TB), sP = smem_addr(sm + PrepSmem::PB);
+        // W = T_beta Ktil is never formed: with YT = Kbar^T T_beta and
+        // ZB = P T_beta, MP = -Kbar^T W = -YT Ktil and QP = Qtil - P W =
+        // Qtil - ZB Ktil, so the record takes two groups of products.
         if (wp == 0) {
             tc_fence_after();
-            const uint32_t idW = idesc_bf16(128, DK, false, true);
+            const uint32_t idY = idesc_bf16(128, C, true, true);
+            const uint32_t idZ = idesc_bf16(128, C, false, true);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)   // [T_beta; P] Ktil: rows 0-63 are W = T_beta Ktil
-                mma_bf16_warp(tmem + 64, smem_desc(sT + ks * 32, 16, 1024, kLayoutSW128),
-                              smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idW, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks) {   // K = 64 tokens
+                // YT = Kbar^T T_beta
+                mma_bf16_warp(tmem + 128, smem_desc(sKb + ks * 2048, 8192, 1024, kLayoutSW128),
+                              smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idY, ks > 0 ? 1u : 0u);
+                // ZB = P T_beta: rows 0-63 of an M = 128 product whose A starts at P
+                mma_bf16_warp(tmem + 192, smem_desc(sP + ks * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idZ, ks > 0 ? 1u : 0u);
+            }
             mma_commit_warp(&B[2]);
         }
         mbar_wait(&B[2], it & 1, abort_flag);
         tc_fence_after();
-        prep::read_w(b, tmem + 64, quad, half, lane);   // -W over Ktil
+        // Kbar, T_beta are no longer read: YT and ZB go over them
+        write_yt(sm + PrepSmem::KBAR, tmem + 128, quad, half, lane);
+        write_zb(sm + PrepSmem::TB, tmem + 192, quad, half, lane);
         fence_async_smem();
         tc_fence_before();
         named_barrier(BAR, prep::kGroupThreads);
         if (wp == 0) {
             tc_fence_after();
-            const uint32_t idM = idesc_bf16(128, DK, true, true);
-            const uint32_t idY = idesc_bf16(128, C, true, true);
-            const uint32_t idZ = idesc_bf16(128, C, false, true);
+            const uint32_t idK = idesc_bf16(128, DK, false, true);   // B = Ktil [t][c] (MN-major)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {   // K = 64 tokens
-                const uint64_t aKb = smem_desc(sKb + ks * 2048, 8192, 1024, kLayoutSW128);   // Kbar^T
-                // MP = Kbar^T (-W)
-                mma_bf16_warp(tmem, aKb, smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idM,
+                const uint64_t bK = smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128);
+                // YT Ktil (= -MP)
+                mma_bf16_warp(tmem, smem_desc(sKb + ks * 32, 16, 1024, kLayoutSW128), bK, idK,
                               ks > 0 ? 1u : 0u);
-                // YT = Kbar^T T_beta
-                mma_bf16_warp(tmem + 128, aKb, smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idY,
+                // ZB Ktil (= Qtil - QP): rows 0-63 of an M = 128 product whose A starts at ZB
+                mma_bf16_warp(tmem + 128, smem_desc(sT + ks * 32, 16, 1024, kLayoutSW128), bK, idK,
                               ks > 0 ? 1u : 0u);
-                // ZB = P T_beta: rows 0-63 of an M = 128 product whose A starts at P
-                mma_bf16_warp(tmem + 192, smem_desc(sP + ks * 32, 16, 1024, kLayoutSW128),
-                              smem_desc(sT + ks * 2048, 8192, 1024, kLayoutSW128), idZ, ks > 0 ? 1u : 0u);
             }
             mma_commit_warp(&B[3]);
         }
         mbar_wait(&B[3], it & 1, abort_flag);
         tc_fence_after();
         write_mp(sm + PrepSmem::KHAT, sm + PrepSmem::GRAW, tmem, quad, half, lane);
-        tc_fence_before();
-        named_barrier(BAR, prep::kGroupThreads);
-        if (wp == 0) {
-            tc_fence_after();
-            const uint32_t idQ = idesc_bf16(128, DK, false, true);
-            // P (-W), into the columns MP has left: rows 0-63 of an M = 128
-            // product whose A starts at P
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_warp(tmem, smem_desc(sP + ks * 32, 16, 1024, kLayoutSW128),
-                              smem_desc(sK + ks * 2048, 16384, 1024, kLayoutSW128), idQ, ks > 0 ? 1u : 0u);
-            mma_commit_warp(&B[4]);
-        }
-        // Kbar, T_beta are no longer read: YT and ZB go over them
-        write_yt(sm + PrepSmem::KBAR, tmem + 128, quad, half, lane);
-        write_zb(sm + PrepSmem::TB, tmem + 192, quad, half, lane);
-        mbar_wait(&B[4], it & 1, abort_flag);
-        tc_fence_after();
-        write_qp(sm + PrepSmem::STK, tmem, quad, half, lane);
+        write_qp(sm + PrepSmem::STK, tmem + 128, quad, half, lane);
         if (leader) next_slot[(it + 1) & 1] = 2 * gridDim.x + drawn;
         fence_async_smem();
         tc_fence_before();
@@ -881,42 +871,50 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 // =============================================================== whole-d_v chain, transposed
 //
 // One CTA per (sequence, head) carrying the state transposed, S^T [j = d_v
-// lanes][c = d_k columns] fp32 in TMEM, with its bf16 copy SB^T also in TMEM
-// as the A operand of the products:
-//     S_{n+1}^T = S_n^T Diag(exp(G_L)) + SB_n^T MP_n^T + V_n^T YT_n^T
+// lanes][c = d_k columns]:
+//     S_{n+1}^T = S_n^T Diag(exp(G_L)) + X_n,   X_n = SB_n^T MP_n^T + V_n^T YT_n^T
 //     O_n^T     = SB_n^T QP_n^T + V_n^T ZB_n^T
-// The record operands keep their layout and descriptors; they only change
-// side (B instead of A), and V (its two 64-column atoms) is the A operand in
-// the MN-major form.  Against the row-major chain this removes the bf16 state
-// from shared memory (its store, the proxy fence, and the two reads per chunk
-// by the products), about a third of the chunk's shared-memory traffic, and
-// makes the output products M = 128.
-// Three rings, each with its own loader: A (MP, YT, exp(G_L)), V (the v
-// tile, read from HBM, so four stages ahead) and B (QP, ZB).
-//   warp 0: ring A;  warp 18: ring B;  warp 19: ring V
+// The fp32 state lives in the chain warps' registers (each thread one lane j
+// and 32 columns c); per chunk they write its bf16 copy SB_n^T into TMEM as
+// the A operand of the products, read the fresh product X_n back, and form
+// S_{n+1} with one FMA per element: no fp32 state goes back to TMEM.  The
+// record operands keep their layout and descriptors; they only change side
+// (B instead of A), and V (its two 64-column atoms) is the A operand in the
+// MN-major form.
+// The state-independent halves of the products, V_n^T YT_n^T into X and
+// V_n^T ZB_n^T into O, are issued ahead, while the chain warps still work on
+// the previous state, so that once SB_n is in TMEM only SB_n^T MP_n^T (8
+// products) stands between it and S_{n+1}; SB_n^T QP_n^T and the next
+// chunk's state-independent products then keep the tensor pipe busy while
+// the chain warps read X_n out.  X and O are double-buffered in TMEM.
+// Four rings, each with its own loader warp (exp(G_L) travels with ring A
+// but has its own deeper ring, since the chain warps read it only after the
+// state products): A (MP, YT), E (exp(G_L)), V (the v tile, read from HBM)
+// and B (QP, ZB).
+//   warp 0: rings A and E;  warp 18: ring B;  warp 19: ring V
 //   warps 1..16: the state; warp w holds lanes j of quadrant w mod 4 and
 //                columns c in 32 ((w - 1) / 4) .. + 31
 //   warp 17: issues the products
 struct ChainT {
     static constexpr int NCW = 16;
     static constexpr int THREADS = 32 * (NCW + 4);
-    static constexpr int NSA = 2, NSB = 2, NSV = 4;
+    static constexpr int NSA = 2, NSB = 2, NSV = 4, NSE = 4;
     static constexpr uint32_t A_MP = 0, A_YT = 32768, A_STRIDE = 49152;
     static constexpr uint32_t B_QP = 0, B_ZB = 16384, B_STRIDE = 24576;
     static constexpr uint32_t V_STRIDE = 16384;
     static constexpr uint32_t RA = 0;
     static constexpr uint32_t RV = NSA * A_STRIDE;
     static constexpr uint32_t RB = RV + NSV * V_STRIDE;
-    static constexpr uint32_t EGLR = RB + NSB * B_STRIDE;   // NSA x exp(G_L), 128 fp32 each
-    static constexpr uint32_t BARS = EGLR + NSA * 512;
+    static constexpr uint32_t EGLR = RB + NSB * B_STRIDE;   // NSE x exp(G_L), 128 fp32 each
+    static constexpr uint32_t BARS = EGLR + NSE * 512;
     static constexpr uint32_t MISC = BARS + 256;
     static constexpr uint32_t SIZE = MISC + 64;
     static constexpr uint32_t ALLOC = SIZE + 1024;
-    // TMEM columns: S^T fp32 (128), SB^T bf16 pairs x 2 (64 each), O^T fp32 x 2 (64 each)
+    // TMEM columns: X fp32 x 2 (128 each), SB^T bf16 pairs x 2 (64 each),
+    // O^T fp32 x 2 (64 each)
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t COL_S = 0, COL_SB = 128, COL_O = 256;
+    static constexpr uint32_t COL_X = 0, COL_SB = 256, COL_O = 384;
     static_assert(ALLOC <= 232448, "chain shared memory");
-    static_assert(2 * NSA + 2 * NSB + 2 * NSV + 5 <= 32, "barrier area");
 };
 
 // MODE (separate instantiations): kChainPlain; kChainTransition forms a
@@ -930,7 +928,7 @@ __global__ void __launch_bounds__(ChainT::THREADS, 1)
 kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     constexpr bool TRANS = MODE == kChainTransition;
     using Cfg = ChainT;
-    constexpr int NSA = Cfg::NSA, NSB = Cfg::NSB, NSV = Cfg::NSV, NCW = Cfg::NCW;
+    constexpr int NSA = Cfg::NSA, NSB = Cfg::NSB, NSV = Cfg::NSV, NSE = Cfg::NSE, NCW = Cfg::NCW;
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *sm = dyn_smem + ((1024u - (smem_addr(dyn_smem) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -944,17 +942,25 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     const size_t rec0 = (size_t)p.chunk_off[seq];
 
     // mbarriers: FULLA[NSA], EMPTYA[NSA], FULLB[NSB], EMPTYB[NSB], FULLV[NSV], EMPTYV[NSV],
-    // SDONE, ODONE[2], FIN, SREADY
+    // FULLE[NSE], EMPTYE[NSE], SDONE, ODONE[2], FIN, SREADY, OFREE[2]
     uint64_t *B = reinterpret_cast<uint64_t *>(sm + Cfg::BARS);
     uint64_t *FULLA = B, *EMPTYA = B + NSA, *FULLB = B + 2 * NSA, *EMPTYB = B + 2 * NSA + NSB;
     uint64_t *FULLV = B + 2 * NSA + 2 * NSB, *EMPTYV = FULLV + NSV;
-    uint64_t *SDONE = EMPTYV + NSV, *ODONE = SDONE + 1, *FIN = SDONE + 3, *SREADY = SDONE + 4;
-    constexpr int kBars = 2 * NSA + 2 * NSB + 2 * NSV + 5;
+    uint64_t *FULLE = EMPTYV + NSV, *EMPTYE = FULLE + NSE;
+    uint64_t *SDONE = EMPTYE + NSE, *ODONE = SDONE + 1, *FIN = SDONE + 3, *SREADY = SDONE + 4;
+    uint64_t *OFREE = SDONE + 5;
+    constexpr int kBars = 2 * NSA + 2 * NSB + 2 * NSV + 2 * NSE + 7;
+    static_assert(kBars * 8 <= 256, "barrier area");
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + Cfg::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     if (tid == 0) {
-        for (int i = 0; i < kBars - 1; ++i) mbar_init(&B[i], 1);
-        mbar_init(SREADY, NCW);   // one arrive per chain warp
+        for (int i = 0; i < kBars; ++i) {
+            // SREADY, EMPTYE and OFREE take one arrive per chain warp
+            const uint64_t *b = &B[i];
+            const bool per_warp = b == SREADY || b == &OFREE[0] || b == &OFREE[1] ||
+                                  (b >= EMPTYE && b < EMPTYE + NSE);
+            mbar_init(&B[i], per_warp ? (uint32_t)NCW : 1u);
+        }
         misc[1] = 0u;
         fence_mbar_init();
     }
@@ -968,25 +974,30 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     const uint32_t tmem = misc[0];
 
     if (warp == 0) {
-        // ---------------------------------------------- ring A: MP, YT, exp(G_L)
+        // ---------------------------------------------- rings A (MP, YT) and E (exp(G_L))
         if (lane == 0 && nchunks > 0) {
-            int issued_a = 0;
+            int issued_a = 0, issued_e = 0;
             for (int n = 0; n < nchunks; ++n) {
-                const int sa = n % NSA;
+                const int sa = n % NSA, se = n % NSE;
                 if (n >= NSA) mbar_wait(&EMPTYA[sa], ((n / NSA) - 1) & 1, abort_flag);
+                if (n >= NSE) mbar_wait(&EMPTYE[se], ((n / NSE) - 1) & 1, abort_flag);
                 if (*abort_flag) break;
                 const size_t ri = (rec0 + n) * p.H + h;
                 const uint8_t *rec = p.recs + ri * Rec::STRIDE;
                 if (p.rec_ready && !acquire_flag(p.rec_ready + ri, abort_flag)) break;   // the record is complete
                 uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
-                mbar_arrive_expect_tx(&FULLA[sa], 49152 + 512);
+                mbar_arrive_expect_tx(&FULLA[sa], 49152);
                 bulk_load(slot_a + Cfg::A_MP, rec + Rec::MP, 49152, &FULLA[sa]);   // MP, YT
-                bulk_load(sm + Cfg::EGLR + sa * 512, rec + Rec::EGL, 512, &FULLA[sa]);
                 issued_a = n + 1;
+                mbar_arrive_expect_tx(&FULLE[se], 512);
+                bulk_load(sm + Cfg::EGLR + se * 512, rec + Rec::EGL, 512, &FULLE[se]);
+                issued_e = n + 1;
             }
             // the copies land before this CTA may exit
             for (int n = (issued_a > NSA ? issued_a - NSA : 0); n < issued_a; ++n)
                 wait_drain(&FULLA[n % NSA], (n / NSA) & 1);
+            for (int n = (issued_e > NSE ? issued_e - NSE : 0); n < issued_e; ++n)
+                wait_drain(&FULLE[n % NSE], (n / NSE) & 1);
         }
     } else if (warp == NCW + 3) {
         // ---------------------------------------------- ring V: the v tile (from HBM)
@@ -1032,51 +1043,61 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         const uint32_t idSV = idesc_bf16(128, 128, true, false);   // A = V^T (MN-major), B = YT^T
         const uint32_t idO = idesc_bf16(128, 64, false, false);    // A = SB^T (TMEM), B = QP^T
         const uint32_t idOV = idesc_bf16(128, 64, true, false);    // A = V^T (MN-major), B = ZB^T
-        for (int n = 0; n < nchunks; ++n) {
-            const int sa = n % NSA, sb = n % NSB, sv = n % NSV;
-            uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
-            uint8_t *slot_b = sm + Cfg::RB + sb * Cfg::B_STRIDE;
-            const uint32_t bM = smem_addr(slot_a + Cfg::A_MP);
-            const uint32_t bY = smem_addr(slot_a + Cfg::A_YT);
+        // The state-independent products of chunk m: X[m mod 2] = V^T YT^T and
+        // O[m mod 2] = V^T ZB^T.  X[m mod 2] was last read by the chain warps
+        // before their SREADY of chunk m - 1, which this warp has passed; O[m
+        // mod 2] is free once they have read O_{m-2} out (OFREE).
+        auto pre = [&](int m) {
+            if (TRANS) return;
+            const int sa = m % NSA, sb = m % NSB, sv = m % NSV;
+            const uint32_t bY = smem_addr(sm + Cfg::RA + sa * Cfg::A_STRIDE + Cfg::A_YT);
+            const uint32_t bZ = smem_addr(sm + Cfg::RB + sb * Cfg::B_STRIDE + Cfg::B_ZB);
             const uint32_t aV = smem_addr(sm + Cfg::RV + sv * Cfg::V_STRIDE);
-            const uint32_t aSB = tmem + Cfg::COL_SB + 64u * (uint32_t)(n & 1);
-            mbar_wait(SREADY, n & 1, abort_flag);
-            mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
-            if (!TRANS) mbar_wait(&FULLV[sv], (n / NSV) & 1, abort_flag);
+            mbar_wait(&FULLA[sa], (m / NSA) & 1, abort_flag);
+            mbar_wait(&FULLV[sv], (m / NSV) & 1, abort_flag);
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)   // S^T += SB^T MP^T  (K = c')
-                mma_bf16_ts_warp(tmem + Cfg::COL_S, aSB + 8 * ks,
-                                 smem_desc(bM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                                 idS, 1u);
-            if (!TRANS) {
+            for (int ks = 0; ks < 4; ++ks)   // X = V^T YT^T  (K = t)
+                mma_bf16_warp(tmem + Cfg::COL_X + 128u * (uint32_t)(m & 1),
+                              smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
+                              smem_desc(bY + ks * 32, 16, 1024, kLayoutSW128), idSV, ks > 0 ? 1u : 0u);
+            mbar_wait(&FULLB[sb], (m / NSB) & 1, abort_flag);
+            if (m >= 2) mbar_wait(&OFREE[m & 1], ((m - 2) >> 1) & 1, abort_flag);
+            tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)   // S^T += V^T YT^T  (K = t)
-                    mma_bf16_warp(tmem + Cfg::COL_S, smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
-                                  smem_desc(bY + ks * 32, 16, 1024, kLayoutSW128), idSV, 1u);
-            }
-            mma_commit_warp(SDONE);
-            if (TRANS) {   // no output: the slot is free once the state products are done
-                mma_commit_warp(&EMPTYA[sa]);
-                continue;
-            }
-            mbar_wait(&FULLB[sb], (n / NSB) & 1, abort_flag);
-            const uint32_t bQ = smem_addr(slot_b + Cfg::B_QP);
-            const uint32_t bZ = smem_addr(slot_b + Cfg::B_ZB);
-            const uint32_t dO = tmem + Cfg::COL_O + 64u * (uint32_t)(n & 1);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)   // O^T = SB^T QP^T  (K = c)
-                mma_bf16_ts_warp(dO, aSB + 8 * ks,
-                                 smem_desc(bQ + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                                 idO, ks > 0 ? 1u : 0u);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)   // O^T += V^T ZB^T  (K = t')
-                mma_bf16_warp(dO, smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
-                              smem_desc(bZ + ks * 32, 16, 1024, kLayoutSW128), idOV, 1u);
-            mma_commit_warp(&ODONE[n & 1]);
-            mma_commit_warp(&EMPTYA[sa]);
-            mma_commit_warp(&EMPTYB[sb]);
+            for (int ks = 0; ks < 4; ++ks)   // O^T = V^T ZB^T  (K = t')
+                mma_bf16_warp(tmem + Cfg::COL_O + 64u * (uint32_t)(m & 1),
+                              smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
+                              smem_desc(bZ + ks * 32, 16, 1024, kLayoutSW128), idOV, ks > 0 ? 1u : 0u);
             mma_commit_warp(&EMPTYV[sv]);
+        };
+        if (nchunks > 0) pre(0);
+        for (int n = 0; n < nchunks; ++n) {
+            const int sa = n % NSA, sb = n % NSB;
+            const uint32_t bM = smem_addr(sm + Cfg::RA + sa * Cfg::A_STRIDE + Cfg::A_MP);
+            const uint32_t aSB = tmem + Cfg::COL_SB + 64u * (uint32_t)(n & 1);
+            if (TRANS) mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
+            mbar_wait(SREADY, n & 1, abort_flag);
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)   // X += SB^T MP^T  (K = c')
+                mma_bf16_ts_warp(tmem + Cfg::COL_X + 128u * (uint32_t)(n & 1), aSB + 8 * ks,
+                                 smem_desc(bM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                                 idS, (TRANS && ks == 0) ? 0u : 1u);
+            mma_commit_warp(SDONE);
+            mma_commit_warp(&EMPTYA[sa]);
+            if (!TRANS) {
+                const uint32_t bQ = smem_addr(sm + Cfg::RB + sb * Cfg::B_STRIDE + Cfg::B_QP);
+                const uint32_t dO = tmem + Cfg::COL_O + 64u * (uint32_t)(n & 1);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)   // O^T += SB^T QP^T  (K = c)
+                    mma_bf16_ts_warp(dO, aSB + 8 * ks,
+                                     smem_desc(bQ + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                                     idO, 1u);
+                mma_commit_warp(&ODONE[n & 1]);
+                mma_commit_warp(&EMPTYB[sb]);
+            }
+            if (n + 1 < nchunks) pre(n + 1);
         }
         if (nchunks > 0) {   // every arrive of the commits above lands before the CTA exits
             mma_commit_warp(FIN);
@@ -1099,13 +1120,17 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] = 0.f;
         }
-        // O^T of chunk m: this warp's 16 t columns, lane j, bf16 to o[t][h][j]
+        // O^T of chunk m: this warp's 16 t columns, lane j, bf16 to o[t][h][j];
+        // the buffer is released (OFREE) as soon as it is in registers
         auto store_o_t = [&](int m) {
             mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
             tc_fence_after();
             float v[16];
             tmem_ld16(tmem_addr(tmem, 32 * quad, Cfg::COL_O + 64 * (m & 1) + 16 * g), v);
             tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&OFREE[m & 1]);
             const int64_t t0 = (int64_t)m * C + 16 * g;
             __nv_bfloat16 *dst = p.o + ((size_t)(bos + t0) * p.H + h) * DV + j;
 #pragma unroll
@@ -1113,37 +1138,43 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 if (t0 + i < len) dst[(size_t)i * p.H * DV] = __float2bfloat16(v[i]);
         };
         for (int n = 0; n < nchunks; ++n) {
-            const int sa = n % NSA;
-            if (n >= 1) {
-                mbar_wait(SDONE, (n - 1) & 1, abort_flag);
-                tc_fence_after();
-                tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + 32 * g), S);
-                tmem_wait_ld();
-            }
-            // SB_n^T: column COL_SB + 64 (n mod 2) + c / 2 holds (c, c + 1)
+            // SB_n^T: column COL_SB + 64 (n mod 2) + c / 2 holds (c, c + 1).  Its
+            // previous contents, SB_{n-2}, were last read by chunk n - 2's
+            // products, which completed before SDONE of chunk n - 1.
             uint32_t w16[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) w16[i] = pack_bf16x2(S[2 * i], S[2 * i + 1]);
             tmem_st16u(tmem_addr(tmem, 32 * quad, Cfg::COL_SB + 64 * (n & 1) + 16 * g), w16);
-            mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
-            const float *egl = reinterpret_cast<const float *>(sm + Cfg::EGLR + sa * 512) + 32 * g;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) S[i] *= egl[i];
-            tmem_st32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + 32 * g), S);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(SREADY);
             if (!TRANS && n >= 1) store_o_t(n - 1);
-        }
-        if (nchunks > 0) {
-            const int m = nchunks - 1;
-            if (!TRANS) store_o_t(m);
-            mbar_wait(SDONE, m & 1, abort_flag);
+            // S_{n+1} = S_n Diag(exp(G_L)) + X_n, in two halves of 16 columns
+            const int se = n % NSE;
+            mbar_wait(&FULLE[se], (n / NSE) & 1, abort_flag);
+            mbar_wait(SDONE, n & 1, abort_flag);
             tc_fence_after();
-            tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + 32 * g), S);
-            tmem_wait_ld();
+            const float4 *egl = reinterpret_cast<const float4 *>(sm + Cfg::EGLR + se * 512) + 8 * g;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float x[16];
+                tmem_ld16(tmem_addr(tmem, 32 * quad, Cfg::COL_X + 128 * (n & 1) + 32 * g + 16 * hh), x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 d = egl[4 * hh + e4];
+                    float *s = S + 16 * hh + 4 * e4;
+                    s[0] = fmaf(s[0], d.x, x[4 * e4 + 0]);
+                    s[1] = fmaf(s[1], d.y, x[4 * e4 + 1]);
+                    s[2] = fmaf(s[2], d.z, x[4 * e4 + 2]);
+                    s[3] = fmaf(s[3], d.w, x[4 * e4 + 3]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&EMPTYE[se]);
         }
+        if (!TRANS && nchunks > 0) store_o_t(nchunks - 1);
         if (p.final_state) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) p.final_state[sbase + (size_t)i * DV] = S[i];
