@@ -92,28 +92,26 @@ static_assert(PrepSmem::KHAT + 64 * prep::kAStride * 4 <= PrepSmem::GRAW &&
 constexpr uint32_t kPrepTmemCols = 512;
 constexpr uint32_t kRawBytes = 4 * 8192 + 16384;   // k, q (2 boxes each), log_alpha
 
-// ---- chain kernel, one CTA per (sequence, head, DVT-column slice of d_v).
+// ---- chain kernel, one CTA per (sequence, head, 32-column slice of d_v).
 // Warp 0 loads ring A, warp NCW + 2 ring B (each ring runs ahead on its own);
 // warps 1 .. NCW hold the state (warp w: TMEM lanes of quadrant w mod 4,
 // columns 32 ((w - 1) / 4) .. + 31 of the slice); warp NCW + 1 issues the
 // products.  Ring A carries MP, YT, the v slice and exp(G_L); ring B QP, ZB.
-// Stages (A, B) and bf16 state copies: (3, 2) and 2 for 32 columns, (3, 1)
-// and 2 for 64, (2, 2) and 1 for 128: what shared memory holds.
+// Three ring-A and two ring-B stages, two bf16 state copies.
 constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 
 template <int DVT_>
 struct ChainCfg {
     static constexpr int DVT = DVT_;
+    static_assert(DVT_ == 32, "the row-major chain runs 32-column slices");
     static constexpr int NTILE = DV / DVT;
     static constexpr int NCW = 4 * (DVT / 32);
     static constexpr int THREADS = 32 * (NCW + 3);
-    static constexpr int NSA = DVT == 128 ? 2 : 3;
-    static constexpr int NSB = DVT == 64 ? 1 : 2;
+    static constexpr int NSA = 3;
+    static constexpr int NSB = 2;
     // Copies of the bf16 state: two let the chain warps write S_{n+1} while
-    // chunk n's output products still read S_n; whole-d_v CTAs keep one (and
-    // a second ring-B stage in its place), the chain warps waiting for those
-    // products first.
-    static constexpr int NSBC = DVT == 128 ? 1 : 2;
+    // chunk n's output products still read S_n.
+    static constexpr int NSBC = 2;
     static constexpr uint32_t V_BYTES = (uint32_t)DVT * C * 2;
     static constexpr uint32_t A_MP = 0, A_YT = 32768, A_V = 49152;
     static constexpr uint32_t A_STRIDE = align1k(A_V + V_BYTES);
@@ -125,14 +123,14 @@ struct ChainCfg {
     static constexpr uint32_t SB = RB + NSB * B_STRIDE;
     static constexpr uint32_t EGLR = SB + NSBC * SB_BYTES;  // NSA x exp(G_L), 128 fp32 each
     static constexpr uint32_t BARS = EGLR + NSA * 512;
-    static constexpr uint32_t MISC = BARS + 128;
+    static constexpr uint32_t MISC = BARS + 256;
     static constexpr uint32_t SIZE = MISC + 64;
     static constexpr uint32_t ALLOC = SIZE + 1024;
-    static constexpr uint32_t TMEM_COLS = DVT == 32 ? 128 : (DVT == 64 ? 256 : 512);
-    static constexpr uint32_t COL_S = 0, COL_O = DVT;   // S; O x2 at DVT + DVT b (M = 64)
+    static constexpr uint32_t TMEM_COLS = 128;
+    // X (the chunk's state products) x2, then O x2 (M = 64 layout)
+    static constexpr uint32_t COL_X = 0, COL_O = 2 * DVT;
     static_assert(ALLOC <= 232448, "chain shared memory");
-    static_assert(3 * DVT <= (int)TMEM_COLS, "chain TMEM");
-    static_assert(2 * NSA + 2 * NSB + 5 <= 16, "barrier area");
+    static_assert(4 * DVT <= (int)TMEM_COLS, "chain TMEM");
 };
 static_assert(Rec::YT == Rec::MP + 32768 && Rec::ZB == Rec::QP + 16384,
               "MP and YT, QP and ZB travel as one copy each");
@@ -636,11 +634,15 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t base, int ks) {
 // reads, lanes 0-15 hold rows.
 template <int DVT>
 __device__ __forceinline__ void store_o(uint32_t tmem, int quad, int lane, int col0, int m,
-                                        int64_t bos, int64_t len, int h, int j0, const Params &p) {
+                                        int64_t bos, int64_t len, int h, int j0, const Params &p,
+                                        uint64_t *ofree) {
     using Cfg = ChainCfg<DVT>;
     float v[32];
     tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_O + DVT * (m & 1) + col0), v);
     tmem_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(ofree);   // the O buffer may be written again
     const int t = 16 * quad + lane;
     if (lane < 16 && (int64_t)m * C + t < len) {
         uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((size_t)(bos + (int64_t)m * C + t) * p.H + h) * DV +
@@ -657,12 +659,16 @@ __device__ __forceinline__ void store_o(uint32_t tmem, int quad, int lane, int c
     }
 }
 
-// Per chunk n, with S_n (fp32) in TMEM:
-//   chain warps: S_n -> bf16 SB[n mod 2];  TMEM S <- Diag(exp(G_L)) S_n
-//   product warp, S products (the serial path):  S += MP SB,  S += YT V
-//                 O products (off it):           O[n mod 2] = QP SB + ZB V
-// The chain warps read the O of chunk n out while chunk n + 1 runs; the
-// product warp issues chunk n's O products while they convert S_{n+1}.
+// Per chunk n, with S_n (fp32) in the chain warps' registers (each thread one
+// row c and 32 columns of the slice):
+//   chain warps: S_n -> bf16 SB[n mod 2] (shared memory, the B operand)
+//   product warp, ahead (state-independent): X[n mod 2] = YT V, O[n mod 2] = ZB V
+//                 after SB_n:  X[n mod 2] += MP SB_n  (the serial path),
+//                              O[n mod 2] += QP SB_n
+//   chain warps: S_{n+1} = Diag(exp(G_L)) S_n + X[n mod 2]
+// The chain warps read the O of chunk n - 1 out while chunk n's state
+// products run.  X[n mod 2] was read by the chain warps before their SREADY
+// of chunk n - 1, O[n mod 2] once they arrive on OFREE after reading O_{n-2}.
 template <int DVT>
 __global__ void __launch_bounds__(ChainCfg<DVT>::THREADS, 1)
 kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -682,16 +688,23 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     const int j0 = tile * DVT;
     const size_t rec0 = (size_t)p.chunk_off[seq];
 
-    // mbarriers: FULLA[NSA], EMPTYA[NSA], FULLB[NSB], EMPTYB[NSB], SDONE, ODONE[2], FIN, SREADY
+    // mbarriers: FULLA[NSA], EMPTYA[NSA], FULLB[NSB], EMPTYB[NSB], SDONE, ODONE[2], FIN,
+    // SREADY, OFREE[2]
     uint64_t *B = reinterpret_cast<uint64_t *>(sm + Cfg::BARS);
     uint64_t *FULLA = B, *EMPTYA = B + NSA, *FULLB = B + 2 * NSA, *EMPTYB = B + 2 * NSA + NSB;
     uint64_t *SDONE = B + 2 * NSA + 2 * NSB, *ODONE = SDONE + 1, *FIN = SDONE + 3, *SREADY = SDONE + 4;
-    constexpr int kBars = 2 * NSA + 2 * NSB + 5;
+    uint64_t *OFREE = SDONE + 5;
+    constexpr int kBars = 2 * NSA + 2 * NSB + 7;
+    static_assert(kBars * 8 <= 256, "barrier area");
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + Cfg::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     if (tid == 0) {
-        for (int i = 0; i < kBars - 1; ++i) mbar_init(&B[i], 1);
-        mbar_init(SREADY, NCW);   // one arrive per chain warp
+        for (int i = 0; i < kBars; ++i) {
+            // SREADY and OFREE take one arrive per chain warp
+            const uint64_t *b = &B[i];
+            const bool per_warp = b == SREADY || b == &OFREE[0] || b == &OFREE[1];
+            mbar_init(&B[i], per_warp ? (uint32_t)NCW : 1u);
+        }
         misc[1] = 0u;
         fence_mbar_init();
     }
@@ -722,7 +735,6 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 bulk_load(slot_a + Cfg::A_MP, rec + Rec::MP, 49152, &FULLA[sa]);   // MP, YT
                 bulk_load(sm + Cfg::EGLR + sa * 512, rec + Rec::EGL, 512, &FULLA[sa]);
                 tma_load_3d(slot_a + Cfg::A_V, &tm_v, &FULLA[sa], j0, h, t);
-                if (DVT == 128) tma_load_3d(slot_a + Cfg::A_V + 8192, &tm_v, &FULLA[sa], j0 + 64, h, t);
                 issued_a = n + 1;
             }
             // the copies land before this CTA may exit
@@ -752,42 +764,52 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         // ---------------------------------------------- tensor-core products
         const uint32_t idS = idesc_bf16(128, DVT, false, true);
         const uint32_t idO = idesc_bf16(64, DVT, false, true);
+        // the state-independent products of chunk m: X[m mod 2] = YT V, O[m mod 2] = ZB V
+        auto pre = [&](int m) {
+            const int sa = m % NSA, sb = m % NSB;
+            uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
+            const uint32_t aY = smem_addr(slot_a + Cfg::A_YT);
+            const uint32_t bV = smem_addr(slot_a + Cfg::A_V);
+            const uint32_t aZ = smem_addr(sm + Cfg::RB + sb * Cfg::B_STRIDE + Cfg::B_ZB);
+            mbar_wait(&FULLA[sa], (m / NSA) & 1, abort_flag);
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)   // X = YT V
+                mma_bf16_warp(tmem + Cfg::COL_X + DVT * (m & 1), smem_desc(aY + ks * 32, 16, 1024, kLayoutSW128),
+                              desc_v<DVT>(bV, ks), idS, ks > 0 ? 1u : 0u);
+            mbar_wait(&FULLB[sb], (m / NSB) & 1, abort_flag);
+            if (m >= 2) mbar_wait(&OFREE[m & 1], ((m - 2) >> 1) & 1, abort_flag);
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)   // O = ZB V
+                mma_bf16_warp(tmem + Cfg::COL_O + DVT * (m & 1), smem_desc(aZ + ks * 32, 16, 1024, kLayoutSW128),
+                              desc_v<DVT>(bV, ks), idO, ks > 0 ? 1u : 0u);
+        };
+        if (nchunks > 0) pre(0);
         for (int n = 0; n < nchunks; ++n) {
             const int sa = n % NSA, sb = n % NSB;
             uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
             uint8_t *slot_b = sm + Cfg::RB + sb * Cfg::B_STRIDE;
             const uint32_t aM = smem_addr(slot_a + Cfg::A_MP);
-            const uint32_t aY = smem_addr(slot_a + Cfg::A_YT);
-            const uint32_t bV = smem_addr(slot_a + Cfg::A_V);
-            const uint32_t bS = smem_addr(sm + Cfg::SB + (Cfg::NSBC == 2 ? (n & 1) : 0) * Cfg::SB_BYTES);
+            const uint32_t bS = smem_addr(sm + Cfg::SB + (n & 1) * Cfg::SB_BYTES);
             mbar_wait(SREADY, n & 1, abort_flag);
-            mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)   // S += MP SB
-                mma_bf16_warp(tmem + Cfg::COL_S,
+            for (int ks = 0; ks < 8; ++ks)   // X += MP SB
+                mma_bf16_warp(tmem + Cfg::COL_X + DVT * (n & 1),
                               smem_desc(aM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
                               desc_sb<DVT>(bS, ks), idS, 1u);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)   // S += YT V
-                mma_bf16_warp(tmem + Cfg::COL_S, smem_desc(aY + ks * 32, 16, 1024, kLayoutSW128),
-                              desc_v<DVT>(bV, ks), idS, 1u);
             mma_commit_warp(SDONE);
-            mbar_wait(&FULLB[sb], (n / NSB) & 1, abort_flag);
             const uint32_t aQ = smem_addr(slot_b + Cfg::B_QP);
-            const uint32_t aZ = smem_addr(slot_b + Cfg::B_ZB);
             const uint32_t dO = tmem + Cfg::COL_O + DVT * (n & 1);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)   // O = QP SB
+            for (int ks = 0; ks < 8; ++ks)   // O += QP SB
                 mma_bf16_warp(dO, smem_desc(aQ + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                              desc_sb<DVT>(bS, ks), idO, ks > 0 ? 1u : 0u);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)   // O += ZB V
-                mma_bf16_warp(dO, smem_desc(aZ + ks * 32, 16, 1024, kLayoutSW128), desc_v<DVT>(bV, ks),
-                              idO, 1u);
+                              desc_sb<DVT>(bS, ks), idO, 1u);
             mma_commit_warp(&ODONE[n & 1]);
             mma_commit_warp(&EMPTYA[sa]);
             mma_commit_warp(&EMPTYB[sb]);
+            if (n + 1 < nchunks) pre(n + 1);
         }
         if (nchunks > 0) {   // every arrive of the commits above lands before the CTA exits
             mma_commit_warp(FIN);
@@ -811,47 +833,33 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] = 0.f;
         }
+        auto store_o_m = [&](int m) {   // O of chunk m; the buffer is released once in registers
+            mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
+            tc_fence_after();
+            store_o<DVT>(tmem, quad, lane, col0, m, bos, len, h, j0, p, &OFREE[m & 1]);
+        };
         for (int n = 0; n < nchunks; ++n) {
             const int sa = n % NSA;
-            const uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
-            if (n >= 1) {
-                mbar_wait(SDONE, (n - 1) & 1, abort_flag);
-                tc_fence_after();
-                tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + col0), S);
-                tmem_wait_ld();
-            }
-            if (Cfg::NSBC == 1 && n >= 1) {   // chunk n-1's output products have read S_{n-1}
-                mbar_wait(&ODONE[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag);
-                tc_fence_after();
-            }
-            store_sb_row<DVT>(sm + Cfg::SB + (Cfg::NSBC == 2 ? (n & 1) : 0) * Cfg::SB_BYTES, crow, col0, S);
+            // SB[n mod 2] was last read by chunk n - 2's products, which
+            // completed before SDONE of chunk n - 1
+            store_sb_row<DVT>(sm + Cfg::SB + (n & 1) * Cfg::SB_BYTES, crow, col0, S);
+            // this row's exp(G_L), read before the slot may be refilled
             mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
             const float d = reinterpret_cast<const float *>(sm + Cfg::EGLR + sa * 512)[crow];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) S[i] *= d;
-            tmem_st32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + col0), S);
-            tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(SREADY);
-            if (n >= 1) {
-                const int m = n - 1;
-                mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
-                tc_fence_after();
-                store_o<DVT>(tmem, quad, lane, col0, m, bos, len, h, j0, p);
-            }
-        }
-        if (nchunks > 0) {
-            const int m = nchunks - 1;
-            mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
+            if (n >= 1) store_o_m(n - 1);
+            mbar_wait(SDONE, n & 1, abort_flag);
             tc_fence_after();
-            store_o<DVT>(tmem, quad, lane, col0, m, bos, len, h, j0, p);
-            mbar_wait(SDONE, m & 1, abort_flag);
-            tc_fence_after();
-            tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_S + col0), S);
+            float x[32];
+            tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_X + DVT * (n & 1) + col0), x);
             tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) S[i] = fmaf(S[i], d, x[i]);
         }
+        if (nchunks > 0) store_o_m(nchunks - 1);
         if (p.final_state) {
             float4 *dst = reinterpret_cast<float4 *>(p.final_state + soff);
 #pragma unroll
