@@ -496,6 +496,9 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only the prefill workload (a lighter command for profiler captures); "
+                         "prints a line without the extra objects")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -517,6 +520,20 @@ def main():
     sampler = ClockSampler(local)
     sampler.start()
     pf = time_prefill(w, args.steps, args.warmup, world)
+    if args.prefill_only:
+        clocks = sampler.stop()
+        work = prefill_work(w, pf["inputs"]["lengths"])
+        ms_step = max_over_ranks(pf["ms_total"] / args.steps, world)
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": world * work["tokens"] / (ms_step * 1e-3),
+                              "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                              "warmup": args.warmup, "ms_per_step": ms_step,
+                              "config": config_of(w, pf["inputs"]["lengths"], world),
+                              "gpu_launches": pf["launches"], "clocks": clocks}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
     extra = []
     for key, name in EXTRA_PREFILL:
         if name != w.name:
