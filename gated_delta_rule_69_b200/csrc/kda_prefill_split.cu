@@ -75,8 +75,7 @@ struct PrepSmem {
     static constexpr uint32_t BETA = 105984;   // 64 fp32
     static constexpr uint32_t CSUM = 106240;   // 4 x 128 fp32
     static constexpr uint32_t BARS = 108288;   // 6 mbarriers
-    static constexpr uint32_t MISC = 108352;   // tmem base, abort, slow flag, next-item slots at 4, 5,
-                                               // their token ranges at 6-9
+    static constexpr uint32_t MISC = 108352;   // tmem base, abort, slow flag, next-item slots at 4, 5
     static constexpr uint32_t NRM = 108416;    // layer prologue: 128 fp32 inverse norms
     static constexpr uint32_t SIZE = 108928;
     static constexpr uint32_t PIPE = 109568;   // per-pipeline stride
@@ -346,7 +345,8 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
     float *beta = reinterpret_cast<float *>(sm + PrepSmem::BETA);
     // The leader publishes a record one step late: it waits only for the
     // stores to have read shared memory before it loads the next item, and
-    // for their writes to complete once those loads are in flight.
+    // for their writes to complete once the next item's first product has
+    // been issued, by which time they have long landed.
     uint32_t *pending = nullptr;
     uint32_t sec_round = 0;   // phases of B[5] (secondary-chunking products) so far
     // Items: each pipeline starts with its own, then takes the next free one
@@ -354,19 +354,13 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
     // share would leave the slowest as the tail).  The leader draws the
     // following item early in the current one and leaves it in a two-entry
     // slot, which every thread reads after the current item's last barrier.
-    // With the item the slot carries its chunk's (first token, length), read
-    // from the plan's table by the leader then, so that no item starts with a
-    // global load before its own loads can be issued.
     volatile uint32_t *next_slot = misc + 4;
-    volatile int32_t *next_ct = reinterpret_cast<volatile int32_t *>(misc + 6);   // [2][2]
     uint32_t item = 2 * blockIdx.x + P;
-    int2 ct_next = make_int2(0, 0);
-    if (item < total_items) ct_next = p.chunk_tab[item / p.H];
 #pragma unroll 1
     for (int it = 0; item < total_items; ++it) {
         const int h = item % p.H;
         const uint32_t chunk = item / p.H;
-        const int2 ct = ct_next;   // the token range was planned
+        const int2 ct = p.chunk_tab[chunk];   // one load: the token range was planned
         const int64_t tok0 = ct.x;
         const int L = ct.y;
         uint8_t *rec = p.recs + ((size_t)chunk * p.H + h) * Rec::STRIDE;
@@ -385,20 +379,6 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
             if (!p.scalar_gate) tma_load_3d(sm + PrepSmem::GRAW, &tm_g, &B[0], 0, h, t);
             bulk_wait_read_all();
             mbar_arrive(&B[0]);
-            // While the loads are in flight: draw the next item and read its
-            // token range, and publish the previous record once its stores
-            // have completed.
-            const uint32_t nxt = 2 * gridDim.x + atomicAdd(p.work_next, 1u);
-            int2 nct = make_int2(0, 0);
-            if (nxt < total_items) nct = p.chunk_tab[nxt / p.H];
-            next_slot[(it + 1) & 1] = nxt;
-            next_ct[2 * ((it + 1) & 1)] = nct.x;
-            next_ct[2 * ((it + 1) & 1) + 1] = nct.y;
-            if (pending) {
-                bulk_wait_all();
-                publish_flag(pending);
-                pending = nullptr;
-            }
         }
         if (pt < C) {
             float bv = (pt < L) ? __bfloat162float(p.beta[(size_t)(tok0 + pt) * p.H + h]) : 0.f;
@@ -444,6 +424,7 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         const int form = prep::gate<BAR, LAYER>(b, pt, L);
         fence_async_smem();
         named_barrier(BAR, prep::kGroupThreads);
+        uint32_t drawn = 0;
         if (wp == 0) {   // tensor-core products: issued by the group's first warp
             tc_fence_after();
             const uint32_t a0 = smem_addr(sm + PrepSmem::STK), b0 = smem_addr(sm + PrepSmem::KHAT);
@@ -454,6 +435,14 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
                               smem_desc(b0 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
                               id, ks > 0 ? 1u : 0u);
             mma_commit_warp(&B[1]);
+        }
+        if (leader) {
+            drawn = atomicAdd(p.work_next, 1u);   // consumed at the end of the item
+            if (pending) {
+                bulk_wait_all();
+                publish_flag(pending);
+                pending = nullptr;
+            }
         }
         mbar_wait(&B[1], it & 1, abort_flag);
         tc_fence_after();
@@ -523,11 +512,11 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         tc_fence_after();
         write_mp(sm + PrepSmem::KHAT, sm + PrepSmem::GRAW, tmem, quad, half, lane);
         write_qp(sm + PrepSmem::STK, tmem + 128, quad, half, lane);
+        if (leader) next_slot[(it + 1) & 1] = 2 * gridDim.x + drawn;
         fence_async_smem();
         tc_fence_before();
         named_barrier(BAR, prep::kGroupThreads);
         const uint32_t next_item = next_slot[(it + 1) & 1];
-        ct_next = make_int2(next_ct[2 * ((it + 1) & 1)], next_ct[2 * ((it + 1) & 1) + 1]);
         if (leader) {
             // first group: the sources the next item's loads overwrite
             bulk_store(rec + Rec::QP, sm + PrepSmem::STK + 8192, 8192);
@@ -678,8 +667,8 @@ __device__ __forceinline__ void store_o(uint32_t tmem, int quad, int lane, int c
 //                              O[n mod 2] += QP SB_n
 //   chain warps: S_{n+1} = Diag(exp(G_L)) S_n + X[n mod 2]
 // The chain warps read the O of chunk n - 1 out while chunk n's state
-// products run.  X[n mod 2] was read by the chain warps before their SB-ready
-// arrival of chunk n - 1, O[n mod 2] once they arrive on OFREE after reading O_{n-2}.
+// products run.  X[n mod 2] was read by the chain warps before their SREADY
+// of chunk n - 1, O[n mod 2] once they arrive on OFREE after reading O_{n-2}.
 template <int DVT>
 __global__ void __launch_bounds__(ChainCfg<DVT>::THREADS, 1)
 kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -700,23 +689,20 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     const size_t rec0 = (size_t)p.chunk_off[seq];
 
     // mbarriers: FULLA[NSA], EMPTYA[NSA], FULLB[NSB], EMPTYB[NSB], SDONE, ODONE[2], FIN,
-    // OFREE[2]
+    // SREADY, OFREE[2]
     uint64_t *B = reinterpret_cast<uint64_t *>(sm + Cfg::BARS);
     uint64_t *FULLA = B, *EMPTYA = B + NSA, *FULLB = B + 2 * NSA, *EMPTYB = B + 2 * NSA + NSB;
-    uint64_t *SDONE = B + 2 * NSA + 2 * NSB, *ODONE = SDONE + 1, *FIN = SDONE + 3;
-    uint64_t *OFREE = SDONE + 4;
-    constexpr int kBars = 2 * NSA + 2 * NSB + 6;
+    uint64_t *SDONE = B + 2 * NSA + 2 * NSB, *ODONE = SDONE + 1, *FIN = SDONE + 3, *SREADY = SDONE + 4;
+    uint64_t *OFREE = SDONE + 5;
+    constexpr int kBars = 2 * NSA + 2 * NSB + 7;
     static_assert(kBars * 8 <= 256, "barrier area");
-    // SB_n ready: the chain warps arrive on a named barrier, the product
-    // warp waits on it
-    constexpr uint32_t kBarSReady = 1, kSReadyThreads = 32 * (NCW + 1);
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + Cfg::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     if (tid == 0) {
         for (int i = 0; i < kBars; ++i) {
-            // OFREE takes one arrive per chain warp
+            // SREADY and OFREE take one arrive per chain warp
             const uint64_t *b = &B[i];
-            const bool per_warp = b == &OFREE[0] || b == &OFREE[1];
+            const bool per_warp = b == SREADY || b == &OFREE[0] || b == &OFREE[1];
             mbar_init(&B[i], per_warp ? (uint32_t)NCW : 1u);
         }
         misc[1] = 0u;
@@ -806,7 +792,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             uint8_t *slot_b = sm + Cfg::RB + sb * Cfg::B_STRIDE;
             const uint32_t aM = smem_addr(slot_a + Cfg::A_MP);
             const uint32_t bS = smem_addr(sm + Cfg::SB + (n & 1) * Cfg::SB_BYTES);
-            named_barrier(kBarSReady, kSReadyThreads);   // SB_n is in shared memory
+            mbar_wait(SREADY, n & 1, abort_flag);
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)   // X += MP SB
@@ -862,7 +848,8 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             const float d = reinterpret_cast<const float *>(sm + Cfg::EGLR + sa * 512)[crow];
             fence_async_smem();
             tc_fence_before();
-            named_barrier_arrive(kBarSReady, kSReadyThreads);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(SREADY);
             if (n >= 1) store_o_m(n - 1);
             mbar_wait(SDONE, n & 1, abort_flag);
             tc_fence_after();
@@ -963,25 +950,23 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     const size_t rec0 = (size_t)p.chunk_off[seq];
 
     // mbarriers: FULLA[NSA], EMPTYA[NSA], FULLB[NSB], EMPTYB[NSB], FULLV[NSV], EMPTYV[NSV],
-    // FULLE[NSE], EMPTYE[NSE], SDONE, ODONE[2], FIN, OFREE[2]
+    // FULLE[NSE], EMPTYE[NSE], SDONE, ODONE[2], FIN, SREADY, OFREE[2]
     uint64_t *B = reinterpret_cast<uint64_t *>(sm + Cfg::BARS);
     uint64_t *FULLA = B, *EMPTYA = B + NSA, *FULLB = B + 2 * NSA, *EMPTYB = B + 2 * NSA + NSB;
     uint64_t *FULLV = B + 2 * NSA + 2 * NSB, *EMPTYV = FULLV + NSV;
     uint64_t *FULLE = EMPTYV + NSV, *EMPTYE = FULLE + NSE;
-    uint64_t *SDONE = EMPTYE + NSE, *ODONE = SDONE + 1, *FIN = SDONE + 3;
-    uint64_t *OFREE = SDONE + 4;
-    constexpr int kBars = 2 * NSA + 2 * NSB + 2 * NSV + 2 * NSE + 6;
+    uint64_t *SDONE = EMPTYE + NSE, *ODONE = SDONE + 1, *FIN = SDONE + 3, *SREADY = SDONE + 4;
+    uint64_t *OFREE = SDONE + 5;
+    constexpr int kBars = 2 * NSA + 2 * NSB + 2 * NSV + 2 * NSE + 7;
     static_assert(kBars * 8 <= 256, "barrier area");
-    // SB_n ready: the chain warps arrive on a named barrier, the product
-    // warp waits on it (a hardware barrier: no polling on the serial path)
-    constexpr uint32_t kBarSReady = 1, kSReadyThreads = 32 * (NCW + 1);
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + Cfg::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     if (tid == 0) {
         for (int i = 0; i < kBars; ++i) {
-            // EMPTYE and OFREE take one arrive per chain warp
+            // SREADY, EMPTYE and OFREE take one arrive per chain warp
             const uint64_t *b = &B[i];
-            const bool per_warp = b == &OFREE[0] || b == &OFREE[1] || (b >= EMPTYE && b < EMPTYE + NSE);
+            const bool per_warp = b == SREADY || b == &OFREE[0] || b == &OFREE[1] ||
+                                  (b >= EMPTYE && b < EMPTYE + NSE);
             mbar_init(&B[i], per_warp ? (uint32_t)NCW : 1u);
         }
         misc[1] = 0u;
@@ -1068,7 +1053,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         const uint32_t idOV = idesc_bf16(128, 64, true, false);    // A = V^T (MN-major), B = ZB^T
         // The state-independent products of chunk m: X[m mod 2] = V^T YT^T and
         // O[m mod 2] = V^T ZB^T.  X[m mod 2] was last read by the chain warps
-        // before their SB-ready arrival of chunk m - 1, which this warp has passed; O[m
+        // before their SREADY of chunk m - 1, which this warp has passed; O[m
         // mod 2] is free once they have read O_{m-2} out (OFREE).
         auto pre = [&](int m) {
             if (TRANS) return;
@@ -1100,7 +1085,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             const uint32_t bM = smem_addr(sm + Cfg::RA + sa * Cfg::A_STRIDE + Cfg::A_MP);
             const uint32_t aSB = tmem + Cfg::COL_SB + 64u * (uint32_t)(n & 1);
             if (TRANS) mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
-            named_barrier(kBarSReady, kSReadyThreads);   // SB_n is in TMEM
+            mbar_wait(SREADY, n & 1, abort_flag);
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)   // X += SB^T MP^T  (K = c')
@@ -1170,22 +1155,24 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             tmem_st16u(tmem_addr(tmem, 32 * quad, Cfg::COL_SB + 64 * (n & 1) + 16 * g), w16);
             tmem_wait_st();
             tc_fence_before();
-            named_barrier_arrive(kBarSReady, kSReadyThreads);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(SREADY);
             if (!TRANS && n >= 1) store_o_t(n - 1);
-            // S_{n+1} = S_n Diag(exp(G_L)) + X_n
+            // S_{n+1} = S_n Diag(exp(G_L)) + X_n, in two halves of 16 columns
             const int se = n % NSE;
             mbar_wait(&FULLE[se], (n / NSE) & 1, abort_flag);
             mbar_wait(SDONE, n & 1, abort_flag);
             tc_fence_after();
             const float4 *egl = reinterpret_cast<const float4 *>(sm + Cfg::EGLR + se * 512) + 8 * g;
-            {
-                float x[32];
-                tmem_ld32(tmem_addr(tmem, 32 * quad, Cfg::COL_X + 128 * (n & 1) + 32 * g), x);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float x[16];
+                tmem_ld16(tmem_addr(tmem, 32 * quad, Cfg::COL_X + 128 * (n & 1) + 32 * g + 16 * hh), x);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 d = egl[e4];
-                    float *s = S + 4 * e4;
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 d = egl[4 * hh + e4];
+                    float *s = S + 16 * hh + 4 * e4;
                     s[0] = fmaf(s[0], d.x, x[4 * e4 + 0]);
                     s[1] = fmaf(s[1], d.y, x[4 * e4 + 1]);
                     s[2] = fmaf(s[2], d.z, x[4 * e4 + 2]);

@@ -116,12 +116,6 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// Arrive on a named barrier without waiting (a producer's half of a
-// producer / consumer hand-off; the consumer waits with named_barrier).
-__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t threads) {
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
 // ---------------------------------------------------------------- TMEM
 
 // Whole warp: allocate `ncols` TMEM columns, base address written to *dst.
