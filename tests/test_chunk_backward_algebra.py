@@ -14,7 +14,10 @@ file's own code; the product has no such path yet).  What it fixes:
     dS = (Diag(e^{G_L}) + MP^T) dS_next + QP^T dO with MP = -Kbar^T W and
     QP = Qtil - P W, the forward's own chunk operands;
   * the chunk-local gradients (through the triangular inverse, both masks,
-    the four gated operands and the running sum) equal the oracle's.
+    the four gated operands and the running sum) equal the oracle's;
+  * the staged form (a forward scan for each chunk's entering state, a
+    reverse scan for dL/dS at each chunk's end, then each chunk's own
+    token-by-token derivative) reproduces the whole sequence's gradients.
 """
 import numpy as np
 import pytest
@@ -130,4 +133,49 @@ def test_chunk_backward_matches_oracle(oracle_mod, C):
                                   d_final_state=d_sT[None, None])
     for name, x, r in zip(("dq", "dk", "dv", "dg", "dbeta"), grads, ref[:5]):
         np.testing.assert_allclose(x, r[:, 0], rtol=1e-8, atol=1e-10, err_msg=name)
+    np.testing.assert_allclose(dS, ref[5][0, 0], rtol=1e-8, atol=1e-10)
+
+
+def test_staged_backward_reproduces_the_oracle(oracle_mod):
+    """The staged form: the forward scan over the chunk operands gives each
+    chunk's entering state, the reverse scan dL/dS at each chunk's end; the
+    token-by-token derivative of each chunk alone, from those two, then equals
+    the whole sequence's (the oracle's backward run per chunk as a sequence of
+    its own with init_state = S_in and d_final_state = dS_next)."""
+    rng = np.random.default_rng(23)
+    T, dk, dv, C = 200, 8, 6, 64
+    q, k, v, g, beta, s0 = _case(rng, T, dk, dv)
+    d_o = rng.normal(size=(T, dv))
+    d_sT = rng.normal(size=(dk, dv))
+    bounds = [(t0, min(t0 + C, T)) for t0 in range(0, T, C)]
+    ops, S_in = [], []
+    S = s0.copy()
+    for t0, t1 in bounds:   # forward scan: S <- Diag(e^GL) S + MP S + YT V
+        c = _chunk(q[t0:t1], k[t0:t1], v[t0:t1], g[t0:t1], beta[t0:t1], S)
+        Tb = c["Tm"] * beta[t0:t1][None, :]
+        MP, YT = -c["Kb"].T @ c["W"], c["Kb"].T @ Tb
+        QP = c["Qt"] - c["P"] @ c["W"]
+        ops.append((np.exp(c["GL"]), MP, YT, QP))
+        S_in.append(S.copy())
+        S = ops[-1][0][:, None] * S + MP @ S + YT @ v[t0:t1]
+    dS_next = [None] * len(bounds)
+    dS = d_sT.copy()
+    for i in reversed(range(len(bounds))):   # reverse scan
+        t0, t1 = bounds[i]
+        egl, MP, _, QP = ops[i]
+        dS_next[i] = dS.copy()
+        dS = egl[:, None] * dS + MP.T @ dS + QP.T @ d_o[t0:t1]
+    ref = oracle_mod.kda_backward(q[:, None], k[:, None], v[:, None], g[:, None], beta[:, None],
+                                  d_o[:, None], init_state=s0[None, None],
+                                  d_final_state=d_sT[None, None])
+    for i, (t0, t1) in enumerate(bounds):
+        sl = slice(t0, t1)
+        part = oracle_mod.kda_backward(q[sl, None], k[sl, None], v[sl, None], g[sl, None],
+                                       beta[sl, None], d_o[sl, None],
+                                       init_state=S_in[i][None, None],
+                                       d_final_state=dS_next[i][None, None])
+        for name, x, r in zip(("dq", "dk", "dv", "dg", "dbeta"), part[:5], ref[:5]):
+            np.testing.assert_allclose(x, r[sl], rtol=1e-8, atol=1e-10, err_msg=f"{name} chunk {i}")
+        if i == 0:
+            np.testing.assert_allclose(part[5], ref[5], rtol=1e-8, atol=1e-10)
     np.testing.assert_allclose(dS, ref[5][0, 0], rtol=1e-8, atol=1e-10)
