@@ -286,15 +286,20 @@ def time_backward(w, steps, warmup, world):
     T, H, dk = q.shape
     dv = v.shape[-1]
     n = len(inp["lengths"])
-    ws = torch.empty(max(256, kda.kda_backward_workspace_size(n, T, H, dk, dv)),
-                     dtype=torch.uint8, device="cuda")
+    # bf16 with d = 128: the chunked backward (plan, preparation, two scans,
+    # chunk steps: five kernels); otherwise the sequential one (one kernel)
+    chunked = w.dtype == "bf16" and dk == 128 and dv == 128
+    fn = kda.kda_backward_chunked if chunked else kda.kda_backward
+    need = (kda.kda_backward_chunked_workspace_size(n, T, H) if chunked
+            else kda.kda_backward_workspace_size(n, T, H, dk, dv))
+    ws = torch.empty(max(256, need), dtype=torch.uint8, device="cuda")
     flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step():
-        kda.kda_backward(q, k, v, g, b, ct["d_o"], init_state=inp["init_state"],
-                         d_final_state=ct["d_final_state"], cu_seqlens=inp["cu_seqlens"],
-                         workspace=ws, stream=stream)
+        fn(q, k, v, g, b, ct["d_o"], init_state=inp["init_state"],
+           d_final_state=ct["d_final_state"], cu_seqlens=inp["cu_seqlens"],
+           workspace=ws, stream=stream)
 
     for _ in range(warmup):
         flush.fill_(1)
@@ -314,8 +319,9 @@ def time_backward(w, steps, warmup, world):
     if kda.kda_check_workspace_error(ws) != kda.KDA_OK:
         raise RuntimeError("device-side check failed during the backward benchmark")
     ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    # one kernel per call (the gradient zeroing is four memsets)
-    return dict(ms_total=sum(ms), ms=ms, lengths=inp["lengths"], launches=steps)
+    # the gradient zeroing is four memsets, not counted
+    return dict(ms_total=sum(ms), ms=ms, lengths=inp["lengths"],
+                launches=steps * (5 if chunked else 1))
 
 
 def time_prefill_e2e(w, steps, warmup):

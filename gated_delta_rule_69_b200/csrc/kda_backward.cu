@@ -248,10 +248,110 @@ __device__ __forceinline__ void flush_group(const float *red, int count, int64_t
     }
 }
 
+// One block of steps [tb, te) backwards, from dS = dL/dS_te: the block run
+// forward again from its entering state S (overwritten) into the scratch,
+// then the backward steps; the row partials are flushed every kBwdGroup
+// steps and at t == t_stop (the first step of the unit).
+template <typename T, int DK>
+__device__ __forceinline__ void block_backward(float4 (&S)[DK / 32], float4 (&dS)[DK / 32],
+                                               const BwdArgs &p, int64_t tb, int64_t te,
+                                               int64_t t_stop, int h, int warp, int lane, int j0,
+                                               int idx, float4 *scratch, float *red, int &buf,
+                                               int &gi, int64_t &g_hi) {
+    using Sh = BwdShape<DK>;
+    constexpr int RPL = Sh::RPL, E = Sh::E, S4 = Sh::STATE4;
+    forward_run<T, DK>(S, p, tb, te, h, lane, j0, scratch, idx);
+
+    // Lane 0 wrote each step's r; the warp's lanes read it below.
+    __syncwarp();
+    // Backward over the block, the next step's inputs and record
+    // loaded one step ahead.
+    constexpr int R4 = scratch_step4<DK>();
+    StepRaw<T, RPL> nxt;
+    float4 Sn[RPL], rn;
+    load_step<T, DK, true>(nxt, p, te - 1, h, lane, j0);
+    {
+        const float4 *rec = scratch + (size_t)(te - 1 - tb) * R4;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) Sn[i] = rec[idx + i * kBwdThreads];
+        rn = rec[S4 + warp];
+    }
+#pragma unroll 1
+    for (int64_t t = te - 1; t >= tb; --t) {
+        StepIn<RPL> cur;
+        decode_step<T, RPL, true>(cur, nxt, p.scalar_gate);
+        float4 sp[RPL];
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) sp[i] = Sn[i];
+        const float4 r = rn;
+        if (t - 1 >= tb) {
+            load_step<T, DK, true>(nxt, p, t - 1, h, lane, j0);
+            const float4 *rec = scratch + (size_t)(t - 1 - tb) * R4;
+#pragma unroll
+            for (int i = 0; i < RPL; ++i) Sn[i] = rec[idx + i * kBwdThreads];
+            rn = rec[S4 + warp];
+        }
+        // Sp = Diag(a) S_{t-1}; r and u as the forward had them
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) sp[i] = mul4(sp[i], cur.a[i]);
+        const float4 vr = sub4(cur.v, r);
+        const float4 uu = mul4(vr, cur.b);
+        // o_t = S_t^T q, S_t = Sp + k u^T
+        float dq_r[RPL], dk_r[RPL], dg_r[RPL];
+        float4 dup = f4(0.f);
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            dS[i] = fma4s(cur.d, cur.q[i], dS[i]);
+            dq_r[i] = dot4(fma4s(uu, cur.k[i], sp[i]), cur.d);
+            dup = fma4s(dS[i], cur.k[i], dup);
+            dk_r[i] = dot4(dS[i], uu);
+        }
+        const float4 du = warp_sum4(dup);
+        const float dbeta = dot4(du, vr);
+        const size_t row = (size_t)t * p.H + h;
+        if (lane == 0)
+            *reinterpret_cast<float4 *>(p.dv + row * p.dv_total + j0) = mul4(du, cur.b);
+        const float4 dr = mul4(du, -cur.b);
+        float gsum = 0.f;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            dS[i] = fma4s(dr, cur.k[i], dS[i]);
+            dk_r[i] += dot4(sp[i], dr);
+            dg_r[i] = dot4(sp[i], dS[i]);
+            gsum += dg_r[i];
+            dS[i] = mul4(dS[i], cur.a[i]);
+        }
+        // this warp's row partials of the step
+        float *slot = red + ((size_t)(buf * kBwdGroup + gi) * kBwdWarps + warp) * E;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            slot[lane + 32 * i] = dq_r[i];
+            slot[DK + lane + 32 * i] = dk_r[i];
+            slot[2 * DK + lane + 32 * i] = dg_r[i];
+        }
+        if (p.scalar_gate) gsum = warp_sum(gsum);
+        if (lane == 0) {
+            slot[3 * DK] = dbeta;
+            slot[3 * DK + 1] = gsum;
+        }
+        if (gi == 0) g_hi = t;
+        ++gi;
+        if (gi == kBwdGroup || t == t_stop) {
+            // One barrier per group: the two buffers alternate, and a
+            // buffer is written again only after the next group's
+            // barrier, which every thread reaches after this flush.
+            __syncthreads();
+            flush_group<DK>(red + (size_t)buf * kBwdGroup * kBwdWarps * E, gi, g_hi, h, p);
+            buf ^= 1;
+            gi = 0;
+        }
+    }
+}
+
 template <typename T, int DK>
 __global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_kernel(const BwdArgs p) {
     using Sh = BwdShape<DK>;
-    constexpr int RPL = Sh::RPL, E = Sh::E, S4 = Sh::STATE4;
+    constexpr int RPL = Sh::RPL, S4 = Sh::STATE4;
     extern __shared__ float red[];   // [2][kBwdGroup][kBwdWarps][E]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // a thread's float4 i of a state slice: key row lane + 32 i, its warp's columns
@@ -315,92 +415,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_kernel(const BwdA
             const float4 *ck = p.ckpt + (((size_t)(slot0 + b) * p.H + h) * p.nslices + s) * S4;
 #pragma unroll
             for (int i = 0; i < RPL; ++i) S[i] = ck[idx + i * kBwdThreads];
-            forward_run<T, DK>(S, p, tb, te, h, lane, j0, scratch, idx);
-
-            // Lane 0 wrote each step's r; the warp's lanes read it below.
-            __syncwarp();
-            // Backward over the block, the next step's inputs and record
-            // loaded one step ahead.
-            constexpr int R4 = scratch_step4<DK>();
-            StepRaw<T, RPL> nxt;
-            float4 Sn[RPL], rn;
-            load_step<T, DK, true>(nxt, p, te - 1, h, lane, j0);
-            {
-                const float4 *rec = scratch + (size_t)(te - 1 - tb) * R4;
-#pragma unroll
-                for (int i = 0; i < RPL; ++i) Sn[i] = rec[idx + i * kBwdThreads];
-                rn = rec[S4 + warp];
-            }
-#pragma unroll 1
-            for (int64_t t = te - 1; t >= tb; --t) {
-                StepIn<RPL> cur;
-                decode_step<T, RPL, true>(cur, nxt, p.scalar_gate);
-                float4 sp[RPL];
-#pragma unroll
-                for (int i = 0; i < RPL; ++i) sp[i] = Sn[i];
-                const float4 r = rn;
-                if (t - 1 >= tb) {
-                    load_step<T, DK, true>(nxt, p, t - 1, h, lane, j0);
-                    const float4 *rec = scratch + (size_t)(t - 1 - tb) * R4;
-#pragma unroll
-                    for (int i = 0; i < RPL; ++i) Sn[i] = rec[idx + i * kBwdThreads];
-                    rn = rec[S4 + warp];
-                }
-                // Sp = Diag(a) S_{t-1}; r and u as the forward had them
-#pragma unroll
-                for (int i = 0; i < RPL; ++i) sp[i] = mul4(sp[i], cur.a[i]);
-                const float4 vr = sub4(cur.v, r);
-                const float4 uu = mul4(vr, cur.b);
-                // o_t = S_t^T q, S_t = Sp + k u^T
-                float dq_r[RPL], dk_r[RPL], dg_r[RPL];
-                float4 dup = f4(0.f);
-#pragma unroll
-                for (int i = 0; i < RPL; ++i) {
-                    dS[i] = fma4s(cur.d, cur.q[i], dS[i]);
-                    dq_r[i] = dot4(fma4s(uu, cur.k[i], sp[i]), cur.d);
-                    dup = fma4s(dS[i], cur.k[i], dup);
-                    dk_r[i] = dot4(dS[i], uu);
-                }
-                const float4 du = warp_sum4(dup);
-                const float dbeta = dot4(du, vr);
-                const size_t row = (size_t)t * p.H + h;
-                if (lane == 0)
-                    *reinterpret_cast<float4 *>(p.dv + row * p.dv_total + j0) = mul4(du, cur.b);
-                const float4 dr = mul4(du, -cur.b);
-                float gsum = 0.f;
-#pragma unroll
-                for (int i = 0; i < RPL; ++i) {
-                    dS[i] = fma4s(dr, cur.k[i], dS[i]);
-                    dk_r[i] += dot4(sp[i], dr);
-                    dg_r[i] = dot4(sp[i], dS[i]);
-                    gsum += dg_r[i];
-                    dS[i] = mul4(dS[i], cur.a[i]);
-                }
-                // this warp's row partials of the step
-                float *slot = red + ((size_t)(buf * kBwdGroup + gi) * kBwdWarps + warp) * E;
-#pragma unroll
-                for (int i = 0; i < RPL; ++i) {
-                    slot[lane + 32 * i] = dq_r[i];
-                    slot[DK + lane + 32 * i] = dk_r[i];
-                    slot[2 * DK + lane + 32 * i] = dg_r[i];
-                }
-                if (p.scalar_gate) gsum = warp_sum(gsum);
-                if (lane == 0) {
-                    slot[3 * DK] = dbeta;
-                    slot[3 * DK + 1] = gsum;
-                }
-                if (gi == 0) g_hi = t;
-                ++gi;
-                if (gi == kBwdGroup || t == bos) {
-                    // One barrier per group: the two buffers alternate, and a
-                    // buffer is written again only after the next group's
-                    // barrier, which every thread reaches after this flush.
-                    __syncthreads();
-                    flush_group<DK>(red + (size_t)buf * kBwdGroup * kBwdWarps * E, gi, g_hi, h, p);
-                    buf ^= 1;
-                    gi = 0;
-                }
-            }
+            block_backward<T, DK>(S, dS, p, tb, te, bos, h, warp, lane, j0, idx, scratch, red, buf,
+                                  gi, g_hi);
         }
         if (p.d_init_state) {
 #pragma unroll
@@ -417,6 +433,179 @@ cudaError_t launch_dk(const BwdArgs &p, int grid, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     kda_backward_kernel<T, DK><<<grid, kBwdThreads, smem, stream>>>(p);
     return cudaGetLastError();
+}
+
+// ---- chunk-parallel variant (bf16, d = 128): the chunk records of the
+// prefill's preparation give every chunk's entering state (a forward scan,
+// S <- Diag(e^{G_L}) S + MP S + YT V) and every chunk's dL/dS_next (a
+// reverse scan, dS <- Diag(e^{G_L}) dS + MP^T dS + QP^T dO: the transpose of
+// the forward transition); the chunks' steps then run independently.
+
+constexpr int kScanThreads = 256;
+struct ScanSmem {
+    static constexpr uint32_t A = 0;         // MP, 128 x 128 bf16 (two 16 KB K-atoms)
+    static constexpr uint32_t B = 32768;     // YT [128][64] or QP [64][128] bf16, 16 KB
+    static constexpr uint32_t X = 49152;     // v or dO slice [64][32] fp32
+    static constexpr uint32_t S = 57344;     // state slice [128][32] fp32
+    static constexpr uint32_t EGL = 73728;   // 128 fp32
+    static constexpr uint32_t SIZE = 74240;
+};
+
+// Byte offset of bf16 element (row, col) of a K-major tile with 128-byte rows
+// of 64 columns, the 16-byte chunk index XORed with (row mod 8); `atom` bytes
+// per 64-column atom.
+__device__ __forceinline__ uint32_t rec_off(uint32_t row, uint32_t col, uint32_t atom) {
+    const uint32_t c = col & 63u;
+    return (col >> 6) * atom + row * 128u + (((c >> 3) ^ (row & 7u)) << 4) + (c & 7u) * 2u;
+}
+
+__device__ __forceinline__ float bf_at(const uint8_t *tile, uint32_t off) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + off));
+}
+
+struct ScanArgs {
+    SplitTables tab;
+    const __nv_bfloat16 *x;   // v (forward scan) or dO (reverse scan), [T, H, 128]
+    const float *s0;          // init_state (forward) or dL/dS_T (reverse), or null
+    float *out;               // [max_chunks, H, 128, 128]: each chunk's entering value
+    float *last;              // reverse: dL/dS_0 per sequence (overwritten later for
+                              // non-empty sequences), or null
+    int H;
+};
+
+// One CTA per (sequence, head, 32-column slice); 256 threads, each 4 key rows
+// x 4 columns of the slice.
+template <bool REV>
+__global__ void __launch_bounds__(kScanThreads) kda_bwd_scan_kernel(const ScanArgs a) {
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const uint8_t *A = sm + ScanSmem::A, *B = sm + ScanSmem::B;
+    float *xs = reinterpret_cast<float *>(sm + ScanSmem::X);
+    float *ss = reinterpret_cast<float *>(sm + ScanSmem::S);
+    float *egl = reinterpret_cast<float *>(sm + ScanSmem::EGL);
+    const int tid = threadIdx.x;
+    const int sl = blockIdx.x & 3, h = (blockIdx.x >> 2) % a.H, n = (blockIdx.x >> 2) / a.H;
+    const int r0 = 4 * (tid >> 3), c0 = 4 * (tid & 7);   // rows r0..r0+3, slice columns c0..c0+3
+    const size_t st = ((size_t)n * a.H + h) * 128 * 128 + (size_t)sl * 32;
+    for (int i = tid; i < 128 * 32; i += kScanThreads)
+        ss[i] = a.s0 ? a.s0[st + (size_t)(i >> 5) * 128 + (i & 31)] : 0.f;
+    const int cb = a.tab.chunk_off[n], ce = a.tab.chunk_off[n + 1];
+#pragma unroll 1
+    for (int it = 0; it < ce - cb; ++it) {
+        const int c = REV ? ce - 1 - it : cb + it;
+        const int2 ct = a.tab.chunk_tab[c];
+        const uint8_t *rec = a.tab.recs + ((size_t)c * a.H + h) * a.tab.rec_stride;
+        __syncthreads();   // the previous chunk's reads and writes of shared memory are done
+        const size_t ob = ((size_t)c * a.H + h) * 128 * 128 + (size_t)sl * 32;
+        for (int i = tid; i < 128 * 32; i += kScanThreads)
+            a.out[ob + (size_t)(i >> 5) * 128 + (i & 31)] = ss[i];
+        for (int i = tid; i < 2048; i += kScanThreads)
+            reinterpret_cast<uint4 *>(sm + ScanSmem::A)[i] =
+                reinterpret_cast<const uint4 *>(rec + a.tab.off_mp)[i];
+        for (int i = tid; i < 1024; i += kScanThreads)
+            reinterpret_cast<uint4 *>(sm + ScanSmem::B)[i] =
+                reinterpret_cast<const uint4 *>(rec + (REV ? a.tab.off_qp : a.tab.off_yt))[i];
+        if (tid < 128) egl[tid] = reinterpret_cast<const float *>(rec + a.tab.off_egl)[tid];
+        for (int i = tid; i < 64 * 32; i += kScanThreads) {
+            const int t = i >> 5;
+            xs[i] = t < ct.y ? __bfloat162float(a.x[((size_t)(ct.x + t) * a.H + h) * 128 + sl * 32 + (i & 31)])
+                             : 0.f;
+        }
+        __syncthreads();
+        float acc[4][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[r][q] = egl[r0 + r] * ss[(r0 + r) * 32 + c0 + q];
+#pragma unroll 4
+        for (int k = 0; k < 128; ++k) {   // (MP S) or (MP^T dS)
+            const float4 sk = *reinterpret_cast<const float4 *>(ss + k * 32 + c0);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const float m = REV ? bf_at(A, rec_off(k, r0 + r, 16384)) : bf_at(A, rec_off(r0 + r, k, 16384));
+                acc[r][0] = fmaf(m, sk.x, acc[r][0]);
+                acc[r][1] = fmaf(m, sk.y, acc[r][1]);
+                acc[r][2] = fmaf(m, sk.z, acc[r][2]);
+                acc[r][3] = fmaf(m, sk.w, acc[r][3]);
+            }
+        }
+#pragma unroll 4
+        for (int t = 0; t < 64; ++t) {   // (YT V) or (QP^T dO)
+            const float4 xt = *reinterpret_cast<const float4 *>(xs + t * 32 + c0);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const float y = REV ? bf_at(B, rec_off(t, r0 + r, 8192)) : bf_at(B, rec_off(r0 + r, t, 16384));
+                acc[r][0] = fmaf(y, xt.x, acc[r][0]);
+                acc[r][1] = fmaf(y, xt.y, acc[r][1]);
+                acc[r][2] = fmaf(y, xt.z, acc[r][2]);
+                acc[r][3] = fmaf(y, xt.w, acc[r][3]);
+            }
+        }
+        __syncthreads();   // every read of the old slice is done
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            *reinterpret_cast<float4 *>(ss + (r0 + r) * 32 + c0) =
+                make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+    }
+    if (REV && a.last) {
+        __syncthreads();
+        for (int i = tid; i < 128 * 32; i += kScanThreads)
+            a.last[st + (size_t)(i >> 5) * 128 + (i & 31)] = ss[i];
+    }
+}
+
+struct ChunkArgs {
+    SplitTables tab;
+    const float *s_in;     // [max_chunks, H, 128, 128] entering states
+    const float *ds_next;  // [max_chunks, H, 128, 128] dL/dS at each chunk's end
+    int num_seqs;
+};
+
+// One unit per (chunk, head, slice): the block_backward of the chunk from its
+// entering state and dL/dS_next; a sequence's first chunk writes dL/dS_0.
+template <typename T, int DK>
+__global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_chunk_kernel(const BwdArgs p,
+                                                                          const ChunkArgs c) {
+    using Sh = BwdShape<DK>;
+    constexpr int RPL = Sh::RPL;
+    extern __shared__ float red[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int idx = warp * 32 + lane;
+    float4 *scratch = p.scratch + (size_t)blockIdx.x * kBwdBlock * scratch_step4<DK>();
+    int buf = 0, gi = 0;
+    int64_t g_hi = 0;
+    const int units = (int)*c.tab.total_chunks * p.H * p.nslices;
+#pragma unroll 1
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        const int s = u % p.nslices;
+        const int h = (u / p.nslices) % p.H;
+        const int ch = u / (p.nslices * p.H);
+        const int2 ct = c.tab.chunk_tab[ch];
+        const int64_t tb = ct.x, te = (int64_t)ct.x + ct.y;
+        const int j0 = s * kBwdSlice + warp * kBwdCols;
+        const size_t base = ((size_t)ch * p.H + h) * DK * p.dv_total + j0;
+        float4 S[RPL], dS[RPL];
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            S[i] = *reinterpret_cast<const float4 *>(c.s_in + base + (size_t)(lane + 32 * i) * p.dv_total);
+            dS[i] = *reinterpret_cast<const float4 *>(c.ds_next + base + (size_t)(lane + 32 * i) * p.dv_total);
+        }
+        block_backward<T, DK>(S, dS, p, tb, te, tb, h, warp, lane, j0, idx, scratch, red, buf, gi,
+                              g_hi);
+        if (p.d_init_state) {
+            int lo = 0, hi = c.num_seqs;   // the last sequence whose first chunk is <= ch
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (c.tab.chunk_off[mid] <= ch) lo = mid;
+                else hi = mid;
+            }
+            if (c.tab.chunk_off[lo] == ch) {
+                const size_t st = ((size_t)lo * p.H + h) * DK * p.dv_total + j0;
+#pragma unroll
+                for (int i = 0; i < RPL; ++i)
+                    *reinterpret_cast<float4 *>(p.d_init_state + st + (size_t)(lane + 32 * i) * p.dv_total) = dS[i];
+            }
+        }
+    }
 }
 
 size_t bwd_slots(int num_seqs, int64_t total_tokens) {
@@ -484,6 +673,102 @@ cudaError_t launch_backward(const void *q, const void *k, const void *v, const v
         case 128: return bf ? launch_dk<__nv_bfloat16, 128>(p, grid, stream) : launch_dk<float, 128>(p, grid, stream);
         default: return cudaErrorInvalidValue;
     }
+}
+
+namespace {
+
+struct ChunkedLayout {
+    size_t split, s_in, ds_next, scratch, total;
+    size_t max_chunks;
+    int grid;
+};
+
+ChunkedLayout chunked_layout(int num_seqs, int64_t total_tokens, int H) {
+    ChunkedLayout l;
+    l.max_chunks = (size_t)(total_tokens / kBwdBlock) + (size_t)num_seqs;
+    const size_t state = (size_t)128 * 128 * sizeof(float);
+    const int64_t units = (int64_t)l.max_chunks * H * (128 / kBwdSlice);
+    l.grid = (int)(units < kBwdMaxCtas ? units : kBwdMaxCtas);
+    l.split = 0;
+    l.s_in = (prefill_split_workspace(num_seqs, total_tokens, H) + 1023) & ~(size_t)1023;
+    l.ds_next = l.s_in + l.max_chunks * H * state;
+    l.scratch = l.ds_next + l.max_chunks * H * state;
+    l.total = l.scratch + (size_t)l.grid * kBwdBlock * scratch_step4<128>() * sizeof(float4);
+    return l;
+}
+
+}  // namespace
+
+size_t backward_chunked_workspace(int num_seqs, int64_t total_tokens, int H) {
+    return chunked_layout(num_seqs, total_tokens, H).total;
+}
+
+cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v, const void *g,
+                                    const void *beta, const float *init_state, const int32_t *cu,
+                                    int num_seqs, int64_t total_tokens, int H, const void *d_o,
+                                    const float *d_final_state, float *dq, float *dk_out,
+                                    float *dv_out, float *dg, float *dbeta, float *d_init_state,
+                                    void *workspace, bool scalar_gate, cudaStream_t stream) {
+    const ChunkedLayout l = chunked_layout(num_seqs, total_tokens, H);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const size_t nk = (size_t)total_tokens * H * 128;
+    const size_t ng = scalar_gate ? (size_t)total_tokens * H : nk;
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(dq, 0, nk * sizeof(float), stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dk_out, 0, nk * sizeof(float), stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dg, 0, ng * sizeof(float), stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dbeta, 0, (size_t)total_tokens * H * sizeof(float), stream)) != cudaSuccess)
+        return e;
+    // 1. the plan and the chunk records (the prefill's preparation, no chain)
+    e = launch_prefill_split(q, k, v, g, beta, nullptr, cu, num_seqs, total_tokens, H, nullptr,
+                             nullptr, ws + l.split, scalar_gate, nullptr, stream, kPrepOnly);
+    if (e != cudaSuccess) return e;
+    const SplitTables tab = split_tables(ws + l.split, num_seqs, total_tokens, H);
+    // 2. the scans: entering states, then dL/dS_next (and a first dL/dS_0)
+    if ((e = set_max_dynamic_smem((const void *)kda_bwd_scan_kernel<false>, (int)ScanSmem::SIZE)) != cudaSuccess)
+        return e;
+    if ((e = set_max_dynamic_smem((const void *)kda_bwd_scan_kernel<true>, (int)ScanSmem::SIZE)) != cudaSuccess)
+        return e;
+    const unsigned scan_grid = (unsigned)((size_t)num_seqs * H * 4);
+    ScanArgs fa;
+    fa.tab = tab;
+    fa.x = static_cast<const __nv_bfloat16 *>(v);
+    fa.s0 = init_state;
+    fa.out = reinterpret_cast<float *>(ws + l.s_in);
+    fa.last = nullptr;
+    fa.H = H;
+    kda_bwd_scan_kernel<false><<<scan_grid, kScanThreads, ScanSmem::SIZE, stream>>>(fa);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ScanArgs ra = fa;
+    ra.x = static_cast<const __nv_bfloat16 *>(d_o);
+    ra.s0 = d_final_state;
+    ra.out = reinterpret_cast<float *>(ws + l.ds_next);
+    ra.last = d_init_state;
+    kda_bwd_scan_kernel<true><<<scan_grid, kScanThreads, ScanSmem::SIZE, stream>>>(ra);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 3. the chunks' steps, all chunks at once
+    BwdArgs p = {};
+    p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.d_o = d_o;
+    p.dq = dq; p.dk = dk_out; p.dv = dv_out; p.dg = dg; p.dbeta = dbeta;
+    p.d_init_state = d_init_state;
+    p.scratch = reinterpret_cast<float4 *>(ws + l.scratch);
+    p.err_word = reinterpret_cast<uint32_t *>(ws);
+    p.total_tokens = total_tokens;
+    p.H = H;
+    p.dv_total = 128;
+    p.nslices = 128 / kBwdSlice;
+    p.scalar_gate = scalar_gate ? 1 : 0;
+    ChunkArgs ca;
+    ca.tab = tab;
+    ca.s_in = reinterpret_cast<const float *>(ws + l.s_in);
+    ca.ds_next = reinterpret_cast<const float *>(ws + l.ds_next);
+    ca.num_seqs = num_seqs;
+    const size_t smem = BwdShape<128>::SMEM;
+    if ((e = set_max_dynamic_smem((const void *)kda_backward_chunk_kernel<__nv_bfloat16, 128>, (int)smem)) !=
+        cudaSuccess)
+        return e;
+    kda_backward_chunk_kernel<__nv_bfloat16, 128><<<l.grid, kBwdThreads, smem, stream>>>(p, ca);
+    return cudaGetLastError();
 }
 
 }  // namespace kda

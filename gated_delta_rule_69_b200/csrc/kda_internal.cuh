@@ -112,7 +112,9 @@ size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H);
 // (final_state then receives the state generated from init_state, o is
 // scratch); kCpFinish runs only the chain over the records a kCpLocal call
 // left in the same workspace.
-enum : int { kCpNone = 0, kCpLocal = 1, kCpFinish = 2 };
+// kPrepOnly: the plan and the chunk records only (no chain), for the
+// backward pass's scans over the records.
+enum : int { kCpNone = 0, kCpLocal = 1, kCpFinish = 2, kPrepOnly = 3 };
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const void *g,
                                  const void *beta, const float *init_state, const int32_t *cu,
                                  int num_seqs, int64_t total_tokens, int H, void *o,
@@ -132,6 +134,31 @@ cudaError_t launch_backward(const void *q, const void *k, const void *v, const v
                             float *dq, float *dk_out, float *dv_out, float *dg, float *dbeta,
                             float *d_init_state, void *workspace, bool scalar_gate,
                             cudaStream_t stream);
+
+// Backward pass through the chunk records (bf16, d_k = d_v = 128): the
+// prefill's preparation, a forward and a reverse scan over the records for
+// each chunk's entering state and dL/dS_next, then every chunk's steps at once.
+size_t backward_chunked_workspace(int num_seqs, int64_t total_tokens, int H);
+cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v, const void *g,
+                                    const void *beta, const float *init_state, const int32_t *cu,
+                                    int num_seqs, int64_t total_tokens, int H, const void *d_o,
+                                    const float *d_final_state, float *dq, float *dk_out,
+                                    float *dv_out, float *dg, float *dbeta, float *d_init_state,
+                                    void *workspace, bool scalar_gate, cudaStream_t stream);
+
+// Where a split-path workspace keeps the plan's tables and the records.
+struct SplitTables {
+    const int32_t *chunk_off;    // [N + 1] first chunk of each sequence
+    const int2 *chunk_tab;       // [chunks] (first token, length)
+    const uint32_t *total_chunks;
+    const uint8_t *recs;         // record (chunk, head) at recs + (chunk * H + head) * rec_stride
+    size_t rec_stride;
+    size_t max_chunks;
+    // record field offsets: MP [128][128], YT [128][64], QP [64][128] bf16
+    // (K-major, 128-byte swizzle, 64-column atoms), e^{G_L} 128 fp32
+    uint32_t off_mp, off_yt, off_qp, off_egl;
+};
+SplitTables split_tables(const void *workspace, int num_seqs, int64_t total_tokens, int H);
 
 // Context parallelism: S_out = the state a segment starts from, given the
 // (M_i, S~_i) of the n_prev segments before it and the sequence's S_0 (or null).

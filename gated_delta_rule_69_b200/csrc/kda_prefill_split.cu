@@ -1524,6 +1524,23 @@ size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H) {
     return split_layout(num_seqs, total_tokens, H).total;
 }
 
+SplitTables split_tables(const void *workspace, int num_seqs, int64_t total_tokens, int H) {
+    const SplitLayout l = split_layout(num_seqs, total_tokens, H);
+    const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+    SplitTables t;
+    t.chunk_off = reinterpret_cast<const int32_t *>(ws + l.chunk_off);
+    t.chunk_tab = reinterpret_cast<const int2 *>(ws + l.chunk_tab);
+    t.total_chunks = reinterpret_cast<const uint32_t *>(ws + 4);
+    t.recs = ws + l.recs;
+    t.rec_stride = split::Rec::STRIDE;
+    t.max_chunks = l.max_chunks;
+    t.off_mp = split::Rec::MP;
+    t.off_yt = split::Rec::YT;
+    t.off_qp = split::Rec::QP;
+    t.off_egl = split::Rec::EGL;
+    return t;
+}
+
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const void *g,
                                  const void *beta, const float *init_state, const int32_t *cu,
                                  int num_seqs, int64_t total_tokens, int H, void *o,
@@ -1577,7 +1594,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     // a segment's transition is d_k x d_k: whole-d_v chain CTAs only
     const ChainPlan plan = choose_chain(units, (uint64_t)(total_tokens / C + num_seqs) * H, total_tokens,
                                         num_seqs, (unsigned)sm_count, cp_mode == kCpLocal);
-    const bool overlap = plan.overlap;
+    const bool overlap = plan.overlap && cp_mode != kPrepOnly;
     const unsigned chain_blocks = units * (unsigned)(DV / plan.dvt);
     uint32_t *rec_ready = overlap ? reinterpret_cast<uint32_t *>(ws + l.flags) : nullptr;
     kda_split_plan_kernel<<<1, kPlanThreads, 0, stream>>>(cu, num_seqs, total_tokens, perm,
@@ -1637,6 +1654,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    if (cp_mode == kPrepOnly) return cudaSuccess;
     if (cp_mode == kCpLocal) {
         // the locally generated state (from zero), then over the same records
         // the segment's transition (from the identity, v counting as zero)

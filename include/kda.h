@@ -322,6 +322,27 @@ kda_status gdn_backward(const void *q, const void *k, const void *v, const void 
                         size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * kda_backward for bf16 inputs with d_k = d_v = 128 by chunks: the prefill's
+ * chunk preparation, a forward and a reverse scan over its per-chunk
+ * transition operands for every chunk's entering state and dL/dS at its end,
+ * then every chunk's steps at once.  Same arguments and outputs as
+ * kda_backward (bf16, d = 128 implied); the workspace (256-byte aligned,
+ * kda_backward_chunked_workspace_size bytes) also holds the prefill's records
+ * and two states per (chunk, head).  The chunk boundary states carry the
+ * records' bf16 rounding: gradients agree with kda_backward to the bf16
+ * tolerance, not to fp32 rounding.
+ */
+size_t kda_backward_chunked_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H);
+
+kda_status kda_backward_chunked(const void *q, const void *k, const void *v, const void *log_alpha,
+                                const void *beta, const float *init_state,
+                                const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                                int32_t H, const void *d_o, const float *d_final_state, float *dq,
+                                float *dk, float *dv, float *dlog_alpha, float *dbeta,
+                                float *d_init_state, void *workspace, size_t workspace_bytes,
+                                kda_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads the error word that the prefill and
  * backward kernels leave at the start of `workspace` (non-zero when a
  * device-side check failed, e.g. cu_seqlens not non-decreasing or not ending
