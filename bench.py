@@ -205,7 +205,7 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # --- the GPU arm -------------------------------------------------------------------
 
-def time_prefill(w, steps, warmup, world, scalar_gate=False, layer=False):
+def time_prefill(w, steps, warmup, world, scalar_gate=False, layer=False, profile_range=False):
     """kda_prefill (or, with ``scalar_gate``, gdn_prefill with channel 0 of
     the gate draw as the per-head gate; with ``layer``, kda_layer_prefill on
     raw activations) on the workload, L2 flushed."""
@@ -266,6 +266,13 @@ def time_prefill(w, steps, warmup, world, scalar_gate=False, layer=False):
     torch.cuda.synchronize()
     barrier(world)
     ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    if profile_range:   # one more call, alone inside a profiler range
+        flush.fill_(7)
+        torch.cuda.synchronize()
+        torch.cuda.profiler.start()
+        step()
+        torch.cuda.synchronize()
+        torch.cuda.profiler.stop()
     if kda.kda_check_workspace_error(ws) != kda.KDA_OK:
         raise RuntimeError("device-side check failed during the benchmark")
     # each call with a full workspace on bf16 d = 128 launches three kernels:
@@ -502,6 +509,10 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=DECODE_STEPS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-range", action="store_true",
+                    help="with --prefill-only: after the timed steps, one more prefill call "
+                         "bracketed by cudaProfilerStart / cudaProfilerStop (for a profiler's "
+                         "range replay over the whole call)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the prefill workload (a lighter command for profiler captures); "
                          "prints a line without the extra objects")
@@ -525,7 +536,7 @@ def main():
 
     sampler = ClockSampler(local)
     sampler.start()
-    pf = time_prefill(w, args.steps, args.warmup, world)
+    pf = time_prefill(w, args.steps, args.warmup, world, profile_range=args.profile_range)
     if args.prefill_only:
         clocks = sampler.stop()
         work = prefill_work(w, pf["inputs"]["lengths"])

@@ -44,14 +44,19 @@ def local_pair(q, k, v, log_alpha, beta, workspace=None, stream=None):
 
 def exchange(m, s_tilde, group=None):
     """All-gather of every rank's (M, S~): returns [world, H, d_k, d_*] each, in
-    rank order."""
+    rank order, on the device of ``m``.  Over NCCL the device tensors travel
+    directly (NVLink); a gloo group exchanges host copies."""
     import torch.distributed as dist
     world = dist.get_world_size(group)
-    ms = [torch.empty_like(m) for _ in range(world)]
-    ss = [torch.empty_like(s_tilde) for _ in range(world)]
-    dist.all_gather(ms, m.contiguous(), group=group)
-    dist.all_gather(ss, s_tilde.contiguous(), group=group)
-    return torch.cat(ms), torch.cat(ss)
+    host = dist.get_backend(group) != "nccl"
+    dev = m.device
+    m_x = m.contiguous().cpu() if host else m.contiguous()
+    s_x = s_tilde.contiguous().cpu() if host else s_tilde.contiguous()
+    ms = [torch.empty_like(m_x) for _ in range(world)]
+    ss = [torch.empty_like(s_x) for _ in range(world)]
+    dist.all_gather(ms, m_x, group=group)
+    dist.all_gather(ss, s_x, group=group)
+    return torch.cat(ms).to(dev), torch.cat(ss).to(dev)
 
 
 def cp_prefill(q, k, v, log_alpha, beta, init_state=None, group=None, workspace=None,

@@ -439,119 +439,8 @@ cudaError_t launch_dk(const BwdArgs &p, int grid, cudaStream_t stream) {
 // prefill's preparation give every chunk's entering state (a forward scan,
 // S <- Diag(e^{G_L}) S + MP S + YT V) and every chunk's dL/dS_next (a
 // reverse scan, dS <- Diag(e^{G_L}) dS + MP^T dS + QP^T dO: the transpose of
-// the forward transition); the chunks' steps then run independently.
-
-constexpr int kScanThreads = 256;
-struct ScanSmem {
-    static constexpr uint32_t A = 0;         // MP, 128 x 128 bf16 (two 16 KB K-atoms)
-    static constexpr uint32_t B = 32768;     // YT [128][64] or QP [64][128] bf16, 16 KB
-    static constexpr uint32_t X = 49152;     // v or dO slice [64][32] fp32
-    static constexpr uint32_t S = 57344;     // state slice [128][32] fp32
-    static constexpr uint32_t EGL = 73728;   // 128 fp32
-    static constexpr uint32_t SIZE = 74240;
-};
-
-// Byte offset of bf16 element (row, col) of a K-major tile with 128-byte rows
-// of 64 columns, the 16-byte chunk index XORed with (row mod 8); `atom` bytes
-// per 64-column atom.
-__device__ __forceinline__ uint32_t rec_off(uint32_t row, uint32_t col, uint32_t atom) {
-    const uint32_t c = col & 63u;
-    return (col >> 6) * atom + row * 128u + (((c >> 3) ^ (row & 7u)) << 4) + (c & 7u) * 2u;
-}
-
-__device__ __forceinline__ float bf_at(const uint8_t *tile, uint32_t off) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + off));
-}
-
-struct ScanArgs {
-    SplitTables tab;
-    const __nv_bfloat16 *x;   // v (forward scan) or dO (reverse scan), [T, H, 128]
-    const float *s0;          // init_state (forward) or dL/dS_T (reverse), or null
-    float *out;               // [max_chunks, H, 128, 128]: each chunk's entering value
-    float *last;              // reverse: dL/dS_0 per sequence (overwritten later for
-                              // non-empty sequences), or null
-    int H;
-};
-
-// One CTA per (sequence, head, 32-column slice); 256 threads, each 4 key rows
-// x 4 columns of the slice.
-template <bool REV>
-__global__ void __launch_bounds__(kScanThreads) kda_bwd_scan_kernel(const ScanArgs a) {
-    extern __shared__ __align__(1024) uint8_t sm[];
-    const uint8_t *A = sm + ScanSmem::A, *B = sm + ScanSmem::B;
-    float *xs = reinterpret_cast<float *>(sm + ScanSmem::X);
-    float *ss = reinterpret_cast<float *>(sm + ScanSmem::S);
-    float *egl = reinterpret_cast<float *>(sm + ScanSmem::EGL);
-    const int tid = threadIdx.x;
-    const int sl = blockIdx.x & 3, h = (blockIdx.x >> 2) % a.H, n = (blockIdx.x >> 2) / a.H;
-    const int r0 = 4 * (tid >> 3), c0 = 4 * (tid & 7);   // rows r0..r0+3, slice columns c0..c0+3
-    const size_t st = ((size_t)n * a.H + h) * 128 * 128 + (size_t)sl * 32;
-    for (int i = tid; i < 128 * 32; i += kScanThreads)
-        ss[i] = a.s0 ? a.s0[st + (size_t)(i >> 5) * 128 + (i & 31)] : 0.f;
-    const int cb = a.tab.chunk_off[n], ce = a.tab.chunk_off[n + 1];
-#pragma unroll 1
-    for (int it = 0; it < ce - cb; ++it) {
-        const int c = REV ? ce - 1 - it : cb + it;
-        const int2 ct = a.tab.chunk_tab[c];
-        const uint8_t *rec = a.tab.recs + ((size_t)c * a.H + h) * a.tab.rec_stride;
-        __syncthreads();   // the previous chunk's reads and writes of shared memory are done
-        const size_t ob = ((size_t)c * a.H + h) * 128 * 128 + (size_t)sl * 32;
-        for (int i = tid; i < 128 * 32; i += kScanThreads)
-            a.out[ob + (size_t)(i >> 5) * 128 + (i & 31)] = ss[i];
-        for (int i = tid; i < 2048; i += kScanThreads)
-            reinterpret_cast<uint4 *>(sm + ScanSmem::A)[i] =
-                reinterpret_cast<const uint4 *>(rec + a.tab.off_mp)[i];
-        for (int i = tid; i < 1024; i += kScanThreads)
-            reinterpret_cast<uint4 *>(sm + ScanSmem::B)[i] =
-                reinterpret_cast<const uint4 *>(rec + (REV ? a.tab.off_qp : a.tab.off_yt))[i];
-        if (tid < 128) egl[tid] = reinterpret_cast<const float *>(rec + a.tab.off_egl)[tid];
-        for (int i = tid; i < 64 * 32; i += kScanThreads) {
-            const int t = i >> 5;
-            xs[i] = t < ct.y ? __bfloat162float(a.x[((size_t)(ct.x + t) * a.H + h) * 128 + sl * 32 + (i & 31)])
-                             : 0.f;
-        }
-        __syncthreads();
-        float acc[4][4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) acc[r][q] = egl[r0 + r] * ss[(r0 + r) * 32 + c0 + q];
-#pragma unroll 4
-        for (int k = 0; k < 128; ++k) {   // (MP S) or (MP^T dS)
-            const float4 sk = *reinterpret_cast<const float4 *>(ss + k * 32 + c0);
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const float m = REV ? bf_at(A, rec_off(k, r0 + r, 16384)) : bf_at(A, rec_off(r0 + r, k, 16384));
-                acc[r][0] = fmaf(m, sk.x, acc[r][0]);
-                acc[r][1] = fmaf(m, sk.y, acc[r][1]);
-                acc[r][2] = fmaf(m, sk.z, acc[r][2]);
-                acc[r][3] = fmaf(m, sk.w, acc[r][3]);
-            }
-        }
-#pragma unroll 4
-        for (int t = 0; t < 64; ++t) {   // (YT V) or (QP^T dO)
-            const float4 xt = *reinterpret_cast<const float4 *>(xs + t * 32 + c0);
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const float y = REV ? bf_at(B, rec_off(t, r0 + r, 8192)) : bf_at(B, rec_off(r0 + r, t, 16384));
-                acc[r][0] = fmaf(y, xt.x, acc[r][0]);
-                acc[r][1] = fmaf(y, xt.y, acc[r][1]);
-                acc[r][2] = fmaf(y, xt.z, acc[r][2]);
-                acc[r][3] = fmaf(y, xt.w, acc[r][3]);
-            }
-        }
-        __syncthreads();   // every read of the old slice is done
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-            *reinterpret_cast<float4 *>(ss + (r0 + r) * 32 + c0) =
-                make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-    }
-    if (REV && a.last) {
-        __syncthreads();
-        for (int i = tid; i < 128 * 32; i += kScanThreads)
-            a.last[st + (size_t)(i >> 5) * 128 + (i & 31)] = ss[i];
-    }
-}
+// the forward transition), both run as the prefill's transposed state chain
+// on the tensor cores; the chunks' steps then run independently.
 
 struct ChunkArgs {
     SplitTables tab;
@@ -724,28 +613,13 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
                              nullptr, ws + l.split, scalar_gate, nullptr, stream, kPrepOnly);
     if (e != cudaSuccess) return e;
     const SplitTables tab = split_tables(ws + l.split, num_seqs, total_tokens, H);
-    // 2. the scans: entering states, then dL/dS_next (and a first dL/dS_0)
-    if ((e = set_max_dynamic_smem((const void *)kda_bwd_scan_kernel<false>, (int)ScanSmem::SIZE)) != cudaSuccess)
-        return e;
-    if ((e = set_max_dynamic_smem((const void *)kda_bwd_scan_kernel<true>, (int)ScanSmem::SIZE)) != cudaSuccess)
-        return e;
-    const unsigned scan_grid = (unsigned)((size_t)num_seqs * H * 4);
-    ScanArgs fa;
-    fa.tab = tab;
-    fa.x = static_cast<const __nv_bfloat16 *>(v);
-    fa.s0 = init_state;
-    fa.out = reinterpret_cast<float *>(ws + l.s_in);
-    fa.last = nullptr;
-    fa.H = H;
-    kda_bwd_scan_kernel<false><<<scan_grid, kScanThreads, ScanSmem::SIZE, stream>>>(fa);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    ScanArgs ra = fa;
-    ra.x = static_cast<const __nv_bfloat16 *>(d_o);
-    ra.s0 = d_final_state;
-    ra.out = reinterpret_cast<float *>(ws + l.ds_next);
-    ra.last = d_init_state;
-    kda_bwd_scan_kernel<true><<<scan_grid, kScanThreads, ScanSmem::SIZE, stream>>>(ra);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 2. the scans over the records on the tensor cores (the transposed state
+    // chain, forward and reverse): every chunk's entering state and dL/dS at
+    // its end, and a first dL/dS_0 per sequence
+    e = launch_backward_scans(v, d_o, init_state, d_final_state, cu, num_seqs, total_tokens, H,
+                              ws + l.split, reinterpret_cast<float *>(ws + l.s_in),
+                              reinterpret_cast<float *>(ws + l.ds_next), d_init_state, stream);
+    if (e != cudaSuccess) return e;
     // 3. the chunks' steps, all chunks at once
     BwdArgs p = {};
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.d_o = d_o;

@@ -160,6 +160,16 @@ struct SplitTables {
 };
 SplitTables split_tables(const void *workspace, int num_seqs, int64_t total_tokens, int H);
 
+// The backward pass's two scans over the records a kPrepOnly launch left in
+// `workspace`, on the tensor cores (the transposed state chain): every chunk's
+// entering state into s_in and dL/dS at every chunk's end into ds_next (both
+// [max_chunks, H, 128, 128] fp32, record order), dL/dS_0 into d_init_state
+// (or not, when null).
+cudaError_t launch_backward_scans(const void *v, const void *d_o, const float *init_state,
+                                  const float *d_final_state, const int32_t *cu, int num_seqs,
+                                  int64_t total_tokens, int H, void *workspace, float *s_in,
+                                  float *ds_next, float *d_init_state, cudaStream_t stream);
+
 // Context parallelism: S_out = the state a segment starts from, given the
 // (M_i, S~_i) of the n_prev segments before it and the sequence's S_0 (or null).
 cudaError_t launch_cp_combine(const float *M, const float *S_tilde, const float *S0, float *S_out,

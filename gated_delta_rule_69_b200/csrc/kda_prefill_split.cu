@@ -159,6 +159,9 @@ struct Params {
                                 // when the chain kernel starts only after the prep grid
     uint32_t *work_next;        // prep items handed out after each pipeline's first one
     uint32_t *err_word;
+    // backward-pass scans of the transposed chain: each chunk's state written
+    // here, [record][128 c][128 j] fp32 (record = chunk * H + head)
+    float *states_out;
     int64_t total_tokens;
     int num_seqs, H;
 };
@@ -929,14 +932,26 @@ struct ChainT {
 // segment's cumulative transition for context parallelism: the state starts
 // as the identity, v counts as zero (the v ring and the YT V products are
 // skipped), no output is formed, and the final state is the transition.
-enum : int { kChainPlain = 0, kChainTransition = 2 };
+// The backward pass's two scans over the records (no output products):
+//   kChainSaveS  - the forward chain, writing every chunk's entering state S_n;
+//   kChainReverse - the chunks in reverse order with the transposed
+//                  transition, G_n = Diag(exp(G_L)) G_{n+1} + MP^T G_{n+1}
+//                  + QP^T dO_n (G = dL/dS; the tensor map carries dO, MP and
+//                  QP are read MN-major), writing dL/dS at each chunk's end;
+//                  init_state is dL/dS_T and final_state receives dL/dS_0.
+enum : int { kChainPlain = 0, kChainTransition = 2, kChainSaveS = 3, kChainReverse = 4 };
 
 template <int MODE>
 __global__ void __launch_bounds__(ChainT::THREADS, 1)
 kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     constexpr bool TRANS = MODE == kChainTransition;
+    constexpr bool SAVE = MODE == kChainSaveS;
+    constexpr bool REV = MODE == kChainReverse;
+    constexpr bool OUT = MODE == kChainPlain;          // output products and stores
+    constexpr bool RING_B = OUT || REV;                // QP (and ZB) travel
     using Cfg = ChainT;
     constexpr int NSA = Cfg::NSA, NSB = Cfg::NSB, NSV = Cfg::NSV, NSE = Cfg::NSE, NCW = Cfg::NCW;
+
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *sm = dyn_smem + ((1024u - (smem_addr(dyn_smem) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -990,12 +1005,14 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 if (n >= NSA) mbar_wait(&EMPTYA[sa], ((n / NSA) - 1) & 1, abort_flag);
                 if (n >= NSE) mbar_wait(&EMPTYE[se], ((n / NSE) - 1) & 1, abort_flag);
                 if (*abort_flag) break;
-                const size_t ri = (rec0 + n) * p.H + h;
+                const int nn = REV ? nchunks - 1 - n : n;
+                const size_t ri = (rec0 + nn) * p.H + h;
                 const uint8_t *rec = p.recs + ri * Rec::STRIDE;
                 if (p.rec_ready && !acquire_flag(p.rec_ready + ri, abort_flag)) break;   // the record is complete
                 uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
-                mbar_arrive_expect_tx(&FULLA[sa], 49152);
-                bulk_load(slot_a + Cfg::A_MP, rec + Rec::MP, 49152, &FULLA[sa]);   // MP, YT
+                constexpr uint32_t kABytes = REV ? 32768 : 49152;   // MP (and YT)
+                mbar_arrive_expect_tx(&FULLA[sa], kABytes);
+                bulk_load(slot_a + Cfg::A_MP, rec + Rec::MP, kABytes, &FULLA[sa]);
                 issued_a = n + 1;
                 mbar_arrive_expect_tx(&FULLE[se], 512);
                 bulk_load(sm + Cfg::EGLR + se * 512, rec + Rec::EGL, 512, &FULLE[se]);
@@ -1008,7 +1025,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 wait_drain(&FULLE[n % NSE], (n / NSE) & 1);
         }
     } else if (warp == NCW + 3) {
-        // ---------------------------------------------- ring V: the v tile (from HBM)
+        // ---------------------------------------------- ring V: the v (or dO) tile (from HBM)
         if (!TRANS && lane == 0 && nchunks > 0) {
             tma_prefetch_desc(&tm_v);
             int issued_v = 0;
@@ -1017,7 +1034,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 if (n >= NSV) mbar_wait(&EMPTYV[sv], ((n / NSV) - 1) & 1, abort_flag);
                 if (*abort_flag) break;
                 uint8_t *slot_v = sm + Cfg::RV + sv * Cfg::V_STRIDE;
-                const int t = (int)(bos + (int64_t)n * C);
+                const int t = (int)(bos + (int64_t)(REV ? nchunks - 1 - n : n) * C);
                 mbar_arrive_expect_tx(&FULLV[sv], 16384);
                 tma_load_3d(slot_v, &tm_v, &FULLV[sv], 0, h, t);
                 tma_load_3d(slot_v + 8192, &tm_v, &FULLV[sv], 64, h, t);
@@ -1028,18 +1045,19 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         }
     } else if (warp == NCW + 2) {
         // ---------------------------------------------- ring B: QP, ZB
-        if (!TRANS && lane == 0 && nchunks > 0) {
+        if (RING_B && lane == 0 && nchunks > 0) {
             int issued_b = 0;
             for (int n = 0; n < nchunks; ++n) {
                 const int sb = n % NSB;
                 if (n >= NSB) mbar_wait(&EMPTYB[sb], ((n / NSB) - 1) & 1, abort_flag);
                 if (*abort_flag) break;
-                const size_t ri = (rec0 + n) * p.H + h;
+                const size_t ri = (rec0 + (REV ? nchunks - 1 - n : n)) * p.H + h;
                 const uint8_t *rec = p.recs + ri * Rec::STRIDE;
                 if (p.rec_ready && !acquire_flag(p.rec_ready + ri, abort_flag)) break;
                 uint8_t *slot_b = sm + Cfg::RB + sb * Cfg::B_STRIDE;
-                mbar_arrive_expect_tx(&FULLB[sb], 24576);
-                bulk_load(slot_b + Cfg::B_QP, rec + Rec::QP, 24576, &FULLB[sb]);   // QP, ZB
+                constexpr uint32_t kBBytes = REV ? 16384 : 24576;   // QP (and ZB)
+                mbar_arrive_expect_tx(&FULLB[sb], kBBytes);
+                bulk_load(slot_b + Cfg::B_QP, rec + Rec::QP, kBBytes, &FULLB[sb]);
                 issued_b = n + 1;
             }
             for (int n = (issued_b > NSB ? issued_b - NSB : 0); n < issued_b; ++n)
@@ -1047,8 +1065,9 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         }
     } else if (warp == NCW + 1) {
         // ---------------------------------------------- tensor-core products
-        const uint32_t idS = idesc_bf16(128, 128, false, false);   // A = SB^T (TMEM), B = MP^T
-        const uint32_t idSV = idesc_bf16(128, 128, true, false);   // A = V^T (MN-major), B = YT^T
+        // reverse scan: B = MP and QP themselves, read MN-major
+        const uint32_t idS = idesc_bf16(128, 128, false, REV);     // A = SB^T (TMEM), B = MP^T (MP)
+        const uint32_t idSV = idesc_bf16(128, 128, true, REV);     // A = V^T (MN-major), B = YT^T (QP)
         const uint32_t idO = idesc_bf16(128, 64, false, false);    // A = SB^T (TMEM), B = QP^T
         const uint32_t idOV = idesc_bf16(128, 64, true, false);    // A = V^T (MN-major), B = ZB^T
         // The state-independent products of chunk m: X[m mod 2] = V^T YT^T and
@@ -1059,16 +1078,25 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             if (TRANS) return;
             const int sa = m % NSA, sb = m % NSB, sv = m % NSV;
             const uint32_t bY = smem_addr(sm + Cfg::RA + sa * Cfg::A_STRIDE + Cfg::A_YT);
+            const uint32_t bQ = smem_addr(sm + Cfg::RB + sb * Cfg::B_STRIDE + Cfg::B_QP);
             const uint32_t bZ = smem_addr(sm + Cfg::RB + sb * Cfg::B_STRIDE + Cfg::B_ZB);
             const uint32_t aV = smem_addr(sm + Cfg::RV + sv * Cfg::V_STRIDE);
             mbar_wait(&FULLA[sa], (m / NSA) & 1, abort_flag);
             mbar_wait(&FULLV[sv], (m / NSV) & 1, abort_flag);
+            if (REV) mbar_wait(&FULLB[sb], (m / NSB) & 1, abort_flag);
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)   // X = V^T YT^T  (K = t)
+            for (int ks = 0; ks < 4; ++ks)   // X = V^T YT^T, or dO^T QP  (K = t)
                 mma_bf16_warp(tmem + Cfg::COL_X + 128u * (uint32_t)(m & 1),
                               smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
-                              smem_desc(bY + ks * 32, 16, 1024, kLayoutSW128), idSV, ks > 0 ? 1u : 0u);
+                              REV ? smem_desc(bQ + ks * 2048, 8192, 1024, kLayoutSW128)
+                                  : smem_desc(bY + ks * 32, 16, 1024, kLayoutSW128),
+                              idSV, ks > 0 ? 1u : 0u);
+            if (!OUT) {   // no output products: v (dO) and QP are free again
+                mma_commit_warp(&EMPTYV[sv]);
+                if (REV) mma_commit_warp(&EMPTYB[sb]);
+                return;
+            }
             mbar_wait(&FULLB[sb], (m / NSB) & 1, abort_flag);
             if (m >= 2) mbar_wait(&OFREE[m & 1], ((m - 2) >> 1) & 1, abort_flag);
             tc_fence_after();
@@ -1088,13 +1116,14 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             mbar_wait(SREADY, n & 1, abort_flag);
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)   // X += SB^T MP^T  (K = c')
+            for (int ks = 0; ks < 8; ++ks)   // X += SB^T MP^T, or GB^T MP  (K = c')
                 mma_bf16_ts_warp(tmem + Cfg::COL_X + 128u * (uint32_t)(n & 1), aSB + 8 * ks,
-                                 smem_desc(bM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                                 REV ? smem_desc(bM + ks * 2048, 16384, 1024, kLayoutSW128)
+                                     : smem_desc(bM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
                                  idS, (TRANS && ks == 0) ? 0u : 1u);
             mma_commit_warp(SDONE);
             mma_commit_warp(&EMPTYA[sa]);
-            if (!TRANS) {
+            if (OUT) {
                 const uint32_t bQ = smem_addr(sm + Cfg::RB + sb * Cfg::B_STRIDE + Cfg::B_QP);
                 const uint32_t dO = tmem + Cfg::COL_O + 64u * (uint32_t)(n & 1);
 #pragma unroll
@@ -1146,6 +1175,13 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
                 if (t0 + i < len) dst[(size_t)i * p.H * DV] = __float2bfloat16(v[i]);
         };
         for (int n = 0; n < nchunks; ++n) {
+            if (SAVE || REV) {   // the state entering (forward) or leaving (reverse) this chunk
+                const int nn = REV ? nchunks - 1 - n : n;
+                float *dst = p.states_out + ((rec0 + nn) * p.H + h) * (size_t)(DK * DV) +
+                             (size_t)(32 * g) * DV + j;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) dst[(size_t)i * DV] = S[i];
+            }
             // SB_n^T: column COL_SB + 64 (n mod 2) + c / 2 holds (c, c + 1).  Its
             // previous contents, SB_{n-2}, were last read by chunk n - 2's
             // products, which completed before SDONE of chunk n - 1.
@@ -1157,7 +1193,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(SREADY);
-            if (!TRANS && n >= 1) store_o_t(n - 1);
+            if (OUT && n >= 1) store_o_t(n - 1);
             // S_{n+1} = S_n Diag(exp(G_L)) + X_n, in two halves of 16 columns
             const int se = n % NSE;
             mbar_wait(&FULLE[se], (n / NSE) & 1, abort_flag);
@@ -1182,7 +1218,7 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&EMPTYE[se]);
         }
-        if (!TRANS && nchunks > 0) store_o_t(nchunks - 1);
+        if (OUT && nchunks > 0) store_o_t(nchunks - 1);
         if (p.final_state) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) p.final_state[sbase + (size_t)i * DV] = S[i];
@@ -1451,10 +1487,11 @@ cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const spl
     if (!make_map_split(&mv, v, total_tokens, H, DV, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     {
-        cudaError_t e = set_max_dynamic_smem((const void *)kda_chain_t_kernel<kChainPlain>,
-                                             (int)ChainT::ALLOC);
-        if (e != cudaSuccess) return e;
-        e = set_max_dynamic_smem((const void *)kda_chain_t_kernel<kChainTransition>, (int)ChainT::ALLOC);
+        const void *fn = mode == kChainTransition ? (const void *)kda_chain_t_kernel<kChainTransition>
+                         : mode == kChainSaveS    ? (const void *)kda_chain_t_kernel<kChainSaveS>
+                         : mode == kChainReverse  ? (const void *)kda_chain_t_kernel<kChainReverse>
+                                                  : (const void *)kda_chain_t_kernel<kChainPlain>;
+        const cudaError_t e = set_max_dynamic_smem(fn, (int)ChainT::ALLOC);
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
@@ -1469,6 +1506,8 @@ cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const spl
     cfg.numAttrs = overlap ? 1 : 0;
     const cudaError_t e =
         mode == kChainTransition ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainTransition>, mv, prm)
+        : mode == kChainSaveS    ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainSaveS>, mv, prm)
+        : mode == kChainReverse  ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainReverse>, mv, prm)
                                  : cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainPlain>, mv, prm);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
@@ -1539,6 +1578,44 @@ SplitTables split_tables(const void *workspace, int num_seqs, int64_t total_toke
     t.off_qp = split::Rec::QP;
     t.off_egl = split::Rec::EGL;
     return t;
+}
+
+cudaError_t launch_backward_scans(const void *v, const void *d_o, const float *init_state,
+                                  const float *d_final_state, const int32_t *cu, int num_seqs,
+                                  int64_t total_tokens, int H, void *workspace, float *s_in,
+                                  float *ds_next, float *d_init_state, cudaStream_t stream) {
+    using namespace split;
+    const SplitLayout l = split_layout(num_seqs, total_tokens, H);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    Params prm = {};
+    prm.cu = cu;
+    prm.perm = cu ? reinterpret_cast<int32_t *>(ws + l.perm) : nullptr;
+    prm.chunk_off = reinterpret_cast<int32_t *>(ws + l.chunk_off);
+    prm.chunk_tab = reinterpret_cast<int2 *>(ws + l.chunk_tab);
+    prm.total_chunks = reinterpret_cast<uint32_t *>(ws + 4);
+    prm.recs = ws + l.recs;
+    prm.rec_ready = nullptr;   // the preparation has completed
+    prm.work_next = reinterpret_cast<uint32_t *>(ws + 8);
+    prm.err_word = reinterpret_cast<uint32_t *>(ws);
+    prm.total_tokens = total_tokens;
+    prm.num_seqs = num_seqs;
+    prm.H = H;
+    const unsigned units = (unsigned)((size_t)num_seqs * H);
+    // each chunk's entering state: the forward chain over the records
+    Params pf = prm;
+    pf.init_state = init_state;
+    pf.final_state = nullptr;
+    pf.states_out = s_in;
+    cudaError_t e = launch_chain_t(v, total_tokens, H, pf, units, false, stream, kChainSaveS);
+    if (e != cudaSuccess) return e;
+    // dL/dS at each chunk's end: the reverse chain (launched after the forward
+    // one in plain stream order, so that the steps kernel that follows finds
+    // both complete)
+    Params pr = prm;
+    pr.init_state = d_final_state;
+    pr.final_state = d_init_state;
+    pr.states_out = ds_next;
+    return launch_chain_t(d_o, total_tokens, H, pr, units, false, stream, kChainReverse);
 }
 
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const void *g,
