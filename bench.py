@@ -16,8 +16,9 @@ decode workload (state 512 MiB, larger than L2, so no flush is needed).  The
 "gdn_prefill" object times gdn_prefill (Gated DeltaNet: one gate value per
 token and head) and "layer_prefill" times kda_layer_prefill (raw activations,
 the layer's prologue and epilogue fused) on the headline workload the same
-way; "backward" times kda_backward (the gradients, given seeded upstream
-gradients) on the 4096-token workload.
+way; "backward" times the backward pass (the gradients, given seeded upstream
+gradients; kda_backward_chunked for bf16 d = 128) on the 4096-token workload,
+"backward_long" on the headline workload.
 Under torchrun every rank runs the same workload as an independent replica
 (the operator needs no exchange between GPUs); value = all ranks' tokens over
 the slowest rank's time.
@@ -513,6 +514,9 @@ def main():
                     help="with --prefill-only: after the timed steps, one more prefill call "
                          "bracketed by cudaProfilerStart / cudaProfilerStop (for a profiler's "
                          "range replay over the whole call)")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the backward pass on --backward-workload (a lighter command "
+                         "for profiler captures); prints a line without the other objects")
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the prefill workload (a lighter command for profiler captures); "
                          "prints a line without the extra objects")
@@ -536,6 +540,22 @@ def main():
 
     sampler = ClockSampler(local)
     sampler.start()
+    if args.backward_only:
+        bw = kin.WORKLOADS[args.backward_workload]
+        bwd = time_backward(bw, args.steps, args.warmup, world)
+        clocks = sampler.stop()
+        bwork = backward_work(bw, bwd["lengths"])
+        bms = max_over_ranks(bwd["ms_total"] / len(bwd["ms"]), world)
+        if rank == 0:
+            print(json.dumps({"metric": "backward tokens/s", "value": world * bwork["tokens"] / (bms * 1e-3),
+                              "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                              "warmup": args.warmup, "ms_per_step": bms,
+                              "config": config_of(bw, bwd["lengths"], world),
+                              "gpu_launches": bwd["launches"], "clocks": clocks}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
     pf = time_prefill(w, args.steps, args.warmup, world, profile_range=args.profile_range)
     if args.prefill_only:
         clocks = sampler.stop()
@@ -562,6 +582,8 @@ def main():
     lay = time_prefill(w, args.steps, args.warmup, world, layer=True)
     bw = kin.WORKLOADS[args.backward_workload]
     bwd = time_backward(bw, max(3, args.steps // 4), args.warmup, world)
+    # the backward on the headline workload too, with few steps (about 0.2 s a call)
+    bwd_long = time_backward(w, 3, 3, world) if w.name != bw.name else None
     clocks = sampler.stop()
 
     lengths = pf["inputs"]["lengths"]
@@ -616,21 +638,36 @@ def main():
                                        "traffic": None, "peak_source": src,
                                        "kernel": "kda_layer_prefill",
                                        "algorithmic_bytes_per_launch": lwork["bytes"]}},
-        "backward": {"workload": bw.name + ", backward pass (kda_backward), seeded upstream gradients",
+        "backward": {"workload": bw.name + ", backward pass (kda_backward_chunked for bf16 d = 128), seeded upstream gradients",
                      "value": world * bwork["tokens"] / (bms * 1e-3), "unit": "tokens/s",
                      "ms_per_step": bms, "steps": len(bwd["ms"]),
                      "roofline": {"bound": "alu", "achieved": btfs, "peak": FP32_SIMT_TFLOPS,
                                   "unit": "TFLOP/s", "frac": btfs / FP32_SIMT_TFLOPS,
                                   "traffic": None,
                                   "peak_source": "nominal fp32 CUDA-core rate (148 SMs x 128 lanes x 2 x 1.965 GHz)",
-                                  "kernel": "kda_backward",
+                                  "kernel": "kda_backward_chunked",
                                   "algorithmic_flop_per_launch": bwork["flop"],
                                   "algorithmic_bytes_per_launch": bwork["bytes"],
                                   "hbm_frac": bwork["bytes"] / (bms * 1e-3) / 1e9 / peaks["hbm"]}},
         "gpu_launches": pf["launches"] + dec["launches"] + gdn["launches"] + lay["launches"]
-                        + bwd["launches"] + sum(x[2]["launches"] for x in extra),
+                        + bwd["launches"] + sum(x[2]["launches"] for x in extra)
+                        + (bwd_long["launches"] if bwd_long else 0),
         "clocks": clocks,
     }
+    if bwd_long:
+        lwk = backward_work(w, bwd_long["lengths"])
+        lbms = max_over_ranks(bwd_long["ms_total"] / len(bwd_long["ms"]), world)
+        ltfs = lwk["flop"] / (lbms * 1e-3) / 1e12
+        line["backward_long"] = {
+            "workload": w.name + ", backward pass (kda_backward_chunked), seeded upstream gradients",
+            "value": world * lwk["tokens"] / (lbms * 1e-3), "unit": "tokens/s", "ms_per_step": lbms,
+            "steps": len(bwd_long["ms"]),
+            "roofline": {"bound": "alu", "achieved": ltfs, "peak": FP32_SIMT_TFLOPS, "unit": "TFLOP/s",
+                         "frac": ltfs / FP32_SIMT_TFLOPS, "traffic": None,
+                         "peak_source": "nominal fp32 CUDA-core rate (148 SMs x 128 lanes x 2 x 1.965 GHz)",
+                         "kernel": "kda_backward_chunked",
+                         "algorithmic_flop_per_launch": lwk["flop"],
+                         "algorithmic_bytes_per_launch": lwk["bytes"]}}
     for key, ew, r in extra:
         ework = prefill_work(ew, r["inputs"]["lengths"])
         ems = max_over_ranks(r["ms_total"] / args.steps, world)

@@ -437,7 +437,10 @@ kda_status kda_backward_chunked(const void *q, const void *k, const void *v, con
 
 kda_status kda_check_workspace_error(const void *workspace, kda_stream_t stream_) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-    if (!workspace) return KDA_ERR_INVALID_ARG;
+    if (!workspace) {   // the no-workspace entry point's array on the current device
+        workspace = kda::noalloc_scratch();
+        if (!workspace) return KDA_ERR_CUDA;
+    }
     if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
     uint32_t word = 0;
     if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)

@@ -41,6 +41,10 @@ constexpr int kBwdSlice = kBwdWarps * kBwdCols;    // d_v columns per CTA
 constexpr int kBwdBlock = 64;                      // steps between kept states
 constexpr int kBwdGroup = 4;                       // steps per shared-memory reduction
 constexpr int kBwdMaxCtas = 2 * 148;               // resident CTAs on a B200 (2 per SM)
+// Sub-block of the chunk-parallel kernel's recompute: the whole 64-step block
+// (16-step sub-blocks with kept states cut its scratch from 1 MB to 330 KB a CTA
+// but their second forward pass made the call 20 % slower on a B200).
+constexpr int kBwdChunkSub = kBwdBlock;
 
 template <int DK>
 struct BwdShape {
@@ -248,12 +252,12 @@ __device__ __forceinline__ void flush_group(const float *red, int count, int64_t
     }
 }
 
-// One block of steps [tb, te) backwards, from dS = dL/dS_te: the block run
+// One range of steps [tb, te) backwards, from dS = dL/dS_te: the range run
 // forward again from its entering state S (overwritten) into the scratch,
 // then the backward steps; the row partials are flushed every kBwdGroup
 // steps and at t == t_stop (the first step of the unit).
 template <typename T, int DK>
-__device__ __forceinline__ void block_backward(float4 (&S)[DK / 32], float4 (&dS)[DK / 32],
+__device__ __forceinline__ void range_backward(float4 (&S)[DK / 32], float4 (&dS)[DK / 32],
                                                const BwdArgs &p, int64_t tb, int64_t te,
                                                int64_t t_stop, int h, int warp, int lane, int j0,
                                                int idx, float4 *scratch, float *red, int &buf,
@@ -348,6 +352,48 @@ __device__ __forceinline__ void block_backward(float4 (&S)[DK / 32], float4 (&dS
     }
 }
 
+// One block of steps [tb, te) backwards (te - tb <= kBwdBlock).  SUB =
+// kBwdBlock: the whole block is run forward into the scratch (kBwdBlock step
+// records), then backwards.  SUB < kBwdBlock: a first forward pass keeps only
+// the state entering each SUB-step sub-block (after the SUB step records in
+// the scratch), then each sub-block from the last is run forward again from
+// its kept state and backwards: SUB + kBwdBlock / SUB state records instead
+// of kBwdBlock, for one more forward pass.  The chunk-parallel kernel keeps
+// many units in flight at once, and the smaller scratch stays in L2.
+template <int SUB>
+constexpr int scratch_records() { return SUB >= kBwdBlock ? kBwdBlock : SUB + kBwdBlock / SUB; }
+
+template <typename T, int DK, int SUB>
+__device__ __forceinline__ void block_backward(float4 (&S)[DK / 32], float4 (&dS)[DK / 32],
+                                               const BwdArgs &p, int64_t tb, int64_t te,
+                                               int64_t t_stop, int h, int warp, int lane, int j0,
+                                               int idx, float4 *scratch, float *red, int &buf,
+                                               int &gi, int64_t &g_hi) {
+    if (SUB >= kBwdBlock) {
+        range_backward<T, DK>(S, dS, p, tb, te, t_stop, h, warp, lane, j0, idx, scratch, red, buf,
+                              gi, g_hi);
+        return;
+    }
+    constexpr int RPL = DK / 32;
+    constexpr int R4 = scratch_step4<DK>();
+    float4 *kept = scratch + (size_t)SUB * R4;   // the state entering sub-block s at kept + s R4
+#pragma unroll 1
+    for (int64_t sb = tb; sb < te; sb += SUB) {
+        float4 *ks = kept + (size_t)((sb - tb) / SUB) * R4;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) ks[idx + i * kBwdThreads] = S[i];
+        forward_run<T, DK>(S, p, sb, sb + SUB < te ? sb + SUB : te, h, lane, j0, nullptr, idx);
+    }
+#pragma unroll 1
+    for (int64_t sb = tb + ((te - tb - 1) / SUB) * SUB; sb >= tb; sb -= SUB) {
+        const float4 *ks = kept + (size_t)((sb - tb) / SUB) * R4;
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) S[i] = ks[idx + i * kBwdThreads];
+        range_backward<T, DK>(S, dS, p, sb, sb + SUB < te ? sb + SUB : te, t_stop, h, warp, lane, j0,
+                              idx, scratch, red, buf, gi, g_hi);
+    }
+}
+
 template <typename T, int DK>
 __global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_kernel(const BwdArgs p) {
     using Sh = BwdShape<DK>;
@@ -415,8 +461,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_kernel(const BwdA
             const float4 *ck = p.ckpt + (((size_t)(slot0 + b) * p.H + h) * p.nslices + s) * S4;
 #pragma unroll
             for (int i = 0; i < RPL; ++i) S[i] = ck[idx + i * kBwdThreads];
-            block_backward<T, DK>(S, dS, p, tb, te, bos, h, warp, lane, j0, idx, scratch, red, buf,
-                                  gi, g_hi);
+            block_backward<T, DK, kBwdBlock>(S, dS, p, tb, te, bos, h, warp, lane, j0, idx, scratch, red,
+                                             buf, gi, g_hi);
         }
         if (p.d_init_state) {
 #pragma unroll
@@ -459,7 +505,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_chunk_kernel(cons
     extern __shared__ float red[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int idx = warp * 32 + lane;
-    float4 *scratch = p.scratch + (size_t)blockIdx.x * kBwdBlock * scratch_step4<DK>();
+    float4 *scratch = p.scratch + (size_t)blockIdx.x * scratch_records<kBwdChunkSub>() * scratch_step4<DK>();
     int buf = 0, gi = 0;
     int64_t g_hi = 0;
     const int units = (int)*c.tab.total_chunks * p.H * p.nslices;
@@ -478,8 +524,8 @@ __global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_chunk_kernel(cons
             S[i] = *reinterpret_cast<const float4 *>(c.s_in + base + (size_t)(lane + 32 * i) * p.dv_total);
             dS[i] = *reinterpret_cast<const float4 *>(c.ds_next + base + (size_t)(lane + 32 * i) * p.dv_total);
         }
-        block_backward<T, DK>(S, dS, p, tb, te, tb, h, warp, lane, j0, idx, scratch, red, buf, gi,
-                              g_hi);
+        block_backward<T, DK, kBwdChunkSub>(S, dS, p, tb, te, tb, h, warp, lane, j0, idx, scratch, red,
+                                            buf, gi, g_hi);
         if (p.d_init_state) {
             int lo = 0, hi = c.num_seqs;   // the last sequence whose first chunk is <= ch
             while (hi - lo > 1) {
@@ -582,7 +628,7 @@ ChunkedLayout chunked_layout(int num_seqs, int64_t total_tokens, int H) {
     l.s_in = (prefill_split_workspace(num_seqs, total_tokens, H) + 1023) & ~(size_t)1023;
     l.ds_next = l.s_in + l.max_chunks * H * state;
     l.scratch = l.ds_next + l.max_chunks * H * state;
-    l.total = l.scratch + (size_t)l.grid * kBwdBlock * scratch_step4<128>() * sizeof(float4);
+    l.total = l.scratch + (size_t)l.grid * scratch_records<kBwdChunkSub>() * scratch_step4<128>() * sizeof(float4);
     return l;
 }
 

@@ -63,6 +63,9 @@ struct Bufs {
     float *nrm;          // 128 fp32, or null
     float neg_eA;        // -exp(A_log[h])
     float qk_eps;
+    // The scalar (Gated DeltaNet) gate: one raw log_alpha per token, 64 fp32
+    // (zero past the chunk end), or null for the per-channel gate in graw.
+    const float *gsc;
 };
 
 // Index of A element (t, i): rows padded to 65 floats, so that a warp
@@ -219,6 +222,98 @@ __device__ int gate(const Bufs &b, int pt, int L) {
         *reinterpret_cast<uint32_t *>(kbar + ok) = pack_bf16x2(k0 * b0, k1 * b1);
     }
     return !slow ? kProductForm : ((flag & 2u) ? kPairwise : kSecondary);
+}
+
+// ---- the same for a scalar gate (b.gsc: one log_alpha per token, every
+// channel decaying alike).  The running sums and the factors e^{G_t},
+// e^{-G_t} and e^{G_L - G_t} are per token, so they are formed once per token
+// (64 exponentials of each kind instead of one per element) and every thread
+// only scales its elements.  Each sum and factor is taken by the very
+// operations, in the same order, that gate() applies per channel, so the
+// operands equal those of the per-channel gate fed the scalar repeated over
+// the channels, bit for bit.  A chunk that takes a slow path also gets the
+// gate spread over the channels in b.graw and the 16-token block sums in
+// b.csum, which those paths read.  Scratch: b.xf (the solve's, free here).
+template <int BAR>
+__device__ int gate_scalar(const Bufs &b, int pt, int L) {
+    const int c = 2 * (pt & 63);
+    const int tg = pt >> 6;
+    const int t0 = tg * 16;
+    const int katom = c >> 6, cc = c & 63;
+    uint8_t *stack = b.stk + katom * 16384;
+    uint8_t *khat = b.khat + katom * 8192;
+    uint8_t *kbar = b.kbar + katom * 8192;
+    float *part = b.xf;                                        // [64] sums within each block
+    float *bsum = b.xf + 64;                                   // [4] block sums
+    float4 *fac = reinterpret_cast<float4 *>(b.xf + 128);     // [64] (e^G, e^-G, Kbar's factor, -)
+
+    if (L < C) {   // rows past the chunk's end: zero operand rows (uniform over the group)
+        for (int v = pt; v < (C - L) * 16; v += kGroupThreads) {
+            const int t = L + (v >> 4), piece = v & 15;
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            uint8_t *atom = b.stk + (piece >> 3) * 16384;
+            *reinterpret_cast<uint4 *>(atom + sw128_off(t, (piece & 7) * 8)) = z;
+            *reinterpret_cast<uint4 *>(atom + sw128_off(64 + t, (piece & 7) * 8)) = z;
+        }
+    }
+    if (pt < 4) {   // block pt's running sum, in token order from zero (base-2 units)
+        float r = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            r = fmaf(clamp_log_alpha(b.gsc[16 * pt + i]), kLog2e, r);
+            part[16 * pt + i] = r;
+        }
+        bsum[pt] = r;
+    }
+    if (pt == 0) *b.slow_flag = 0u;
+    named_barrier(BAR, kGroupThreads);
+    constexpr float kSlow2 = kSlowPathLogDecay * kLog2e;
+    float GL = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) GL += bsum[j];
+    const bool slow = GL < kSlow2;
+    bool pairwise = false;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) pairwise |= bsum[j] < kSlow2;
+    const float eL = exp2_f(GL);
+    constexpr float kMaxInv2 = 80.f * kLog2e;   // Khat's factor is capped at e^80
+    if (pt < C) {   // token pt's factors
+        const int j = pt >> 4;
+        float off = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 3; ++jj)
+            if (jj < j) off += bsum[jj];
+        const float G = part[pt] + off;
+        const float ih = exp2_f(fminf(-G, kMaxInv2));
+        fac[pt] = make_float4(exp2_f(G), ih, slow ? exp2_f(GL - G) : eL * ih, 0.f);
+    }
+    if (pt < 128) b.egl[pt] = eL;
+    if (slow) {   // what the slow paths read: the gate per channel and the block sums
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat16 gv = __float2bfloat16_rn(b.gsc[t0 + i]);   // exact: a bf16 value
+            *reinterpret_cast<__nv_bfloat162 *>(const_cast<uint8_t *>(b.graw) + (t0 + i) * 256 + c * 2) =
+                __halves2bfloat162(gv, gv);
+        }
+        b.csum[tg * 128 + c] = bsum[tg];
+        b.csum[tg * 128 + c + 1] = bsum[tg];
+    }
+    named_barrier(BAR, kGroupThreads);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int t = t0 + i;
+        const float4 f = fac[t];
+        const __nv_bfloat162 kv = *reinterpret_cast<const __nv_bfloat162 *>(stack + sw128_off(t, cc));
+        const __nv_bfloat162 qv = *reinterpret_cast<const __nv_bfloat162 *>(stack + sw128_off(64 + t, cc));
+        const float k0 = __low2float(kv), k1 = __high2float(kv);
+        const float q0 = __low2float(qv), q1 = __high2float(qv);
+        const uint32_t ok = sw128_off(t, cc);
+        *reinterpret_cast<uint32_t *>(stack + ok) = pack_bf16x2(k0 * f.x, k1 * f.x);
+        *reinterpret_cast<uint32_t *>(stack + sw128_off(64 + t, cc)) = pack_bf16x2(q0 * f.x, q1 * f.x);
+        *reinterpret_cast<uint32_t *>(khat + ok) = pack_bf16x2(k0 * f.y, k1 * f.y);
+        *reinterpret_cast<uint32_t *>(kbar + ok) = pack_bf16x2(k0 * f.z, k1 * f.z);
+    }
+    return !slow ? kProductForm : (pairwise ? kPairwise : kSecondary);
 }
 
 // ---- secondary chunking, for a chunk that decays too fast for one reference
@@ -491,37 +586,43 @@ __device__ __forceinline__ void merge(const float *__restrict__ AF, float *__res
     named_barrier(BAR, kGroupThreads);
 }
 
-// ---- T = (I + A)^-1 by recursive doubling from closed-form 4x4 diagonal
-// blocks; writes T diag(beta) as bf16 into b.tb.  Starts and ends with every
+// ---- T = (I + A)^-1: the 16 x 16 diagonal blocks by forward substitution,
+// then recursive doubling (merges at 16 and 32); writes T diag(beta) as bf16
+// into b.tb.  Starts and ends with every
 // thread of the group past a barrier on its buffers.
 template <int BAR>
 __device__ void solve(const Bufs &b, int pt) {
     const float *__restrict__ AF = b.af;
     float *__restrict__ TF = b.tf;
     float *__restrict__ XF = b.xf;
-    for (int v = pt; v < 1024; v += kGroupThreads) {   // zero outside the 4x4 diagonal blocks
-        const int row = v >> 4, g4 = v & 15;
-        if (g4 != (row >> 2))
+    if (pt < 64) {
+        // The four 16 x 16 diagonal blocks of T, one column per lane (two warps,
+        // a half-warp per block), by forward substitution in fp32: for rows
+        // i > j of column j, x_i = -sum_{k < i} A_ik x_k with x_j = 1 and
+        // x_k = 0 above it.  The half-warp's lanes read the same A element at
+        // once (a broadcast), and only the last term of each row waits for the
+        // row before.
+        const int b0 = 16 * (pt >> 4), j = pt & 15;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 1; i < 16; ++i) {
+            float acc = 0.f;
+#pragma unroll
+            for (int k = 0; k < i; ++k) acc = fmaf(AF[fidx(b0 + i, b0 + k)], x[k], acc);
+            if (i > j) x[i] = -acc;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) TF[tfi(b0 + i, b0 + j)] = x[i];
+    } else {   // zero outside the 16 x 16 diagonal blocks
+        for (int v = pt - 64; v < 768; v += kGroupThreads - 64) {
+            const int row = v / 12, g = v % 12;               // 12 float4 off the block per row
+            const int g4 = g + (g >= 4 * (row >> 4) ? 4 : 0);  // skip the row's diagonal block
             *reinterpret_cast<float4 *>(&TF[tfi(row, 4 * g4)]) = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    if (pt < 16) {   // 4x4 unit lower-triangular inverses, written out
-        const int b0 = 4 * pt;
-        const float n10 = AF[fidx(b0 + 1, b0)];
-        const float n20 = AF[fidx(b0 + 2, b0)], n21 = AF[fidx(b0 + 2, b0 + 1)];
-        const float n30 = AF[fidx(b0 + 3, b0)], n31 = AF[fidx(b0 + 3, b0 + 1)],
-                    n32 = AF[fidx(b0 + 3, b0 + 2)];
-        const float t10 = -n10, t21 = -n21, t32 = -n32;
-        const float t20 = -(n20 + n21 * t10);
-        const float t31 = -(n31 + n32 * t21);
-        const float t30 = -(n30 + n31 * t10 + n32 * t20);
-        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 0, b0)]) = make_float4(1.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 1, b0)]) = make_float4(t10, 1.f, 0.f, 0.f);
-        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 2, b0)]) = make_float4(t20, t21, 1.f, 0.f);
-        *reinterpret_cast<float4 *>(&TF[tfi(b0 + 3, b0)]) = make_float4(t30, t31, t32, 1.f);
+        }
     }
     named_barrier(BAR, kGroupThreads);
-    merge<4, BAR>(AF, TF, XF, pt);
-    merge<8, BAR>(AF, TF, XF, pt);
     merge<16, BAR>(AF, TF, XF, pt);
     merge<32, BAR>(AF, TF, XF, pt);
 

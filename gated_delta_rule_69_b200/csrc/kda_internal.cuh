@@ -170,6 +170,9 @@ cudaError_t launch_backward_scans(const void *v, const void *d_o, const float *i
                                   int64_t total_tokens, int H, void *workspace, float *s_in,
                                   float *ds_next, float *d_init_state, cudaStream_t stream);
 
+// The fixed scratch array of kda_prefill_noalloc on the current device.
+void *noalloc_scratch();
+
 // Context parallelism: S_out = the state a segment starts from, given the
 // (M_i, S~_i) of the n_prev segments before it and the sequence's S_0 (or null).
 cudaError_t launch_cp_combine(const float *M, const float *S_tilde, const float *S0, float *S_out,

@@ -45,6 +45,12 @@ void *scratch_for_current_device() {
 
 }  // namespace
 
+namespace kda {
+// The array's device address on the current device (null on failure), for
+// kda_check_workspace_error(NULL, ...), which reads its error word.
+void *noalloc_scratch() { return scratch_for_current_device(); }
+}  // namespace kda
+
 extern "C" kda_status kda_prefill_noalloc(const void *q, const void *k, const void *v,
                                           const void *log_alpha, const void *beta,
                                           const float *init_state, const int32_t *cu_seqlens,

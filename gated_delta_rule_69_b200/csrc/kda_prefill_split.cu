@@ -77,7 +77,8 @@ struct PrepSmem {
     static constexpr uint32_t BARS = 108288;   // 6 mbarriers
     static constexpr uint32_t MISC = 108352;   // tmem base, abort, slow flag, next-item slots at 4, 5
     static constexpr uint32_t NRM = 108416;    // layer prologue: 128 fp32 inverse norms
-    static constexpr uint32_t SIZE = 108928;
+    static constexpr uint32_t GSC = 108928;    // scalar gate: 64 fp32 raw log_alpha
+    static constexpr uint32_t SIZE = 109184;
     static constexpr uint32_t PIPE = 109568;   // per-pipeline stride
     static constexpr uint32_t ALLOC = 2 * PIPE + 1024;
 };
@@ -331,7 +332,7 @@ __device__ __forceinline__ void write_qp(uint8_t *stk, uint32_t tmem, int quad, 
     }
 }
 
-template <int P, bool LAYER>
+template <int P, bool LAYER, bool SCALAR>
 __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int tid, int warp, int lane,
                                               const CUtensorMap &tm_k, const CUtensorMap &tm_q,
                                               const CUtensorMap &tm_g, const Params &p,
@@ -359,6 +360,7 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
     // slot, which every thread reads after the current item's last barrier.
     volatile uint32_t *next_slot = misc + 4;
     uint32_t item = 2 * blockIdx.x + P;
+    uint32_t drawn = 0;   // the next item, drawn while the current one's loads are in flight
 #pragma unroll 1
     for (int it = 0; item < total_items; ++it) {
         const int h = item % p.H;
@@ -373,33 +375,31 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         // the rest of the record may still be leaving shared memory, so the
         // leader's arrive, which lets the group write again, waits for that.
         if (leader) {
-            mbar_expect_tx(&B[0], p.scalar_gate ? kRawBytes - 16384 : kRawBytes);
+            mbar_expect_tx(&B[0], SCALAR ? kRawBytes - 16384 : kRawBytes);
             const int t = (int)tok0;
             tma_load_3d(sm + PrepSmem::STK, &tm_k, &B[0], 0, h, t);
             tma_load_3d(sm + PrepSmem::STK + 16384, &tm_k, &B[0], 64, h, t);
             tma_load_3d(sm + PrepSmem::STK + 8192, &tm_q, &B[0], 0, h, t);
             tma_load_3d(sm + PrepSmem::STK + 16384 + 8192, &tm_q, &B[0], 64, h, t);
-            if (!p.scalar_gate) tma_load_3d(sm + PrepSmem::GRAW, &tm_g, &B[0], 0, h, t);
+            if (!SCALAR) tma_load_3d(sm + PrepSmem::GRAW, &tm_g, &B[0], 0, h, t);
             bulk_wait_read_all();
             mbar_arrive(&B[0]);
+            // while the loads are in flight: draw the next item, and publish the
+            // previous record once its stores have completed
+            drawn = atomicAdd(p.work_next, 1u);   // consumed at the end of the item
+            if (pending) {
+                bulk_wait_all();
+                publish_flag(pending);
+                pending = nullptr;
+            }
         }
         if (pt < C) {
             float bv = (pt < L) ? __bfloat162float(p.beta[(size_t)(tok0 + pt) * p.H + h]) : 0.f;
             if (LAYER && pt < L) bv = 1.f / (1.f + __expf(-bv));   // beta = sigmoid(logit)
             beta[pt] = bv;
-            if (p.scalar_gate) {
-                // One log_alpha per token, broadcast over its 128 channels.  GRAW
-                // is a source of the previous record's stores: the leader has
-                // waited for every store to read its source before this
-                // barrier of the 64 threads that write it.
-                __nv_bfloat16 gv = __float2bfloat16(0.f);
-                if (pt < L) gv = p.g[(size_t)(tok0 + pt) * p.H + h];
-                named_barrier(BAR + 2, C);
-                const __nv_bfloat162 g2 = __halves2bfloat162(gv, gv);
-                const uint32_t gw = *reinterpret_cast<const uint32_t *>(&g2);
-                uint4 *row = reinterpret_cast<uint4 *>(sm + PrepSmem::GRAW + pt * 256);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) row[i] = make_uint4(gw, gw, gw, gw);
+            if (SCALAR) {   // one log_alpha per token (zero past the chunk end)
+                reinterpret_cast<float *>(sm + PrepSmem::GSC)[pt] =
+                    pt < L ? __bfloat162float(p.g[(size_t)(tok0 + pt) * p.H + h]) : 0.f;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&B[0]);
@@ -422,12 +422,12 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         b.nrm = LAYER ? reinterpret_cast<float *>(sm + PrepSmem::NRM) : nullptr;
         b.neg_eA = LAYER ? -__expf(p.A_log[h]) : 0.f;
         b.qk_eps = p.qk_eps;
+        b.gsc = SCALAR ? reinterpret_cast<const float *>(sm + PrepSmem::GSC) : nullptr;
 
         mbar_wait(&B[0], it & 1, abort_flag);
-        const int form = prep::gate<BAR, LAYER>(b, pt, L);
+        const int form = SCALAR ? prep::gate_scalar<BAR>(b, pt, L) : prep::gate<BAR, LAYER>(b, pt, L);
         fence_async_smem();
         named_barrier(BAR, prep::kGroupThreads);
-        uint32_t drawn = 0;
         if (wp == 0) {   // tensor-core products: issued by the group's first warp
             tc_fence_after();
             const uint32_t a0 = smem_addr(sm + PrepSmem::STK), b0 = smem_addr(sm + PrepSmem::KHAT);
@@ -438,14 +438,6 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
                               smem_desc(b0 + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
                               id, ks > 0 ? 1u : 0u);
             mma_commit_warp(&B[1]);
-        }
-        if (leader) {
-            drawn = atomicAdd(p.work_next, 1u);   // consumed at the end of the item
-            if (pending) {
-                bulk_wait_all();
-                publish_flag(pending);
-                pending = nullptr;
-            }
         }
         mbar_wait(&B[1], it & 1, abort_flag);
         tc_fence_after();
@@ -544,8 +536,9 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
 }
 
 // LAYER: the layer prologue (gate activation, q / k normalisation, beta
-// sigmoid) fused in; a separate instantiation keeps the plain kernel as it is.
-template <bool LAYER>
+// sigmoid) fused in; SCALAR: the Gated DeltaNet gate (one log_alpha per
+// token); separate instantiations keep the plain kernel as it is.
+template <bool LAYER, bool SCALAR>
 __global__ void __launch_bounds__(kPrepThreads, 1)
 kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_g, const Params p) {
@@ -583,8 +576,8 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t total_items = *p.total_chunks * (uint32_t)p.H;
     const uint32_t tmem = misc0[0] + 256u * P;
     if (2 * blockIdx.x < total_items) {
-        if (P == 0) prep_pipeline<0, LAYER>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
-        else prep_pipeline<1, LAYER>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
+        if (P == 0) prep_pipeline<0, LAYER, SCALAR>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
+        else prep_pipeline<1, LAYER, SCALAR>(sm, tmem, tid, warp, lane, tm_k, tm_q, tm_g, p, total_items);
     }
     tc_fence_before();
     __syncthreads();
@@ -1680,9 +1673,11 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                                           work_next);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = set_max_dynamic_smem((const void *)kda_prep_kernel<false>, (int)PrepSmem::ALLOC);
+    e = set_max_dynamic_smem((const void *)kda_prep_kernel<false, false>, (int)PrepSmem::ALLOC);
     if (e != cudaSuccess) return e;
-    e = set_max_dynamic_smem((const void *)kda_prep_kernel<true>, (int)PrepSmem::ALLOC);
+    e = set_max_dynamic_smem((const void *)kda_prep_kernel<true, false>, (int)PrepSmem::ALLOC);
+    if (e != cudaSuccess) return e;
+    e = set_max_dynamic_smem((const void *)kda_prep_kernel<false, true>, (int)PrepSmem::ALLOC);
     if (e != cudaSuccess) return e;
     Params prm;
     prm.k = static_cast<const __nv_bfloat16 *>(k);
@@ -1725,8 +1720,9 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = layer ? cudaLaunchKernelEx(&cfg, kda_prep_kernel<true>, mk, mq, mg, prm)
-                  : cudaLaunchKernelEx(&cfg, kda_prep_kernel<false>, mk, mq, mg, prm);
+        e = layer         ? cudaLaunchKernelEx(&cfg, kda_prep_kernel<true, false>, mk, mq, mg, prm)
+            : scalar_gate ? cudaLaunchKernelEx(&cfg, kda_prep_kernel<false, true>, mk, mq, mg, prm)
+                          : cudaLaunchKernelEx(&cfg, kda_prep_kernel<false, false>, mk, mq, mg, prm);
         if (e != cudaSuccess) return e;
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

@@ -217,9 +217,11 @@ def _decode(fn, q, k, v, log_alpha, beta, state, o, stream):
     return o
 
 
-def kda_check_workspace_error(workspace, stream=None) -> int:
-    """Synchronise and return the status of the device-side checks."""
-    return int(lib().kda_check_workspace_error(_ptr(workspace), _stream(stream, workspace.device)))
+def kda_check_workspace_error(workspace=None, stream=None) -> int:
+    """Synchronise and return the status of the device-side checks; with
+    workspace None, those of kda_prefill_noalloc on the current device."""
+    device = workspace.device if workspace is not None else torch.device("cuda", torch.cuda.current_device())
+    return int(lib().kda_check_workspace_error(_ptr(workspace), _stream(stream, device)))
 
 
 def kda_prefill_noalloc(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None,

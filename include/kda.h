@@ -346,9 +346,11 @@ kda_status kda_backward_chunked(const void *q, const void *k, const void *v, con
  * Synchronises `stream`, then reads the error word that the prefill and
  * backward kernels leave at the start of `workspace` (non-zero when a
  * device-side check failed, e.g. cu_seqlens not non-decreasing or not ending
- * at T_total).  Returns
- * KDA_ERR_INVALID_ARG in that case, KDA_OK otherwise.  Debugging aid; the
- * only call here that blocks.
+ * at T_total).  With workspace NULL it reads the word that
+ * kda_prefill_noalloc leaves in its fixed array on the current device.
+ * Returns KDA_ERR_INVALID_ARG in that case, KDA_OK otherwise (KDA_ERR_CUDA
+ * if the word cannot be read).  Debugging aid; the only call here that
+ * blocks.
  */
 kda_status kda_check_workspace_error(const void *workspace,
                                      kda_stream_t stream);
@@ -372,8 +374,12 @@ kda_status kda_check_workspace_error(const void *workspace,
  * array's device address and caches it; make that first call before any
  * stream capture.  All calls share the one array: calls that may overlap on
  * the GPU (different streams, or several host threads) race on it and must
- * be serialised by the caller.  kda_check_workspace_error cannot be used
- * with this entry point.
+ * be serialised by the caller.  The device-side checks of a call (a bad
+ * cu_seqlens) leave their error word in the array: kda_check_workspace_error
+ * with a NULL workspace reads it for the current device (it synchronises
+ * `stream`).  The array's device address is looked up once per device and
+ * kept for the life of the process; a cudaDeviceReset invalidates it, so a
+ * process that resets a device must not call this entry point on it again.
  */
 #define KDA_NOALLOC_MAX_SEQS 4096
 

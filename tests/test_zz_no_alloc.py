@@ -57,3 +57,22 @@ def test_noalloc_matches_prefill_two_calls(dtype, dk, dv, tol):
         assert torch.isfinite(o.float()).all()
         assert ((o.float() - ref_o.float()).abs().max() / scale_o).item() <= tol
         assert ((s - ref_s).abs().max() / scale_s).item() <= tol
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("fp32", 16)])
+def test_noalloc_reports_device_errors(dtype, d):
+    """The device-side check of cu_seqlens (a non-monotone one here) leaves
+    its error word in the built-in array, where kda_check_workspace_error with
+    no workspace reads it; the next good call clears it."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    kda = _kda()
+    w = kin.Workload("noalloc_err", "prefill", H=1, d_k=d, d_v=d, dtype=dtype, seed=4343, T=0)
+    inp = kin.generate(w, device="cuda", lengths=[10, 10])
+    args = (inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"])
+    bad = torch.tensor([0, 15, 10, 20], dtype=torch.int32, device="cuda")
+    kda.kda_prefill_noalloc(*args, cu_seqlens=bad)
+    assert kda.kda_check_workspace_error() == kda.KDA_ERR_INVALID_ARG
+    kda.kda_prefill_noalloc(*args, cu_seqlens=inp["cu_seqlens"])
+    assert kda.kda_check_workspace_error() == kda.KDA_OK
