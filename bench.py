@@ -43,6 +43,12 @@ EXTRA_PREFILL = (("prefill_T4096", "prefill_T4096_H16_d128"),
                  ("varlen", "varlen_16seq_256to16384_H32_d128"))
 BACKWARD_DEFAULT = "prefill_T4096_H16_d128"
 DECODE_DEFAULT = "decode_B256_H32_d128"
+# DRAM bytes (read + write) of one whole kda_prefill call, from an ncu
+# application-range capture over one call of the 16384-token, 32-head workload
+# (547.5 MB read + 693.4 MB written), scaled by the token count to the
+# 131072-token workload, which runs the same plan and per-chunk schedule
+# (profiles/kda_prefill_T131072_H32_d128.md); null for other workloads.
+CALL_TRAFFIC = {"prefill_T131072_H32_d128": (547.5e6 + 693.4e6) * 131072 / 16384}
 # the oracle's sample: whole heads of the first sequence, at most this many
 # of its first tokens (its cost is linear in (token, head) pairs)
 ORACLE_PREFIX = 32768
@@ -613,7 +619,8 @@ def main():
         "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
         "config": config_of(w, lengths, world),
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": gbs / peaks["hbm"], "traffic": None, "peak_source": src,
+                     "frac": gbs / peaks["hbm"], "traffic": CALL_TRAFFIC.get(w.name),
+                     "traffic_unit": "bytes per call (DRAM read + write)", "peak_source": src,
                      "kernel": "kda_prefill", "algorithmic_bytes_per_launch": work["bytes"],
                      "tensor_tflops": tfs, "tensor_frac": tfs / peaks["bf16"],
                      "algorithmic_flop_per_launch": work["flop"]},
