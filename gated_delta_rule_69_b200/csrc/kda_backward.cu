@@ -32,6 +32,15 @@
 #include "kda_internal.cuh"
 
 namespace kda {
+
+// kda_backward_tc.cu: the chunk-local gradients on the tensor cores
+size_t backward_tc_scratch(int grid);
+cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                               const void *d_o, int64_t total_tokens, int H, const int2 *chunk_tab,
+                               const uint32_t *total_chunks, const float *s_in, const float *ds_next, float *dq,
+                               float *dk, float *dv, float *dg, float *dbeta, uint32_t *slow, float *gscr,
+                               uint32_t *err_word, int grid, cudaStream_t stream);
+
 namespace {
 
 constexpr int kBwdWarps = 8;
@@ -41,6 +50,7 @@ constexpr int kBwdSlice = kBwdWarps * kBwdCols;    // d_v columns per CTA
 constexpr int kBwdBlock = 64;                      // steps between kept states
 constexpr int kBwdGroup = 4;                       // steps per shared-memory reduction
 constexpr int kBwdMaxCtas = 2 * 148;               // resident CTAs on a B200 (2 per SM)
+constexpr int kBwdTcMaxCtas = 148;                 // tensor-core chunk kernel: one CTA per SM
 // Sub-block of the chunk-parallel kernel's recompute: the whole 64-step block
 // (16-step sub-blocks with kept states cut its scratch from 1 MB to 330 KB a CTA
 // but their second forward pass made the call 20 % slower on a B200).
@@ -492,6 +502,7 @@ struct ChunkArgs {
     SplitTables tab;
     const float *s_in;     // [max_chunks, H, 128, 128] entering states
     const float *ds_next;  // [max_chunks, H, 128, 128] dL/dS at each chunk's end
+    const uint32_t *only;  // [max_chunks * H] or null: run only the (chunk, head) items flagged 1
     int num_seqs;
 };
 
@@ -514,6 +525,7 @@ __global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_chunk_kernel(cons
         const int s = u % p.nslices;
         const int h = (u / p.nslices) % p.H;
         const int ch = u / (p.nslices * p.H);
+        if (c.only && !c.only[(size_t)ch * p.H + h]) continue;
         const int2 ct = c.tab.chunk_tab[ch];
         const int64_t tb = ct.x, te = (int64_t)ct.x + ct.y;
         const int j0 = s * kBwdSlice + warp * kBwdCols;
@@ -613,9 +625,9 @@ cudaError_t launch_backward(const void *q, const void *k, const void *v, const v
 namespace {
 
 struct ChunkedLayout {
-    size_t split, s_in, ds_next, scratch, total;
+    size_t split, s_in, ds_next, scratch, slow, gscr, total;
     size_t max_chunks;
-    int grid;
+    int grid, grid_tc;
 };
 
 ChunkedLayout chunked_layout(int num_seqs, int64_t total_tokens, int H) {
@@ -628,7 +640,11 @@ ChunkedLayout chunked_layout(int num_seqs, int64_t total_tokens, int H) {
     l.s_in = (prefill_split_workspace(num_seqs, total_tokens, H) + 1023) & ~(size_t)1023;
     l.ds_next = l.s_in + l.max_chunks * H * state;
     l.scratch = l.ds_next + l.max_chunks * H * state;
-    l.total = l.scratch + (size_t)l.grid * scratch_records<kBwdChunkSub>() * scratch_step4<128>() * sizeof(float4);
+    l.slow = l.scratch + (size_t)l.grid * scratch_records<kBwdChunkSub>() * scratch_step4<128>() * sizeof(float4);
+    l.gscr = (l.slow + l.max_chunks * H * sizeof(uint32_t) + 255) & ~(size_t)255;
+    const size_t items = l.max_chunks * (size_t)H;
+    l.grid_tc = (int)(items < (size_t)kBwdTcMaxCtas ? items : (size_t)kBwdTcMaxCtas);
+    l.total = l.gscr + backward_tc_scratch(l.grid_tc);
     return l;
 }
 
@@ -666,7 +682,19 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
                               ws + l.split, reinterpret_cast<float *>(ws + l.s_in),
                               reinterpret_cast<float *>(ws + l.ds_next), d_init_state, stream);
     if (e != cudaSuccess) return e;
-    // 3. the chunks' steps, all chunks at once
+    // 3. the chunk-local gradients: on the tensor cores for every chunk that
+    // decays within e^80 (per-channel gate), then the token-by-token kernel for
+    // the rest (all chunks for a scalar gate)
+    uint32_t *slow = reinterpret_cast<uint32_t *>(ws + l.slow);
+    if (!scalar_gate) {
+        if ((e = cudaMemsetAsync(slow, 0, l.max_chunks * H * sizeof(uint32_t), stream)) != cudaSuccess) return e;
+        e = launch_backward_tc(q, k, v, g, beta, d_o, total_tokens, H, tab.chunk_tab, tab.total_chunks,
+                               reinterpret_cast<const float *>(ws + l.s_in),
+                               reinterpret_cast<const float *>(ws + l.ds_next), dq, dk_out, dv_out, dg, dbeta,
+                               slow, reinterpret_cast<float *>(ws + l.gscr), reinterpret_cast<uint32_t *>(ws),
+                               l.grid_tc, stream);
+        if (e != cudaSuccess) return e;
+    }
     BwdArgs p = {};
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.d_o = d_o;
     p.dq = dq; p.dk = dk_out; p.dv = dv_out; p.dg = dg; p.dbeta = dbeta;
@@ -682,6 +710,7 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
     ca.tab = tab;
     ca.s_in = reinterpret_cast<const float *>(ws + l.s_in);
     ca.ds_next = reinterpret_cast<const float *>(ws + l.ds_next);
+    ca.only = scalar_gate ? nullptr : slow;
     ca.num_seqs = num_seqs;
     const size_t smem = BwdShape<128>::SMEM;
     if ((e = set_max_dynamic_smem((const void *)kda_backward_chunk_kernel<__nv_bfloat16, 128>, (int)smem)) !=

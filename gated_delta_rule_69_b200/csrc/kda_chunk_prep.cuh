@@ -66,6 +66,9 @@ struct Bufs {
     // The scalar (Gated DeltaNet) gate: one raw log_alpha per token, 64 fp32
     // (zero past the chunk end), or null for the per-channel gate in graw.
     const float *gsc;
+    // gate<BAR, LAYER, true> also writes the running sums G (base-2 units,
+    // fp32 [64 t][128 c] row-major) here, for the backward pass
+    float *gout;
 };
 
 // Index of A element (t, i): rows padded to 65 floats, so that a warp
@@ -90,7 +93,7 @@ __device__ __forceinline__ int tfi(int row, int col) { return row * kTStride + c
 // reference per block) or kPairwise.
 enum : int { kProductForm = 0, kSecondary = 1, kPairwise = 2 };
 
-template <int BAR, bool LAYER>
+template <int BAR, bool LAYER, bool GOUT = false>
 __device__ int gate(const Bufs &b, int pt, int L) {
     const int c = 2 * (pt & 63);
     const int tg = pt >> 6;
@@ -209,6 +212,7 @@ __device__ int gate(const Bufs &b, int pt, int L) {
         const float k0 = __low2float(kv) * nk, k1 = __high2float(kv) * nk;
         const float q0 = __low2float(qv) * nq, q1 = __high2float(qv) * nq;
         const float G0 = g0[i] + off0, G1 = g1[i] + off1;
+        if (GOUT) *reinterpret_cast<float2 *>(b.gout + t * 128 + c) = make_float2(G0, G1);
         const float e0 = exp2_f(G0), e1 = exp2_f(G1);
         const float ih0 = exp2_f(fminf(-G0, kMaxInv2)), ih1 = exp2_f(fminf(-G1, kMaxInv2));
         // Kbar's factor e^{G_L - G}: a product of two factors, or (pairwise
@@ -441,7 +445,7 @@ __device__ __forceinline__ void load_row32(const __nv_bfloat16 *src, float (&v)[
 // the chunk for this head; row_stride is H * d_k elements).  All lanes of a
 // warp walk the same rows (from the warp's first column), so the shuffles
 // stay converged.
-__device__ void pairwise(const Bufs &b, int pt, int L, const __nv_bfloat16 *kt0,
+__device__ inline void pairwise(const Bufs &b, int pt, int L, const __nv_bfloat16 *kt0,
                          const __nv_bfloat16 *qt0, size_t row_stride) {
     const int i = pt >> 2, cg = pt & 3, c0 = 32 * cg;
     const bool lead = cg == 0;

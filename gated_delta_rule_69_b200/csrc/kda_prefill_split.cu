@@ -1552,6 +1552,12 @@ ChainPlan choose_chain(unsigned units, uint64_t items, int64_t total_tokens, int
 
 }  // namespace
 
+// A [T, H, inner] bf16 tensor as [64 tokens][box_inner] boxes (one head).
+bool make_bf16_map_3d(CUtensorMap *m, const void *base, int64_t T, int H, int inner, int box_inner,
+                      CUtensorMapSwizzle sw) {
+    return make_map_split(m, base, T, H, inner, box_inner, sw);
+}
+
 size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H) {
     return split_layout(num_seqs, total_tokens, H).total;
 }
