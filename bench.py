@@ -92,13 +92,54 @@ BWD_FLOP_PER_ELEM = 5 + 18
 FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
+# The chunk form of the backward pass (bf16, d = 128, C = 64) on the tensor
+# cores: per (chunk, head) the products its algebra takes, 2 m n k FLOP each.
+#   records:          [Ktil; Qtil] Khat^T, YT = Kbar^T T_beta, ZB = P T_beta,
+#                     MP = -YT Ktil, ZB Ktil
+#   forward scan:     MP S, YT V
+#   reverse scan:     MP^T dS, QP^T dO
+#   chunk gradients:  [Ktil; Qtil] Khat^T, Ktil S, Kbar dS_C, P^T dO,
+#                     T_beta R, T_beta^T dU, dU R^T, U dS_C^T, dO U^T, dT T^T,
+#                     dO S^T, dR S^T, T^T Z, dP Khat, BdA Khat, dP^T Qtil, BdA^T Ktil
+def _mm(m, n, k):
+    return 2 * m * n * k
+
+
+def chunk_backward_flop(C=64, d=128):
+    rec = _mm(2 * C, C, d) + _mm(d, C, C) + _mm(C, C, C) + _mm(d, d, C) + _mm(C, d, C)
+    scans = 2 * (_mm(d, d, d) + _mm(d, d, C))
+    local = _mm(2 * C, C, d) + 5 * _mm(C, d, d) + 9 * _mm(C, C, d) + 2 * _mm(C, C, C)
+    return rec + scans + local
+
+
 def backward_work(w, lengths):
     T, n = sum(lengths), len(lengths)
     eb = 2 if w.dtype == "bf16" else 4
     per_tok = (3 * w.d_k + 2 * w.d_v) * eb + eb + (3 * w.d_k + w.d_v + 1) * 4
     states = n * w.H * w.d_k * w.d_v * 4 * 3
+    chunks = sum((L + 63) // 64 for L in lengths)
     return dict(tokens=T, flop=BWD_FLOP_PER_ELEM * w.d_k * w.d_v * T * w.H,
+                chunk_flop=chunk_backward_flop() * chunks * w.H,
                 bytes=per_tok * T * w.H + states)
+
+
+def backward_roofline(work, ms, peaks, src):
+    """The chunked pass against the bf16 tensor peak (its chunk-form
+    products), the sequential one against the fp32 CUDA-core rate."""
+    if work.get("chunked"):
+        tf = work["chunk_flop"] / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": tf, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                "frac": tf / peaks["bf16"], "traffic": None, "peak_source": src + " (bf16 burst)",
+                "kernel": "kda_backward_chunked", "algorithmic_flop_per_launch": work["chunk_flop"],
+                "algorithmic_bytes_per_launch": work["bytes"],
+                "hbm_frac": work["bytes"] / (ms * 1e-3) / 1e9 / peaks["hbm"]}
+    tf = work["flop"] / (ms * 1e-3) / 1e12
+    return {"bound": "alu", "achieved": tf, "peak": FP32_SIMT_TFLOPS, "unit": "TFLOP/s",
+            "frac": tf / FP32_SIMT_TFLOPS, "traffic": None,
+            "peak_source": "nominal fp32 CUDA-core rate (148 SMs x 128 lanes x 2 x 1.965 GHz)",
+            "kernel": "kda_backward", "algorithmic_flop_per_launch": work["flop"],
+            "algorithmic_bytes_per_launch": work["bytes"],
+            "hbm_frac": work["bytes"] / (ms * 1e-3) / 1e9 / peaks["hbm"]}
 
 
 def decode_work(w):
@@ -333,9 +374,11 @@ def time_backward(w, steps, warmup, world):
     if kda.kda_check_workspace_error(ws) != kda.KDA_OK:
         raise RuntimeError("device-side check failed during the backward benchmark")
     ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    # the gradient zeroing is four memsets, not counted
-    return dict(ms_total=sum(ms), ms=ms, lengths=inp["lengths"],
-                launches=steps * (5 if chunked else 1))
+    # chunked: the plan, the preparation, two scans, the tensor-core chunk
+    # kernel and the step kernel for chunks it leaves; the gradient zeroing
+    # (memsets) is not counted
+    return dict(ms_total=sum(ms), ms=ms, lengths=inp["lengths"], chunked=chunked,
+                launches=steps * (6 if chunked else 1))
 
 
 def time_prefill_e2e(w, steps, warmup):
@@ -608,8 +651,8 @@ def main():
     lms = max_over_ranks(lay["ms_total"] / args.steps, world)
     lgbs = lwork["bytes"] / (lms * 1e-3) / 1e9
     bwork = backward_work(bw, bwd["lengths"])
+    bwork["chunked"] = bwd["chunked"]
     bms = max_over_ranks(bwd["ms_total"] / len(bwd["ms"]), world)
-    btfs = bwork["flop"] / (bms * 1e-3) / 1e12
     src = "of " + peaks["source"]
 
     line = {
@@ -648,14 +691,7 @@ def main():
         "backward": {"workload": bw.name + ", backward pass (kda_backward_chunked for bf16 d = 128), seeded upstream gradients",
                      "value": world * bwork["tokens"] / (bms * 1e-3), "unit": "tokens/s",
                      "ms_per_step": bms, "steps": len(bwd["ms"]),
-                     "roofline": {"bound": "alu", "achieved": btfs, "peak": FP32_SIMT_TFLOPS,
-                                  "unit": "TFLOP/s", "frac": btfs / FP32_SIMT_TFLOPS,
-                                  "traffic": None,
-                                  "peak_source": "nominal fp32 CUDA-core rate (148 SMs x 128 lanes x 2 x 1.965 GHz)",
-                                  "kernel": "kda_backward_chunked",
-                                  "algorithmic_flop_per_launch": bwork["flop"],
-                                  "algorithmic_bytes_per_launch": bwork["bytes"],
-                                  "hbm_frac": bwork["bytes"] / (bms * 1e-3) / 1e9 / peaks["hbm"]}},
+                     "roofline": backward_roofline(bwork, bms, peaks, src)},
         "gpu_launches": pf["launches"] + dec["launches"] + gdn["launches"] + lay["launches"]
                         + bwd["launches"] + sum(x[2]["launches"] for x in extra)
                         + (bwd_long["launches"] if bwd_long else 0),
@@ -663,18 +699,13 @@ def main():
     }
     if bwd_long:
         lwk = backward_work(w, bwd_long["lengths"])
+        lwk["chunked"] = bwd_long["chunked"]
         lbms = max_over_ranks(bwd_long["ms_total"] / len(bwd_long["ms"]), world)
-        ltfs = lwk["flop"] / (lbms * 1e-3) / 1e12
         line["backward_long"] = {
             "workload": w.name + ", backward pass (kda_backward_chunked), seeded upstream gradients",
             "value": world * lwk["tokens"] / (lbms * 1e-3), "unit": "tokens/s", "ms_per_step": lbms,
             "steps": len(bwd_long["ms"]),
-            "roofline": {"bound": "alu", "achieved": ltfs, "peak": FP32_SIMT_TFLOPS, "unit": "TFLOP/s",
-                         "frac": ltfs / FP32_SIMT_TFLOPS, "traffic": None,
-                         "peak_source": "nominal fp32 CUDA-core rate (148 SMs x 128 lanes x 2 x 1.965 GHz)",
-                         "kernel": "kda_backward_chunked",
-                         "algorithmic_flop_per_launch": lwk["flop"],
-                         "algorithmic_bytes_per_launch": lwk["bytes"]}}
+            "roofline": backward_roofline(lwk, lbms, peaks, src)}
     for key, ew, r in extra:
         ework = prefill_work(ew, r["inputs"]["lengths"])
         ems = max_over_ranks(r["ms_total"] / args.steps, world)

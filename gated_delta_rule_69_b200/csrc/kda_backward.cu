@@ -37,7 +37,7 @@ namespace kda {
 size_t backward_tc_scratch(int grid);
 cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, const void *g, const void *beta,
                                const void *d_o, int64_t total_tokens, int H, const int2 *chunk_tab,
-                               const uint32_t *total_chunks, const float *s_in, const float *ds_next, float *dq,
+                               const uint32_t *total_chunks, const uint8_t *s_in, const uint8_t *ds_next, float *dq,
                                float *dk, float *dv, float *dg, float *dbeta, uint32_t *slow, float *gscr,
                                uint32_t *err_word, int grid, cudaStream_t stream);
 
@@ -78,6 +78,12 @@ struct BwdArgs {
 };
 
 __device__ __forceinline__ float4 f4(float x) { return make_float4(x, x, x, x); }
+
+// Byte offset of element (row, col) in a 128-byte-swizzled K-atom of 64
+// bf16 columns (the layout the backward scans write the states in).
+__device__ __forceinline__ uint32_t sw128_tile_off(uint32_t row, uint32_t col) {
+    return row * 128u + (((col >> 3) ^ (row & 7u)) << 4) + (col & 7u) * 2u;
+}
 __device__ __forceinline__ float4 sub4(float4 a, float4 b) {
     return make_float4(a.x - b.x, a.y - b.y, a.z - b.z, a.w - b.w);
 }
@@ -500,8 +506,8 @@ cudaError_t launch_dk(const BwdArgs &p, int grid, cudaStream_t stream) {
 
 struct ChunkArgs {
     SplitTables tab;
-    const float *s_in;     // [max_chunks, H, 128, 128] entering states
-    const float *ds_next;  // [max_chunks, H, 128, 128] dL/dS at each chunk's end
+    const uint8_t *s_in;     // entering states, bf16 tiles (launch_backward_scans)
+    const uint8_t *ds_next;  // dL/dS at each chunk's end, bf16 tiles
     const uint32_t *only;  // [max_chunks * H] or null: run only the (chunk, head) items flagged 1
     int num_seqs;
 };
@@ -529,12 +535,14 @@ __global__ void __launch_bounds__(kBwdThreads, 2) kda_backward_chunk_kernel(cons
         const int2 ct = c.tab.chunk_tab[ch];
         const int64_t tb = ct.x, te = (int64_t)ct.x + ct.y;
         const int j0 = s * kBwdSlice + warp * kBwdCols;
-        const size_t base = ((size_t)ch * p.H + h) * DK * p.dv_total + j0;
+        // the 4 columns j0 .. j0 + 3 of row c share one 16-byte piece of the tile
+        const size_t tile = ((size_t)ch * p.H + h) * 32768 + (size_t)(j0 >> 6) * 16384;
         float4 S[RPL], dS[RPL];
 #pragma unroll
         for (int i = 0; i < RPL; ++i) {
-            S[i] = *reinterpret_cast<const float4 *>(c.s_in + base + (size_t)(lane + 32 * i) * p.dv_total);
-            dS[i] = *reinterpret_cast<const float4 *>(c.ds_next + base + (size_t)(lane + 32 * i) * p.dv_total);
+            const uint32_t off = sw128_tile_off(lane + 32 * i, j0 & 63);
+            S[i] = to_f4(*reinterpret_cast<const uint2 *>(c.s_in + tile + off));
+            dS[i] = to_f4(*reinterpret_cast<const uint2 *>(c.ds_next + tile + off));
         }
         block_backward<T, DK, kBwdChunkSub>(S, dS, p, tb, te, tb, h, warp, lane, j0, idx, scratch, red,
                                             buf, gi, g_hi);
@@ -633,7 +641,7 @@ struct ChunkedLayout {
 ChunkedLayout chunked_layout(int num_seqs, int64_t total_tokens, int H) {
     ChunkedLayout l;
     l.max_chunks = (size_t)(total_tokens / kBwdBlock) + (size_t)num_seqs;
-    const size_t state = (size_t)128 * 128 * sizeof(float);
+    const size_t state = (size_t)128 * 128 * sizeof(__nv_bfloat16);   // a bf16 tile per record
     const int64_t units = (int64_t)l.max_chunks * H * (128 / kBwdSlice);
     l.grid = (int)(units < kBwdMaxCtas ? units : kBwdMaxCtas);
     l.split = 0;
@@ -679,8 +687,7 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
     // chain, forward and reverse): every chunk's entering state and dL/dS at
     // its end, and a first dL/dS_0 per sequence
     e = launch_backward_scans(v, d_o, init_state, d_final_state, cu, num_seqs, total_tokens, H,
-                              ws + l.split, reinterpret_cast<float *>(ws + l.s_in),
-                              reinterpret_cast<float *>(ws + l.ds_next), d_init_state, stream);
+                              ws + l.split, ws + l.s_in, ws + l.ds_next, d_init_state, stream);
     if (e != cudaSuccess) return e;
     // 3. the chunk-local gradients: on the tensor cores for every chunk that
     // decays within e^80 (per-channel gate), then the token-by-token kernel for
@@ -689,8 +696,7 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
     if (!scalar_gate) {
         if ((e = cudaMemsetAsync(slow, 0, l.max_chunks * H * sizeof(uint32_t), stream)) != cudaSuccess) return e;
         e = launch_backward_tc(q, k, v, g, beta, d_o, total_tokens, H, tab.chunk_tab, tab.total_chunks,
-                               reinterpret_cast<const float *>(ws + l.s_in),
-                               reinterpret_cast<const float *>(ws + l.ds_next), dq, dk_out, dv_out, dg, dbeta,
+                               ws + l.s_in, ws + l.ds_next, dq, dk_out, dv_out, dg, dbeta,
                                slow, reinterpret_cast<float *>(ws + l.gscr), reinterpret_cast<uint32_t *>(ws),
                                l.grid_tc, stream);
         if (e != cudaSuccess) return e;
@@ -708,8 +714,8 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
     p.scalar_gate = scalar_gate ? 1 : 0;
     ChunkArgs ca;
     ca.tab = tab;
-    ca.s_in = reinterpret_cast<const float *>(ws + l.s_in);
-    ca.ds_next = reinterpret_cast<const float *>(ws + l.ds_next);
+    ca.s_in = ws + l.s_in;
+    ca.ds_next = ws + l.ds_next;
     ca.only = scalar_gate ? nullptr : slow;
     ca.num_seqs = num_seqs;
     const size_t smem = BwdShape<128>::SMEM;

@@ -24,14 +24,19 @@
 //   dG = dKtil.Ktil + dQtil.Qtil - dKhat.Khat - dKbar.Kbar
 //   dg_t = sum_{s >= t} dG_s + sum_s dKbar.Kbar|_s + e^{G_L} rowsum(S .* dS_C)
 //
-// Five rounds of products, each one commit: {Ktil S, dU}, {U, dR, dT_beta},
-// {dKbar, dP, dT T^T, [dO; -dR] S^T}, {T^T Z}, {[dP; BdA] Khat, dKhat}.  A
-// round's results are read from TMEM by the warps of quadrants 0 and 1 (rows
-// 0-63; the M = 128 products' rows 64-127 multiply whatever follows an
-// operand in shared memory and are not read), converted to bf16 tiles and
-// fed to the next round.  Two products are stacked to fill all 128 rows:
-// [dO; -dR] S^T and [dP; BdA] Khat accumulate into one TMEM tile whose rows
-// 0-63 are dQtil and rows 64-127 dKtil.
+// Five rounds of products: {Ktil S, dU}, {U, dR, dT_beta}, {dP, dT T^T},
+// {T^T Z}, {dKhat}; the products the gradients need only at the end are
+// issued early and committed apart.  The first rounds' results (64 x 64 and
+// 64 x 128, token in the TMEM lane) are read by the warps of quadrants 0 and
+// 1 (the M = 128 products' rows 64-127 multiply whatever follows an operand
+// in shared memory and are not read), converted to bf16 tiles and fed to the
+// next round.  The final ones are formed transposed, channel in the lane
+// (M = 128 = d_k): dKbar^T = dS_C U^T, [dQtil^T | dKtil^T] = S [dO; -dR]^T +
+// Khat^T [dP; BdA]^T (one N = 128 tile), dKhat^T = Qtil^T dP + Ktil^T BdA, so
+// that every warp combines them, each thread one channel and 32 tokens, with
+// the running sum of dG along its own tokens.  S and dS_C arrive as bf16
+// tiles (the scans write them in this layout) by bulk copies issued while
+// the previous item's gradients are combined.
 //
 // A chunk that decays below e^-80 within itself on some channel (the
 // prefill's slow forms: Khat's factor would overflow) is left to the
@@ -57,8 +62,11 @@ constexpr int kThreads = 256;
 constexpr uint32_t BAR = 1;   // named barrier of the CTA's 256 threads
 
 // Shared memory (bytes; tiles bf16, K-major, 128-byte swizzle, 64 columns per
-// K-atom).  Phase A (the prefill's preparation: gating, [A; P], the solve)
-// and phase B (the products) share the region from AF on.
+// K-atom).  S and dS_C arrive as such tiles (the scans write them so) by bulk
+// copies issued one item ahead; the region from DU on serves phase A (the
+// prefill's preparation: gating, [A; P], the solve) and then phase B (the
+// products).  dU and U serve as M = 128 A operands whose rows 64-127 read the
+// 8 KB after each K-atom, so each is followed by another tile.
 struct Sm {
     static constexpr uint32_t STK = 0;         // [Ktil rows 0-63 | Qtil rows 64-127], 2 x 16 KB
     static constexpr uint32_t KHAT = 32768;    // Khat [64 t][128 c], 2 x 8 KB
@@ -66,51 +74,49 @@ struct Sm {
     static constexpr uint32_t TB16 = 57344;    // T [64 t][64 i]
     static constexpr uint32_t KBAR = 65536;    // Kbar [64][128], then R, then PA = [dP; BdA] [128][64]
     static constexpr uint32_t PB = 81920;      // P [64 t][64 i], then dT
+    static constexpr uint32_t S0 = 90112;      // S [128 c][128 j], 2 x 16 KB
+    static constexpr uint32_t DSC = 122880;    // dS_C [128 c][128 j], 2 x 16 KB
     // phase A
-    static constexpr uint32_t AF = 90112;      // A fp32, rows of 65
-    static constexpr uint32_t TF = 107520;     // T fp32, rows of 68
-    static constexpr uint32_t GRAW = 124928;   // raw log_alpha [64][128] bf16
-    static constexpr uint32_t XF = 141312;     // solve scratch (4608 bytes)
+    static constexpr uint32_t AF = 155648;     // A fp32, rows of 65
+    static constexpr uint32_t TF = 172288;     // T fp32, rows of 68
+    static constexpr uint32_t GRAW = 190464;   // raw log_alpha [64][128] bf16
+    static constexpr uint32_t XF = 206848;     // solve scratch (4608 bytes)
     // phase B
-    // (dU and U serve as M = 128 A operands whose rows 64-127 read the 8 KB
-    // after each K-atom: each is followed by another tile, not by the end)
-    static constexpr uint32_t S0 = 90112;      // S [128 c][128 j], 2 x 16 KB; then the final exchange
-    static constexpr uint32_t DOR = 122880;    // [dO rows 0-63 | -dR rows 64-127] [128][128], 2 x 16 KB
     static constexpr uint32_t DU = 155648;     // dU [64 t][128 j], 2 x 8 KB
     static constexpr uint32_t U = 172032;      // U [64 t][128 j], 2 x 8 KB
-    static constexpr uint32_t DSC = 188416;    // dS_C [128 c][128 j], 2 x 16 KB
-    static constexpr uint32_t XCH = S0;        // fp32 [64 t][128 c] (32 KB), 16-byte pieces swizzled
+    static constexpr uint32_t DOR = 188416;    // [dO rows 0-63 | -dR rows 64-127] [128][128], 2 x 16 KB
     static constexpr uint32_t BETA = 221184;   // 64 fp32
     static constexpr uint32_t EGL = 221440;    // 128 fp32: e^{G_L}
-    static constexpr uint32_t CSUM = 221952;   // 4 x 128 fp32
+    static constexpr uint32_t CSUM = 221952;   // 4 x 128 fp32 (the gate's; the final exchange after)
     static constexpr uint32_t DB = 224000;     // 64 fp32: dbeta of the item
-    static constexpr uint32_t DGL = 224256;    // 128 fp32: column sums of dKbar.Kbar
     static constexpr uint32_t ES = 224768;     // 128 fp32: rowsum(S .* dS_C)
-    static constexpr uint32_t BARS = 225280;   // mbarriers: raw loads, dO, products
+    static constexpr uint32_t BARS = 225280;   // mbarriers
     static constexpr uint32_t MISC = 225344;   // tmem base, abort, slow flag
     static constexpr uint32_t SIZE = 225408;
     static constexpr uint32_t ALLOC = SIZE + 1024;
 };
 static_assert(Sm::ALLOC <= 232448, "shared memory");
 static_assert(Sm::AF + 64 * prep::kAStride * 4 <= Sm::TF && Sm::TF + 64 * prep::kTStride * 4 <= Sm::GRAW &&
-                  Sm::GRAW + 16384 <= Sm::XF && Sm::XF + 4608 <= Sm::DU,
+                  Sm::GRAW + 16384 <= Sm::XF && Sm::XF + 4608 <= Sm::BETA && Sm::TF % 16 == 0,
               "phase A buffers");
-static_assert(Sm::DU + 16384 == Sm::U && Sm::U + 16384 == Sm::DSC && Sm::DSC + 32768 <= Sm::BETA &&
-                  Sm::XCH + 32768 <= Sm::GRAW,
+static_assert(Sm::DU + 16384 == Sm::U && Sm::U + 16384 == Sm::DOR && Sm::DOR + 32768 <= Sm::BETA &&
+                  Sm::DU + 32768 <= Sm::GRAW &&
+                  Sm::S0 + 32768 == Sm::DSC && Sm::DSC + 32768 <= Sm::DU && Sm::PB + 8192 == Sm::S0,
               "phase B buffers");
 
-// TMEM columns (512): [A; P] (KK in rows 0-63) until round 3; the stacked
-// [dQtil; dKtil]; then per round the products listed.
-constexpr uint32_t kColAP = 0;
-constexpr uint32_t kColD1 = 64;     // rows 0-63 dQtil, 64-127 dKtil
-constexpr uint32_t kColX = 192;     // Ktil S (round 0), U (1), dKbar (2 - end)
-constexpr uint32_t kColY = 320;     // dU (0), dR (1), dP (2, 64 cols), dKhat (4 - end)
+// TMEM columns (512).  Rounds 0 and 1 give row-major (token in the lane)
+// results; the final ones are transposed (channel in the lane), so that all
+// eight warps combine them.
+constexpr uint32_t kColAP = 0;      // [A; P] (KK in rows 0-63) until round 3
+constexpr uint32_t kColD1 = 64;     // [dQtil^T | dKtil^T] [128 c][64 t | 64 t] (rounds 2 and 4)
+constexpr uint32_t kColX = 192;     // Ktil S (round 0), U (1), dKbar^T [c][t] (2 - end, 64 cols)
+constexpr uint32_t kColY = 320;     // dU (0), dR (1), dP (2, 64 cols), dKhat^T [c][t] (4 - end, 64 cols)
 constexpr uint32_t kColZ = 384;     // Z (2, 64 cols)
 constexpr uint32_t kColW = 448;     // dT_beta (1), T^T Z (3)
 
 struct Args {
     const __nv_bfloat16 *q, *k, *v, *g, *beta, *d_o;
-    const float *s_in, *ds_next;     // [record][128][128] fp32, record = chunk * H + head
+    const uint8_t *s_in, *ds_next;   // bf16 tiles, 32 KB per record (record = chunk * H + head)
     const int2 *chunk_tab;
     const uint32_t *total_chunks;
     float *dq, *dk, *dv, *dg, *dbeta;
@@ -166,11 +172,6 @@ __device__ __forceinline__ void gload32(const __nv_bfloat16 *src, bool valid, fl
     }
 }
 
-// fp32 [64 t][128 c] exchange tile: 16-byte piece p of row t at piece p ^ (t mod 32)
-__device__ __forceinline__ float4 *xch_at(uint8_t *sm, int t, int piece) {
-    return reinterpret_cast<float4 *>(sm + Sm::XCH + t * 512 + ((piece ^ (t & 31)) << 4));
-}
-
 // Sums v[j] over the warp's 32 lanes for j = 0..31; lane l returns the sum of v[l].
 __device__ __forceinline__ float column_sums(float (&v)[32], int lane) {
 #pragma unroll
@@ -185,6 +186,19 @@ __device__ __forceinline__ float column_sums(float (&v)[32], int lane) {
         }
     }
     return v[0];
+}
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
+}
+
+// S and dS_C of an item (64 KB) into their tiles
+__device__ __forceinline__ void issue_states(uint8_t *sm, uint64_t *bar, const Args &p, uint32_t item) {
+    mbar_arrive_expect_tx(bar, 65536);
+    bulk_load(sm + Sm::S0, p.s_in + (size_t)item * 32768, 32768, bar);
+    bulk_load(sm + Sm::DSC, p.ds_next + (size_t)item * 32768, 32768, bar);
 }
 
 __device__ __forceinline__ void issue_raw(uint8_t *sm, uint64_t *bar, const CUtensorMap &tm_k,
@@ -210,18 +224,19 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     const int quad = warp & 3, half = warp >> 2;
     const bool leader = pt == 0;
     uint64_t *BLD = reinterpret_cast<uint64_t *>(sm + Sm::BARS);
-    uint64_t *BDO = BLD + 1, *BMMA = BLD + 2;
+    uint64_t *BDO = BLD + 1, *BMMA = BLD + 2, *BMMA2 = BLD + 3, *BSD = BLD + 4;
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + Sm::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     float *beta = reinterpret_cast<float *>(sm + Sm::BETA);
     float *egl = reinterpret_cast<float *>(sm + Sm::EGL);
     float *db = reinterpret_cast<float *>(sm + Sm::DB);
-    float *dgl = reinterpret_cast<float *>(sm + Sm::DGL);
     float *es = reinterpret_cast<float *>(sm + Sm::ES);
     if (leader) {
         mbar_init(BLD, 3);   // the leader's copies, one arrive per beta warp
         mbar_init(BDO, 1);
         mbar_init(BMMA, 1);
+        mbar_init(BMMA2, 1);
+        mbar_init(BSD, 1);
         misc[1] = 0u;
         fence_mbar_init();
         tma_prefetch_desc(&tm_k);
@@ -239,7 +254,7 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     const uint32_t tmem = misc[0];
     const uint32_t total = *p.total_chunks * (uint32_t)p.H;
     float *gscr = p.gscr + (size_t)blockIdx.x * (C * DK);
-    uint32_t n_mma = 0, n_do = 0;   // completed phases of BMMA, BDO
+    uint32_t n_mma = 0, n_mma2 = 0, n_sd = 0, n_do = 0;   // completed phases of BMMA, BMMA2, BSD, BDO
     auto mma_wait = [&]() {
         mbar_wait(BMMA, n_mma & 1u, abort_flag);
         ++n_mma;
@@ -252,7 +267,10 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         named_barrier(BAR, kThreads);
     };
 
-    if (leader && blockIdx.x < total) issue_raw(sm, BLD, tm_k, tm_q, tm_g, p, blockIdx.x);
+    if (leader && blockIdx.x < total) {
+        issue_raw(sm, BLD, tm_k, tm_q, tm_g, p, blockIdx.x);
+        issue_states(sm, BSD, p, blockIdx.x);
+    }
 #pragma unroll 1
     for (uint32_t item = blockIdx.x, it = 0; item < total; item += gridDim.x, ++it) {
         const int h = (int)(item % (uint32_t)p.H);
@@ -266,8 +284,6 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
             db[pt] = 0.f;
             __syncwarp();
             if (lane == 0) mbar_arrive(BLD);
-        } else if (pt < C + 128) {
-            dgl[pt - C] = 0.f;
         }
         prep::Bufs b = {};
         b.stk = sm + Sm::STK;
@@ -289,9 +305,15 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         fence_async_smem();
         named_barrier(BAR, kThreads);
         if (form != prep::kProductForm) {   // left to the step kernel
+            mbar_wait(BSD, n_sd & 1u, abort_flag);   // the item's states have landed
+            ++n_sd;
+            named_barrier(BAR, kThreads);
             if (leader) {
                 p.slow[item] = 1u;
-                if (next < total) issue_raw(sm, BLD, tm_k, tm_q, tm_g, p, next);
+                if (next < total) {
+                    issue_raw(sm, BLD, tm_k, tm_q, tm_g, p, next);
+                    issue_states(sm, BSD, p, next);
+                }
             }
             continue;
         }
@@ -331,29 +353,26 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         }
         named_barrier(BAR, kThreads);   // phase A's fp32 buffers are free
 
-        // ---- phase B inputs: dO by TMA, S and dS_C converted to bf16
+        // ---- phase B inputs: dO by TMA over phase A's buffers; S and dS_C (bulk
+        // copies issued an item ahead) give rowsum(S .* dS_C)
         if (leader) {
             mbar_arrive_expect_tx(BDO, 16384);
             tma_load_3d(sm + Sm::DOR, &tm_do, BDO, 0, h, (int)tok0);
             tma_load_3d(sm + Sm::DOR + 16384, &tm_do, BDO, 64, h, (int)tok0);
         }
+        mbar_wait(BSD, n_sd & 1u, abort_flag);
+        ++n_sd;
         {
-            const size_t rec = (size_t)chunk * p.H + h;
-            const int c = pt >> 1, j0 = (pt & 1) * 64;
-            const float4 *s4 = reinterpret_cast<const float4 *>(p.s_in + (rec * DK + c) * 128 + j0);
-            const float4 *d4 = reinterpret_cast<const float4 *>(p.ds_next + (rec * DK + c) * 128 + j0);
-            uint8_t *sa = sm + Sm::S0 + (pt & 1) * 16384, *da = sm + Sm::DSC + (pt & 1) * 16384;
+            const int c = pt >> 1;
+            const uint8_t *sa = sm + Sm::S0 + (pt & 1) * 16384, *da = sm + Sm::DSC + (pt & 1) * 16384;
+            float sv[32], dv[32];
             float dot = 0.f;
 #pragma unroll
-            for (int j = 0; j < 64; j += 8) {
-                const float4 a0 = s4[j / 4], a1 = s4[j / 4 + 1];
-                const float4 b0 = d4[j / 4], b1 = d4[j / 4 + 1];
-                const float sv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                const float dv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            for (int j = 0; j < 64; j += 32) {
+                get32(sa, c, j, sv);
+                get32(da, c, j, dv);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) dot = fmaf(sv[e], dv[e], dot);
-                *reinterpret_cast<uint4 *>(sa + sw128_off(c, j)) = pack8(sv);
-                *reinterpret_cast<uint4 *>(da + sw128_off(c, j)) = pack8(dv);
+                for (int e = 0; e < 32; ++e) dot = fmaf(sv[e], dv[e], dot);
             }
             dot += __shfl_xor_sync(0xffffffffu, dot, 1);
             if ((pt & 1) == 0) es[c] = dot;
@@ -469,27 +488,33 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         }
         round_barrier();
 
-        // ---- round 2: dKbar = U dS_C^T, dP = dO U^T, Z = dT T^T, [dO; -dR] S^T
+        // ---- round 2: dP = dO U^T and Z = dT T^T (one commit: the next rounds
+        // wait for them), then, transposed, dKbar^T = dS_C U^T and
+        // [dQtil^T | dKtil^T] = S [dO; -dR]^T (a second commit, waited for only
+        // before the gradients)
         if (warp == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {   // K = 128 (j)
-                const uint64_t aUk = smem_desc(aU + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128);
-                const uint64_t aDk = smem_desc(aDOR + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128);
-                mma_bf16_warp(tmem + kColX, aUk,
-                              smem_desc(aDSC + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                              idesc_bf16(128, 128, false, false), ks > 0 ? 1u : 0u);
-                mma_bf16_warp(tmem + kColY, aDk, aUk, idesc_bf16(128, 64, false, false), ks > 0 ? 1u : 0u);
-                mma_bf16_warp(tmem + kColD1, aDk,
-                              smem_desc(aS0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                              idesc_bf16(128, 128, false, false), ks > 0 ? 1u : 0u);
-            }
+            for (int ks = 0; ks < 8; ++ks)   // K = 128 (j)
+                mma_bf16_warp(tmem + kColY, smem_desc(aDOR + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(aU + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              idesc_bf16(128, 64, false, false), ks > 0 ? 1u : 0u);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)   // K = 64 (k)
                 mma_bf16_warp(tmem + kColZ, smem_desc(aPB + ks * 32, 16, 1024, kLayoutSW128),
                               smem_desc(aT16 + ks * 32, 16, 1024, kLayoutSW128), idesc_bf16(128, 64, false, false),
                               ks > 0 ? 1u : 0u);
             mma_commit_warp(BMMA);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {   // K = 128 (j)
+                mma_bf16_warp(tmem + kColX, smem_desc(aDSC + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(aU + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              idesc_bf16(128, 64, false, false), ks > 0 ? 1u : 0u);
+                mma_bf16_warp(tmem + kColD1, smem_desc(aS0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              smem_desc(aDOR + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+                              idesc_bf16(128, 128, false, false), ks > 0 ? 1u : 0u);
+            }
+            mma_commit_warp(BMMA2);
         }
         mma_wait();
         if (quad < 2) {
@@ -539,108 +564,100 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         }
         round_barrier();
 
-        // ---- round 4: [dQtil; dKtil] += [dP; BdA] Khat, dKhat = dP^T Qtil + BdA^T Ktil
+        // ---- round 4, transposed: [dQtil^T | dKtil^T] += Khat^T [dP; BdA]^T,
+        // dKhat^T = Qtil^T dP + Ktil^T BdA
         if (warp == 0) {
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)   // K = 64 (i)
-                mma_bf16_warp(tmem + kColD1, smem_desc(aKB + ks * 32, 16, 1024, kLayoutSW128),
-                              smem_desc(aKH + ks * 2048, 8192, 1024, kLayoutSW128), idesc_bf16(128, 128, false, true),
+                mma_bf16_warp(tmem + kColD1, smem_desc(aKH + ks * 2048, 8192, 1024, kLayoutSW128),
+                              smem_desc(aKB + ks * 32, 16, 1024, kLayoutSW128), idesc_bf16(128, 128, true, false),
                               1u);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)   // K = 64 (t)
-                mma_bf16_warp(tmem + kColY, smem_desc(aKB + ks * 2048, 8192, 1024, kLayoutSW128),
-                              smem_desc(aSTK + 8192 + ks * 2048, 16384, 1024, kLayoutSW128),
-                              idesc_bf16(128, 128, true, true), ks > 0 ? 1u : 0u);
+                mma_bf16_warp(tmem + kColY, smem_desc(aSTK + 8192 + ks * 2048, 16384, 1024, kLayoutSW128),
+                              smem_desc(aKB + ks * 2048, 8192, 1024, kLayoutSW128), idesc_bf16(128, 64, true, true),
+                              ks > 0 ? 1u : 0u);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16_warp(tmem + kColY, smem_desc(aKB + 8192 + ks * 2048, 8192, 1024, kLayoutSW128),
-                              smem_desc(aSTK + ks * 2048, 16384, 1024, kLayoutSW128), idesc_bf16(128, 128, true, true),
-                              1u);
+                mma_bf16_warp(tmem + kColY, smem_desc(aSTK + ks * 2048, 16384, 1024, kLayoutSW128),
+                              smem_desc(aKB + 8192 + ks * 2048, 8192, 1024, kLayoutSW128),
+                              idesc_bf16(128, 64, true, true), 1u);
             mma_commit_warp(BMMA);
         }
         mma_wait();
-        // the next item's k, q, log_alpha go over tiles no product reads again
-        if (leader && next < total) issue_raw(sm, BLD, tm_k, tm_q, tm_g, p, next);
+        // round 4's commit tracks every product issued before it, round 2's second
+        // group included; its barrier phase is consumed here
+        mbar_wait(BMMA2, n_mma2 & 1u, abort_flag);
+        ++n_mma2;
+        // the next item's inputs go over tiles no product reads again
+        if (leader && next < total) {
+            issue_raw(sm, BLD, tm_k, tm_q, tm_g, p, next);
+            issue_states(sm, BSD, p, next);
+        }
 
-        // ---- the gradients
-        if (quad >= 2) {   // dKtil e^G (rows 64-127 of the stacked tile) into the exchange
-            const int t = 32 * (quad - 2) + lane;
+        // ---- the gradients: thread (quad, half, lane) owns channel c = 32 quad
+        // + lane (its TMEM lane) and tokens t0 .. t0 + 31
+        {
+            const int c = 32 * quad + lane;
+            const int t0 = 32 * half;
+            const float el = egl[c];
+            // dG [64 t][128 c] fp32 over dU and U (free past round 4)
+            float *dGs = reinterpret_cast<float *>(sm + Sm::DU);
+            float sx = 0.f, up = 0.f;
+#pragma unroll 1
+            for (int pass = 0; pass < 2; ++pass) {
+                const int tp = t0 + 16 * pass;
+                float dQ[16], dKt[16], dKh[16], dKb[16], G[16], kr[16], qr[16];
+                tmem_ld16(tmem_addr(tmem + kColD1, 32 * quad, tp), dQ);
+                tmem_ld16(tmem_addr(tmem + kColD1, 32 * quad, 64 + tp), dKt);
+                tmem_ld16(tmem_addr(tmem + kColY, 32 * quad, tp), dKh);
+                tmem_ld16(tmem_addr(tmem + kColX, 32 * quad, tp), dKb);
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * half + 32 * part;
-                float x[32];
-                tmem_ld32(tmem_addr(tmem + kColD1, 32 * quad, c0), x);
+                for (int i = 0; i < 16; ++i) {
+                    const int t = tp + i;
+                    const bool valid = t < L;
+                    const size_t e = ((size_t)(tok0 + t) * p.H + h) * 128 + c;
+                    G[i] = gscr[t * 128 + c];
+                    kr[i] = valid ? __bfloat162float(p.k[e]) : 0.f;
+                    qr[i] = valid ? __bfloat162float(p.q[e]) : 0.f;
+                }
                 tmem_wait_ld();
-                const float4 *G4 = reinterpret_cast<const float4 *>(gscr + t * 128 + c0);
 #pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const float4 G = G4[m];
-                    *xch_at(sm, t, c0 / 4 + m) = make_float4(x[4 * m] * prep::exp2_f(G.x), x[4 * m + 1] * prep::exp2_f(G.y),
-                                                             x[4 * m + 2] * prep::exp2_f(G.z), x[4 * m + 3] * prep::exp2_f(G.w));
+                for (int i = 0; i < 16; ++i) {
+                    const int t = tp + i;
+                    const float eG = prep::exp2_f(G[i]), eiG = prep::exp2_f(-G[i]);
+                    const float dq = dQ[i] * eG, X = dKt[i] * eG;
+                    const float hk = dKh[i] * eiG, bk = dKb[i] * (el * eiG);
+                    const float xb = kr[i] * bk;
+                    const float dGv = kr[i] * (X - hk) - xb + qr[i] * dq;
+                    dGs[t * 128 + c] = dGv;
+                    up += dGv;
+                    sx += xb;
+                    if (t < L) {
+                        const size_t e = ((size_t)(tok0 + t) * p.H + h) * 128 + c;
+                        p.dq[e] = dq;
+                        p.dk[e] = X + hk + bk;
+                    }
                 }
             }
+            // dg_t = sum_{s >= t} dG_s + sum_s dKbar.Kbar|_s + e^{G_L} rowsum(S .* dS_C):
+            // the second half's running total and each half's Kbar sum through
+            // shared memory (the gate's scratch, free here)
+            float *xs = reinterpret_cast<float *>(sm + Sm::CSUM);   // [2][128] Kbar sums, [128] upper total
+            xs[half * 128 + c] = sx;
+            if (half) xs[256 + c] = up;
+            named_barrier(BAR, kThreads);
+            float acc = xs[c] + xs[128 + c] + el * es[c] + (half ? 0.f : xs[256 + c]);
+#pragma unroll 4
+            for (int i = 31; i >= 0; --i) {
+                const int t = t0 + i;
+                acc += dGs[t * 128 + c];
+                if (t < L) p.dg[((size_t)(tok0 + t) * p.H + h) * 128 + c] = acc;
+            }
+            if (pt < L) p.dbeta[(size_t)(tok0 + pt) * p.H + h] = db[pt];
         }
         tc_fence_before();
-        named_barrier(BAR, kThreads);
-        if (quad < 2) {
-            tc_fence_after();
-            const int t = 32 * quad + lane;
-            const bool valid = t < L;
-            const size_t row = (size_t)(tok0 + t) * p.H + h;
-#pragma unroll 1
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * half + 32 * part;
-                float dQ[32], dKh[32], dKb[32], kr[32], qr[32];
-                tmem_ld32(tmem_addr(tmem + kColD1, 32 * quad, c0), dQ);
-                tmem_ld32(tmem_addr(tmem + kColY, 32 * quad, c0), dKh);
-                tmem_ld32(tmem_addr(tmem + kColX, 32 * quad, c0), dKb);
-                gload32(p.k + row * 128 + c0, valid, kr);
-                gload32(p.q + row * 128 + c0, valid, qr);
-                tmem_wait_ld();
-                const float4 *G4 = reinterpret_cast<const float4 *>(gscr + t * 128 + c0);
-                float xb[32];
-#pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const float4 G = G4[m];
-                    const float4 X = *xch_at(sm, t, c0 / 4 + m);
-                    const float Gs[4] = {G.x, G.y, G.z, G.w}, Xs[4] = {X.x, X.y, X.z, X.w};
-                    float dq4[4], dk4[4], dG4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = 4 * m + e;
-                        const float eG = prep::exp2_f(Gs[e]), eiG = prep::exp2_f(-Gs[e]);
-                        const float eb = egl[c0 + j] * eiG;
-                        const float hk = dKh[j] * eiG, bk = dKb[j] * eb;
-                        dq4[e] = dQ[j] * eG;
-                        dk4[e] = Xs[e] + hk + bk;
-                        xb[j] = kr[j] * bk;
-                        dG4[e] = kr[j] * (Xs[e] - hk) - xb[j] + qr[j] * dq4[e];
-                    }
-                    if (valid) {
-                        *reinterpret_cast<float4 *>(p.dq + row * 128 + c0 + 4 * m) =
-                            make_float4(dq4[0], dq4[1], dq4[2], dq4[3]);
-                        *reinterpret_cast<float4 *>(p.dk + row * 128 + c0 + 4 * m) =
-                            make_float4(dk4[0], dk4[1], dk4[2], dk4[3]);
-                    }
-                    *xch_at(sm, t, c0 / 4 + m) = make_float4(dG4[0], dG4[1], dG4[2], dG4[3]);
-                }
-                atomicAdd(&dgl[c0 + lane], column_sums(xb, lane));
-            }
-        }
-        named_barrier(BAR, kThreads);
-        if (pt < 128) {   // dg: the running sum from the chunk end, plus the terms of G_L
-            const int c = pt;
-            const float tot = dgl[c] + egl[c] * es[c];
-            float acc = 0.f;
-            for (int t = L - 1; t >= 0; --t) {
-                acc += reinterpret_cast<const float *>(xch_at(sm, t, c >> 2))[c & 3];
-                p.dg[((size_t)(tok0 + t) * p.H + h) * 128 + c] = acc + tot;
-            }
-        } else if (pt - 128 < L) {
-            const int t = pt - 128;
-            p.dbeta[(size_t)(tok0 + t) * p.H + h] = db[t];
-        }
         named_barrier(BAR, kThreads);
     }
     if (leader && *abort_flag) atomicOr(p.err_word, kDevErrTimeout);
@@ -658,7 +675,7 @@ size_t backward_tc_scratch(int grid) { return (size_t)grid * bwdtc::C * bwdtc::D
 
 cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, const void *g, const void *beta,
                                const void *d_o, int64_t total_tokens, int H, const int2 *chunk_tab,
-                               const uint32_t *total_chunks, const float *s_in, const float *ds_next, float *dq,
+                               const uint32_t *total_chunks, const uint8_t *s_in, const uint8_t *ds_next, float *dq,
                                float *dk, float *dv, float *dg, float *dbeta, uint32_t *slow, float *gscr,
                                uint32_t *err_word, int grid, cudaStream_t stream) {
     using namespace bwdtc;

@@ -163,12 +163,13 @@ SplitTables split_tables(const void *workspace, int num_seqs, int64_t total_toke
 // The backward pass's two scans over the records a kPrepOnly launch left in
 // `workspace`, on the tensor cores (the transposed state chain): every chunk's
 // entering state into s_in and dL/dS at every chunk's end into ds_next (both
-// [max_chunks, H, 128, 128] fp32, record order), dL/dS_0 into d_init_state
-// (or not, when null).
+// bf16 tiles [128 c][128 j] in the 128-byte-swizzled K-major layout of a
+// tensor-core operand, two 16 KB K-atoms of 64 j, 32 KB per record, record
+// order), dL/dS_0 into d_init_state (or not, when null).
 cudaError_t launch_backward_scans(const void *v, const void *d_o, const float *init_state,
                                   const float *d_final_state, const int32_t *cu, int num_seqs,
-                                  int64_t total_tokens, int H, void *workspace, float *s_in,
-                                  float *ds_next, float *d_init_state, cudaStream_t stream);
+                                  int64_t total_tokens, int H, void *workspace, void *s_in,
+                                  void *ds_next, float *d_init_state, cudaStream_t stream);
 
 // The fixed scratch array of kda_prefill_noalloc on the current device.
 void *noalloc_scratch();

@@ -161,8 +161,10 @@ struct Params {
     uint32_t *work_next;        // prep items handed out after each pipeline's first one
     uint32_t *err_word;
     // backward-pass scans of the transposed chain: each chunk's state written
-    // here, [record][128 c][128 j] fp32 (record = chunk * H + head)
-    float *states_out;
+    // here as a bf16 tile [128 c][128 j] (two 16 KB K-atoms of 64 j, 128-byte
+    // swizzle: the layout of a tensor-core operand), 32 KB per record
+    // (record = chunk * H + head)
+    uint8_t *states_out;
     int64_t total_tokens;
     int num_seqs, H;
 };
@@ -1170,10 +1172,10 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         for (int n = 0; n < nchunks; ++n) {
             if (SAVE || REV) {   // the state entering (forward) or leaving (reverse) this chunk
                 const int nn = REV ? nchunks - 1 - n : n;
-                float *dst = p.states_out + ((rec0 + nn) * p.H + h) * (size_t)(DK * DV) +
-                             (size_t)(32 * g) * DV + j;
+                uint8_t *tile = p.states_out + ((rec0 + nn) * p.H + h) * (size_t)32768 + (j >> 6) * 16384;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) dst[(size_t)i * DV] = S[i];
+                for (int i = 0; i < 32; ++i)
+                    *reinterpret_cast<__nv_bfloat16 *>(tile + sw128_off(32 * g + i, j & 63)) = __float2bfloat16(S[i]);
             }
             // SB_n^T: column COL_SB + 64 (n mod 2) + c / 2 holds (c, c + 1).  Its
             // previous contents, SB_{n-2}, were last read by chunk n - 2's
@@ -1581,8 +1583,8 @@ SplitTables split_tables(const void *workspace, int num_seqs, int64_t total_toke
 
 cudaError_t launch_backward_scans(const void *v, const void *d_o, const float *init_state,
                                   const float *d_final_state, const int32_t *cu, int num_seqs,
-                                  int64_t total_tokens, int H, void *workspace, float *s_in,
-                                  float *ds_next, float *d_init_state, cudaStream_t stream) {
+                                  int64_t total_tokens, int H, void *workspace, void *s_in,
+                                  void *ds_next, float *d_init_state, cudaStream_t stream) {
     using namespace split;
     const SplitLayout l = split_layout(num_seqs, total_tokens, H);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1604,7 +1606,7 @@ cudaError_t launch_backward_scans(const void *v, const void *d_o, const float *i
     Params pf = prm;
     pf.init_state = init_state;
     pf.final_state = nullptr;
-    pf.states_out = s_in;
+    pf.states_out = static_cast<uint8_t *>(s_in);
     cudaError_t e = launch_chain_t(v, total_tokens, H, pf, units, false, stream, kChainSaveS);
     if (e != cudaSuccess) return e;
     // dL/dS at each chunk's end: the reverse chain (launched after the forward
@@ -1613,7 +1615,7 @@ cudaError_t launch_backward_scans(const void *v, const void *d_o, const float *i
     Params pr = prm;
     pr.init_state = d_final_state;
     pr.final_state = d_init_state;
-    pr.states_out = ds_next;
+    pr.states_out = static_cast<uint8_t *>(ds_next);
     return launch_chain_t(d_o, total_tokens, H, pr, units, false, stream, kChainReverse);
 }
 

@@ -1,7 +1,10 @@
 """kda_backward_chunked (bf16, d = 128, chunk boundary states from the chunk
 records) against the fp64 oracle's derivative, at the bf16 tolerance: the
 boundary states carry the records' bf16 rounding, as the prefill's own states
-do (per (sequence, head) slice, max|x - ref| / max|ref| <= 2e-2)."""
+do (per (sequence, head) slice, max|x - ref| / max|ref| <= 2e-2).  The
+chunk-local gradients run on the tensor cores except for chunks that decay
+past e^-80 on some channel, which the token-by-token kernel takes; one case
+mixes both within a sequence and a head."""
 import numpy as np
 import pytest
 import torch
@@ -87,4 +90,20 @@ def test_backward_chunked_full_size_sampled_heads():
     gpu = run(inp)
     ref, cu, hs = run_oracle(inp, heads=[0, 11])
     errs = errors(gpu, ref, cu, hs)
+    assert all(e <= TOL for e in errs.values()), errs
+
+
+def test_backward_chunked_slow_chunks_take_the_step_kernel():
+    """Chunks whose decay passes e^-80 on one channel (over the chunk: the
+    prefill's secondary form; within a 16-token block: the pairwise form) sit
+    between ordinary chunks of the same sequence and head; their gradients
+    come from the token-by-token kernel, the others' from the tensor cores."""
+    inp = case([300, 140], 2, seed=6)
+    g = inp["log_alpha"].float()
+    g[64:128, 0, 5] = -2.0     # -128 over the chunk, -32 per 16-token block
+    g[128:192, 1, 9] = -6.0    # -96 within a 16-token block
+    g[300 + 64:300 + 128, 0, 17] = -1.5
+    inp["log_alpha"] = g.to(inp["log_alpha"].dtype)
+    ref, cu, hs = run_oracle(inp)
+    errs = errors(run(inp), ref, cu, hs)
     assert all(e <= TOL for e in errs.values()), errs
