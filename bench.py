@@ -374,11 +374,10 @@ def time_backward(w, steps, warmup, world):
     if kda.kda_check_workspace_error(ws) != kda.KDA_OK:
         raise RuntimeError("device-side check failed during the backward benchmark")
     ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    # chunked: the plan, the preparation, two scans, the tensor-core chunk
-    # kernel and the step kernel for chunks it leaves; the gradient zeroing
-    # (memsets) is not counted
+    # chunked: the plan, the preparation, the two scans (one grid), the
+    # tensor-core chunk kernel and the step kernel for the chunks it leaves
     return dict(ms_total=sum(ms), ms=ms, lengths=inp["lengths"], chunked=chunked,
-                launches=steps * (6 if chunked else 1))
+                launches=steps * (5 if chunked else 1))
 
 
 def time_prefill_e2e(w, steps, warmup):

@@ -673,11 +673,14 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
     const size_t nk = (size_t)total_tokens * H * 128;
     const size_t ng = scalar_gate ? (size_t)total_tokens * H : nk;
     cudaError_t e;
-    if ((e = cudaMemsetAsync(dq, 0, nk * sizeof(float), stream)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(dk_out, 0, nk * sizeof(float), stream)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(dg, 0, ng * sizeof(float), stream)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(dbeta, 0, (size_t)total_tokens * H * sizeof(float), stream)) != cudaSuccess)
-        return e;
+    if (scalar_gate) {   // the step kernel adds into zeroed gradients (the tensor-core
+                         // kernel writes every row of its items and zeroes the others)
+        if ((e = cudaMemsetAsync(dq, 0, nk * sizeof(float), stream)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(dk_out, 0, nk * sizeof(float), stream)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(dg, 0, ng * sizeof(float), stream)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(dbeta, 0, (size_t)total_tokens * H * sizeof(float), stream)) != cudaSuccess)
+            return e;
+    }
     // 1. the plan and the chunk records (the prefill's preparation, no chain)
     e = launch_prefill_split(q, k, v, g, beta, nullptr, cu, num_seqs, total_tokens, H, nullptr,
                              nullptr, ws + l.split, scalar_gate, nullptr, stream, kPrepOnly);

@@ -305,6 +305,15 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         fence_async_smem();
         named_barrier(BAR, kThreads);
         if (form != prep::kProductForm) {   // left to the step kernel
+            // which adds its (chunk, head, slice) units' row sums into zeroed rows
+            for (int v = pt; v < 32 * L; v += kThreads) {
+                const size_t e = ((size_t)(tok0 + (v >> 5)) * p.H + h) * 128 + 4 * (v & 31);
+                const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4 *>(p.dq + e) = z;
+                *reinterpret_cast<float4 *>(p.dk + e) = z;
+                *reinterpret_cast<float4 *>(p.dg + e) = z;
+            }
+            if (pt < L) p.dbeta[(size_t)(tok0 + pt) * p.H + h] = 0.f;
             mbar_wait(BSD, n_sd & 1u, abort_flag);   // the item's states have landed
             ++n_sd;
             named_barrier(BAR, kThreads);

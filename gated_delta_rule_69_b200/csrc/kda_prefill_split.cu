@@ -936,9 +936,10 @@ struct ChainT {
 //                  init_state is dL/dS_T and final_state receives dL/dS_0.
 enum : int { kChainPlain = 0, kChainTransition = 2, kChainSaveS = 3, kChainReverse = 4 };
 
+// The chain of one (sequence, head) unit (rank `unit` in the longest-first
+// order); the kernels below run one unit per CTA.
 template <int MODE>
-__global__ void __launch_bounds__(ChainT::THREADS, 1)
-kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
+__device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const Params &p, int unit) {
     constexpr bool TRANS = MODE == kChainTransition;
     constexpr bool SAVE = MODE == kChainSaveS;
     constexpr bool REV = MODE == kChainReverse;
@@ -950,8 +951,8 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *sm = dyn_smem + ((1024u - (smem_addr(dyn_smem) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x % p.H;
-    const int rank = blockIdx.x / p.H;
+    const int h = unit % p.H;
+    const int rank = unit / p.H;
     const int seq = p.perm ? p.perm[rank] : rank;
     int64_t bos, eos;
     seq_bounds(p, seq, bos, eos);
@@ -1226,6 +1227,22 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
         tmem_dealloc(tmem, Cfg::TMEM_COLS);
     }
     if (tid == 0 && *abort_flag) atomicOr(p.err_word, kDevErrTimeout);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(ChainT::THREADS, 1)
+kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    chain_t_unit<MODE>(tm_v, p, (int)blockIdx.x);
+}
+
+// The backward pass's two scans in one grid: CTAs [0, units) run the forward
+// scan (each chunk's entering state), CTAs [units, 2 units) the reverse one
+// (dL/dS at each chunk's end); they share only the records, which both read.
+__global__ void __launch_bounds__(ChainT::THREADS, 1)
+kda_backward_scans_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                          const Params pf, const Params pr, int units) {
+    if ((int)blockIdx.x < units) chain_t_unit<kChainSaveS>(tm_v, pf, (int)blockIdx.x);
+    else chain_t_unit<kChainReverse>(tm_do, pr, (int)blockIdx.x - units);
 }
 
 // =============================================================== layer epilogue
@@ -1607,16 +1624,21 @@ cudaError_t launch_backward_scans(const void *v, const void *d_o, const float *i
     pf.init_state = init_state;
     pf.final_state = nullptr;
     pf.states_out = static_cast<uint8_t *>(s_in);
-    cudaError_t e = launch_chain_t(v, total_tokens, H, pf, units, false, stream, kChainSaveS);
-    if (e != cudaSuccess) return e;
-    // dL/dS at each chunk's end: the reverse chain (launched after the forward
-    // one in plain stream order, so that the steps kernel that follows finds
-    // both complete)
+    // dL/dS at each chunk's end: the reverse chain over the same records
     Params pr = prm;
     pr.init_state = d_final_state;
     pr.final_state = d_init_state;
     pr.states_out = static_cast<uint8_t *>(ds_next);
-    return launch_chain_t(d_o, total_tokens, H, pr, units, false, stream, kChainReverse);
+    // both at once, in one grid
+    CUtensorMap mv, mdo;
+    if (!make_map_split(&mv, v, total_tokens, H, DV, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_split(&mdo, d_o, total_tokens, H, DV, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    cudaError_t e = set_max_dynamic_smem((const void *)kda_backward_scans_kernel, (int)ChainT::ALLOC);
+    if (e != cudaSuccess) return e;
+    if (units == 0) return cudaSuccess;
+    kda_backward_scans_kernel<<<2 * units, ChainT::THREADS, ChainT::ALLOC, stream>>>(mv, mdo, pf, pr, (int)units);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const void *g,
