@@ -322,15 +322,21 @@ kda_status gdn_backward(const void *q, const void *k, const void *v, const void 
                         size_t workspace_bytes, kda_stream_t stream);
 
 /*
- * kda_backward for bf16 inputs with d_k = d_v = 128 by chunks: the prefill's
- * chunk preparation, a forward and a reverse scan over its per-chunk
- * transition operands for every chunk's entering state and dL/dS at its end,
- * then every chunk's steps at once.  Same arguments and outputs as
- * kda_backward (bf16, d = 128 implied); the workspace (256-byte aligned,
+ * kda_backward for bf16 inputs with d_k = d_v = 128 by chunks (news digest
+ * page on Kimi Linear, section "Algorithme parallele par chunks": the chunk
+ * algebra, here differentiated): the prefill's chunk preparation, a forward
+ * and a reverse scan over its per-chunk transition operands (one grid) for
+ * every chunk's entering state and dL/dS at its end, then every (chunk,
+ * head) item's gradients at once as products on the tensor cores.  A chunk
+ * that decays below e^-80 within itself on some channel (log_alpha summing
+ * below -80 over it) takes the token-by-token steps instead.  Same
+ * arguments and outputs as kda_backward (bf16, d = 128 implied); the
+ * workspace (256-byte aligned,
  * kda_backward_chunked_workspace_size bytes) also holds the prefill's records
- * and two states per (chunk, head).  The chunk boundary states carry the
- * records' bf16 rounding: gradients agree with kda_backward to the bf16
- * tolerance, not to fp32 rounding.
+ * and two bf16 states per (chunk, head).  The chunk boundary states and the
+ * products' operands are bf16: gradients agree with kda_backward to the bf16
+ * tolerance, not to fp32 rounding.  Every gradient element is written (the
+ * per-channel path needs no zeroed outputs).
  */
 size_t kda_backward_chunked_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H);
 
