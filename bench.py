@@ -289,8 +289,9 @@ def time_prefill(w, steps, warmup, world, scalar_gate=False, layer=False, profil
     n = len(inp["lengths"])
     o = torch.empty((T, H, dv), dtype=q.dtype, device="cuda")
     fs = torch.empty((n, H, dk, dv), dtype=torch.float32, device="cuda")
-    ws = torch.empty(max(256, kda.kda_prefill_workspace_size(n, T, H, dk, dv)),
-                     dtype=torch.uint8, device="cuda")
+    need = (kda.kda_layer_prefill_workspace_size(n, T, H, dk, dv) if layer
+            else kda.kda_prefill_workspace_size(n, T, H, dk, dv))
+    ws = torch.empty(max(256, need), dtype=torch.uint8, device="cuda")
     flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 

@@ -89,6 +89,10 @@ kda_status prefill_impl(const void *q, const void *k, const void *v,
             overlaps(o, nv, layer->out_gate, nv))
             return KDA_ERR_INVALID_ARG;
     }
+    if (layer && total_tokens > 0 &&
+        workspace_bytes >= kda::layer_prefill_workspace(num_seqs, total_tokens, H))
+        return from_cuda(kda::launch_layer_prefill_split(q, k, v, *layer, init_state, cu_seqlens, num_seqs,
+                                                         total_tokens, H, o, final_state, workspace, stream));
     if (use_tensor_cores(dtype, d_k, d_v, total_tokens) &&
         workspace_bytes >= kda::prefill_split_workspace(num_seqs, total_tokens, H))
         return from_cuda(kda::launch_prefill_split(q, k, v, log_alpha, beta, init_state,
@@ -268,6 +272,12 @@ kda_status gdn_decode_step(const void *q, const void *k, const void *v,
                            kda_stream_t stream) {
     return decode_impl(q, k, v, log_alpha, beta, state, batch, H, d_k, d_v, dtype, o, stream,
                        true);
+}
+
+size_t kda_layer_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t d_k,
+                                        int32_t d_v) {
+    if (num_seqs < 1 || total_tokens < 0 || H < 1 || d_k != 128 || d_v != 128) return 0;
+    return kda::layer_prefill_workspace(num_seqs, total_tokens, H);
 }
 
 kda_status kda_layer_prefill(const void *q, const void *k, const void *v, const void *gate_z,

@@ -115,6 +115,15 @@ size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H);
 // kPrepOnly: the plan and the chunk records only (no chain), for the
 // backward pass's scans over the records.
 enum : int { kCpNone = 0, kCpLocal = 1, kCpFinish = 2, kPrepOnly = 3 };
+
+// The layer with its prologue as a pass of its own (the activations turned
+// into the operator's bf16 inputs in the workspace), then the split path and
+// the epilogue; its workspace is layer_prefill_workspace bytes.
+size_t layer_prefill_workspace(int num_seqs, int64_t total_tokens, int H);
+cudaError_t launch_layer_prefill_split(const void *q, const void *k, const void *v, const LayerArgs &la,
+                                       const float *init_state, const int32_t *cu, int num_seqs,
+                                       int64_t total_tokens, int H, void *o, float *final_state,
+                                       void *workspace, cudaStream_t stream);
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const void *g,
                                  const void *beta, const float *init_state, const int32_t *cu,
                                  int num_seqs, int64_t total_tokens, int H, void *o,

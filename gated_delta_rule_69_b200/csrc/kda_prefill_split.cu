@@ -1245,48 +1245,115 @@ kda_backward_scans_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid
     else chain_t_unit<kChainReverse>(tm_do, pr, (int)blockIdx.x - units);
 }
 
+// =============================================================== layer prologue
+// The layer's activations as the operator's inputs: q and k L2-normalised
+// (x rsqrt(sum x^2 + eps)), log_alpha = -e^{A_log[h]} softplus(z), beta =
+// sigmoid(logit), all written in bf16.  A half-warp per (token, head) row of
+// 128 channels (16-byte pieces, eight channels per lane).  A pass of its own ahead of the
+// operator: inside the chunk preparation the same arithmetic sat on that
+// kernel's latency-bound path, while as a stream over the activations it is
+// bound by HBM.
+constexpr int kProThreads = 256;
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &w, float (&x)[8]) {
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&ww[e]);
+        x[2 * e] = __low2float(h2);
+        x[2 * e + 1] = __high2float(h2);
+    }
+}
+
+__device__ __forceinline__ uint4 f32x8_to_bf16(const float (&x)[8], float s) {
+    uint4 w;
+    w.x = pack_bf16x2(x[0] * s, x[1] * s);
+    w.y = pack_bf16x2(x[2] * s, x[3] * s);
+    w.z = pack_bf16x2(x[4] * s, x[5] * s);
+    w.w = pack_bf16x2(x[6] * s, x[7] * s);
+    return w;
+}
+
+__global__ void __launch_bounds__(kProThreads)
+kda_layer_prologue_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                          const __nv_bfloat16 *__restrict__ z, const __nv_bfloat16 *__restrict__ blogit,
+                          const float *__restrict__ A_log, float eps, int H, int64_t rows,
+                          __nv_bfloat16 *__restrict__ qn, __nv_bfloat16 *__restrict__ kn,
+                          __nv_bfloat16 *__restrict__ la, __nv_bfloat16 *__restrict__ bt) {
+    const int lane = threadIdx.x & 31, sub = lane & 15;
+    // a warp's two rows (half-warps); the shuffles take all 32 lanes, so a row
+    // past the end is masked, not skipped
+    const int64_t row = ((int64_t)blockIdx.x * (kProThreads / 32) + (threadIdx.x >> 5)) * 2 + (lane >> 4);
+    const bool valid = row < rows;
+    const size_t at = (size_t)row * 16 + sub;
+    uint4 qv = make_uint4(0u, 0u, 0u, 0u), kv = qv, zv = qv;
+    if (valid) {
+        qv = reinterpret_cast<const uint4 *>(q)[at];
+        kv = reinterpret_cast<const uint4 *>(k)[at];
+        zv = reinterpret_cast<const uint4 *>(z)[at];
+    }
+    float xq[8], xk[8], xz[8];
+    bf16x8_to_f32(qv, xq);
+    bf16x8_to_f32(kv, xk);
+    bf16x8_to_f32(zv, xz);
+    float sq = 0.f, sk = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        sq = fmaf(xq[e], xq[e], sq);
+        sk = fmaf(xk[e], xk[e], sk);
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) {   // within the half-warp
+        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+    }
+    if (!valid) return;
+    const float c = -__expf(A_log[row % H]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)   // softplus as the in-kernel prologue takes it
+        xz[e] = c * (xz[e] > 15.f ? xz[e] : __logf(1.f + __expf(xz[e])));
+    reinterpret_cast<uint4 *>(qn)[at] = f32x8_to_bf16(xq, rsqrtf(sq + eps));
+    reinterpret_cast<uint4 *>(kn)[at] = f32x8_to_bf16(xk, rsqrtf(sk + eps));
+    reinterpret_cast<uint4 *>(la)[at] = f32x8_to_bf16(xz, 1.f);
+    if (sub == 0) bt[row] = __float2bfloat16(1.f / (1.f + __expf(-__bfloat162float(blogit[row]))));
+}
+
 // =============================================================== layer epilogue
 // o <- o / sqrt(mean_j o_j^2 + eps) * w_j * sigmoid(g_j) per (token, head) row,
-// in place after the chain: one warp per row of 128, four channels per lane.
-// A pass of its own: inside the chain's loop the same work sat on the serial
-// state path (about 1.5 us per chunk); here it is a stream over o and the gate.
+// in place after the chain: a half-warp per row of 128 (eight channels per
+// lane, 16-byte pieces).  A pass of its own: inside the chain's loop the same
+// work sat on the serial state path (about 1.5 us per chunk); here it is a
+// stream over o and the gate.
 constexpr int kEpiThreads = 256;
 
 __global__ void __launch_bounds__(kEpiThreads)
 kda_layer_epilogue_kernel(__nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ gate,
                           const float *__restrict__ w, float eps, int64_t rows) {
-    const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * (kEpiThreads / 32) + (threadIdx.x >> 5);
-    if (row >= rows) return;
-    uint2 *orow = reinterpret_cast<uint2 *>(o + row * DV) + lane;
-    const uint2 ov = *orow;
-    float x[4];
-    {
-        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&ov.x);
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&ov.y);
-        x[0] = __low2float(a); x[1] = __high2float(a); x[2] = __low2float(b); x[3] = __high2float(b);
+    const int lane = threadIdx.x & 31, sub = lane & 15;
+    const int64_t row = ((int64_t)blockIdx.x * (kEpiThreads / 32) + (threadIdx.x >> 5)) * 2 + (lane >> 4);
+    const bool valid = row < rows;   // masked, not skipped: the shuffles take all 32 lanes
+    const size_t at = (size_t)row * (DV / 8) + sub;
+    uint4 ov = make_uint4(0u, 0u, 0u, 0u), gv4 = ov;
+    if (valid) {
+        ov = reinterpret_cast<const uint4 *>(o)[at];
+        if (gate) gv4 = reinterpret_cast<const uint4 *>(gate)[at];
     }
-    float gv[4] = {0.f, 0.f, 0.f, 0.f};
-    if (gate) {
-        const uint2 g2 = reinterpret_cast<const uint2 *>(gate + row * DV)[lane];
-        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(&g2.x);
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&g2.y);
-        gv[0] = __low2float(a); gv[1] = __high2float(a); gv[2] = __low2float(b); gv[3] = __high2float(b);
-    }
-    float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
+    float x[8], gv[8];
+    bf16x8_to_f32(ov, x);
+    bf16x8_to_f32(gv4, gv);
+    float ss = 0.f;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if (!valid) return;
     const float r = rsqrtf(ss * (1.f / DV) + eps);
-    float y[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        y[e] = x[e] * r * (w ? w[4 * lane + e] : 1.f);
-        if (gate) y[e] *= 1.f / (1.f + __expf(-gv[e]));
+    for (int e = 0; e < 8; ++e) {
+        x[e] *= r * (w ? w[8 * sub + e] : 1.f);
+        if (gate) x[e] *= 1.f / (1.f + __expf(-gv[e]));
     }
-    uint2 out;
-    out.x = pack_bf16x2(y[0], y[1]);
-    out.y = pack_bf16x2(y[2], y[3]);
-    *orow = out;
+    reinterpret_cast<uint4 *>(o)[at] = f32x8_to_bf16(x, 1.f);
 }
 
 // =============================================================== plan kernel
@@ -1577,6 +1644,59 @@ bool make_bf16_map_3d(CUtensorMap *m, const void *base, int64_t T, int H, int in
     return make_map_split(m, base, T, H, inner, box_inner, sw);
 }
 
+// The layer path with its prologue as a pass of its own: the split
+// workspace, then the prologue's outputs (q, k, log_alpha [T, H, 128] and
+// beta [T, H], bf16), 256-byte aligned.
+struct LayerLayout {
+    size_t qn, kn, la, bt, total;
+};
+
+LayerLayout layer_layout(int num_seqs, int64_t total_tokens, int H) {
+    LayerLayout l;
+    const size_t tile = (size_t)total_tokens * H * 128 * sizeof(__nv_bfloat16);
+    l.qn = round_up(split_layout(num_seqs, total_tokens, H).total, 256);
+    l.kn = l.qn + round_up(tile, 256);
+    l.la = l.kn + round_up(tile, 256);
+    l.bt = l.la + round_up(tile, 256);
+    l.total = l.bt + round_up((size_t)total_tokens * H * sizeof(__nv_bfloat16), 256);
+    return l;
+}
+
+size_t layer_prefill_workspace(int num_seqs, int64_t total_tokens, int H) {
+    return layer_layout(num_seqs, total_tokens, H).total;
+}
+
+cudaError_t launch_layer_prefill_split(const void *q, const void *k, const void *v, const LayerArgs &la,
+                                       const float *init_state, const int32_t *cu, int num_seqs,
+                                       int64_t total_tokens, int H, void *o, float *final_state,
+                                       void *workspace, cudaStream_t stream) {
+    using namespace split;
+    const LayerLayout l = layer_layout(num_seqs, total_tokens, H);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    auto *qn = reinterpret_cast<__nv_bfloat16 *>(ws + l.qn);
+    auto *kn = reinterpret_cast<__nv_bfloat16 *>(ws + l.kn);
+    auto *lg = reinterpret_cast<__nv_bfloat16 *>(ws + l.la);
+    auto *bt = reinterpret_cast<__nv_bfloat16 *>(ws + l.bt);
+    const int64_t rows = total_tokens * H;
+    if (rows > 0) {
+        const int64_t per = kProThreads / 16;   // rows per CTA
+        kda_layer_prologue_kernel<<<(unsigned)((rows + per - 1) / per), kProThreads, 0, stream>>>(
+            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+            static_cast<const __nv_bfloat16 *>(la.gate_z), static_cast<const __nv_bfloat16 *>(la.beta_logit),
+            la.A_log, la.qk_eps, H, rows, qn, kn, lg, bt);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = launch_prefill_split(qn, kn, v, lg, bt, init_state, cu, num_seqs, total_tokens, H, o,
+                                         final_state, workspace, false, nullptr, stream, kCpNone, nullptr);
+    if (e != cudaSuccess || rows == 0) return e;
+    kda_layer_epilogue_kernel<<<(unsigned)((rows + kEpiThreads / 16 - 1) / (kEpiThreads / 16)), kEpiThreads, 0,
+                                stream>>>(static_cast<__nv_bfloat16 *>(o),
+                                          static_cast<const __nv_bfloat16 *>(la.out_gate), la.norm_weight,
+                                          la.norm_eps, rows);
+    return cudaGetLastError();
+}
+
 size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H) {
     return split_layout(num_seqs, total_tokens, H).total;
 }
@@ -1773,7 +1893,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                        : launch_chain_t(v, total_tokens, H, prm, units, overlap, stream);
     if (e != cudaSuccess || !layer) return e;
     const int64_t rows = total_tokens * H;
-    kda_layer_epilogue_kernel<<<(unsigned)((rows + kEpiThreads / 32 - 1) / (kEpiThreads / 32)),
+    kda_layer_epilogue_kernel<<<(unsigned)((rows + kEpiThreads / 16 - 1) / (kEpiThreads / 16)),
                                 kEpiThreads, 0, stream>>>(
         static_cast<__nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(layer->out_gate),
         layer->norm_weight, layer->norm_eps, rows);

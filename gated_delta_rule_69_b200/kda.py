@@ -48,6 +48,8 @@ def lib():
         L.kda_version.restype = ctypes.c_int
         L.kda_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32]
         L.kda_prefill_workspace_size.restype = sz
+        L.kda_layer_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32]
+        L.kda_layer_prefill_workspace_size.restype = sz
         L.kda_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
                                   ctypes.c_int, vp, vp, vp, sz, vp]
         L.kda_prefill.restype = ctypes.c_int
@@ -127,6 +129,12 @@ def _check_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def kda_layer_prefill_workspace_size(num_seqs: int, total_tokens: int, H: int, d_k: int, d_v: int) -> int:
+    """Workspace for kda_layer_prefill with its prologue as a pass of its own
+    (0 for shapes the layer path does not take)."""
+    return int(lib().kda_layer_prefill_workspace_size(num_seqs, total_tokens, H, d_k, d_v))
 
 
 def kda_prefill_workspace_size(num_seqs: int, total_tokens: int, H: int, d_k: int, d_v: int) -> int:
@@ -257,10 +265,12 @@ def kda_layer_prefill(q, k, v, gate_z, A_log, beta_logit, out_gate=None, norm_we
                       qk_eps=1e-6, norm_eps=1e-6, init_state=None, cu_seqlens=None,
                       num_seqs=None, o=None, final_state=None, workspace=None,
                       output_final_state=True, stream=None):
-    """KDA prefill with the layer prologue / epilogue fused in (see
-    include/kda.h): raw q, k, gate pre-activation gate_z [T, H, d_k], A_log [H]
-    fp32, beta_logit [T, H]; optional out_gate [T, H, d_v] and norm_weight
-    [d_v] fp32.  bf16, d = 128."""
+    """KDA prefill with the layer prologue and epilogue (see include/kda.h):
+    raw q, k, gate pre-activation gate_z [T, H, d_k], A_log [H] fp32,
+    beta_logit [T, H]; optional out_gate [T, H, d_v] and norm_weight [d_v]
+    fp32.  bf16, d = 128.  The default workspace takes the path with the
+    prologue as a pass of its own; one of kda_prefill_workspace_size bytes
+    runs it inside the chunk preparation."""
     T, H, dk = q.shape
     dv = v.shape[-1]
     if gate_z.shape != q.shape or beta_logit.shape != q.shape[:2] or A_log.shape != (H,):
@@ -273,7 +283,7 @@ def kda_layer_prefill(q, k, v, gate_z, A_log, beta_logit, out_gate=None, norm_we
             raise TypeError("cu_seqlens must be int32")
     else:
         n = 1 if num_seqs is None else int(num_seqs)
-    need = kda_prefill_workspace_size(n, T, H, dk, dv)
+    need = kda_layer_prefill_workspace_size(n, T, H, dk, dv) or kda_prefill_workspace_size(n, T, H, dk, dv)
     with _on(stream):
         if o is None:
             o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)

@@ -206,13 +206,20 @@ kda_status gdn_decode_step(const void *q, const void *k, const void *v,
  *   norm_weight  : [d_v] fp32 (device), or NULL (weight 1)
  * Other arguments, layouts and errors as kda_prefill / kda_decode_step.
  * kda_layer_prefill runs on the two-kernel tensor-core path only: bf16,
- * d_k = d_v = 128 and a workspace of kda_prefill_workspace_size(...) bytes
- * (else KDA_ERR_UNSUPPORTED / KDA_ERR_WORKSPACE); its prologue runs inside
- * the chunk preparation and its epilogue as one pass over o after the state
- * chain.  kda_layer_decode_step takes every shape
- * kda_decode_step takes.  Weights of the projections that produce these
- * activations are the caller's.
+ * d_k = d_v = 128 and a workspace of at least kda_prefill_workspace_size(...)
+ * bytes (else KDA_ERR_UNSUPPORTED / KDA_ERR_WORKSPACE).  With a workspace of
+ * kda_layer_prefill_workspace_size(...) bytes its prologue runs as a pass of
+ * its own that writes the operator's inputs (normalised q and k, log_alpha
+ * and beta, bf16) into the workspace, then the operator's kernels; with less,
+ * the prologue runs inside the chunk preparation (log_alpha kept in fp32
+ * there; slower: the arithmetic lands on that kernel's latency-bound path).
+ * Either way the epilogue is one pass over o after the state chain.
+ * kda_layer_decode_step takes every shape kda_decode_step takes.  Weights of
+ * the projections that produce these activations are the caller's.
  */
+size_t kda_layer_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t H,
+                                        int32_t d_k, int32_t d_v);
+
 kda_status kda_layer_prefill(const void *q, const void *k, const void *v, const void *gate_z,
                              const float *A_log, const void *beta_logit, const void *out_gate,
                              const float *norm_weight, float qk_eps, float norm_eps,

@@ -165,6 +165,25 @@ def test_layer_prefill(lengths, gates):
     assert skipped <= rows // 5, (skipped, rows)
 
 
+@pytest.mark.parametrize("A_mean", [0.0, 2.6])
+def test_layer_prefill_prologue_inside_the_preparation(A_mean):
+    """A workspace of kda_prefill_workspace_size bytes (no room for the
+    prologue's outputs): the prologue runs inside the chunk preparation."""
+    lengths = [1, 64, 130, 200, 63]
+    inp = layer_case(sum(lengths), 3, 128, 128, seed=36, lengths=lengths, A_mean=A_mean)
+    n = len(lengths)
+    T, H = inp["q"].shape[:2]
+    need = kda().kda_prefill_workspace_size(n, T, H, 128, 128)
+    assert kda().kda_layer_prefill_workspace_size(n, T, H, 128, 128) > need
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    o, fs = run_layer(inp, workspace=ws)
+    ref_o, ref_s, cu, to_o = oracle_layer(inp)
+    assert o_err(to_o(f64(o)), ref_o, cu, 3) <= TOL["bf16"]
+    assert state_err(f64(fs), ref_s) <= TOL["bf16"]
+    ratio, skipped, rows = y_within_bound(o, inp, TOL["bf16"])
+    assert ratio <= 1.0, ratio
+
+
 @pytest.mark.parametrize("A_mean", [1.3, 2.6])
 def test_layer_prefill_fast_decay(A_mean):
     """e^A softplus(z) near 2.5 and 10 per token: chunks that take the
