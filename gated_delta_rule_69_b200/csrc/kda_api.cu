@@ -329,7 +329,7 @@ kda_status kda_cp_local(const void *q, const void *k, const void *v, const void 
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (total_tokens < 1 || H < 1) return KDA_ERR_INVALID_ARG;
     if (!use_tensor_cores(dtype, d_k, d_v, total_tokens)) return KDA_ERR_UNSUPPORTED;
-    if (!q || !k || !v || !log_alpha || !beta || !M || !S_tilde || !o_scratch)
+    if (!q || !k || !v || !log_alpha || !beta || !M || !S_tilde)
         return KDA_ERR_INVALID_ARG;
     const void *ptrs[] = {q, k, v, log_alpha, M, S_tilde, o_scratch};
     for (const void *p : ptrs)

@@ -1171,7 +1171,7 @@ __device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const Para
                 if (t0 + i < len) dst[(size_t)i * p.H * DV] = __float2bfloat16(v[i]);
         };
         for (int n = 0; n < nchunks; ++n) {
-            if (SAVE || REV) {   // the state entering (forward) or leaving (reverse) this chunk
+            if ((SAVE || REV) && p.states_out) {   // the state entering (forward) or leaving (reverse) this chunk
                 const int nn = REV ? nchunks - 1 - n : n;
                 uint8_t *tile = p.states_out + ((rec0 + nn) * p.H + h) * (size_t)32768 + (j >> 6) * 16384;
 #pragma unroll
@@ -1243,6 +1243,17 @@ kda_backward_scans_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid
                           const Params pf, const Params pr, int units) {
     if ((int)blockIdx.x < units) chain_t_unit<kChainSaveS>(tm_v, pf, (int)blockIdx.x);
     else chain_t_unit<kChainReverse>(tm_do, pr, (int)blockIdx.x - units);
+}
+
+// A segment's two local chains for context parallelism in one grid: CTAs
+// [0, units) run the chain from a zero state with v (the state the segment
+// generates), CTAs [units, 2 units) from the identity with v counting as zero
+// (its transition); both over the same records, neither writing o.
+__global__ void __launch_bounds__(ChainT::THREADS, 1)
+kda_cp_local_chains_kernel(const __grid_constant__ CUtensorMap tm_v, const Params pl, const Params pt,
+                           int units) {
+    if ((int)blockIdx.x < units) chain_t_unit<kChainSaveS>(tm_v, pl, (int)blockIdx.x);
+    else chain_t_unit<kChainTransition>(tm_v, pt, (int)blockIdx.x - units);
 }
 
 // =============================================================== layer prologue
@@ -1814,8 +1825,10 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     // a segment's transition is d_k x d_k: whole-d_v chain CTAs only
     const ChainPlan plan = choose_chain(units, (uint64_t)(total_tokens / C + num_seqs) * H, total_tokens,
                                         num_seqs, (unsigned)sm_count, cp_mode == kCpLocal);
-    const bool overlap = plan.overlap && cp_mode != kPrepOnly;
-    const unsigned chain_blocks = units * (unsigned)(DV / plan.dvt);
+    // a segment's two local chains run side by side (twice the chain CTAs)
+    const unsigned chain_blocks = units * (unsigned)(DV / plan.dvt) * (cp_mode == kCpLocal ? 2u : 1u);
+    const bool overlap = (cp_mode == kCpLocal ? chain_blocks < (unsigned)sm_count : plan.overlap) &&
+                         cp_mode != kPrepOnly;
     uint32_t *rec_ready = overlap ? reinterpret_cast<uint32_t *>(ws + l.flags) : nullptr;
     kda_split_plan_kernel<<<1, kPlanThreads, 0, stream>>>(cu, num_seqs, total_tokens, perm,
                                                           chunk_off, chunk_tab, total_chunks, err,
@@ -1879,15 +1892,33 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     }
     if (cp_mode == kPrepOnly) return cudaSuccess;
     if (cp_mode == kCpLocal) {
-        // the locally generated state (from zero), then over the same records
-        // the segment's transition (from the identity, v counting as zero)
-        e = launch_chain_t(v, total_tokens, H, prm, units, overlap, stream);
-        if (e != cudaSuccess) return e;
+        // the locally generated state (from zero) and, over the same records, the
+        // segment's transition (from the identity, v counting as zero), in one
+        // grid, consuming the records as the preparation publishes them
+        Params pl = prm;
+        pl.init_state = nullptr;
+        pl.states_out = nullptr;
         Params pt = prm;
         pt.init_state = nullptr;
         pt.final_state = cp_transition;
-        pt.rec_ready = nullptr;   // the records are complete once the first chain has run
-        return launch_chain_t(v, total_tokens, H, pt, units, false, stream, kChainTransition);
+        CUtensorMap mv;
+        if (!make_map_split(&mv, v, total_tokens, H, DV, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        e = set_max_dynamic_smem((const void *)kda_cp_local_chains_kernel, (int)ChainT::ALLOC);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * units);
+        cfg.blockDim = dim3(ChainT::THREADS);
+        cfg.dynamicSmemBytes = ChainT::ALLOC;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = overlap ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, kda_cp_local_chains_kernel, mv, pl, pt, (int)units);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
     }
     e = plan.dvt == 32 ? launch_chain<32>(v, total_tokens, H, prm, units, overlap, stream)
                        : launch_chain_t(v, total_tokens, H, prm, units, overlap, stream);

@@ -345,14 +345,13 @@ def kda_cp_combine(M, S_tilde, S0=None, S_in=None, stream=None):
 
 def kda_cp_local(q, k, v, log_alpha, beta, workspace, o_scratch=None, stream=None):
     """One segment's (M [1, H, d_k, d_k], S~ [1, H, d_k, d_v]); the chunk records
-    stay in ``workspace`` for kda_cp_finish.  bf16, d = 128, one sequence."""
+    stay in ``workspace`` for kda_cp_finish.  bf16, d = 128, one sequence.
+    ``o_scratch`` is accepted for the interface and not written."""
     T, H, dk = q.shape
     dv = v.shape[-1]
     with _on(stream):
         M = torch.empty((1, H, dk, dk), dtype=torch.float32, device=q.device)
         S = torch.empty((1, H, dk, dv), dtype=torch.float32, device=q.device)
-        if o_scratch is None:
-            o_scratch = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
     _check_cuda(q, k, v, log_alpha, beta, workspace, o_scratch)
     st = lib().kda_cp_local(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), T, H, dk, dv,
                             _dtype_code(q), _ptr(M), _ptr(S), _ptr(o_scratch), _ptr(workspace),

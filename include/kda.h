@@ -261,10 +261,10 @@ kda_status kda_cp_combine(const float *M, const float *S_tilde, const float *S0,
  * bf16, d_k = d_v = 128, a workspace of kda_prefill_workspace_size(1,
  * total_tokens, H) bytes), sharing one chunk preparation:
  *   kda_cp_local  prepares every chunk (the records stay in `workspace`) and
- *                 runs the state chain twice over them: S_tilde [1, H, d_k, d_v]
- *                 from a zero state, M [1, H, d_k, d_k] from the identity with
- *                 v counting as zero; o_scratch [T, H, d_v] is written and
- *                 holds nothing useful.
+ *                 runs the state chain twice over them, side by side:
+ *                 S_tilde [1, H, d_k, d_v] from a zero state, M [1, H, d_k, d_k]
+ *                 from the identity with v counting as zero; o_scratch is not
+ *                 written (it stays in the interface; may be NULL).
  *   kda_cp_finish runs the chain once more over the same workspace's records
  *                 from S_in [1, H, d_k, d_v] (NULL: zero), writing o and
  *                 final_state (NULL: not written).  The workspace must not have
