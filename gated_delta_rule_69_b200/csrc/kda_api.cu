@@ -416,33 +416,63 @@ size_t kda_backward_chunked_workspace_size(int32_t num_seqs, int64_t total_token
     return kda::backward_chunked_workspace(num_seqs, total_tokens, H);
 }
 
-kda_status kda_backward_chunked(const void *q, const void *k, const void *v, const void *log_alpha,
-                                const void *beta, const float *init_state,
-                                const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
-                                int32_t H, const void *d_o, const float *d_final_state, float *dq,
-                                float *dk, float *dv, float *dlog_alpha, float *dbeta,
-                                float *d_init_state, void *workspace, size_t workspace_bytes,
-                                kda_stream_t stream_) {
+namespace {
+
+kda_status backward_chunked_impl(const void *q, const void *k, const void *v, const void *log_alpha,
+                                 const void *beta, const float *init_state,
+                                 const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                                 int32_t H, const void *d_o, const float *d_final_state, float *dq,
+                                 float *dk, float *dv, float *dlog_alpha, float *dbeta,
+                                 float *d_init_state, void *workspace, size_t workspace_bytes,
+                                 kda_stream_t stream_, bool scalar_gate) {
     cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
     if (num_seqs < 1 || total_tokens < 1 || total_tokens > INT_MAX || H < 1)
         return KDA_ERR_INVALID_ARG;
     if (!cu_seqlens && total_tokens % num_seqs != 0) return KDA_ERR_INVALID_ARG;
     if (!q || !k || !v || !log_alpha || !beta || !d_o || !dq || !dk || !dv || !dlog_alpha || !dbeta)
         return KDA_ERR_INVALID_ARG;
-    const void *p16[] = {q, k, v, log_alpha, d_o, init_state, d_final_state, dv, d_init_state};
+    const void *p16[] = {q, k, v, scalar_gate ? nullptr : log_alpha, d_o, init_state, d_final_state, dv,
+                         d_init_state};
     for (const void *p : p16)
         if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
     const void *p4[] = {dq, dk, dlog_alpha, dbeta, cu_seqlens};
     for (const void *p : p4)
         if (p && !aligned_to(p, 4)) return KDA_ERR_INVALID_ARG;
     if (beta && !aligned_to(beta, 2)) return KDA_ERR_INVALID_ARG;
+    if (scalar_gate && !aligned_to(log_alpha, 2)) return KDA_ERR_INVALID_ARG;
     if (!workspace || workspace_bytes < kda::backward_chunked_workspace(num_seqs, total_tokens, H))
         return KDA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_INVALID_ARG;
     return from_cuda(kda::launch_backward_chunked(q, k, v, log_alpha, beta, init_state, cu_seqlens,
                                                   num_seqs, total_tokens, H, d_o, d_final_state,
                                                   dq, dk, dv, dlog_alpha, dbeta, d_init_state,
-                                                  workspace, false, stream));
+                                                  workspace, scalar_gate, stream));
+}
+
+}  // namespace
+
+kda_status kda_backward_chunked(const void *q, const void *k, const void *v, const void *log_alpha,
+                                const void *beta, const float *init_state,
+                                const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                                int32_t H, const void *d_o, const float *d_final_state, float *dq,
+                                float *dk, float *dv, float *dlog_alpha, float *dbeta,
+                                float *d_init_state, void *workspace, size_t workspace_bytes,
+                                kda_stream_t stream) {
+    return backward_chunked_impl(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, total_tokens,
+                                 H, d_o, d_final_state, dq, dk, dv, dlog_alpha, dbeta, d_init_state,
+                                 workspace, workspace_bytes, stream, false);
+}
+
+kda_status gdn_backward_chunked(const void *q, const void *k, const void *v, const void *log_alpha,
+                                const void *beta, const float *init_state,
+                                const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                                int32_t H, const void *d_o, const float *d_final_state, float *dq,
+                                float *dk, float *dv, float *dlog_alpha, float *dbeta,
+                                float *d_init_state, void *workspace, size_t workspace_bytes,
+                                kda_stream_t stream) {
+    return backward_chunked_impl(q, k, v, log_alpha, beta, init_state, cu_seqlens, num_seqs, total_tokens,
+                                 H, d_o, d_final_state, dq, dk, dv, dlog_alpha, dbeta, d_init_state,
+                                 workspace, workspace_bytes, stream, true);
 }
 
 kda_status kda_check_workspace_error(const void *workspace, kda_stream_t stream_) {

@@ -39,7 +39,7 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
                                const void *d_o, int64_t total_tokens, int H, const int2 *chunk_tab,
                                const uint32_t *total_chunks, const uint8_t *s_in, const uint8_t *ds_next, float *dq,
                                float *dk, float *dv, float *dg, float *dbeta, uint32_t *slow, float *gscr,
-                               uint32_t *err_word, int grid, cudaStream_t stream);
+                               uint32_t *err_word, int grid, bool scalar_gate, cudaStream_t stream);
 
 namespace {
 
@@ -672,15 +672,11 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const size_t nk = (size_t)total_tokens * H * 128;
     const size_t ng = scalar_gate ? (size_t)total_tokens * H : nk;
+    // no zeroing: the tensor-core kernel writes every row of its items and
+    // zeroes those of the items it leaves, into which the step kernel adds
+    (void)nk;
+    (void)ng;
     cudaError_t e;
-    if (scalar_gate) {   // the step kernel adds into zeroed gradients (the tensor-core
-                         // kernel writes every row of its items and zeroes the others)
-        if ((e = cudaMemsetAsync(dq, 0, nk * sizeof(float), stream)) != cudaSuccess) return e;
-        if ((e = cudaMemsetAsync(dk_out, 0, nk * sizeof(float), stream)) != cudaSuccess) return e;
-        if ((e = cudaMemsetAsync(dg, 0, ng * sizeof(float), stream)) != cudaSuccess) return e;
-        if ((e = cudaMemsetAsync(dbeta, 0, (size_t)total_tokens * H * sizeof(float), stream)) != cudaSuccess)
-            return e;
-    }
     // 1. the plan and the chunk records (the prefill's preparation, no chain)
     e = launch_prefill_split(q, k, v, g, beta, nullptr, cu, num_seqs, total_tokens, H, nullptr,
                              nullptr, ws + l.split, scalar_gate, nullptr, stream, kPrepOnly);
@@ -693,17 +689,14 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
                               ws + l.split, ws + l.s_in, ws + l.ds_next, d_init_state, stream);
     if (e != cudaSuccess) return e;
     // 3. the chunk-local gradients: on the tensor cores for every chunk that
-    // decays within e^80 (per-channel gate), then the token-by-token kernel for
-    // the rest (all chunks for a scalar gate)
+    // decays within e^80, then the token-by-token kernel for the rest
     uint32_t *slow = reinterpret_cast<uint32_t *>(ws + l.slow);
-    if (!scalar_gate) {
-        if ((e = cudaMemsetAsync(slow, 0, l.max_chunks * H * sizeof(uint32_t), stream)) != cudaSuccess) return e;
-        e = launch_backward_tc(q, k, v, g, beta, d_o, total_tokens, H, tab.chunk_tab, tab.total_chunks,
-                               ws + l.s_in, ws + l.ds_next, dq, dk_out, dv_out, dg, dbeta,
-                               slow, reinterpret_cast<float *>(ws + l.gscr), reinterpret_cast<uint32_t *>(ws),
-                               l.grid_tc, stream);
-        if (e != cudaSuccess) return e;
-    }
+    if ((e = cudaMemsetAsync(slow, 0, l.max_chunks * H * sizeof(uint32_t), stream)) != cudaSuccess) return e;
+    e = launch_backward_tc(q, k, v, g, beta, d_o, total_tokens, H, tab.chunk_tab, tab.total_chunks,
+                           ws + l.s_in, ws + l.ds_next, dq, dk_out, dv_out, dg, dbeta,
+                           slow, reinterpret_cast<float *>(ws + l.gscr), reinterpret_cast<uint32_t *>(ws),
+                           l.grid_tc, scalar_gate, stream);
+    if (e != cudaSuccess) return e;
     BwdArgs p = {};
     p.q = q; p.k = k; p.v = v; p.g = g; p.beta = beta; p.d_o = d_o;
     p.dq = dq; p.dk = dk_out; p.dv = dv_out; p.dg = dg; p.dbeta = dbeta;
@@ -719,7 +712,7 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
     ca.tab = tab;
     ca.s_in = ws + l.s_in;
     ca.ds_next = ws + l.ds_next;
-    ca.only = scalar_gate ? nullptr : slow;
+    ca.only = slow;
     ca.num_seqs = num_seqs;
     const size_t smem = BwdShape<128>::SMEM;
     if ((e = set_max_dynamic_smem((const void *)kda_backward_chunk_kernel<__nv_bfloat16, 128>, (int)smem)) !=

@@ -89,6 +89,7 @@ struct Sm {
     static constexpr uint32_t EGL = 221440;    // 128 fp32: e^{G_L}
     static constexpr uint32_t CSUM = 221952;   // 4 x 128 fp32 (the gate's; the final exchange after)
     static constexpr uint32_t DB = 224000;     // 64 fp32: dbeta of the item
+    static constexpr uint32_t GSC = 224256;    // 64 fp32: a scalar gate's raw log_alpha
     static constexpr uint32_t ES = 224768;     // 128 fp32: rowsum(S .* dS_C)
     static constexpr uint32_t BARS = 225280;   // mbarriers
     static constexpr uint32_t MISC = 225344;   // tmem base, abort, slow flag
@@ -201,19 +202,24 @@ __device__ __forceinline__ void issue_states(uint8_t *sm, uint64_t *bar, const A
     bulk_load(sm + Sm::DSC, p.ds_next + (size_t)item * 32768, 32768, bar);
 }
 
+// k, q (and, for a per-channel gate, log_alpha) of an item
+template <bool SCALAR>
 __device__ __forceinline__ void issue_raw(uint8_t *sm, uint64_t *bar, const CUtensorMap &tm_k,
                                           const CUtensorMap &tm_q, const CUtensorMap &tm_g, const Args &p,
                                           uint32_t item) {
     const int h = (int)(item % (uint32_t)p.H);
     const int t = p.chunk_tab[item / (uint32_t)p.H].x;
-    mbar_arrive_expect_tx(bar, 4 * 8192 + 16384);
+    mbar_arrive_expect_tx(bar, 4 * 8192 + (SCALAR ? 0 : 16384));
     tma_load_3d(sm + Sm::STK, &tm_k, bar, 0, h, t);
     tma_load_3d(sm + Sm::STK + 16384, &tm_k, bar, 64, h, t);
     tma_load_3d(sm + Sm::STK + 8192, &tm_q, bar, 0, h, t);
     tma_load_3d(sm + Sm::STK + 16384 + 8192, &tm_q, bar, 64, h, t);
-    tma_load_3d(sm + Sm::GRAW, &tm_g, bar, 0, h, t);
+    if (!SCALAR) tma_load_3d(sm + Sm::GRAW, &tm_g, bar, 0, h, t);
 }
 
+// SCALAR: the Gated DeltaNet gate (log_alpha and dlog_alpha one value per
+// token and head).
+template <bool SCALAR>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_do,
@@ -241,7 +247,7 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         fence_mbar_init();
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_g);
+        if (!SCALAR) tma_prefetch_desc(&tm_g);
         tma_prefetch_desc(&tm_do);
     }
     if (warp == 0) {
@@ -267,8 +273,9 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         named_barrier(BAR, kThreads);
     };
 
+    float *gsc = reinterpret_cast<float *>(sm + Sm::GSC);
     if (leader && blockIdx.x < total) {
-        issue_raw(sm, BLD, tm_k, tm_q, tm_g, p, blockIdx.x);
+        issue_raw<SCALAR>(sm, BLD, tm_k, tm_q, tm_g, p, blockIdx.x);
         issue_states(sm, BSD, p, blockIdx.x);
     }
 #pragma unroll 1
@@ -280,7 +287,9 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         const int L = ct.y;
         const uint32_t next = item + gridDim.x;
         if (pt < C) {
-            beta[pt] = pt < L ? __bfloat162float(p.beta[(size_t)(tok0 + pt) * p.H + h]) : 0.f;
+            const size_t at = (size_t)(tok0 + pt) * p.H + h;
+            beta[pt] = pt < L ? __bfloat162float(p.beta[at]) : 0.f;
+            if (SCALAR) gsc[pt] = pt < L ? __bfloat162float(p.g[at]) : 0.f;
             db[pt] = 0.f;
             __syncwarp();
             if (lane == 0) mbar_arrive(BLD);
@@ -300,8 +309,9 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         b.csum = reinterpret_cast<float *>(sm + Sm::CSUM);
         b.slow_flag = misc + 2;
         b.gout = gscr;
+        b.gsc = SCALAR ? gsc : nullptr;
         mbar_wait(BLD, it & 1u, abort_flag);
-        const int form = prep::gate<BAR, false, true>(b, pt, L);
+        const int form = SCALAR ? prep::gate_scalar<BAR, true>(b, pt, L) : prep::gate<BAR, false, true>(b, pt, L);
         fence_async_smem();
         named_barrier(BAR, kThreads);
         if (form != prep::kProductForm) {   // left to the step kernel
@@ -311,16 +321,19 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
                 const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
                 *reinterpret_cast<float4 *>(p.dq + e) = z;
                 *reinterpret_cast<float4 *>(p.dk + e) = z;
-                *reinterpret_cast<float4 *>(p.dg + e) = z;
+                if (!SCALAR) *reinterpret_cast<float4 *>(p.dg + e) = z;
             }
-            if (pt < L) p.dbeta[(size_t)(tok0 + pt) * p.H + h] = 0.f;
+            if (pt < L) {
+                p.dbeta[(size_t)(tok0 + pt) * p.H + h] = 0.f;
+                if (SCALAR) p.dg[(size_t)(tok0 + pt) * p.H + h] = 0.f;
+            }
             mbar_wait(BSD, n_sd & 1u, abort_flag);   // the item's states have landed
             ++n_sd;
             named_barrier(BAR, kThreads);
             if (leader) {
                 p.slow[item] = 1u;
                 if (next < total) {
-                    issue_raw(sm, BLD, tm_k, tm_q, tm_g, p, next);
+                    issue_raw<SCALAR>(sm, BLD, tm_k, tm_q, tm_g, p, next);
                     issue_states(sm, BSD, p, next);
                 }
             }
@@ -601,7 +614,7 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         ++n_mma2;
         // the next item's inputs go over tiles no product reads again
         if (leader && next < total) {
-            issue_raw(sm, BLD, tm_k, tm_q, tm_g, p, next);
+            issue_raw<SCALAR>(sm, BLD, tm_k, tm_q, tm_g, p, next);
             issue_states(sm, BSD, p, next);
         }
 
@@ -627,7 +640,7 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
                     const int t = tp + i;
                     const bool valid = t < L;
                     const size_t e = ((size_t)(tok0 + t) * p.H + h) * 128 + c;
-                    G[i] = gscr[t * 128 + c];
+                    G[i] = SCALAR ? gscr[t] : gscr[t * 128 + c];
                     kr[i] = valid ? __bfloat162float(p.k[e]) : 0.f;
                     qr[i] = valid ? __bfloat162float(p.q[e]) : 0.f;
                 }
@@ -657,12 +670,49 @@ kda_bwd_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
             xs[half * 128 + c] = sx;
             if (half) xs[256 + c] = up;
             named_barrier(BAR, kThreads);
-            float acc = xs[c] + xs[128 + c] + el * es[c] + (half ? 0.f : xs[256 + c]);
+            if (!SCALAR) {
+                float acc = xs[c] + xs[128 + c] + el * es[c] + (half ? 0.f : xs[256 + c]);
 #pragma unroll 4
-            for (int i = 31; i >= 0; --i) {
-                const int t = t0 + i;
-                acc += dGs[t * 128 + c];
-                if (t < L) p.dg[((size_t)(tok0 + t) * p.H + h) * 128 + c] = acc;
+                for (int i = 31; i >= 0; --i) {
+                    const int t = t0 + i;
+                    acc += dGs[t * 128 + c];
+                    if (t < L) p.dg[((size_t)(tok0 + t) * p.H + h) * 128 + c] = acc;
+                }
+            } else {
+                // one gate per token: dg_t = sum_{s >= t} sum_c dG[s][c] + sum_c (the
+                // G_L terms); four threads per token sum its row, then warp 0
+                // takes the running sum from the chunk end
+                float *rows = xs + 384;   // [64]
+                {
+                    const int t = pt >> 2, c0 = 32 * (pt & 3);
+                    float r = 0.f;
+#pragma unroll 8
+                    for (int j = 0; j < 32; ++j) r += dGs[t * 128 + c0 + j];
+                    r += __shfl_xor_sync(0xffffffffu, r, 1);
+                    r += __shfl_xor_sync(0xffffffffu, r, 2);
+                    if ((pt & 3) == 0) rows[t] = r;
+                }
+                named_barrier(BAR, kThreads);
+                if (warp == 0) {
+                    float base = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int cc = 4 * lane + e;
+                        base += xs[cc] + xs[128 + cc] + egl[cc] * es[cc];
+                    }
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) base += __shfl_xor_sync(0xffffffffu, base, off);
+                    const float a = rows[2 * lane], bb = rows[2 * lane + 1];
+                    float suf = a + bb;   // rows 2 lane .. 63, by a suffix scan over the lanes
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float v = __shfl_down_sync(0xffffffffu, suf, off);
+                        if (lane + off < 32) suf += v;
+                    }
+                    const size_t r0 = (size_t)(tok0 + 2 * lane) * p.H + h;
+                    if (2 * lane < L) p.dg[r0] = base + suf;
+                    if (2 * lane + 1 < L) p.dg[r0 + p.H] = base + suf - a;
+                }
             }
             if (pt < L) p.dbeta[(size_t)(tok0 + pt) * p.H + h] = db[pt];
         }
@@ -686,15 +736,19 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
                                const void *d_o, int64_t total_tokens, int H, const int2 *chunk_tab,
                                const uint32_t *total_chunks, const uint8_t *s_in, const uint8_t *ds_next, float *dq,
                                float *dk, float *dv, float *dg, float *dbeta, uint32_t *slow, float *gscr,
-                               uint32_t *err_word, int grid, cudaStream_t stream) {
+                               uint32_t *err_word, int grid, bool scalar_gate, cudaStream_t stream) {
     using namespace bwdtc;
     CUtensorMap mk, mq, mg, mdo;
     if (!make_bf16_map_3d(&mk, k, total_tokens, H, DK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_bf16_map_3d(&mq, q, total_tokens, H, DK, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_bf16_map_3d(&mg, g, total_tokens, H, DK, 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_bf16_map_3d(&mdo, d_o, total_tokens, H, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    cudaError_t e = set_max_dynamic_smem((const void *)kda_bwd_chunk_tc_kernel, (int)Sm::ALLOC);
+    if (scalar_gate) mg = mk;   // never read: the scalar gate comes in by plain loads
+    else if (!make_bf16_map_3d(&mg, g, total_tokens, H, DK, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    const void *fn = scalar_gate ? (const void *)kda_bwd_chunk_tc_kernel<true>
+                                 : (const void *)kda_bwd_chunk_tc_kernel<false>;
+    cudaError_t e = set_max_dynamic_smem(fn, (int)Sm::ALLOC);
     if (e != cudaSuccess) return e;
     Args a;
     a.q = static_cast<const __nv_bfloat16 *>(q);
@@ -716,7 +770,8 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
     a.gscr = gscr;
     a.err_word = err_word;
     a.H = H;
-    kda_bwd_chunk_tc_kernel<<<grid, kThreads, Sm::ALLOC, stream>>>(mk, mq, mg, mdo, a);
+    if (scalar_gate) kda_bwd_chunk_tc_kernel<true><<<grid, kThreads, Sm::ALLOC, stream>>>(mk, mq, mg, mdo, a);
+    else kda_bwd_chunk_tc_kernel<false><<<grid, kThreads, Sm::ALLOC, stream>>>(mk, mq, mg, mdo, a);
     return cudaGetLastError();
 }
 

@@ -67,7 +67,8 @@ struct Bufs {
     // (zero past the chunk end), or null for the per-channel gate in graw.
     const float *gsc;
     // gate<BAR, LAYER, true> also writes the running sums G (base-2 units,
-    // fp32 [64 t][128 c] row-major) here, for the backward pass
+    // fp32 [64 t][128 c] row-major) here, gate_scalar<BAR, true> the 64 per
+    // token, for the backward pass
     float *gout;
 };
 
@@ -238,7 +239,7 @@ __device__ int gate(const Bufs &b, int pt, int L) {
 // the channels, bit for bit.  A chunk that takes a slow path also gets the
 // gate spread over the channels in b.graw and the 16-token block sums in
 // b.csum, which those paths read.  Scratch: b.xf (the solve's, free here).
-template <int BAR>
+template <int BAR, bool GOUT = false>
 __device__ int gate_scalar(const Bufs &b, int pt, int L) {
     const int c = 2 * (pt & 63);
     const int tg = pt >> 6;
@@ -288,6 +289,7 @@ __device__ int gate_scalar(const Bufs &b, int pt, int L) {
         for (int jj = 0; jj < 3; ++jj)
             if (jj < j) off += bsum[jj];
         const float G = part[pt] + off;
+        if (GOUT) b.gout[pt] = G;   // one running sum per token (base-2 units)
         const float ih = exp2_f(fminf(-G, kMaxInv2));
         fac[pt] = make_float4(exp2_f(G), ih, slow ? exp2_f(GL - G) : eL * ih, 0.f);
     }

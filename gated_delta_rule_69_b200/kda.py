@@ -24,7 +24,8 @@ EXPORTED = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
             "kda_prefill_noalloc", "gdn_prefill", "gdn_decode_step", "kda_layer_prefill",
             "kda_layer_decode_step", "kda_cp_combine", "kda_cp_local", "kda_cp_finish",
             "kda_backward_workspace_size", "kda_backward", "gdn_backward",
-            "kda_backward_chunked_workspace_size", "kda_backward_chunked")
+            "kda_backward_chunked_workspace_size", "kda_backward_chunked", "gdn_backward_chunked",
+            "kda_layer_prefill_workspace_size")
 
 
 class KdaError(RuntimeError):
@@ -89,6 +90,8 @@ def lib():
         L.kda_backward_chunked.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, vp,
                                            vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.kda_backward_chunked.restype = ctypes.c_int
+        L.gdn_backward_chunked.argtypes = L.kda_backward_chunked.argtypes
+        L.gdn_backward_chunked.restype = ctypes.c_int
         L.kda_check_workspace_error.argtypes = [vp, vp]
         L.kda_check_workspace_error.restype = ctypes.c_int
         _lib = L
@@ -447,10 +450,27 @@ def kda_backward_chunked(q, k, v, log_alpha, beta, d_o, init_state=None, d_final
                          cu_seqlens=None, num_seqs=None, workspace=None, want_d_init_state=True,
                          stream=None):
     """kda_backward by chunks (bf16, d = 128): same arguments and outputs."""
-    T, H, dk = q.shape
-    dv = v.shape[-1]
     if log_alpha.shape != q.shape:
         raise ValueError("log_alpha must have q's shape [T, H, d_k]")
+    return _backward_chunked("kda_backward_chunked", q, k, v, log_alpha, beta, d_o, init_state,
+                             d_final_state, cu_seqlens, num_seqs, workspace, want_d_init_state, stream)
+
+
+def gdn_backward_chunked(q, k, v, log_alpha, beta, d_o, init_state=None, d_final_state=None,
+                         cu_seqlens=None, num_seqs=None, workspace=None, want_d_init_state=True,
+                         stream=None):
+    """kda_backward_chunked for the Gated DeltaNet gate (log_alpha and
+    dlog_alpha [T, H])."""
+    if log_alpha.shape != q.shape[:2]:
+        raise ValueError("log_alpha must be [T, H]")
+    return _backward_chunked("gdn_backward_chunked", q, k, v, log_alpha, beta, d_o, init_state,
+                             d_final_state, cu_seqlens, num_seqs, workspace, want_d_init_state, stream)
+
+
+def _backward_chunked(fn, q, k, v, log_alpha, beta, d_o, init_state, d_final_state, cu_seqlens,
+                      num_seqs, workspace, want_d_init_state, stream):
+    T, H, dk = q.shape
+    dv = v.shape[-1]
     if cu_seqlens is not None:
         n = cu_seqlens.numel() - 1
         if cu_seqlens.dtype != torch.int32:
@@ -462,18 +482,18 @@ def kda_backward_chunked(q, k, v, log_alpha, beta, d_o, init_state=None, d_final
         dq = torch.empty((T, H, dk), **f32)
         dkk = torch.empty((T, H, dk), **f32)
         dvv = torch.empty((T, H, dv), **f32)
-        dg = torch.empty((T, H, dk), **f32)
+        dg = torch.empty(tuple(log_alpha.shape), **f32)
         db = torch.empty((T, H), **f32)
         ds0 = torch.empty((n, H, dk, dv), **f32) if want_d_init_state else None
         if workspace is None:
             need = kda_backward_chunked_workspace_size(n, T, H)
             workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     _check_cuda(q, k, v, log_alpha, beta, d_o, init_state, d_final_state, cu_seqlens, workspace)
-    st = lib().kda_backward_chunked(
+    st = getattr(lib(), fn)(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
         _ptr(cu_seqlens), n, T, H, _ptr(d_o), _ptr(d_final_state), _ptr(dq), _ptr(dkk),
         _ptr(dvv), _ptr(dg), _ptr(db), _ptr(ds0), _ptr(workspace), workspace.numel(),
         _stream(stream, q.device))
     if st != KDA_OK:
-        raise KdaError(st, "kda_backward_chunked")
+        raise KdaError(st, fn)
     return dq, dkk, dvv, dg, db, ds0

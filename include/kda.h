@@ -356,6 +356,20 @@ kda_status kda_backward_chunked(const void *q, const void *k, const void *v, con
                                 kda_stream_t stream);
 
 /*
+ * gdn_backward_chunked: kda_backward_chunked for the Gated DeltaNet gate
+ * (log_alpha and dlog_alpha one value per token and head, [T_total, H]; the
+ * gradient is the channel sum of the per-channel one), the same stages and
+ * workspace size.
+ */
+kda_status gdn_backward_chunked(const void *q, const void *k, const void *v, const void *log_alpha,
+                                const void *beta, const float *init_state,
+                                const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                                int32_t H, const void *d_o, const float *d_final_state, float *dq,
+                                float *dk, float *dv, float *dlog_alpha, float *dbeta,
+                                float *d_init_state, void *workspace, size_t workspace_bytes,
+                                kda_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads the error word that the prefill and
  * backward kernels leave at the start of `workspace` (non-zero when a
  * device-side check failed, e.g. cu_seqlens not non-decreasing or not ending

@@ -107,3 +107,37 @@ def test_backward_chunked_slow_chunks_take_the_step_kernel():
     ref, cu, hs = run_oracle(inp)
     errs = errors(run(inp), ref, cu, hs)
     assert all(e <= TOL for e in errs.values()), errs
+
+
+@pytest.mark.parametrize("lengths", [[300], [1, 64, 65, 0, 190, 128]])
+def test_gdn_backward_chunked(lengths):
+    """The Gated DeltaNet gate (one log_alpha per token and head) through the
+    same chunked path, against the oracle's gdn derivative; dlog_alpha is the
+    channel sum of the per-channel one."""
+    inp = case(lengths, 3, seed=8)
+    inp["log_alpha"] = inp["log_alpha"][..., 0].contiguous()
+    ref, cu, hs = run_oracle(inp, scalar_gate=True)
+    out = kda().gdn_backward_chunked(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                                     inp["d_o"], init_state=inp["init_state"],
+                                     d_final_state=inp["d_final_state"], cu_seqlens=inp["cu_seqlens"])
+    torch.cuda.synchronize()
+    errs = errors([f64(x) for x in out], ref, cu, hs)
+    assert all(e <= TOL for e in errs.values()), errs
+
+
+def test_gdn_backward_chunked_slow_chunks():
+    """A scalar gate of -2 per token over one chunk of one head (-128 over the
+    chunk) and of -6 within a 16-token block of another: those chunks take the
+    step kernel, the rest the tensor cores."""
+    inp = case([300, 140], 2, seed=9)
+    g = inp["log_alpha"][..., 0].float().contiguous()
+    g[64:128, 0] = -2.0
+    g[128:192, 1] = -6.0
+    inp["log_alpha"] = g.to(inp["q"].dtype)
+    ref, cu, hs = run_oracle(inp, scalar_gate=True)
+    out = kda().gdn_backward_chunked(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                                     inp["d_o"], init_state=inp["init_state"],
+                                     d_final_state=inp["d_final_state"], cu_seqlens=inp["cu_seqlens"])
+    torch.cuda.synchronize()
+    errs = errors([f64(x) for x in out], ref, cu, hs)
+    assert all(e <= TOL for e in errs.values()), errs
