@@ -887,39 +887,53 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 // record operands keep their layout and descriptors; they only change side
 // (B instead of A), and V (its two 64-column atoms) is the A operand in the
 // MN-major form.
-// The state-independent halves of the products, V_n^T YT_n^T into X and
-// V_n^T ZB_n^T into O, are issued ahead, while the chain warps still work on
-// the previous state, so that once SB_n is in TMEM only SB_n^T MP_n^T (8
-// products) stands between it and S_{n+1}; SB_n^T QP_n^T and the next
-// chunk's state-independent products then keep the tensor pipe busy while
-// the chain warps read X_n out.  X and O are double-buffered in TMEM.
-// Four rings, each with its own loader warp (exp(G_L) travels with ring A
-// but has its own deeper ring, since the chain warps read it only after the
-// state products): A (MP, YT), E (exp(G_L)), V (the v tile, read from HBM)
-// and B (QP, ZB).
-//   warp 0: rings A and E;  warp 18: ring B;  warp 19: ring V
+// A tcgen05 product costs about the same whatever its N up to 192 (~100
+// cycles per M = 128, K = 16 instruction with A in shared memory, ~116 with
+// A in TMEM, against ~134 at N = 256), so the products that share their A
+// operand are issued as one: X and O^T lie side by side in TMEM (X in 128
+// columns, O^T in the next 64) and the record's B operands side by side in
+// shared memory (MP over QP, YT over ZB):
+//     [X | O^T]  = V_n^T [YT_n; ZB_n]^T        (4 products, N = 192)
+//     [X | O^T] += SB_n^T [MP_n; QP_n]^T       (8 products, N = 192)
+// The state-independent group is issued ahead, while the chain warps still
+// work on the previous state, so that once SB_n is in TMEM only the second
+// group stands between it and S_{n+1}.  [X | O^T] is double-buffered in TMEM.
+// The chain warps read O^T out together with X and, once SB_{n+1} is handed
+// over, write it in bf16 to a shared-memory staging tile that a store warp
+// copies to o with one tensor store per chunk (stores from the chain warps'
+// registers straight to global memory, 16 of 64 bytes per warp and chunk,
+// took most of a chunk's period).  The backward scan modes stage the state tiles they
+// save the same way, and one bulk copy per chunk writes each out.
+// Rings, each with its loader warp: R (MP, QP, YT, ZB of a record in the
+// layout above), E (exp(G_L); its own deeper ring, since the chain warps read
+// it only after the state products) and V (the v tile, read from HBM).
+//   warp 0: rings R and E;  warp 18: the stores;  warp 19: ring V
 //   warps 1..16: the state; warp w holds lanes j of quadrant w mod 4 and
 //                columns c in 32 ((w - 1) / 4) .. + 31
 //   warp 17: issues the products
 struct ChainT {
     static constexpr int NCW = 16;
     static constexpr int THREADS = 32 * (NCW + 4);
-    static constexpr int NSA = 2, NSB = 2, NSV = 4, NSE = 4;
-    static constexpr uint32_t A_MP = 0, A_YT = 32768, A_STRIDE = 49152;
-    static constexpr uint32_t B_QP = 0, B_ZB = 16384, B_STRIDE = 24576;
+    static constexpr int NSR = 2, NSV = 3, NSE = 3;
+    // ring R stage: K-atom 0 of MP (128 rows c) over K-atom 0 of QP (64 rows t),
+    // the same for K-atom 1, then YT (128 rows c) over ZB (64 rows t)
+    static constexpr uint32_t R_MP = 0, R_QP = 16384, R_KATOM = 24576, R_YT = 49152, R_ZB = 65536;
+    static constexpr uint32_t R_STRIDE = 73728;
     static constexpr uint32_t V_STRIDE = 16384;
-    static constexpr uint32_t RA = 0;
-    static constexpr uint32_t RV = NSA * A_STRIDE;
-    static constexpr uint32_t RB = RV + NSV * V_STRIDE;
-    static constexpr uint32_t EGLR = RB + NSB * B_STRIDE;   // NSE x exp(G_L), 128 fp32 each
+    static constexpr uint32_t RR = 0;
+    static constexpr uint32_t RV = NSR * R_STRIDE;
+    static constexpr uint32_t STG = RV + NSV * V_STRIDE;   // 2 x 16 KB of o rows, or one 32 KB state tile
+    static constexpr uint32_t EGLR = STG + 32768;          // NSE x exp(G_L), 128 fp32 each
     static constexpr uint32_t BARS = EGLR + NSE * 512;
     static constexpr uint32_t MISC = BARS + 256;
     static constexpr uint32_t SIZE = MISC + 64;
     static constexpr uint32_t ALLOC = SIZE + 1024;
-    // TMEM columns: X fp32 x 2 (128 each), SB^T bf16 pairs x 2 (64 each),
-    // O^T fp32 x 2 (64 each)
+    // TMEM columns: [X | O^T] x 2 (X fp32 in 128 columns, O^T fp32 in 64),
+    // SB^T bf16 pairs x 2 (64 each)
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t COL_X = 0, COL_SB = 256, COL_O = 384;
+    static constexpr uint32_t COL_XO = 0, XO_STRIDE = 192, COL_O = 128, COL_SB = 384;
+    static_assert(R_QP == 16384 && R_KATOM == R_QP + 8192 && R_ZB == R_YT + 16384,
+                  "B operands of one product group must be contiguous rows");
     static_assert(ALLOC <= 232448, "chain shared memory");
 };
 
@@ -938,15 +952,16 @@ enum : int { kChainPlain = 0, kChainTransition = 2, kChainSaveS = 3, kChainRever
 
 // The chain of one (sequence, head) unit (rank `unit` in the longest-first
 // order); the kernels below run one unit per CTA.
+// tm_o (the output mode only): o as [64 tokens][128 channels] boxes of one head.
 template <int MODE>
-__device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const Params &p, int unit) {
+__device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const CUtensorMap *tm_o, const Params &p,
+                                             int unit) {
     constexpr bool TRANS = MODE == kChainTransition;
     constexpr bool SAVE = MODE == kChainSaveS;
     constexpr bool REV = MODE == kChainReverse;
     constexpr bool OUT = MODE == kChainPlain;          // output products and stores
-    constexpr bool RING_B = OUT || REV;                // QP (and ZB) travel
     using Cfg = ChainT;
-    constexpr int NSA = Cfg::NSA, NSB = Cfg::NSB, NSV = Cfg::NSV, NSE = Cfg::NSE, NCW = Cfg::NCW;
+    constexpr int NSR = Cfg::NSR, NSV = Cfg::NSV, NSE = Cfg::NSE, NCW = Cfg::NCW;
 
     extern __shared__ uint8_t dyn_smem[];
     uint8_t *sm = dyn_smem + ((1024u - (smem_addr(dyn_smem) & 1023u)) & 1023u);
@@ -959,24 +974,24 @@ __device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const Para
     const int64_t len = eos - bos;
     const int nchunks = (int)((len + C - 1) / C);
     const size_t rec0 = (size_t)p.chunk_off[seq];
+    const bool stage_states = (SAVE || REV) && p.states_out != nullptr;
 
-    // mbarriers: FULLA[NSA], EMPTYA[NSA], FULLB[NSB], EMPTYB[NSB], FULLV[NSV], EMPTYV[NSV],
-    // FULLE[NSE], EMPTYE[NSE], SDONE, ODONE[2], FIN, SREADY, OFREE[2]
+    // mbarriers: FULLR[NSR], EMPTYR[NSR], FULLV[NSV], EMPTYV[NSV], FULLE[NSE],
+    // EMPTYE[NSE], SDONE, FIN, SREADY, STGF[2], STGE[2]
     uint64_t *B = reinterpret_cast<uint64_t *>(sm + Cfg::BARS);
-    uint64_t *FULLA = B, *EMPTYA = B + NSA, *FULLB = B + 2 * NSA, *EMPTYB = B + 2 * NSA + NSB;
-    uint64_t *FULLV = B + 2 * NSA + 2 * NSB, *EMPTYV = FULLV + NSV;
+    uint64_t *FULLR = B, *EMPTYR = B + NSR, *FULLV = B + 2 * NSR, *EMPTYV = FULLV + NSV;
     uint64_t *FULLE = EMPTYV + NSV, *EMPTYE = FULLE + NSE;
-    uint64_t *SDONE = EMPTYE + NSE, *ODONE = SDONE + 1, *FIN = SDONE + 3, *SREADY = SDONE + 4;
-    uint64_t *OFREE = SDONE + 5;
-    constexpr int kBars = 2 * NSA + 2 * NSB + 2 * NSV + 2 * NSE + 7;
+    uint64_t *SDONE = EMPTYE + NSE, *FIN = SDONE + 1, *SREADY = SDONE + 2;
+    uint64_t *STGF = SDONE + 3, *STGE = SDONE + 5;
+    constexpr int kBars = 2 * NSR + 2 * NSV + 2 * NSE + 7;
     static_assert(kBars * 8 <= 256, "barrier area");
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + Cfg::MISC);
     volatile uint32_t *abort_flag = misc + 1;
     if (tid == 0) {
         for (int i = 0; i < kBars; ++i) {
-            // SREADY, EMPTYE and OFREE take one arrive per chain warp
+            // SREADY, EMPTYE and STGF take one arrive per chain warp
             const uint64_t *b = &B[i];
-            const bool per_warp = b == SREADY || b == &OFREE[0] || b == &OFREE[1] ||
+            const bool per_warp = b == SREADY || b == &STGF[0] || b == &STGF[1] ||
                                   (b >= EMPTYE && b < EMPTYE + NSE);
             mbar_init(&B[i], per_warp ? (uint32_t)NCW : 1u);
         }
@@ -993,30 +1008,40 @@ __device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const Para
     const uint32_t tmem = misc[0];
 
     if (warp == 0) {
-        // ---------------------------------------------- rings A (MP, YT) and E (exp(G_L))
+        // ---------------------------------------------- rings R (MP, QP, YT, ZB) and E (exp(G_L))
         if (lane == 0 && nchunks > 0) {
-            int issued_a = 0, issued_e = 0;
+            int issued_r = 0, issued_e = 0;
             for (int n = 0; n < nchunks; ++n) {
-                const int sa = n % NSA, se = n % NSE;
-                if (n >= NSA) mbar_wait(&EMPTYA[sa], ((n / NSA) - 1) & 1, abort_flag);
+                const int sr = n % NSR, se = n % NSE;
+                if (n >= NSR) mbar_wait(&EMPTYR[sr], ((n / NSR) - 1) & 1, abort_flag);
                 if (n >= NSE) mbar_wait(&EMPTYE[se], ((n / NSE) - 1) & 1, abort_flag);
                 if (*abort_flag) break;
                 const int nn = REV ? nchunks - 1 - n : n;
                 const size_t ri = (rec0 + nn) * p.H + h;
                 const uint8_t *rec = p.recs + ri * Rec::STRIDE;
                 if (p.rec_ready && !acquire_flag(p.rec_ready + ri, abort_flag)) break;   // the record is complete
-                uint8_t *slot_a = sm + Cfg::RA + sa * Cfg::A_STRIDE;
-                constexpr uint32_t kABytes = REV ? 32768 : 49152;   // MP (and YT)
-                mbar_arrive_expect_tx(&FULLA[sa], kABytes);
-                bulk_load(slot_a + Cfg::A_MP, rec + Rec::MP, kABytes, &FULLA[sa]);
-                issued_a = n + 1;
+                uint8_t *slot = sm + Cfg::RR + sr * Cfg::R_STRIDE;
+                // MP always; QP for the output (and, read MN-major, the reverse scan);
+                // YT wherever v enters; ZB for the output
+                constexpr uint32_t kRBytes = 32768 + ((OUT || REV) ? 16384 : 0) + ((OUT || SAVE) ? 16384 : 0) +
+                                             (OUT ? 8192 : 0);
+                mbar_arrive_expect_tx(&FULLR[sr], kRBytes);
+                bulk_load(slot + Cfg::R_MP, rec + Rec::MP, 16384, &FULLR[sr]);
+                bulk_load(slot + Cfg::R_MP + Cfg::R_KATOM, rec + Rec::MP + 16384, 16384, &FULLR[sr]);
+                if (OUT || REV) {
+                    bulk_load(slot + Cfg::R_QP, rec + Rec::QP, 8192, &FULLR[sr]);
+                    bulk_load(slot + Cfg::R_QP + Cfg::R_KATOM, rec + Rec::QP + 8192, 8192, &FULLR[sr]);
+                }
+                if (OUT || SAVE) bulk_load(slot + Cfg::R_YT, rec + Rec::YT, 16384, &FULLR[sr]);
+                if (OUT) bulk_load(slot + Cfg::R_ZB, rec + Rec::ZB, 8192, &FULLR[sr]);
+                issued_r = n + 1;
                 mbar_arrive_expect_tx(&FULLE[se], 512);
                 bulk_load(sm + Cfg::EGLR + se * 512, rec + Rec::EGL, 512, &FULLE[se]);
                 issued_e = n + 1;
             }
             // the copies land before this CTA may exit
-            for (int n = (issued_a > NSA ? issued_a - NSA : 0); n < issued_a; ++n)
-                wait_drain(&FULLA[n % NSA], (n / NSA) & 1);
+            for (int n = (issued_r > NSR ? issued_r - NSR : 0); n < issued_r; ++n)
+                wait_drain(&FULLR[n % NSR], (n / NSR) & 1);
             for (int n = (issued_e > NSE ? issued_e - NSE : 0); n < issued_e; ++n)
                 wait_drain(&FULLE[n % NSE], (n / NSE) & 1);
         }
@@ -1040,96 +1065,98 @@ __device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const Para
                 wait_drain(&FULLV[n % NSV], (n / NSV) & 1);
         }
     } else if (warp == NCW + 2) {
-        // ---------------------------------------------- ring B: QP, ZB
-        if (RING_B && lane == 0 && nchunks > 0) {
-            int issued_b = 0;
-            for (int n = 0; n < nchunks; ++n) {
-                const int sb = n % NSB;
-                if (n >= NSB) mbar_wait(&EMPTYB[sb], ((n / NSB) - 1) & 1, abort_flag);
+        // ---------------------------------------------- stores from the staging tiles
+        if (OUT && nchunks > 0) {
+            // chunk m's o rows: buffer m mod 2, row r (token m C + r) at r * 256
+            // bytes.  A whole chunk goes out as one tensor store; a sequence's
+            // partial last chunk row by row in 16-byte pieces (16 lanes per row),
+            // since the box's further rows belong to the next sequence.
+            if (lane == 0) tma_prefetch_desc(tm_o);
+            for (int m = 0; m < nchunks; ++m) {
+                const int b = m & 1;
+                mbar_wait(&STGF[b], (m >> 1) & 1, abort_flag);
                 if (*abort_flag) break;
-                const size_t ri = (rec0 + (REV ? nchunks - 1 - n : n)) * p.H + h;
-                const uint8_t *rec = p.recs + ri * Rec::STRIDE;
-                if (p.rec_ready && !acquire_flag(p.rec_ready + ri, abort_flag)) break;
-                uint8_t *slot_b = sm + Cfg::RB + sb * Cfg::B_STRIDE;
-                constexpr uint32_t kBBytes = REV ? 16384 : 24576;   // QP (and ZB)
-                mbar_arrive_expect_tx(&FULLB[sb], kBBytes);
-                bulk_load(slot_b + Cfg::B_QP, rec + Rec::QP, kBBytes, &FULLB[sb]);
-                issued_b = n + 1;
+                const uint8_t *src = sm + Cfg::STG + b * 16384;
+                const int rows = (int)min((int64_t)C, len - (int64_t)m * C);
+                if (rows == C) {
+                    if (lane == 0) {
+                        tma_store_3d(tm_o, src, 0, h, (int)(bos + (int64_t)m * C));
+                        bulk_commit();
+                        bulk_wait_read_all();
+                    }
+                } else {
+#pragma unroll 4
+                    for (int it = 0; it < 32; ++it) {
+                        const int r = 2 * it + (lane >> 4), piece = lane & 15;
+                        if (r < rows) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(src + r * 256 + piece * 16);
+                            *reinterpret_cast<uint4 *>(p.o + ((size_t)(bos + (int64_t)m * C + r) * p.H + h) * DV +
+                                                       piece * 8) = v;
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&STGE[b]);
             }
-            for (int n = (issued_b > NSB ? issued_b - NSB : 0); n < issued_b; ++n)
-                wait_drain(&FULLB[n % NSB], (n / NSB) & 1);
+            if (lane == 0) bulk_wait_all();
+        } else if (stage_states && lane == 0 && nchunks > 0) {
+            // the state tile (two 16 KB halves over j) of each chunk
+            for (int n = 0; n < nchunks; ++n) {
+                mbar_wait(&STGF[0], n & 1, abort_flag);
+                if (*abort_flag) break;
+                const int nn = REV ? nchunks - 1 - n : n;
+                bulk_store(p.states_out + ((rec0 + nn) * p.H + h) * (size_t)32768, sm + Cfg::STG, 32768);
+                bulk_commit();
+                bulk_wait_read_all();
+                mbar_arrive(&STGE[0]);
+            }
+            bulk_wait_all();
         }
     } else if (warp == NCW + 1) {
         // ---------------------------------------------- tensor-core products
-        // reverse scan: B = MP and QP themselves, read MN-major
-        const uint32_t idS = idesc_bf16(128, 128, false, REV);     // A = SB^T (TMEM), B = MP^T (MP)
-        const uint32_t idSV = idesc_bf16(128, 128, true, REV);     // A = V^T (MN-major), B = YT^T (QP)
-        const uint32_t idO = idesc_bf16(128, 64, false, false);    // A = SB^T (TMEM), B = QP^T
-        const uint32_t idOV = idesc_bf16(128, 64, true, false);    // A = V^T (MN-major), B = ZB^T
-        // The state-independent products of chunk m: X[m mod 2] = V^T YT^T and
-        // O[m mod 2] = V^T ZB^T.  X[m mod 2] was last read by the chain warps
-        // before their SREADY of chunk m - 1, which this warp has passed; O[m
-        // mod 2] is free once they have read O_{m-2} out (OFREE).
+        // N = 192 where the output products ride along, else 128; the reverse
+        // scan's B operands (MP and QP themselves) are read MN-major
+        constexpr int NP = OUT ? 192 : 128;
+        const uint32_t idS = idesc_bf16(128, NP, false, REV);   // A = SB^T (TMEM), B = [MP; QP]^T
+        const uint32_t idP = idesc_bf16(128, NP, true, REV);    // A = V^T (MN-major), B = [YT; ZB]^T
+        // The state-independent group of chunk m into [X | O^T][m mod 2], which
+        // the chain warps read out (X and O^T) before their SREADY of chunk m - 1,
+        // which this warp has passed.
         auto pre = [&](int m) {
             if (TRANS) return;
-            const int sa = m % NSA, sb = m % NSB, sv = m % NSV;
-            const uint32_t bY = smem_addr(sm + Cfg::RA + sa * Cfg::A_STRIDE + Cfg::A_YT);
-            const uint32_t bQ = smem_addr(sm + Cfg::RB + sb * Cfg::B_STRIDE + Cfg::B_QP);
-            const uint32_t bZ = smem_addr(sm + Cfg::RB + sb * Cfg::B_STRIDE + Cfg::B_ZB);
+            const int sr = m % NSR, sv = m % NSV;
+            const uint32_t slot = smem_addr(sm + Cfg::RR + sr * Cfg::R_STRIDE);
             const uint32_t aV = smem_addr(sm + Cfg::RV + sv * Cfg::V_STRIDE);
-            mbar_wait(&FULLA[sa], (m / NSA) & 1, abort_flag);
+            const uint32_t d = tmem + Cfg::COL_XO + Cfg::XO_STRIDE * (uint32_t)(m & 1);
+            mbar_wait(&FULLR[sr], (m / NSR) & 1, abort_flag);
             mbar_wait(&FULLV[sv], (m / NSV) & 1, abort_flag);
-            if (REV) mbar_wait(&FULLB[sb], (m / NSB) & 1, abort_flag);
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)   // X = V^T YT^T, or dO^T QP  (K = t)
-                mma_bf16_warp(tmem + Cfg::COL_X + 128u * (uint32_t)(m & 1),
-                              smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
-                              REV ? smem_desc(bQ + ks * 2048, 8192, 1024, kLayoutSW128)
-                                  : smem_desc(bY + ks * 32, 16, 1024, kLayoutSW128),
-                              idSV, ks > 0 ? 1u : 0u);
-            if (!OUT) {   // no output products: v (dO) and QP are free again
-                mma_commit_warp(&EMPTYV[sv]);
-                if (REV) mma_commit_warp(&EMPTYB[sb]);
-                return;
-            }
-            mbar_wait(&FULLB[sb], (m / NSB) & 1, abort_flag);
-            if (m >= 2) mbar_wait(&OFREE[m & 1], ((m - 2) >> 1) & 1, abort_flag);
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)   // O^T = V^T ZB^T  (K = t')
-                mma_bf16_warp(tmem + Cfg::COL_O + 64u * (uint32_t)(m & 1),
-                              smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
-                              smem_desc(bZ + ks * 32, 16, 1024, kLayoutSW128), idOV, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks)   // V^T [YT; ZB]^T, or dO^T QP  (K = t)
+                mma_bf16_warp(d, smem_desc(aV + ks * 2048, 8192, 1024, kLayoutSW128),
+                              REV ? smem_desc(slot + Cfg::R_QP + ks * 2048, Cfg::R_KATOM, 1024, kLayoutSW128)
+                                  : smem_desc(slot + Cfg::R_YT + ks * 32, 16, 1024, kLayoutSW128),
+                              idP, ks > 0 ? 1u : 0u);
             mma_commit_warp(&EMPTYV[sv]);
         };
         if (nchunks > 0) pre(0);
         for (int n = 0; n < nchunks; ++n) {
-            const int sa = n % NSA, sb = n % NSB;
-            const uint32_t bM = smem_addr(sm + Cfg::RA + sa * Cfg::A_STRIDE + Cfg::A_MP);
+            const int sr = n % NSR;
+            const uint32_t slot = smem_addr(sm + Cfg::RR + sr * Cfg::R_STRIDE);
             const uint32_t aSB = tmem + Cfg::COL_SB + 64u * (uint32_t)(n & 1);
-            if (TRANS) mbar_wait(&FULLA[sa], (n / NSA) & 1, abort_flag);
+            const uint32_t d = tmem + Cfg::COL_XO + Cfg::XO_STRIDE * (uint32_t)(n & 1);
+            if (TRANS) mbar_wait(&FULLR[sr], (n / NSR) & 1, abort_flag);
             mbar_wait(SREADY, n & 1, abort_flag);
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)   // X += SB^T MP^T, or GB^T MP  (K = c')
-                mma_bf16_ts_warp(tmem + Cfg::COL_X + 128u * (uint32_t)(n & 1), aSB + 8 * ks,
-                                 REV ? smem_desc(bM + ks * 2048, 16384, 1024, kLayoutSW128)
-                                     : smem_desc(bM + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
+            for (int ks = 0; ks < 8; ++ks)   // SB^T [MP; QP]^T, or GB^T MP  (K = c')
+                mma_bf16_ts_warp(d, aSB + 8 * ks,
+                                 REV ? smem_desc(slot + Cfg::R_MP + ks * 2048, Cfg::R_KATOM, 1024, kLayoutSW128)
+                                     : smem_desc(slot + Cfg::R_MP + (ks >> 2) * Cfg::R_KATOM + (ks & 3) * 32, 16,
+                                                 1024, kLayoutSW128),
                                  idS, (TRANS && ks == 0) ? 0u : 1u);
             mma_commit_warp(SDONE);
-            mma_commit_warp(&EMPTYA[sa]);
-            if (OUT) {
-                const uint32_t bQ = smem_addr(sm + Cfg::RB + sb * Cfg::B_STRIDE + Cfg::B_QP);
-                const uint32_t dO = tmem + Cfg::COL_O + 64u * (uint32_t)(n & 1);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)   // O^T += SB^T QP^T  (K = c)
-                    mma_bf16_ts_warp(dO, aSB + 8 * ks,
-                                     smem_desc(bQ + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                                     idO, 1u);
-                mma_commit_warp(&ODONE[n & 1]);
-                mma_commit_warp(&EMPTYB[sb]);
-            }
+            mma_commit_warp(&EMPTYR[sr]);
             if (n + 1 < nchunks) pre(n + 1);
         }
         if (nchunks > 0) {   // every arrive of the commits above lands before the CTA exits
@@ -1153,31 +1180,21 @@ __device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const Para
 #pragma unroll
             for (int i = 0; i < 32; ++i) S[i] = 0.f;
         }
-        // O^T of chunk m: this warp's 16 t columns, lane j, bf16 to o[t][h][j];
-        // the buffer is released (OFREE) as soon as it is in registers
-        auto store_o_t = [&](int m) {
-            mbar_wait(&ODONE[m & 1], (m >> 1) & 1, abort_flag);
-            tc_fence_after();
-            float v[16];
-            tmem_ld16(tmem_addr(tmem, 32 * quad, Cfg::COL_O + 64 * (m & 1) + 16 * g), v);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&OFREE[m & 1]);
-            const int64_t t0 = (int64_t)m * C + 16 * g;
-            __nv_bfloat16 *dst = p.o + ((size_t)(bos + t0) * p.H + h) * DV + j;
+        // O^T of chunk m (this warp's 16 t columns, lane j), read out with X_m,
+        // into staging buffer m mod 2 as o rows [t][j]; the buffer's previous
+        // rows (chunk m - 2) have been copied out once STGE says so
+        float ov[16];
+        auto stage_o = [&](int m) {
+            const int b = m & 1;
+            if (m >= 2) mbar_wait(&STGE[b], ((m - 2) >> 1) & 1, abort_flag);
+            __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(sm + Cfg::STG + b * 16384) + (16 * g) * DV + j;
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (t0 + i < len) dst[(size_t)i * p.H * DV] = __float2bfloat16(v[i]);
+            for (int i = 0; i < 16; ++i) st[i * DV] = __float2bfloat16(ov[i]);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&STGF[b]);
         };
         for (int n = 0; n < nchunks; ++n) {
-            if ((SAVE || REV) && p.states_out) {   // the state entering (forward) or leaving (reverse) this chunk
-                const int nn = REV ? nchunks - 1 - n : n;
-                uint8_t *tile = p.states_out + ((rec0 + nn) * p.H + h) * (size_t)32768 + (j >> 6) * 16384;
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    *reinterpret_cast<__nv_bfloat16 *>(tile + sw128_off(32 * g + i, j & 63)) = __float2bfloat16(S[i]);
-            }
             // SB_n^T: column COL_SB + 64 (n mod 2) + c / 2 holds (c, c + 1).  Its
             // previous contents, SB_{n-2}, were last read by chunk n - 2's
             // products, which completed before SDONE of chunk n - 1.
@@ -1189,17 +1206,29 @@ __device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const Para
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(SREADY);
-            if (OUT && n >= 1) store_o_t(n - 1);
+            if (stage_states) {   // the state entering (forward) or leaving (reverse) this chunk
+                if (n >= 1) mbar_wait(&STGE[0], (n - 1) & 1, abort_flag);
+                uint8_t *tile = sm + Cfg::STG + (j >> 6) * 16384;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    *reinterpret_cast<__nv_bfloat16 *>(tile + sw128_off(32 * g + i, j & 63)) = __float2bfloat16(S[i]);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&STGF[0]);
+            }
+            if (OUT && n >= 1) stage_o(n - 1);
             // S_{n+1} = S_n Diag(exp(G_L)) + X_n, in two halves of 16 columns
             const int se = n % NSE;
             mbar_wait(&FULLE[se], (n / NSE) & 1, abort_flag);
             mbar_wait(SDONE, n & 1, abort_flag);
             tc_fence_after();
             const float4 *egl = reinterpret_cast<const float4 *>(sm + Cfg::EGLR + se * 512) + 8 * g;
+            const uint32_t xo = Cfg::COL_XO + Cfg::XO_STRIDE * (n & 1);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 float x[16];
-                tmem_ld16(tmem_addr(tmem, 32 * quad, Cfg::COL_X + 128 * (n & 1) + 32 * g + 16 * hh), x);
+                tmem_ld16(tmem_addr(tmem, 32 * quad, xo + 32 * g + 16 * hh), x);
+                if (OUT && hh == 1) tmem_ld16(tmem_addr(tmem, 32 * quad, xo + Cfg::COL_O + 16 * g), ov);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
@@ -1214,7 +1243,7 @@ __device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const Para
             __syncwarp();
             if (lane == 0) mbar_arrive(&EMPTYE[se]);
         }
-        if (OUT && nchunks > 0) store_o_t(nchunks - 1);
+        if (OUT && nchunks > 0) stage_o(nchunks - 1);
         if (p.final_state) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) p.final_state[sbase + (size_t)i * DV] = S[i];
@@ -1231,8 +1260,9 @@ __device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const Para
 
 template <int MODE>
 __global__ void __launch_bounds__(ChainT::THREADS, 1)
-kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
-    chain_t_unit<MODE>(tm_v, p, (int)blockIdx.x);
+kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                   const Params p) {
+    chain_t_unit<MODE>(tm_v, &tm_o, p, (int)blockIdx.x);
 }
 
 // The backward pass's two scans in one grid: CTAs [0, units) run the forward
@@ -1241,8 +1271,8 @@ kda_chain_t_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 __global__ void __launch_bounds__(ChainT::THREADS, 1)
 kda_backward_scans_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                           const Params pf, const Params pr, int units) {
-    if ((int)blockIdx.x < units) chain_t_unit<kChainSaveS>(tm_v, pf, (int)blockIdx.x);
-    else chain_t_unit<kChainReverse>(tm_do, pr, (int)blockIdx.x - units);
+    if ((int)blockIdx.x < units) chain_t_unit<kChainSaveS>(tm_v, nullptr, pf, (int)blockIdx.x);
+    else chain_t_unit<kChainReverse>(tm_do, nullptr, pr, (int)blockIdx.x - units);
 }
 
 // A segment's two local chains for context parallelism in one grid: CTAs
@@ -1252,8 +1282,8 @@ kda_backward_scans_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid
 __global__ void __launch_bounds__(ChainT::THREADS, 1)
 kda_cp_local_chains_kernel(const __grid_constant__ CUtensorMap tm_v, const Params pl, const Params pt,
                            int units) {
-    if ((int)blockIdx.x < units) chain_t_unit<kChainSaveS>(tm_v, pl, (int)blockIdx.x);
-    else chain_t_unit<kChainTransition>(tm_v, pt, (int)blockIdx.x - units);
+    if ((int)blockIdx.x < units) chain_t_unit<kChainSaveS>(tm_v, nullptr, pl, (int)blockIdx.x);
+    else chain_t_unit<kChainTransition>(tm_v, nullptr, pt, (int)blockIdx.x - units);
 }
 
 // =============================================================== layer prologue
@@ -1573,8 +1603,11 @@ cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const spl
                            unsigned units, bool overlap, cudaStream_t stream,
                            int mode = split::kChainPlain) {
     using namespace split;
-    CUtensorMap mv;
+    CUtensorMap mv, mo;
     if (!make_map_split(&mv, v, total_tokens, H, DV, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (mode != kChainPlain) mo = mv;   // not read
+    else if (!make_map_split(&mo, prm.o, total_tokens, H, DV, DV, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     {
         const void *fn = mode == kChainTransition ? (const void *)kda_chain_t_kernel<kChainTransition>
@@ -1595,10 +1628,10 @@ cudaError_t launch_chain_t(const void *v, int64_t total_tokens, int H, const spl
     cfg.attrs = attr;
     cfg.numAttrs = overlap ? 1 : 0;
     const cudaError_t e =
-        mode == kChainTransition ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainTransition>, mv, prm)
-        : mode == kChainSaveS    ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainSaveS>, mv, prm)
-        : mode == kChainReverse  ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainReverse>, mv, prm)
-                                 : cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainPlain>, mv, prm);
+        mode == kChainTransition ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainTransition>, mv, mo, prm)
+        : mode == kChainSaveS    ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainSaveS>, mv, mo, prm)
+        : mode == kChainReverse  ? cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainReverse>, mv, mo, prm)
+                                 : cudaLaunchKernelEx(&cfg, kda_chain_t_kernel<kChainPlain>, mv, mo, prm);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
