@@ -45,10 +45,10 @@ BACKWARD_DEFAULT = "prefill_T4096_H16_d128"
 DECODE_DEFAULT = "decode_B256_H32_d128"
 # DRAM bytes (read + write) of one whole kda_prefill call, from an ncu
 # application-range capture over one call of the 16384-token, 32-head workload
-# (547.5 MB read + 693.4 MB written), scaled by the token count to the
+# (597.9 MB read + 694.3 MB written), scaled by the token count to the
 # 131072-token workload, which runs the same plan and per-chunk schedule
 # (profiles/kda_prefill_T131072_H32_d128.md); null for other workloads.
-CALL_TRAFFIC = {"prefill_T131072_H32_d128": (547.5e6 + 693.4e6) * 131072 / 16384}
+CALL_TRAFFIC = {"prefill_T131072_H32_d128": (597.9e6 + 694.3e6) * 131072 / 16384}
 # the oracle's sample: whole heads of the first sequence, at most this many
 # of its first tokens (its cost is linear in (token, head) pairs)
 ORACLE_PREFIX = 32768
