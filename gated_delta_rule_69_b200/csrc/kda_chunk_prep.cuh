@@ -94,7 +94,10 @@ __device__ __forceinline__ int tfi(int row, int col) { return row * kTStride + c
 // reference per block) or kPairwise.
 enum : int { kProductForm = 0, kSecondary = 1, kPairwise = 2 };
 
-template <int BAR, bool LAYER, bool GOUT = false>
+// LAYER: 0 plain; 1 the layer prologue (z -> log_alpha, the norms of the raw
+// q and k rows formed here and left in b.nrm); 2 raw q and k scaled by the
+// inverse norms already in b.nrm.
+template <int BAR, int LAYER, bool GOUT = false>
 __device__ int gate(const Bufs &b, int pt, int L) {
     const int c = 2 * (pt & 63);
     const int tg = pt >> 6;
@@ -117,7 +120,8 @@ __device__ int gate(const Bufs &b, int pt, int L) {
         named_barrier(BAR, kGroupThreads);
     }
 
-    constexpr bool layer = LAYER;   // the prologue (b.nrm set)
+    constexpr bool layer = LAYER == 1;    // the prologue
+    constexpr bool scaled = LAYER != 0;   // q and k scaled by b.nrm
     uint32_t graw_v[16], k_v[16], q_v[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -209,7 +213,7 @@ __device__ int gate(const Bufs &b, int pt, int L) {
         const int t = t0 + i;
         const __nv_bfloat162 kv = *reinterpret_cast<const __nv_bfloat162 *>(&k_v[i]);
         const __nv_bfloat162 qv = *reinterpret_cast<const __nv_bfloat162 *>(&q_v[i]);
-        const float nk = layer ? b.nrm[t] : 1.f, nq = layer ? b.nrm[64 + t] : 1.f;
+        const float nk = scaled ? b.nrm[t] : 1.f, nq = scaled ? b.nrm[64 + t] : 1.f;
         const float k0 = __low2float(kv) * nk, k1 = __high2float(kv) * nk;
         const float q0 = __low2float(qv) * nq, q1 = __high2float(qv) * nq;
         const float G0 = g0[i] + off0, G1 = g1[i] + off1;

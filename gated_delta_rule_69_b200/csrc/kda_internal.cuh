@@ -116,9 +116,10 @@ size_t prefill_split_workspace(int num_seqs, int64_t total_tokens, int H);
 // backward pass's scans over the records.
 enum : int { kCpNone = 0, kCpLocal = 1, kCpFinish = 2, kPrepOnly = 3 };
 
-// The layer with its prologue as a pass of its own (the activations turned
-// into the operator's bf16 inputs in the workspace), then the split path and
-// the epilogue; its workspace is layer_prefill_workspace bytes.
+// The layer with its prologue as a pass of its own (log_alpha, beta and the
+// inverse norms of q and k into the workspace), then the split path on the raw
+// q and k scaled by those norms, and the epilogue; its workspace is
+// layer_prefill_workspace bytes.
 size_t layer_prefill_workspace(int num_seqs, int64_t total_tokens, int H);
 cudaError_t launch_layer_prefill_split(const void *q, const void *k, const void *v, const LayerArgs &la,
                                        const float *init_state, const int32_t *cu, int num_seqs,
@@ -129,7 +130,8 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                  int num_seqs, int64_t total_tokens, int H, void *o,
                                  float *final_state, void *workspace, bool scalar_gate,
                                  const LayerArgs *layer, cudaStream_t stream,
-                                 int cp_mode = kCpNone, float *cp_transition = nullptr);
+                                 int cp_mode = kCpNone, float *cp_transition = nullptr,
+                                 const float *nrm_in = nullptr);
 
 // Backward pass (fp32 gradients; d_k and d_v multiples of 32 up to 128).
 // Its workspace keeps the state entering every 64-step block of every

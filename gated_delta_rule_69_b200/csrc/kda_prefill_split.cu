@@ -143,6 +143,9 @@ struct Params {
     // layer prologue / epilogue (layer != 0): the g map carries the gate
     // pre-activation, beta holds logits; the chain normalises and gates o
     int layer;
+    // the layer prologue's inverse L2 norms of k and q, fp32 [T * H][2] (k, q),
+    // for raw q and k (the preparation scales every operand by them); or null
+    const float *nrm_in;
     const float *A_log;
     const __nv_bfloat16 *out_gate;
     const float *norm_weight;
@@ -334,7 +337,10 @@ __device__ __forceinline__ void write_qp(uint8_t *stk, uint32_t tmem, int quad, 
     }
 }
 
-template <int P, bool LAYER, bool SCALAR>
+// LAYER: 0 the plain operator; 1 the layer prologue inside (gate activation,
+// beta sigmoid and the q / k norms from the raw rows); 2 the operator on raw q
+// and k with their inverse norms given (p.nrm_in).
+template <int P, int LAYER, bool SCALAR>
 __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int tid, int warp, int lane,
                                               const CUtensorMap &tm_k, const CUtensorMap &tm_q,
                                               const CUtensorMap &tm_g, const Params &p,
@@ -397,8 +403,15 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         }
         if (pt < C) {
             float bv = (pt < L) ? __bfloat162float(p.beta[(size_t)(tok0 + pt) * p.H + h]) : 0.f;
-            if (LAYER && pt < L) bv = 1.f / (1.f + __expf(-bv));   // beta = sigmoid(logit)
+            if (LAYER == 1 && pt < L) bv = 1.f / (1.f + __expf(-bv));   // beta = sigmoid(logit)
             beta[pt] = bv;
+            if (LAYER == 2) {   // the given inverse norms (none past the chunk end)
+                float2 nv = make_float2(0.f, 0.f);
+                if (pt < L) nv = *reinterpret_cast<const float2 *>(p.nrm_in + ((size_t)(tok0 + pt) * p.H + h) * 2);
+                float *nrm = reinterpret_cast<float *>(sm + PrepSmem::NRM);
+                nrm[pt] = nv.x;
+                nrm[64 + pt] = nv.y;
+            }
             if (SCALAR) {   // one log_alpha per token (zero past the chunk end)
                 reinterpret_cast<float *>(sm + PrepSmem::GSC)[pt] =
                     pt < L ? __bfloat162float(p.g[(size_t)(tok0 + pt) * p.H + h]) : 0.f;
@@ -422,7 +435,7 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
         b.csum = reinterpret_cast<float *>(sm + PrepSmem::CSUM);
         b.slow_flag = misc + 2;
         b.nrm = LAYER ? reinterpret_cast<float *>(sm + PrepSmem::NRM) : nullptr;
-        b.neg_eA = LAYER ? -__expf(p.A_log[h]) : 0.f;
+        b.neg_eA = LAYER == 1 ? -__expf(p.A_log[h]) : 0.f;
         b.qk_eps = p.qk_eps;
         b.gsc = SCALAR ? reinterpret_cast<const float *>(sm + PrepSmem::GSC) : nullptr;
 
@@ -537,10 +550,11 @@ __device__ __forceinline__ void prep_pipeline(uint8_t *sm, uint32_t tmem, int ti
     }
 }
 
-// LAYER: the layer prologue (gate activation, q / k normalisation, beta
-// sigmoid) fused in; SCALAR: the Gated DeltaNet gate (one log_alpha per
-// token); separate instantiations keep the plain kernel as it is.
-template <bool LAYER, bool SCALAR>
+// LAYER (as prep_pipeline): 1 the layer prologue (gate activation, q / k
+// normalisation, beta sigmoid) fused in, 2 raw q and k with given inverse
+// norms; SCALAR: the Gated DeltaNet gate (one log_alpha per token); separate
+// instantiations keep the plain kernel as it is.
+template <int LAYER, bool SCALAR>
 __global__ void __launch_bounds__(kPrepThreads, 1)
 kda_prep_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_g, const Params p) {
@@ -1287,13 +1301,15 @@ kda_cp_local_chains_kernel(const __grid_constant__ CUtensorMap tm_v, const Param
 }
 
 // =============================================================== layer prologue
-// The layer's activations as the operator's inputs: q and k L2-normalised
-// (x rsqrt(sum x^2 + eps)), log_alpha = -e^{A_log[h]} softplus(z), beta =
-// sigmoid(logit), all written in bf16.  A half-warp per (token, head) row of
-// 128 channels (16-byte pieces, eight channels per lane).  A pass of its own ahead of the
-// operator: inside the chunk preparation the same arithmetic sat on that
-// kernel's latency-bound path, while as a stream over the activations it is
-// bound by HBM.
+// The layer's activations as the operator's inputs: log_alpha = -e^{A_log[h]}
+// softplus(z) and beta = sigmoid(logit) in bf16, and the inverse L2 norms
+// rsqrt(sum x^2 + eps) of every k and q row in fp32 ([row][k, q]); the
+// preparation reads the raw q and k and scales every operand by the norms, so
+// the normalised rows are never written out.  A half-warp per (token, head) row
+// of 128 channels (16-byte pieces, eight channels per lane).  A pass of its own
+// ahead of the operator: inside the chunk preparation the same arithmetic sat
+// on that kernel's latency-bound path, while as a stream over the activations
+// it is bound by HBM.
 constexpr int kProThreads = 256;
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 &w, float (&x)[8]) {
@@ -1319,8 +1335,8 @@ __global__ void __launch_bounds__(kProThreads)
 kda_layer_prologue_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                           const __nv_bfloat16 *__restrict__ z, const __nv_bfloat16 *__restrict__ blogit,
                           const float *__restrict__ A_log, float eps, int H, int64_t rows,
-                          __nv_bfloat16 *__restrict__ qn, __nv_bfloat16 *__restrict__ kn,
-                          __nv_bfloat16 *__restrict__ la, __nv_bfloat16 *__restrict__ bt) {
+                          float *__restrict__ nrm, __nv_bfloat16 *__restrict__ la,
+                          __nv_bfloat16 *__restrict__ bt) {
     const int lane = threadIdx.x & 31, sub = lane & 15;
     // a warp's two rows (half-warps); the shuffles take all 32 lanes, so a row
     // past the end is masked, not skipped
@@ -1353,10 +1369,11 @@ kda_layer_prologue_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat
 #pragma unroll
     for (int e = 0; e < 8; ++e)   // softplus as the in-kernel prologue takes it
         xz[e] = c * (xz[e] > 15.f ? xz[e] : __logf(1.f + __expf(xz[e])));
-    reinterpret_cast<uint4 *>(qn)[at] = f32x8_to_bf16(xq, rsqrtf(sq + eps));
-    reinterpret_cast<uint4 *>(kn)[at] = f32x8_to_bf16(xk, rsqrtf(sk + eps));
     reinterpret_cast<uint4 *>(la)[at] = f32x8_to_bf16(xz, 1.f);
-    if (sub == 0) bt[row] = __float2bfloat16(1.f / (1.f + __expf(-__bfloat162float(blogit[row]))));
+    if (sub == 0) {
+        reinterpret_cast<float2 *>(nrm)[row] = make_float2(rsqrtf(sk + eps), rsqrtf(sq + eps));
+        bt[row] = __float2bfloat16(1.f / (1.f + __expf(-__bfloat162float(blogit[row]))));
+    }
 }
 
 // =============================================================== layer epilogue
@@ -1689,18 +1706,17 @@ bool make_bf16_map_3d(CUtensorMap *m, const void *base, int64_t T, int H, int in
 }
 
 // The layer path with its prologue as a pass of its own: the split
-// workspace, then the prologue's outputs (q, k, log_alpha [T, H, 128] and
-// beta [T, H], bf16), 256-byte aligned.
+// workspace, then the prologue's outputs (log_alpha [T, H, 128] and beta
+// [T, H] in bf16, the inverse norms [T, H, 2] in fp32), 256-byte aligned.
 struct LayerLayout {
-    size_t qn, kn, la, bt, total;
+    size_t nrm, la, bt, total;
 };
 
 LayerLayout layer_layout(int num_seqs, int64_t total_tokens, int H) {
     LayerLayout l;
     const size_t tile = (size_t)total_tokens * H * 128 * sizeof(__nv_bfloat16);
-    l.qn = round_up(split_layout(num_seqs, total_tokens, H).total, 256);
-    l.kn = l.qn + round_up(tile, 256);
-    l.la = l.kn + round_up(tile, 256);
+    l.nrm = round_up(split_layout(num_seqs, total_tokens, H).total, 256);
+    l.la = l.nrm + round_up((size_t)total_tokens * H * 2 * sizeof(float), 256);
     l.bt = l.la + round_up(tile, 256);
     l.total = l.bt + round_up((size_t)total_tokens * H * sizeof(__nv_bfloat16), 256);
     return l;
@@ -1717,8 +1733,7 @@ cudaError_t launch_layer_prefill_split(const void *q, const void *k, const void 
     using namespace split;
     const LayerLayout l = layer_layout(num_seqs, total_tokens, H);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    auto *qn = reinterpret_cast<__nv_bfloat16 *>(ws + l.qn);
-    auto *kn = reinterpret_cast<__nv_bfloat16 *>(ws + l.kn);
+    auto *nrm = reinterpret_cast<float *>(ws + l.nrm);
     auto *lg = reinterpret_cast<__nv_bfloat16 *>(ws + l.la);
     auto *bt = reinterpret_cast<__nv_bfloat16 *>(ws + l.bt);
     const int64_t rows = total_tokens * H;
@@ -1727,12 +1742,12 @@ cudaError_t launch_layer_prefill_split(const void *q, const void *k, const void 
         kda_layer_prologue_kernel<<<(unsigned)((rows + per - 1) / per), kProThreads, 0, stream>>>(
             static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
             static_cast<const __nv_bfloat16 *>(la.gate_z), static_cast<const __nv_bfloat16 *>(la.beta_logit),
-            la.A_log, la.qk_eps, H, rows, qn, kn, lg, bt);
+            la.A_log, la.qk_eps, H, rows, nrm, lg, bt);
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    cudaError_t e = launch_prefill_split(qn, kn, v, lg, bt, init_state, cu, num_seqs, total_tokens, H, o,
-                                         final_state, workspace, false, nullptr, stream, kCpNone, nullptr);
+    cudaError_t e = launch_prefill_split(q, k, v, lg, bt, init_state, cu, num_seqs, total_tokens, H, o,
+                                         final_state, workspace, false, nullptr, stream, kCpNone, nullptr, nrm);
     if (e != cudaSuccess || rows == 0) return e;
     kda_layer_epilogue_kernel<<<(unsigned)((rows + kEpiThreads / 16 - 1) / (kEpiThreads / 16)), kEpiThreads, 0,
                                 stream>>>(static_cast<__nv_bfloat16 *>(o),
@@ -1810,7 +1825,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                  int num_seqs, int64_t total_tokens, int H, void *o,
                                  float *final_state, void *workspace, bool scalar_gate,
                                  const LayerArgs *layer, cudaStream_t stream, int cp_mode,
-                                 float *cp_transition) {
+                                 float *cp_transition, const float *nrm_in) {
     using namespace split;
     const SplitLayout l = split_layout(num_seqs, total_tokens, H);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1869,11 +1884,13 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                                           work_next);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = set_max_dynamic_smem((const void *)kda_prep_kernel<false, false>, (int)PrepSmem::ALLOC);
+    e = set_max_dynamic_smem((const void *)kda_prep_kernel<0, false>, (int)PrepSmem::ALLOC);
     if (e != cudaSuccess) return e;
-    e = set_max_dynamic_smem((const void *)kda_prep_kernel<true, false>, (int)PrepSmem::ALLOC);
+    e = set_max_dynamic_smem((const void *)kda_prep_kernel<1, false>, (int)PrepSmem::ALLOC);
     if (e != cudaSuccess) return e;
-    e = set_max_dynamic_smem((const void *)kda_prep_kernel<false, true>, (int)PrepSmem::ALLOC);
+    e = set_max_dynamic_smem((const void *)kda_prep_kernel<2, false>, (int)PrepSmem::ALLOC);
+    if (e != cudaSuccess) return e;
+    e = set_max_dynamic_smem((const void *)kda_prep_kernel<0, true>, (int)PrepSmem::ALLOC);
     if (e != cudaSuccess) return e;
     Params prm;
     prm.k = static_cast<const __nv_bfloat16 *>(k);
@@ -1882,6 +1899,7 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     prm.g = static_cast<const __nv_bfloat16 *>(g);
     prm.scalar_gate = scalar_gate ? 1 : 0;
     prm.layer = layer ? 1 : 0;
+    prm.nrm_in = nrm_in;
     prm.A_log = layer ? layer->A_log : nullptr;
     prm.out_gate = layer ? static_cast<const __nv_bfloat16 *>(layer->out_gate) : nullptr;
     prm.norm_weight = layer ? layer->norm_weight : nullptr;
@@ -1916,9 +1934,10 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = layer         ? cudaLaunchKernelEx(&cfg, kda_prep_kernel<true, false>, mk, mq, mg, prm)
-            : scalar_gate ? cudaLaunchKernelEx(&cfg, kda_prep_kernel<false, true>, mk, mq, mg, prm)
-                          : cudaLaunchKernelEx(&cfg, kda_prep_kernel<false, false>, mk, mq, mg, prm);
+        e = layer         ? cudaLaunchKernelEx(&cfg, kda_prep_kernel<1, false>, mk, mq, mg, prm)
+            : nrm_in      ? cudaLaunchKernelEx(&cfg, kda_prep_kernel<2, false>, mk, mq, mg, prm)
+            : scalar_gate ? cudaLaunchKernelEx(&cfg, kda_prep_kernel<0, true>, mk, mq, mg, prm)
+                          : cudaLaunchKernelEx(&cfg, kda_prep_kernel<0, false>, mk, mq, mg, prm);
         if (e != cudaSuccess) return e;
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

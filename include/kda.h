@@ -209,8 +209,9 @@ kda_status gdn_decode_step(const void *q, const void *k, const void *v,
  * d_k = d_v = 128 and a workspace of at least kda_prefill_workspace_size(...)
  * bytes (else KDA_ERR_UNSUPPORTED / KDA_ERR_WORKSPACE).  With a workspace of
  * kda_layer_prefill_workspace_size(...) bytes its prologue runs as a pass of
- * its own that writes the operator's inputs (normalised q and k, log_alpha
- * and beta, bf16) into the workspace, then the operator's kernels; with less,
+ * its own that writes log_alpha and beta (bf16) and the inverse L2 norms of
+ * the q and k rows (fp32) into the workspace, then the operator's kernels,
+ * whose preparation scales the raw q and k by those norms; with less,
  * the prologue runs inside the chunk preparation (log_alpha kept in fp32
  * there; slower: the arithmetic lands on that kernel's latency-bound path).
  * Either way the epilogue is one pass over o after the state chain.
