@@ -1238,12 +1238,14 @@ __device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const CUte
             tc_fence_after();
             const float4 *egl = reinterpret_cast<const float4 *>(sm + Cfg::EGLR + se * 512) + 8 * g;
             const uint32_t xo = Cfg::COL_XO + Cfg::XO_STRIDE * (n & 1);
+            float x0[16], x1[16];   // X's two halves (and O^T) in one round trip
+            tmem_ld16(tmem_addr(tmem, 32 * quad, xo + 32 * g), x0);
+            tmem_ld16(tmem_addr(tmem, 32 * quad, xo + 32 * g + 16), x1);
+            if (OUT) tmem_ld16(tmem_addr(tmem, 32 * quad, xo + Cfg::COL_O + 16 * g), ov);
+            tmem_wait_ld();
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                float x[16];
-                tmem_ld16(tmem_addr(tmem, 32 * quad, xo + 32 * g + 16 * hh), x);
-                if (OUT && hh == 1) tmem_ld16(tmem_addr(tmem, 32 * quad, xo + Cfg::COL_O + 16 * g), ov);
-                tmem_wait_ld();
+                const float *x = hh ? x1 : x0;
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
                     const float4 d = egl[4 * hh + e4];
