@@ -325,8 +325,11 @@ def time_prefill(w, steps, warmup, world, scalar_gate=False, layer=False, profil
     if kda.kda_check_workspace_error(ws) != kda.KDA_OK:
         raise RuntimeError("device-side check failed during the benchmark")
     # each call with a full workspace on bf16 d = 128 launches three kernels:
-    # the plan, the preparation and the state chain
+    # the plan, the preparation and the state chain (the layer two more: its
+    # prologue pass and its epilogue)
     per_call = 3 if (w.dtype == "bf16" and w.d_k == 128 and w.d_v == 128) else 2
+    if layer:
+        per_call += 2
     return dict(ms_total=sum(ms), ms=ms, inputs=inp, launches=steps * per_call)
 
 
