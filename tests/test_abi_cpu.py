@@ -58,6 +58,20 @@ def test_workspace_size(L):
     assert ws(1, -1, 1, 16, 16) == 0
 
 
+def test_layer_workspace_size(L):
+    """The layer's workspace is the prefill's plus what its prologue pass
+    leaves for the operator: the inverse norms of the k and q rows (fp32 pairs),
+    log_alpha per (token, head, channel) and beta per (token, head) in bf16,
+    each 256-byte aligned; the normalised q and k are never written."""
+    up = lambda x: (x + 255) // 256 * 256
+    for n, T, H in ((1, 4096, 16), (1, 131072, 32), (16, 133_000, 32), (3, 1, 1)):
+        base = L.kda_prefill_workspace_size(n, T, H, 128, 128)
+        lay = L.kda_layer_prefill_workspace_size(n, T, H, 128, 128)
+        assert lay == up(base) + up(T * H * 8) + up(T * H * 128 * 2) + up(T * H * 2), (n, T, H)
+    assert L.kda_layer_prefill_workspace_size(1, 4096, 16, 64, 128) == 0
+    assert L.kda_layer_prefill_workspace_size(0, 4096, 16, 128, 128) == 0
+
+
 FAKE = 1 << 20  # 16-byte aligned, never dereferenced on the host
 
 
