@@ -1088,8 +1088,9 @@ __device__ __forceinline__ void chain_t_unit(const CUtensorMap &tm_v, const CUte
             if (lane == 0) tma_prefetch_desc(tm_o);
             for (int m = 0; m < nchunks; ++m) {
                 const int b = m & 1;
-                mbar_wait(&STGF[b], (m >> 1) & 1, abort_flag);
-                if (*abort_flag) break;
+                const bool ok = mbar_wait(&STGF[b], (m >> 1) & 1, abort_flag);
+                // one decision for the whole warp: the loop below synchronises it
+                if (__any_sync(0xffffffffu, !ok || *abort_flag != 0u)) break;
                 const uint8_t *src = sm + Cfg::STG + b * 16384;
                 const int rows = (int)min((int64_t)C, len - (int64_t)m * C);
                 if (rows == C) {
