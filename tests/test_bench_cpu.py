@@ -43,3 +43,37 @@ def test_warmup_below_three_rejected():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
                         "--warmup", "2"], capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert r.returncode != 0
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    sys.path.insert(0, ROOT)
+    import bench
+    bench.barrier(world)
+    # per-rank step times; every rank must report the slowest
+    got = bench.max_over_ranks([3.0, 7.5, 5.25][rank], world)
+    bench.barrier(world)
+    dist.destroy_process_group()
+    with open(os.path.join(out, f"rank{rank}.json"), "w") as f:
+        json.dump(got, f)
+
+
+def test_max_over_ranks_under_gloo(tmp_path):
+    """The bench's cross-rank reduction (max of the per-rank step times, which
+    sets value = all ranks' tokens / slowest time) with 2 and 3 gloo ranks on
+    the CPU."""
+    import socket
+    import torch.multiprocessing as mp
+    for world in (2, 3):
+        with socket.socket() as s:
+            s.bind(("127.0.0.1", 0))
+            port = s.getsockname()[1]
+        out = tmp_path / f"w{world}"
+        out.mkdir()
+        mp.start_processes(_rank_main, args=(world, port, str(out)), nprocs=world, join=True,
+                           start_method="spawn")
+        want = max([3.0, 7.5, 5.25][:world])
+        for r in range(world):
+            assert json.load(open(out / f"rank{r}.json")) == want
