@@ -898,9 +898,9 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 // and 32 columns c); per chunk they write its bf16 copy SB_n^T into TMEM as
 // the A operand of the products, read the fresh product X_n back, and form
 // S_{n+1} with one FMA per element: no fp32 state goes back to TMEM.  The
-// record operands keep their layout and descriptors; they only change side
-// (B instead of A), and V (its two 64-column atoms) is the A operand in the
-// MN-major form.
+// record operands keep their tile layout (K-major, 128-byte swizzle); they
+// only change side (B instead of A), and V (its two 64-column atoms) is the A
+// operand in the MN-major form.
 // A tcgen05 product costs about the same whatever its N up to 192 (~100
 // cycles per M = 128, K = 16 instruction with A in shared memory, ~116 with
 // A in TMEM, against ~134 at N = 256), so the products that share their A
@@ -916,8 +916,8 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_v, const Params p) {
 // over, write it in bf16 to a shared-memory staging tile that a store warp
 // copies to o with one tensor store per chunk (stores from the chain warps'
 // registers straight to global memory, 16 of 64 bytes per warp and chunk,
-// took most of a chunk's period).  The backward scan modes stage the state tiles they
-// save the same way, and one bulk copy per chunk writes each out.
+// took most of a chunk's period).  The backward scan modes stage the state
+// tiles they save the same way, and one bulk copy per chunk writes each out.
 // Rings, each with its loader warp: R (MP, QP, YT, ZB of a record in the
 // layout above), E (exp(G_L); its own deeper ring, since the chain warps read
 // it only after the state products) and V (the v tile, read from HBM).
