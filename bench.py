@@ -546,6 +546,7 @@ def config_of(w, lengths, n_gpus):
     c = {"workload": w.name, "tokens": sum(lengths), "num_seqs": len(lengths), "H": w.H,
          "d_k": w.d_k, "d_v": w.d_v, "chunk": CHUNK, "io_dtype": w.dtype,
          "state_dtype": "fp32", "init_state": "N(0, 0.02)" if w.init_std > 0 else "zeros",
+         "seed": w.seed,
          "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
          "l2": "flushed by a 256 MiB write before each timed prefill step"}
     return c

@@ -31,6 +31,7 @@ def test_reference_arm_json_line():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"] == "tiny_T64_H1_d16_fp32"
+    assert isinstance(line["config"]["seed"], int)   # the input draw's seed travels with the line
 
 
 def test_reference_arm_other_ranks_silent():
