@@ -200,3 +200,42 @@ def test_binding_checks_backward_gate_shape():
         kda.kda_backward(x, x, x, b, b, x)
     with pytest.raises(ValueError):   # per-channel gate given to the per-head entry
         kda.gdn_backward(x, x, x, x, b, x)
+
+
+def _backward_chunked(L, fn="kda_backward_chunked", **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, g=FAKE * 4, b=FAKE * 5, s0=None, cu=None,
+             n=1, T=64, H=1, do=FAKE * 6, dfs=None, dq=FAKE * 64, dkk=FAKE * 65,
+             dvv=FAKE * 66, dg=FAKE * 67, db=FAKE * 68, ds0=None, ws=FAKE * 128, wsb=1 << 40)
+    a.update(kw)
+    return getattr(L, fn)(a["q"], a["k"], a["v"], a["g"], a["b"], a["s0"], a["cu"], a["n"],
+                          a["T"], a["H"], a["do"], a["dfs"], a["dq"], a["dkk"], a["dvv"],
+                          a["dg"], a["db"], a["ds0"], a["ws"], a["wsb"], None)
+
+
+def test_backward_chunked_workspace_size(L):
+    ws = L.kda_backward_chunked_workspace_size
+    # at least the prefill's split workspace and two bf16 state tiles (32 KB each) per record
+    for n, T, H in ((1, 4096, 16), (3, 1000, 2)):
+        chunks = T // 64 + n
+        assert ws(n, T, H) >= L.kda_prefill_workspace_size(n, T, H, 128, 128) + 2 * chunks * H * 32768
+    assert ws(0, 64, 1) == 0
+
+
+def test_backward_chunked_rejects_on_host(L):
+    """Every refusal is decided on the host, before any CUDA call."""
+    for fn in ("kda_backward_chunked", "gdn_backward_chunked"):
+        assert _backward_chunked(L, fn, n=0) == 1
+        assert _backward_chunked(L, fn, T=0) == 1
+        assert _backward_chunked(L, fn, n=3) == 1                # T % N != 0 without cu_seqlens
+        assert _backward_chunked(L, fn, do=None) == 1
+        assert _backward_chunked(L, fn, dq=None) == 1
+        assert _backward_chunked(L, fn, q=FAKE + 4) == 1         # q not 16-byte aligned
+        assert _backward_chunked(L, fn, dvv=FAKE * 66 + 8) == 1  # dv not 16-byte aligned
+        assert _backward_chunked(L, fn, dq=FAKE * 64 + 2) == 1   # dq not 4-byte aligned
+        assert _backward_chunked(L, fn, b=FAKE * 5 + 1) == 1     # beta not 2-byte aligned
+        assert _backward_chunked(L, fn, wsb=1024) == 3           # workspace too small
+        assert _backward_chunked(L, fn, ws=None) == 3
+        assert _backward_chunked(L, fn, ws=FAKE * 128 + 16) == 1  # workspace not 256-aligned
+    # the per-channel gate is a 16-byte aligned tile; the scalar gate needs 2 bytes only
+    assert _backward_chunked(L, "kda_backward_chunked", g=FAKE * 4 + 2) == 1
+    assert _backward_chunked(L, "gdn_backward_chunked", g=FAKE * 4 + 1) == 1
