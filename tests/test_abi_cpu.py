@@ -239,3 +239,56 @@ def test_backward_chunked_rejects_on_host(L):
     # the per-channel gate is a 16-byte aligned tile; the scalar gate needs 2 bytes only
     assert _backward_chunked(L, "kda_backward_chunked", g=FAKE * 4 + 2) == 1
     assert _backward_chunked(L, "gdn_backward_chunked", g=FAKE * 4 + 1) == 1
+
+
+BF16, FP32 = 0, 1   # kda_dtype
+
+
+def test_cp_entries_reject_on_host(L):
+    """kda_cp_combine / kda_cp_local / kda_cp_finish decide every refusal on the
+    host: shapes without a kernel, null or misaligned pointers, too small or
+    misaligned workspaces, outputs over inputs."""
+    big = 1 << 40
+    ws = FAKE * 1024
+    # combine: S_in [H, d_k, d_v] from n_prev (M, S~) pairs
+    cmb = lambda **kw: L.kda_cp_combine(kw.get("M", FAKE), kw.get("St", FAKE * 2), kw.get("S0", None),
+                                        kw.get("Sin", FAKE * 8), kw.get("n", 1), kw.get("H", 1),
+                                        kw.get("dk", 32), kw.get("dv", 32), None)
+    assert cmb(n=-1) == 1
+    assert cmb(H=0) == 1
+    assert cmb(dv=16) == 2                       # d_v below 32
+    assert cmb(dk=48) == 2
+    assert cmb(Sin=None) == 1
+    assert cmb(M=None) == 1                      # n_prev > 0 needs M and S~
+    assert cmb(Sin=FAKE * 8 + 2) == 1            # not 4-byte aligned
+    assert cmb(Sin=FAKE + 64) == 1               # S_in inside M
+    # local: bf16, d = 128 only
+    loc = lambda **kw: L.kda_cp_local(kw.get("q", FAKE), kw.get("k", FAKE * 2), kw.get("v", FAKE * 3),
+                                      kw.get("g", FAKE * 4), kw.get("b", FAKE * 5), kw.get("T", 64),
+                                      kw.get("H", 1), kw.get("dk", 128), kw.get("dv", 128),
+                                      kw.get("dt", BF16), kw.get("M", FAKE * 8), kw.get("St", FAKE * 9),
+                                      kw.get("os", None), kw.get("ws", ws), kw.get("wsb", big), None)
+    assert loc(T=0) == 1
+    assert loc(dt=FP32) == 2
+    assert loc(dk=64) == 2
+    assert loc(M=None) == 1
+    assert loc(q=FAKE + 8) == 1                  # not 16-byte aligned
+    assert loc(b=FAKE * 5 + 1) == 1
+    assert loc(wsb=1024) == 3
+    assert loc(ws=None) == 3
+    assert loc(ws=ws + 16) == 1                  # workspace not 256-aligned
+    assert loc(M=FAKE * 3) == 1                  # M over v
+    assert loc(St=FAKE * 8) == 1                 # S~ over M
+    # finish: the chain again over the kept records
+    fin = lambda **kw: L.kda_cp_finish(kw.get("v", FAKE * 3), kw.get("Sin", FAKE * 8), kw.get("T", 64),
+                                       kw.get("H", 1), kw.get("dk", 128), kw.get("dv", 128),
+                                       kw.get("dt", BF16), kw.get("o", FAKE * 16), kw.get("fs", None),
+                                       kw.get("ws", ws), kw.get("wsb", big), None)
+    assert fin(T=0) == 1
+    assert fin(dv=64) == 2
+    assert fin(o=None) == 1
+    assert fin(o=FAKE * 16 + 4) == 1
+    assert fin(wsb=16) == 3
+    assert fin(ws=ws + 64) == 1
+    assert fin(o=FAKE * 3) == 1                  # o over v
+    assert fin(fs=FAKE * 16 + 1024) == 1         # final state inside o
