@@ -292,3 +292,33 @@ def test_cp_entries_reject_on_host(L):
     assert fin(ws=ws + 64) == 1
     assert fin(o=FAKE * 3) == 1                  # o over v
     assert fin(fs=FAKE * 16 + 1024) == 1         # final state inside o
+
+
+def test_layer_prefill_rejects_on_host(L):
+    """kda_layer_prefill: the two-kernel tensor-core path only (bf16, d = 128,
+    at least the prefill's workspace), A_log required, eps >= 0, the output
+    gate not under o; all decided on the host."""
+    T, H = 64, 1
+    big = 1 << 40
+    ws = FAKE * 1024
+
+    def lay(**kw):
+        a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, z=FAKE * 4, A=FAKE * 5, bl=FAKE * 6, og=None, nw=None,
+                 qe=1e-6, ne=1e-6, s0=None, cu=None, n=1, T=T, H=H, dk=128, dv=128, dt=BF16,
+                 o=FAKE * 16, fs=None, ws=ws, wsb=big)
+        a.update(kw)
+        return L.kda_layer_prefill(a["q"], a["k"], a["v"], a["z"], a["A"], a["bl"], a["og"], a["nw"],
+                                   a["qe"], a["ne"], a["s0"], a["cu"], a["n"], a["T"], a["H"], a["dk"],
+                                   a["dv"], a["dt"], a["o"], a["fs"], a["ws"], a["wsb"], None)
+    assert lay(n=0) == 1
+    assert lay(dt=FP32) == 2                     # the layer has no fp32 path
+    assert lay(dk=64, dv=64) == 2
+    assert lay(A=None) == 1
+    assert lay(A=FAKE * 5 + 2) == 1              # A_log not 4-byte aligned
+    assert lay(nw=FAKE * 7 + 1) == 1
+    assert lay(og=FAKE * 8 + 8) == 1             # out_gate not 16-byte aligned
+    assert lay(og=FAKE * 16 + 4096) == 1         # out_gate under o
+    assert lay(qe=-1.0) == 1
+    assert lay(ne=float("nan")) == 1
+    assert lay(wsb=1024) == 3
+    assert lay(ws=ws + 128) == 1                 # workspace not 256-aligned
