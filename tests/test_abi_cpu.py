@@ -322,3 +322,13 @@ def test_layer_prefill_rejects_on_host(L):
     assert lay(ne=float("nan")) == 1
     assert lay(wsb=1024) == 3
     assert lay(ws=ws + 128) == 1                 # workspace not 256-aligned
+
+
+def test_noalloc_refuses_more_sequences_than_its_array_holds(L):
+    """kda_prefill_noalloc keeps its scratch in a fixed array sized for
+    KDA_NOALLOC_MAX_SEQS sequences; more is refused before any CUDA call."""
+    text = open(os.path.join(ROOT, "include", "kda.h")).read()
+    cap = int(re.search(r"#define KDA_NOALLOC_MAX_SEQS (\d+)", text).group(1))
+    st = L.kda_prefill_noalloc(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, FAKE * 5, None, FAKE * 6,
+                               cap + 1, 64 * (cap + 1), 1, 128, 128, BF16, FAKE * 16, None, None)
+    assert st == 2
