@@ -332,3 +332,27 @@ def test_noalloc_refuses_more_sequences_than_its_array_holds(L):
     st = L.kda_prefill_noalloc(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, FAKE * 5, None, FAKE * 6,
                                cap + 1, 64 * (cap + 1), 1, 128, 128, BF16, FAKE * 16, None, None)
     assert st == 2
+
+
+def test_layer_decode_rejects_on_host(L):
+    """kda_layer_decode_step: kda_decode_step's checks plus the layer's own
+    (A_log required and 4-byte aligned, eps >= 0, the output gate aligned and
+    not under o)."""
+    def lay(**kw):
+        a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, z=FAKE * 4, A=FAKE * 5, bl=FAKE * 6, og=None, nw=None,
+                 qe=1e-6, ne=1e-6, s=FAKE * 16, B=4, H=2, dk=16, dv=16, dt=FP32, o=FAKE * 64)
+        a.update(kw)
+        return L.kda_layer_decode_step(a["q"], a["k"], a["v"], a["z"], a["A"], a["bl"], a["og"], a["nw"],
+                                       a["qe"], a["ne"], a["s"], a["B"], a["H"], a["dk"], a["dv"],
+                                       a["dt"], a["o"], None)
+    assert lay(B=0) == 0                         # empty batch: no-op
+    assert lay(B=-1) == 1
+    assert lay(dk=48) == 2
+    assert lay(A=None) == 1
+    assert lay(A=FAKE * 5 + 2) == 1
+    assert lay(nw=FAKE * 7 + 2) == 1
+    assert lay(og=FAKE * 8 + 2) == 1             # fp32 gate not 4-byte aligned
+    assert lay(og=FAKE * 64 + 64) == 1           # out_gate under o
+    assert lay(qe=-0.5) == 1
+    assert lay(ne=float("nan")) == 1
+    assert lay(s=FAKE * 16 + 8) == 1             # state not 16-byte aligned
