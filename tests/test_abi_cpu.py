@@ -356,3 +356,14 @@ def test_layer_decode_rejects_on_host(L):
     assert lay(qe=-0.5) == 1
     assert lay(ne=float("nan")) == 1
     assert lay(s=FAKE * 16 + 8) == 1             # state not 16-byte aligned
+
+
+def test_binding_checks_chunked_backward_gate_shape():
+    import torch
+    from gated_delta_rule_69_b200 import kda
+    x = torch.zeros(4, 2, 128, dtype=torch.bfloat16)
+    b = torch.zeros(4, 2, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):   # per-head gate given to the per-channel entry
+        kda.kda_backward_chunked(x, x, x, b, b, x)
+    with pytest.raises(ValueError):   # per-channel gate given to the Gated DeltaNet entry
+        kda.gdn_backward_chunked(x, x, x, x, b, x)
